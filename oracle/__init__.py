@@ -1,0 +1,174 @@
+"""fp64 CPU oracle for RoPE context extension + causal attention prefill.
+
+TEST INFRASTRUCTURE ONLY: the test suite, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg are the only callers.  The CUDA library never
+imports or links anything here, and this package imports nothing from it.
+
+Thin ctypes wrappers around ``liblcx_oracle.so`` (plain C, fp64); see
+``lcx_oracle.c`` for the definitions and their sources.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+MODES = {"none": 0, "plain": 1, "pi": 2, "ntk": 3, "yarn": 4}
+PAIRINGS = {"half": 0, "interleaved": 1}
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        f32p = ctypes.POINTER(ctypes.c_float)
+        f64p = ctypes.POINTER(ctypes.c_double)
+        i32p = ctypes.POINTER(ctypes.c_int)
+        lib.orc_rope_theta_fp64.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                            ctypes.c_double, ctypes.c_int64, ctypes.c_double,
+                                            ctypes.c_double, f64p, f64p]
+        lib.orc_rope_table.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                       ctypes.c_double, ctypes.c_int64, ctypes.c_double,
+                                       ctypes.c_double, f32p, f32p, f64p, i32p]
+        lib.orc_rotate_rows.argtypes = [f32p, f64p, ctypes.c_int64, ctypes.c_int, i64p,
+                                        f32p, ctypes.c_float, ctypes.c_int]
+        lib.orc_visible.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                    ctypes.c_int, ctypes.c_int64, ctypes.c_int64]
+        lib.orc_mask.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
+                                 ctypes.POINTER(ctypes.c_uint8)]
+        lib.orc_mask.restype = None
+        lib.orc_attn_rows.argtypes = [f32p, i64p, i64p, i64p, ctypes.c_int64, f32p, f32p,
+                                      ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                      ctypes.c_int64, ctypes.c_int64, f32p, ctypes.c_float,
+                                      ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+                                      ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
+                                      f64p, f64p, ctypes.c_int]
+        lib.orc_num_threads.argtypes = [ctypes.c_int]
+        _lib = lib
+    return _lib
+
+
+def _ptr(a, ct):
+    return a.ctypes.data_as(ctypes.POINTER(ct))
+
+
+def rope_theta_fp64(mode, D, base=10000.0, scale=1.0, original_max_pos=4096,
+                    alpha=1.0, beta=32.0):
+    """theta'_i in fp64 (before the fp32 rounding) and mscale in fp64."""
+    lib = _load()
+    out = np.zeros(D // 2, dtype=np.float64)
+    ms = ctypes.c_double(0.0)
+    rc = lib.orc_rope_theta_fp64(MODES[mode], D, base, scale, original_max_pos, alpha, beta,
+                                 _ptr(out, ctypes.c_double), ctypes.byref(ms))
+    if rc:
+        raise ValueError("orc_rope_theta_fp64: invalid argument")
+    return out, ms.value
+
+
+def rope_table(mode, D, base=10000.0, scale=1.0, original_max_pos=4096, alpha=1.0, beta=32.0):
+    """fp32 table (theta'_i rounded to nearest even), fp32 mscale, midpoint flags.
+
+    flags has D/2 + 1 entries (the last one for mscale); a 1 marks a value whose
+    fp32 rounding is too close to a midpoint to be trusted bit for bit.
+    """
+    lib = _load()
+    table = np.zeros(D // 2, dtype=np.float32)
+    ms = ctypes.c_float(0.0)
+    flags = np.zeros(D // 2 + 1, dtype=np.int32)
+    rc = lib.orc_rope_table(MODES[mode], D, base, scale, original_max_pos, alpha, beta,
+                            _ptr(table, ctypes.c_float), ctypes.byref(ms), None,
+                            _ptr(flags, ctypes.c_int))
+    if rc:
+        raise ValueError("orc_rope_table: invalid argument")
+    return table, np.float32(ms.value), flags
+
+
+def rotate_rows(x, pos, table, mscale, pairing="half"):
+    """Rotate rows x[n, D] (fp32 values) at integer positions pos[n]; fp64 out."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    n, D = x.shape
+    pos = np.ascontiguousarray(pos, dtype=np.int64)
+    assert pos.shape == (n,)
+    table = np.ascontiguousarray(table, dtype=np.float32)
+    y = np.zeros((n, D), dtype=np.float64)
+    rc = lib.orc_rotate_rows(_ptr(x, ctypes.c_float), _ptr(y, ctypes.c_double), n, D,
+                             _ptr(pos, ctypes.c_int64), _ptr(table, ctypes.c_float),
+                             float(mscale), PAIRINGS[pairing])
+    if rc:
+        raise ValueError("orc_rotate_rows: invalid argument")
+    return y
+
+
+def visible(i, j, L, causal=True, window=0, sinks=0):
+    return bool(_load().orc_visible(i, j, L, int(causal), window, sinks))
+
+
+def mask(L, causal=True, window=0, sinks=0):
+    """[L, L] bool visibility mask (True = key j visible to query i)."""
+    m = np.zeros((L, L), dtype=np.uint8)
+    _load().orc_mask(L, int(causal), window, sinks, _ptr(m, ctypes.c_uint8))
+    return m.astype(bool)
+
+
+def attn_rows(q_rows, row_b, row_h, row_i, k, v, Hq, table, mscale, pairing="half",
+                 pos_offset=0, causal=True, window=0, sinks=0, scale=None, nthreads=0):
+    """Attention output o[n, D] and lse[n] (fp64) for selected query rows.
+
+    q_rows: [n, D] raw (un-rotated) query rows; row_b/row_h/row_i: batch, query
+    head and query index of each row; k, v: [B, Hkv, L, D] raw keys / values
+    (fp32 arrays holding the exact input values); Hq: number of query heads
+    (query head h reads kv head h // (Hq // Hkv)).
+    """
+    lib = _load()
+    q_rows = np.ascontiguousarray(q_rows, dtype=np.float32)
+    k = np.ascontiguousarray(k, dtype=np.float32)
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    row_b = np.ascontiguousarray(row_b, dtype=np.int64)
+    row_h = np.ascontiguousarray(row_h, dtype=np.int64)
+    row_i = np.ascontiguousarray(row_i, dtype=np.int64)
+    return _attn_rows_impl(lib, q_rows, row_b, row_h, row_i, k, v, Hq, table, mscale,
+                           pairing, pos_offset, causal, window, sinks, scale, nthreads)
+
+
+def _attn_rows_impl(lib, q_rows, row_b, row_h, row_i, k, v, Hq, table, mscale, pairing,
+                    pos_offset, causal, window, sinks, scale, nthreads):
+    B, Hkv, L, D = k.shape
+    n = q_rows.shape[0]
+    assert q_rows.shape == (n, D)
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    table = np.ascontiguousarray(table, dtype=np.float32)
+    o = np.zeros((n, D), dtype=np.float64)
+    lse = np.zeros(n, dtype=np.float64)
+    rc = lib.orc_attn_rows(_ptr(q_rows, ctypes.c_float), _ptr(row_b, ctypes.c_int64),
+                           _ptr(row_h, ctypes.c_int64), _ptr(row_i, ctypes.c_int64), n,
+                           _ptr(k, ctypes.c_float), _ptr(v, ctypes.c_float),
+                           B, Hq, Hkv, L, D, _ptr(table, ctypes.c_float), float(mscale),
+                           PAIRINGS[pairing], int(pos_offset), int(causal), int(window),
+                           int(sinks), float(scale), _ptr(o, ctypes.c_double),
+                           _ptr(lse, ctypes.c_double), int(nthreads))
+    if rc:
+        raise ValueError("orc_attn_rows: invalid argument (rc=%d)" % rc)
+    return o, lse
+
+
+def attn_full(q, k, v, table, mscale, pairing="half", pos_offset=0, causal=True,
+              window=0, sinks=0, scale=None, nthreads=0):
+    """All rows: q [B, Hq, L, D], k/v [B, Hkv, L, D] -> o [B, Hq, L, D], lse [B, Hq, L]."""
+    q = np.asarray(q, dtype=np.float32)
+    B, Hq, L, D = q.shape
+    bb, hh, ii = np.meshgrid(np.arange(B), np.arange(Hq), np.arange(L), indexing="ij")
+    o, lse = attn_rows(q.reshape(-1, D), bb.ravel(), hh.ravel(), ii.ravel(), k, v, Hq,
+                          table, mscale, pairing, pos_offset, causal, window, sinks, scale,
+                          nthreads)
+    return o.reshape(B, Hq, L, D), lse.reshape(B, Hq, L)
+
+
+def num_threads(nthreads=0):
+    return int(_load().orc_num_threads(nthreads))
