@@ -1,0 +1,387 @@
+"""Benchmark: fused YaRN-RoPE causal attention prefill on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one pass of the hot path over one batch of the workload: the RoPE
+table for the mode (host) and the fused rotate + QK^T + online softmax + PV
+kernel (lcx_attn_fwd).  Prints ONE JSON line (rank 0).
+
+* value      : attention TFLOP/s, algorithmic FLOPs = 4 * D * (visible query/key
+               pairs) * B * Hq summed over all ranks, divided by the max over ranks
+               of the device time of K steps (CUDA events, inputs resident in HBM).
+* e2e        : the same metric through attn_fwd_host (pinned host q/k/v copied in,
+               o copied out, inside the timed region).
+* roofline   : the attention kernel against the measured dense BF16 peak.
+* cpu_baseline: the fp64 CPU oracle on a bounded sample of the same workload.
+* --impl reference: the oracle alone, as the reference arm (rank 0 only).
+
+Multi-GPU (torchrun): every rank runs an independent replica (its own seeded
+batch) -- the path has no exchange step, so there is no data-path collective and
+scaling is weak.  Inputs are larger than L2 (126 MB), so no flush is needed.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from workloads import HEADLINE, WORKLOADS, attn_flops, make_inputs, rope_bytes, \
+    visible_pairs  # noqa: E402
+
+METRIC = "fused YaRN-RoPE causal attention prefill TFLOP/s and % dense BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic (read + write bytes) of one attention launch on the headline
+# workload from an ncu capture of the current kernel; None until captured.
+ATTN_TRAFFIC_BYTES = None
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        loaded = [s for s in sm if s >= 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ oracle
+def oracle_sample(w, budget_s=15.0, seed=0):
+    """Time the fp64 oracle on a bounded sample of the workload: one (batch, kv
+    head) with its query heads, rows taken from the end of the sequence (the
+    heaviest rows).  Returns (TFLOP/s, seconds, threads, description)."""
+    import oracle
+    g = torch.Generator().manual_seed(seed)
+    L, D = w.L, w.D
+    k = torch.randn((1, 1, L, D), generator=g).to(w.torch_dtype).float().numpy()
+    v = torch.randn((1, 1, L, D), generator=g).to(w.torch_dtype).float().numpy()
+    G = w.Hq // w.Hkv
+    table, ms, _ = oracle.rope_table(w.mode, D, w.base, w.scale, w.original_max_pos,
+                                     w.alpha, w.beta)
+    nthreads = oracle.num_threads(0)
+    scale = w.softmax_scale if w.softmax_scale > 0 else None
+    # calibrate with a few rows, then size the sample to the time budget
+    n_rows = 2 * nthreads
+    while True:
+        rows = np.arange(L - n_rows, L) % L
+        heads = np.arange(n_rows) % G
+        q = torch.randn((n_rows, D), generator=g).to(w.torch_dtype).float().numpy()
+        t0 = time.perf_counter()
+        oracle.attn_rows(q, np.zeros(n_rows), heads, rows, k, v, G, table, ms, w.pairing, 0,
+                         w.causal, w.window, w.sinks, scale, 0)
+        dt = time.perf_counter() - t0
+        flops = sum(4 * D * _row_visible(w, int(i)) for i in rows)
+        if dt >= budget_s / 3 or n_rows >= 1 << 16:
+            break
+        n_rows = int(min(n_rows * max(2.0, budget_s / max(dt, 1e-3) * 0.5), 1 << 16))
+    desc = ("fp64 oracle, 1 kv head of %s: %d query rows (the last %d positions, %d query "
+            "heads) incl. rotating all %d keys" % (w.name, n_rows, n_rows, G, L))
+    return flops / dt / 1e12, dt, nthreads, desc
+
+
+def _row_visible(w, i):
+    if not w.causal:
+        return w.L
+    n = i + 1
+    if w.window > 0 and i - w.window + 1 > 0:
+        lo = i - w.window + 1
+        n = w.window + min(w.sinks, lo)
+    return n
+
+
+# ------------------------------------------------------------------ GPU arm
+def bench_gpu(args, world, rank, local):
+    import ntk_rope_flashattn_b200 as lcx
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    q, k, v = make_inputs(w, device=dev, seed=w.seed + rank)
+    rope = lcx.RopeParams(w.mode, w.D, w.base, w.scale, w.original_max_pos, w.alpha, w.beta,
+                          w.pairing)
+    o = torch.empty_like(q)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    kw = dict(causal=w.causal, window=w.window, sinks=w.sinks, softmax_scale=w.softmax_scale,
+              out=o, status=status)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        lcx.attn_fwd(q, k, v, rope, **kw)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, "device watchdog fired during warm-up"
+
+    # --- device-timed steps (per-launch events on the launching stream)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    total_ms = start.elapsed_time(end)
+    launch_ms = [a.elapsed_time(b) for a, b in evs]
+    assert int(status.item()) == 0, "device watchdog fired"
+    total_ms = max_over_ranks(total_ms, world)
+    flops_rank = attn_flops(w)
+    tflops = flops_rank * world * args.steps / (total_ms * 1e-3) / 1e12
+
+    # --- apply_rope (the unfused rotate-pairs pass) on Q and K, for its own roofline
+    qr, kr = torch.empty_like(q), torch.empty_like(k)
+    for _ in range(3):
+        lcx.apply_rope(q, rope, out=qr)
+        lcx.apply_rope(k, rope, out=kr)
+    torch.cuda.synchronize()
+    rope_ev = []
+    for _ in range(max(3, args.steps)):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        lcx.apply_rope(q, rope, out=qr)
+        lcx.apply_rope(k, rope, out=kr)
+        b.record(stream)
+        rope_ev.append((a, b))
+    torch.cuda.synchronize()
+    rope_ms = statistics.median(a.elapsed_time(b) for a, b in rope_ev)
+    del qr, kr
+
+    # --- end to end through host buffers
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    ws = {}
+    for _ in range(max(1, min(args.warmup, 2))):
+        lcx.attn_fwd_host(qh, kh, vh, rope, device=dev, workspace=ws, causal=w.causal,
+                          window=w.window, sinks=w.sinks, softmax_scale=w.softmax_scale)
+    torch.cuda.synchronize()
+    barrier(world)
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(args.steps):
+        oh = lcx.attn_fwd_host(qh, kh, vh, rope, device=dev, workspace=ws, causal=w.causal,
+                               window=w.window, sinks=w.sinks, softmax_scale=w.softmax_scale)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), world)
+    e2e_tflops = flops_rank * world * args.steps / (e2e_ms * 1e-3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size()
+    del qh, kh, vh, ws
+
+    peaks, peak_src = load_peaks()
+    avg_launch = statistics.mean(launch_ms)
+    achieved = flops_rank / (avg_launch * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops_sustained"])
+    rope_gbs = rope_bytes(w) / (rope_ms * 1e-3) / 1e9
+    res = {
+        "metric": METRIC,
+        "value": round(tflops, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) q/k/v, seed 0 + rank)",
+        "impl": "lcx",
+        "config": {
+            "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D,
+            "rope": w.mode, "scale": w.scale, "original_max_pos": w.original_max_pos,
+            "alpha": w.alpha, "beta": w.beta, "causal": w.causal, "window": w.window,
+            "sinks": w.sinks, "visible_pairs_per_head": visible_pairs(w.L, w.causal, w.window,
+                                                                      w.sinks),
+            "flops_per_step_per_gpu": flops_rank,
+            "l2": "inputs larger than L2 (q+k+v = %.2f GB), no flush" % (
+                sum(t.numel() * t.element_size() for t in (q, k, v)) / 1e9),
+            "parallelism": "replicas x%d (independent batches, no collective)" % world,
+        },
+        "gpu_launches": args.steps,
+        "roofline": {
+            "bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+            "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+            "peak_kind": "bf16_tflops_sustained of %s" % peak_src,
+            "frac_of_burst": round(achieved / float(peaks["bf16_tflops"]), 4),
+            "traffic": ATTN_TRAFFIC_BYTES,
+            "kernel": "attn_fwd_kernel", "avg_launch_ms": round(avg_launch, 3),
+        },
+        "apply_rope": {
+            "bound": "hbm", "bytes": rope_bytes(w), "ms": round(rope_ms, 4),
+            "achieved": round(rope_gbs, 1), "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+            "frac": round(rope_gbs / float(peaks["hbm_gbs"]), 4),
+        },
+        "e2e": {"value": round(e2e_tflops, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "clocks": clk.summary(),
+    }
+    del q, k, v, o
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, secs, cores, desc = oracle_sample(w, budget_s=args.cpu_budget)
+        res["cpu_baseline"] = {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                               "sample": desc, "seconds": round(secs, 2)}
+    return res
+
+
+def bench_reference(args, world, rank):
+    """The reference arm: the fp64 oracle as it stands, on host cores."""
+    if rank != 0:
+        return None
+    w = WORKLOADS[args.workload]
+    vals, secs_all = [], 0.0
+    for s in range(args.warmup + args.steps):
+        val, secs, cores, desc = oracle_sample(w, budget_s=args.cpu_budget / max(1, args.steps),
+                                               seed=s)
+        if s >= args.warmup:
+            vals.append(val)
+            secs_all += secs
+    value = statistics.mean(vals)
+    return {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs_all / args.steps * 1e3, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "impl": "reference",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D,
+                   "rope": w.mode},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="lcx", choices=["lcx", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        res = bench_reference(args, world, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        res = bench_gpu(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,183 @@
+/*
+ * lcx.h -- C ABI of the long-context RoPE + causal attention prefill library
+ * (liblcx.so, sm_100a).
+ *
+ * Three calls make up the hot path:
+ *   lcx_rope_table  per-pair RoPE frequencies theta'_i and the attention scale
+ *                   for plain RoPE, Position Interpolation, NTK-aware base
+ *                   scaling and YaRN (NTK-by-parts ramp + 0.1 ln s + 1).
+ *   lcx_apply_rope  the memory-bound rotate-pairs pass over a Q or K tensor.
+ *   lcx_attn_fwd    blockwise online-softmax causal attention prefill that
+ *                   rotates Q/K tiles on chip, with GQA, an optional sliding
+ *                   window and attention sinks.
+ *
+ * Sources (page title, section):
+ *   [LC]  "Long Context: RoPE / YaRN / NTK / MLA" (mathieu0905.github.io):
+ *         2.1-2.4 RoPE and rope_attention, 4.2 PI, 5.2 NTK-aware base,
+ *         6.2-6.6 YaRN, 10.1 sliding window, 10.2 attention sinks.
+ *   [B83] "8.3 长上下文技术" (paper.xwysyy.cn llm-fullstack-book): 8.3.1-8.3.3
+ *         frequencies, PI, NTK-aware, NTK-by-parts, YaRN recipe; 8.3.4
+ *         FlashAttention tiling and online softmax.
+ *
+ * Conventions shared by every call:
+ *   - Ownership: the caller owns every buffer.  The library allocates no device
+ *     memory, keeps no state besides a per-thread last-error string, and never
+ *     synchronises a stream.  Device work is enqueued on `stream` (a
+ *     cudaStream_t passed as void*; NULL = the legacy default stream).
+ *   - Tensors are [B, H, L, D] with element strides given per dimension; the
+ *     last dimension must be contiguous (stride 1).  Pointers and strides must
+ *     keep every row 16-byte aligned.
+ *   - Errors: argument problems are detected on the host before any device
+ *     work and return LCX_ERR_INVALID_ARG (malformed) or LCX_ERR_UNSUPPORTED
+ *     (well-formed but outside what the kernels implement).  A failed launch
+ *     returns LCX_ERR_CUDA.  lcx_last_error() describes the last failure on
+ *     the calling thread.  Device-side watchdog expiries are reported through
+ *     the optional device status word of lcx_attn_fwd.
+ *   - Thread safety: every call is reentrant.
+ */
+#ifndef LCX_H
+#define LCX_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LCX_VERSION 100
+
+#if defined(__GNUC__)
+#define LCX_API __attribute__((visibility("default")))
+#else
+#define LCX_API
+#endif
+
+typedef enum {
+    LCX_OK = 0,
+    LCX_ERR_INVALID_ARG = 1,
+    LCX_ERR_UNSUPPORTED = 2,
+    LCX_ERR_CUDA = 3,
+    LCX_ERR_TIMEOUT = 4
+} lcx_status;
+
+/* Frequency-scaling modes ([LC] 2.3, 4.2, 5.2, 6.2; [B83] 8.3.2-8.3.3).
+ * NONE leaves vectors unrotated (theta' = 0) and is meant for testing. */
+typedef enum {
+    LCX_ROPE_NONE = 0,
+    LCX_ROPE_PLAIN = 1,   /* theta'_i = b^(-2i/D)                              */
+    LCX_ROPE_PI = 2,      /* theta'_i = theta_i / s  (positions m -> m/s)      */
+    LCX_ROPE_NTK = 3,     /* theta'_i = (b s^(D/(D-2)))^(-2i/D)                */
+    LCX_ROPE_YARN = 4     /* theta'_i = theta_i ((1-g_i)/s + g_i), g_i = clip((r_i-alpha)/(beta-alpha),0,1),
+                             r_i = L_train theta_i / (2 pi); mscale = 0.1 ln s + 1 (s > 1) */
+} lcx_rope_mode;
+
+/* Which dimensions form a rotated pair ([LC] 2.4): HALF pairs (i, i + D/2)
+ * (HuggingFace halves), INTERLEAVED pairs (2i, 2i + 1) (adjacent, [LC] 2.1). */
+typedef enum { LCX_PAIR_HALF = 0, LCX_PAIR_INTERLEAVED = 1 } lcx_pairing;
+
+typedef enum { LCX_BF16 = 0, LCX_F32 = 1 } lcx_dtype;
+
+typedef struct {
+    int32_t mode;              /* lcx_rope_mode                                  */
+    int32_t head_dim;          /* D: even, 2..512                                */
+    int32_t pairing;           /* lcx_pairing                                    */
+    int32_t reserved;          /* must be 0                                      */
+    double base;               /* b > 1 (10000 in the pages)                     */
+    double scale;              /* s = L_new / L_train > 0 (PI, NTK, YARN)        */
+    int64_t original_max_pos;  /* L_train > 0 (YARN)                             */
+    double alpha;              /* YARN ramp lower bound in turns (default 1)     */
+    double beta;               /* YARN ramp upper bound in turns (default 32)    */
+} lcx_rope_params;
+
+/*
+ * lcx_rope_table -- the per-pair frequencies of a mode, rounded once from fp64
+ * to fp32 (nearest even), and the attention scale sqrt(1/t).
+ *   Defines: [LC] 2.4 (theta_i = b^(-2i/D)), 4.2 (PI), 5.2 (NTK-aware base),
+ *            6.2 (NTK-by-parts ramp), 6.3/6.6 (sqrt(1/t) = 0.1 ln s + 1);
+ *            [B83] 8.3.3 five-step YaRN recipe.
+ *   inv_freq: HOST array of head_dim/2 floats, written on success.
+ *   mscale  : HOST float, written on success (1 unless YARN with s > 1).
+ *   Host-only; touches no GPU.  Returns LCX_OK or LCX_ERR_INVALID_ARG.
+ */
+LCX_API lcx_status lcx_rope_table(const lcx_rope_params *params, float *inv_freq, float *mscale);
+
+/*
+ * lcx_apply_rope -- rotate every pair of x by m * theta'_i and multiply by
+ * mscale: (x_p, x_q) -> ms (x_p cos - x_q sin, x_p sin + x_q cos), with
+ * m = pos_offset + l for sequence index l.
+ *   Defines: [LC] 2.2 (rotation matrix), 2.4 apply_rope, 6.4 (mscale folded
+ *            into cos/sin); [B83] 8.3.3 step 4-5.
+ *   x, y      : DEVICE pointers to [B, H, L, D] tensors of `dtype`; y may equal
+ *               x (in place; then the strides must match).  16-byte aligned.
+ *   x_strides : element strides of x for (B, H, L, D); D's stride must be 1.
+ *   y_strides : element strides of y, or NULL for "same as x".
+ *   Angles are evaluated from the exact product m * theta'_i (fp64), so the
+ *   result is accurate for positions up to 2^31.
+ *   Supported: head_dim % 16 == 0, head_dim <= 512, strides multiples of 16
+ *   bytes.  Enqueued on `stream`; returns before the work completes.
+ */
+LCX_API lcx_status lcx_apply_rope(const lcx_rope_params *params, const void *x, void *y, int32_t dtype,
+                          int64_t B, int64_t H, int64_t L, const int64_t *x_strides,
+                          const int64_t *y_strides, int64_t pos_offset, void *stream);
+
+/* lcx_attn_args.flags */
+#define LCX_ATTN_PREROTATED 1u  /* q and k already hold rotated vectors (e.g. from
+                                   lcx_apply_rope with the same params, mscale
+                                   included): skip the on-chip rotation and the
+                                   mscale^2 factor on the logits.             */
+
+typedef struct {
+    const void *q;             /* DEVICE [B, Hq, L, D]                            */
+    const void *k;             /* DEVICE [B, Hkv, L, D]                           */
+    const void *v;             /* DEVICE [B, Hkv, L, D]                           */
+    void *o;                   /* DEVICE [B, Hq, L, D], same dtype as q           */
+    float *lse;                /* DEVICE [B, Hq, L] fp32 natural-log sum-exp of the
+                                  scaled logits, or NULL                          */
+    int32_t *dev_status;       /* DEVICE int32 or NULL: set to LCX_ERR_TIMEOUT by a
+                                  kernel whose bounded wait expired; never cleared */
+    int32_t dtype;             /* lcx_dtype of q, k, v, o                         */
+    int32_t causal;            /* 1 = key j visible to query i only if j <= i    */
+    int64_t B, Hq, Hkv, L, D;  /* Hq % Hkv == 0; D in {64, 128}                   */
+    int64_t q_strides[4], k_strides[4], v_strides[4], o_strides[4];  /* elements  */
+    lcx_rope_params rope;      /* head_dim must equal D                           */
+    int64_t window;            /* W > 0: key j visible only if i - j < W (W counts
+                                  the query itself); 0 = no window.  Needs causal */
+    int64_t sinks;             /* S: keys j < S stay visible to every i >= j when
+                                  a window is set; 0 = none                       */
+    float softmax_scale;       /* logit scale; 0 -> 1/sqrt(D)                     */
+    uint32_t flags;            /* LCX_ATTN_* bits                                 */
+} lcx_attn_args;
+
+/*
+ * lcx_attn_fwd -- o_i = sum_j softmax_j(c <q'_i, k'_j>) v_j over the visible
+ * keys, q' and k' the RoPE-rotated vectors times mscale, c = softmax_scale;
+ * query head h reads kv head h / (Hq / Hkv) (GQA).
+ *   Defines: [LC] 2.4 rope_attention (rotate, QK^T / sqrt(d), mask, softmax,
+ *            times V), 6.3-6.4 (temperature via mscale on q and k), 10.1
+ *            sliding window, 10.2 sinks; [B83] 8.3.4 (blockwise tiling with an
+ *            exact online softmax), 8.3.3 (YaRN attention scaling).
+ *   Visibility in prefill (queries and keys share positions 0..L-1): j <= i if
+ *   causal; with W > 0 also i - j < W or j < S.  Rows with no visible key get
+ *   o = 0 and lse = -inf.
+ *   Arithmetic: q', k' rounded to bf16 on chip, QK^T and PV on bf16 tensor
+ *   cores with fp32 accumulation, softmax statistics in fp32, o rounded once
+ *   to the output dtype.  fp32 inputs are rounded to bf16 operands.
+ *   Supported: D in {64, 128}; bf16 or fp32; pointers 16-byte aligned, strides
+ *   multiples of 16 bytes, D's stride 1.  Enqueued on `stream`.
+ */
+LCX_API lcx_status lcx_attn_fwd(const lcx_attn_args *args, void *stream);
+
+/* Static description of a status code. */
+LCX_API const char *lcx_status_string(lcx_status status);
+
+/* Description of the last failure on the calling thread ("" if none). */
+LCX_API const char *lcx_last_error(void);
+
+/* LCX_VERSION of the built library. */
+LCX_API int32_t lcx_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LCX_H */

@@ -1,0 +1,247 @@
+"""ntk_rope_flashattn_b200 -- RoPE context extension fused into causal attention
+prefill on B200 (sm_100a).
+
+Python binding of the C-ABI library ``liblcx.so`` (see ``include/lcx.h``).  It
+only marshals arguments: tensors stay PyTorch tensors (device memory and the
+current stream come from torch), and every step of the computation runs in the
+library's CUDA kernels.  If the library is missing the calls raise; there is no
+fallback implementation.
+
+    import torch, ntk_rope_flashattn_b200 as lcx
+    rope = lcx.RopeParams("yarn", head_dim=128, scale=16, original_max_pos=8192)
+    o = lcx.attn_fwd(q, k, v, rope, causal=True)          # q, k, v: [B, H, L, D]
+"""
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblcx.so")
+
+LCX_OK, LCX_ERR_INVALID_ARG, LCX_ERR_UNSUPPORTED, LCX_ERR_CUDA, LCX_ERR_TIMEOUT = range(5)
+MODES = {"none": 0, "plain": 1, "pi": 2, "ntk": 3, "yarn": 4}
+PAIRINGS = {"half": 0, "interleaved": 1}
+DTYPES = {"bf16": 0, "f32": 1}
+LCX_ATTN_PREROTATED = 1
+
+# Symbols include/lcx.h declares; the library must export every one of them.
+EXPORTED = ("lcx_rope_table", "lcx_apply_rope", "lcx_attn_fwd", "lcx_status_string",
+            "lcx_last_error", "lcx_version")
+
+
+class LcxError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__("%s (status %d): %s" % (STATUS_NAMES.get(status, "?"), status, msg))
+        self.status = status
+
+
+STATUS_NAMES = {0: "LCX_OK", 1: "LCX_ERR_INVALID_ARG", 2: "LCX_ERR_UNSUPPORTED",
+                3: "LCX_ERR_CUDA", 4: "LCX_ERR_TIMEOUT"}
+
+
+class _RopeParams(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("pairing", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("base", ctypes.c_double), ("scale", ctypes.c_double),
+                ("original_max_pos", ctypes.c_int64), ("alpha", ctypes.c_double),
+                ("beta", ctypes.c_double)]
+
+
+class _AttnArgs(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+                ("dev_status", ctypes.c_void_p), ("dtype", ctypes.c_int32),
+                ("causal", ctypes.c_int32), ("B", ctypes.c_int64), ("Hq", ctypes.c_int64),
+                ("Hkv", ctypes.c_int64), ("L", ctypes.c_int64), ("D", ctypes.c_int64),
+                ("q_strides", ctypes.c_int64 * 4), ("k_strides", ctypes.c_int64 * 4),
+                ("v_strides", ctypes.c_int64 * 4), ("o_strides", ctypes.c_int64 * 4),
+                ("rope", _RopeParams), ("window", ctypes.c_int64), ("sinks", ctypes.c_int64),
+                ("softmax_scale", ctypes.c_float), ("flags", ctypes.c_uint32)]
+
+
+@dataclass
+class RopeParams:
+    """RoPE frequency scaling (mirrors ``lcx_rope_params``)."""
+    mode: str = "plain"
+    head_dim: int = 128
+    base: float = 10000.0
+    scale: float = 1.0
+    original_max_pos: int = 4096
+    alpha: float = 1.0
+    beta: float = 32.0
+    pairing: str = "half"
+
+    @classmethod
+    def from_hf(cls, cfg: dict, head_dim: int):
+        """From a HuggingFace-style ``rope_scaling`` dict plus ``rope_theta``
+        (keys: type/rope_type, factor, original_max_position_embeddings,
+        beta_slow -> alpha, beta_fast -> beta, rope_theta)."""
+        kind = cfg.get("rope_type", cfg.get("type", "default"))
+        mode = {"default": "plain", "linear": "pi", "dynamic": "ntk", "ntk": "ntk",
+                "yarn": "yarn"}.get(kind, kind)
+        return cls(mode=mode, head_dim=head_dim, base=float(cfg.get("rope_theta", 10000.0)),
+                   scale=float(cfg.get("factor", 1.0)),
+                   original_max_pos=int(cfg.get("original_max_position_embeddings", 4096)),
+                   alpha=float(cfg.get("beta_slow", 1.0)), beta=float(cfg.get("beta_fast", 32.0)))
+
+    def _c(self):
+        return _RopeParams(MODES[self.mode], int(self.head_dim), PAIRINGS[self.pairing], 0,
+                           float(self.base), float(self.scale), int(self.original_max_pos),
+                           float(self.alpha), float(self.beta))
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load liblcx.so (built by ``python -m ntk_rope_flashattn_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError("liblcx.so not found at %s: build it with "
+                           "`python -m ntk_rope_flashattn_b200.build`" % path)
+    lib = ctypes.CDLL(path)
+    lib.lcx_rope_table.argtypes = [ctypes.POINTER(_RopeParams), ctypes.POINTER(ctypes.c_float),
+                                   ctypes.POINTER(ctypes.c_float)]
+    lib.lcx_rope_table.restype = ctypes.c_int
+    lib.lcx_apply_rope.argtypes = [ctypes.POINTER(_RopeParams), ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_int32, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                   ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64),
+                                   ctypes.c_int64, ctypes.c_void_p]
+    lib.lcx_apply_rope.restype = ctypes.c_int
+    lib.lcx_attn_fwd.argtypes = [ctypes.POINTER(_AttnArgs), ctypes.c_void_p]
+    lib.lcx_attn_fwd.restype = ctypes.c_int
+    lib.lcx_status_string.argtypes = [ctypes.c_int]
+    lib.lcx_status_string.restype = ctypes.c_char_p
+    lib.lcx_last_error.argtypes = []
+    lib.lcx_last_error.restype = ctypes.c_char_p
+    lib.lcx_version.argtypes = []
+    lib.lcx_version.restype = ctypes.c_int32
+    _lib = lib
+    return lib
+
+
+def _check(st):
+    if st != LCX_OK:
+        raise LcxError(st, load().lcx_last_error().decode())
+
+
+def version() -> int:
+    return int(load().lcx_version())
+
+
+def rope_table(rope: RopeParams):
+    """(theta' float32[head_dim/2], mscale float32) from ``lcx_rope_table``."""
+    lib = load()
+    out = np.zeros(rope.head_dim // 2, dtype=np.float32)
+    ms = ctypes.c_float(0.0)
+    p = rope._c()
+    _check(lib.lcx_rope_table(ctypes.byref(p), out.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),
+                              ctypes.byref(ms)))
+    return out, np.float32(ms.value)
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return DTYPES["bf16"]
+    if t.dtype == torch.float32:
+        return DTYPES["f32"]
+    raise TypeError("unsupported dtype %s (bf16 or fp32)" % t.dtype)
+
+
+def _strides(t):
+    return (ctypes.c_int64 * 4)(*[int(s) for s in t.stride()])
+
+
+def _stream(t):
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def apply_rope(x, rope: RopeParams, out=None, pos_offset: int = 0, inplace: bool = False):
+    """Rotate x [B, H, L, D] (bf16/fp32, CUDA) by positions pos_offset + l."""
+    import torch
+    if x.dim() != 4 or not x.is_cuda:
+        raise ValueError("x must be a 4-D CUDA tensor [B, H, L, D]")
+    y = x if inplace else (out if out is not None else torch.empty_like(x))
+    B, H, L, D = x.shape
+    if D != rope.head_dim:
+        raise ValueError("x head_dim %d != rope.head_dim %d" % (D, rope.head_dim))
+    p = rope._c()
+    _check(load().lcx_apply_rope(ctypes.byref(p), ctypes.c_void_p(x.data_ptr()),
+                                 ctypes.c_void_p(y.data_ptr()), _dtype_code(x), B, H, L,
+                                 _strides(x), _strides(y), int(pos_offset), _stream(x)))
+    return y
+
+
+def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, sinks: int = 0,
+             softmax_scale: float = 0.0, return_lse: bool = False, prerotated: bool = False,
+             out=None, lse=None, status=None):
+    """Fused RoPE + causal attention prefill.
+
+    q [B, Hq, L, D], k/v [B, Hkv, L, D] CUDA tensors (bf16 or fp32, last dim
+    contiguous).  Returns o [B, Hq, L, D] (and lse [B, Hq, L] fp32 if asked).
+    ``status`` (optional int32 CUDA tensor of one element) receives
+    LCX_ERR_TIMEOUT if a kernel's bounded wait expired.
+    """
+    import torch
+    for t in (q, k, v):
+        if t.dim() != 4 or not t.is_cuda:
+            raise ValueError("q, k, v must be 4-D CUDA tensors [B, H, L, D]")
+    B, Hq, L, D = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, L, D) or v.shape != k.shape:
+        raise ValueError("shape mismatch: q %s k %s v %s" % (q.shape, k.shape, v.shape))
+    if not (q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must share a dtype")
+    o = out if out is not None else torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
+    a = _AttnArgs()
+    a.q, a.k, a.v, a.o = q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr()
+    a.lse = lse.data_ptr() if lse is not None else None
+    a.dev_status = status.data_ptr() if status is not None else None
+    a.dtype = _dtype_code(q)
+    a.causal = 1 if causal else 0
+    a.B, a.Hq, a.Hkv, a.L, a.D = B, Hq, Hkv, L, D
+    a.q_strides, a.k_strides, a.v_strides, a.o_strides = (_strides(q), _strides(k),
+                                                          _strides(v), _strides(o))
+    a.rope = rope._c()
+    a.window, a.sinks = int(window), int(sinks)
+    a.softmax_scale = float(softmax_scale)
+    a.flags = LCX_ATTN_PREROTATED if prerotated else 0
+    _check(load().lcx_attn_fwd(ctypes.byref(a), _stream(q)))
+    return (o, lse) if return_lse else o
+
+
+def attn_fwd_host(q, k, v, rope: RopeParams, device="cuda", workspace=None, **kw):
+    """attn_fwd on HOST tensors: copies q/k/v to the device (pinned memory makes
+    the copies asynchronous), runs the kernel and copies o back to the host.
+
+    ``workspace`` (dict) keeps the device buffers between calls.
+    """
+    import torch
+    ws = workspace if workspace is not None else {}
+    dev = {}
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        buf = ws.get(name)
+        if buf is None or buf.shape != t.shape or buf.dtype != t.dtype:
+            buf = torch.empty(t.shape, dtype=t.dtype, device=device)
+            ws[name] = buf
+        buf.copy_(t, non_blocking=True)
+        dev[name] = buf
+    o_dev = ws.get("o")
+    if o_dev is None or o_dev.shape != q.shape or o_dev.dtype != q.dtype:
+        o_dev = torch.empty(q.shape, dtype=q.dtype, device=device)
+        ws["o"] = o_dev
+    attn_fwd(dev["q"], dev["k"], dev["v"], rope, out=o_dev, **kw)
+    o_host = ws.get("o_host")
+    if o_host is None or o_host.shape != q.shape or o_host.dtype != q.dtype:
+        o_host = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        ws["o_host"] = o_host
+    o_host.copy_(o_dev, non_blocking=True)
+    return o_host

@@ -1,0 +1,845 @@
+// attn_fwd.cu -- fused RoPE + blockwise online-softmax causal attention prefill
+// on sm_100a tensor cores (lcx_attn_fwd).
+//
+// What it computes ("Long Context: RoPE / YaRN / NTK / MLA", section 2.4
+// rope_attention with the masks of 10.1/10.2 and the YaRN scale of 6.3-6.4):
+//   o_i = sum_j softmax_j(c <q'_i, k'_j>) v_j over visible keys j,
+// q', k' the rotated vectors (times mscale).  The blockwise evaluation with a
+// running max and sum is the exact online softmax of "8.3 长上下文技术",
+// section 8.3.4.
+//
+// Design (one CTA per work unit, 14 warps):
+//   unit      = (batch b, two query heads of one GQA group, 128 query rows);
+//               both query tiles read the same K/V tiles, so each K tile is
+//               loaded and rotated once for 256 query rows.
+//   warp 12   TMA producer: Q tiles once, then K/V tiles into a ring of stages.
+//   warps 8-11 rotation warpgroup: rotates the Q tiles and every K tile in
+//               shared memory (bf16 -> fp32 -> rotate -> bf16) right after the
+//               TMA lands, then hands the tile to the tensor core.
+//   warp 13   MMA issuer: S_t = Q_t K^T (tcgen05.mma, fp32 accumulators in
+//               TMEM), then O_t += P_t V with P_t read from TMEM.  The two
+//               query tiles ping-pong so one tile's softmax overlaps the other
+//               tile's matrix products.
+//   warps 0-3 / 4-7  softmax for query tile 0 / 1: one thread per query row
+//               reads its S row from TMEM, masks partial tiles, keeps the
+//               running max/sum, writes P (bf16) back over S, rescales its O
+//               row only when the max grew by more than 2^8, and finally
+//               normalises O and stores it.
+// Tiles entirely hidden by the causal/window mask are never visited; tiles
+// entirely visible skip the per-element mask.  Every barrier wait is bounded
+// (wall-clock timeout); on expiry the CTA winds down, releases TMEM and
+// reports LCX_ERR_TIMEOUT through the optional status word.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+
+#include "lcx_internal.h"
+#include "rope_angle.cuh"
+#include "sm100.cuh"
+
+namespace lcx {
+namespace {
+
+constexpr int kThreads = 448;           // 14 warps
+constexpr int kBM = 128;                // query rows per tile
+constexpr int kBN = 128;                // keys per tile
+constexpr int kBoxBytes = 128 * 128;    // one TMA box: 128 rows x 128 bytes
+constexpr float kRescaleLog2 = 8.0f;    // rescale O only if the max grows by > 2^8
+constexpr int kWarpMma = 13;
+constexpr int kWarpTma = 12;
+constexpr int kWarpRot0 = 8;
+
+struct AttnParams {
+    const char *q, *k, *v;             // raw pointers (fp32 operands path)
+    char *o;
+    float *lse;
+    int *status;
+    long long qs[3], ks[3], vs[3], os[3];  // element strides of B, H, L
+    int B, Hq, Hkv, L, G;
+    int causal, window, sinks;
+    int n_qb, heads_per_unit, units_per_qb;
+    int rotate;
+    float c_log2;                      // logit scale in log2 units
+    unsigned long long timeout_ns;
+    float theta[64];
+};
+
+template <int D>
+struct Cfg {
+    static constexpr int kTile = kBM * D * 2;  // bytes of a 128 x D bf16 tile
+    static constexpr int kStages = (D == 128) ? 2 : 4;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = 2 * kTile;
+    static constexpr int kOffV = kOffK + kStages * kTile;
+    static constexpr int kOffBar = kOffV + kStages * kTile;
+    static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers + alignment slack
+};
+
+template <int NS>
+struct Bars {
+    uint64_t full_q, ready_q;
+    uint64_t full_k[NS], ready_k[NS], empty_k[NS];
+    uint64_t full_v[NS], empty_v[NS];
+    uint64_t s_ready[2], p_ready[2], o_ready[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// ---------------------------------------------------------------- schedule
+struct Unit {
+    int b, g, hq0, nt, q0;
+};
+
+// Work units are numbered heaviest first (query blocks from the end of the
+// sequence, which see the most keys), so the block scheduler hands out the
+// longest units first.
+__device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
+    const int u = blockIdx.x;
+    const int hu = u % p.units_per_qb;
+    const int qb = p.n_qb - 1 - u / p.units_per_qb;
+    Unit r;
+    r.q0 = qb * kBM;
+    r.nt = p.heads_per_unit;
+    const int per_b = p.units_per_qb / p.B;
+    r.b = hu / per_b;
+    const int rem = hu % per_b;
+    if (p.heads_per_unit == 2) {
+        const int ppg = p.G / 2;
+        r.g = rem / ppg;
+        r.hq0 = r.g * p.G + 2 * (rem % ppg);
+    } else {
+        r.hq0 = rem;
+        r.g = rem / p.G;
+    }
+    return r;
+}
+
+// K tiles a query block visits: the sink tiles [0, ns) then the window tiles
+// [jlo, jhi]; every listed tile has at least one visible key.
+struct Tiles {
+    int ns, jlo, n;
+    __device__ __forceinline__ int tile(int j) const { return j < ns ? j : jlo + (j - ns); }
+};
+
+__device__ __forceinline__ Tiles make_tiles(int q0, const AttnParams &p) {
+    const int i1 = min(q0 + kBM - 1, p.L - 1);
+    const int jhi = p.causal ? i1 / kBN : (p.L - 1) / kBN;
+    int jlo = 0, ns = 0;
+    if (p.causal && p.window > 0) {
+        jlo = max(0, q0 - p.window + 1) / kBN;
+        if (p.sinks > 0) ns = min((p.sinks + kBN - 1) / kBN, jlo);
+    }
+    Tiles t;
+    t.ns = ns;
+    t.jlo = jlo;
+    t.n = ns + (jhi - jlo + 1);
+    return t;
+}
+
+// True when every (query row of the block, key of the tile) pair is visible.
+__device__ __forceinline__ bool tile_full(int q0, int jt, const AttnParams &p) {
+    const int j0 = jt * kBN, j1 = j0 + kBN - 1;
+    const int i0 = q0, i1 = q0 + kBM - 1;
+    if (j1 > p.L - 1) return false;
+    if (!p.causal) return true;
+    if (j1 > i0) return false;
+    if (p.window > 0 && !(j0 >= i1 - p.window + 1 || j1 < p.sinks)) return false;
+    return true;
+}
+
+// ---------------------------------------------------------------- smem tiles
+// A 128 x D bf16 tile is stored as D/64 TMA boxes of 128 rows x 128 bytes with
+// the 128-byte swizzle: the 16-byte chunk c of row r sits at chunk c ^ (r & 7).
+__device__ __forceinline__ uint32_t chunk_off(int r, int fc) {
+    return (fc >> 3) * kBoxBytes + r * 128 + (((fc & 7) ^ (r & 7)) << 4);
+}
+
+template <int D, bool kHalf>
+struct Rot {
+    static constexpr int CPR = kHalf ? D / 16 : D / 8;  // jobs per row
+    static constexpr int RP = 128 / CPR;                 // rows per pass of the WG
+    static constexpr int NJ = 128 / RP;                  // jobs per thread
+    static constexpr int PPJ = kHalf ? 8 : 4;            // pairs per job
+};
+
+// Rotate one job's pairs: x1/x2 are the pair members, (c, s) the phasor.
+template <int N>
+__device__ __forceinline__ void rot_pairs(float (&x1)[N], float (&x2)[N], const float *c,
+                                          const float *s) {
+#pragma unroll
+    for (int e = 0; e < N; ++e) {
+        const float a = x1[e], b = x2[e];
+        x1[e] = fmaf(a, c[e], -b * s[e]);
+        x2[e] = fmaf(a, s[e], b * c[e]);
+    }
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &v, float (&x)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        x[2 * k] = bf16lo_to_f32(w[k]);
+        x[2 * k + 1] = bf16hi_to_f32(w[k]);
+    }
+}
+__device__ __forceinline__ uint4 pack8(const float (&y)[8]) {
+    return make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
+                      pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
+}
+
+// Per-thread phasor state of the rotation warpgroup: the thread always handles
+// the same pairs i0..i0+PPJ-1 and rows r0 + RP k, so it starts each tile at
+// e^{i (pos0 + r0) theta} and steps by e^{i RP theta}.
+template <int D, bool kHalf>
+struct Phasor {
+    using R = Rot<D, kHalf>;
+    float sc[R::PPJ], ss[R::PPJ];  // step
+    int q, r0, i0;
+    __device__ __forceinline__ void init(int tw, const AttnParams &p) {
+        q = tw % R::CPR;
+        r0 = tw / R::CPR;
+        i0 = q * R::PPJ;
+#pragma unroll
+        for (int e = 0; e < R::PPJ; ++e) rope_sincos(R::RP, p.theta[i0 + e], &sc[e], &ss[e]);
+    }
+    __device__ __forceinline__ void start(long long pos0, const AttnParams &p, float (&c)[R::PPJ],
+                                          float (&s)[R::PPJ]) const {
+#pragma unroll
+        for (int e = 0; e < R::PPJ; ++e) rope_sincos_fast(pos0 + r0, p.theta[i0 + e], &c[e], &s[e]);
+    }
+    __device__ __forceinline__ void step(float (&c)[R::PPJ], float (&s)[R::PPJ]) const {
+#pragma unroll
+        for (int e = 0; e < R::PPJ; ++e) {
+            const float nc = fmaf(c[e], sc[e], -s[e] * ss[e]);
+            const float ns = fmaf(c[e], ss[e], s[e] * sc[e]);
+            c[e] = nc;
+            s[e] = ns;
+        }
+    }
+};
+
+// Rotate a bf16 tile in place (rows at positions pos0 + r).
+template <int D, bool kHalf>
+__device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, long long pos0,
+                                                 const Phasor<D, kHalf> &ph,
+                                                 const AttnParams &p) {
+    using R = Rot<D, kHalf>;
+    float c[R::PPJ], s[R::PPJ];
+    ph.start(pos0, p, c, s);
+#pragma unroll 2
+    for (int k = 0; k < R::NJ; ++k) {
+        const int r = ph.r0 + k * R::RP;
+        if (kHalf) {
+            uint4 *pa = reinterpret_cast<uint4 *>(tile + chunk_off(r, ph.q));
+            uint4 *pb = reinterpret_cast<uint4 *>(tile + chunk_off(r, ph.q + D / 16));
+            float x1[8], x2[8];
+            unpack8(*pa, x1);
+            unpack8(*pb, x2);
+            rot_pairs<8>(x1, x2, c, s);
+            *pa = pack8(x1);
+            *pb = pack8(x2);
+        } else {
+            uint4 *pa = reinterpret_cast<uint4 *>(tile + chunk_off(r, ph.q));
+            float x[8];
+            unpack8(*pa, x);
+            float x1[4], x2[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                x1[e] = x[2 * e];
+                x2[e] = x[2 * e + 1];
+            }
+            rot_pairs<4>(x1, x2, c, s);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                x[2 * e] = x1[e];
+                x[2 * e + 1] = x2[e];
+            }
+            *pa = pack8(x);
+        }
+        ph.step(c, s);
+    }
+}
+
+// fp32 operands: load 128 rows from global (rows >= L read as zero), rotate in
+// fp32 when asked, round to bf16 into the swizzled tile.
+template <int D, bool kHalf>
+__device__ __forceinline__ void load_tile_f32(uint8_t *tile, const float *base, long long rs,
+                                              int row0, int L, bool rotate,
+                                              const Phasor<D, kHalf> &ph, const AttnParams &p) {
+    using R = Rot<D, kHalf>;
+    float c[R::PPJ], s[R::PPJ];
+    if (rotate) ph.start(row0, p, c, s);
+    for (int k = 0; k < R::NJ; ++k) {
+        const int r = ph.r0 + k * R::RP;
+        const bool valid = row0 + r < L;
+        const float *src = base + (long long)(row0 + r) * rs;
+        if (kHalf) {
+            float x1[8], x2[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                x1[e] = valid ? src[ph.i0 + e] : 0.f;
+                x2[e] = valid ? src[ph.i0 + e + D / 2] : 0.f;
+            }
+            if (rotate) rot_pairs<8>(x1, x2, c, s);
+            *reinterpret_cast<uint4 *>(tile + chunk_off(r, ph.q)) = pack8(x1);
+            *reinterpret_cast<uint4 *>(tile + chunk_off(r, ph.q + D / 16)) = pack8(x2);
+        } else {
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = valid ? src[8 * ph.q + e] : 0.f;
+            if (rotate) {
+                float x1[4], x2[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    x1[e] = x[2 * e];
+                    x2[e] = x[2 * e + 1];
+                }
+                rot_pairs<4>(x1, x2, c, s);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    x[2 * e] = x1[e];
+                    x[2 * e + 1] = x2[e];
+                }
+            }
+            *reinterpret_cast<uint4 *>(tile + chunk_off(r, ph.q)) = pack8(x);
+        }
+        if (rotate) ph.step(c, s);
+    }
+}
+
+// fp32 V tile: convert only.
+template <int D>
+__device__ __forceinline__ void load_v_f32(uint8_t *tile, const float *base, long long rs, int row0,
+                                           int L, int tw) {
+    constexpr int CPR = D / 8;
+    for (int idx = tw; idx < kBN * CPR; idx += 128) {
+        const int r = idx / CPR, fc = idx % CPR;
+        const bool valid = row0 + r < L;
+        const float *src = base + (long long)(row0 + r) * rs + fc * 8;
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = valid ? src[e] : 0.f;
+        *reinterpret_cast<uint4 *>(tile + chunk_off(r, fc)) = pack8(x);
+    }
+}
+
+// ---------------------------------------------------------------- kernel
+template <int D, bool kF32, bool kHalf>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq,
+                    const __grid_constant__ CUtensorMap tmk,
+                    const __grid_constant__ CUtensorMap tmv, const __grid_constant__ AttnParams p) {
+    using C = Cfg<D>;
+    constexpr int NS = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = smem + C::kOffQ;
+    uint8_t *sK = smem + C::kOffK;
+    uint8_t *sV = smem + C::kOffV;
+    Bars<NS> &bar = *reinterpret_cast<Bars<NS> *>(smem + C::kOffBar);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const Unit U = decode_unit(p);
+    const Tiles T = make_tiles(U.q0, p);
+    volatile int *abort = &bar.abort;
+    const uint64_t tmo = p.timeout_ns;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bar.full_q, 1);
+        mbar_init(&bar.ready_q, 128);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&bar.full_k[s], 1);
+            mbar_init(&bar.ready_k[s], 128);
+            mbar_init(&bar.empty_k[s], 1);
+            mbar_init(&bar.full_v[s], kF32 ? 128 : 1);
+            mbar_init(&bar.empty_v[s], 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&bar.s_ready[t], 1);
+            mbar_init(&bar.p_ready[t], 128);
+            mbar_init(&bar.o_ready[t], 1);
+        }
+        mbar_init(&bar.drain, 1);
+        // A CTA that starts after another one's watchdog fired does no work.
+        bar.abort = p.status ? *reinterpret_cast<volatile int *>(p.status) : 0;
+        fence_mbar_init();
+    }
+    if (warp == kWarpMma) {
+        tmem_alloc(&bar.tmem_base, 512);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bar.tmem_base;
+    const bool skip = bar.abort != 0;
+
+    if (skip) {
+        // nothing to do: fall through to the common exit
+    } else if (warp == kWarpTma) {
+        // ------------------------------------------------ TMA producer
+        if (!kF32 && lane == 0) {
+            tma_prefetch_desc(&tmq);
+            tma_prefetch_desc(&tmk);
+            tma_prefetch_desc(&tmv);
+            int issued_k[NS] = {}, issued_v[NS] = {};
+            mbar_arrive_expect_tx(&bar.full_q, U.nt * C::kTile);
+            for (int t = 0; t < U.nt; ++t)
+                for (int bx = 0; bx < D / 64; ++bx)
+                    tma_load_4d(sQ + t * C::kTile + bx * kBoxBytes, &tmq, &bar.full_q, bx * 64,
+                                U.q0, U.hq0 + t, U.b);
+            bool ok = true;
+            for (int j = 0; ok && j < T.n; ++j) {
+                const int s = j % NS, use = j / NS, jt = T.tile(j);
+                if (use > 0) ok = mbar_wait(&bar.empty_k[s], (use - 1) & 1, abort, tmo);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&bar.full_k[s], C::kTile);
+                for (int bx = 0; bx < D / 64; ++bx)
+                    tma_load_4d(sK + s * C::kTile + bx * kBoxBytes, &tmk, &bar.full_k[s], bx * 64,
+                                jt * kBN, U.g, U.b);
+                ++issued_k[s];
+                if (use > 0) ok = mbar_wait(&bar.empty_v[s], (use - 1) & 1, abort, tmo);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&bar.full_v[s], C::kTile);
+                for (int bx = 0; bx < D / 64; ++bx)
+                    tma_load_4d(sV + s * C::kTile + bx * kBoxBytes, &tmv, &bar.full_v[s], bx * 64,
+                                jt * kBN, U.g, U.b);
+                ++issued_v[s];
+            }
+            // Never leave the CTA with copies in flight: wait (bounded, even
+            // after an abort) for the last load issued to every buffer.
+            mbar_wait(&bar.full_q, 0, nullptr, tmo);
+            for (int s = 0; s < NS; ++s) {
+                if (issued_k[s]) mbar_wait(&bar.full_k[s], (issued_k[s] - 1) & 1, nullptr, tmo);
+                if (issued_v[s]) mbar_wait(&bar.full_v[s], (issued_v[s] - 1) & 1, nullptr, tmo);
+            }
+        }
+    } else if (warp >= kWarpRot0 && warp < kWarpRot0 + 4) {
+        // ------------------------------------------------ rotation warpgroup
+        const int tw = threadIdx.x - kWarpRot0 * 32;
+        Phasor<D, kHalf> ph;
+        ph.init(tw, p);
+        bool ok = true;
+        if (!kF32) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_q, 0, abort, tmo));
+            if (ok && p.rotate)
+                for (int t = 0; t < U.nt; ++t)
+                    rotate_tile_bf16<D, kHalf>(sQ + t * C::kTile, U.q0, ph, p);
+        } else {
+            for (int t = 0; t < U.nt; ++t) {
+                const float *base = reinterpret_cast<const float *>(p.q) + U.b * p.qs[0] +
+                                    (long long)(U.hq0 + t) * p.qs[1];
+                load_tile_f32<D, kHalf>(sQ + t * C::kTile, base, p.qs[2], U.q0, p.L, p.rotate != 0,
+                                        ph, p);
+            }
+        }
+        if (ok) {
+            fence_proxy_async_smem();
+            mbar_arrive(&bar.ready_q);
+        }
+        for (int j = 0; ok && j < T.n; ++j) {
+            const int s = j % NS, use = j / NS, jt = T.tile(j);
+            uint8_t *tk = sK + s * C::kTile;
+            if (!kF32) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_k[s], use & 1, abort, tmo));
+                if (!ok) break;
+                if (p.rotate) rotate_tile_bf16<D, kHalf>(tk, (long long)jt * kBN, ph, p);
+            } else {
+                if (use > 0)
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(&bar.empty_k[s], (use - 1) & 1, abort, tmo));
+                if (!ok) break;
+                const float *base = reinterpret_cast<const float *>(p.k) + U.b * p.ks[0] +
+                                    (long long)U.g * p.ks[1];
+                load_tile_f32<D, kHalf>(tk, base, p.ks[2], jt * kBN, p.L, p.rotate != 0, ph, p);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&bar.ready_k[s]);
+            if (kF32) {
+                if (use > 0)
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(&bar.empty_v[s], (use - 1) & 1, abort, tmo));
+                if (!ok) break;
+                const float *base = reinterpret_cast<const float *>(p.v) + U.b * p.vs[0] +
+                                    (long long)U.g * p.vs[1];
+                load_v_f32<D>(sV + s * C::kTile, base, p.vs[2], jt * kBN, p.L, tw);
+                fence_proxy_async_smem();
+                mbar_arrive(&bar.full_v[s]);
+            }
+        }
+    } else if (warp == kWarpMma) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdS = idesc_bf16_f32(128, kBN, 0, 0);
+            constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, 0, 1);
+            const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+            auto issue_s = [&](int t, int s) {
+                const uint32_t qa = q_addr + t * C::kTile, ka = k_addr + s * C::kTile;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+                    mma_ss(tmem + t * 128, sdesc_sw128(qa + off, 16, 1024),
+                           sdesc_sw128(ka + off, 16, 1024), kIdS, kk > 0);
+                }
+            };
+            auto issue_pv = [&](int t, int s, bool acc) {
+                const uint32_t va = v_addr + s * C::kTile;
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk)
+                    mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8,
+                           sdesc_sw128(va + kk * 2048, kBoxBytes, 1024), kIdPV, (acc || kk > 0));
+            };
+            bool ok = mbar_wait(&bar.ready_q, 0, abort, tmo);
+            if (ok) ok = mbar_wait(&bar.ready_k[0], 0, abort, tmo);
+            tc_fence_after();
+            if (ok) {
+                for (int t = 0; t < U.nt; ++t) {
+                    issue_s(t, 0);
+                    mma_commit(&bar.s_ready[t]);
+                }
+                mma_commit(&bar.empty_k[0]);
+            }
+            for (int j = 0; ok && j < T.n; ++j) {
+                const int sv = j % NS;
+                ok = mbar_wait(&bar.full_v[sv], (j / NS) & 1, abort, tmo);
+                for (int t = 0; ok && t < U.nt; ++t) {
+                    ok = mbar_wait(&bar.p_ready[t], j & 1, abort, tmo);
+                    tc_fence_after();
+                    if (!ok) break;
+                    issue_pv(t, sv, j > 0);
+                    if (j + 1 < T.n) {
+                        const int sk = (j + 1) % NS;
+                        if (t == 0) {
+                            ok = mbar_wait(&bar.ready_k[sk], ((j + 1) / NS) & 1, abort, tmo);
+                            tc_fence_after();
+                            if (!ok) break;
+                        }
+                        issue_s(t, sk);
+                        mma_commit(&bar.s_ready[t]);
+                    }
+                }
+                if (ok) {
+                    mma_commit(&bar.empty_v[sv]);
+                    if (j + 1 < T.n) mma_commit(&bar.empty_k[(j + 1) % NS]);
+                }
+            }
+            if (ok)
+                for (int t = 0; t < U.nt; ++t) mma_commit(&bar.o_ready[t]);
+            // Drain: all issued MMAs complete before TMEM is released.
+            mma_commit(&bar.drain);
+            mbar_wait(&bar.drain, 0, nullptr, tmo);
+        }
+    } else if (warp < 8 && (warp >> 2) < U.nt) {
+        // ------------------------------------------------ softmax, tile t
+        const int t = warp >> 2;
+        const int wq = warp & 3;
+        const int row = wq * 32 + lane;
+        const uint32_t trow = tmem + (uint32_t(wq * 32) << 16);
+        const uint32_t s_col = t * 128, o_col = 256 + t * D;
+        const int i = U.q0 + row;
+        const float cl2 = p.c_log2;
+        float m = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < T.n; ++j) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_ready[t], j & 1, abort, tmo));
+            if (!ok) break;
+            tc_fence_after();
+            const int jt = T.tile(j), k0 = jt * kBN;
+            const bool partial = !tile_full(U.q0, jt, p);
+            // visible columns: col <= hi and (no window or col >= lo or col < sk)
+            const int hi = p.causal ? min(i - k0, p.L - 1 - k0) : p.L - 1 - k0;
+            const int lo = i - p.window + 1 - k0;
+            const int sk = p.sinks - k0;
+            const bool win = p.causal && p.window > 0;
+            auto vis = [&](int col) { return col <= hi && (!win || col >= lo || col < sk); };
+
+            // pass 1: row max
+            float mx = -INFINITY;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                float v[32];
+                tmem_ld32(trow + s_col + c * 32, v);
+                if (partial) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (!vis(c * 32 + e)) v[e] = -INFINITY;
+                }
+                float m0 = v[0], m1 = v[1], m2 = v[2], m3 = v[3];
+#pragma unroll
+                for (int e = 4; e < 32; e += 4) {
+                    m0 = fmaxf(m0, v[e]);
+                    m1 = fmaxf(m1, v[e + 1]);
+                    m2 = fmaxf(m2, v[e + 2]);
+                    m3 = fmaxf(m3, v[e + 3]);
+                }
+                mx = fmaxf(mx, fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)));
+            }
+            const float m_new = fmaxf(m, mx * cl2);
+            // Keep the old reference unless the max grew by more than 2^8: the
+            // result is exact either way, only O's rescale is saved.
+            const bool need = (m != -INFINITY) && (m_new > m + kRescaleLog2);
+            if (__any_sync(0xffffffffu, need)) {
+                const float alpha = need ? ex2_approx(m - m_new) : 1.f;
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    float v[32];
+                    tmem_ld32(trow + o_col + c * 32, v);
+                    uint32_t u[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(v[e] * alpha);
+                    tmem_st32(trow + o_col + c * 32, u);
+                }
+                if (need) {
+                    l *= alpha;
+                    m = m_new;
+                }
+            }
+            if (m == -INFINITY) m = m_new;
+            const float mref = (m == -INFINITY) ? 0.f : m;
+            // pass 2: P = 2^(s c - m) as bf16 written over the first half of S
+            float lsum = 0.f;
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+                float a[32], b[32];
+                tmem_ld32(trow + s_col + h * 64, a);
+                tmem_ld32(trow + s_col + h * 64 + 32, b);
+                if (partial) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        if (!vis(h * 64 + e)) a[e] = -INFINITY;
+                        if (!vis(h * 64 + 32 + e)) b[e] = -INFINITY;
+                    }
+                }
+                uint32_t pk[32];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = ex2_approx(fmaf(a[2 * e], cl2, -mref));
+                    const float p1 = ex2_approx(fmaf(a[2 * e + 1], cl2, -mref));
+                    lsum += p0 + p1;
+                    pk[e] = pack_bf16x2(p0, p1);
+                }
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = ex2_approx(fmaf(b[2 * e], cl2, -mref));
+                    const float p1 = ex2_approx(fmaf(b[2 * e + 1], cl2, -mref));
+                    lsum += p0 + p1;
+                    pk[16 + e] = pack_bf16x2(p0, p1);
+                }
+                tmem_st32(trow + s_col + h * 32, pk);
+            }
+            l += lsum;
+            tc_fence_before();
+            mbar_arrive(&bar.p_ready[t]);
+        }
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.o_ready[t], 0, abort, tmo));
+        if (ok) {
+            tc_fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const int h = U.hq0 + t;
+            const bool valid = i < p.L;
+            const long long ob = U.b * p.os[0] + (long long)h * p.os[1] + (long long)i * p.os[2];
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                float v[32];
+                tmem_ld32(trow + o_col + c * 32, v);
+                if (!valid) continue;
+                if (kF32) {
+                    float4 *dst = reinterpret_cast<float4 *>(
+                        reinterpret_cast<float *>(p.o) + ob + c * 32);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        dst[e] = make_float4(v[4 * e] * inv, v[4 * e + 1] * inv,
+                                             v[4 * e + 2] * inv, v[4 * e + 3] * inv);
+                } else {
+                    uint4 *dst = reinterpret_cast<uint4 *>(
+                        reinterpret_cast<__nv_bfloat16 *>(p.o) + ob + c * 32);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_uint4(pack_bf16x2(v[8 * e] * inv, v[8 * e + 1] * inv),
+                                            pack_bf16x2(v[8 * e + 2] * inv, v[8 * e + 3] * inv),
+                                            pack_bf16x2(v[8 * e + 4] * inv, v[8 * e + 5] * inv),
+                                            pack_bf16x2(v[8 * e + 6] * inv, v[8 * e + 7] * inv));
+                }
+            }
+            if (valid && p.lse) {
+                const float ln2 = 0.69314718055994531f;
+                p.lse[(U.b * (long long)p.Hq + h) * p.L + i] =
+                    l > 0.f ? (m + __log2f(l)) * ln2 : -INFINITY;
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+    if (threadIdx.x == 0 && !skip && bar.abort && p.status)
+        atomicExch(p.status, int(LCX_ERR_TIMEOUT));
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(ptr);
+    }();
+    return fn;
+}
+
+// [B, H, L, D] bf16 tensor -> 4-D tensor map with 64 x 128 boxes, 128-byte swizzle.
+lcx_status make_map(CUtensorMap *map, const void *ptr, int64_t B, int64_t H, int64_t L, int64_t D,
+                    const int64_t *st, const char *name) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(LCX_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(L), cuuint64_t(H), cuuint64_t(B)};
+    cuuint64_t strides[3] = {cuuint64_t(st[2] * 2), cuuint64_t(st[1] * 2), cuuint64_t(st[0] * 2)};
+    cuuint32_t box[4] = {64, 128, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(LCX_ERR_UNSUPPORTED, "tensor map for %s rejected (CUresult %d)", name, int(r));
+    return LCX_OK;
+}
+
+template <int D, bool kF32, bool kHalf>
+lcx_status launch(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                  const AttnParams &p, unsigned grid, cudaStream_t s) {
+    auto kern = attn_fwd_kernel<D, kF32, kHalf>;
+    const int smem = Cfg<D>::kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess)
+        return fail(LCX_ERR_CUDA, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
+    kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return fail(LCX_ERR_CUDA, "attn_fwd launch failed: %s", cudaGetErrorString(e));
+    return LCX_OK;
+}
+
+template <int D>
+lcx_status launch_d(bool f32, bool half, const CUtensorMap &mq, const CUtensorMap &mk,
+                    const CUtensorMap &mv, const AttnParams &p, unsigned grid, cudaStream_t s) {
+    if (f32)
+        return half ? launch<D, true, true>(mq, mk, mv, p, grid, s)
+                    : launch<D, true, false>(mq, mk, mv, p, grid, s);
+    return half ? launch<D, false, true>(mq, mk, mv, p, grid, s)
+                : launch<D, false, false>(mq, mk, mv, p, grid, s);
+}
+
+lcx_status check_tensor(const void *ptr, const int64_t *st, int es, const char *name) {
+    if (!ptr) return fail(LCX_ERR_INVALID_ARG, "%s is NULL", name);
+    if (!aligned16(ptr)) return fail(LCX_ERR_UNSUPPORTED, "%s must be 16-byte aligned", name);
+    if (st[3] != 1) return fail(LCX_ERR_UNSUPPORTED, "%s: head_dim stride must be 1", name);
+    for (int d = 0; d < 3; ++d) {
+        if (st[d] < 0) return fail(LCX_ERR_UNSUPPORTED, "%s: negative stride", name);
+        if ((st[d] * es) % 16 != 0)
+            return fail(LCX_ERR_UNSUPPORTED, "%s: strides must be multiples of 16 bytes", name);
+    }
+    return LCX_OK;
+}
+
+}  // namespace
+}  // namespace lcx
+
+extern "C" lcx_status lcx_attn_fwd(const lcx_attn_args *a, void *stream) {
+    using namespace lcx;
+    clear_error();
+    if (!a) return fail(LCX_ERR_INVALID_ARG, "args is NULL");
+    lcx_status st = check_rope_params(&a->rope);
+    if (st != LCX_OK) return st;
+    if (a->dtype != LCX_BF16 && a->dtype != LCX_F32)
+        return fail(LCX_ERR_INVALID_ARG, "unknown dtype %d", a->dtype);
+    if (a->B < 0 || a->Hq <= 0 || a->Hkv <= 0 || a->L < 0 || a->D <= 0)
+        return fail(LCX_ERR_INVALID_ARG, "bad sizes");
+    if (a->Hq % a->Hkv != 0)
+        return fail(LCX_ERR_INVALID_ARG, "Hq (%lld) must be a multiple of Hkv (%lld)",
+                    (long long)a->Hq, (long long)a->Hkv);
+    if (a->rope.head_dim != a->D) return fail(LCX_ERR_INVALID_ARG, "rope.head_dim != D");
+    if (a->causal != 0 && a->causal != 1) return fail(LCX_ERR_INVALID_ARG, "causal must be 0 or 1");
+    if (a->window < 0 || a->sinks < 0)
+        return fail(LCX_ERR_INVALID_ARG, "window and sinks must be >= 0");
+    if (!a->causal && (a->window != 0 || a->sinks != 0))
+        return fail(LCX_ERR_UNSUPPORTED, "window / sinks need causal attention");
+    if (a->flags & ~uint32_t(LCX_ATTN_PREROTATED)) return fail(LCX_ERR_INVALID_ARG, "unknown flags");
+    if (!(a->softmax_scale >= 0.f) || !std::isfinite(a->softmax_scale))
+        return fail(LCX_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+    if (a->D != 64 && a->D != 128)
+        return fail(LCX_ERR_UNSUPPORTED, "head_dim %lld: only 64 and 128", (long long)a->D);
+    if (a->B == 0 || a->L == 0) return LCX_OK;
+    if (a->L > (int64_t(1) << 30) || a->B > (int64_t(1) << 20) || a->Hq > 65536)
+        return fail(LCX_ERR_UNSUPPORTED, "sizes too large");
+    const int es = a->dtype == LCX_BF16 ? 2 : 4;
+    if ((st = check_tensor(a->q, a->q_strides, es, "q")) != LCX_OK) return st;
+    if ((st = check_tensor(a->k, a->k_strides, es, "k")) != LCX_OK) return st;
+    if ((st = check_tensor(a->v, a->v_strides, es, "v")) != LCX_OK) return st;
+    if ((st = check_tensor(a->o, a->o_strides, es, "o")) != LCX_OK) return st;
+
+    AttnParams p;
+    memset(&p, 0, sizeof(p));
+    p.q = static_cast<const char *>(a->q);
+    p.k = static_cast<const char *>(a->k);
+    p.v = static_cast<const char *>(a->v);
+    p.o = static_cast<char *>(a->o);
+    p.lse = a->lse;
+    p.status = a->dev_status;
+    for (int d = 0; d < 3; ++d) {
+        p.qs[d] = a->q_strides[d];
+        p.ks[d] = a->k_strides[d];
+        p.vs[d] = a->v_strides[d];
+        p.os[d] = a->o_strides[d];
+    }
+    p.B = int(a->B);
+    p.Hq = int(a->Hq);
+    p.Hkv = int(a->Hkv);
+    p.L = int(a->L);
+    p.G = int(a->Hq / a->Hkv);
+    p.causal = a->causal;
+    p.window = int(a->window > a->L ? a->L : a->window);
+    p.sinks = int(a->sinks > a->L ? a->L : a->sinks);
+    p.n_qb = int((a->L + kBM - 1) / kBM);
+    p.heads_per_unit = (p.G % 2 == 0) ? 2 : 1;
+    p.units_per_qb = p.B * p.Hq / p.heads_per_unit;
+    const long long grid = (long long)p.n_qb * p.units_per_qb;
+    if (grid > 0x7fffffffLL) return fail(LCX_ERR_UNSUPPORTED, "too many work units");
+    p.rotate = (a->flags & LCX_ATTN_PREROTATED) ? 0 : 1;
+    float ms = 1.f;
+    rope_table_unchecked(&a->rope, p.theta, &ms);
+    const double scale = a->softmax_scale > 0.f ? double(a->softmax_scale) : 1.0 / std::sqrt(double(a->D));
+    const double msq = p.rotate ? double(ms) * double(ms) : 1.0;
+    p.c_log2 = float(scale * msq * 1.4426950408889634);
+    p.timeout_ns = 2000000000ull;  // 2 s: legitimate waits last microseconds
+
+    CUtensorMap mq, mk, mv;
+    memset(&mq, 0, sizeof(mq));
+    memset(&mk, 0, sizeof(mk));
+    memset(&mv, 0, sizeof(mv));
+    if (a->dtype == LCX_BF16) {
+        if ((st = make_map(&mq, a->q, a->B, a->Hq, a->L, a->D, a->q_strides, "q")) != LCX_OK) return st;
+        if ((st = make_map(&mk, a->k, a->B, a->Hkv, a->L, a->D, a->k_strides, "k")) != LCX_OK) return st;
+        if ((st = make_map(&mv, a->v, a->B, a->Hkv, a->L, a->D, a->v_strides, "v")) != LCX_OK) return st;
+    }
+    const bool f32 = a->dtype == LCX_F32;
+    const bool half = a->rope.pairing == LCX_PAIR_HALF;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (a->D == 128) return launch_d<128>(f32, half, mq, mk, mv, p, unsigned(grid), s);
+    return launch_d<64>(f32, half, mq, mk, mv, p, unsigned(grid), s);
+}

@@ -1,0 +1,170 @@
+"""GPU parity of lcx_attn_fwd (fused RoPE + causal attention prefill) against the
+fp64 oracle.
+
+Tolerance (from the target): output max-abs <= 2e-2 and mean-abs <= 2e-3 against
+the fp64 result; LSE max-abs <= 2e-2.  Small cases compare every element and span
+several 128-row tiles with ragged tails; the full-size workloads compare sampled
+query rows (boundary rows plus seeded random rows, all heads).
+"""
+import numpy as np
+import pytest
+import torch
+
+import ntk_rope_flashattn_b200 as lcx
+import oracle
+from workloads import WORKLOADS, Workload, make_inputs, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, MEAN_ABS, LSE_ABS = 2e-2, 2e-3, 2e-2
+
+
+def rope_of(w):
+    return lcx.RopeParams(w.mode, w.D, w.base, w.scale, w.original_max_pos, w.alpha, w.beta,
+                          w.pairing)
+
+
+def table_of(w):
+    t, ms, _ = oracle.rope_table(w.mode, w.D, w.base, w.scale, w.original_max_pos, w.alpha,
+                                 w.beta)
+    return t, ms
+
+
+def run_gpu(w, q, k, v, **kw):
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = lcx.attn_fwd(q, k, v, rope_of(w), causal=w.causal, window=w.window, sinks=w.sinks,
+                          softmax_scale=w.softmax_scale, return_lse=True, status=status, **kw)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, "device watchdog fired"
+    return o, lse
+
+
+def compare(got_o, got_lse, ref_o, ref_lse):
+    err = np.abs(got_o.astype(np.float64) - ref_o)
+    assert np.isfinite(got_o).all()
+    assert err.max() <= MAX_ABS, "max-abs %.4g" % err.max()
+    assert err.mean() <= MEAN_ABS, "mean-abs %.4g" % err.mean()
+    lerr = np.abs(got_lse.astype(np.float64) - ref_lse)
+    assert lerr.max() <= LSE_ABS, "lse max-abs %.4g" % lerr.max()
+    return err.max(), err.mean()
+
+
+def full_check(w, **kw):
+    q, k, v = make_inputs(w, device="cuda")
+    o, lse = run_gpu(w, q, k, v, **kw)
+    table, ms = table_of(w)
+    scale = w.softmax_scale if w.softmax_scale > 0 else None
+    ref_o, ref_lse = oracle.attn_full(q.float().cpu().numpy(), k.float().cpu().numpy(),
+                                      v.float().cpu().numpy(), table, ms, w.pairing, 0,
+                                      w.causal, w.window, w.sinks, scale)
+    return compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_lse)
+
+
+BASE = Workload("case", B=1, Hq=4, Hkv=2, L=256, D=128, dtype="bf16", mode="plain")
+
+SMALL = {
+    "L1": dict(L=1, Hq=2, Hkv=1),
+    "L127_yarn_G2": dict(L=127, mode="yarn", scale=4.0, original_max_pos=64),
+    "L129_ntk_G4": dict(L=129, Hq=8, Hkv=2, mode="ntk", scale=4.0),
+    "L300_pi_MHA_B2": dict(L=300, B=2, Hq=2, Hkv=2, mode="pi", scale=2.0),
+    "L300_G3": dict(L=300, Hq=3, Hkv=1),
+    "L1000_window_sinks": dict(L=1000, mode="yarn", scale=8.0, original_max_pos=128,
+                               window=300, sinks=4),
+    "L1000_window": dict(L=1000, window=200),
+    "L700_D64": dict(L=700, D=64, mode="yarn", scale=4.0, original_max_pos=128),
+    "L500_noncausal": dict(L=500, Hq=2, Hkv=1, causal=False),
+    "L400_interleaved": dict(L=400, pairing="interleaved", mode="yarn", scale=16.0,
+                             original_max_pos=32),
+    "L333_D64_interleaved_window": dict(L=333, D=64, pairing="interleaved", window=64, sinks=130),
+    "L600_f32": dict(L=600, dtype="f32", mode="ntk", scale=2.0),
+    "L390_f32_D64_interleaved": dict(L=390, D=64, dtype="f32", pairing="interleaved"),
+    "L2000_W1": dict(L=2000, Hq=2, Hkv=1, window=1),
+    "L513_bigwindow": dict(L=513, window=5000, sinks=3),
+    "L640_outliers": dict(L=640, mode="yarn", scale=8.0, original_max_pos=128,
+                          outlier_frac=0.01, window=256, sinks=4),
+    "L256_scale": dict(L=256, softmax_scale=0.05),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_attn_small_cases(name):
+    full_check(BASE.with_(**SMALL[name]))
+
+
+def test_attn_tiny_workload_full():
+    """The 256-token fp32 workload (head_dim 64, scale 1/8), every element."""
+    full_check(WORKLOADS["tiny_L256_D64"])
+
+
+def test_attn_window_one_returns_v():
+    """W = 1 without sinks: every query sees only itself, so o_i = v_i (bf16 exact)."""
+    w = BASE.with_(L=300, window=1)
+    q, k, v = make_inputs(w, device="cuda")
+    o, _ = run_gpu(w, q, k, v)
+    vv = v.repeat_interleave(w.Hq // w.Hkv, dim=1)
+    assert torch.equal(o, vv)
+
+
+def test_attn_prerotated_matches_fused():
+    """lcx_apply_rope on q and k followed by the PREROTATED kernel equals the
+    oracle (and the fused rotation within tolerance)."""
+    w = BASE.with_(L=777, mode="yarn", scale=16.0, original_max_pos=64, Hq=8, Hkv=2,
+                   window=400, sinks=4)
+    q, k, v = make_inputs(w, device="cuda")
+    rope = rope_of(w)
+    qr, kr = lcx.apply_rope(q, rope), lcx.apply_rope(k, rope)
+    o_pre, lse_pre = run_gpu(w, qr, kr, v, prerotated=True)
+    o_fused, lse_fused = run_gpu(w, q, k, v)
+    table, ms = table_of(w)
+    ref_o, ref_lse = oracle.attn_full(q.float().cpu().numpy(), k.float().cpu().numpy(),
+                                      v.float().cpu().numpy(), table, ms, "half", 0, True,
+                                      w.window, w.sinks)
+    compare(o_pre.float().cpu().numpy(), lse_pre.cpu().numpy(), ref_o, ref_lse)
+    compare(o_fused.float().cpu().numpy(), lse_fused.cpu().numpy(), ref_o, ref_lse)
+
+
+def test_attn_strided_views_and_determinism():
+    """q/k/v/o given as [B, L, H, D] buffers viewed as [B, H, L, D]; two calls give
+    bit-identical results."""
+    w = BASE.with_(L=333, B=2, mode="yarn", scale=4.0, original_max_pos=64)
+    q, k, v = make_inputs(w, device="cuda")
+    qs, ks, vs = (t.transpose(1, 2).contiguous().transpose(1, 2) for t in (q, k, v))
+    assert not qs.is_contiguous()
+    out = torch.empty((w.B, w.L, w.Hq, w.D), dtype=q.dtype, device="cuda").transpose(1, 2)
+    o1, _ = run_gpu(w, qs, ks, vs, out=out)
+    o2, _ = run_gpu(w, q, k, v)
+    assert torch.equal(o1, o2)
+    o3, _ = run_gpu(w, q, k, v)
+    assert torch.equal(o2, o3)
+
+
+def sampled_check(w, n_random=16, max_heads=None):
+    q, k, v = make_inputs(w, device="cuda")
+    o, lse = run_gpu(w, q, k, v)
+    rows, batches = sample_rows(w, n_random=n_random)
+    heads = list(range(w.Hq)) if max_heads is None else list(range(0, w.Hq, w.Hq // max_heads))
+    idx = torch.tensor(rows, device="cuda")
+    table, ms = table_of(w)
+    scale = w.softmax_scale if w.softmax_scale > 0 else None
+    errs = []
+    for b in batches:
+        qb = q[b].index_select(1, idx)[heads]                      # [h, r, D]
+        ob = o[b].index_select(1, idx)[heads].float().cpu().numpy()
+        lb = lse[b].index_select(1, idx)[heads].cpu().numpy()
+        kb = k[b:b + 1].float().cpu().numpy()
+        vb = v[b:b + 1].float().cpu().numpy()
+        hh, rr = np.meshgrid(heads, rows, indexing="ij")
+        ref_o, ref_l = oracle.attn_rows(qb.float().cpu().numpy().reshape(-1, w.D),
+                                        np.zeros(hh.size), hh.ravel(), rr.ravel(), kb, vb, w.Hq,
+                                        table, ms, w.pairing, 0, w.causal, w.window, w.sinks,
+                                        scale)
+        errs.append(compare(ob.reshape(-1, w.D), lb.ravel(), ref_o, ref_l))
+    del q, k, v, o, lse
+    torch.cuda.empty_cache()
+    return errs
+
+
+@pytest.mark.parametrize("name", ["llama3_8b_L8192", "pi_L32768_s4", "ntk_L32768_s4",
+                                  "yarn_L131072_s16", "sink_window_L65536"])
+def test_attn_full_size_sampled_rows(name):
+    sampled_check(WORKLOADS[name])
