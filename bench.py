@@ -308,6 +308,7 @@ def bench_gpu(args, world, rank, local):
             "frac_of_burst": round(achieved / float(peaks["bf16_tflops"]), 4),
             "traffic": ATTN_TRAFFIC_BYTES,
             "kernel": "attn_fwd_kernel", "avg_launch_ms": round(avg_launch, 3),
+            "launch_ms": [round(x, 3) for x in launch_ms],
         },
         "apply_rope": {
             "bound": "hbm", "bytes": rope_bytes(w), "ms": round(rope_ms, 4),
