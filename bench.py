@@ -198,7 +198,7 @@ def bench_gpu(args, world, rank, local):
     o = torch.empty_like(q)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     kw = dict(causal=w.causal, window=w.window, sinks=w.sinks, softmax_scale=w.softmax_scale,
-              out=o, status=status)
+              split_qk=w.split_qk, out=o, status=status)
     stream = torch.cuda.current_stream(dev)
 
     def step():
@@ -254,14 +254,16 @@ def bench_gpu(args, world, rank, local):
     ws = {}
     for _ in range(max(1, min(args.warmup, 2))):
         lcx.attn_fwd_host(qh, kh, vh, rope, device=dev, workspace=ws, causal=w.causal,
-                          window=w.window, sinks=w.sinks, softmax_scale=w.softmax_scale)
+                          window=w.window, sinks=w.sinks, softmax_scale=w.softmax_scale,
+                          split_qk=w.split_qk)
     torch.cuda.synchronize()
     barrier(world)
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e_start.record(stream)
     for _ in range(args.steps):
         oh = lcx.attn_fwd_host(qh, kh, vh, rope, device=dev, workspace=ws, causal=w.causal,
-                               window=w.window, sinks=w.sinks, softmax_scale=w.softmax_scale)
+                               window=w.window, sinks=w.sinks, softmax_scale=w.softmax_scale,
+                               split_qk=w.split_qk)
     e_end.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), world)
@@ -293,7 +295,7 @@ def bench_gpu(args, world, rank, local):
             "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D,
             "rope": w.mode, "scale": w.scale, "original_max_pos": w.original_max_pos,
             "alpha": w.alpha, "beta": w.beta, "causal": w.causal, "window": w.window,
-            "sinks": w.sinks, "visible_pairs_per_head": visible_pairs(w.L, w.causal, w.window,
+            "sinks": w.sinks, "split_qk": w.split_qk, "visible_pairs_per_head": visible_pairs(w.L, w.causal, w.window,
                                                                       w.sinks),
             "flops_per_step_per_gpu": flops_rank,
             "l2": "inputs larger than L2 (q+k+v = %.2f GB), no flush" % (

@@ -125,6 +125,13 @@ LCX_API lcx_status lcx_apply_rope(const lcx_rope_params *params, const void *x, 
                                    lcx_apply_rope with the same params, mscale
                                    included): skip the on-chip rotation and the
                                    mscale^2 factor on the logits.             */
+#define LCX_ATTN_SPLIT_QK 2u    /* split mode: hold each rotated q' and k' as a bf16
+                                   pair hi + lo (lo = bf16(x' - hi)) and form
+                                   QK^T as hi.hi + hi.lo + lo.hi, so the logits
+                                   are no longer limited by bf16 rounding of the
+                                   rotated operands (needed when the logits are
+                                   large, e.g. outlier-heavy activations); about
+                                   twice the tensor-core work for QK^T        */
 
 typedef struct {
     const void *q;             /* DEVICE [B, Hq, L, D]                            */

@@ -25,6 +25,7 @@ MODES = {"none": 0, "plain": 1, "pi": 2, "ntk": 3, "yarn": 4}
 PAIRINGS = {"half": 0, "interleaved": 1}
 DTYPES = {"bf16": 0, "f32": 1}
 LCX_ATTN_PREROTATED = 1
+LCX_ATTN_SPLIT_QK = 2
 
 # Symbols include/lcx.h declares; the library must export every one of them.
 EXPORTED = ("lcx_rope_table", "lcx_apply_rope", "lcx_attn_fwd", "lcx_status_string",
@@ -180,11 +181,13 @@ def apply_rope(x, rope: RopeParams, out=None, pos_offset: int = 0, inplace: bool
 
 def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, sinks: int = 0,
              softmax_scale: float = 0.0, return_lse: bool = False, prerotated: bool = False,
-             out=None, lse=None, status=None):
+             split_qk: bool = False, out=None, lse=None, status=None):
     """Fused RoPE + causal attention prefill.
 
     q [B, Hq, L, D], k/v [B, Hkv, L, D] CUDA tensors (bf16 or fp32, last dim
     contiguous).  Returns o [B, Hq, L, D] (and lse [B, Hq, L] fp32 if asked).
+    ``split_qk`` forms QK^T from hi/lo bf16 parts of the rotated operands
+    (LCX_ATTN_SPLIT_QK) for inputs whose large logits bf16 rounding would spoil.
     ``status`` (optional int32 CUDA tensor of one element) receives
     LCX_ERR_TIMEOUT if a kernel's bounded wait expired.
     """
@@ -213,7 +216,7 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
     a.rope = rope._c()
     a.window, a.sinks = int(window), int(sinks)
     a.softmax_scale = float(softmax_scale)
-    a.flags = LCX_ATTN_PREROTATED if prerotated else 0
+    a.flags = (LCX_ATTN_PREROTATED if prerotated else 0) | (LCX_ATTN_SPLIT_QK if split_qk else 0)
     _check(load().lcx_attn_fwd(ctypes.byref(a), _stream(q)))
     return (o, lse) if return_lse else o
 

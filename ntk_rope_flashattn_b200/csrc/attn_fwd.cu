@@ -45,8 +45,6 @@ namespace {
 
 constexpr int kThreads = 448;           // 14 warps
 constexpr int kBM = 128;                // query rows per tile
-constexpr int kBN = 128;                // keys per tile
-constexpr int kBoxBytes = 128 * 128;    // one TMA box: 128 rows x 128 bytes
 constexpr float kRescaleLog2 = 8.0f;    // rescale O only if the max grows by > 2^8
 constexpr int kWarpMma = 13;
 constexpr int kWarpTma = 12;
@@ -67,15 +65,28 @@ struct AttnParams {
     float theta[64];
 };
 
-template <int D>
+// Shared-memory plan.  A tile of R rows x D bf16 is stored as D/64 TMA boxes of
+// R rows x 128 bytes with the 128-byte swizzle.  In the split mode every Q and
+// K tile has a second "lo" part holding bf16(x' - bf16(x')), and key tiles are
+// 64 rows so that both parts fit.
+template <int D, bool kSplit>
 struct Cfg {
-    static constexpr int kTile = kBM * D * 2;  // bytes of a 128 x D bf16 tile
+    static constexpr int BN = kSplit ? 64 : 128;        // keys per tile
+    static constexpr int kParts = kSplit ? 2 : 1;       // hi (+ lo) parts of Q and K
+    static constexpr int kTileQ = kBM * D * 2;          // one part of a Q tile
+    static constexpr int kTileK = BN * D * 2;           // one part of a K tile / a V tile
+    static constexpr int kBoxQ = kBM * 128;
+    static constexpr int kBoxK = BN * 128;
     static constexpr int kStages = (D == 128) ? 2 : 4;
     static constexpr int kOffQ = 0;
-    static constexpr int kOffK = 2 * kTile;
-    static constexpr int kOffV = kOffK + kStages * kTile;
-    static constexpr int kOffBar = kOffV + kStages * kTile;
+    static constexpr int kOffK = kOffQ + 2 * kParts * kTileQ;
+    static constexpr int kOffV = kOffK + kStages * kParts * kTileK;
+    static constexpr int kOffBar = kOffV + kStages * kTileK;
     static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers + alignment slack
+    // TMEM columns: S_t at t*BN (P_t aliased over its first BN/2 columns), O_t after.
+    static constexpr int kColO = 2 * BN;
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
 };
 
 template <int NS>
@@ -125,13 +136,14 @@ struct Tiles {
     __device__ __forceinline__ int tile(int j) const { return j < ns ? j : jlo + (j - ns); }
 };
 
+template <int BN>
 __device__ __forceinline__ Tiles make_tiles(int q0, const AttnParams &p) {
     const int i1 = min(q0 + kBM - 1, p.L - 1);
-    const int jhi = p.causal ? i1 / kBN : (p.L - 1) / kBN;
+    const int jhi = p.causal ? i1 / BN : (p.L - 1) / BN;
     int jlo = 0, ns = 0;
     if (p.causal && p.window > 0) {
-        jlo = max(0, q0 - p.window + 1) / kBN;
-        if (p.sinks > 0) ns = min((p.sinks + kBN - 1) / kBN, jlo);
+        jlo = max(0, q0 - p.window + 1) / BN;
+        if (p.sinks > 0) ns = min((p.sinks + BN - 1) / BN, jlo);
     }
     Tiles t;
     t.ns = ns;
@@ -141,8 +153,9 @@ __device__ __forceinline__ Tiles make_tiles(int q0, const AttnParams &p) {
 }
 
 // True when every (query row of the block, key of the tile) pair is visible.
+template <int BN>
 __device__ __forceinline__ bool tile_full(int q0, int jt, const AttnParams &p) {
-    const int j0 = jt * kBN, j1 = j0 + kBN - 1;
+    const int j0 = jt * BN, j1 = j0 + BN - 1;
     const int i0 = q0, i1 = q0 + kBM - 1;
     if (j1 > p.L - 1) return false;
     if (!p.causal) return true;
@@ -152,17 +165,16 @@ __device__ __forceinline__ bool tile_full(int q0, int jt, const AttnParams &p) {
 }
 
 // ---------------------------------------------------------------- smem tiles
-// A 128 x D bf16 tile is stored as D/64 TMA boxes of 128 rows x 128 bytes with
-// the 128-byte swizzle: the 16-byte chunk c of row r sits at chunk c ^ (r & 7).
-__device__ __forceinline__ uint32_t chunk_off(int r, int fc) {
-    return (fc >> 3) * kBoxBytes + r * 128 + (((fc & 7) ^ (r & 7)) << 4);
+// Byte offset of the 16-byte chunk fc (8 bf16 columns) of row r in a tile whose
+// boxes are box_bytes long: the chunk c of row r sits at chunk c ^ (r & 7).
+__device__ __forceinline__ uint32_t chunk_off(int r, int fc, int box_bytes) {
+    return (fc >> 3) * box_bytes + r * 128 + (((fc & 7) ^ (r & 7)) << 4);
 }
 
 template <int D, bool kHalf>
 struct Rot {
     static constexpr int CPR = kHalf ? D / 16 : D / 8;  // jobs per row
     static constexpr int RP = 128 / CPR;                 // rows per pass of the WG
-    static constexpr int NJ = 128 / RP;                  // jobs per thread
     static constexpr int PPJ = kHalf ? 8 : 4;            // pairs per job
 };
 
@@ -189,6 +201,27 @@ __device__ __forceinline__ void unpack8(const uint4 &v, float (&x)[8]) {
 __device__ __forceinline__ uint4 pack8(const float (&y)[8]) {
     return make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
                       pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
+}
+// hi = bf16(y) (returned packed), y -= hi (the residual, for the lo part).
+__device__ __forceinline__ uint4 pack8_hi(float (&y)[8]) {
+    const uint4 h = pack8(y);
+    float hf[8];
+    unpack8(h, hf);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] -= hf[e];
+    return h;
+}
+
+// Store 8 rotated values: bf16 hi part at `hi`, and in the split mode the bf16
+// residual at the same offset of the lo part.
+template <bool kSplit>
+__device__ __forceinline__ void store8(uint8_t *hi, uint8_t *lo, uint32_t off, float (&y)[8]) {
+    if (kSplit) {
+        *reinterpret_cast<uint4 *>(hi + off) = pack8_hi(y);
+        *reinterpret_cast<uint4 *>(lo + off) = pack8(y);
+    } else {
+        *reinterpret_cast<uint4 *>(hi + off) = pack8(y);
+    }
 }
 
 // Per-thread phasor state of the rotation warpgroup: the thread always handles
@@ -222,58 +255,64 @@ struct Phasor {
     }
 };
 
-// Rotate a bf16 tile in place (rows at positions pos0 + r).
-template <int D, bool kHalf>
-__device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, long long pos0,
-                                                 const Phasor<D, kHalf> &ph,
-                                                 const AttnParams &p) {
+// Rotate a ROWS x D bf16 tile in place (row r at position pos0 + r); in the
+// split mode also write the residual part into `lo`.
+template <int D, bool kHalf, bool kSplit, int ROWS>
+__device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, uint8_t *lo, long long pos0,
+                                                 const Phasor<D, kHalf> &ph, const AttnParams &p,
+                                                 bool rotate) {
     using R = Rot<D, kHalf>;
+    constexpr int NJ = ROWS / R::RP;
+    constexpr int BOX = ROWS * 128;
     float c[R::PPJ], s[R::PPJ];
-    ph.start(pos0, p, c, s);
+    if (rotate) ph.start(pos0, p, c, s);
 #pragma unroll 2
-    for (int k = 0; k < R::NJ; ++k) {
+    for (int k = 0; k < NJ; ++k) {
         const int r = ph.r0 + k * R::RP;
         if (kHalf) {
-            uint4 *pa = reinterpret_cast<uint4 *>(tile + chunk_off(r, ph.q));
-            uint4 *pb = reinterpret_cast<uint4 *>(tile + chunk_off(r, ph.q + D / 16));
+            const uint32_t oa = chunk_off(r, ph.q, BOX), ob = chunk_off(r, ph.q + D / 16, BOX);
             float x1[8], x2[8];
-            unpack8(*pa, x1);
-            unpack8(*pb, x2);
-            rot_pairs<8>(x1, x2, c, s);
-            *pa = pack8(x1);
-            *pb = pack8(x2);
+            unpack8(*reinterpret_cast<const uint4 *>(tile + oa), x1);
+            unpack8(*reinterpret_cast<const uint4 *>(tile + ob), x2);
+            if (rotate) rot_pairs<8>(x1, x2, c, s);
+            store8<kSplit>(tile, lo, oa, x1);
+            store8<kSplit>(tile, lo, ob, x2);
         } else {
-            uint4 *pa = reinterpret_cast<uint4 *>(tile + chunk_off(r, ph.q));
+            const uint32_t oa = chunk_off(r, ph.q, BOX);
             float x[8];
-            unpack8(*pa, x);
-            float x1[4], x2[4];
+            unpack8(*reinterpret_cast<const uint4 *>(tile + oa), x);
+            if (rotate) {
+                float x1[4], x2[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                x1[e] = x[2 * e];
-                x2[e] = x[2 * e + 1];
-            }
-            rot_pairs<4>(x1, x2, c, s);
+                for (int e = 0; e < 4; ++e) {
+                    x1[e] = x[2 * e];
+                    x2[e] = x[2 * e + 1];
+                }
+                rot_pairs<4>(x1, x2, c, s);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                x[2 * e] = x1[e];
-                x[2 * e + 1] = x2[e];
+                for (int e = 0; e < 4; ++e) {
+                    x[2 * e] = x1[e];
+                    x[2 * e + 1] = x2[e];
+                }
             }
-            *pa = pack8(x);
+            store8<kSplit>(tile, lo, oa, x);
         }
-        ph.step(c, s);
+        if (rotate) ph.step(c, s);
     }
 }
 
-// fp32 operands: load 128 rows from global (rows >= L read as zero), rotate in
-// fp32 when asked, round to bf16 into the swizzled tile.
-template <int D, bool kHalf>
-__device__ __forceinline__ void load_tile_f32(uint8_t *tile, const float *base, long long rs,
-                                              int row0, int L, bool rotate,
+// fp32 operands: load ROWS rows from global (rows >= L read as zero), rotate in
+// fp32 when asked, round to bf16 (hi, and lo in the split mode) into the tile.
+template <int D, bool kHalf, bool kSplit, int ROWS>
+__device__ __forceinline__ void load_tile_f32(uint8_t *tile, uint8_t *lo, const float *base,
+                                              long long rs, int row0, int L, bool rotate,
                                               const Phasor<D, kHalf> &ph, const AttnParams &p) {
     using R = Rot<D, kHalf>;
+    constexpr int NJ = ROWS / R::RP;
+    constexpr int BOX = ROWS * 128;
     float c[R::PPJ], s[R::PPJ];
     if (rotate) ph.start(row0, p, c, s);
-    for (int k = 0; k < R::NJ; ++k) {
+    for (int k = 0; k < NJ; ++k) {
         const int r = ph.r0 + k * R::RP;
         const bool valid = row0 + r < L;
         const float *src = base + (long long)(row0 + r) * rs;
@@ -285,8 +324,8 @@ __device__ __forceinline__ void load_tile_f32(uint8_t *tile, const float *base, 
                 x2[e] = valid ? src[ph.i0 + e + D / 2] : 0.f;
             }
             if (rotate) rot_pairs<8>(x1, x2, c, s);
-            *reinterpret_cast<uint4 *>(tile + chunk_off(r, ph.q)) = pack8(x1);
-            *reinterpret_cast<uint4 *>(tile + chunk_off(r, ph.q + D / 16)) = pack8(x2);
+            store8<kSplit>(tile, lo, chunk_off(r, ph.q, BOX), x1);
+            store8<kSplit>(tile, lo, chunk_off(r, ph.q + D / 16, BOX), x2);
         } else {
             float x[8];
 #pragma unroll
@@ -305,39 +344,43 @@ __device__ __forceinline__ void load_tile_f32(uint8_t *tile, const float *base, 
                     x[2 * e + 1] = x2[e];
                 }
             }
-            *reinterpret_cast<uint4 *>(tile + chunk_off(r, ph.q)) = pack8(x);
+            store8<kSplit>(tile, lo, chunk_off(r, ph.q, BOX), x);
         }
         if (rotate) ph.step(c, s);
     }
 }
 
 // fp32 V tile: convert only.
-template <int D>
+template <int D, int ROWS>
 __device__ __forceinline__ void load_v_f32(uint8_t *tile, const float *base, long long rs, int row0,
                                            int L, int tw) {
     constexpr int CPR = D / 8;
-    for (int idx = tw; idx < kBN * CPR; idx += 128) {
+    constexpr int BOX = ROWS * 128;
+    for (int idx = tw; idx < ROWS * CPR; idx += 128) {
         const int r = idx / CPR, fc = idx % CPR;
         const bool valid = row0 + r < L;
         const float *src = base + (long long)(row0 + r) * rs + fc * 8;
         float x[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[e] = valid ? src[e] : 0.f;
-        *reinterpret_cast<uint4 *>(tile + chunk_off(r, fc)) = pack8(x);
+        *reinterpret_cast<uint4 *>(tile + chunk_off(r, fc, BOX)) = pack8(x);
     }
 }
 
 // ---------------------------------------------------------------- kernel
-template <int D, bool kF32, bool kHalf>
+template <int D, bool kF32, bool kHalf, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq,
                     const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, const __grid_constant__ AttnParams p) {
-    using C = Cfg<D>;
+    using C = Cfg<D, kSplit>;
     constexpr int NS = C::kStages;
+    constexpr int BN = C::BN;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // Q part x of tile t at sQ + (t * kParts + x) * kTileQ; K part x of stage s at
+    // sK + (s * kParts + x) * kTileK; V stage s at sV + s * kTileK.
     uint8_t *sQ = smem + C::kOffQ;
     uint8_t *sK = smem + C::kOffK;
     uint8_t *sV = smem + C::kOffV;
@@ -346,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const Unit U = decode_unit(p);
-    const Tiles T = make_tiles(U.q0, p);
+    const Tiles T = make_tiles<BN>(U.q0, p);
     volatile int *abort = &bar.abort;
     const uint64_t tmo = p.timeout_ns;
 
@@ -389,27 +432,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tmk);
             tma_prefetch_desc(&tmv);
             int issued_k[NS] = {}, issued_v[NS] = {};
-            mbar_arrive_expect_tx(&bar.full_q, U.nt * C::kTile);
+            mbar_arrive_expect_tx(&bar.full_q, U.nt * C::kTileQ);
             for (int t = 0; t < U.nt; ++t)
                 for (int bx = 0; bx < D / 64; ++bx)
-                    tma_load_4d(sQ + t * C::kTile + bx * kBoxBytes, &tmq, &bar.full_q, bx * 64,
-                                U.q0, U.hq0 + t, U.b);
+                    tma_load_4d(sQ + t * C::kParts * C::kTileQ + bx * C::kBoxQ, &tmq, &bar.full_q,
+                                bx * 64, U.q0, U.hq0 + t, U.b);
             bool ok = true;
             for (int j = 0; ok && j < T.n; ++j) {
                 const int s = j % NS, use = j / NS, jt = T.tile(j);
                 if (use > 0) ok = mbar_wait(&bar.empty_k[s], (use - 1) & 1, abort, tmo);
                 if (!ok) break;
-                mbar_arrive_expect_tx(&bar.full_k[s], C::kTile);
+                mbar_arrive_expect_tx(&bar.full_k[s], C::kTileK);
                 for (int bx = 0; bx < D / 64; ++bx)
-                    tma_load_4d(sK + s * C::kTile + bx * kBoxBytes, &tmk, &bar.full_k[s], bx * 64,
-                                jt * kBN, U.g, U.b);
+                    tma_load_4d(sK + s * C::kParts * C::kTileK + bx * C::kBoxK, &tmk,
+                                &bar.full_k[s], bx * 64, jt * BN, U.g, U.b);
                 ++issued_k[s];
                 if (use > 0) ok = mbar_wait(&bar.empty_v[s], (use - 1) & 1, abort, tmo);
                 if (!ok) break;
-                mbar_arrive_expect_tx(&bar.full_v[s], C::kTile);
+                mbar_arrive_expect_tx(&bar.full_v[s], C::kTileK);
                 for (int bx = 0; bx < D / 64; ++bx)
-                    tma_load_4d(sV + s * C::kTile + bx * kBoxBytes, &tmv, &bar.full_v[s], bx * 64,
-                                jt * kBN, U.g, U.b);
+                    tma_load_4d(sV + s * C::kTileK + bx * C::kBoxK, &tmv, &bar.full_v[s], bx * 64,
+                                jt * BN, U.g, U.b);
                 ++issued_v[s];
             }
             // Never leave the CTA with copies in flight: wait (bounded, even
@@ -423,20 +466,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp >= kWarpRot0 && warp < kWarpRot0 + 4) {
         // ------------------------------------------------ rotation warpgroup
         const int tw = threadIdx.x - kWarpRot0 * 32;
+        const bool rot = p.rotate != 0;
         Phasor<D, kHalf> ph;
         ph.init(tw, p);
         bool ok = true;
         if (!kF32) {
             ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_q, 0, abort, tmo));
-            if (ok && p.rotate)
-                for (int t = 0; t < U.nt; ++t)
-                    rotate_tile_bf16<D, kHalf>(sQ + t * C::kTile, U.q0, ph, p);
+            if (ok && (rot || kSplit))
+                for (int t = 0; t < U.nt; ++t) {
+                    uint8_t *qt = sQ + t * C::kParts * C::kTileQ;
+                    rotate_tile_bf16<D, kHalf, kSplit, kBM>(qt, qt + C::kTileQ, U.q0, ph, p, rot);
+                }
         } else {
             for (int t = 0; t < U.nt; ++t) {
                 const float *base = reinterpret_cast<const float *>(p.q) + U.b * p.qs[0] +
                                     (long long)(U.hq0 + t) * p.qs[1];
-                load_tile_f32<D, kHalf>(sQ + t * C::kTile, base, p.qs[2], U.q0, p.L, p.rotate != 0,
-                                        ph, p);
+                uint8_t *qt = sQ + t * C::kParts * C::kTileQ;
+                load_tile_f32<D, kHalf, kSplit, kBM>(qt, qt + C::kTileQ, base, p.qs[2], U.q0, p.L,
+                                                     rot, ph, p);
             }
         }
         if (ok) {
@@ -445,11 +492,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int j = 0; ok && j < T.n; ++j) {
             const int s = j % NS, use = j / NS, jt = T.tile(j);
-            uint8_t *tk = sK + s * C::kTile;
+            uint8_t *tk = sK + s * C::kParts * C::kTileK;
             if (!kF32) {
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_k[s], use & 1, abort, tmo));
                 if (!ok) break;
-                if (p.rotate) rotate_tile_bf16<D, kHalf>(tk, (long long)jt * kBN, ph, p);
+                if (rot || kSplit)
+                    rotate_tile_bf16<D, kHalf, kSplit, BN>(tk, tk + C::kTileK, (long long)jt * BN,
+                                                           ph, p, rot);
             } else {
                 if (use > 0)
                     ok = __all_sync(0xffffffffu,
@@ -457,7 +506,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 const float *base = reinterpret_cast<const float *>(p.k) + U.b * p.ks[0] +
                                     (long long)U.g * p.ks[1];
-                load_tile_f32<D, kHalf>(tk, base, p.ks[2], jt * kBN, p.L, p.rotate != 0, ph, p);
+                load_tile_f32<D, kHalf, kSplit, BN>(tk, tk + C::kTileK, base, p.ks[2], jt * BN,
+                                                    p.L, rot, ph, p);
             }
             fence_proxy_async_smem();
             mbar_arrive(&bar.ready_k[s]);
@@ -468,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 const float *base = reinterpret_cast<const float *>(p.v) + U.b * p.vs[0] +
                                     (long long)U.g * p.vs[1];
-                load_v_f32<D>(sV + s * C::kTile, base, p.vs[2], jt * kBN, p.L, tw);
+                load_v_f32<D, BN>(sV + s * C::kTileK, base, p.vs[2], jt * BN, p.L, tw);
                 fence_proxy_async_smem();
                 mbar_arrive(&bar.full_v[s]);
             }
@@ -476,24 +526,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kWarpMma) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t kIdS = idesc_bf16_f32(128, kBN, 0, 0);
+            constexpr uint32_t kIdS = idesc_bf16_f32(128, BN, 0, 0);
             constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, 0, 1);
             const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+            // S_t = Q_t K^T over D in steps of 16 (32 bytes inside a 128-byte
+            // swizzle row, then the next 64-column box).  Split mode:
+            // S = Qhi Klo + Qlo Khi + Qhi Khi, all accumulated in fp32.
             auto issue_s = [&](int t, int s) {
-                const uint32_t qa = q_addr + t * C::kTile, ka = k_addr + s * C::kTile;
+                const uint32_t qa = q_addr + t * C::kParts * C::kTileQ;
+                const uint32_t ka = k_addr + s * C::kParts * C::kTileK;
+                constexpr int NPROD = kSplit ? 3 : 1;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                    mma_ss(tmem + t * 128, sdesc_sw128(qa + off, 16, 1024),
-                           sdesc_sw128(ka + off, 16, 1024), kIdS, kk > 0);
+                for (int pr = 0; pr < NPROD; ++pr) {
+                    const uint32_t qp = qa + ((kSplit && pr == 1) ? C::kTileQ : 0);
+                    const uint32_t kp = ka + ((kSplit && pr == 0) ? C::kTileK : 0);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t oq = (kk >> 2) * C::kBoxQ + (kk & 3) * 32;
+                        const uint32_t ok_ = (kk >> 2) * C::kBoxK + (kk & 3) * 32;
+                        mma_ss(tmem + t * BN, sdesc_sw128(qp + oq, 16, 1024),
+                               sdesc_sw128(kp + ok_, 16, 1024), kIdS, (pr > 0 || kk > 0));
+                    }
                 }
             };
+            // O_t += P_t V: P from TMEM (BN/2 columns of bf16 pairs), V MN-major.
             auto issue_pv = [&](int t, int s, bool acc) {
-                const uint32_t va = v_addr + s * C::kTile;
+                const uint32_t va = v_addr + s * C::kTileK;
 #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk)
-                    mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8,
-                           sdesc_sw128(va + kk * 2048, kBoxBytes, 1024), kIdPV, (acc || kk > 0));
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    mma_ts(tmem + C::kColO + t * D, tmem + t * BN + kk * 8,
+                           sdesc_sw128(va + kk * 2048, C::kBoxK, 1024), kIdPV, (acc || kk > 0));
             };
             bool ok = mbar_wait(&bar.ready_q, 0, abort, tmo);
             if (ok) ok = mbar_wait(&bar.ready_k[0], 0, abort, tmo);
@@ -541,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
         const uint32_t trow = tmem + (uint32_t(wq * 32) << 16);
-        const uint32_t s_col = t * 128, o_col = 256 + t * D;
+        const uint32_t s_col = t * BN, o_col = C::kColO + t * D;
         const int i = U.q0 + row;
         const float cl2 = p.c_log2;
         float m = -INFINITY, l = 0.f;
@@ -550,8 +612,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_ready[t], j & 1, abort, tmo));
             if (!ok) break;
             tc_fence_after();
-            const int jt = T.tile(j), k0 = jt * kBN;
-            const bool partial = !tile_full(U.q0, jt, p);
+            const int jt = T.tile(j), k0 = jt * BN;
+            const bool partial = !tile_full<BN>(U.q0, jt, p);
             // visible columns: col <= hi and (no window or col >= lo or col < sk)
             const int hi = p.causal ? min(i - k0, p.L - 1 - k0) : p.L - 1 - k0;
             const int lo = i - p.window + 1 - k0;
@@ -559,20 +621,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool win = p.causal && p.window > 0;
             auto vis = [&](int col) { return col <= hi && (!win || col >= lo || col < sk); };
 
-            // pass 1: row max
+            // pass 1: row max, 64 columns per TMEM load
             float mx = -INFINITY;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                float v[32];
-                tmem_ld32(trow + s_col + c * 32, v);
+            for (int c = 0; c < BN / 64; ++c) {
+                float v[64];
+                tmem_ld64(trow + s_col + c * 64, v);
                 if (partial) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (!vis(c * 32 + e)) v[e] = -INFINITY;
+                    for (int e = 0; e < 64; ++e)
+                        if (!vis(c * 64 + e)) v[e] = -INFINITY;
                 }
                 float m0 = v[0], m1 = v[1], m2 = v[2], m3 = v[3];
 #pragma unroll
-                for (int e = 4; e < 32; e += 4) {
+                for (int e = 4; e < 64; e += 4) {
                     m0 = fmaxf(m0, v[e]);
                     m1 = fmaxf(m1, v[e + 1]);
                     m2 = fmaxf(m2, v[e + 2]);
@@ -603,37 +665,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (m == -INFINITY) m = m_new;
             const float mref = (m == -INFINITY) ? 0.f : m;
             // pass 2: P = 2^(s c - m) as bf16 written over the first half of S
-            float lsum = 0.f;
+            float lsum0 = 0.f, lsum1 = 0.f;
 #pragma unroll 1
-            for (int h = 0; h < 2; ++h) {
-                float a[32], b[32];
-                tmem_ld32(trow + s_col + h * 64, a);
-                tmem_ld32(trow + s_col + h * 64 + 32, b);
+            for (int h = 0; h < BN / 64; ++h) {
+                float a[64];
+                tmem_ld64(trow + s_col + h * 64, a);
                 if (partial) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
+                    for (int e = 0; e < 64; ++e)
                         if (!vis(h * 64 + e)) a[e] = -INFINITY;
-                        if (!vis(h * 64 + 32 + e)) b[e] = -INFINITY;
-                    }
                 }
                 uint32_t pk[32];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
+                for (int e = 0; e < 32; ++e) {
                     const float p0 = ex2_approx(fmaf(a[2 * e], cl2, -mref));
                     const float p1 = ex2_approx(fmaf(a[2 * e + 1], cl2, -mref));
-                    lsum += p0 + p1;
+                    lsum0 += p0;
+                    lsum1 += p1;
                     pk[e] = pack_bf16x2(p0, p1);
-                }
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float p0 = ex2_approx(fmaf(b[2 * e], cl2, -mref));
-                    const float p1 = ex2_approx(fmaf(b[2 * e + 1], cl2, -mref));
-                    lsum += p0 + p1;
-                    pk[16 + e] = pack_bf16x2(p0, p1);
                 }
                 tmem_st32(trow + s_col + h * 32, pk);
             }
-            l += lsum;
+            l += lsum0 + lsum1;
             tc_fence_before();
             mbar_arrive(&bar.p_ready[t]);
         }
@@ -703,14 +756,14 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [B, H, L, D] bf16 tensor -> 4-D tensor map with 64 x 128 boxes, 128-byte swizzle.
+// [B, H, L, D] bf16 tensor -> 4-D tensor map with 64 x box_rows boxes, 128-byte swizzle.
 lcx_status make_map(CUtensorMap *map, const void *ptr, int64_t B, int64_t H, int64_t L, int64_t D,
-                    const int64_t *st, const char *name) {
+                    const int64_t *st, uint32_t box_rows, const char *name) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(LCX_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(L), cuuint64_t(H), cuuint64_t(B)};
     cuuint64_t strides[3] = {cuuint64_t(st[2] * 2), cuuint64_t(st[1] * 2), cuuint64_t(st[0] * 2)};
-    cuuint32_t box[4] = {64, 128, 1, 1};
+    cuuint32_t box[4] = {64, box_rows, 1, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -720,11 +773,11 @@ lcx_status make_map(CUtensorMap *map, const void *ptr, int64_t B, int64_t H, int
     return LCX_OK;
 }
 
-template <int D, bool kF32, bool kHalf>
+template <int D, bool kF32, bool kHalf, bool kSplit>
 lcx_status launch(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                   const AttnParams &p, unsigned grid, cudaStream_t s) {
-    auto kern = attn_fwd_kernel<D, kF32, kHalf>;
-    const int smem = Cfg<D>::kSmemBytes;
+    auto kern = attn_fwd_kernel<D, kF32, kHalf, kSplit>;
+    const int smem = Cfg<D, kSplit>::kSmemBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
         return fail(LCX_ERR_CUDA, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
@@ -735,14 +788,14 @@ lcx_status launch(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMa
     return LCX_OK;
 }
 
-template <int D>
+template <int D, bool kSplit>
 lcx_status launch_d(bool f32, bool half, const CUtensorMap &mq, const CUtensorMap &mk,
                     const CUtensorMap &mv, const AttnParams &p, unsigned grid, cudaStream_t s) {
     if (f32)
-        return half ? launch<D, true, true>(mq, mk, mv, p, grid, s)
-                    : launch<D, true, false>(mq, mk, mv, p, grid, s);
-    return half ? launch<D, false, true>(mq, mk, mv, p, grid, s)
-                : launch<D, false, false>(mq, mk, mv, p, grid, s);
+        return half ? launch<D, true, true, kSplit>(mq, mk, mv, p, grid, s)
+                    : launch<D, true, false, kSplit>(mq, mk, mv, p, grid, s);
+    return half ? launch<D, false, true, kSplit>(mq, mk, mv, p, grid, s)
+                : launch<D, false, false, kSplit>(mq, mk, mv, p, grid, s);
 }
 
 lcx_status check_tensor(const void *ptr, const int64_t *st, int es, const char *name) {
@@ -779,7 +832,8 @@ extern "C" lcx_status lcx_attn_fwd(const lcx_attn_args *a, void *stream) {
         return fail(LCX_ERR_INVALID_ARG, "window and sinks must be >= 0");
     if (!a->causal && (a->window != 0 || a->sinks != 0))
         return fail(LCX_ERR_UNSUPPORTED, "window / sinks need causal attention");
-    if (a->flags & ~uint32_t(LCX_ATTN_PREROTATED)) return fail(LCX_ERR_INVALID_ARG, "unknown flags");
+    if (a->flags & ~uint32_t(LCX_ATTN_PREROTATED | LCX_ATTN_SPLIT_QK))
+        return fail(LCX_ERR_INVALID_ARG, "unknown flags");
     if (!(a->softmax_scale >= 0.f) || !std::isfinite(a->softmax_scale))
         return fail(LCX_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
     if (a->D != 64 && a->D != 128)
@@ -828,18 +882,26 @@ extern "C" lcx_status lcx_attn_fwd(const lcx_attn_args *a, void *stream) {
     p.c_log2 = float(scale * msq * 1.4426950408889634);
     p.timeout_ns = 2000000000ull;  // 2 s: legitimate waits last microseconds
 
+    const bool split = (a->flags & LCX_ATTN_SPLIT_QK) != 0;
+    const uint32_t bn = split ? 64u : 128u;
     CUtensorMap mq, mk, mv;
     memset(&mq, 0, sizeof(mq));
     memset(&mk, 0, sizeof(mk));
     memset(&mv, 0, sizeof(mv));
     if (a->dtype == LCX_BF16) {
-        if ((st = make_map(&mq, a->q, a->B, a->Hq, a->L, a->D, a->q_strides, "q")) != LCX_OK) return st;
-        if ((st = make_map(&mk, a->k, a->B, a->Hkv, a->L, a->D, a->k_strides, "k")) != LCX_OK) return st;
-        if ((st = make_map(&mv, a->v, a->B, a->Hkv, a->L, a->D, a->v_strides, "v")) != LCX_OK) return st;
+        if ((st = make_map(&mq, a->q, a->B, a->Hq, a->L, a->D, a->q_strides, 128, "q")) != LCX_OK)
+            return st;
+        if ((st = make_map(&mk, a->k, a->B, a->Hkv, a->L, a->D, a->k_strides, bn, "k")) != LCX_OK)
+            return st;
+        if ((st = make_map(&mv, a->v, a->B, a->Hkv, a->L, a->D, a->v_strides, bn, "v")) != LCX_OK)
+            return st;
     }
     const bool f32 = a->dtype == LCX_F32;
     const bool half = a->rope.pairing == LCX_PAIR_HALF;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (a->D == 128) return launch_d<128>(f32, half, mq, mk, mv, p, unsigned(grid), s);
-    return launch_d<64>(f32, half, mq, mk, mv, p, unsigned(grid), s);
+    if (a->D == 128)
+        return split ? launch_d<128, true>(f32, half, mq, mk, mv, p, unsigned(grid), s)
+                     : launch_d<128, false>(f32, half, mq, mk, mv, p, unsigned(grid), s);
+    return split ? launch_d<64, true>(f32, half, mq, mk, mv, p, unsigned(grid), s)
+                 : launch_d<64, false>(f32, half, mq, mk, mv, p, unsigned(grid), s);
 }

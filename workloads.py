@@ -39,6 +39,7 @@ class Workload:
     softmax_scale: float = 0.0  # 0 -> 1/sqrt(D)
     outlier_frac: float = 0.0
     outlier_mult: float = 8.0
+    split_qk: bool = False     # form QK^T from hi/lo bf16 parts (outlier-heavy inputs)
     seed: int = 0
     description: str = ""
 
@@ -81,7 +82,7 @@ WORKLOADS = {
     "sink_window_L65536": Workload(
         "sink_window_L65536", B=4, Hq=32, Hkv=8, L=65536, D=128, dtype="bf16", mode="yarn",
         scale=8.0, original_max_pos=8192, alpha=1.0, beta=32.0, window=4096, sinks=4,
-        outlier_frac=0.01, outlier_mult=8.0,
+        outlier_frac=0.01, outlier_mult=8.0, split_qk=True,
         description="4 sink tokens + window 4096, batch 4, seq 65536, YaRN s=8, 1% outliers x8"),
 }
 
