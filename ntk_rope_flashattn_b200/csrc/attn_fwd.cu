@@ -680,9 +680,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = 0; e < 32; ++e) {
                     const float p0 = ex2_approx(fmaf(a[2 * e], cl2, -mref));
                     const float p1 = ex2_approx(fmaf(a[2 * e + 1], cl2, -mref));
-                    lsum0 += p0;
-                    lsum1 += p1;
                     pk[e] = pack_bf16x2(p0, p1);
+                    if (kSplit) {
+                        // Normalise by the weights the tensor core actually
+                        // multiplies V with (bf16), not their fp32 values: with
+                        // the stale max reference the dominant weight is 2^d,
+                        // d in [0, 8], and its rounding must cancel in o.
+                        lsum0 += bf16lo_to_f32(pk[e]);
+                        lsum1 += bf16hi_to_f32(pk[e]);
+                    } else {
+                        lsum0 += p0;
+                        lsum1 += p1;
+                    }
                 }
                 tmem_st32(trow + s_col + h * 32, pk);
             }
