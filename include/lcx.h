@@ -132,6 +132,11 @@ LCX_API lcx_status lcx_apply_rope(const lcx_rope_params *params, const void *x, 
                                    rotated operands (needed when the logits are
                                    large, e.g. outlier-heavy activations); about
                                    twice the tensor-core work for QK^T        */
+#define LCX_ATTN_TEST_STALL 0x80000000u /* test hook for the watchdog: the loader
+                                   issues no copies, so every wait of the
+                                   kernel expires after watchdog_ms and the
+                                   status word receives LCX_ERR_TIMEOUT; o is
+                                   left unwritten.  Never set in production.  */
 
 typedef struct {
     const void *q;             /* DEVICE [B, Hq, L, D]                            */
@@ -153,6 +158,8 @@ typedef struct {
                                   a window is set; 0 = none                       */
     float softmax_scale;       /* logit scale; 0 -> 1/sqrt(D)                     */
     uint32_t flags;            /* LCX_ATTN_* bits                                 */
+    int32_t watchdog_ms;       /* wall-clock limit of every device wait, 1..60000;
+                                  0 -> 2000 ms                                    */
 } lcx_attn_args;
 
 /*

@@ -26,6 +26,7 @@ PAIRINGS = {"half": 0, "interleaved": 1}
 DTYPES = {"bf16": 0, "f32": 1}
 LCX_ATTN_PREROTATED = 1
 LCX_ATTN_SPLIT_QK = 2
+LCX_ATTN_TEST_STALL = 0x80000000
 
 # Symbols include/lcx.h declares; the library must export every one of them.
 EXPORTED = ("lcx_rope_table", "lcx_apply_rope", "lcx_attn_fwd", "lcx_status_string",
@@ -59,7 +60,8 @@ class _AttnArgs(ctypes.Structure):
                 ("q_strides", ctypes.c_int64 * 4), ("k_strides", ctypes.c_int64 * 4),
                 ("v_strides", ctypes.c_int64 * 4), ("o_strides", ctypes.c_int64 * 4),
                 ("rope", _RopeParams), ("window", ctypes.c_int64), ("sinks", ctypes.c_int64),
-                ("softmax_scale", ctypes.c_float), ("flags", ctypes.c_uint32)]
+                ("softmax_scale", ctypes.c_float), ("flags", ctypes.c_uint32),
+                ("watchdog_ms", ctypes.c_int32)]
 
 
 @dataclass
@@ -181,7 +183,8 @@ def apply_rope(x, rope: RopeParams, out=None, pos_offset: int = 0, inplace: bool
 
 def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, sinks: int = 0,
              softmax_scale: float = 0.0, return_lse: bool = False, prerotated: bool = False,
-             split_qk: bool = False, out=None, lse=None, status=None):
+             split_qk: bool = False, out=None, lse=None, status=None, watchdog_ms: int = 0,
+             _test_stall: bool = False):
     """Fused RoPE + causal attention prefill.
 
     q [B, Hq, L, D], k/v [B, Hkv, L, D] CUDA tensors (bf16 or fp32, last dim
@@ -216,7 +219,9 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
     a.rope = rope._c()
     a.window, a.sinks = int(window), int(sinks)
     a.softmax_scale = float(softmax_scale)
-    a.flags = (LCX_ATTN_PREROTATED if prerotated else 0) | (LCX_ATTN_SPLIT_QK if split_qk else 0)
+    a.flags = ((LCX_ATTN_PREROTATED if prerotated else 0) | (LCX_ATTN_SPLIT_QK if split_qk else 0)
+               | (LCX_ATTN_TEST_STALL if _test_stall else 0))
+    a.watchdog_ms = int(watchdog_ms)
     _check(load().lcx_attn_fwd(ctypes.byref(a), _stream(q)))
     return (o, lse) if return_lse else o
 

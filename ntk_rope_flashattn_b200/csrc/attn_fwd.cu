@@ -60,6 +60,7 @@ struct AttnParams {
     int causal, window, sinks;
     int n_qb, heads_per_unit, units_per_qb;
     int rotate;
+    int test_stall;                    // loader issues nothing (watchdog test hook)
     float c_log2;                      // logit scale in log2 units
     unsigned long long timeout_ns;
     float theta[64];
@@ -427,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // nothing to do: fall through to the common exit
     } else if (warp == kWarpTma) {
         // ------------------------------------------------ TMA producer
-        if (!kF32 && lane == 0) {
+        if (!kF32 && lane == 0 && !p.test_stall) {
             tma_prefetch_desc(&tmq);
             tma_prefetch_desc(&tmk);
             tma_prefetch_desc(&tmv);
@@ -841,8 +842,12 @@ extern "C" lcx_status lcx_attn_fwd(const lcx_attn_args *a, void *stream) {
         return fail(LCX_ERR_INVALID_ARG, "window and sinks must be >= 0");
     if (!a->causal && (a->window != 0 || a->sinks != 0))
         return fail(LCX_ERR_UNSUPPORTED, "window / sinks need causal attention");
-    if (a->flags & ~uint32_t(LCX_ATTN_PREROTATED | LCX_ATTN_SPLIT_QK))
+    if (a->flags & ~uint32_t(LCX_ATTN_PREROTATED | LCX_ATTN_SPLIT_QK | LCX_ATTN_TEST_STALL))
         return fail(LCX_ERR_INVALID_ARG, "unknown flags");
+    if (a->watchdog_ms < 0 || a->watchdog_ms > 60000)
+        return fail(LCX_ERR_INVALID_ARG, "watchdog_ms must be in [0, 60000]");
+    if ((a->flags & LCX_ATTN_TEST_STALL) && a->dtype != LCX_BF16)
+        return fail(LCX_ERR_UNSUPPORTED, "the stall test hook needs bf16 operands");
     if (!(a->softmax_scale >= 0.f) || !std::isfinite(a->softmax_scale))
         return fail(LCX_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
     if (a->D != 64 && a->D != 128)
@@ -889,7 +894,9 @@ extern "C" lcx_status lcx_attn_fwd(const lcx_attn_args *a, void *stream) {
     const double scale = a->softmax_scale > 0.f ? double(a->softmax_scale) : 1.0 / std::sqrt(double(a->D));
     const double msq = p.rotate ? double(ms) * double(ms) : 1.0;
     p.c_log2 = float(scale * msq * 1.4426950408889634);
-    p.timeout_ns = 2000000000ull;  // 2 s: legitimate waits last microseconds
+    // Legitimate waits last microseconds; the default limit is 2 s.
+    p.timeout_ns = 1000000ull * (unsigned long long)(a->watchdog_ms > 0 ? a->watchdog_ms : 2000);
+    p.test_stall = (a->flags & LCX_ATTN_TEST_STALL) ? 1 : 0;
 
     const bool split = (a->flags & LCX_ATTN_SPLIT_QK) != 0;
     const uint32_t bn = split ? 64u : 128u;

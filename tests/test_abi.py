@@ -65,7 +65,7 @@ int main(void) {
   P(lcx_attn_args, dev_status) P(lcx_attn_args, dtype) P(lcx_attn_args, B) P(lcx_attn_args, D)
   P(lcx_attn_args, q_strides) P(lcx_attn_args, o_strides) P(lcx_attn_args, rope)
   P(lcx_attn_args, window) P(lcx_attn_args, sinks) P(lcx_attn_args, softmax_scale)
-  P(lcx_attn_args, flags)
+  P(lcx_attn_args, flags) P(lcx_attn_args, watchdog_ms)
   return 0;
 }
 ''')
@@ -195,6 +195,9 @@ def _attn_args(**kw):
     (dict(q_strides=[8 * 256 * 128, 256 * 128, 132, 1]), lcx.LCX_ERR_UNSUPPORTED),
     (dict(v_strides=[2 * 256 * 128, 256 * 128, 128, 2]), lcx.LCX_ERR_UNSUPPORTED),
     (dict(Hq=0), lcx.LCX_ERR_INVALID_ARG),
+    (dict(watchdog_ms=-1), lcx.LCX_ERR_INVALID_ARG),
+    (dict(watchdog_ms=60001), lcx.LCX_ERR_INVALID_ARG),
+    (dict(dtype=1, flags=0x80000000), lcx.LCX_ERR_UNSUPPORTED),
 ])
 def test_attn_validation_without_device(lib, kw, expect):
     a = _attn_args(**kw)
