@@ -43,9 +43,24 @@
 namespace lcx {
 namespace {
 
-constexpr int kThreads = 448;           // 14 warps
+constexpr int kThreads = 512;           // 16 warps = 4 warpgroups
+// Registers per thread after the warpgroups re-balance (launch: 128 each;
+// 176 + 176 + 96 + 64 = 4 x 128, so the file is exactly used).
+constexpr int kRegsSoftmax = 176;       // warpgroups 0, 1: a whole S row in registers
+constexpr int kRegsRotate = 96;         // warpgroup 2
+constexpr int kRegsIssue = 64;          // warpgroup 3: TMA and MMA issuing warps
+static_assert(2 * kRegsSoftmax + kRegsRotate + kRegsIssue == 4 * 128, "register file split");
 constexpr int kBM = 128;                // query rows per tile
 constexpr float kRescaleLog2 = 8.0f;    // rescale O only if the max grows by > 2^8
+#ifndef LCX_EMU_EVERY
+#define LCX_EMU_EVERY 0
+#endif
+#ifndef LCX_KSTAGES_D128
+#define LCX_KSTAGES_D128 2
+#endif
+// 1 column pair in kEmuEvery takes 2^x on the FMA pipe (0 = all on the MUFU:
+// measured fastest here, since the MUFU is not the binding limit).
+constexpr int kEmuEvery = LCX_EMU_EVERY;
 constexpr int kWarpMma = 13;
 constexpr int kWarpTma = 12;
 constexpr int kWarpRot0 = 8;
@@ -78,11 +93,12 @@ struct Cfg {
     static constexpr int kTileK = BN * D * 2;           // one part of a K tile / a V tile
     static constexpr int kBoxQ = kBM * 128;
     static constexpr int kBoxK = BN * 128;
-    static constexpr int kStages = (D == 128) ? 2 : 4;
+    static constexpr int kStagesK = (D == 128) ? (kSplit ? 2 : LCX_KSTAGES_D128) : 4;
+    static constexpr int kStagesV = (D == 128) ? 2 : 4;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + 2 * kParts * kTileQ;
-    static constexpr int kOffV = kOffK + kStages * kParts * kTileK;
-    static constexpr int kOffBar = kOffV + kStages * kTileK;
+    static constexpr int kOffV = kOffK + kStagesK * kParts * kTileK;
+    static constexpr int kOffBar = kOffV + kStagesV * kTileK;
     static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers + alignment slack
     // TMEM columns: S_t at t*BN (P_t aliased over its first BN/2 columns), O_t after.
     static constexpr int kColO = 2 * BN;
@@ -90,11 +106,11 @@ struct Cfg {
     static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
 };
 
-template <int NS>
+template <int NSK, int NSV>
 struct Bars {
     uint64_t full_q, ready_q;
-    uint64_t full_k[NS], ready_k[NS], empty_k[NS];
-    uint64_t full_v[NS], empty_v[NS];
+    uint64_t full_k[NSK], ready_k[NSK], empty_k[NSK];
+    uint64_t full_v[NSV], empty_v[NSV];
     uint64_t s_ready[2], p_ready[2], o_ready[2];
     uint64_t drain;
     uint32_t tmem_base;
@@ -179,15 +195,22 @@ struct Rot {
     static constexpr int PPJ = kHalf ? 8 : 4;            // pairs per job
 };
 
-// Rotate one job's pairs: x1/x2 are the pair members, (c, s) the phasor.
+// Rotate one job's pairs, two pairs per packed instruction: x1/x2 are the pair
+// members, (c, s) the phasor: x1' = x1 c - x2 s, x2' = x1 s + x2 c.
 template <int N>
 __device__ __forceinline__ void rot_pairs(float (&x1)[N], float (&x2)[N], const float *c,
                                           const float *s) {
 #pragma unroll
-    for (int e = 0; e < N; ++e) {
-        const float a = x1[e], b = x2[e];
-        x1[e] = fmaf(a, c[e], -b * s[e]);
-        x2[e] = fmaf(a, s[e], b * c[e]);
+    for (int e = 0; e < N; e += 2) {
+        const float2 a = make_float2(x1[e], x1[e + 1]), b = make_float2(x2[e], x2[e + 1]);
+        const float2 cc = make_float2(c[e], c[e + 1]), ss = make_float2(s[e], s[e + 1]);
+        const float2 nss = make_float2(-s[e], -s[e + 1]);
+        const float2 y1 = fma2(b, nss, mul2(a, cc));
+        const float2 y2 = fma2(a, ss, mul2(b, cc));
+        x1[e] = y1.x;
+        x1[e + 1] = y1.y;
+        x2[e] = y2.x;
+        x2[e + 1] = y2.y;
     }
 }
 
@@ -247,11 +270,16 @@ struct Phasor {
     }
     __device__ __forceinline__ void step(float (&c)[R::PPJ], float (&s)[R::PPJ]) const {
 #pragma unroll
-        for (int e = 0; e < R::PPJ; ++e) {
-            const float nc = fmaf(c[e], sc[e], -s[e] * ss[e]);
-            const float ns = fmaf(c[e], ss[e], s[e] * sc[e]);
-            c[e] = nc;
-            s[e] = ns;
+        for (int e = 0; e < R::PPJ; e += 2) {
+            const float2 cc = make_float2(c[e], c[e + 1]), s2 = make_float2(s[e], s[e + 1]);
+            const float2 stc = make_float2(sc[e], sc[e + 1]), sts = make_float2(ss[e], ss[e + 1]);
+            const float2 nsts = make_float2(-ss[e], -ss[e + 1]);
+            const float2 nc = fma2(cc, stc, mul2(s2, nsts));
+            const float2 ns = fma2(cc, sts, mul2(s2, stc));
+            c[e] = nc.x;
+            c[e + 1] = nc.y;
+            s[e] = ns.x;
+            s[e + 1] = ns.y;
         }
     }
 };
@@ -368,6 +396,35 @@ __device__ __forceinline__ void load_v_f32(uint8_t *tile, const float *base, lon
     }
 }
 
+// Whole-row TMEM access for the softmax (128 or 64 columns).
+__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, float (&v)[128]) { tmem_ld128(taddr, v); }
+__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, float (&v)[64]) { tmem_ld64(taddr, v); }
+__device__ __forceinline__ void tmem_st_row(uint32_t taddr, const uint32_t (&u)[64]) {
+    tmem_st64(taddr, u);
+}
+__device__ __forceinline__ void tmem_st_row(uint32_t taddr, const uint32_t (&u)[32]) {
+    tmem_st32(taddr, u);
+}
+
+// Max of N values (N % 8 == 0) with four independent chains of 3-input max:
+// v[0..3] start the chains, v[4 .. N-5] are taken 8 at a time, v[N-4 .. N-1]
+// close them.
+template <int N>
+__device__ __forceinline__ float row_max(const float (&v)[N]) {
+    static_assert(N % 8 == 0 && N >= 16, "row_max layout");
+    float m0 = v[0], m1 = v[1], m2 = v[2], m3 = v[3];
+#pragma unroll
+    for (int e = 4; e + 8 <= N - 4; e += 8) {
+        m0 = max3(m0, v[e], v[e + 1]);
+        m1 = max3(m1, v[e + 2], v[e + 3]);
+        m2 = max3(m2, v[e + 4], v[e + 5]);
+        m3 = max3(m3, v[e + 6], v[e + 7]);
+    }
+    m0 = max3(m0, v[N - 4], v[N - 3]);
+    m1 = max3(m1, v[N - 2], v[N - 1]);
+    return fmaxf(max3(m0, m1, m2), m3);
+}
+
 // ---------------------------------------------------------------- kernel
 template <int D, bool kF32, bool kHalf, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -375,7 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, const __grid_constant__ AttnParams p) {
     using C = Cfg<D, kSplit>;
-    constexpr int NS = C::kStages;
+    constexpr int NSK = C::kStagesK;
+    constexpr int NSV = C::kStagesV;
     constexpr int BN = C::BN;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -385,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *sQ = smem + C::kOffQ;
     uint8_t *sK = smem + C::kOffK;
     uint8_t *sV = smem + C::kOffV;
-    Bars<NS> &bar = *reinterpret_cast<Bars<NS> *>(smem + C::kOffBar);
+    Bars<NSK, NSV> &bar = *reinterpret_cast<Bars<NSK, NSV> *>(smem + C::kOffBar);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -397,10 +455,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(&bar.full_q, 1);
         mbar_init(&bar.ready_q, 128);
-        for (int s = 0; s < NS; ++s) {
+        for (int s = 0; s < NSK; ++s) {
             mbar_init(&bar.full_k[s], 1);
             mbar_init(&bar.ready_k[s], 128);
             mbar_init(&bar.empty_k[s], 1);
+        }
+        for (int s = 0; s < NSV; ++s) {
             mbar_init(&bar.full_v[s], kF32 ? 128 : 1);
             mbar_init(&bar.empty_v[s], 1);
         }
@@ -424,47 +484,128 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = bar.tmem_base;
     const bool skip = bar.abort != 0;
 
+
     if (skip) {
         // nothing to do: fall through to the common exit
-    } else if (warp == kWarpTma) {
-        // ------------------------------------------------ TMA producer
-        if (!kF32 && lane == 0 && !p.test_stall) {
-            tma_prefetch_desc(&tmq);
-            tma_prefetch_desc(&tmk);
-            tma_prefetch_desc(&tmv);
-            int issued_k[NS] = {}, issued_v[NS] = {};
-            mbar_arrive_expect_tx(&bar.full_q, U.nt * C::kTileQ);
-            for (int t = 0; t < U.nt; ++t)
-                for (int bx = 0; bx < D / 64; ++bx)
-                    tma_load_4d(sQ + t * C::kParts * C::kTileQ + bx * C::kBoxQ, &tmq, &bar.full_q,
-                                bx * 64, U.q0, U.hq0 + t, U.b);
-            bool ok = true;
-            for (int j = 0; ok && j < T.n; ++j) {
-                const int s = j % NS, use = j / NS, jt = T.tile(j);
-                if (use > 0) ok = mbar_wait(&bar.empty_k[s], (use - 1) & 1, abort, tmo);
-                if (!ok) break;
-                mbar_arrive_expect_tx(&bar.full_k[s], C::kTileK);
-                for (int bx = 0; bx < D / 64; ++bx)
-                    tma_load_4d(sK + s * C::kParts * C::kTileK + bx * C::kBoxK, &tmk,
-                                &bar.full_k[s], bx * 64, jt * BN, U.g, U.b);
-                ++issued_k[s];
-                if (use > 0) ok = mbar_wait(&bar.empty_v[s], (use - 1) & 1, abort, tmo);
-                if (!ok) break;
-                mbar_arrive_expect_tx(&bar.full_v[s], C::kTileK);
-                for (int bx = 0; bx < D / 64; ++bx)
-                    tma_load_4d(sV + s * C::kTileK + bx * C::kBoxK, &tmv, &bar.full_v[s], bx * 64,
-                                jt * BN, U.g, U.b);
-                ++issued_v[s];
+    } else if ((warp >> 2) == 3) {
+        // warpgroup 3: warp 12 issues the TMA copies, warp 13 the MMAs
+        setmaxnreg_dec<kRegsIssue>();
+        if (warp == kWarpTma) {
+            // ------------------------------------------------ TMA producer
+            if (!kF32 && lane == 0 && !p.test_stall) {
+                tma_prefetch_desc(&tmq);
+                tma_prefetch_desc(&tmk);
+                tma_prefetch_desc(&tmv);
+                int issued_k[NSK] = {}, issued_v[NSV] = {};
+                mbar_arrive_expect_tx(&bar.full_q, U.nt * C::kTileQ);
+                for (int t = 0; t < U.nt; ++t)
+                    for (int bx = 0; bx < D / 64; ++bx)
+                        tma_load_4d(sQ + t * C::kParts * C::kTileQ + bx * C::kBoxQ, &tmq, &bar.full_q,
+                                    bx * 64, U.q0, U.hq0 + t, U.b);
+                bool ok = true;
+                for (int j = 0; ok && j < T.n; ++j) {
+                    const int jt = T.tile(j);
+                    const int sk = j % NSK, uk = j / NSK, sv = j % NSV, uv = j / NSV;
+                    if (uk > 0) ok = mbar_wait(&bar.empty_k[sk], (uk - 1) & 1, abort, tmo);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&bar.full_k[sk], C::kTileK);
+                    for (int bx = 0; bx < D / 64; ++bx)
+                        tma_load_4d(sK + sk * C::kParts * C::kTileK + bx * C::kBoxK, &tmk,
+                                    &bar.full_k[sk], bx * 64, jt * BN, U.g, U.b);
+                    ++issued_k[sk];
+                    if (uv > 0) ok = mbar_wait(&bar.empty_v[sv], (uv - 1) & 1, abort, tmo);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&bar.full_v[sv], C::kTileK);
+                    for (int bx = 0; bx < D / 64; ++bx)
+                        tma_load_4d(sV + sv * C::kTileK + bx * C::kBoxK, &tmv, &bar.full_v[sv],
+                                    bx * 64, jt * BN, U.g, U.b);
+                    ++issued_v[sv];
+                }
+                // Never leave the CTA with copies in flight: wait (bounded, even
+                // after an abort) for the last load issued to every buffer.
+                mbar_wait(&bar.full_q, 0, nullptr, tmo);
+                for (int s = 0; s < NSK; ++s)
+                    if (issued_k[s]) mbar_wait(&bar.full_k[s], (issued_k[s] - 1) & 1, nullptr, tmo);
+                for (int s = 0; s < NSV; ++s)
+                    if (issued_v[s]) mbar_wait(&bar.full_v[s], (issued_v[s] - 1) & 1, nullptr, tmo);
             }
-            // Never leave the CTA with copies in flight: wait (bounded, even
-            // after an abort) for the last load issued to every buffer.
-            mbar_wait(&bar.full_q, 0, nullptr, tmo);
-            for (int s = 0; s < NS; ++s) {
-                if (issued_k[s]) mbar_wait(&bar.full_k[s], (issued_k[s] - 1) & 1, nullptr, tmo);
-                if (issued_v[s]) mbar_wait(&bar.full_v[s], (issued_v[s] - 1) & 1, nullptr, tmo);
+        } else if (warp == kWarpMma) {
+            // ------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t kIdS = idesc_bf16_f32(128, BN, 0, 0);
+                constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, 0, 1);
+                const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+                // S_t = Q_t K^T over D in steps of 16 (32 bytes inside a 128-byte
+                // swizzle row, then the next 64-column box).  Split mode:
+                // S = Qhi Klo + Qlo Khi + Qhi Khi, all accumulated in fp32.
+                auto issue_s = [&](int t, int s) {
+                    const uint32_t qa = q_addr + t * C::kParts * C::kTileQ;
+                    const uint32_t ka = k_addr + s * C::kParts * C::kTileK;
+                    constexpr int NPROD = kSplit ? 3 : 1;
+    #pragma unroll
+                    for (int pr = 0; pr < NPROD; ++pr) {
+                        const uint32_t qp = qa + ((kSplit && pr == 1) ? C::kTileQ : 0);
+                        const uint32_t kp = ka + ((kSplit && pr == 0) ? C::kTileK : 0);
+    #pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t oq = (kk >> 2) * C::kBoxQ + (kk & 3) * 32;
+                            const uint32_t ok_ = (kk >> 2) * C::kBoxK + (kk & 3) * 32;
+                            mma_ss(tmem + t * BN, sdesc_sw128(qp + oq, 16, 1024),
+                                   sdesc_sw128(kp + ok_, 16, 1024), kIdS, (pr > 0 || kk > 0));
+                        }
+                    }
+                };
+                // O_t += P_t V: P from TMEM (BN/2 columns of bf16 pairs), V MN-major.
+                auto issue_pv = [&](int t, int s, bool acc) {
+                    const uint32_t va = v_addr + s * C::kTileK;
+    #pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        mma_ts(tmem + C::kColO + t * D, tmem + t * BN + kk * 8,
+                               sdesc_sw128(va + kk * 2048, C::kBoxK, 1024), kIdPV, (acc || kk > 0));
+                };
+                bool ok = mbar_wait(&bar.ready_q, 0, abort, tmo);
+                if (ok) ok = mbar_wait(&bar.ready_k[0], 0, abort, tmo);
+                tc_fence_after();
+                if (ok) {
+                    for (int t = 0; t < U.nt; ++t) {
+                        issue_s(t, 0);
+                        mma_commit(&bar.s_ready[t]);
+                    }
+                    mma_commit(&bar.empty_k[0]);
+                }
+                for (int j = 0; ok && j < T.n; ++j) {
+                    const int sv = j % NSV;
+                    ok = mbar_wait(&bar.full_v[sv], (j / NSV) & 1, abort, tmo);
+                    for (int t = 0; ok && t < U.nt; ++t) {
+                        ok = mbar_wait(&bar.p_ready[t], j & 1, abort, tmo);
+                        tc_fence_after();
+                        if (!ok) break;
+                        issue_pv(t, sv, j > 0);
+                        if (j + 1 < T.n) {
+                            const int sk = (j + 1) % NSK;
+                            if (t == 0) {
+                                ok = mbar_wait(&bar.ready_k[sk], ((j + 1) / NSK) & 1, abort, tmo);
+                                tc_fence_after();
+                                if (!ok) break;
+                            }
+                            issue_s(t, sk);
+                            mma_commit(&bar.s_ready[t]);
+                        }
+                    }
+                    if (ok) {
+                        mma_commit(&bar.empty_v[sv]);
+                        if (j + 1 < T.n) mma_commit(&bar.empty_k[(j + 1) % NSK]);
+                    }
+                }
+                if (ok)
+                    for (int t = 0; t < U.nt; ++t) mma_commit(&bar.o_ready[t]);
+                // Drain: all issued MMAs complete before TMEM is released.
+                mma_commit(&bar.drain);
+                mbar_wait(&bar.drain, 0, nullptr, tmo);
             }
         }
-    } else if (warp >= kWarpRot0 && warp < kWarpRot0 + 4) {
+    } else if ((warp >> 2) == 2) {
+        setmaxnreg_dec<kRegsRotate>();
         // ------------------------------------------------ rotation warpgroup
         const int tw = threadIdx.x - kWarpRot0 * 32;
         const bool rot = p.rotate != 0;
@@ -492,7 +633,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&bar.ready_q);
         }
         for (int j = 0; ok && j < T.n; ++j) {
-            const int s = j % NS, use = j / NS, jt = T.tile(j);
+            const int jt = T.tile(j);
+            const int s = j % NSK, use = j / NSK, sv = j % NSV, usev = j / NSV;
             uint8_t *tk = sK + s * C::kParts * C::kTileK;
             if (!kF32) {
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_k[s], use & 1, abort, tmo));
@@ -513,227 +655,138 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             mbar_arrive(&bar.ready_k[s]);
             if (kF32) {
-                if (use > 0)
+                if (usev > 0)
                     ok = __all_sync(0xffffffffu,
-                                    mbar_wait(&bar.empty_v[s], (use - 1) & 1, abort, tmo));
+                                    mbar_wait(&bar.empty_v[sv], (usev - 1) & 1, abort, tmo));
                 if (!ok) break;
                 const float *base = reinterpret_cast<const float *>(p.v) + U.b * p.vs[0] +
                                     (long long)U.g * p.vs[1];
-                load_v_f32<D, BN>(sV + s * C::kTileK, base, p.vs[2], jt * BN, p.L, tw);
+                load_v_f32<D, BN>(sV + sv * C::kTileK, base, p.vs[2], jt * BN, p.L, tw);
                 fence_proxy_async_smem();
-                mbar_arrive(&bar.full_v[s]);
+                mbar_arrive(&bar.full_v[sv]);
             }
         }
-    } else if (warp == kWarpMma) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t kIdS = idesc_bf16_f32(128, BN, 0, 0);
-            constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, 0, 1);
-            const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-            // S_t = Q_t K^T over D in steps of 16 (32 bytes inside a 128-byte
-            // swizzle row, then the next 64-column box).  Split mode:
-            // S = Qhi Klo + Qlo Khi + Qhi Khi, all accumulated in fp32.
-            auto issue_s = [&](int t, int s) {
-                const uint32_t qa = q_addr + t * C::kParts * C::kTileQ;
-                const uint32_t ka = k_addr + s * C::kParts * C::kTileK;
-                constexpr int NPROD = kSplit ? 3 : 1;
-#pragma unroll
-                for (int pr = 0; pr < NPROD; ++pr) {
-                    const uint32_t qp = qa + ((kSplit && pr == 1) ? C::kTileQ : 0);
-                    const uint32_t kp = ka + ((kSplit && pr == 0) ? C::kTileK : 0);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t oq = (kk >> 2) * C::kBoxQ + (kk & 3) * 32;
-                        const uint32_t ok_ = (kk >> 2) * C::kBoxK + (kk & 3) * 32;
-                        mma_ss(tmem + t * BN, sdesc_sw128(qp + oq, 16, 1024),
-                               sdesc_sw128(kp + ok_, 16, 1024), kIdS, (pr > 0 || kk > 0));
-                    }
-                }
-            };
-            // O_t += P_t V: P from TMEM (BN/2 columns of bf16 pairs), V MN-major.
-            auto issue_pv = [&](int t, int s, bool acc) {
-                const uint32_t va = v_addr + s * C::kTileK;
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)
-                    mma_ts(tmem + C::kColO + t * D, tmem + t * BN + kk * 8,
-                           sdesc_sw128(va + kk * 2048, C::kBoxK, 1024), kIdPV, (acc || kk > 0));
-            };
-            bool ok = mbar_wait(&bar.ready_q, 0, abort, tmo);
-            if (ok) ok = mbar_wait(&bar.ready_k[0], 0, abort, tmo);
-            tc_fence_after();
-            if (ok) {
-                for (int t = 0; t < U.nt; ++t) {
-                    issue_s(t, 0);
-                    mma_commit(&bar.s_ready[t]);
-                }
-                mma_commit(&bar.empty_k[0]);
-            }
-            for (int j = 0; ok && j < T.n; ++j) {
-                const int sv = j % NS;
-                ok = mbar_wait(&bar.full_v[sv], (j / NS) & 1, abort, tmo);
-                for (int t = 0; ok && t < U.nt; ++t) {
-                    ok = mbar_wait(&bar.p_ready[t], j & 1, abort, tmo);
-                    tc_fence_after();
-                    if (!ok) break;
-                    issue_pv(t, sv, j > 0);
-                    if (j + 1 < T.n) {
-                        const int sk = (j + 1) % NS;
-                        if (t == 0) {
-                            ok = mbar_wait(&bar.ready_k[sk], ((j + 1) / NS) & 1, abort, tmo);
-                            tc_fence_after();
-                            if (!ok) break;
-                        }
-                        issue_s(t, sk);
-                        mma_commit(&bar.s_ready[t]);
-                    }
-                }
-                if (ok) {
-                    mma_commit(&bar.empty_v[sv]);
-                    if (j + 1 < T.n) mma_commit(&bar.empty_k[(j + 1) % NS]);
-                }
-            }
-            if (ok)
-                for (int t = 0; t < U.nt; ++t) mma_commit(&bar.o_ready[t]);
-            // Drain: all issued MMAs complete before TMEM is released.
-            mma_commit(&bar.drain);
-            mbar_wait(&bar.drain, 0, nullptr, tmo);
-        }
-    } else if (warp < 8 && (warp >> 2) < U.nt) {
-        // ------------------------------------------------ softmax, tile t
-        const int t = warp >> 2;
-        const int wq = warp & 3;
-        const int row = wq * 32 + lane;
-        const uint32_t trow = tmem + (uint32_t(wq * 32) << 16);
-        const uint32_t s_col = t * BN, o_col = C::kColO + t * D;
-        const int i = U.q0 + row;
-        const float cl2 = p.c_log2;
-        float m = -INFINITY, l = 0.f;
-        bool ok = true;
-        for (int j = 0; j < T.n; ++j) {
-            ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_ready[t], j & 1, abort, tmo));
-            if (!ok) break;
-            tc_fence_after();
-            const int jt = T.tile(j), k0 = jt * BN;
-            const bool partial = !tile_full<BN>(U.q0, jt, p);
-            // visible columns: col <= hi and (no window or col >= lo or col < sk)
-            const int hi = p.causal ? min(i - k0, p.L - 1 - k0) : p.L - 1 - k0;
-            const int lo = i - p.window + 1 - k0;
-            const int sk = p.sinks - k0;
-            const bool win = p.causal && p.window > 0;
-            auto vis = [&](int col) { return col <= hi && (!win || col >= lo || col < sk); };
+    } else {
+        setmaxnreg_inc<kRegsSoftmax>();
+        if ((warp >> 2) < U.nt) {
+            // ------------------------------------------------ softmax, tile t
+            const int t = warp >> 2;
+            const int wq = warp & 3;
+            const int row = wq * 32 + lane;
+            const uint32_t trow = tmem + (uint32_t(wq * 32) << 16);
+            const uint32_t s_col = t * BN, o_col = C::kColO + t * D;
+            const int i = U.q0 + row;
+            const float cl2 = p.c_log2;
+            float m = -INFINITY, l = 0.f;
+            bool ok = true;
+            for (int j = 0; j < T.n; ++j) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_ready[t], j & 1, abort, tmo));
+                if (!ok) break;
+                tc_fence_after();
+                const int jt = T.tile(j), k0 = jt * BN;
+                const bool partial = !tile_full<BN>(U.q0, jt, p);
+                // visible columns: col <= hi and (no window or col >= lo or col < sk)
+                const int hi = p.causal ? min(i - k0, p.L - 1 - k0) : p.L - 1 - k0;
+                const int lo = i - p.window + 1 - k0;
+                const int sk = p.sinks - k0;
+                const bool win = p.causal && p.window > 0;
+                auto vis = [&](int col) { return col <= hi && (!win || col >= lo || col < sk); };
 
-            // pass 1: row max, 64 columns per TMEM load
-            float mx = -INFINITY;
-#pragma unroll 1
-            for (int c = 0; c < BN / 64; ++c) {
-                float v[64];
-                tmem_ld64(trow + s_col + c * 64, v);
+                // The whole S row of this thread in one TMEM load.
+                float v[BN];
+                tmem_ld_row(trow + s_col, v);
                 if (partial) {
-#pragma unroll
-                    for (int e = 0; e < 64; ++e)
-                        if (!vis(c * 64 + e)) v[e] = -INFINITY;
+    #pragma unroll
+                    for (int e = 0; e < BN; ++e)
+                        if (!vis(e)) v[e] = -INFINITY;
                 }
-                float m0 = v[0], m1 = v[1], m2 = v[2], m3 = v[3];
-#pragma unroll
-                for (int e = 4; e < 64; e += 4) {
-                    m0 = fmaxf(m0, v[e]);
-                    m1 = fmaxf(m1, v[e + 1]);
-                    m2 = fmaxf(m2, v[e + 2]);
-                    m3 = fmaxf(m3, v[e + 3]);
+                const float mx = row_max(v);
+                const float m_new = fmaxf(m, mx * cl2);
+                // Keep the old reference unless the max grew by more than 2^8: the
+                // result is exact either way, only O's rescale is saved.
+                const bool need = (m != -INFINITY) && (m_new > m + kRescaleLog2);
+                if (__any_sync(0xffffffffu, need)) {
+                    const float alpha = need ? ex2_approx(m - m_new) : 1.f;
+    #pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        float o[32];
+                        tmem_ld32(trow + o_col + c * 32, o);
+                        uint32_t u[32];
+    #pragma unroll
+                        for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(o[e] * alpha);
+                        tmem_st32(trow + o_col + c * 32, u);
+                    }
+                    if (need) {
+                        l *= alpha;
+                        m = m_new;
+                    }
                 }
-                mx = fmaxf(mx, fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)));
-            }
-            const float m_new = fmaxf(m, mx * cl2);
-            // Keep the old reference unless the max grew by more than 2^8: the
-            // result is exact either way, only O's rescale is saved.
-            const bool need = (m != -INFINITY) && (m_new > m + kRescaleLog2);
-            if (__any_sync(0xffffffffu, need)) {
-                const float alpha = need ? ex2_approx(m - m_new) : 1.f;
-#pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    float v[32];
-                    tmem_ld32(trow + o_col + c * 32, v);
-                    uint32_t u[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(v[e] * alpha);
-                    tmem_st32(trow + o_col + c * 32, u);
-                }
-                if (need) {
-                    l *= alpha;
-                    m = m_new;
-                }
-            }
-            if (m == -INFINITY) m = m_new;
-            const float mref = (m == -INFINITY) ? 0.f : m;
-            // pass 2: P = 2^(s c - m) as bf16 written over the first half of S
-            float lsum0 = 0.f, lsum1 = 0.f;
-#pragma unroll 1
-            for (int h = 0; h < BN / 64; ++h) {
-                float a[64];
-                tmem_ld64(trow + s_col + h * 64, a);
-                if (partial) {
-#pragma unroll
-                    for (int e = 0; e < 64; ++e)
-                        if (!vis(h * 64 + e)) a[e] = -INFINITY;
-                }
-                uint32_t pk[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float p0 = ex2_approx(fmaf(a[2 * e], cl2, -mref));
-                    const float p1 = ex2_approx(fmaf(a[2 * e + 1], cl2, -mref));
-                    pk[e] = pack_bf16x2(p0, p1);
+                if (m == -INFINITY) m = m_new;
+                const float mref = (m == -INFINITY) ? 0.f : m;
+                // P = 2^(s c - m) as bf16 pairs, written over the first half of S.
+                // One column pair in kEmuEvery takes 2^x on the FMA pipe.
+                const float2 c2 = make_float2(cl2, cl2), nm2 = make_float2(-mref, -mref);
+                float2 lsum = make_float2(0.f, 0.f);
+                uint32_t pk[BN / 2];
+    #pragma unroll
+                for (int e = 0; e < BN / 2; ++e) {
+                    const float2 x = fma2(make_float2(v[2 * e], v[2 * e + 1]), c2, nm2);
+                    float2 pe;
+                    if (kEmuEvery > 0 && (e % kEmuEvery) == kEmuEvery - 1)
+                        pe = exp2_fma2(x);
+                    else
+                        pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                    pk[e] = pack_bf16x2(pe.x, pe.y);
                     if (kSplit) {
                         // Normalise by the weights the tensor core actually
                         // multiplies V with (bf16), not their fp32 values: with
                         // the stale max reference the dominant weight is 2^d,
                         // d in [0, 8], and its rounding must cancel in o.
-                        lsum0 += bf16lo_to_f32(pk[e]);
-                        lsum1 += bf16hi_to_f32(pk[e]);
+                        lsum = add2(lsum, make_float2(bf16lo_to_f32(pk[e]), bf16hi_to_f32(pk[e])));
                     } else {
-                        lsum0 += p0;
-                        lsum1 += p1;
+                        lsum = add2(lsum, pe);
                     }
                 }
-                tmem_st32(trow + s_col + h * 32, pk);
+                tmem_st_row(trow + s_col, pk);
+                l += lsum.x + lsum.y;
+                tc_fence_before();
+                mbar_arrive(&bar.p_ready[t]);
             }
-            l += lsum0 + lsum1;
-            tc_fence_before();
-            mbar_arrive(&bar.p_ready[t]);
-        }
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.o_ready[t], 0, abort, tmo));
-        if (ok) {
-            tc_fence_after();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            const int h = U.hq0 + t;
-            const bool valid = i < p.L;
-            const long long ob = U.b * p.os[0] + (long long)h * p.os[1] + (long long)i * p.os[2];
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                float v[32];
-                tmem_ld32(trow + o_col + c * 32, v);
-                if (!valid) continue;
-                if (kF32) {
-                    float4 *dst = reinterpret_cast<float4 *>(
-                        reinterpret_cast<float *>(p.o) + ob + c * 32);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        dst[e] = make_float4(v[4 * e] * inv, v[4 * e + 1] * inv,
-                                             v[4 * e + 2] * inv, v[4 * e + 3] * inv);
-                } else {
-                    uint4 *dst = reinterpret_cast<uint4 *>(
-                        reinterpret_cast<__nv_bfloat16 *>(p.o) + ob + c * 32);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dst[e] = make_uint4(pack_bf16x2(v[8 * e] * inv, v[8 * e + 1] * inv),
-                                            pack_bf16x2(v[8 * e + 2] * inv, v[8 * e + 3] * inv),
-                                            pack_bf16x2(v[8 * e + 4] * inv, v[8 * e + 5] * inv),
-                                            pack_bf16x2(v[8 * e + 6] * inv, v[8 * e + 7] * inv));
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.o_ready[t], 0, abort, tmo));
+            if (ok) {
+                tc_fence_after();
+                const float inv = l > 0.f ? 1.f / l : 0.f;
+                const int h = U.hq0 + t;
+                const bool valid = i < p.L;
+                const long long ob = U.b * p.os[0] + (long long)h * p.os[1] + (long long)i * p.os[2];
+    #pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    float v[32];
+                    tmem_ld32(trow + o_col + c * 32, v);
+                    if (!valid) continue;
+                    if (kF32) {
+                        float4 *dst = reinterpret_cast<float4 *>(
+                            reinterpret_cast<float *>(p.o) + ob + c * 32);
+    #pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            dst[e] = make_float4(v[4 * e] * inv, v[4 * e + 1] * inv,
+                                                 v[4 * e + 2] * inv, v[4 * e + 3] * inv);
+                    } else {
+                        uint4 *dst = reinterpret_cast<uint4 *>(
+                            reinterpret_cast<__nv_bfloat16 *>(p.o) + ob + c * 32);
+    #pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            dst[e] = make_uint4(pack_bf16x2(v[8 * e] * inv, v[8 * e + 1] * inv),
+                                                pack_bf16x2(v[8 * e + 2] * inv, v[8 * e + 3] * inv),
+                                                pack_bf16x2(v[8 * e + 4] * inv, v[8 * e + 5] * inv),
+                                                pack_bf16x2(v[8 * e + 6] * inv, v[8 * e + 7] * inv));
+                    }
                 }
-            }
-            if (valid && p.lse) {
-                const float ln2 = 0.69314718055994531f;
-                p.lse[(U.b * (long long)p.Hq + h) * p.L + i] =
-                    l > 0.f ? (m + __log2f(l)) * ln2 : -INFINITY;
+                if (valid && p.lse) {
+                    const float ln2 = 0.69314718055994531f;
+                    p.lse[(U.b * (long long)p.Hq + h) * p.L + i] =
+                        l > 0.f ? (m + __log2f(l)) * ln2 : -INFINITY;
+                }
             }
         }
     }
@@ -788,6 +841,17 @@ lcx_status launch(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMa
                   const AttnParams &p, unsigned grid, cudaStream_t s) {
     auto kern = attn_fwd_kernel<D, kF32, kHalf, kSplit>;
     const int smem = Cfg<D, kSplit>::kSmemBytes;
+    // The warpgroups re-balance registers with setmaxnreg, which waits until the
+    // registers it asks for are free: the launch must hold the whole split.
+    static const int regs = []() {
+        cudaFuncAttributes fa;
+        return cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kF32, kHalf, kSplit>) == cudaSuccess
+                   ? fa.numRegs
+                   : -1;
+    }();
+    if (regs * kThreads < (2 * kRegsSoftmax + kRegsRotate + kRegsIssue) * 128)
+        return fail(LCX_ERR_CUDA, "attn_fwd kernel built with %d registers per thread; the "
+                    "warpgroup register split needs 128", regs);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
         return fail(LCX_ERR_CUDA, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
