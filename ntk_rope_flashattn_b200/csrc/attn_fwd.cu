@@ -538,30 +538,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // S_t = Q_t K^T over D in steps of 16 (32 bytes inside a 128-byte
                 // swizzle row, then the next 64-column box).  Split mode:
                 // S = Qhi Klo + Qlo Khi + Qhi Khi, all accumulated in fp32.
+                // Descriptors of the first K step; later steps only move the start
+                // address (in 16-byte units, well inside the 14-bit field).
+                const uint64_t dq0 = sdesc_sw128(q_addr, 16, 1024);
+                const uint64_t dk0 = sdesc_sw128(k_addr, 16, 1024);
+                const uint64_t dv0 = sdesc_sw128(v_addr, C::kBoxK, 1024);
                 auto issue_s = [&](int t, int s) {
-                    const uint32_t qa = q_addr + t * C::kParts * C::kTileQ;
-                    const uint32_t ka = k_addr + s * C::kParts * C::kTileK;
+                    const uint64_t qa = dq0 + ((t * C::kParts * C::kTileQ) >> 4);
+                    const uint64_t ka = dk0 + ((s * C::kParts * C::kTileK) >> 4);
+                    const uint32_t dst = tmem + t * BN;
                     constexpr int NPROD = kSplit ? 3 : 1;
-    #pragma unroll
+#pragma unroll
                     for (int pr = 0; pr < NPROD; ++pr) {
-                        const uint32_t qp = qa + ((kSplit && pr == 1) ? C::kTileQ : 0);
-                        const uint32_t kp = ka + ((kSplit && pr == 0) ? C::kTileK : 0);
-    #pragma unroll
+                        const uint64_t qp = qa + (((kSplit && pr == 1) ? C::kTileQ : 0) >> 4);
+                        const uint64_t kp = ka + (((kSplit && pr == 0) ? C::kTileK : 0) >> 4);
+#pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t oq = (kk >> 2) * C::kBoxQ + (kk & 3) * 32;
-                            const uint32_t ok_ = (kk >> 2) * C::kBoxK + (kk & 3) * 32;
-                            mma_ss(tmem + t * BN, sdesc_sw128(qp + oq, 16, 1024),
-                                   sdesc_sw128(kp + ok_, 16, 1024), kIdS, (pr > 0 || kk > 0));
+                            const uint32_t oq = ((kk >> 2) * C::kBoxQ + (kk & 3) * 32) >> 4;
+                            const uint32_t ok_ = ((kk >> 2) * C::kBoxK + (kk & 3) * 32) >> 4;
+                            mma_ss(dst, qp + oq, kp + ok_, kIdS, (pr > 0 || kk > 0));
                         }
                     }
                 };
                 // O_t += P_t V: P from TMEM (BN/2 columns of bf16 pairs), V MN-major.
                 auto issue_pv = [&](int t, int s, bool acc) {
-                    const uint32_t va = v_addr + s * C::kTileK;
-    #pragma unroll
+                    const uint64_t va = dv0 + ((s * C::kTileK) >> 4);
+                    const uint32_t dst = tmem + C::kColO + t * D, pa = tmem + t * BN;
+#pragma unroll
                     for (int kk = 0; kk < BN / 16; ++kk)
-                        mma_ts(tmem + C::kColO + t * D, tmem + t * BN + kk * 8,
-                               sdesc_sw128(va + kk * 2048, C::kBoxK, 1024), kIdPV, (acc || kk > 0));
+                        mma_ts(dst, pa + kk * 8, va + ((kk * 2048) >> 4), kIdPV, (acc || kk > 0));
                 };
                 bool ok = mbar_wait(&bar.ready_q, 0, abort, tmo);
                 if (ok) ok = mbar_wait(&bar.ready_k[0], 0, abort, tmo);
@@ -732,7 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = 0; e < BN / 2; ++e) {
                     const float2 x = fma2(make_float2(v[2 * e], v[2 * e + 1]), c2, nm2);
                     float2 pe;
-                    if (kEmuEvery > 0 && (e % kEmuEvery) == kEmuEvery - 1)
+                    if (kEmuEvery > 0 && (e % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1)
                         pe = exp2_fma2(x);
                     else
                         pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));

@@ -55,6 +55,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep in the instruction for up to
+// hint_ns (it wakes as soon as the phase completes), so a waiting warp does
+// not take issue slots from the warps that share its scheduler.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity to complete.  Gives up when
 // another thread of the CTA has already raised *abort (returns false at once),
 // or after timeout_ns of wall time (raises *abort, returns false).  With
@@ -65,9 +81,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
-#pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+        // sleep in the wait for up to 0.5 ms at a time; the phase completing
+        // wakes the thread at once
+        if (mbar_try_wait_sleep(bar, parity, 500000u)) return true;
         if (abort && *abort) return false;
         if (globaltimer_ns() - t0 > timeout_ns) {
             if (abort) *abort = 1;
