@@ -58,6 +58,13 @@ constexpr float kRescaleLog2 = 8.0f;    // rescale O only if the max grows by > 
 #ifndef LCX_KSTAGES_D128
 #define LCX_KSTAGES_D128 2
 #endif
+#ifndef LCX_ROT_UNROLL
+#define LCX_ROT_UNROLL 2
+#endif
+#ifndef LCX_PHASOR_CARRY
+#define LCX_PHASOR_CARRY 1
+#endif
+constexpr int kRotUnroll = LCX_ROT_UNROLL;  // rows in flight per rotation thread
 // 1 column pair in kEmuEvery takes 2^x on the FMA pipe (0 = all on the MUFU:
 // measured fastest here, since the MUFU is not the binding limit).
 constexpr int kEmuEvery = LCX_EMU_EVERY;
@@ -284,18 +291,43 @@ struct Phasor {
     }
 };
 
+// The phasor a rotation thread ends a K tile with already points at the first
+// row of the next tile; consecutive tiles reuse it, and every kReseed tiles
+// (or after a jump, e.g. from the sink tiles to the window) it is evaluated
+// afresh from the exact angle, which bounds the drift of the recurrence.
+template <int PPJ>
+struct PhasorCarry {
+    float c[PPJ], s[PPJ];
+    long long next = -1;
+    int age = 0;
+};
+constexpr int kReseed = 16;
+
 // Rotate a ROWS x D bf16 tile in place (row r at position pos0 + r); in the
 // split mode also write the residual part into `lo`.
 template <int D, bool kHalf, bool kSplit, int ROWS>
 __device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, uint8_t *lo, long long pos0,
                                                  const Phasor<D, kHalf> &ph, const AttnParams &p,
-                                                 bool rotate) {
+                                                 bool rotate,
+                                                 PhasorCarry<Rot<D, kHalf>::PPJ> *carry = nullptr) {
     using R = Rot<D, kHalf>;
     constexpr int NJ = ROWS / R::RP;
     constexpr int BOX = ROWS * 128;
     float c[R::PPJ], s[R::PPJ];
-    if (rotate) ph.start(pos0, p, c, s);
-#pragma unroll 2
+    if (rotate) {
+        if (LCX_PHASOR_CARRY && carry && carry->next == pos0 && carry->age < kReseed) {
+#pragma unroll
+            for (int e = 0; e < R::PPJ; ++e) {
+                c[e] = carry->c[e];
+                s[e] = carry->s[e];
+            }
+            ++carry->age;
+        } else {
+            ph.start(pos0, p, c, s);
+            if (carry) carry->age = 0;
+        }
+    }
+#pragma unroll kRotUnroll
     for (int k = 0; k < NJ; ++k) {
         const int r = ph.r0 + k * R::RP;
         if (kHalf) {
@@ -327,6 +359,14 @@ __device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, uint8_t *lo, lon
             store8<kSplit>(tile, lo, oa, x);
         }
         if (rotate) ph.step(c, s);
+    }
+    if (LCX_PHASOR_CARRY && carry && rotate) {
+#pragma unroll
+        for (int e = 0; e < R::PPJ; ++e) {
+            carry->c[e] = c[e];
+            carry->s[e] = s[e];
+        }
+        carry->next = pos0 + ROWS;
     }
 }
 
@@ -616,6 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool rot = p.rotate != 0;
         Phasor<D, kHalf> ph;
         ph.init(tw, p);
+        PhasorCarry<Rot<D, kHalf>::PPJ> kcarry;
         bool ok = true;
         if (!kF32) {
             ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_q, 0, abort, tmo));
@@ -646,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 if (rot || kSplit)
                     rotate_tile_bf16<D, kHalf, kSplit, BN>(tk, tk + C::kTileK, (long long)jt * BN,
-                                                           ph, p, rot);
+                                                           ph, p, rot, &kcarry);
             } else {
                 if (use > 0)
                     ok = __all_sync(0xffffffffu,
