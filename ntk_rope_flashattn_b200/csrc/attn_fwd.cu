@@ -659,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         PhasorCarry<Rot<D, kHalf>::PPJ> kcarry;
         bool ok = true;
         if (!kF32) {
-            ok = mbar_wait_warp(&bar.full_q, 0, abort, tmo);
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_q, 0, abort, tmo));
             if (ok && (rot || kSplit))
                 for (int t = 0; t < U.nt; ++t) {
                     uint8_t *qt = sQ + t * C::kParts * C::kTileQ;
@@ -683,14 +683,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int s = j % NSK, use = j / NSK, sv = j % NSV, usev = j / NSV;
             uint8_t *tk = sK + s * C::kParts * C::kTileK;
             if (!kF32) {
-                ok = mbar_wait_warp(&bar.full_k[s], use & 1, abort, tmo);
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_k[s], use & 1, abort, tmo));
                 if (!ok) break;
                 if (rot || kSplit)
                     rotate_tile_bf16<D, kHalf, kSplit, BN>(tk, tk + C::kTileK, (long long)jt * BN,
                                                            ph, p, rot, &kcarry);
             } else {
                 if (use > 0)
-                    ok = mbar_wait_warp(&bar.empty_k[s], (use - 1) & 1, abort, tmo);
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(&bar.empty_k[s], (use - 1) & 1, abort, tmo));
                 if (!ok) break;
                 const float *base = reinterpret_cast<const float *>(p.k) + U.b * p.ks[0] +
                                     (long long)U.g * p.ks[1];
@@ -701,7 +702,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&bar.ready_k[s]);
             if (kF32) {
                 if (usev > 0)
-                    ok = mbar_wait_warp(&bar.empty_v[sv], (usev - 1) & 1, abort, tmo);
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(&bar.empty_v[sv], (usev - 1) & 1, abort, tmo));
                 if (!ok) break;
                 const float *base = reinterpret_cast<const float *>(p.v) + U.b * p.vs[0] +
                                     (long long)U.g * p.vs[1];
@@ -724,7 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float m = -INFINITY, l = 0.f;
             bool ok = true;
             for (int j = 0; j < T.n; ++j) {
-                ok = mbar_wait_warp(&bar.s_ready[t], j & 1, abort, tmo);
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_ready[t], j & 1, abort, tmo));
                 if (!ok) break;
                 tc_fence_after();
                 const int jt = T.tile(j), k0 = jt * BN;
@@ -796,7 +798,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 mbar_arrive(&bar.p_ready[t]);
             }
-            if (ok) ok = mbar_wait_warp(&bar.o_ready[t], 0, abort, tmo);
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.o_ready[t], 0, abort, tmo));
             if (ok) {
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.f / l : 0.f;

@@ -92,18 +92,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
-// Warp-wide bounded wait: lane 0 alone polls the barrier (32 lanes polling one
-// word would serialise in the shared-memory pipe), then the warp synchronises,
-// which orders lane 0's acquire before every lane's subsequent accesses, and
-// the outcome is broadcast.  All 32 lanes must call it.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                               uint64_t timeout_ns) {
-    int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, timeout_ns) ? 1 : 0;
-    __syncwarp();
-    return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-
 // Make generic-proxy shared-memory writes visible to the async proxy (tensor
 // core / TMA) before signalling a barrier.
 __device__ __forceinline__ void fence_proxy_async_smem() {
