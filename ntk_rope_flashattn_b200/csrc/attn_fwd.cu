@@ -129,27 +129,22 @@ struct Unit {
     int b, g, hq0, nt, q0;
 };
 
-// Work units are numbered heaviest first (query blocks from the end of the
-// sequence, which see the most keys), so the block scheduler hands out the
-// longest units first.
+// Work units are grouped by (batch, kv head) and, inside a group, numbered
+// heaviest first (query blocks from the end of the sequence, which see the
+// most keys).  The block scheduler therefore runs many query blocks of the same
+// kv head side by side -- they stream the same K/V tiles, which L2 then serves
+// -- and still hands out the longest units of every group first.
 __device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
     const int u = blockIdx.x;
-    const int hu = u % p.units_per_qb;
-    const int qb = p.n_qb - 1 - u / p.units_per_qb;
+    const int upq = p.G / p.heads_per_unit;          // units per query block of a group
+    const int per_group = p.n_qb * upq;
+    const int grp = u / per_group, rem = u % per_group;
     Unit r;
-    r.q0 = qb * kBM;
+    r.b = grp / p.Hkv;
+    r.g = grp % p.Hkv;
+    r.q0 = (p.n_qb - 1 - rem / upq) * kBM;
     r.nt = p.heads_per_unit;
-    const int per_b = p.units_per_qb / p.B;
-    r.b = hu / per_b;
-    const int rem = hu % per_b;
-    if (p.heads_per_unit == 2) {
-        const int ppg = p.G / 2;
-        r.g = rem / ppg;
-        r.hq0 = r.g * p.G + 2 * (rem % ppg);
-    } else {
-        r.hq0 = rem;
-        r.g = rem / p.G;
-    }
+    r.hq0 = r.g * p.G + p.heads_per_unit * (rem % upq);
     return r;
 }
 
