@@ -40,9 +40,11 @@ from workloads import HEADLINE, WORKLOADS, attn_flops, make_inputs, rope_bytes, 
 METRIC = "fused YaRN-RoPE causal attention prefill TFLOP/s and % dense BF16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM traffic (read + write bytes) of one attention launch on the headline
-# workload from an ncu capture of the current kernel; None until captured.
-ATTN_TRAFFIC_BYTES = None
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
+# launch on the headline workload (yarn_L131072_s16), from a one-pass ncu capture
+# of the current kernel: 3.03 GB read + 1.08 GB written (algorithmic: q, k, v
+# read once = 1.61 GB, o written once = 1.07 GB).  Only valid for that workload.
+ATTN_TRAFFIC_BYTES = {"yarn_L131072_s16": 4.11e9}
 
 
 def load_peaks():
@@ -135,12 +137,24 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The largest of the ranks' values (device times are reported as the max)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(w, rank):
+    """Each rank runs an independent replica of the workload with its own seed."""
+    return w.seed + rank
+
+
+def job_tflops(flops_per_rank, world, steps, max_ms):
+    """Whole-job throughput: the work of all ranks over the slowest rank's time."""
+    return flops_per_rank * world * steps / (max_ms * 1e-3) / 1e12
 
 
 # ------------------------------------------------------------------ oracle
@@ -192,7 +206,7 @@ def bench_gpu(args, world, rank, local):
     import ntk_rope_flashattn_b200 as lcx
     w = WORKLOADS[args.workload]
     dev = torch.device("cuda", local)
-    q, k, v = make_inputs(w, device=dev, seed=w.seed + rank)
+    q, k, v = make_inputs(w, device=dev, seed=rank_seed(w, rank))
     rope = lcx.RopeParams(w.mode, w.D, w.base, w.scale, w.original_max_pos, w.alpha, w.beta,
                           w.pairing)
     o = torch.empty_like(q)
@@ -229,7 +243,7 @@ def bench_gpu(args, world, rank, local):
     assert int(status.item()) == 0, "device watchdog fired"
     total_ms = max_over_ranks(total_ms, world)
     flops_rank = attn_flops(w)
-    tflops = flops_rank * world * args.steps / (total_ms * 1e-3) / 1e12
+    tflops = job_tflops(flops_rank, world, args.steps, total_ms)
 
     # --- apply_rope (the unfused rotate-pairs pass) on Q and K, for its own roofline
     qr, kr = torch.empty_like(q), torch.empty_like(k)
@@ -267,7 +281,7 @@ def bench_gpu(args, world, rank, local):
     e_end.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), world)
-    e2e_tflops = flops_rank * world * args.steps / (e2e_ms * 1e-3) / 1e12
+    e2e_tflops = job_tflops(flops_rank, world, args.steps, e2e_ms)
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
     d2h = oh.numel() * oh.element_size()
     del qh, kh, vh, ws
@@ -308,7 +322,9 @@ def bench_gpu(args, world, rank, local):
             "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
             "peak_kind": "bf16_tflops_sustained of %s" % peak_src,
             "frac_of_burst": round(achieved / float(peaks["bf16_tflops"]), 4),
-            "traffic": ATTN_TRAFFIC_BYTES,
+            "traffic": ATTN_TRAFFIC_BYTES.get(w.name),
+            "algorithmic_bytes": (sum(t.numel() * t.element_size() for t in (q, k, v))
+                                  + o.numel() * o.element_size()),
             "kernel": "attn_fwd_kernel", "avg_launch_ms": round(avg_launch, 3),
             "launch_ms": [round(x, 3) for x in launch_ms],
         },
