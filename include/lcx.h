@@ -60,15 +60,21 @@ typedef enum {
     LCX_ERR_TIMEOUT = 4
 } lcx_status;
 
-/* Frequency-scaling modes ([LC] 2.3, 4.2, 5.2, 6.2; [B83] 8.3.2-8.3.3).
+/* Frequency-scaling modes ([LC] 2.3, 4.2, 5.2, 6.2, 7.3; [B83] 8.3.2-8.3.3).
  * NONE leaves vectors unrotated (theta' = 0) and is meant for testing. */
 typedef enum {
     LCX_ROPE_NONE = 0,
     LCX_ROPE_PLAIN = 1,   /* theta'_i = b^(-2i/D)                              */
     LCX_ROPE_PI = 2,      /* theta'_i = theta_i / s  (positions m -> m/s)      */
     LCX_ROPE_NTK = 3,     /* theta'_i = (b s^(D/(D-2)))^(-2i/D)                */
-    LCX_ROPE_YARN = 4     /* theta'_i = theta_i ((1-g_i)/s + g_i), g_i = clip((r_i-alpha)/(beta-alpha),0,1),
+    LCX_ROPE_YARN = 4,    /* theta'_i = theta_i ((1-g_i)/s + g_i), g_i = clip((r_i-alpha)/(beta-alpha),0,1),
                              r_i = L_train theta_i / (2 pi); mscale = 0.1 ln s + 1 (s > 1) */
+    LCX_ROPE_DYNAMIC_NTK = 5, /* NTK-aware base with s = seq_len / L_train when
+                             seq_len > L_train, plain RoPE otherwise ("AI Day 9:
+                             长上下文技术", RoPE extension list, Dynamic NTK)     */
+    LCX_ROPE_FACTORS = 6  /* theta'_i = theta_i / lambda_i with caller-supplied
+                             per-pair factors ([LC] 7.3 LongRoPE); the optional
+                             short table applies while seq_len <= L_train ([LC] 7.4) */
 } lcx_rope_mode;
 
 /* Which dimensions form a rotated pair ([LC] 2.4): HALF pairs (i, i + D/2)
@@ -87,6 +93,13 @@ typedef struct {
     int64_t original_max_pos;  /* L_train > 0 (YARN)                             */
     double alpha;              /* YARN ramp lower bound in turns (default 1)     */
     double beta;               /* YARN ramp upper bound in turns (default 32)    */
+    int64_t seq_len;           /* DYNAMIC_NTK, FACTORS: the actual context length.
+                                  lcx_rope_table needs it > 0; lcx_apply_rope and
+                                  lcx_attn_fwd use their own length when it is 0
+                                  (pos_offset + L, resp. L)                       */
+    const double *factors;     /* FACTORS: HOST array of head_dim/2 factors > 0  */
+    const double *factors_short; /* FACTORS: optional HOST table of head_dim/2
+                                  factors used while seq_len <= original_max_pos */
 } lcx_rope_params;
 
 /*

@@ -21,7 +21,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblcx.so")
 
 LCX_OK, LCX_ERR_INVALID_ARG, LCX_ERR_UNSUPPORTED, LCX_ERR_CUDA, LCX_ERR_TIMEOUT = range(5)
-MODES = {"none": 0, "plain": 1, "pi": 2, "ntk": 3, "yarn": 4}
+MODES = {"none": 0, "plain": 1, "pi": 2, "ntk": 3, "yarn": 4, "dynamic_ntk": 5, "factors": 6}
 PAIRINGS = {"half": 0, "interleaved": 1}
 DTYPES = {"bf16": 0, "f32": 1}
 LCX_ATTN_PREROTATED = 1
@@ -48,7 +48,8 @@ class _RopeParams(ctypes.Structure):
                 ("pairing", ctypes.c_int32), ("reserved", ctypes.c_int32),
                 ("base", ctypes.c_double), ("scale", ctypes.c_double),
                 ("original_max_pos", ctypes.c_int64), ("alpha", ctypes.c_double),
-                ("beta", ctypes.c_double)]
+                ("beta", ctypes.c_double), ("seq_len", ctypes.c_int64),
+                ("factors", ctypes.c_void_p), ("factors_short", ctypes.c_void_p)]
 
 
 class _AttnArgs(ctypes.Structure):
@@ -75,6 +76,9 @@ class RopeParams:
     alpha: float = 1.0
     beta: float = 32.0
     pairing: str = "half"
+    seq_len: int = 0              # dynamic_ntk / factors: actual length (0: the call's length)
+    factors: object = None        # factors: per-pair lambda_i (head_dim/2 values)
+    factors_short: object = None  # factors: optional table for seq_len <= original_max_pos
 
     @classmethod
     def from_hf(cls, cfg: dict, head_dim: int):
@@ -90,9 +94,17 @@ class RopeParams:
                    alpha=float(cfg.get("beta_slow", 1.0)), beta=float(cfg.get("beta_fast", 32.0)))
 
     def _c(self):
-        return _RopeParams(MODES[self.mode], int(self.head_dim), PAIRINGS[self.pairing], 0,
-                           float(self.base), float(self.scale), int(self.original_max_pos),
-                           float(self.alpha), float(self.beta))
+        """The C struct; it keeps the factor arrays it points to alive."""
+        fl = None if self.factors is None else np.ascontiguousarray(self.factors, np.float64)
+        fs = (None if self.factors_short is None
+              else np.ascontiguousarray(self.factors_short, np.float64))
+        c = _RopeParams(MODES[self.mode], int(self.head_dim), PAIRINGS[self.pairing], 0,
+                        float(self.base), float(self.scale), int(self.original_max_pos),
+                        float(self.alpha), float(self.beta), int(self.seq_len),
+                        None if fl is None else fl.ctypes.data,
+                        None if fs is None else fs.ctypes.data)
+        c._keep = (fl, fs)
+        return c
 
 
 _lib = None
@@ -216,13 +228,15 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
     a.B, a.Hq, a.Hkv, a.L, a.D = B, Hq, Hkv, L, D
     a.q_strides, a.k_strides, a.v_strides, a.o_strides = (_strides(q), _strides(k),
                                                           _strides(v), _strides(o))
-    a.rope = rope._c()
+    rope_c = rope._c()
+    a.rope = rope_c
     a.window, a.sinks = int(window), int(sinks)
     a.softmax_scale = float(softmax_scale)
     a.flags = ((LCX_ATTN_PREROTATED if prerotated else 0) | (LCX_ATTN_SPLIT_QK if split_qk else 0)
                | (LCX_ATTN_TEST_STALL if _test_stall else 0))
     a.watchdog_ms = int(watchdog_ms)
     _check(load().lcx_attn_fwd(ctypes.byref(a), _stream(q)))
+    del rope_c
     return (o, lse) if return_lse else o
 
 

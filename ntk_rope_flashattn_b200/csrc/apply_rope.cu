@@ -200,7 +200,7 @@ extern "C" lcx_status lcx_apply_rope(const lcx_rope_params *params, const void *
     a.H = int(H);
     a.L = int(L);
     a.pos_offset = pos_offset;
-    rope_table_unchecked(params, a.theta, &a.ms);
+    rope_table_unchecked(params, effective_seq_len(params, pos_offset + L), a.theta, &a.ms);
     const bool half = params->pairing == LCX_PAIR_HALF;
     a.jobs_per_row = half ? (D / 2) / vec : D / vec;
     a.rows_per_cta = 256 / a.jobs_per_row;

@@ -995,7 +995,7 @@ extern "C" lcx_status lcx_attn_fwd(const lcx_attn_args *a, void *stream) {
     if (grid > 0x7fffffffLL) return fail(LCX_ERR_UNSUPPORTED, "too many work units");
     p.rotate = (a->flags & LCX_ATTN_PREROTATED) ? 0 : 1;
     float ms = 1.f;
-    rope_table_unchecked(&a->rope, p.theta, &ms);
+    rope_table_unchecked(&a->rope, effective_seq_len(&a->rope, a->L), p.theta, &ms);
     const double scale = a->softmax_scale > 0.f ? double(a->softmax_scale) : 1.0 / std::sqrt(double(a->D));
     const double msq = p.rotate ? double(ms) * double(ms) : 1.0;
     p.c_log2 = float(scale * msq * 1.4426950408889634);

@@ -18,8 +18,15 @@ void clear_error();
 // Validate RoPE parameters (shared by every entry point).
 lcx_status check_rope_params(const lcx_rope_params *p);
 
-// Fill theta'_i (fp32, head_dim/2 entries) and mscale for validated params.
-void rope_table_unchecked(const lcx_rope_params *p, float *inv_freq, float *mscale);
+// Fill theta'_i (fp32, head_dim/2 entries) and mscale for validated params;
+// seq_len is the actual context length the length-dependent modes use.
+void rope_table_unchecked(const lcx_rope_params *p, int64_t seq_len, float *inv_freq,
+                          float *mscale);
+
+// The context length a call uses for the length-dependent modes.
+inline int64_t effective_seq_len(const lcx_rope_params *p, int64_t call_len) {
+    return p->seq_len > 0 ? p->seq_len : call_len;
+}
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

@@ -14,7 +14,7 @@ import numpy as np
 
 from . import build as _build
 
-MODES = {"none": 0, "plain": 1, "pi": 2, "ntk": 3, "yarn": 4}
+MODES = {"none": 0, "plain": 1, "pi": 2, "ntk": 3, "yarn": 4, "dynamic_ntk": 5, "factors": 6}
 PAIRINGS = {"half": 0, "interleaved": 1}
 
 _lib = None
@@ -35,6 +35,14 @@ def _load():
         lib.orc_rope_table.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                        ctypes.c_double, ctypes.c_int64, ctypes.c_double,
                                        ctypes.c_double, f32p, f32p, f64p, i32p]
+        lib.orc_rope_table_ext.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                           ctypes.c_double, ctypes.c_int64, ctypes.c_double,
+                                           ctypes.c_double, ctypes.c_int64, f64p, f64p, f32p,
+                                           f32p, f64p, i32p]
+        lib.orc_rope_theta_ext.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                           ctypes.c_double, ctypes.c_int64, ctypes.c_double,
+                                           ctypes.c_double, ctypes.c_int64, f64p, f64p, f64p,
+                                           f64p]
         lib.orc_rotate_rows.argtypes = [f32p, f64p, ctypes.c_int64, ctypes.c_int, i64p,
                                         f32p, ctypes.c_float, ctypes.c_int]
         lib.orc_visible.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
@@ -70,22 +78,49 @@ def rope_theta_fp64(mode, D, base=10000.0, scale=1.0, original_max_pos=4096,
     return out, ms.value
 
 
-def rope_table(mode, D, base=10000.0, scale=1.0, original_max_pos=4096, alpha=1.0, beta=32.0):
+def _f64_or_null(a):
+    if a is None:
+        return None, None
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    return a, _ptr(a, ctypes.c_double)
+
+
+def rope_table(mode, D, base=10000.0, scale=1.0, original_max_pos=4096, alpha=1.0, beta=32.0,
+               seq_len=0, factors=None, factors_short=None):
     """fp32 table (theta'_i rounded to nearest even), fp32 mscale, midpoint flags.
 
     flags has D/2 + 1 entries (the last one for mscale); a 1 marks a value whose
     fp32 rounding is too close to a midpoint to be trusted bit for bit.
+    seq_len / factors / factors_short are used by the dynamic_ntk and factors modes.
     """
     lib = _load()
     table = np.zeros(D // 2, dtype=np.float32)
     ms = ctypes.c_float(0.0)
     flags = np.zeros(D // 2 + 1, dtype=np.int32)
-    rc = lib.orc_rope_table(MODES[mode], D, base, scale, original_max_pos, alpha, beta,
-                            _ptr(table, ctypes.c_float), ctypes.byref(ms), None,
-                            _ptr(flags, ctypes.c_int))
+    fa, fp = _f64_or_null(factors)
+    fsa, fsp = _f64_or_null(factors_short)
+    rc = lib.orc_rope_table_ext(MODES[mode], D, base, scale, original_max_pos, alpha, beta,
+                                int(seq_len), fp, fsp, _ptr(table, ctypes.c_float),
+                                ctypes.byref(ms), None, _ptr(flags, ctypes.c_int))
     if rc:
         raise ValueError("orc_rope_table: invalid argument")
     return table, np.float32(ms.value), flags
+
+
+def rope_theta_ext(mode, D, base=10000.0, scale=1.0, original_max_pos=4096, alpha=1.0,
+                   beta=32.0, seq_len=0, factors=None, factors_short=None):
+    """fp64 theta'_i and mscale for every mode, including the length-dependent ones."""
+    lib = _load()
+    out = np.zeros(D // 2, dtype=np.float64)
+    ms = ctypes.c_double(0.0)
+    fa, fp = _f64_or_null(factors)
+    fsa, fsp = _f64_or_null(factors_short)
+    rc = lib.orc_rope_theta_ext(MODES[mode], D, base, scale, original_max_pos, alpha, beta,
+                                int(seq_len), fp, fsp, _ptr(out, ctypes.c_double),
+                                ctypes.byref(ms))
+    if rc:
+        raise ValueError("orc_rope_theta_ext: invalid argument")
+    return out, ms.value
 
 
 def rotate_rows(x, pos, table, mscale, pairing="half"):

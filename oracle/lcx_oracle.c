@@ -37,6 +37,8 @@
 #define ORC_PI 2
 #define ORC_NTK 3
 #define ORC_YARN 4
+#define ORC_DYNAMIC_NTK 5
+#define ORC_FACTORS 6
 
 #define ORC_PAIR_HALF 0
 #define ORC_PAIR_INTERLEAVED 1
@@ -100,6 +102,42 @@ int orc_rope_theta_fp64(int mode, int D, double base, double s, int64_t L_train,
 }
 
 /*
+ * Table variants that depend on the actual context length seq_len:
+ *   DYNAMIC_NTK ("AI Day 9: 长上下文技术", RoPE extension list, item 4 Dynamic
+ *     NTK: the base is adjusted at inference time to the actual sequence
+ *     length; no change for short sequences): s = seq_len / L_train when
+ *     seq_len > L_train, else 1, and the NTK-aware base b' = b s^(D/(D-2)).
+ *   FACTORS ("Long Context: RoPE / YaRN / NTK / MLA", 7.3-7.4, LongRoPE):
+ *     theta'_i = theta_i / lambda_i with per-pair factors lambda_i; with a
+ *     second (short) table, that table is used while seq_len <= L_train.
+ *   Both keep mscale = 1.  Other modes ignore seq_len and the factor tables.
+ */
+int orc_rope_theta_ext(int mode, int D, double base, double s, int64_t L_train, double alpha,
+                       double beta, int64_t seq_len, const double *factors,
+                       const double *factors_short, double *theta_prime, double *mscale)
+{
+    if (mode == ORC_DYNAMIC_NTK) {
+        if (D < 4 || (D % 2) != 0 || !(base > 1.0) || L_train <= 0 || seq_len <= 0) return 1;
+        double se = (seq_len > L_train) ? (double)seq_len / (double)L_train : 1.0;
+        if (se == 1.0) return orc_rope_theta_fp64(ORC_PLAIN, D, base, 1.0, L_train, alpha, beta,
+                                                  theta_prime, mscale);
+        return orc_rope_theta_fp64(ORC_NTK, D, base, se, L_train, alpha, beta, theta_prime,
+                                   mscale);
+    }
+    if (mode == ORC_FACTORS) {
+        if (D <= 0 || (D % 2) != 0 || !(base > 1.0) || !factors) return 1;
+        const double *lam = (factors_short && seq_len <= L_train) ? factors_short : factors;
+        for (int i = 0; i < D / 2; i++) {
+            if (!(lam[i] > 0.0) || !isfinite(lam[i])) return 1;
+            theta_prime[i] = pow(base, -2.0 * (double)i / (double)D) / lam[i];
+        }
+        *mscale = 1.0;
+        return 0;
+    }
+    return orc_rope_theta_fp64(mode, D, base, s, L_train, alpha, beta, theta_prime, mscale);
+}
+
+/*
  * 1 if the fp64 value v lies within a relative 2^-40 of a midpoint between two
  * adjacent fp32 numbers (where its fp32 rounding could depend on the last bits
  * of the fp64 evaluation), else 0.
@@ -121,14 +159,16 @@ static int near_fp32_midpoint(double v)
  * from fp64.  flags[i] (nullable) is set to 1 where that rounding sits too
  * close to an fp32 midpoint to be trusted bit for bit.
  */
-int orc_rope_table(int mode, int D, double base, double s, int64_t L_train,
-                   double alpha, double beta, float *table, float *mscale,
-                   double *theta_fp64, int *flags)
+int orc_rope_table_ext(int mode, int D, double base, double s, int64_t L_train,
+                       double alpha, double beta, int64_t seq_len, const double *factors,
+                       const double *factors_short, float *table, float *mscale,
+                       double *theta_fp64, int *flags)
 {
     if (D <= 0 || D > 4096 || (D % 2) != 0) return 1;
     double tp[2048];
     double ms;
-    int rc = orc_rope_theta_fp64(mode, D, base, s, L_train, alpha, beta, tp, &ms);
+    int rc = orc_rope_theta_ext(mode, D, base, s, L_train, alpha, beta, seq_len, factors,
+                                factors_short, tp, &ms);
     if (rc) return rc;
     for (int i = 0; i < D / 2; i++) {
         table[i] = (float)tp[i];
@@ -138,6 +178,14 @@ int orc_rope_table(int mode, int D, double base, double s, int64_t L_train,
     *mscale = (float)ms;
     if (flags) flags[D / 2] = near_fp32_midpoint(ms);
     return 0;
+}
+
+int orc_rope_table(int mode, int D, double base, double s, int64_t L_train,
+                   double alpha, double beta, float *table, float *mscale,
+                   double *theta_fp64, int *flags)
+{
+    return orc_rope_table_ext(mode, D, base, s, L_train, alpha, beta, 0, NULL, NULL, table,
+                              mscale, theta_fp64, flags);
 }
 
 /*

@@ -62,6 +62,7 @@ int main(void) {
   printf("lcx_rope_params %zu\n", sizeof(lcx_rope_params));
   printf("lcx_attn_args %zu\n", sizeof(lcx_attn_args));
   P(lcx_rope_params, base) P(lcx_rope_params, original_max_pos) P(lcx_rope_params, beta)
+  P(lcx_rope_params, seq_len) P(lcx_rope_params, factors) P(lcx_rope_params, factors_short)
   P(lcx_attn_args, dev_status) P(lcx_attn_args, dtype) P(lcx_attn_args, B) P(lcx_attn_args, D)
   P(lcx_attn_args, q_strides) P(lcx_attn_args, o_strides) P(lcx_attn_args, rope)
   P(lcx_attn_args, window) P(lcx_attn_args, sinks) P(lcx_attn_args, softmax_scale)
@@ -111,11 +112,37 @@ def test_rope_table_bit_exact_with_oracle(lib):
     assert checked > 10000
 
 
+def test_length_dependent_tables_bit_exact_with_oracle(lib):
+    """Dynamic NTK and factor tables (with and without the short table) equal the
+    oracle's bit for bit across lengths below, at and above the training length."""
+    rng = np.random.default_rng(5)
+    for D in (64, 128):
+        lam = rng.uniform(1.0, 16.0, D // 2)
+        lam_s = rng.uniform(1.0, 1.5, D // 2)
+        for seq in (1, 4095, 4096, 4097, 20000, 131072, 1 << 20):
+            for mode, kw in (("dynamic_ntk", {}), ("factors", dict(factors=lam)),
+                             ("factors", dict(factors=lam, factors_short=lam_s))):
+                ref, ref_ms, flags = oracle.rope_table(mode, D, 5e5, 1.0, 4096, 1.0, 32.0,
+                                                       seq_len=seq, **kw)
+                got, ms = lcx.rope_table(lcx.RopeParams(mode, D, base=5e5,
+                                                        original_max_pos=4096, seq_len=seq,
+                                                        **kw))
+                ok = flags[:-1] == 0
+                np.testing.assert_array_equal(got.view(np.uint32)[ok], ref.view(np.uint32)[ok])
+                assert ms == ref_ms == 1.0
+
+
 @pytest.mark.parametrize("bad", [
     dict(head_dim=63), dict(head_dim=0), dict(head_dim=1024), dict(mode="plain", base=1.0),
     dict(mode="pi", scale=0.0), dict(mode="yarn", alpha=32.0, beta=1.0),
     dict(mode="yarn", original_max_pos=0), dict(mode="ntk", head_dim=2),
     dict(mode="yarn", scale=float("nan")),
+    dict(mode="factors", seq_len=10),
+    dict(mode="factors", seq_len=10, factors=[1.0] * 63 + [0.0]),
+    dict(mode="factors", seq_len=10, factors=[1.0] * 64, factors_short=[float("inf")] * 64),
+    dict(mode="dynamic_ntk", seq_len=0),
+    dict(mode="dynamic_ntk", seq_len=10, original_max_pos=0),
+    dict(mode="plain", seq_len=-1),
 ])
 def test_rope_table_rejects_bad_params(lib, bad):
     p = dict(mode="yarn", head_dim=128, scale=4.0, original_max_pos=4096)

@@ -208,3 +208,31 @@ def sampled_check(w, n_random=16, max_heads=None):
                                   "yarn_L131072_s16", "sink_window_L65536"])
 def test_attn_full_size_sampled_rows(name):
     sampled_check(WORKLOADS[name])
+
+
+@pytest.mark.parametrize("mode", ["dynamic_ntk", "factors", "factors_short"])
+def test_attn_length_dependent_tables(mode):
+    """Dynamic NTK (base from the call's own length L) and per-pair factor tables
+    (long table, or the short one while L <= L_train) against the oracle."""
+    w = BASE.with_(L=700, Hq=4, Hkv=2, original_max_pos=256 if mode != "factors_short" else 1024,
+                   window=300, sinks=2)
+    q, k, v = make_inputs(w, device="cuda")
+    rng = np.random.default_rng(11)
+    kw = {}
+    if mode.startswith("factors"):
+        kw["factors"] = rng.uniform(1.0, 8.0, w.D // 2)
+        if mode == "factors_short":
+            kw["factors_short"] = rng.uniform(1.0, 1.2, w.D // 2)
+    omode = "dynamic_ntk" if mode == "dynamic_ntk" else "factors"
+    rope = lcx.RopeParams(omode, w.D, original_max_pos=w.original_max_pos, **kw)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = lcx.attn_fwd(q, k, v, rope, window=w.window, sinks=w.sinks, return_lse=True,
+                          status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    table, ms, _ = oracle.rope_table(omode, w.D, original_max_pos=w.original_max_pos,
+                                     seq_len=w.L, **kw)
+    ref_o, ref_lse = oracle.attn_full(q.float().cpu().numpy(), k.float().cpu().numpy(),
+                                      v.float().cpu().numpy(), table, ms, "half", 0, True,
+                                      w.window, w.sinks)
+    compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_lse)

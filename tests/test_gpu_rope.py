@@ -107,3 +107,20 @@ def test_apply_rope_full_size_sampled(name):
             tol = delta + 0.5 * ulp(np.abs(ref) + delta, torch.bfloat16)
             assert (np.abs(got - ref) <= tol).all()
         del y
+
+
+def test_apply_rope_dynamic_ntk_uses_offset_plus_length():
+    """Dynamic NTK in lcx_apply_rope takes the context length pos_offset + L."""
+    g = torch.Generator(device="cuda").manual_seed(3)
+    x = torch.randn((1, 2, 100, 128), generator=g, device="cuda").bfloat16()
+    rope = lcx.RopeParams("dynamic_ntk", 128, original_max_pos=4096)
+    y = lcx.apply_rope(x, rope, pos_offset=30000)
+    torch.cuda.synchronize()
+    table, ms, _ = oracle.rope_table("dynamic_ntk", 128, original_max_pos=4096, seq_len=30100)
+    xs = x.float().cpu().numpy().reshape(-1, 128)
+    pos = np.tile(np.arange(100) + 30000, 2)
+    ref = oracle.rotate_rows(xs, pos, table, ms, "half")
+    partner = np.concatenate([np.arange(64, 128), np.arange(64)])
+    delta = 2.0 ** -19 * (np.abs(xs) + np.abs(xs[:, partner]))
+    tol = delta + 0.5 * ulp(np.abs(ref) + delta, torch.bfloat16)
+    assert (np.abs(y.float().cpu().numpy().reshape(-1, 128) - ref) <= tol).all()

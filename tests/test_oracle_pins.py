@@ -465,3 +465,65 @@ def test_invalid_arguments_rejected():
     with pytest.raises(ValueError):   # window without causal
         oracle.attn_rows(np.zeros((1, 8), np.float32), [0], [0], [0], k, k, 2, table, ms,
                          causal=False, window=2)
+
+
+# --------------------------------------------------------------------------
+# length-dependent table variants
+# --------------------------------------------------------------------------
+
+def test_dynamic_ntk_keeps_short_sequences_plain():
+    """"AI Day 9: 长上下文技术", RoPE extension list item 4 (Dynamic NTK): the base
+    follows the actual sequence length and short sequences are unchanged."""
+    for seq in (1, 4096, 8192):
+        t, ms, _ = oracle.rope_table("dynamic_ntk", 128, original_max_pos=8192, seq_len=seq)
+        plain, _, _ = oracle.rope_table("plain", 128)
+        np.testing.assert_array_equal(t, plain)
+        assert ms == 1.0
+
+
+def test_dynamic_ntk_base_for_8k_to_128k():
+    """With the actual length 131072 over a training length of 8192 the dynamic
+    base is the NTK-aware base for s = 16: about 1.7e5 ("长上下文推理" plumephp NTK
+    comment); longer sequences get lower low frequencies."""
+    th, _ = oracle.rope_theta_ext("dynamic_ntk", 128, original_max_pos=8192, seq_len=131072)
+    pin("ntk_b1e4_d128_s16", ntk_base_from_table(th, 128))
+    prev = None
+    for seq in (16384, 32768, 65536, 131072):
+        th, _ = oracle.rope_theta_ext("dynamic_ntk", 128, original_max_pos=8192, seq_len=seq)
+        assert th[0] == 1.0
+        if prev is not None:
+            assert (th[1:] < prev[1:]).all()
+        prev = th
+
+
+def test_factor_tables():
+    """"Long Context: RoPE / YaRN / NTK / MLA", 7.3: theta'_i = theta_i / lambda_i.
+    lambda = s everywhere is PI (7.4's uniform row), lambda = 1 is plain, the
+    inverse YaRN multipliers reproduce YaRN (7.4: a three-segment ramp is one
+    choice of lambda), and 7.4's short-context rescue switches to the short table
+    while the actual length is within the training length."""
+    D, s = 128, 8.0
+    plain, _, _ = oracle.rope_table("plain", D)
+    pi, _, _ = oracle.rope_table("pi", D, scale=s)
+    t, ms, _ = oracle.rope_table("factors", D, factors=np.full(D // 2, s), seq_len=10 ** 6)
+    np.testing.assert_array_equal(t, pi)
+    assert ms == 1.0
+    t, _, _ = oracle.rope_table("factors", D, factors=np.ones(D // 2), seq_len=10 ** 6)
+    np.testing.assert_array_equal(t, plain)
+    th, _ = oracle.rope_theta_fp64("plain", D)
+    yarn, _ = oracle.rope_theta_fp64("yarn", D, scale=s, original_max_pos=8192)
+    lam = th / yarn
+    tf, _ = oracle.rope_theta_ext("factors", D, factors=lam, seq_len=10 ** 6)
+    np.testing.assert_allclose(tf, yarn, rtol=1e-15)
+    short = np.ones(D // 2)
+    long_ = np.full(D // 2, 4.0)
+    ts, _, _ = oracle.rope_table("factors", D, original_max_pos=4096, seq_len=4096,
+                                 factors=long_, factors_short=short)
+    tl, _, _ = oracle.rope_table("factors", D, original_max_pos=4096, seq_len=4097,
+                                 factors=long_, factors_short=short)
+    np.testing.assert_array_equal(ts, plain)
+    np.testing.assert_array_equal(tl, oracle.rope_table("pi", D, scale=4.0)[0])
+    with pytest.raises(ValueError):
+        oracle.rope_table("factors", D, factors=np.zeros(D // 2), seq_len=1)
+    with pytest.raises(ValueError):
+        oracle.rope_table("dynamic_ntk", D, seq_len=0)
