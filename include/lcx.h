@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define LCX_VERSION 100
+#define LCX_VERSION 101
 
 #if defined(__GNUC__)
 #define LCX_API __attribute__((visibility("default")))
@@ -145,6 +145,10 @@ LCX_API lcx_status lcx_apply_rope(const lcx_rope_params *params, const void *x, 
                                    rotated operands (needed when the logits are
                                    large, e.g. outlier-heavy activations); about
                                    twice the tensor-core work for QK^T        */
+#define LCX_ATTN_PREROTATED_K 4u /* k alone already holds rotated vectors (a KV
+                                   cache filled by lcx_apply_rope with the same
+                                   params, mscale included); q is rotated on
+                                   chip.  Ignored when LCX_ATTN_PREROTATED is set */
 #define LCX_ATTN_TEST_STALL 0x80000000u /* test hook for the watchdog: the loader
                                    issues no copies, so every wait of the
                                    kernel expires after watchdog_ms and the
@@ -153,8 +157,8 @@ LCX_API lcx_status lcx_apply_rope(const lcx_rope_params *params, const void *x, 
 
 typedef struct {
     const void *q;             /* DEVICE [B, Hq, L, D]                            */
-    const void *k;             /* DEVICE [B, Hkv, L, D]                           */
-    const void *v;             /* DEVICE [B, Hkv, L, D]                           */
+    const void *k;             /* DEVICE [B, Hkv, Lk, D]                          */
+    const void *v;             /* DEVICE [B, Hkv, Lk, D]                          */
     void *o;                   /* DEVICE [B, Hq, L, D], same dtype as q           */
     float *lse;                /* DEVICE [B, Hq, L] fp32 natural-log sum-exp of the
                                   scaled logits, or NULL                          */
@@ -173,6 +177,14 @@ typedef struct {
     uint32_t flags;            /* LCX_ATTN_* bits                                 */
     int32_t watchdog_ms;       /* wall-clock limit of every device wait, 1..60000;
                                   0 -> 2000 ms                                    */
+    int32_t reserved0;         /* must be 0                                       */
+    int64_t Lk;                /* key / value rows; 0 -> L (prefill)              */
+    int64_t q_offset;          /* position of query row 0: query i sits at
+                                  q_offset + i, key j at position j.  Chunked
+                                  prefill and decode pass the chunk's start
+                                  (decode: Lk - L).  With causal masking
+                                  q_offset + L <= Lk (every query sees its own
+                                  key); 0 for plain prefill                      */
 } lcx_attn_args;
 
 /*
@@ -183,9 +195,14 @@ typedef struct {
  *            times V), 6.3-6.4 (temperature via mscale on q and k), 10.1
  *            sliding window, 10.2 sinks; [B83] 8.3.4 (blockwise tiling with an
  *            exact online softmax), 8.3.3 (YaRN attention scaling).
- *   Visibility in prefill (queries and keys share positions 0..L-1): j <= i if
- *   causal; with W > 0 also i - j < W or j < S.  Rows with no visible key get
- *   o = 0 and lse = -inf.
+ *   Positions: query i at p_i = q_offset + i, key j at j (prefill: q_offset = 0,
+ *   Lk = L).  Visibility: j <= p_i if causal; with W > 0 also p_i - j < W or
+ *   j < S.  Chunked prefill / decode ([LC] 10.3, position offsets) passes the
+ *   new queries with the whole key cache; a StreamingLLM cache (sink entries
+ *   then the recent window, keys stored un-rotated) passes its entries in that
+ *   order, so every key is re-rotated on chip at its logical position (its
+ *   index in the cache) on every call.  Rows with no visible key get o = 0 and
+ *   lse = -inf.
  *   Arithmetic: q', k' rounded to bf16 on chip, QK^T and PV on bf16 tensor
  *   cores with fp32 accumulation, softmax statistics in fp32, o rounded once
  *   to the output dtype.  fp32 inputs are rounded to bf16 operands.

@@ -26,6 +26,7 @@ PAIRINGS = {"half": 0, "interleaved": 1}
 DTYPES = {"bf16": 0, "f32": 1}
 LCX_ATTN_PREROTATED = 1
 LCX_ATTN_SPLIT_QK = 2
+LCX_ATTN_PREROTATED_K = 4
 LCX_ATTN_TEST_STALL = 0x80000000
 
 # Symbols include/lcx.h declares; the library must export every one of them.
@@ -62,7 +63,8 @@ class _AttnArgs(ctypes.Structure):
                 ("v_strides", ctypes.c_int64 * 4), ("o_strides", ctypes.c_int64 * 4),
                 ("rope", _RopeParams), ("window", ctypes.c_int64), ("sinks", ctypes.c_int64),
                 ("softmax_scale", ctypes.c_float), ("flags", ctypes.c_uint32),
-                ("watchdog_ms", ctypes.c_int32)]
+                ("watchdog_ms", ctypes.c_int32), ("reserved0", ctypes.c_int32),
+                ("Lk", ctypes.c_int64), ("q_offset", ctypes.c_int64)]
 
 
 @dataclass
@@ -196,11 +198,16 @@ def apply_rope(x, rope: RopeParams, out=None, pos_offset: int = 0, inplace: bool
 def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, sinks: int = 0,
              softmax_scale: float = 0.0, return_lse: bool = False, prerotated: bool = False,
              split_qk: bool = False, out=None, lse=None, status=None, watchdog_ms: int = 0,
-             _test_stall: bool = False):
-    """Fused RoPE + causal attention prefill.
+             q_offset: int = 0, k_prerotated: bool = False, _test_stall: bool = False):
+    """Fused RoPE + causal attention (prefill, chunked prefill, decode).
 
-    q [B, Hq, L, D], k/v [B, Hkv, L, D] CUDA tensors (bf16 or fp32, last dim
-    contiguous).  Returns o [B, Hq, L, D] (and lse [B, Hq, L] fp32 if asked).
+    q [B, Hq, L, D], k/v [B, Hkv, Lk, D] CUDA tensors (bf16 or fp32, last dim
+    contiguous).  Query row i sits at position q_offset + i and key j at j
+    (prefill: q_offset 0 and Lk = L; decode of L new tokens against a cache of
+    Lk keys that already holds them: q_offset = Lk - L).  Returns o [B, Hq, L, D]
+    (and lse [B, Hq, L] fp32 if asked).
+    ``k_prerotated``: k already holds rotated keys (LCX_ATTN_PREROTATED_K), q is
+    rotated on chip; ``prerotated``: both are (LCX_ATTN_PREROTATED).
     ``split_qk`` forms QK^T from hi/lo bf16 parts of the rotated operands
     (LCX_ATTN_SPLIT_QK) for inputs whose large logits bf16 rounding would spoil.
     ``status`` (optional int32 CUDA tensor of one element) receives
@@ -211,8 +218,8 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
         if t.dim() != 4 or not t.is_cuda:
             raise ValueError("q, k, v must be 4-D CUDA tensors [B, H, L, D]")
     B, Hq, L, D = q.shape
-    Hkv = k.shape[1]
-    if k.shape != (B, Hkv, L, D) or v.shape != k.shape:
+    Hkv, Lk = k.shape[1], k.shape[2]
+    if k.shape != (B, Hkv, Lk, D) or v.shape != k.shape:
         raise ValueError("shape mismatch: q %s k %s v %s" % (q.shape, k.shape, v.shape))
     if not (q.dtype == k.dtype == v.dtype):
         raise ValueError("q, k, v must share a dtype")
@@ -233,8 +240,12 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
     a.window, a.sinks = int(window), int(sinks)
     a.softmax_scale = float(softmax_scale)
     a.flags = ((LCX_ATTN_PREROTATED if prerotated else 0) | (LCX_ATTN_SPLIT_QK if split_qk else 0)
+               | (LCX_ATTN_PREROTATED_K if k_prerotated else 0)
                | (LCX_ATTN_TEST_STALL if _test_stall else 0))
     a.watchdog_ms = int(watchdog_ms)
+    a.reserved0 = 0
+    a.Lk = Lk
+    a.q_offset = int(q_offset)
     _check(load().lcx_attn_fwd(ctypes.byref(a), _stream(q)))
     del rope_c
     return (o, lse) if return_lse else o

@@ -25,6 +25,10 @@
 //               running max/sum, writes P (bf16) back over S, rescales its O
 //               row only when the max grew by more than 2^8, and finally
 //               normalises O and stores it.
+// Positions: query row i sits at q_offset + i and key j at j, so one kernel
+// serves prefill (q_offset 0, Lk = L), chunked prefill and decode (the new
+// queries against the whole key cache), and a StreamingLLM cache whose
+// un-rotated keys are re-rotated at their cache index on every call.
 // Tiles entirely hidden by the causal/window mask are never visited; tiles
 // entirely visible skip the per-element mask.  Every barrier wait is bounded
 // (wall-clock timeout); on expiry the CTA winds down, releases TMEM and
@@ -78,10 +82,11 @@ struct AttnParams {
     float *lse;
     int *status;
     long long qs[3], ks[3], vs[3], os[3];  // element strides of B, H, L
-    int B, Hq, Hkv, L, G;
+    int B, Hq, Hkv, L, G;              // L: query rows
+    int Lk, qoff;                      // key rows; position of query row 0
     int causal, window, sinks;
     int n_qb, heads_per_unit, units_per_qb;
-    int rotate;
+    int rotate_q, rotate_k;
     int test_stall;                    // loader issues nothing (watchdog test hook)
     float c_log2;                      // logit scale in log2 units
     unsigned long long timeout_ns;
@@ -149,7 +154,8 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
 }
 
 // K tiles a query block visits: the sink tiles [0, ns) then the window tiles
-// [jlo, jhi]; every listed tile has at least one visible key.
+// [jlo, jhi]; every listed tile has at least one visible key.  Query row i sits
+// at position qoff + i, key j at position j.
 struct Tiles {
     int ns, jlo, n;
     __device__ __forceinline__ int tile(int j) const { return j < ns ? j : jlo + (j - ns); }
@@ -157,11 +163,11 @@ struct Tiles {
 
 template <int BN>
 __device__ __forceinline__ Tiles make_tiles(int q0, const AttnParams &p) {
-    const int i1 = min(q0 + kBM - 1, p.L - 1);
-    const int jhi = p.causal ? i1 / BN : (p.L - 1) / BN;
+    const int i1 = min(q0 + kBM - 1, p.L - 1) + p.qoff;
+    const int jhi = p.causal ? i1 / BN : (p.Lk - 1) / BN;
     int jlo = 0, ns = 0;
     if (p.causal && p.window > 0) {
-        jlo = max(0, q0 - p.window + 1) / BN;
+        jlo = max(0, q0 + p.qoff - p.window + 1) / BN;
         if (p.sinks > 0) ns = min((p.sinks + BN - 1) / BN, jlo);
     }
     Tiles t;
@@ -175,8 +181,8 @@ __device__ __forceinline__ Tiles make_tiles(int q0, const AttnParams &p) {
 template <int BN>
 __device__ __forceinline__ bool tile_full(int q0, int jt, const AttnParams &p) {
     const int j0 = jt * BN, j1 = j0 + BN - 1;
-    const int i0 = q0, i1 = q0 + kBM - 1;
-    if (j1 > p.L - 1) return false;
+    const int i0 = q0 + p.qoff, i1 = i0 + kBM - 1;
+    if (j1 > p.Lk - 1) return false;
     if (!p.causal) return true;
     if (j1 > i0) return false;
     if (p.window > 0 && !(j0 >= i1 - p.window + 1 || j1 < p.sinks)) return false;
@@ -366,16 +372,18 @@ __device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, uint8_t *lo, lon
 }
 
 // fp32 operands: load ROWS rows from global (rows >= L read as zero), rotate in
-// fp32 when asked, round to bf16 (hi, and lo in the split mode) into the tile.
+// fp32 when asked (row r at position pos0 + r), round to bf16 (hi, and lo in
+// the split mode) into the tile.
 template <int D, bool kHalf, bool kSplit, int ROWS>
 __device__ __forceinline__ void load_tile_f32(uint8_t *tile, uint8_t *lo, const float *base,
-                                              long long rs, int row0, int L, bool rotate,
-                                              const Phasor<D, kHalf> &ph, const AttnParams &p) {
+                                              long long rs, int row0, int L, long long pos0,
+                                              bool rotate, const Phasor<D, kHalf> &ph,
+                                              const AttnParams &p) {
     using R = Rot<D, kHalf>;
     constexpr int NJ = ROWS / R::RP;
     constexpr int BOX = ROWS * 128;
     float c[R::PPJ], s[R::PPJ];
-    if (rotate) ph.start(row0, p, c, s);
+    if (rotate) ph.start(pos0, p, c, s);
     for (int k = 0; k < NJ; ++k) {
         const int r = ph.r0 + k * R::RP;
         const bool valid = row0 + r < L;
@@ -648,17 +656,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         setmaxnreg_dec<kRegsRotate>();
         // ------------------------------------------------ rotation warpgroup
         const int tw = threadIdx.x - kWarpRot0 * 32;
-        const bool rot = p.rotate != 0;
+        const bool rotq = p.rotate_q != 0, rotk = p.rotate_k != 0;
         Phasor<D, kHalf> ph;
         ph.init(tw, p);
         PhasorCarry<Rot<D, kHalf>::PPJ> kcarry;
         bool ok = true;
         if (!kF32) {
             ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_q, 0, abort, tmo));
-            if (ok && (rot || kSplit))
+            if (ok && (rotq || kSplit))
                 for (int t = 0; t < U.nt; ++t) {
                     uint8_t *qt = sQ + t * C::kParts * C::kTileQ;
-                    rotate_tile_bf16<D, kHalf, kSplit, kBM>(qt, qt + C::kTileQ, U.q0, ph, p, rot);
+                    rotate_tile_bf16<D, kHalf, kSplit, kBM>(qt, qt + C::kTileQ,
+                                                            (long long)U.q0 + p.qoff, ph, p, rotq);
                 }
         } else {
             for (int t = 0; t < U.nt; ++t) {
@@ -666,7 +675,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     (long long)(U.hq0 + t) * p.qs[1];
                 uint8_t *qt = sQ + t * C::kParts * C::kTileQ;
                 load_tile_f32<D, kHalf, kSplit, kBM>(qt, qt + C::kTileQ, base, p.qs[2], U.q0, p.L,
-                                                     rot, ph, p);
+                                                     (long long)U.q0 + p.qoff, rotq, ph, p);
             }
         }
         if (ok) {
@@ -680,9 +689,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!kF32) {
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_k[s], use & 1, abort, tmo));
                 if (!ok) break;
-                if (rot || kSplit)
+                if (rotk || kSplit)
                     rotate_tile_bf16<D, kHalf, kSplit, BN>(tk, tk + C::kTileK, (long long)jt * BN,
-                                                           ph, p, rot, &kcarry);
+                                                           ph, p, rotk, &kcarry);
             } else {
                 if (use > 0)
                     ok = __all_sync(0xffffffffu,
@@ -691,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float *base = reinterpret_cast<const float *>(p.k) + U.b * p.ks[0] +
                                     (long long)U.g * p.ks[1];
                 load_tile_f32<D, kHalf, kSplit, BN>(tk, tk + C::kTileK, base, p.ks[2], jt * BN,
-                                                    p.L, rot, ph, p);
+                                                    p.Lk, (long long)jt * BN, rotk, ph, p);
             }
             fence_proxy_async_smem();
             mbar_arrive(&bar.ready_k[s]);
@@ -702,7 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 const float *base = reinterpret_cast<const float *>(p.v) + U.b * p.vs[0] +
                                     (long long)U.g * p.vs[1];
-                load_v_f32<D, BN>(sV + sv * C::kTileK, base, p.vs[2], jt * BN, p.L, tw);
+                load_v_f32<D, BN>(sV + sv * C::kTileK, base, p.vs[2], jt * BN, p.Lk, tw);
                 fence_proxy_async_smem();
                 mbar_arrive(&bar.full_v[sv]);
             }
@@ -716,7 +725,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int row = wq * 32 + lane;
             const uint32_t trow = tmem + (uint32_t(wq * 32) << 16);
             const uint32_t s_col = t * BN, o_col = C::kColO + t * D;
-            const int i = U.q0 + row;
+            const int i = U.q0 + row;      // query row; its position is qoff + i
+            const int pi = i + p.qoff;
             const float cl2 = p.c_log2;
             float m = -INFINITY, l = 0.f;
             bool ok = true;
@@ -727,8 +737,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int jt = T.tile(j), k0 = jt * BN;
                 const bool partial = !tile_full<BN>(U.q0, jt, p);
                 // visible columns: col <= hi and (no window or col >= lo or col < sk)
-                const int hi = p.causal ? min(i - k0, p.L - 1 - k0) : p.L - 1 - k0;
-                const int lo = i - p.window + 1 - k0;
+                const int hi = p.causal ? min(pi - k0, p.Lk - 1 - k0) : p.Lk - 1 - k0;
+                const int lo = pi - p.window + 1 - k0;
                 const int sk = p.sinks - k0;
                 const bool win = p.causal && p.window > 0;
                 auto vis = [&](int col) { return col <= hi && (!win || col >= lo || col < sk); };
@@ -947,8 +957,17 @@ extern "C" lcx_status lcx_attn_fwd(const lcx_attn_args *a, void *stream) {
         return fail(LCX_ERR_INVALID_ARG, "window and sinks must be >= 0");
     if (!a->causal && (a->window != 0 || a->sinks != 0))
         return fail(LCX_ERR_UNSUPPORTED, "window / sinks need causal attention");
-    if (a->flags & ~uint32_t(LCX_ATTN_PREROTATED | LCX_ATTN_SPLIT_QK | LCX_ATTN_TEST_STALL))
+    if (a->flags & ~uint32_t(LCX_ATTN_PREROTATED | LCX_ATTN_PREROTATED_K | LCX_ATTN_SPLIT_QK |
+                             LCX_ATTN_TEST_STALL))
         return fail(LCX_ERR_INVALID_ARG, "unknown flags");
+    if (a->reserved0 != 0) return fail(LCX_ERR_INVALID_ARG, "reserved0 must be 0");
+    const int64_t Lk = a->Lk > 0 ? a->Lk : a->L;
+    if (a->Lk < 0 || a->q_offset < 0)
+        return fail(LCX_ERR_INVALID_ARG, "Lk and q_offset must be >= 0");
+    if (a->causal && a->L > 0 && a->q_offset + a->L > Lk)
+        return fail(LCX_ERR_INVALID_ARG,
+                    "causal attention needs q_offset + L <= Lk (got %lld + %lld > %lld)",
+                    (long long)a->q_offset, (long long)a->L, (long long)Lk);
     if (a->watchdog_ms < 0 || a->watchdog_ms > 60000)
         return fail(LCX_ERR_INVALID_ARG, "watchdog_ms must be in [0, 60000]");
     if ((a->flags & LCX_ATTN_TEST_STALL) && a->dtype != LCX_BF16)
@@ -958,7 +977,8 @@ extern "C" lcx_status lcx_attn_fwd(const lcx_attn_args *a, void *stream) {
     if (a->D != 64 && a->D != 128)
         return fail(LCX_ERR_UNSUPPORTED, "head_dim %lld: only 64 and 128", (long long)a->D);
     if (a->B == 0 || a->L == 0) return LCX_OK;
-    if (a->L > (int64_t(1) << 30) || a->B > (int64_t(1) << 20) || a->Hq > 65536)
+    if (a->L > (int64_t(1) << 30) || Lk > (int64_t(1) << 30) ||
+        a->q_offset + a->L > (int64_t(1) << 30) || a->B > (int64_t(1) << 20) || a->Hq > 65536)
         return fail(LCX_ERR_UNSUPPORTED, "sizes too large");
     const int es = a->dtype == LCX_BF16 ? 2 : 4;
     if ((st = check_tensor(a->q, a->q_strides, es, "q")) != LCX_OK) return st;
@@ -984,20 +1004,27 @@ extern "C" lcx_status lcx_attn_fwd(const lcx_attn_args *a, void *stream) {
     p.Hq = int(a->Hq);
     p.Hkv = int(a->Hkv);
     p.L = int(a->L);
+    p.Lk = int(Lk);
+    p.qoff = int(a->q_offset);
     p.G = int(a->Hq / a->Hkv);
     p.causal = a->causal;
-    p.window = int(a->window > a->L ? a->L : a->window);
-    p.sinks = int(a->sinks > a->L ? a->L : a->sinks);
+    // A window of Lk or more keys, or Lk sinks, no longer restricts anything.
+    p.window = int(a->window > Lk ? Lk : a->window);
+    p.sinks = int(a->sinks > Lk ? Lk : a->sinks);
     p.n_qb = int((a->L + kBM - 1) / kBM);
     p.heads_per_unit = (p.G % 2 == 0) ? 2 : 1;
     p.units_per_qb = p.B * p.Hq / p.heads_per_unit;
     const long long grid = (long long)p.n_qb * p.units_per_qb;
     if (grid > 0x7fffffffLL) return fail(LCX_ERR_UNSUPPORTED, "too many work units");
-    p.rotate = (a->flags & LCX_ATTN_PREROTATED) ? 0 : 1;
+    p.rotate_q = (a->flags & LCX_ATTN_PREROTATED) ? 0 : 1;
+    p.rotate_k = (a->flags & (LCX_ATTN_PREROTATED | LCX_ATTN_PREROTATED_K)) ? 0 : 1;
     float ms = 1.f;
-    rope_table_unchecked(&a->rope, effective_seq_len(&a->rope, a->L), p.theta, &ms);
+    // The length-dependent modes see the whole context: the Lk keys.
+    rope_table_unchecked(&a->rope, effective_seq_len(&a->rope, Lk), p.theta, &ms);
     const double scale = a->softmax_scale > 0.f ? double(a->softmax_scale) : 1.0 / std::sqrt(double(a->D));
-    const double msq = p.rotate ? double(ms) * double(ms) : 1.0;
+    // Each operand rotated on chip contributes its mscale factor to the logits
+    // (pre-rotated operands already carry theirs).
+    const double msq = (p.rotate_q ? double(ms) : 1.0) * (p.rotate_k ? double(ms) : 1.0);
     p.c_log2 = float(scale * msq * 1.4426950408889634);
     // Legitimate waits last microseconds; the default limit is 2 s.
     p.timeout_ns = 1000000ull * (unsigned long long)(a->watchdog_ms > 0 ? a->watchdog_ms : 2000);
@@ -1012,9 +1039,9 @@ extern "C" lcx_status lcx_attn_fwd(const lcx_attn_args *a, void *stream) {
     if (a->dtype == LCX_BF16) {
         if ((st = make_map(&mq, a->q, a->B, a->Hq, a->L, a->D, a->q_strides, 128, "q")) != LCX_OK)
             return st;
-        if ((st = make_map(&mk, a->k, a->B, a->Hkv, a->L, a->D, a->k_strides, bn, "k")) != LCX_OK)
+        if ((st = make_map(&mk, a->k, a->B, a->Hkv, Lk, a->D, a->k_strides, bn, "k")) != LCX_OK)
             return st;
-        if ((st = make_map(&mv, a->v, a->B, a->Hkv, a->L, a->D, a->v_strides, bn, "v")) != LCX_OK)
+        if ((st = make_map(&mv, a->v, a->B, a->Hkv, Lk, a->D, a->v_strides, bn, "v")) != LCX_OK)
             return st;
     }
     const bool f32 = a->dtype == LCX_F32;

@@ -43,7 +43,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lcx.version() == 100
+    assert lcx.version() == 101
     for st in range(5):
         assert lib.lcx_status_string(st).decode()
     assert lib.lcx_status_string(99).decode() == "unknown status"
@@ -66,7 +66,8 @@ int main(void) {
   P(lcx_attn_args, dev_status) P(lcx_attn_args, dtype) P(lcx_attn_args, B) P(lcx_attn_args, D)
   P(lcx_attn_args, q_strides) P(lcx_attn_args, o_strides) P(lcx_attn_args, rope)
   P(lcx_attn_args, window) P(lcx_attn_args, sinks) P(lcx_attn_args, softmax_scale)
-  P(lcx_attn_args, flags) P(lcx_attn_args, watchdog_ms)
+  P(lcx_attn_args, flags) P(lcx_attn_args, watchdog_ms) P(lcx_attn_args, reserved0)
+  P(lcx_attn_args, Lk) P(lcx_attn_args, q_offset)
   return 0;
 }
 ''')
@@ -225,6 +226,12 @@ def _attn_args(**kw):
     (dict(watchdog_ms=-1), lcx.LCX_ERR_INVALID_ARG),
     (dict(watchdog_ms=60001), lcx.LCX_ERR_INVALID_ARG),
     (dict(dtype=1, flags=0x80000000), lcx.LCX_ERR_UNSUPPORTED),
+    (dict(reserved0=1), lcx.LCX_ERR_INVALID_ARG),
+    (dict(Lk=-1), lcx.LCX_ERR_INVALID_ARG),
+    (dict(q_offset=-1), lcx.LCX_ERR_INVALID_ARG),
+    (dict(q_offset=1), lcx.LCX_ERR_INVALID_ARG),            # causal: q_offset + L > Lk
+    (dict(Lk=255), lcx.LCX_ERR_INVALID_ARG),                # causal: L > Lk
+    (dict(Lk=1 << 31, q_offset=(1 << 31) - 256), lcx.LCX_ERR_UNSUPPORTED),
 ])
 def test_attn_validation_without_device(lib, kw, expect):
     a = _attn_args(**kw)

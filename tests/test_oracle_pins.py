@@ -527,3 +527,53 @@ def test_factor_tables():
         oracle.rope_table("factors", D, factors=np.zeros(D // 2), seq_len=1)
     with pytest.raises(ValueError):
         oracle.rope_table("dynamic_ntk", D, seq_len=0)
+
+
+# --------------------------------------------------------------------------
+# Chunked prefill, decode and the StreamingLLM cache ("Long Context: RoPE /
+# YaRN / NTK / MLA", section 10.3): the oracle evaluates query rows at any index
+# into the key arrays; these pin what the decode-time readings compute.
+
+def test_chunked_rows_equal_prefill_rows():
+    """A query chunk evaluated against only the keys up to its end equals the
+    same rows of the full causal prefill (keys beyond a causal row are masked)."""
+    B, Hq, Hkv, L, D = 1, 4, 2, 50, 32
+    table, ms, _ = oracle.rope_table("yarn", D, scale=4.0, original_max_pos=16)
+    q, k, v = _rand((B, Hq, L, D), 40), _rand((B, Hkv, L, D), 41), _rand((B, Hkv, L, D), 42)
+    o_full, l_full = oracle.attn_full(q, k, v, table, ms, window=11, sinks=2)
+    a, b = 17, 33
+    hh, ii = np.meshgrid(np.arange(Hq), np.arange(a, b), indexing="ij")
+    o, lse = oracle.attn_rows(q[0][hh.ravel(), ii.ravel()], np.zeros(hh.size, np.int64),
+                              hh.ravel(), ii.ravel(), k[:, :, :b], v[:, :, :b], Hq, table, ms,
+                              window=11, sinks=2)
+    np.testing.assert_array_equal(o.reshape(Hq, b - a, D), o_full[0, :, a:b])
+    np.testing.assert_array_equal(lse.reshape(Hq, b - a), l_full[0, :, a:b])
+
+
+def test_streaming_cache_without_sinks_is_a_sliding_window():
+    """With no sink tokens, a StreamingLLM step (the W most recent un-rotated keys
+    re-indexed to positions 0..W-1, the new token at position W) sees the same
+    keys at the same relative distances as sliding-window attention over the
+    absolute sequence with a window of W + 1 (the query included), so by the
+    relative-position property of RoPE (section 2.2) the outputs agree."""
+    H, N, D, W = 2, 64, 32, 12
+    table, ms, _ = oracle.rope_table("yarn", D, scale=8.0, original_max_pos=16)
+    q, k, v = _rand((1, H, N, D), 43), _rand((1, H, N, D), 44), _rand((1, H, N, D), 45)
+    o_abs, l_abs = oracle.attn_full(q, k, v, table, ms, window=W + 1)
+    for t in (W, W + 5, N - 1):
+        kc, vc = k[:, :, t - W:t + 1], v[:, :, t - W:t + 1]
+        o, lse = oracle.attn_rows(q[0, :, t], np.zeros(H, np.int64), np.arange(H),
+                                  np.full(H, W), kc, vc, H, table, ms)
+        np.testing.assert_allclose(o, o_abs[0, :, t], atol=1e-10, rtol=0)
+        np.testing.assert_allclose(lse, l_abs[0, :, t], atol=1e-10, rtol=0)
+
+
+def test_streaming_cache_before_eviction_is_plain_causal():
+    """While the sequence fits in S + W entries nothing is evicted, every key keeps
+    its index as position, and a decode step equals the last causal row."""
+    H, N, D = 1, 20, 16
+    table, ms, _ = oracle.rope_table("plain", D)
+    q, k, v = _rand((1, H, N, D), 46), _rand((1, H, N, D), 47), _rand((1, H, N, D), 48)
+    o_full, _ = oracle.attn_full(q, k, v, table, ms)
+    o, _ = oracle.attn_rows(q[0, :, N - 1], [0], [0], [N - 1], k, v, H, table, ms)
+    np.testing.assert_array_equal(o[0], o_full[0, 0, N - 1])
