@@ -56,6 +56,11 @@ def _load():
                                       ctypes.c_int, ctypes.c_int64, ctypes.c_int,
                                       ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
                                       f64p, f64p, ctypes.c_int]
+        lib.orc_attn_rows_keys.argtypes = (lib.orc_attn_rows.argtypes[:19] +
+                                           [ctypes.c_int64, ctypes.c_int64] +
+                                           lib.orc_attn_rows.argtypes[19:])
+        lib.orc_merge.argtypes = [f64p, f64p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                  f64p, f64p]
         lib.orc_num_threads.argtypes = [ctypes.c_int]
         _lib = lib
     return _lib
@@ -152,13 +157,15 @@ def mask(L, causal=True, window=0, sinks=0):
 
 
 def attn_rows(q_rows, row_b, row_h, row_i, k, v, Hq, table, mscale, pairing="half",
-                 pos_offset=0, causal=True, window=0, sinks=0, scale=None, nthreads=0):
+                 pos_offset=0, causal=True, window=0, sinks=0, scale=None, nthreads=0,
+                 k_begin=0, k_end=None):
     """Attention output o[n, D] and lse[n] (fp64) for selected query rows.
 
     q_rows: [n, D] raw (un-rotated) query rows; row_b/row_h/row_i: batch, query
     head and query index of each row; k, v: [B, Hkv, L, D] raw keys / values
     (fp32 arrays holding the exact input values); Hq: number of query heads
-    (query head h reads kv head h // (Hq // Hkv)).
+    (query head h reads kv head h // (Hq // Hkv)).  k_begin/k_end restrict the
+    keys to k_begin <= j < k_end (a partial result for merge()).
     """
     lib = _load()
     q_rows = np.ascontiguousarray(q_rows, dtype=np.float32)
@@ -168,12 +175,15 @@ def attn_rows(q_rows, row_b, row_h, row_i, k, v, Hq, table, mscale, pairing="hal
     row_h = np.ascontiguousarray(row_h, dtype=np.int64)
     row_i = np.ascontiguousarray(row_i, dtype=np.int64)
     return _attn_rows_impl(lib, q_rows, row_b, row_h, row_i, k, v, Hq, table, mscale,
-                           pairing, pos_offset, causal, window, sinks, scale, nthreads)
+                           pairing, pos_offset, causal, window, sinks, scale, nthreads,
+                           k_begin, k_end)
 
 
 def _attn_rows_impl(lib, q_rows, row_b, row_h, row_i, k, v, Hq, table, mscale, pairing,
-                    pos_offset, causal, window, sinks, scale, nthreads):
+                    pos_offset, causal, window, sinks, scale, nthreads, k_begin=0, k_end=None):
     B, Hkv, L, D = k.shape
+    if k_end is None:
+        k_end = L
     n = q_rows.shape[0]
     assert q_rows.shape == (n, D)
     if scale is None:
@@ -181,13 +191,14 @@ def _attn_rows_impl(lib, q_rows, row_b, row_h, row_i, k, v, Hq, table, mscale, p
     table = np.ascontiguousarray(table, dtype=np.float32)
     o = np.zeros((n, D), dtype=np.float64)
     lse = np.zeros(n, dtype=np.float64)
-    rc = lib.orc_attn_rows(_ptr(q_rows, ctypes.c_float), _ptr(row_b, ctypes.c_int64),
-                           _ptr(row_h, ctypes.c_int64), _ptr(row_i, ctypes.c_int64), n,
-                           _ptr(k, ctypes.c_float), _ptr(v, ctypes.c_float),
-                           B, Hq, Hkv, L, D, _ptr(table, ctypes.c_float), float(mscale),
-                           PAIRINGS[pairing], int(pos_offset), int(causal), int(window),
-                           int(sinks), float(scale), _ptr(o, ctypes.c_double),
-                           _ptr(lse, ctypes.c_double), int(nthreads))
+    rc = lib.orc_attn_rows_keys(_ptr(q_rows, ctypes.c_float), _ptr(row_b, ctypes.c_int64),
+                                _ptr(row_h, ctypes.c_int64), _ptr(row_i, ctypes.c_int64), n,
+                                _ptr(k, ctypes.c_float), _ptr(v, ctypes.c_float),
+                                B, Hq, Hkv, L, D, _ptr(table, ctypes.c_float), float(mscale),
+                                PAIRINGS[pairing], int(pos_offset), int(causal), int(window),
+                                int(sinks), int(k_begin), int(k_end), float(scale),
+                                _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double),
+                                int(nthreads))
     if rc:
         raise ValueError("orc_attn_rows: invalid argument (rc=%d)" % rc)
     return o, lse
@@ -207,3 +218,21 @@ def attn_full(q, k, v, table, mscale, pairing="half", pos_offset=0, causal=True,
 
 def num_threads(nthreads=0):
     return int(_load().orc_num_threads(nthreads))
+
+
+def merge(o_parts, lse_parts):
+    """Combine partial results over disjoint key sets: o_parts [n, ..., D] and
+    lse_parts [n, ...] (fp64) -> o [..., D], lse [...] (see orc_merge)."""
+    o_parts = np.ascontiguousarray(o_parts, dtype=np.float64)
+    lse_parts = np.ascontiguousarray(lse_parts, dtype=np.float64)
+    n, D = o_parts.shape[0], o_parts.shape[-1]
+    lead = lse_parts.shape[1:]
+    assert o_parts.shape == (n,) + lead + (D,)
+    rows = int(np.prod(lead)) if lead else 1
+    o = np.zeros(lead + (D,), dtype=np.float64)
+    lse = np.zeros(lead, dtype=np.float64)
+    rc = _load().orc_merge(_ptr(o_parts, ctypes.c_double), _ptr(lse_parts, ctypes.c_double),
+                           n, rows, D, _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    if rc:
+        raise ValueError("orc_merge: invalid argument (rc=%d)" % rc)
+    return o, lse

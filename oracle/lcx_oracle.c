@@ -338,6 +338,7 @@ typedef struct {
     double ms;
     int pairing, causal;
     int64_t window, sinks;
+    int64_t k_begin, k_end;  /* only keys k_begin <= j < k_end take part */
     double scale;
     double *o;               /* [nrows, D] */
     double *lse;             /* [nrows] */
@@ -361,7 +362,8 @@ static void row_body(void *vctx, int64_t t)
     double *s = (double *)malloc(sizeof(double) * (size_t)L);
     double mx = -INFINITY;
     for (int64_t j = 0; j < L; j++) {
-        if (!orc_visible(i, j, L, c->causal, c->window, c->sinks)) { s[j] = -INFINITY; continue; }
+        if (j < c->k_begin || j >= c->k_end ||
+            !orc_visible(i, j, L, c->causal, c->window, c->sinks)) { s[j] = -INFINITY; continue; }
         double dot = 0.0;
         const double *kj = c->kr + j * D;
         for (int64_t d = 0; d < D; d++) dot += qr[d] * kj[d];
@@ -401,14 +403,15 @@ static void row_body(void *vctx, int64_t t)
  * Outputs o [nrows, D] and lse [nrows] in fp64.  Keys of one (b, kv head) are
  * rotated once and reused by all selected rows of that head.
  */
-int orc_attn_rows(const float *q, const int64_t *row_b, const int64_t *row_h,
-                  const int64_t *row_i, int64_t nrows,
-                  const float *k, const float *v,
-                  int64_t B, int64_t Hq, int64_t Hkv, int64_t L, int64_t D,
-                  const float *table, float mscale, int pairing, int64_t pos_offset,
-                  int causal, int64_t window, int64_t sinks, double scale,
-                  double *o, double *lse, int nthreads)
+int orc_attn_rows_keys(const float *q, const int64_t *row_b, const int64_t *row_h,
+                       const int64_t *row_i, int64_t nrows,
+                       const float *k, const float *v,
+                       int64_t B, int64_t Hq, int64_t Hkv, int64_t L, int64_t D,
+                       const float *table, float mscale, int pairing, int64_t pos_offset,
+                       int causal, int64_t window, int64_t sinks, int64_t k_begin,
+                       int64_t k_end, double scale, double *o, double *lse, int nthreads)
 {
+    if (k_begin < 0 || k_end < k_begin || k_end > L) return 1;
     if (D <= 0 || D > 4096 || (D % 2) != 0) return 1;
     if (Hkv <= 0 || Hq <= 0 || (Hq % Hkv) != 0 || L <= 0 || B <= 0) return 1;
     if (!causal && (window != 0 || sinks != 0)) return 1;
@@ -431,12 +434,65 @@ int orc_attn_rows(const float *q, const int64_t *row_b, const int64_t *row_h,
             rot_keys_ctx rk = {k, kr, b, g, Hkv, L, D, pos_offset, table, (double)mscale, pairing};
             orc_parallel_for(L, nthreads, rot_keys_body, &rk);
             row_ctx rc = {q, row_i, sel, kr, v, b, g, Hkv, L, D, pos_offset, table,
-                          (double)mscale, pairing, causal, window, sinks, scale, o, lse};
+                          (double)mscale, pairing, causal, window, sinks, k_begin, k_end,
+                          scale, o, lse};
             orc_parallel_for(ns, nthreads, row_body, &rc);
         }
     }
     free(sel);
     free(kr);
+    return 0;
+}
+
+/* orc_attn_rows_keys over all keys. */
+int orc_attn_rows(const float *q, const int64_t *row_b, const int64_t *row_h,
+                  const int64_t *row_i, int64_t nrows,
+                  const float *k, const float *v,
+                  int64_t B, int64_t Hq, int64_t Hkv, int64_t L, int64_t D,
+                  const float *table, float mscale, int pairing, int64_t pos_offset,
+                  int causal, int64_t window, int64_t sinks, double scale,
+                  double *o, double *lse, int nthreads)
+{
+    return orc_attn_rows_keys(q, row_b, row_h, row_i, nrows, k, v, B, Hq, Hkv, L, D, table,
+                              mscale, pairing, pos_offset, causal, window, sinks, 0, L, scale,
+                              o, lse, nthreads);
+}
+
+/*
+ * Combine partial attention results of the same query rows over disjoint key
+ * sets ("8.3 长上下文技术", 8.3.4 online softmax and 8.3.5 Ring Attention step 3:
+ * partial outputs are merged by rescaling with their softmax statistics).
+ * Part s of a row holds o_s = sum_{j in K_s} e^{s_j} v_j / Z_s and
+ * lse_s = ln Z_s (Z_s = sum_{j in K_s} e^{s_j}; an empty K_s has lse_s = -inf).
+ * Then Z = sum_s Z_s = e^m sum_s e^{lse_s - m} with m = max_s lse_s, and
+ *   o = sum_s Z_s o_s / Z = sum_s e^{lse_s - m} o_s / sum_s e^{lse_s - m},
+ *   lse = m + ln sum_s e^{lse_s - m}.
+ * o_parts [n_parts, rows, D], lse_parts [n_parts, rows]; o [rows, D], lse [rows].
+ * A row whose parts are all empty gets o = 0, lse = -inf.
+ */
+int orc_merge(const double *o_parts, const double *lse_parts, int64_t n_parts, int64_t rows,
+              int64_t D, double *o, double *lse)
+{
+    if (n_parts <= 0 || rows < 0 || D <= 0) return 1;
+    for (int64_t r = 0; r < rows; r++) {
+        double m = -INFINITY;
+        for (int64_t s = 0; s < n_parts; s++)
+            if (lse_parts[s * rows + r] > m) m = lse_parts[s * rows + r];
+        double *orow = o + r * D;
+        for (int64_t d = 0; d < D; d++) orow[d] = 0.0;
+        if (m == -INFINITY) { lse[r] = -INFINITY; continue; }
+        double z = 0.0;
+        for (int64_t s = 0; s < n_parts; s++) {
+            double l = lse_parts[s * rows + r];
+            if (l == -INFINITY) continue;
+            double w = exp(l - m);
+            z += w;
+            const double *op = o_parts + (s * rows + r) * D;
+            for (int64_t d = 0; d < D; d++) orow[d] += w * op[d];
+        }
+        for (int64_t d = 0; d < D; d++) orow[d] /= z;
+        lse[r] = m + log(z);
+    }
     return 0;
 }
 

@@ -577,3 +577,58 @@ def test_streaming_cache_before_eviction_is_plain_causal():
     o_full, _ = oracle.attn_full(q, k, v, table, ms)
     o, _ = oracle.attn_rows(q[0, :, N - 1], [0], [0], [N - 1], k, v, H, table, ms)
     np.testing.assert_array_equal(o[0], o_full[0, 0, N - 1])
+
+
+# --------------------------------------------------------------------------
+# Split-KV partial attention and the (O, LSE) merge ("8.3 长上下文技术", 8.3.4
+# online softmax, 8.3.5 Ring Attention step 3).
+
+@pytest.mark.parametrize("causal,W,S", [(True, 0, 0), (True, 9, 3), (False, 0, 0)])
+def test_merge_of_key_partitions_is_full_attention(causal, W, S):
+    """Partial results over a partition of the keys (some parts empty for some
+    rows) merge to the full attention result: the softmax identity behind
+    split-KV and ring attention."""
+    B, Hq, Hkv, L, D = 1, 4, 2, 41, 32
+    table, ms, _ = oracle.rope_table("yarn", D, scale=4.0, original_max_pos=16)
+    q, k, v = _rand((B, Hq, L, D), 50), _rand((B, Hkv, L, D), 51), _rand((B, Hkv, L, D), 52)
+    o_full, l_full = oracle.attn_full(q, k, v, table, ms, "half", 0, causal, W, S)
+    hh, ii = np.meshgrid(np.arange(Hq), np.arange(L), indexing="ij")
+    rows = dict(q_rows=q[0][hh.ravel(), ii.ravel()], row_b=np.zeros(hh.size, np.int64),
+                row_h=hh.ravel(), row_i=ii.ravel(), k=k, v=v, Hq=Hq, table=table, mscale=ms,
+                causal=causal, window=W, sinks=S)
+    cuts = [0, 5, 6, 20, 33, 41]
+    parts = [oracle.attn_rows(**rows, k_begin=a, k_end=b) for a, b in zip(cuts, cuts[1:])]
+    o, lse = oracle.merge(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+    np.testing.assert_allclose(o.reshape(Hq, L, D), o_full[0], atol=1e-12, rtol=0)
+    np.testing.assert_allclose(lse.reshape(Hq, L), l_full[0], atol=1e-12, rtol=0)
+    # a part with no visible key is the empty sum
+    assert np.isneginf(parts[-1][1][:5]).all() or not causal
+
+
+def test_merge_closed_forms():
+    rng = np.random.default_rng(53)
+    o1, o2 = rng.standard_normal((2, 3, 8))
+    l1 = rng.standard_normal(3)
+    # one part: identity
+    o, lse = oracle.merge(o1[None], l1[None])
+    np.testing.assert_array_equal(o, o1)
+    np.testing.assert_array_equal(lse, l1)
+    # equal weights: the mean, lse + ln 2
+    o, lse = oracle.merge(np.stack([o1, o2]), np.stack([l1, l1]))
+    np.testing.assert_allclose(o, (o1 + o2) / 2, atol=1e-15)
+    np.testing.assert_allclose(lse, l1 + math.log(2), atol=1e-15)
+    # an empty part changes nothing; all parts empty -> o = 0, lse = -inf
+    o, lse = oracle.merge(np.stack([o1, o2]), np.stack([l1, np.full(3, -np.inf)]))
+    np.testing.assert_array_equal(o, o1)
+    np.testing.assert_array_equal(lse, l1)
+    o, lse = oracle.merge(np.stack([o1, o2]), np.full((2, 3), -np.inf))
+    assert (o == 0).all() and np.isneginf(lse).all()
+    # weights e^{lse_s}: a part 10 nats heavier dominates with weight 1/(1+e^-10)
+    o, _ = oracle.merge(np.stack([o1, o2]), np.stack([l1 + 10.0, l1]))
+    w = 1.0 / (1.0 + math.exp(-10.0))
+    np.testing.assert_allclose(o, w * o1 + (1 - w) * o2, atol=1e-14)
+    # order of the parts does not matter
+    oa, la = oracle.merge(np.stack([o1, o2]), np.stack([l1, l1 - 1]))
+    ob, lb = oracle.merge(np.stack([o2, o1]), np.stack([l1 - 1, l1]))
+    np.testing.assert_allclose(oa, ob, atol=1e-15)
+    np.testing.assert_allclose(la, lb, atol=1e-15)
