@@ -263,6 +263,9 @@ def bench_gpu(args, world, rank, local):
     rope_ms = statistics.median(a.elapsed_time(b) for a, b in rope_ev)
     del qr, kr
 
+    # --- split-KV decode: one new token per query head against the whole cache
+    decode = bench_decode(lcx, w, q, k, v, rope, stream, status)
+
     # --- end to end through host buffers
     qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
     ws = {}
@@ -336,7 +339,12 @@ def bench_gpu(args, world, rank, local):
         "e2e": {"value": round(e2e_tflops, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "clocks": clk.summary(),
+        "splitkv_decode": decode,
     }
+    if decode is not None:
+        decode["peak"] = float(peaks["hbm_gbs"])
+        decode["frac"] = round(decode["achieved"] / decode["peak"], 4)
+        res["gpu_launches_decode"] = decode["launches"]
     del q, k, v, o
     torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -344,6 +352,43 @@ def bench_gpu(args, world, rank, local):
         res["cpu_baseline"] = {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                                "sample": desc, "seconds": round(secs, 2)}
     return res
+
+
+def bench_decode(lcx, w, q, k, v, rope, stream, status, reps=20):
+    """Decode step on the workload's cache: the last query position of every
+    head (q_offset = L - 1) against all L keys, through lcx_attn_fwd_split for a
+    few split counts.  HBM-bound: the algorithmic bytes are K and V read once
+    (plus q and o); reported against the measured copy bandwidth."""
+    if not w.causal or w.L < 2 * 128:
+        return None
+    qd = q[:, :, -1:].contiguous()
+    od = torch.empty_like(qd)
+    kw = dict(causal=True, window=w.window, sinks=w.sinks, softmax_scale=w.softmax_scale,
+              split_qk=w.split_qk, out=od, status=status, q_offset=w.L - 1)
+    nbytes = sum(t.numel() * t.element_size() for t in (k, v, qd, od))
+    sweep = {}
+    for splits in (1, 8, 16, 32, 64):
+        ws = torch.empty(max(1, lcx.split_workspace_bytes(w.B, w.Hq, 1, w.D, splits)),
+                         dtype=torch.uint8, device=q.device)
+        for _ in range(3):
+            lcx.attn_fwd(qd, k, v, rope, num_splits=splits, workspace=ws, **kw)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            lcx.attn_fwd(qd, k, v, rope, num_splits=splits, workspace=ws, **kw)
+        b.record(stream)
+        torch.cuda.synchronize()
+        sweep[splits] = a.elapsed_time(b) / reps
+    assert int(status.item()) == 0, "device watchdog fired in decode"
+    best = min(sweep, key=sweep.get)
+    us = sweep[best] * 1e3
+    return {"what": "1 new token per head (B=%d, Hq=%d) against %d cached keys, q_offset = "
+                    "L - 1, keys rotated on chip" % (w.B, w.Hq, w.L),
+            "bound": "hbm", "num_splits": best, "us_per_call": round(us, 2),
+            "us_by_splits": {str(s_): round(t * 1e3, 2) for s_, t in sweep.items()},
+            "bytes": nbytes, "achieved": round(nbytes / (us * 1e-6) / 1e9, 1), "unit": "GB/s",
+            "launches": (1 if best == 1 else 2) * reps}
 
 
 def bench_reference(args, world, rank):

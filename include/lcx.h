@@ -2,7 +2,8 @@
  * lcx.h -- C ABI of the long-context RoPE + causal attention prefill library
  * (liblcx.so, sm_100a).
  *
- * Three calls make up the hot path:
+ * Three calls make up the hot path (lcx_attn_fwd_split and lcx_attn_merge
+ * add split-KV evaluation for decode-sized problems):
  *   lcx_rope_table  per-pair RoPE frequencies theta'_i and the attention scale
  *                   for plain RoPE, Position Interpolation, NTK-aware base
  *                   scaling and YaRN (NTK-by-parts ramp + 0.1 ln s + 1).
@@ -210,6 +211,57 @@ typedef struct {
  *   multiples of 16 bytes, D's stride 1.  Enqueued on `stream`.
  */
 LCX_API lcx_status lcx_attn_fwd(const lcx_attn_args *args, void *stream);
+
+/*
+ * lcx_attn_fwd_split -- lcx_attn_fwd evaluated as num_splits partial
+ * attentions, each over a consecutive stretch of a query block's key tiles
+ * (split-KV), combined by the merge of lcx_attn_merge.  It runs num_splits
+ * times more CTAs, which fills the GPU when there are few query blocks
+ * (decode, short chunks against a long cache); the result equals
+ * lcx_attn_fwd's up to rounding (the partial outputs are fp32).
+ *   Defines: [B83] 8.3.4 (online softmax), 8.3.5 step 3 (a KV block's partial
+ *            output folded in by rescaling with its softmax statistics).
+ *   num_splits     : 1..256; 1 is lcx_attn_fwd and uses no workspace.  Splits
+ *                    beyond a query block's tile count are empty and cost a
+ *                    CTA each.
+ *   workspace      : DEVICE buffer, 256-byte aligned, of at least
+ *                    lcx_attn_split_workspace_bytes(B, Hq, L, D, num_splits)
+ *                    bytes.  Owned by the caller; its contents on entry are
+ *                    ignored and overwritten; two calls in flight at the same
+ *                    time must not share it.
+ *   Enqueues two kernels on `stream` (attention, then merge).  Errors as for
+ *   lcx_attn_fwd; a short workspace is LCX_ERR_INVALID_ARG.
+ */
+LCX_API lcx_status lcx_attn_fwd_split(const lcx_attn_args *args, int32_t num_splits,
+                                      void *workspace, int64_t workspace_bytes, void *stream);
+
+/* Workspace bytes lcx_attn_fwd_split needs: [num_splits, B, Hq, L, D] fp32
+ * partial outputs then [num_splits, B, Hq, L] fp32 partial LSEs, each block
+ * rounded up to 256 bytes.  0 when num_splits == 1; -1 for invalid sizes
+ * (D not 64/128, num_splits outside 1..256, or more than 2^40 query rows). */
+LCX_API int64_t lcx_attn_split_workspace_bytes(int64_t B, int64_t Hq, int64_t L, int64_t D,
+                                               int32_t num_splits);
+
+/*
+ * lcx_attn_merge -- combine n_parts partial attention results of the same
+ * query rows over disjoint key sets: with m = max_s lse_s and
+ * w_s = exp(lse_s - m), o = sum_s w_s o_s / sum_s w_s and
+ * lse = m + ln sum_s w_s.  Parts with lse_s = -inf (no key) weigh nothing; a
+ * row with no non-empty part gets o = 0, lse = -inf.
+ *   Defines: [B83] 8.3.4 (online softmax rescaling), 8.3.5 step 3 (Ring
+ *            Attention: partial outputs combined by their statistics).
+ *   o_parts  : DEVICE fp32 [n_parts, B, Hq, L, D], contiguous, 16-byte
+ *              aligned; row r of part s normalised over that part's keys.
+ *   lse_parts: DEVICE fp32 [n_parts, B, Hq, L], contiguous (natural log).
+ *   o        : DEVICE [B, Hq, L, D] of `dtype`, element strides o_strides
+ *              (D's stride 1, others multiples of 16 bytes), 16-byte aligned.
+ *   lse      : DEVICE fp32 [B, Hq, L] contiguous, or NULL.
+ *   Supported: D in {64, 128}, n_parts 1..4096.  Enqueued on `stream`.
+ */
+LCX_API lcx_status lcx_attn_merge(const float *o_parts, const float *lse_parts, int32_t n_parts,
+                                  int64_t B, int64_t Hq, int64_t L, int64_t D, void *o,
+                                  int32_t dtype, const int64_t *o_strides, float *lse,
+                                  void *stream);
 
 /* Static description of a status code. */
 LCX_API const char *lcx_status_string(lcx_status status);

@@ -30,7 +30,8 @@ LCX_ATTN_PREROTATED_K = 4
 LCX_ATTN_TEST_STALL = 0x80000000
 
 # Symbols include/lcx.h declares; the library must export every one of them.
-EXPORTED = ("lcx_rope_table", "lcx_apply_rope", "lcx_attn_fwd", "lcx_status_string",
+EXPORTED = ("lcx_rope_table", "lcx_apply_rope", "lcx_attn_fwd", "lcx_attn_fwd_split",
+            "lcx_attn_split_workspace_bytes", "lcx_attn_merge", "lcx_status_string",
             "lcx_last_error", "lcx_version")
 
 
@@ -131,6 +132,17 @@ def load(path: str = LIB_PATH):
     lib.lcx_apply_rope.restype = ctypes.c_int
     lib.lcx_attn_fwd.argtypes = [ctypes.POINTER(_AttnArgs), ctypes.c_void_p]
     lib.lcx_attn_fwd.restype = ctypes.c_int
+    lib.lcx_attn_fwd_split.argtypes = [ctypes.POINTER(_AttnArgs), ctypes.c_int32, ctypes.c_void_p,
+                                       ctypes.c_int64, ctypes.c_void_p]
+    lib.lcx_attn_fwd_split.restype = ctypes.c_int
+    lib.lcx_attn_split_workspace_bytes.argtypes = [ctypes.c_int64] * 4 + [ctypes.c_int32]
+    lib.lcx_attn_split_workspace_bytes.restype = ctypes.c_int64
+    lib.lcx_attn_merge.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                   ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                   ctypes.c_void_p, ctypes.c_int32,
+                                   ctypes.POINTER(ctypes.c_int64), ctypes.c_void_p,
+                                   ctypes.c_void_p]
+    lib.lcx_attn_merge.restype = ctypes.c_int
     lib.lcx_status_string.argtypes = [ctypes.c_int]
     lib.lcx_status_string.restype = ctypes.c_char_p
     lib.lcx_last_error.argtypes = []
@@ -198,7 +210,8 @@ def apply_rope(x, rope: RopeParams, out=None, pos_offset: int = 0, inplace: bool
 def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, sinks: int = 0,
              softmax_scale: float = 0.0, return_lse: bool = False, prerotated: bool = False,
              split_qk: bool = False, out=None, lse=None, status=None, watchdog_ms: int = 0,
-             q_offset: int = 0, k_prerotated: bool = False, _test_stall: bool = False):
+             q_offset: int = 0, k_prerotated: bool = False, num_splits: int = 1,
+             workspace=None, _test_stall: bool = False):
     """Fused RoPE + causal attention (prefill, chunked prefill, decode).
 
     q [B, Hq, L, D], k/v [B, Hkv, Lk, D] CUDA tensors (bf16 or fp32, last dim
@@ -208,6 +221,9 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
     (and lse [B, Hq, L] fp32 if asked).
     ``k_prerotated``: k already holds rotated keys (LCX_ATTN_PREROTATED_K), q is
     rotated on chip; ``prerotated``: both are (LCX_ATTN_PREROTATED).
+    ``num_splits`` > 1 runs split-KV (lcx_attn_fwd_split): each query block's
+    key tiles are shared among that many CTAs and the partial results merged;
+    ``workspace`` (uint8 CUDA tensor) is allocated when not given.
     ``split_qk`` forms QK^T from hi/lo bf16 parts of the rotated operands
     (LCX_ATTN_SPLIT_QK) for inputs whose large logits bf16 rounding would spoil.
     ``status`` (optional int32 CUDA tensor of one element) receives
@@ -246,9 +262,52 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
     a.reserved0 = 0
     a.Lk = Lk
     a.q_offset = int(q_offset)
-    _check(load().lcx_attn_fwd(ctypes.byref(a), _stream(q)))
+    if num_splits == 1:
+        _check(load().lcx_attn_fwd(ctypes.byref(a), _stream(q)))
+    else:
+        need = split_workspace_bytes(B, Hq, L, D, num_splits)
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _check(load().lcx_attn_fwd_split(ctypes.byref(a), int(num_splits),
+                                         ctypes.c_void_p(workspace.data_ptr()),
+                                         workspace.numel() * workspace.element_size(),
+                                         _stream(q)))
     del rope_c
     return (o, lse) if return_lse else o
+
+
+def split_workspace_bytes(B, Hq, L, D, num_splits):
+    """Bytes of workspace lcx_attn_fwd_split needs (0 for one split)."""
+    n = int(load().lcx_attn_split_workspace_bytes(B, Hq, L, D, int(num_splits)))
+    if n < 0:
+        raise ValueError("invalid split-KV sizes")
+    return n
+
+
+def attn_merge(o_parts, lse_parts, out=None, lse=None, dtype=None):
+    """Merge partial results over disjoint key sets (lcx_attn_merge).
+
+    o_parts [n, B, Hq, L, D] and lse_parts [n, B, Hq, L] fp32 contiguous CUDA
+    tensors -> o [B, Hq, L, D] (bf16 unless ``dtype`` or ``out`` says
+    otherwise) and lse [B, Hq, L] fp32.
+    """
+    import torch
+    if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32:
+        raise ValueError("partial results must be fp32")
+    if not (o_parts.is_contiguous() and lse_parts.is_contiguous()):
+        raise ValueError("partial results must be contiguous")
+    n, B, Hq, L, D = o_parts.shape
+    if lse_parts.shape != (n, B, Hq, L):
+        raise ValueError("lse_parts shape %s != %s" % (tuple(lse_parts.shape), (n, B, Hq, L)))
+    if out is None:
+        out = torch.empty((B, Hq, L, D), dtype=dtype or torch.bfloat16, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=o_parts.device)
+    _check(load().lcx_attn_merge(ctypes.c_void_p(o_parts.data_ptr()),
+                                 ctypes.c_void_p(lse_parts.data_ptr()), n, B, Hq, L, D,
+                                 ctypes.c_void_p(out.data_ptr()), _dtype_code(out), _strides(out),
+                                 ctypes.c_void_p(lse.data_ptr()), _stream(o_parts)))
+    return out, lse
 
 
 def attn_fwd_host(q, k, v, rope: RopeParams, device="cuda", workspace=None, **kw):

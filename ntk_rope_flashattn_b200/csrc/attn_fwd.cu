@@ -87,6 +87,9 @@ struct AttnParams {
     int causal, window, sinks;
     int n_qb, heads_per_unit, units_per_qb;
     int rotate_q, rotate_k;
+    int n_split;                       // key-range splits per unit (1: plain output)
+    float *part_o;                     // n_split > 1: [n_split, B, Hq, L, D] partial o
+    float *part_lse;                   //              [n_split, B, Hq, L] partial lse
     int test_stall;                    // loader issues nothing (watchdog test hook)
     float c_log2;                      // logit scale in log2 units
     unsigned long long timeout_ns;
@@ -131,16 +134,17 @@ struct Bars {
 
 // ---------------------------------------------------------------- schedule
 struct Unit {
-    int b, g, hq0, nt, q0;
+    int b, g, hq0, nt, q0, split;
 };
 
 // Work units are grouped by (batch, kv head) and, inside a group, numbered
 // heaviest first (query blocks from the end of the sequence, which see the
 // most keys).  The block scheduler therefore runs many query blocks of the same
 // kv head side by side -- they stream the same K/V tiles, which L2 then serves
-// -- and still hands out the longest units of every group first.
+// -- and still hands out the longest units of every group first.  With key
+// splits, the n_split CTAs of a unit are consecutive.
 __device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
-    const int u = blockIdx.x;
+    const int u = blockIdx.x / p.n_split;
     const int upq = p.G / p.heads_per_unit;          // units per query block of a group
     const int per_group = p.n_qb * upq;
     const int grp = u / per_group, rem = u % per_group;
@@ -150,15 +154,20 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
     r.q0 = (p.n_qb - 1 - rem / upq) * kBM;
     r.nt = p.heads_per_unit;
     r.hq0 = r.g * p.G + p.heads_per_unit * (rem % upq);
+    r.split = blockIdx.x % p.n_split;
     return r;
 }
 
 // K tiles a query block visits: the sink tiles [0, ns) then the window tiles
 // [jlo, jhi]; every listed tile has at least one visible key.  Query row i sits
 // at position qoff + i, key j at position j.
+// A key split takes the consecutive stretch [j0, j0 + n) of that list.
 struct Tiles {
-    int ns, jlo, n;
-    __device__ __forceinline__ int tile(int j) const { return j < ns ? j : jlo + (j - ns); }
+    int ns, jlo, n, j0;
+    __device__ __forceinline__ int tile(int j) const {
+        const int x = j + j0;
+        return x < ns ? x : jlo + (x - ns);
+    }
 };
 
 template <int BN>
@@ -174,6 +183,15 @@ __device__ __forceinline__ Tiles make_tiles(int q0, const AttnParams &p) {
     t.ns = ns;
     t.jlo = jlo;
     t.n = ns + (jhi - jlo + 1);
+    t.j0 = 0;
+    if (p.n_split > 1) {
+        // split s of S takes tiles [n s / S, n (s + 1) / S); it may be empty
+        const int s = blockIdx.x % p.n_split;
+        const int jb = int((long long)t.n * s / p.n_split);
+        const int je = int((long long)t.n * (s + 1) / p.n_split);
+        t.j0 = jb;
+        t.n = je - jb;
+    }
     return t;
 }
 
@@ -468,6 +486,48 @@ __device__ __forceinline__ float row_max(const float (&v)[N]) {
     return fmaxf(max3(m0, m1, m2), m3);
 }
 
+// Store 32 output columns [c*32, c*32+32) of query row i of head h, scaled by
+// inv: fp32 into the partial buffer of the unit's key split when there is one,
+// else rounded once to the output type.
+template <int D, bool kF32>
+__device__ __forceinline__ void store_o32(const AttnParams &p, const Unit &U, int h, int i, int c,
+                                          const float (&v)[32], float inv) {
+    if (p.part_o) {
+        const long long prow = (((long long)U.split * p.B + U.b) * p.Hq + h) * p.L + i;
+        float4 *dst = reinterpret_cast<float4 *>(p.part_o + prow * D + c * 32);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(v[4 * e] * inv, v[4 * e + 1] * inv, v[4 * e + 2] * inv,
+                                 v[4 * e + 3] * inv);
+        return;
+    }
+    const long long ob = U.b * p.os[0] + (long long)h * p.os[1] + (long long)i * p.os[2] + c * 32;
+    if (kF32) {
+        float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.o) + ob);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(v[4 * e] * inv, v[4 * e + 1] * inv, v[4 * e + 2] * inv,
+                                 v[4 * e + 3] * inv);
+    } else {
+        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.o) + ob);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pack_bf16x2(v[8 * e] * inv, v[8 * e + 1] * inv),
+                                pack_bf16x2(v[8 * e + 2] * inv, v[8 * e + 3] * inv),
+                                pack_bf16x2(v[8 * e + 4] * inv, v[8 * e + 5] * inv),
+                                pack_bf16x2(v[8 * e + 6] * inv, v[8 * e + 7] * inv));
+    }
+}
+
+// The row's log-sum-exp (natural log) into the partial buffer or the output.
+__device__ __forceinline__ void store_lse(const AttnParams &p, const Unit &U, int h, int i,
+                                          float lse) {
+    if (p.part_o)
+        p.part_lse[(((long long)U.split * p.B + U.b) * p.Hq + h) * p.L + i] = lse;
+    else if (p.lse)
+        p.lse[(U.b * (long long)p.Hq + h) * p.L + i] = lse;
+}
+
 // ---------------------------------------------------------------- kernel
 template <int D, bool kF32, bool kHalf, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -491,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const Unit U = decode_unit(p);
-    const Tiles T = make_tiles<BN>(U.q0, p);
+    const Tiles T = make_tiles<BN>(U.q0, p);   // this CTA's key tiles (its split's share)
     volatile int *abort = &bar.abort;
     const uint64_t tmo = p.timeout_ns;
 
@@ -530,6 +590,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (skip) {
         // nothing to do: fall through to the common exit
+    } else if (T.n == 0) {
+        // A key split that received no tile (more splits than tiles): the
+        // empty partial result, o = 0 and lse = -inf.
+        if (warp < 8 && (warp >> 2) < U.nt) {
+            const int h = U.hq0 + (warp >> 2), i = U.q0 + (warp & 3) * 32 + lane;
+            if (i < p.L) {
+                float z[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) z[e] = 0.f;
+                for (int c = 0; c < D / 32; ++c) store_o32<D, kF32>(p, U, h, i, c, z, 0.f);
+                store_lse(p, U, h, i, -INFINITY);
+            }
+        }
     } else if ((warp >> 2) == 3) {
         // warpgroup 3: warp 12 issues the TMA copies, warp 13 the MMAs
         setmaxnreg_dec<kRegsIssue>();
@@ -809,34 +882,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float inv = l > 0.f ? 1.f / l : 0.f;
                 const int h = U.hq0 + t;
                 const bool valid = i < p.L;
-                const long long ob = U.b * p.os[0] + (long long)h * p.os[1] + (long long)i * p.os[2];
     #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     float v[32];
                     tmem_ld32(trow + o_col + c * 32, v);
-                    if (!valid) continue;
-                    if (kF32) {
-                        float4 *dst = reinterpret_cast<float4 *>(
-                            reinterpret_cast<float *>(p.o) + ob + c * 32);
-    #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            dst[e] = make_float4(v[4 * e] * inv, v[4 * e + 1] * inv,
-                                                 v[4 * e + 2] * inv, v[4 * e + 3] * inv);
-                    } else {
-                        uint4 *dst = reinterpret_cast<uint4 *>(
-                            reinterpret_cast<__nv_bfloat16 *>(p.o) + ob + c * 32);
-    #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            dst[e] = make_uint4(pack_bf16x2(v[8 * e] * inv, v[8 * e + 1] * inv),
-                                                pack_bf16x2(v[8 * e + 2] * inv, v[8 * e + 3] * inv),
-                                                pack_bf16x2(v[8 * e + 4] * inv, v[8 * e + 5] * inv),
-                                                pack_bf16x2(v[8 * e + 6] * inv, v[8 * e + 7] * inv));
-                    }
+                    if (valid) store_o32<D, kF32>(p, U, h, i, c, v, inv);
                 }
-                if (valid && p.lse) {
+                if (valid) {
                     const float ln2 = 0.69314718055994531f;
-                    p.lse[(U.b * (long long)p.Hq + h) * p.L + i] =
-                        l > 0.f ? (m + __log2f(l)) * ln2 : -INFINITY;
+                    store_lse(p, U, h, i, l > 0.f ? (m + __log2f(l)) * ln2 : -INFINITY);
                 }
             }
         }
@@ -938,9 +992,22 @@ lcx_status check_tensor(const void *ptr, const int64_t *st, int es, const char *
 }  // namespace
 }  // namespace lcx
 
-extern "C" lcx_status lcx_attn_fwd(const lcx_attn_args *a, void *stream) {
-    using namespace lcx;
-    clear_error();
+namespace lcx {
+namespace {
+
+// Everything one attn_fwd launch needs, derived from validated arguments.
+struct AttnLaunch {
+    AttnParams p;
+    CUtensorMap mq, mk, mv;
+    long long units;  // CTAs without key splits
+    bool f32, half, split_qk;
+    int D;
+};
+
+// Validate `a` and fill `x`.  *noop is set for empty problems (B or L zero),
+// which succeed without device work.
+lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
+    *noop = false;
     if (!a) return fail(LCX_ERR_INVALID_ARG, "args is NULL");
     lcx_status st = check_rope_params(&a->rope);
     if (st != LCX_OK) return st;
@@ -976,7 +1043,10 @@ extern "C" lcx_status lcx_attn_fwd(const lcx_attn_args *a, void *stream) {
         return fail(LCX_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
     if (a->D != 64 && a->D != 128)
         return fail(LCX_ERR_UNSUPPORTED, "head_dim %lld: only 64 and 128", (long long)a->D);
-    if (a->B == 0 || a->L == 0) return LCX_OK;
+    if (a->B == 0 || a->L == 0) {
+        *noop = true;
+        return LCX_OK;
+    }
     if (a->L > (int64_t(1) << 30) || Lk > (int64_t(1) << 30) ||
         a->q_offset + a->L > (int64_t(1) << 30) || a->B > (int64_t(1) << 20) || a->Hq > 65536)
         return fail(LCX_ERR_UNSUPPORTED, "sizes too large");
@@ -986,8 +1056,8 @@ extern "C" lcx_status lcx_attn_fwd(const lcx_attn_args *a, void *stream) {
     if ((st = check_tensor(a->v, a->v_strides, es, "v")) != LCX_OK) return st;
     if ((st = check_tensor(a->o, a->o_strides, es, "o")) != LCX_OK) return st;
 
-    AttnParams p;
-    memset(&p, 0, sizeof(p));
+    memset(&x, 0, sizeof(x));
+    AttnParams &p = x.p;
     p.q = static_cast<const char *>(a->q);
     p.k = static_cast<const char *>(a->k);
     p.v = static_cast<const char *>(a->v);
@@ -1014,8 +1084,9 @@ extern "C" lcx_status lcx_attn_fwd(const lcx_attn_args *a, void *stream) {
     p.n_qb = int((a->L + kBM - 1) / kBM);
     p.heads_per_unit = (p.G % 2 == 0) ? 2 : 1;
     p.units_per_qb = p.B * p.Hq / p.heads_per_unit;
-    const long long grid = (long long)p.n_qb * p.units_per_qb;
-    if (grid > 0x7fffffffLL) return fail(LCX_ERR_UNSUPPORTED, "too many work units");
+    p.n_split = 1;
+    x.units = (long long)p.n_qb * p.units_per_qb;
+    if (x.units > 0x7fffffffLL) return fail(LCX_ERR_UNSUPPORTED, "too many work units");
     p.rotate_q = (a->flags & LCX_ATTN_PREROTATED) ? 0 : 1;
     p.rotate_k = (a->flags & (LCX_ATTN_PREROTATED | LCX_ATTN_PREROTATED_K)) ? 0 : 1;
     float ms = 1.f;
@@ -1030,26 +1101,97 @@ extern "C" lcx_status lcx_attn_fwd(const lcx_attn_args *a, void *stream) {
     p.timeout_ns = 1000000ull * (unsigned long long)(a->watchdog_ms > 0 ? a->watchdog_ms : 2000);
     p.test_stall = (a->flags & LCX_ATTN_TEST_STALL) ? 1 : 0;
 
-    const bool split = (a->flags & LCX_ATTN_SPLIT_QK) != 0;
-    const uint32_t bn = split ? 64u : 128u;
-    CUtensorMap mq, mk, mv;
-    memset(&mq, 0, sizeof(mq));
-    memset(&mk, 0, sizeof(mk));
-    memset(&mv, 0, sizeof(mv));
-    if (a->dtype == LCX_BF16) {
-        if ((st = make_map(&mq, a->q, a->B, a->Hq, a->L, a->D, a->q_strides, 128, "q")) != LCX_OK)
+    x.split_qk = (a->flags & LCX_ATTN_SPLIT_QK) != 0;
+    x.f32 = a->dtype == LCX_F32;
+    x.half = a->rope.pairing == LCX_PAIR_HALF;
+    x.D = int(a->D);
+    const uint32_t bn = x.split_qk ? 64u : 128u;
+    if (!x.f32) {
+        if ((st = make_map(&x.mq, a->q, a->B, a->Hq, a->L, a->D, a->q_strides, 128, "q")) != LCX_OK)
             return st;
-        if ((st = make_map(&mk, a->k, a->B, a->Hkv, Lk, a->D, a->k_strides, bn, "k")) != LCX_OK)
+        if ((st = make_map(&x.mk, a->k, a->B, a->Hkv, Lk, a->D, a->k_strides, bn, "k")) != LCX_OK)
             return st;
-        if ((st = make_map(&mv, a->v, a->B, a->Hkv, Lk, a->D, a->v_strides, bn, "v")) != LCX_OK)
+        if ((st = make_map(&x.mv, a->v, a->B, a->Hkv, Lk, a->D, a->v_strides, bn, "v")) != LCX_OK)
             return st;
     }
-    const bool f32 = a->dtype == LCX_F32;
-    const bool half = a->rope.pairing == LCX_PAIR_HALF;
+    return LCX_OK;
+}
+
+// Launch the attention kernel described by x (x.p.n_split CTAs per unit).
+lcx_status attn_enqueue(const AttnLaunch &x, cudaStream_t s) {
+    const long long grid = x.units * x.p.n_split;
+    if (grid > 0x7fffffffLL) return fail(LCX_ERR_UNSUPPORTED, "too many work units");
+    const unsigned g = unsigned(grid);
+    if (x.D == 128)
+        return x.split_qk ? launch_d<128, true>(x.f32, x.half, x.mq, x.mk, x.mv, x.p, g, s)
+                          : launch_d<128, false>(x.f32, x.half, x.mq, x.mk, x.mv, x.p, g, s);
+    return x.split_qk ? launch_d<64, true>(x.f32, x.half, x.mq, x.mk, x.mv, x.p, g, s)
+                      : launch_d<64, false>(x.f32, x.half, x.mq, x.mk, x.mv, x.p, g, s);
+}
+
+constexpr int kMaxKvSplits = 256;
+constexpr int64_t kMaxSplitRows = int64_t(1) << 40;  // keeps workspace sizes far from overflow
+
+// Workspace of the split path: the partial o block then the partial lse block,
+// each starting on a 256-byte boundary.
+int64_t split_o_bytes(int64_t rows, int64_t D, int64_t n) {
+    return ((n * rows * D * 4) + 255) / 256 * 256;
+}
+int64_t split_ws_bytes(int64_t rows, int64_t D, int64_t n) {
+    return split_o_bytes(rows, D, n) + ((n * rows * 4) + 255) / 256 * 256;
+}
+
+}  // namespace
+}  // namespace lcx
+
+extern "C" lcx_status lcx_attn_fwd(const lcx_attn_args *a, void *stream) {
+    using namespace lcx;
+    clear_error();
+    AttnLaunch x;
+    bool noop = false;
+    lcx_status st = attn_prepare(a, x, &noop);
+    if (st != LCX_OK || noop) return st;
+    return attn_enqueue(x, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int64_t lcx_attn_split_workspace_bytes(int64_t B, int64_t Hq, int64_t L, int64_t D,
+                                                  int32_t num_splits) {
+    if (B < 0 || Hq < 0 || L < 0 || (D != 64 && D != 128) || num_splits < 1 ||
+        num_splits > lcx::kMaxKvSplits || B > (int64_t(1) << 20) || Hq > 65536 ||
+        L > (int64_t(1) << 30) || B * Hq > (int64_t(1) << 30) ||
+        B * Hq * L > lcx::kMaxSplitRows)
+        return -1;
+    if (num_splits == 1) return 0;
+    return lcx::split_ws_bytes(B * Hq * L, D, num_splits);
+}
+
+extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_splits,
+                                         void *workspace, int64_t workspace_bytes, void *stream) {
+    using namespace lcx;
+    clear_error();
+    if (num_splits < 1 || num_splits > kMaxKvSplits)
+        return fail(LCX_ERR_INVALID_ARG, "num_splits must be in [1, %d]", kMaxKvSplits);
+    AttnLaunch x;
+    bool noop = false;
+    lcx_status st = attn_prepare(a, x, &noop);
+    if (st != LCX_OK || noop) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (a->D == 128)
-        return split ? launch_d<128, true>(f32, half, mq, mk, mv, p, unsigned(grid), s)
-                     : launch_d<128, false>(f32, half, mq, mk, mv, p, unsigned(grid), s);
-    return split ? launch_d<64, true>(f32, half, mq, mk, mv, p, unsigned(grid), s)
-                 : launch_d<64, false>(f32, half, mq, mk, mv, p, unsigned(grid), s);
+    if (num_splits == 1) return attn_enqueue(x, s);
+    const int64_t rows = a->B * a->Hq * a->L;
+    if (rows > kMaxSplitRows) return fail(LCX_ERR_UNSUPPORTED, "too many query rows to split");
+    const int64_t need = split_ws_bytes(rows, a->D, num_splits);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(LCX_ERR_INVALID_ARG, "workspace must be a 256-byte aligned device pointer");
+    if (workspace_bytes < need)
+        return fail(LCX_ERR_INVALID_ARG, "workspace holds %lld bytes; %lld needed",
+                    (long long)workspace_bytes, (long long)need);
+    float *part_o = static_cast<float *>(workspace);
+    float *part_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                                split_o_bytes(rows, a->D, num_splits));
+    x.p.n_split = num_splits;
+    x.p.part_o = part_o;
+    x.p.part_lse = part_lse;
+    if ((st = attn_enqueue(x, s)) != LCX_OK) return st;
+    return launch_merge(part_o, part_lse, num_splits, a->B, a->Hq, a->L, a->D, a->o, a->dtype,
+                        a->o_strides, a->lse, s);
 }

@@ -5,6 +5,8 @@
 #include <cstdio>
 #include <string>
 
+#include <cuda_runtime.h>
+
 #include "../../include/lcx.h"
 
 namespace lcx {
@@ -29,5 +31,12 @@ inline int64_t effective_seq_len(const lcx_rope_params *p, int64_t call_len) {
 }
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Enqueue the merge of n_parts partial results ([n_parts, B, Hq, L, D] fp32 o,
+// [n_parts, B, Hq, L] fp32 lse) into o (dtype, strides) and optionally lse.
+// Arguments are assumed valid.
+lcx_status launch_merge(const float *o_parts, const float *lse_parts, int n_parts, int64_t B,
+                        int64_t Hq, int64_t L, int64_t D, void *o, int32_t dtype,
+                        const int64_t *o_strides, float *lse_out, cudaStream_t stream);
 
 }  // namespace lcx

@@ -239,6 +239,47 @@ def test_attn_validation_without_device(lib, kw, expect):
     assert lib.lcx_last_error().decode()
 
 
+@pytest.mark.parametrize("splits,ws,nbytes", [
+    (0, 0x10000000, 1 << 30),        # num_splits out of range
+    (257, 0x10000000, 1 << 30),
+    (4, 0, 1 << 30),                 # NULL workspace
+    (4, 0x10000010, 1 << 30),        # not 256-byte aligned
+    (4, 0x10000000, 1000),           # too small
+])
+def test_attn_split_validation_without_device(lib, splits, ws, nbytes):
+    """fp32 operands (no tensor maps are built), so every case stops at the
+    split arguments, before any device work."""
+    a = _attn_args(dtype=1, q_strides=[8 * 256 * 128, 256 * 128, 128, 1],
+                   o_strides=[8 * 256 * 128, 256 * 128, 128, 1])
+    assert lib.lcx_attn_fwd_split(ctypes.byref(a), splits, ws, nbytes, None) == \
+        lcx.LCX_ERR_INVALID_ARG
+    assert lib.lcx_last_error().decode()
+
+
+def test_split_workspace_bytes(lib):
+    f = lib.lcx_attn_split_workspace_bytes
+    assert f(1, 32, 1, 128, 1) == 0
+    assert f(1, 32, 1, 128, 16) == 16 * 32 * 128 * 4 + 2048
+    assert f(2, 3, 5, 64, 3) == -(-(3 * 30 * 64 * 4) // 256) * 256 + 512
+    for bad in ((1, 32, 1, 96, 4), (1, 32, 1, 128, 0), (1, 32, 1, 128, 257), (-1, 1, 1, 64, 2),
+                (1 << 20, 65536, 1 << 30, 128, 2)):
+        assert f(*bad) == -1
+
+
+def test_merge_validation_without_device(lib):
+    st = (ctypes.c_int64 * 4)(4 * 8 * 128, 8 * 128, 128, 1)
+    m = lib.lcx_attn_merge
+    F = 0x10000000
+    assert m(F, F, 0, 1, 4, 8, 128, F, 0, st, None, None) == lcx.LCX_ERR_INVALID_ARG
+    assert m(F, F, 2, 1, 4, 8, 96, F, 0, st, None, None) == lcx.LCX_ERR_UNSUPPORTED
+    assert m(F, F, 2, 1, 4, 8, 128, F, 7, st, None, None) == lcx.LCX_ERR_INVALID_ARG
+    assert m(0, F, 2, 1, 4, 8, 128, F, 0, st, None, None) == lcx.LCX_ERR_INVALID_ARG
+    assert m(F + 4, F, 2, 1, 4, 8, 128, F, 0, st, None, None) == lcx.LCX_ERR_UNSUPPORTED
+    bad = (ctypes.c_int64 * 4)(4 * 8 * 128, 8 * 128, 132, 1)
+    assert m(F, F, 2, 1, 4, 8, 128, F, 0, bad, None, None) == lcx.LCX_ERR_UNSUPPORTED
+    assert m(0, 0, 2, 0, 4, 8, 128, 0, 0, st, None, None) == lcx.LCX_OK   # empty: no-op
+
+
 def test_attn_empty_is_noop(lib):
     a = _attn_args(L=0, q=0, k=0, v=0, o=0)
     assert lib.lcx_attn_fwd(ctypes.byref(a), None) == lcx.LCX_OK

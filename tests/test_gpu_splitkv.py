@@ -1,0 +1,114 @@
+"""GPU parity of split-KV attention (lcx_attn_fwd_split) and the (O, LSE) merge
+(lcx_attn_merge) against the fp64 oracle ("8.3 长上下文技术", 8.3.4 online
+softmax and 8.3.5 step 3: partial results over disjoint key sets combined by
+their softmax statistics).
+
+Split-KV must give the unsplit result up to rounding, for any split count
+(including more splits than a query block has key tiles, which leaves empty
+splits), so every case is checked against the oracle with the prefill
+tolerances; the merge kernel is checked against the oracle's merge.
+"""
+import numpy as np
+import pytest
+import torch
+
+import ntk_rope_flashattn_b200 as lcx
+import oracle
+from test_gpu_attn import compare
+from test_gpu_decode import W0, oracle_rows, rope_of
+from workloads import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def run_split(q, k, v, rope, num_splits, **kw):
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = lcx.attn_fwd(q, k, v, rope, return_lse=True, status=status, num_splits=num_splits,
+                          **kw)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return o, lse
+
+
+@pytest.mark.parametrize("L,Lk,splits,extra", [
+    (1, 777, 3, {}),
+    (1, 777, 16, {}),                        # more splits than the 7 key tiles
+    (4, 5000, 8, dict(window=1000, sinks=4)),
+    (1, 4096, 32, dict(Hq=8, Hkv=2)),
+    (2, 900, 5, dict(split_qk=True, window=300, sinks=2)),
+    (3, 640, 4, dict(dtype="f32", mode="pi", scale=2.0)),
+    (1, 500, 7, dict(D=64, pairing="interleaved")),
+])
+def test_splitkv_decode(L, Lk, splits, extra):
+    w = W0.with_(**extra, L=Lk)
+    q_all, k, v = make_inputs(w, device="cuda")
+    q = q_all[:, :, Lk - L:]
+    rope = rope_of(w)
+    o, lse = run_split(q, k, v, rope, splits, window=w.window, sinks=w.sinks, q_offset=Lk - L,
+                       split_qk=w.split_qk)
+    ref = oracle_rows(q, k, v, rope, Lk - L, True, w.window, w.sinks)
+    compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref[0], ref[1],
+            24 if w.dtype == "f32" else 8)
+
+
+@pytest.mark.parametrize("splits", [2, 5])
+def test_splitkv_prefill(splits):
+    """Prefill with split keys: causal rows of every length, window and sinks."""
+    w = W0.with_(L=700, window=250, sinks=3)
+    q, k, v = make_inputs(w, device="cuda")
+    rope = rope_of(w)
+    o, lse = run_split(q, k, v, rope, splits, window=w.window, sinks=w.sinks)
+    ref = oracle_rows(q, k, v, rope, 0, True, w.window, w.sinks)
+    compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref[0], ref[1])
+    o1, _ = run_split(q, k, v, rope, 1, window=w.window, sinks=w.sinks)
+    assert (o.float() - o1.float()).abs().max().item() <= 2e-2
+
+
+def test_splitkv_deterministic_and_workspace_reuse():
+    w = W0.with_(L=3000)
+    q_all, k, v = make_inputs(w, device="cuda")
+    q = q_all[:, :, -2:]
+    rope = rope_of(w)
+    ws = torch.empty(lcx.split_workspace_bytes(1, w.Hq, 2, w.D, 6), dtype=torch.uint8,
+                     device="cuda")
+    a = lcx.attn_fwd(q, k, v, rope, q_offset=2998, num_splits=6, workspace=ws)
+    ws.fill_(0xFF)                            # stale contents must not matter
+    b = lcx.attn_fwd(q, k, v, rope, q_offset=2998, num_splits=6, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_splitkv_long_cache_sampled():
+    """One new token per head against the 131072-key cache of the YaRN s=16
+    workload, 16 splits."""
+    w = WORKLOADS["yarn_L131072_s16"]
+    q_all, k, v = make_inputs(w, device="cuda")
+    q = q_all[:, :, -1:].contiguous()
+    del q_all
+    rope = rope_of(w)
+    o, lse = run_split(q, k, v, rope, 16, q_offset=w.L - 1)
+    ref = oracle_rows(q, k, v, rope, w.L - 1)
+    compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref[0], ref[1])
+
+
+@pytest.mark.parametrize("D,dtype", [(128, torch.bfloat16), (64, torch.float32)])
+def test_merge_matches_oracle(D, dtype):
+    n, B, Hq, L = 5, 2, 3, 37
+    g = torch.Generator(device="cuda").manual_seed(7)
+    o_parts = torch.randn((n, B, Hq, L, D), generator=g, device="cuda")
+    lse_parts = 3.0 * torch.randn((n, B, Hq, L), generator=g, device="cuda")
+    lse_parts[1, 0, 0, :5] = -float("inf")        # empty parts
+    lse_parts[:, 1, 2, 7] = -float("inf")         # a row with no key at all
+    base = torch.empty((B, L, Hq, D + 8), dtype=dtype, device="cuda")
+    out = base[..., :D].permute(0, 2, 1, 3)      # strided output [B, Hq, L, D]
+    o, lse = lcx.attn_merge(o_parts, lse_parts, out=out)
+    torch.cuda.synchronize()
+    ref_o, ref_lse = oracle.merge(o_parts.double().cpu().numpy(), lse_parts.double().cpu().numpy())
+    got = o.float().cpu().numpy()
+    bits = 8 if dtype == torch.bfloat16 else 24
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref_o), 1e-30))) - bits)
+    assert (np.abs(got - ref_o) <= 1e-5 + ulp).all()
+    lse_np = lse.cpu().numpy()
+    finite = np.isfinite(ref_lse)
+    assert np.isneginf(lse_np[~finite]).all() and (got[~finite] == 0).all()
+    assert np.abs(lse_np[finite] - ref_lse[finite]).max() <= 1e-5
