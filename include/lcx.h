@@ -263,6 +263,35 @@ LCX_API lcx_status lcx_attn_merge(const float *o_parts, const float *lse_parts, 
                                   int32_t dtype, const int64_t *o_strides, float *lse,
                                   void *stream);
 
+/* Size of the static device scratch of lcx_attn_fwd_split_static (32 MiB). */
+#define LCX_STATIC_SCRATCH_BYTES (32 * 1024 * 1024)
+
+/*
+ * lcx_attn_fwd_split_static -- lcx_attn_fwd_split with the library's own
+ * static device scratch in place of a caller workspace: the call allocates
+ * nothing (no cudaMalloc, no caller buffer besides the tensors of `args`).
+ * The pages describe no counterpart of this call; it exists for callers that
+ * have no device allocator at hand.
+ *   Scratch : one static __device__ array of LCX_STATIC_SCRATCH_BYTES per
+ *             device (256-byte aligned), resolved with cudaGetSymbolAddress
+ *             on the first call on each device (a checked call; failure is
+ *             LCX_ERR_CUDA; under lazy module loading the CUDA runtime also
+ *             materialises the array at that point).  Make that first call
+ *             before capturing the stream into a graph; later calls allocate
+ *             nothing.  Nothing in it must start at zero (every partial
+ *             row the merge reads is written earlier in the same call), so it
+ *             is never cleared.
+ *   Limit   : requests whose lcx_attn_split_workspace_bytes exceeds
+ *             LCX_STATIC_SCRATCH_BYTES return LCX_ERR_UNSUPPORTED before any
+ *             device work.
+ *   Races   : every call on a device shares the one array, so two calls whose
+ *             executions overlap (different streams, or threads without
+ *             ordering) corrupt each other's partial results; order them.
+ *   Otherwise as lcx_attn_fwd_split (num_splits 1..256; 1 uses no scratch).
+ */
+LCX_API lcx_status lcx_attn_fwd_split_static(const lcx_attn_args *args, int32_t num_splits,
+                                             void *stream);
+
 /* Static description of a status code. */
 LCX_API const char *lcx_status_string(lcx_status status);
 

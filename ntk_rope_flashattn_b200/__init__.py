@@ -31,7 +31,8 @@ LCX_ATTN_TEST_STALL = 0x80000000
 
 # Symbols include/lcx.h declares; the library must export every one of them.
 EXPORTED = ("lcx_rope_table", "lcx_apply_rope", "lcx_attn_fwd", "lcx_attn_fwd_split",
-            "lcx_attn_split_workspace_bytes", "lcx_attn_merge", "lcx_status_string",
+            "lcx_attn_split_workspace_bytes", "lcx_attn_merge", "lcx_attn_fwd_split_static",
+            "lcx_status_string",
             "lcx_last_error", "lcx_version")
 
 
@@ -135,6 +136,9 @@ def load(path: str = LIB_PATH):
     lib.lcx_attn_fwd_split.argtypes = [ctypes.POINTER(_AttnArgs), ctypes.c_int32, ctypes.c_void_p,
                                        ctypes.c_int64, ctypes.c_void_p]
     lib.lcx_attn_fwd_split.restype = ctypes.c_int
+    lib.lcx_attn_fwd_split_static.argtypes = [ctypes.POINTER(_AttnArgs), ctypes.c_int32,
+                                              ctypes.c_void_p]
+    lib.lcx_attn_fwd_split_static.restype = ctypes.c_int
     lib.lcx_attn_split_workspace_bytes.argtypes = [ctypes.c_int64] * 4 + [ctypes.c_int32]
     lib.lcx_attn_split_workspace_bytes.restype = ctypes.c_int64
     lib.lcx_attn_merge.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
@@ -274,6 +278,43 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
                                          _stream(q)))
     del rope_c
     return (o, lse) if return_lse else o
+
+
+def attn_fwd_split_static(q, k, v, rope: RopeParams, num_splits: int, causal: bool = True,
+                          window: int = 0, sinks: int = 0, softmax_scale: float = 0.0,
+                          q_offset: int = 0, out=None, lse=None, status=None):
+    """Split-KV attention through lcx_attn_fwd_split_static: the partial results
+    live in the library's static device scratch (LCX_STATIC_SCRATCH_BYTES per
+    device), so nothing is allocated for them.  Calls on one device must not
+    overlap in time (they share the scratch).  q [B, Hq, L, D], k/v
+    [B, Hkv, Lk, D]; returns o (and fills ``lse`` when given)."""
+    import torch
+    B, Hq, L, D = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    if k.shape != (B, Hkv, Lk, D) or v.shape != k.shape or not (q.dtype == k.dtype == v.dtype):
+        raise ValueError("shape / dtype mismatch: q %s k %s v %s" % (q.shape, k.shape, v.shape))
+    o = out if out is not None else torch.empty_like(q)
+    a = _AttnArgs()
+    a.q, a.k, a.v, a.o = q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr()
+    a.lse = lse.data_ptr() if lse is not None else None
+    a.dev_status = status.data_ptr() if status is not None else None
+    a.dtype = _dtype_code(q)
+    a.causal = 1 if causal else 0
+    a.B, a.Hq, a.Hkv, a.L, a.D = B, Hq, Hkv, L, D
+    a.q_strides, a.k_strides, a.v_strides, a.o_strides = (_strides(q), _strides(k),
+                                                          _strides(v), _strides(o))
+    rope_c = rope._c()
+    a.rope = rope_c
+    a.window, a.sinks = int(window), int(sinks)
+    a.softmax_scale = float(softmax_scale)
+    a.flags = 0
+    a.watchdog_ms = 0
+    a.reserved0 = 0
+    a.Lk = Lk
+    a.q_offset = int(q_offset)
+    _check(load().lcx_attn_fwd_split_static(ctypes.byref(a), int(num_splits), _stream(q)))
+    del rope_c
+    return o
 
 
 def split_workspace_bytes(B, Hq, L, D, num_splits):

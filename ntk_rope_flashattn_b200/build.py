@@ -17,7 +17,7 @@ BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "liblcx.so")
 INCLUDE = os.path.join(ROOT, "include")
 
-SOURCES = ["lcx_table.cpp", "apply_rope.cu", "attn_fwd.cu", "merge.cu"]
+SOURCES = ["lcx_table.cpp", "apply_rope.cu", "attn_fwd.cu", "merge.cu", "static_scratch.cu"]
 HEADERS = ["lcx_internal.h", "sm100.cuh", "rope_angle.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
