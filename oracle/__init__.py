@@ -61,6 +61,11 @@ def _load():
                                            lib.orc_attn_rows.argtypes[19:])
         lib.orc_merge.argtypes = [f64p, f64p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                   f64p, f64p]
+        lib.orc_attn_rows_mla.argtypes = [f32p, i64p, i64p, i64p, ctypes.c_int64, f32p, f32p,
+                                          f32p] + [ctypes.c_int64] * 7 + [
+                                          f32p, ctypes.c_float, ctypes.c_int, ctypes.c_int64,
+                                          ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
+                                          ctypes.c_double, f64p, f64p, ctypes.c_int]
         lib.orc_num_threads.argtypes = [ctypes.c_int]
         _lib = lib
     return _lib
@@ -235,4 +240,41 @@ def merge(o_parts, lse_parts):
                            n, rows, D, _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double))
     if rc:
         raise ValueError("orc_merge: invalid argument (rc=%d)" % rc)
+    return o, lse
+
+
+def attn_rows_mla(q_rows, row_b, row_h, row_i, kc, kr, v, Hq, table, mscale, pairing="half",
+                  pos_offset=0, causal=True, window=0, sinks=0, scale=None, nthreads=0):
+    """Decoupled-RoPE attention (see orc_attn_rows_mla) for selected query rows.
+
+    q_rows [n, Dc + Dr]; kc [B, Hkv, L, Dc] (Dc may be 0); kr [B, L, Dr] shared by
+    all heads; v [B, Hkv, L, Dv]; table of a Dr-dim RoPE.  Default scale
+    1/sqrt(Dc + Dr).  Returns o [n, Dv], lse [n] in fp64.
+    """
+    q_rows = np.ascontiguousarray(q_rows, dtype=np.float32)
+    kc = np.ascontiguousarray(kc, dtype=np.float32)
+    kr = np.ascontiguousarray(kr, dtype=np.float32)
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    B, Hkv, L, Dc = kc.shape
+    Dr, Dv = kr.shape[2], v.shape[3]
+    assert kr.shape == (B, L, Dr) and v.shape[:3] == (B, Hkv, L)
+    n = q_rows.shape[0]
+    assert q_rows.shape == (n, Dc + Dr)
+    if scale is None:
+        scale = 1.0 / np.sqrt(Dc + Dr)
+    row_b, row_h, row_i = (np.ascontiguousarray(x, dtype=np.int64) for x in (row_b, row_h, row_i))
+    table = np.ascontiguousarray(table, dtype=np.float32)
+    o = np.zeros((n, Dv), dtype=np.float64)
+    lse = np.zeros(n, dtype=np.float64)
+    kc_p = kc if kc.size else np.zeros(1, np.float32)
+    rc = _load().orc_attn_rows_mla(_ptr(q_rows, ctypes.c_float), _ptr(row_b, ctypes.c_int64),
+                                   _ptr(row_h, ctypes.c_int64), _ptr(row_i, ctypes.c_int64), n,
+                                   _ptr(kc_p, ctypes.c_float), _ptr(kr, ctypes.c_float),
+                                   _ptr(v, ctypes.c_float), B, Hq, Hkv, L, Dc, Dr, Dv,
+                                   _ptr(table, ctypes.c_float), float(mscale), PAIRINGS[pairing],
+                                   int(pos_offset), int(causal), int(window), int(sinks),
+                                   float(scale), _ptr(o, ctypes.c_double),
+                                   _ptr(lse, ctypes.c_double), int(nthreads))
+    if rc:
+        raise ValueError("orc_attn_rows_mla: invalid argument (rc=%d)" % rc)
     return o, lse

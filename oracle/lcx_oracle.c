@@ -496,5 +496,103 @@ int orc_merge(const double *o_parts, const double *lse_parts, int64_t n_parts, i
     return 0;
 }
 
+/* ------------------------------------------------------------------------ */
+/* decoupled RoPE ("Long Context: RoPE / YaRN / NTK / MLA", 9.5 and 9.7):     */
+/* a query is [q_C ; q_R], the key of head h is [k_C^(h) ; k_R] with one      */
+/* rotary key k_R shared by all heads, only the d_R-dim parts are rotated    */
+/* (RoPE of dimension d_R, mscale on the rotated parts as cos/sin carry it), */
+/* scores use 1/sqrt(d_C + d_R) unless a scale is given, values are v^(h).   */
+
+typedef struct {
+    const float *q;          /* [nrows, Dc + Dr] raw query rows */
+    const int64_t *row_b, *row_h, *row_i;
+    const float *kc;         /* [B, Hkv, L, Dc] */
+    const double *krr;       /* [B, L, Dr] rotated shared rope keys */
+    const float *v;          /* [B, Hkv, L, Dv] */
+    int64_t B, Hq, Hkv, L, Dc, Dr, Dv;
+    int64_t pos_offset;
+    const float *table;
+    double ms;
+    int pairing, causal;
+    int64_t window, sinks;
+    double scale;
+    double *o, *lse;
+} mla_ctx;
+
+static void mla_row(void *vctx, int64_t r)
+{
+    mla_ctx *c = (mla_ctx *)vctx;
+    const int64_t b = c->row_b[r], h = c->row_h[r], i = c->row_i[r];
+    const int64_t g = h / (c->Hq / c->Hkv), Dq = c->Dc + c->Dr, L = c->L;
+    double xr[4096], qr[4096];
+    for (int64_t d = 0; d < c->Dr; d++) xr[d] = (double)c->q[r * Dq + c->Dc + d];
+    rotate_row(xr, qr, (int)c->Dr, c->pos_offset + i, c->table, c->ms, c->pairing);
+    double *s = (double *)malloc(sizeof(double) * (size_t)L);
+    double mx = -INFINITY;
+    for (int64_t j = 0; j < L; j++) {
+        if (!orc_visible(i, j, L, c->causal, c->window, c->sinks)) { s[j] = -INFINITY; continue; }
+        const float *kc = c->kc + (((b * c->Hkv) + g) * L + j) * c->Dc;
+        const double *kr = c->krr + (b * L + j) * c->Dr;
+        double dot = 0.0;
+        for (int64_t d = 0; d < c->Dc; d++) dot += (double)c->q[r * Dq + d] * (double)kc[d];
+        for (int64_t d = 0; d < c->Dr; d++) dot += qr[d] * kr[d];
+        s[j] = c->scale * dot;
+        if (s[j] > mx) mx = s[j];
+    }
+    double *o = c->o + r * c->Dv;
+    for (int64_t d = 0; d < c->Dv; d++) o[d] = 0.0;
+    if (mx == -INFINITY) { c->lse[r] = -INFINITY; free(s); return; }
+    double Z = 0.0;
+    for (int64_t j = 0; j < L; j++) {
+        if (s[j] == -INFINITY) continue;
+        double p = exp(s[j] - mx);
+        Z += p;
+        const float *vj = c->v + (((b * c->Hkv) + g) * L + j) * c->Dv;
+        for (int64_t d = 0; d < c->Dv; d++) o[d] += p * (double)vj[d];
+    }
+    for (int64_t d = 0; d < c->Dv; d++) o[d] /= Z;
+    c->lse[r] = mx + log(Z);
+    free(s);
+}
+
+/*
+ * Attention rows with decoupled RoPE.
+ *   q  : [nrows, Dc + Dr] raw query rows ([q_C ; q_R])
+ *   kc : [B, Hkv, L, Dc] per-head non-rotary keys (Dc may be 0)
+ *   kr : [B, L, Dr] raw rotary keys shared by every head
+ *   v  : [B, Hkv, L, Dv]
+ *   table, mscale, pairing : a RoPE table of dimension Dr
+ *   scale : score scale (the caller passes 1/sqrt(Dc + Dr) for the default)
+ * Other arguments as orc_attn_rows.  Outputs o [nrows, Dv], lse [nrows].
+ */
+int orc_attn_rows_mla(const float *q, const int64_t *row_b, const int64_t *row_h,
+                      const int64_t *row_i, int64_t nrows, const float *kc, const float *kr,
+                      const float *v, int64_t B, int64_t Hq, int64_t Hkv, int64_t L,
+                      int64_t Dc, int64_t Dr, int64_t Dv, const float *table, float mscale,
+                      int pairing, int64_t pos_offset, int causal, int64_t window,
+                      int64_t sinks, double scale, double *o, double *lse, int nthreads)
+{
+    if (Dc < 0 || Dr <= 0 || (Dr % 2) != 0 || Dv <= 0 || Dc + Dr > 4096 || Dr > 4096) return 1;
+    if (Hkv <= 0 || Hq <= 0 || (Hq % Hkv) != 0 || L <= 0 || B <= 0) return 1;
+    if (!causal && (window != 0 || sinks != 0)) return 1;
+    if (window < 0 || sinks < 0) return 1;
+    for (int64_t r = 0; r < nrows; r++)
+        if (row_b[r] < 0 || row_b[r] >= B || row_h[r] < 0 || row_h[r] >= Hq ||
+            row_i[r] < 0 || row_i[r] >= L) return 1;
+    double *krr = (double *)malloc(sizeof(double) * (size_t)(B * L * Dr));
+    if (!krr) return 2;
+    double xr[4096];
+    for (int64_t t = 0; t < B * L; t++) {
+        for (int64_t d = 0; d < Dr; d++) xr[d] = (double)kr[t * Dr + d];
+        rotate_row(xr, krr + t * Dr, (int)Dr, pos_offset + t % L, table, (double)mscale,
+                   pairing);
+    }
+    mla_ctx c = {q, row_b, row_h, row_i, kc, krr, v, B, Hq, Hkv, L, Dc, Dr, Dv, pos_offset,
+                 table, (double)mscale, pairing, causal, window, sinks, scale, o, lse};
+    orc_parallel_for(nrows, nthreads, mla_row, &c);
+    free(krr);
+    return 0;
+}
+
 /* Number of threads orc_attn_rows uses for a given request (0 = all cores). */
 int orc_num_threads(int nthreads) { return orc_threads(nthreads); }

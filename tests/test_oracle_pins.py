@@ -632,3 +632,73 @@ def test_merge_closed_forms():
     ob, lb = oracle.merge(np.stack([o2, o1]), np.stack([l1 - 1, l1]))
     np.testing.assert_allclose(oa, ob, atol=1e-15)
     np.testing.assert_allclose(la, lb, atol=1e-15)
+
+
+# --------------------------------------------------------------------------
+# Decoupled RoPE ("Long Context: RoPE / YaRN / NTK / MLA", 9.5 and 9.7; A.1):
+# q = [q_C ; RoPE(q_R)], k^(h) = [k_C^(h) ; RoPE(k_R)] with k_R shared by all
+# heads, scores scaled by 1/sqrt(d_C + d_R).
+
+def _mla_inputs(B, Hq, Hkv, L, Dc, Dr, Dv, seed):
+    return (_rand((B, Hq, L, Dc + Dr), seed), _rand((B, Hkv, L, Dc), seed + 1),
+            _rand((B, L, Dr), seed + 2), _rand((B, Hkv, L, Dv), seed + 3))
+
+
+def _all_rows(B, Hq, L):
+    bb, hh, ii = np.meshgrid(np.arange(B), np.arange(Hq), np.arange(L), indexing="ij")
+    return bb.ravel(), hh.ravel(), ii.ravel()
+
+
+def test_mla_without_nope_part_is_shared_key_attention():
+    """With d_C = 0 every head attends with the one shared rotary key: the
+    standard oracle with a single kv head (GQA over all heads)."""
+    B, Hq, L, Dr = 1, 4, 33, 32
+    table, ms, _ = oracle.rope_table("yarn", Dr, scale=4.0, original_max_pos=8)
+    q, kc, kr, v = _mla_inputs(B, Hq, 1, L, 0, Dr, Dr, 60)
+    bb, hh, ii = _all_rows(B, Hq, L)
+    o, lse = oracle.attn_rows_mla(q.reshape(-1, Dr), bb, hh, ii, kc, kr, v, Hq, table, ms,
+                                  window=9, sinks=2)
+    ref_o, ref_l = oracle.attn_full(q, kr[:, None], v, table, ms, window=9, sinks=2)
+    np.testing.assert_allclose(o.reshape(B, Hq, L, Dr), ref_o, atol=1e-12, rtol=0)
+    np.testing.assert_allclose(lse.reshape(B, Hq, L), ref_l, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("pairing", ["half", "interleaved"])
+def test_mla_matches_torch_sdpa_on_concatenated_vectors(pairing):
+    """Reduction to a library routine: torch's fp64 scaled_dot_product_attention
+    on explicitly concatenated [q_C ; rotated q_R] and [k_C ; rotated k_R] (the
+    rotation pinned above, mscale on the rotated parts), value dim d_v != d_qk."""
+    B, Hq, Hkv, L, Dc, Dr, Dv = 2, 4, 4, 29, 48, 16, 24
+    table, ms, _ = oracle.rope_table("yarn", Dr, scale=8.0, original_max_pos=4)
+    assert ms > 1.0
+    q, kc, kr, v = _mla_inputs(B, Hq, Hkv, L, Dc, Dr, Dv, 61)
+    bb, hh, ii = _all_rows(B, Hq, L)
+    o, lse = oracle.attn_rows_mla(q.reshape(-1, Dc + Dr), bb, hh, ii, kc, kr, v, Hq, table, ms,
+                                  pairing, causal=True, window=11, sinks=3)
+    qr = oracle.rotate_rows(q[..., Dc:].reshape(-1, Dr), np.tile(np.arange(L), B * Hq), table,
+                            ms, pairing).reshape(B, Hq, L, Dr)
+    krr = oracle.rotate_rows(kr.reshape(-1, Dr), np.tile(np.arange(L), B), table, ms,
+                             pairing).reshape(B, 1, L, Dr)
+    qcat = torch.from_numpy(np.concatenate([q[..., :Dc].astype(np.float64), qr], axis=-1))
+    kcat = torch.from_numpy(np.concatenate([kc.astype(np.float64),
+                                            np.repeat(krr, Hkv, axis=1)], axis=-1))
+    m = torch.from_numpy(oracle.mask(L, True, 11, 3))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        qcat, kcat, torch.from_numpy(v.astype(np.float64)), attn_mask=m,
+        scale=1.0 / math.sqrt(Dc + Dr))
+    np.testing.assert_allclose(o.reshape(B, Hq, L, Dv), ref.numpy(), atol=1e-12, rtol=0)
+    logits = (qcat @ kcat.transpose(-1, -2)) / math.sqrt(Dc + Dr)
+    ref_l = torch.logsumexp(logits.masked_fill(~m, float("-inf")), dim=-1)
+    np.testing.assert_allclose(lse.reshape(B, Hq, L), ref_l.numpy(), atol=1e-12, rtol=0)
+
+
+def test_mla_relative_positions_only():
+    B, Hq, L, Dc, Dr = 1, 2, 20, 32, 32
+    table, ms, _ = oracle.rope_table("ntk", Dr, scale=4.0)
+    q, kc, kr, v = _mla_inputs(B, Hq, Hq, L, Dc, Dr, 32, 62)
+    bb, hh, ii = _all_rows(B, Hq, L)
+    a = oracle.attn_rows_mla(q.reshape(-1, Dc + Dr), bb, hh, ii, kc, kr, v, Hq, table, ms)
+    b = oracle.attn_rows_mla(q.reshape(-1, Dc + Dr), bb, hh, ii, kc, kr, v, Hq, table, ms,
+                             pos_offset=77777)
+    np.testing.assert_allclose(a[0], b[0], atol=1e-9)
+    np.testing.assert_allclose(a[1], b[1], atol=1e-9)
