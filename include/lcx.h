@@ -158,18 +158,19 @@ LCX_API lcx_status lcx_apply_rope(const lcx_rope_params *params, const void *x, 
 
 typedef struct {
     const void *q;             /* DEVICE [B, Hq, L, D]                            */
-    const void *k;             /* DEVICE [B, Hkv, Lk, D]                          */
-    const void *v;             /* DEVICE [B, Hkv, Lk, D]                          */
-    void *o;                   /* DEVICE [B, Hq, L, D], same dtype as q           */
+    const void *k;             /* DEVICE [B, Hkv, Lk, D] ([.., D - d_R] with k_rope) */
+    const void *v;             /* DEVICE [B, Hkv, Lk, Dv]                         */
+    void *o;                   /* DEVICE [B, Hq, L, Dv], same dtype as q          */
     float *lse;                /* DEVICE [B, Hq, L] fp32 natural-log sum-exp of the
                                   scaled logits, or NULL                          */
     int32_t *dev_status;       /* DEVICE int32 or NULL: set to LCX_ERR_TIMEOUT by a
                                   kernel whose bounded wait expired; never cleared */
     int32_t dtype;             /* lcx_dtype of q, k, v, o                         */
     int32_t causal;            /* 1 = key j visible to query i only if j <= i    */
-    int64_t B, Hq, Hkv, L, D;  /* Hq % Hkv == 0; D in {64, 128}                   */
+    int64_t B, Hq, Hkv, L, D;  /* Hq % Hkv == 0; D = query/key head dim           */
     int64_t q_strides[4], k_strides[4], v_strides[4], o_strides[4];  /* elements  */
-    lcx_rope_params rope;      /* head_dim must equal D                           */
+    lcx_rope_params rope;      /* head_dim = D (every dim rotated) or, partial
+                                  rotary, the number of LAST dims rotated      */
     int64_t window;            /* W > 0: key j visible only if i - j < W (W counts
                                   the query itself); 0 = no window.  Needs causal */
     int64_t sinks;             /* S: keys j < S stay visible to every i >= j when
@@ -186,6 +187,12 @@ typedef struct {
                                   (decode: Lk - L).  With causal masking
                                   q_offset + L <= Lk (every query sees its own
                                   key); 0 for plain prefill                      */
+    int64_t Dv;                /* value / output head dim; 0 -> D                 */
+    const void *k_rope;        /* DEVICE [B, 1, Lk, rope.head_dim] or NULL: the
+                                  rotary key part shared by every head (decoupled
+                                  RoPE).  When set, k holds only the first
+                                  D - rope.head_dim columns of each key       */
+    int64_t k_rope_strides[4]; /* elements; the head stride is not used        */
 } lcx_attn_args;
 
 /*
@@ -204,11 +211,18 @@ typedef struct {
  *   order, so every key is re-rotated on chip at its logical position (its
  *   index in the cache) on every call.  Rows with no visible key get o = 0 and
  *   lse = -inf.
+ *   Decoupled RoPE ([LC] 9.5, 9.7, A.1): with rope.head_dim = d_R < D only the
+ *   last d_R dims of q and k are rotated (by a d_R-dim RoPE; mscale multiplies
+ *   the rotated parts only, as the scaled cos/sin do), the first D - d_R are
+ *   used as they are, and the default scale 1/sqrt(D) is 1/sqrt(d_h + d_R).
+ *   k_rope supplies the rotated key part once for all heads.
  *   Arithmetic: q', k' rounded to bf16 on chip, QK^T and PV on bf16 tensor
  *   cores with fp32 accumulation, softmax statistics in fp32, o rounded once
  *   to the output dtype.  fp32 inputs are rounded to bf16 operands.
- *   Supported: D in {64, 128}; bf16 or fp32; pointers 16-byte aligned, strides
- *   multiples of 16 bytes, D's stride 1.  Enqueued on `stream`.
+ *   Supported (D, Dv, rope.head_dim): (64, 64, 64), (128, 128, 128) with bf16
+ *   or fp32 and either QK^T mode; (128, 128, 64) and (192, 128, 64) with bf16
+ *   and plain QK^T.  Pointers 16-byte aligned, strides multiples of 16 bytes,
+ *   D's stride 1.  Enqueued on `stream`.
  */
 LCX_API lcx_status lcx_attn_fwd(const lcx_attn_args *args, void *stream);
 
@@ -236,7 +250,8 @@ LCX_API lcx_status lcx_attn_fwd_split(const lcx_attn_args *args, int32_t num_spl
                                       void *workspace, int64_t workspace_bytes, void *stream);
 
 /* Workspace bytes lcx_attn_fwd_split needs: [num_splits, B, Hq, L, D] fp32
- * partial outputs then [num_splits, B, Hq, L] fp32 partial LSEs, each block
+ * partial outputs (D here: the output head dim, args.Dv or args.D when Dv is
+ * 0) then [num_splits, B, Hq, L] fp32 partial LSEs, each block
  * rounded up to 256 bytes.  0 when num_splits == 1; -1 for invalid sizes
  * (D not 64/128, num_splits outside 1..256, or more than 2^40 query rows). */
 LCX_API int64_t lcx_attn_split_workspace_bytes(int64_t B, int64_t Hq, int64_t L, int64_t D,

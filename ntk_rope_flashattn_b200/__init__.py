@@ -66,7 +66,8 @@ class _AttnArgs(ctypes.Structure):
                 ("rope", _RopeParams), ("window", ctypes.c_int64), ("sinks", ctypes.c_int64),
                 ("softmax_scale", ctypes.c_float), ("flags", ctypes.c_uint32),
                 ("watchdog_ms", ctypes.c_int32), ("reserved0", ctypes.c_int32),
-                ("Lk", ctypes.c_int64), ("q_offset", ctypes.c_int64)]
+                ("Lk", ctypes.c_int64), ("q_offset", ctypes.c_int64), ("Dv", ctypes.c_int64),
+                ("k_rope", ctypes.c_void_p), ("k_rope_strides", ctypes.c_int64 * 4)]
 
 
 @dataclass
@@ -215,7 +216,7 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
              softmax_scale: float = 0.0, return_lse: bool = False, prerotated: bool = False,
              split_qk: bool = False, out=None, lse=None, status=None, watchdog_ms: int = 0,
              q_offset: int = 0, k_prerotated: bool = False, num_splits: int = 1,
-             workspace=None, _test_stall: bool = False):
+             workspace=None, k_rope=None, _test_stall: bool = False):
     """Fused RoPE + causal attention (prefill, chunked prefill, decode).
 
     q [B, Hq, L, D], k/v [B, Hkv, Lk, D] CUDA tensors (bf16 or fp32, last dim
@@ -228,6 +229,10 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
     ``num_splits`` > 1 runs split-KV (lcx_attn_fwd_split): each query block's
     key tiles are shared among that many CTAs and the partial results merged;
     ``workspace`` (uint8 CUDA tensor) is allocated when not given.
+    Decoupled RoPE: ``rope.head_dim`` < D rotates only the last
+    rope.head_dim dims of q and k; ``k_rope`` [B, 1, Lk, rope.head_dim] then
+    supplies that part of every key once for all heads and k holds the first
+    D - rope.head_dim dims.  v / o may have their own head dim (v.shape[-1]).
     ``split_qk`` forms QK^T from hi/lo bf16 parts of the rotated operands
     (LCX_ATTN_SPLIT_QK) for inputs whose large logits bf16 rounding would spoil.
     ``status`` (optional int32 CUDA tensor of one element) receives
@@ -239,11 +244,15 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
             raise ValueError("q, k, v must be 4-D CUDA tensors [B, H, L, D]")
     B, Hq, L, D = q.shape
     Hkv, Lk = k.shape[1], k.shape[2]
-    if k.shape != (B, Hkv, Lk, D) or v.shape != k.shape:
+    Dv = v.shape[3]
+    Dk = D - rope.head_dim if k_rope is not None else D
+    if k.shape != (B, Hkv, Lk, Dk) or v.shape != (B, Hkv, Lk, Dv):
         raise ValueError("shape mismatch: q %s k %s v %s" % (q.shape, k.shape, v.shape))
-    if not (q.dtype == k.dtype == v.dtype):
-        raise ValueError("q, k, v must share a dtype")
-    o = out if out is not None else torch.empty_like(q)
+    if k_rope is not None and (k_rope.dim() != 4 or k_rope.shape != (B, 1, Lk, rope.head_dim)):
+        raise ValueError("k_rope must be [B, 1, Lk, rope.head_dim], got %s" % (k_rope.shape,))
+    if not (q.dtype == k.dtype == v.dtype) or (k_rope is not None and k_rope.dtype != q.dtype):
+        raise ValueError("q, k, v (and k_rope) must share a dtype")
+    o = out if out is not None else torch.empty((B, Hq, L, Dv), dtype=q.dtype, device=q.device)
     if return_lse and lse is None:
         lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
     a = _AttnArgs()
@@ -266,10 +275,14 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
     a.reserved0 = 0
     a.Lk = Lk
     a.q_offset = int(q_offset)
+    a.Dv = Dv
+    if k_rope is not None:
+        a.k_rope = k_rope.data_ptr()
+        a.k_rope_strides = _strides(k_rope)
     if num_splits == 1:
         _check(load().lcx_attn_fwd(ctypes.byref(a), _stream(q)))
     else:
-        need = split_workspace_bytes(B, Hq, L, D, num_splits)
+        need = split_workspace_bytes(B, Hq, L, Dv, num_splits)
         if workspace is None:
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
         _check(load().lcx_attn_fwd_split(ctypes.byref(a), int(num_splits),

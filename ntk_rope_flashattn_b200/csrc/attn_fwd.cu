@@ -88,9 +88,12 @@ struct AttnParams {
     int n_qb, heads_per_unit, units_per_qb;
     int rotate_q, rotate_k;
     int n_split;                       // key-range splits per unit (1: plain output)
+    float split_recip;                 // 1 / n_split, rounded up
     float *part_o;                     // n_split > 1: [n_split, B, Hq, L, D] partial o
     float *part_lse;                   //              [n_split, B, Hq, L] partial lse
     int test_stall;                    // loader issues nothing (watchdog test hook)
+    int k_rope_shared;                 // rotated key columns come from one shared head
+    float rot_ms;                      // factor on rotated values (partial rotary: mscale)
     float c_log2;                      // logit scale in log2 units
     unsigned long long timeout_ns;
     float theta[64];
@@ -99,26 +102,30 @@ struct AttnParams {
 // Shared-memory plan.  A tile of R rows x D bf16 is stored as D/64 TMA boxes of
 // R rows x 128 bytes with the 128-byte swizzle.  In the split mode every Q and
 // K tile has a second "lo" part holding bf16(x' - bf16(x')), and key tiles are
-// 64 rows so that both parts fit.
-template <int D, bool kSplit>
+// 64 rows so that both parts fit.  D is the query/key head dim, DV the
+// value/output head dim; at D = 192 (decoupled RoPE: 128 + 64) one query tile
+// per CTA leaves room for two K and two V stages.
+template <int D, int DV, bool kSplit>
 struct Cfg {
     static constexpr int BN = kSplit ? 64 : 128;        // keys per tile
     static constexpr int kParts = kSplit ? 2 : 1;       // hi (+ lo) parts of Q and K
+    static constexpr int kNTQ = D > 128 ? 1 : 2;        // query tiles per CTA
     static constexpr int kTileQ = kBM * D * 2;          // one part of a Q tile
-    static constexpr int kTileK = BN * D * 2;           // one part of a K tile / a V tile
+    static constexpr int kTileK = BN * D * 2;           // one part of a K tile
+    static constexpr int kTileV = BN * DV * 2;          // a V tile
     static constexpr int kBoxQ = kBM * 128;
     static constexpr int kBoxK = BN * 128;
-    static constexpr int kStagesK = (D == 128) ? (kSplit ? 2 : LCX_KSTAGES_D128) : 4;
-    static constexpr int kStagesV = (D == 128) ? 2 : 4;
+    static constexpr int kStagesK = (D == 64) ? 4 : (D == 128 && !kSplit) ? LCX_KSTAGES_D128 : 2;
+    static constexpr int kStagesV = (D == 64) ? 4 : 2;
     static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + 2 * kParts * kTileQ;
+    static constexpr int kOffK = kOffQ + kNTQ * kParts * kTileQ;
     static constexpr int kOffV = kOffK + kStagesK * kParts * kTileK;
-    static constexpr int kOffBar = kOffV + kStagesV * kTileK;
+    static constexpr int kOffBar = kOffV + kStagesV * kTileV;
     static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers + alignment slack
     // TMEM columns: S_t at t*BN (P_t aliased over its first BN/2 columns), O_t after.
     static constexpr int kColO = 2 * BN;
     static_assert(kSmemBytes <= 232448, "shared memory budget");
-    static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
+    static_assert(2 * BN + 2 * DV <= 512, "TMEM budget");
 };
 
 template <int NSK, int NSV>
@@ -142,9 +149,10 @@ struct Unit {
 // most keys).  The block scheduler therefore runs many query blocks of the same
 // kv head side by side -- they stream the same K/V tiles, which L2 then serves
 // -- and still hands out the longest units of every group first.  With key
-// splits, the n_split CTAs of a unit are consecutive.
+// splits (kKvSplit), the n_split CTAs of a unit are consecutive.
+template <bool kKvSplit>
 __device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
-    const int u = blockIdx.x / p.n_split;
+    const int u = kKvSplit ? int(blockIdx.x) / p.n_split : int(blockIdx.x);
     const int upq = p.G / p.heads_per_unit;          // units per query block of a group
     const int per_group = p.n_qb * upq;
     const int grp = u / per_group, rem = u % per_group;
@@ -154,7 +162,7 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
     r.q0 = (p.n_qb - 1 - rem / upq) * kBM;
     r.nt = p.heads_per_unit;
     r.hq0 = r.g * p.G + p.heads_per_unit * (rem % upq);
-    r.split = blockIdx.x % p.n_split;
+    r.split = kKvSplit ? int(blockIdx.x) % p.n_split : 0;
     return r;
 }
 
@@ -170,8 +178,8 @@ struct Tiles {
     }
 };
 
-template <int BN>
-__device__ __forceinline__ Tiles make_tiles(int q0, const AttnParams &p) {
+template <int BN, bool kKvSplit>
+__device__ __forceinline__ Tiles make_tiles(int q0, int split, const AttnParams &p) {
     const int i1 = min(q0 + kBM - 1, p.L - 1) + p.qoff;
     const int jhi = p.causal ? i1 / BN : (p.Lk - 1) / BN;
     int jlo = 0, ns = 0;
@@ -184,13 +192,14 @@ __device__ __forceinline__ Tiles make_tiles(int q0, const AttnParams &p) {
     t.jlo = jlo;
     t.n = ns + (jhi - jlo + 1);
     t.j0 = 0;
-    if (p.n_split > 1) {
-        // split s of S takes tiles [n s / S, n (s + 1) / S); it may be empty
-        const int s = blockIdx.x % p.n_split;
-        const int jb = int((long long)t.n * s / p.n_split);
-        const int je = int((long long)t.n * (s + 1) / p.n_split);
+    if constexpr (kKvSplit) {
+        // split s of S takes tiles [s c, min(n, (s + 1) c)) with c >= n / S
+        // (c = n / S rounded up in fp32, never below the exact quotient for
+        // n < 2^24); the last splits may be empty.
+        const int per = int(ceilf(float(t.n) * p.split_recip));
+        const int jb = min(t.n, split * per);
         t.j0 = jb;
-        t.n = je - jb;
+        t.n = min(t.n, jb + per) - jb;
     }
     return t;
 }
@@ -289,10 +298,19 @@ struct Phasor {
 #pragma unroll
         for (int e = 0; e < R::PPJ; ++e) rope_sincos(R::RP, p.theta[i0 + e], &sc[e], &ss[e]);
     }
+    // kScaled: multiply by p.rot_ms (partial rotary, where mscale is not folded
+    // into the logit scale).
+    template <bool kScaled = false>
     __device__ __forceinline__ void start(long long pos0, const AttnParams &p, float (&c)[R::PPJ],
                                           float (&s)[R::PPJ]) const {
 #pragma unroll
-        for (int e = 0; e < R::PPJ; ++e) rope_sincos_fast(pos0 + r0, p.theta[i0 + e], &c[e], &s[e]);
+        for (int e = 0; e < R::PPJ; ++e) {
+            rope_sincos_fast(pos0 + r0, p.theta[i0 + e], &c[e], &s[e]);
+            if constexpr (kScaled) {
+                c[e] *= p.rot_ms;
+                s[e] *= p.rot_ms;
+            }
+        }
     }
     __device__ __forceinline__ void step(float (&c)[R::PPJ], float (&s)[R::PPJ]) const {
 #pragma unroll
@@ -322,14 +340,16 @@ struct PhasorCarry {
 };
 constexpr int kReseed = 16;
 
-// Rotate a ROWS x D bf16 tile in place (row r at position pos0 + r); in the
-// split mode also write the residual part into `lo`.
-template <int D, bool kHalf, bool kSplit, int ROWS>
+// Rotate a ROWS x D bf16 tile in place (row r at position pos0 + r); only its
+// last RD columns are rotated (RD = D: all of them).  In the split mode also
+// write the residual part into `lo`.
+template <int D, int RD, bool kHalf, bool kSplit, int ROWS>
 __device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, uint8_t *lo, long long pos0,
-                                                 const Phasor<D, kHalf> &ph, const AttnParams &p,
+                                                 const Phasor<RD, kHalf> &ph, const AttnParams &p,
                                                  bool rotate,
-                                                 PhasorCarry<Rot<D, kHalf>::PPJ> *carry = nullptr) {
-    using R = Rot<D, kHalf>;
+                                                 PhasorCarry<Rot<RD, kHalf>::PPJ> *carry = nullptr) {
+    using R = Rot<RD, kHalf>;
+    constexpr int C0 = (D - RD) / 8;  // first rotated 16-byte chunk of a row
     constexpr int NJ = ROWS / R::RP;
     constexpr int BOX = ROWS * 128;
     float c[R::PPJ], s[R::PPJ];
@@ -342,7 +362,7 @@ __device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, uint8_t *lo, lon
             }
             ++carry->age;
         } else {
-            ph.start(pos0, p, c, s);
+            ph.template start<(RD < D)>(pos0, p, c, s);
             if (carry) carry->age = 0;
         }
     }
@@ -350,7 +370,8 @@ __device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, uint8_t *lo, lon
     for (int k = 0; k < NJ; ++k) {
         const int r = ph.r0 + k * R::RP;
         if (kHalf) {
-            const uint32_t oa = chunk_off(r, ph.q, BOX), ob = chunk_off(r, ph.q + D / 16, BOX);
+            const uint32_t oa = chunk_off(r, C0 + ph.q, BOX);
+            const uint32_t ob = chunk_off(r, C0 + ph.q + RD / 16, BOX);
             float x1[8], x2[8];
             unpack8(*reinterpret_cast<const uint4 *>(tile + oa), x1);
             unpack8(*reinterpret_cast<const uint4 *>(tile + ob), x2);
@@ -358,7 +379,7 @@ __device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, uint8_t *lo, lon
             store8<kSplit>(tile, lo, oa, x1);
             store8<kSplit>(tile, lo, ob, x2);
         } else {
-            const uint32_t oa = chunk_off(r, ph.q, BOX);
+            const uint32_t oa = chunk_off(r, C0 + ph.q, BOX);
             float x[8];
             unpack8(*reinterpret_cast<const uint4 *>(tile + oa), x);
             if (rotate) {
@@ -489,10 +510,10 @@ __device__ __forceinline__ float row_max(const float (&v)[N]) {
 // Store 32 output columns [c*32, c*32+32) of query row i of head h, scaled by
 // inv: fp32 into the partial buffer of the unit's key split when there is one,
 // else rounded once to the output type.
-template <int D, bool kF32>
+template <int D, bool kF32, bool kKvSplit>
 __device__ __forceinline__ void store_o32(const AttnParams &p, const Unit &U, int h, int i, int c,
                                           const float (&v)[32], float inv) {
-    if (p.part_o) {
+    if constexpr (kKvSplit) {
         const long long prow = (((long long)U.split * p.B + U.b) * p.Hq + h) * p.L + i;
         float4 *dst = reinterpret_cast<float4 *>(p.part_o + prow * D + c * 32);
 #pragma unroll
@@ -520,21 +541,27 @@ __device__ __forceinline__ void store_o32(const AttnParams &p, const Unit &U, in
 }
 
 // The row's log-sum-exp (natural log) into the partial buffer or the output.
+template <bool kKvSplit>
 __device__ __forceinline__ void store_lse(const AttnParams &p, const Unit &U, int h, int i,
                                           float lse) {
-    if (p.part_o)
+    if constexpr (kKvSplit)
         p.part_lse[(((long long)U.split * p.B + U.b) * p.Hq + h) * p.L + i] = lse;
     else if (p.lse)
         p.lse[(U.b * (long long)p.Hq + h) * p.L + i] = lse;
 }
 
 // ---------------------------------------------------------------- kernel
-template <int D, bool kF32, bool kHalf, bool kSplit>
+// D: query/key head dim, DV: value/output head dim, RD: rotated (last) dims;
+// kKvSplit: this launch is one pass of split-KV (partial results per split).
+template <int D, int DV, int RD, bool kF32, bool kHalf, bool kSplit, bool kKvSplit>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq,
                     const __grid_constant__ CUtensorMap tmk,
-                    const __grid_constant__ CUtensorMap tmv, const __grid_constant__ AttnParams p) {
-    using C = Cfg<D, kSplit>;
+                    const __grid_constant__ CUtensorMap tmv,
+                    const __grid_constant__ CUtensorMap tmkr, const __grid_constant__ AttnParams p) {
+    using C = Cfg<D, DV, kSplit>;
+    static_assert(!kF32 || (RD == D && DV == D), "fp32 operands: full rotary, DV = D");
+    static_assert(!kSplit || (RD == D && DV == D), "split QK^T: full rotary, DV = D");
     constexpr int NSK = C::kStagesK;
     constexpr int NSV = C::kStagesV;
     constexpr int BN = C::BN;
@@ -550,8 +577,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const Unit U = decode_unit(p);
-    const Tiles T = make_tiles<BN>(U.q0, p);   // this CTA's key tiles (its split's share)
+    const Unit U = decode_unit<kKvSplit>(p);
+    const Tiles T = make_tiles<BN, kKvSplit>(U.q0, U.split, p);   // this CTA's key tiles
     volatile int *abort = &bar.abort;
     const uint64_t tmo = p.timeout_ns;
 
@@ -590,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (skip) {
         // nothing to do: fall through to the common exit
-    } else if (T.n == 0) {
+    } else if (kKvSplit && T.n == 0) {
         // A key split that received no tile (more splits than tiles): the
         // empty partial result, o = 0 and lse = -inf.
         if (warp < 8 && (warp >> 2) < U.nt) {
@@ -599,8 +626,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float z[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) z[e] = 0.f;
-                for (int c = 0; c < D / 32; ++c) store_o32<D, kF32>(p, U, h, i, c, z, 0.f);
-                store_lse(p, U, h, i, -INFINITY);
+                for (int c = 0; c < DV / 32; ++c)
+                    store_o32<DV, kF32, kKvSplit>(p, U, h, i, c, z, 0.f);
+                store_lse<kKvSplit>(p, U, h, i, -INFINITY);
             }
         }
     } else if ((warp >> 2) == 3) {
@@ -612,6 +640,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_prefetch_desc(&tmq);
                 tma_prefetch_desc(&tmk);
                 tma_prefetch_desc(&tmv);
+                if (RD < D && p.k_rope_shared) tma_prefetch_desc(&tmkr);
+                // With a shared rotary key, the K boxes from column D - RD on
+                // come from that tensor's single head.
+                constexpr int kNopeBoxes = (D - RD) / 64;
                 int issued_k[NSK] = {}, issued_v[NSV] = {};
                 mbar_arrive_expect_tx(&bar.full_q, U.nt * C::kTileQ);
                 for (int t = 0; t < U.nt; ++t)
@@ -625,15 +657,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (uk > 0) ok = mbar_wait(&bar.empty_k[sk], (uk - 1) & 1, abort, tmo);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&bar.full_k[sk], C::kTileK);
-                    for (int bx = 0; bx < D / 64; ++bx)
-                        tma_load_4d(sK + sk * C::kParts * C::kTileK + bx * C::kBoxK, &tmk,
-                                    &bar.full_k[sk], bx * 64, jt * BN, U.g, U.b);
+                    for (int bx = 0; bx < D / 64; ++bx) {
+                        uint8_t *dst = sK + sk * C::kParts * C::kTileK + bx * C::kBoxK;
+                        if constexpr (RD < D) {
+                            if (p.k_rope_shared && bx >= kNopeBoxes) {
+                                tma_load_4d(dst, &tmkr, &bar.full_k[sk], (bx - kNopeBoxes) * 64,
+                                            jt * BN, 0, U.b);
+                                continue;
+                            }
+                        }
+                        tma_load_4d(dst, &tmk, &bar.full_k[sk], bx * 64, jt * BN, U.g, U.b);
+                    }
                     ++issued_k[sk];
                     if (uv > 0) ok = mbar_wait(&bar.empty_v[sv], (uv - 1) & 1, abort, tmo);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(&bar.full_v[sv], C::kTileK);
-                    for (int bx = 0; bx < D / 64; ++bx)
-                        tma_load_4d(sV + sv * C::kTileK + bx * C::kBoxK, &tmv, &bar.full_v[sv],
+                    mbar_arrive_expect_tx(&bar.full_v[sv], C::kTileV);
+                    for (int bx = 0; bx < DV / 64; ++bx)
+                        tma_load_4d(sV + sv * C::kTileV + bx * C::kBoxK, &tmv, &bar.full_v[sv],
                                     bx * 64, jt * BN, U.g, U.b);
                     ++issued_v[sv];
                 }
@@ -649,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // ------------------------------------------------ MMA issuer
             if (lane == 0) {
                 constexpr uint32_t kIdS = idesc_bf16_f32(128, BN, 0, 0);
-                constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, 0, 1);
+                constexpr uint32_t kIdPV = idesc_bf16_f32(128, DV, 0, 1);
                 const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
                 // S_t = Q_t K^T over D in steps of 16 (32 bytes inside a 128-byte
                 // swizzle row, then the next 64-column box).  Split mode:
@@ -678,8 +718,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 };
                 // O_t += P_t V: P from TMEM (BN/2 columns of bf16 pairs), V MN-major.
                 auto issue_pv = [&](int t, int s, bool acc) {
-                    const uint64_t va = dv0 + ((s * C::kTileK) >> 4);
-                    const uint32_t dst = tmem + C::kColO + t * D, pa = tmem + t * BN;
+                    const uint64_t va = dv0 + ((s * C::kTileV) >> 4);
+                    const uint32_t dst = tmem + C::kColO + t * DV, pa = tmem + t * BN;
 #pragma unroll
                     for (int kk = 0; kk < BN / 16; ++kk)
                         mma_ts(dst, pa + kk * 8, va + ((kk * 2048) >> 4), kIdPV, (acc || kk > 0));
@@ -730,17 +770,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------ rotation warpgroup
         const int tw = threadIdx.x - kWarpRot0 * 32;
         const bool rotq = p.rotate_q != 0, rotk = p.rotate_k != 0;
-        Phasor<D, kHalf> ph;
+        Phasor<RD, kHalf> ph;
         ph.init(tw, p);
-        PhasorCarry<Rot<D, kHalf>::PPJ> kcarry;
+        PhasorCarry<Rot<RD, kHalf>::PPJ> kcarry;
         bool ok = true;
-        if (!kF32) {
+        if constexpr (!kF32) {
             ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_q, 0, abort, tmo));
             if (ok && (rotq || kSplit))
                 for (int t = 0; t < U.nt; ++t) {
                     uint8_t *qt = sQ + t * C::kParts * C::kTileQ;
-                    rotate_tile_bf16<D, kHalf, kSplit, kBM>(qt, qt + C::kTileQ,
-                                                            (long long)U.q0 + p.qoff, ph, p, rotq);
+                    rotate_tile_bf16<D, RD, kHalf, kSplit, kBM>(
+                        qt, qt + C::kTileQ, (long long)U.q0 + p.qoff, ph, p, rotq);
                 }
         } else {
             for (int t = 0; t < U.nt; ++t) {
@@ -759,12 +799,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int jt = T.tile(j);
             const int s = j % NSK, use = j / NSK, sv = j % NSV, usev = j / NSV;
             uint8_t *tk = sK + s * C::kParts * C::kTileK;
-            if (!kF32) {
+            if constexpr (!kF32) {
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_k[s], use & 1, abort, tmo));
                 if (!ok) break;
                 if (rotk || kSplit)
-                    rotate_tile_bf16<D, kHalf, kSplit, BN>(tk, tk + C::kTileK, (long long)jt * BN,
-                                                           ph, p, rotk, &kcarry);
+                    rotate_tile_bf16<D, RD, kHalf, kSplit, BN>(
+                        tk, tk + C::kTileK, (long long)jt * BN, ph, p, rotk, &kcarry);
             } else {
                 if (use > 0)
                     ok = __all_sync(0xffffffffu,
@@ -777,14 +817,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             fence_proxy_async_smem();
             mbar_arrive(&bar.ready_k[s]);
-            if (kF32) {
+            if constexpr (kF32) {
                 if (usev > 0)
                     ok = __all_sync(0xffffffffu,
                                     mbar_wait(&bar.empty_v[sv], (usev - 1) & 1, abort, tmo));
                 if (!ok) break;
                 const float *base = reinterpret_cast<const float *>(p.v) + U.b * p.vs[0] +
                                     (long long)U.g * p.vs[1];
-                load_v_f32<D, BN>(sV + sv * C::kTileK, base, p.vs[2], jt * BN, p.Lk, tw);
+                load_v_f32<D, BN>(sV + sv * C::kTileV, base, p.vs[2], jt * BN, p.Lk, tw);
                 fence_proxy_async_smem();
                 mbar_arrive(&bar.full_v[sv]);
             }
@@ -797,7 +837,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int wq = warp & 3;
             const int row = wq * 32 + lane;
             const uint32_t trow = tmem + (uint32_t(wq * 32) << 16);
-            const uint32_t s_col = t * BN, o_col = C::kColO + t * D;
+            const uint32_t s_col = t * BN, o_col = C::kColO + t * DV;
             const int i = U.q0 + row;      // query row; its position is qoff + i
             const int pi = i + p.qoff;
             const float cl2 = p.c_log2;
@@ -832,7 +872,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (__any_sync(0xffffffffu, need)) {
                     const float alpha = need ? ex2_approx(m - m_new) : 1.f;
     #pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
+                    for (int c = 0; c < DV / 32; ++c) {
                         float o[32];
                         tmem_ld32(trow + o_col + c * 32, o);
                         uint32_t u[32];
@@ -883,14 +923,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int h = U.hq0 + t;
                 const bool valid = i < p.L;
     #pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < DV / 32; ++c) {
                     float v[32];
                     tmem_ld32(trow + o_col + c * 32, v);
-                    if (valid) store_o32<D, kF32>(p, U, h, i, c, v, inv);
+                    if (valid) store_o32<DV, kF32, kKvSplit>(p, U, h, i, c, v, inv);
                 }
                 if (valid) {
                     const float ln2 = 0.69314718055994531f;
-                    store_lse(p, U, h, i, l > 0.f ? (m + __log2f(l)) * ln2 : -INFINITY);
+                    store_lse<kKvSplit>(p, U, h, i, l > 0.f ? (m + __log2f(l)) * ln2 : -INFINITY);
                 }
             }
         }
@@ -941,16 +981,28 @@ lcx_status make_map(CUtensorMap *map, const void *ptr, int64_t B, int64_t H, int
     return LCX_OK;
 }
 
-template <int D, bool kF32, bool kHalf, bool kSplit>
-lcx_status launch(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
-                  const AttnParams &p, unsigned grid, cudaStream_t s) {
-    auto kern = attn_fwd_kernel<D, kF32, kHalf, kSplit>;
-    const int smem = Cfg<D, kSplit>::kSmemBytes;
+// The four tensor maps of a launch: q, k (its non-shared columns), v, and the
+// shared rotary key (unused unless AttnParams::k_rope_shared).
+struct Maps {
+    CUtensorMap q, k, v, kr;
+};
+
+// Which kernel instance a launch needs.
+struct AttnLaunchShape {
+    bool f32, half, split_qk;
+    int D, DV, RD;    // query/key head dim, value head dim, rotated dims
+};
+
+template <int D, int DV, int RD, bool kF32, bool kHalf, bool kSplit, bool kKvSplit>
+lcx_status launch(const Maps &m, const AttnParams &p, unsigned grid, cudaStream_t s) {
+    auto kern = attn_fwd_kernel<D, DV, RD, kF32, kHalf, kSplit, kKvSplit>;
+    const int smem = Cfg<D, DV, kSplit>::kSmemBytes;
     // The warpgroups re-balance registers with setmaxnreg, which waits until the
     // registers it asks for are free: the launch must hold the whole split.
     static const int regs = []() {
         cudaFuncAttributes fa;
-        return cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kF32, kHalf, kSplit>) == cudaSuccess
+        return cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, DV, RD, kF32, kHalf, kSplit,
+                                                         kKvSplit>) == cudaSuccess
                    ? fa.numRegs
                    : -1;
     }();
@@ -960,21 +1012,42 @@ lcx_status launch(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMa
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
         return fail(LCX_ERR_CUDA, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
-    kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, p);
+    kern<<<grid, kThreads, smem, s>>>(m.q, m.k, m.v, m.kr, p);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return fail(LCX_ERR_CUDA, "attn_fwd launch failed: %s", cudaGetErrorString(e));
     return LCX_OK;
 }
 
-template <int D, bool kSplit>
-lcx_status launch_d(bool f32, bool half, const CUtensorMap &mq, const CUtensorMap &mk,
-                    const CUtensorMap &mv, const AttnParams &p, unsigned grid, cudaStream_t s) {
+// Full rotary (RD = D = DV): bf16 or fp32 operands, plain or split QK^T.
+template <int D, bool kSplit, bool kKv>
+lcx_status launch_full(bool f32, bool half, const Maps &m, const AttnParams &p, unsigned grid,
+                       cudaStream_t s) {
     if (f32)
-        return half ? launch<D, true, true, kSplit>(mq, mk, mv, p, grid, s)
-                    : launch<D, true, false, kSplit>(mq, mk, mv, p, grid, s);
-    return half ? launch<D, false, true, kSplit>(mq, mk, mv, p, grid, s)
-                : launch<D, false, false, kSplit>(mq, mk, mv, p, grid, s);
+        return half ? launch<D, D, D, true, true, kSplit, kKv>(m, p, grid, s)
+                    : launch<D, D, D, true, false, kSplit, kKv>(m, p, grid, s);
+    return half ? launch<D, D, D, false, true, kSplit, kKv>(m, p, grid, s)
+                : launch<D, D, D, false, false, kSplit, kKv>(m, p, grid, s);
+}
+
+// Partial rotary (the last RD of D dims): bf16 operands, plain QK^T.
+template <int D, int DV, int RD, bool kKv>
+lcx_status launch_partial(bool half, const Maps &m, const AttnParams &p, unsigned grid,
+                          cudaStream_t s) {
+    return half ? launch<D, DV, RD, false, true, false, kKv>(m, p, grid, s)
+                : launch<D, DV, RD, false, false, false, kKv>(m, p, grid, s);
+}
+
+template <bool kKv>
+lcx_status launch_shape(const AttnLaunchShape &x, const Maps &m, const AttnParams &p,
+                        unsigned g, cudaStream_t s) {
+    if (x.D == 192) return launch_partial<192, 128, 64, kKv>(x.half, m, p, g, s);
+    if (x.D == 128 && x.RD == 64) return launch_partial<128, 128, 64, kKv>(x.half, m, p, g, s);
+    if (x.D == 128)
+        return x.split_qk ? launch_full<128, true, kKv>(x.f32, x.half, m, p, g, s)
+                          : launch_full<128, false, kKv>(x.f32, x.half, m, p, g, s);
+    return x.split_qk ? launch_full<64, true, kKv>(x.f32, x.half, m, p, g, s)
+                      : launch_full<64, false, kKv>(x.f32, x.half, m, p, g, s);
 }
 
 lcx_status check_tensor(const void *ptr, const int64_t *st, int es, const char *name) {
@@ -996,12 +1069,10 @@ namespace lcx {
 namespace {
 
 // Everything one attn_fwd launch needs, derived from validated arguments.
-struct AttnLaunch {
+struct AttnLaunch : AttnLaunchShape {
     AttnParams p;
-    CUtensorMap mq, mk, mv;
+    Maps m;
     long long units;  // CTAs without key splits
-    bool f32, half, split_qk;
-    int D;
 };
 
 // Validate `a` and fill `x`.  *noop is set for empty problems (B or L zero),
@@ -1018,7 +1089,11 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     if (a->Hq % a->Hkv != 0)
         return fail(LCX_ERR_INVALID_ARG, "Hq (%lld) must be a multiple of Hkv (%lld)",
                     (long long)a->Hq, (long long)a->Hkv);
-    if (a->rope.head_dim != a->D) return fail(LCX_ERR_INVALID_ARG, "rope.head_dim != D");
+    const int64_t Dv = a->Dv > 0 ? a->Dv : a->D;
+    const int64_t RD = a->rope.head_dim;
+    if (a->Dv < 0) return fail(LCX_ERR_INVALID_ARG, "Dv must be >= 0");
+    if (RD > a->D) return fail(LCX_ERR_INVALID_ARG, "rope.head_dim > D");
+    const bool partial = RD < a->D;
     if (a->causal != 0 && a->causal != 1) return fail(LCX_ERR_INVALID_ARG, "causal must be 0 or 1");
     if (a->window < 0 || a->sinks < 0)
         return fail(LCX_ERR_INVALID_ARG, "window and sinks must be >= 0");
@@ -1041,8 +1116,18 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
         return fail(LCX_ERR_UNSUPPORTED, "the stall test hook needs bf16 operands");
     if (!(a->softmax_scale >= 0.f) || !std::isfinite(a->softmax_scale))
         return fail(LCX_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
-    if (a->D != 64 && a->D != 128)
-        return fail(LCX_ERR_UNSUPPORTED, "head_dim %lld: only 64 and 128", (long long)a->D);
+    const bool shape_ok = (a->D == 64 && Dv == 64 && RD == 64) ||
+                          (a->D == 128 && Dv == 128 && (RD == 128 || RD == 64)) ||
+                          (a->D == 192 && Dv == 128 && RD == 64);
+    if (!shape_ok)
+        return fail(LCX_ERR_UNSUPPORTED,
+                    "(D, Dv, rotated dims) = (%lld, %lld, %lld): supported are (64, 64, 64), "
+                    "(128, 128, 128), (128, 128, 64), (192, 128, 64)",
+                    (long long)a->D, (long long)Dv, (long long)RD);
+    if (partial && (a->dtype != LCX_BF16 || (a->flags & LCX_ATTN_SPLIT_QK)))
+        return fail(LCX_ERR_UNSUPPORTED, "partial rotary needs bf16 operands and plain QK^T");
+    if (a->k_rope && !partial)
+        return fail(LCX_ERR_INVALID_ARG, "k_rope needs rope.head_dim < D");
     if (a->B == 0 || a->L == 0) {
         *noop = true;
         return LCX_OK;
@@ -1055,6 +1140,8 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     if ((st = check_tensor(a->k, a->k_strides, es, "k")) != LCX_OK) return st;
     if ((st = check_tensor(a->v, a->v_strides, es, "v")) != LCX_OK) return st;
     if ((st = check_tensor(a->o, a->o_strides, es, "o")) != LCX_OK) return st;
+    if (a->k_rope && (st = check_tensor(a->k_rope, a->k_rope_strides, es, "k_rope")) != LCX_OK)
+        return st;
 
     memset(&x, 0, sizeof(x));
     AttnParams &p = x.p;
@@ -1082,7 +1169,9 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     p.window = int(a->window > Lk ? Lk : a->window);
     p.sinks = int(a->sinks > Lk ? Lk : a->sinks);
     p.n_qb = int((a->L + kBM - 1) / kBM);
-    p.heads_per_unit = (p.G % 2 == 0) ? 2 : 1;
+    // Two query heads share a CTA's K/V tiles when the group allows it and
+    // two query tiles fit (D = 192 leaves room for one).
+    p.heads_per_unit = (p.G % 2 == 0 && a->D <= 128) ? 2 : 1;
     p.units_per_qb = p.B * p.Hq / p.heads_per_unit;
     p.n_split = 1;
     x.units = (long long)p.n_qb * p.units_per_qb;
@@ -1093,10 +1182,19 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     // The length-dependent modes see the whole context: the Lk keys.
     rope_table_unchecked(&a->rope, effective_seq_len(&a->rope, Lk), p.theta, &ms);
     const double scale = a->softmax_scale > 0.f ? double(a->softmax_scale) : 1.0 / std::sqrt(double(a->D));
-    // Each operand rotated on chip contributes its mscale factor to the logits
-    // (pre-rotated operands already carry theirs).
-    const double msq = (p.rotate_q ? double(ms) : 1.0) * (p.rotate_k ? double(ms) : 1.0);
+    double msq = 1.0;
+    p.rot_ms = 1.f;
+    if (!partial) {
+        // Each operand rotated on chip contributes its mscale factor to the
+        // logits (pre-rotated operands already carry theirs): folded into the
+        // logit scale.
+        msq = (p.rotate_q ? double(ms) : 1.0) * (p.rotate_k ? double(ms) : 1.0);
+    } else {
+        // Only the rotated dims carry mscale: applied to the rotated values.
+        p.rot_ms = ms;
+    }
     p.c_log2 = float(scale * msq * 1.4426950408889634);
+    p.k_rope_shared = a->k_rope ? 1 : 0;
     // Legitimate waits last microseconds; the default limit is 2 s.
     p.timeout_ns = 1000000ull * (unsigned long long)(a->watchdog_ms > 0 ? a->watchdog_ms : 2000);
     p.test_stall = (a->flags & LCX_ATTN_TEST_STALL) ? 1 : 0;
@@ -1105,14 +1203,23 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     x.f32 = a->dtype == LCX_F32;
     x.half = a->rope.pairing == LCX_PAIR_HALF;
     x.D = int(a->D);
+    x.DV = int(Dv);
+    x.RD = int(RD);
     const uint32_t bn = x.split_qk ? 64u : 128u;
     if (!x.f32) {
-        if ((st = make_map(&x.mq, a->q, a->B, a->Hq, a->L, a->D, a->q_strides, 128, "q")) != LCX_OK)
+        const int64_t dk = a->k_rope ? a->D - RD : a->D;   // columns k itself holds
+        if ((st = make_map(&x.m.q, a->q, a->B, a->Hq, a->L, a->D, a->q_strides, 128, "q")) != LCX_OK)
             return st;
-        if ((st = make_map(&x.mk, a->k, a->B, a->Hkv, Lk, a->D, a->k_strides, bn, "k")) != LCX_OK)
+        if ((st = make_map(&x.m.k, a->k, a->B, a->Hkv, Lk, dk, a->k_strides, bn, "k")) != LCX_OK)
             return st;
-        if ((st = make_map(&x.mv, a->v, a->B, a->Hkv, Lk, a->D, a->v_strides, bn, "v")) != LCX_OK)
+        if ((st = make_map(&x.m.v, a->v, a->B, a->Hkv, Lk, Dv, a->v_strides, bn, "v")) != LCX_OK)
             return st;
+        if (a->k_rope) {
+            // one head: the head stride never matters, any valid value will do
+            int64_t krs[4] = {a->k_rope_strides[0], Lk * RD, a->k_rope_strides[2], 1};
+            if ((st = make_map(&x.m.kr, a->k_rope, a->B, 1, Lk, RD, krs, bn, "k_rope")) != LCX_OK)
+                return st;
+        }
     }
     return LCX_OK;
 }
@@ -1122,11 +1229,8 @@ lcx_status attn_enqueue(const AttnLaunch &x, cudaStream_t s) {
     const long long grid = x.units * x.p.n_split;
     if (grid > 0x7fffffffLL) return fail(LCX_ERR_UNSUPPORTED, "too many work units");
     const unsigned g = unsigned(grid);
-    if (x.D == 128)
-        return x.split_qk ? launch_d<128, true>(x.f32, x.half, x.mq, x.mk, x.mv, x.p, g, s)
-                          : launch_d<128, false>(x.f32, x.half, x.mq, x.mk, x.mv, x.p, g, s);
-    return x.split_qk ? launch_d<64, true>(x.f32, x.half, x.mq, x.mk, x.mv, x.p, g, s)
-                      : launch_d<64, false>(x.f32, x.half, x.mq, x.mk, x.mv, x.p, g, s);
+    return x.p.n_split > 1 ? launch_shape<true>(x, x.m, x.p, g, s)
+                           : launch_shape<false>(x, x.m, x.p, g, s);
 }
 
 constexpr int kMaxKvSplits = 256;
@@ -1179,7 +1283,7 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
     if (num_splits == 1) return attn_enqueue(x, s);
     const int64_t rows = a->B * a->Hq * a->L;
     if (rows > kMaxSplitRows) return fail(LCX_ERR_UNSUPPORTED, "too many query rows to split");
-    const int64_t need = split_ws_bytes(rows, a->D, num_splits);
+    const int64_t need = split_ws_bytes(rows, x.DV, num_splits);
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(LCX_ERR_INVALID_ARG, "workspace must be a 256-byte aligned device pointer");
     if (workspace_bytes < need)
@@ -1187,11 +1291,12 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
                     (long long)workspace_bytes, (long long)need);
     float *part_o = static_cast<float *>(workspace);
     float *part_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) +
-                                                split_o_bytes(rows, a->D, num_splits));
+                                                split_o_bytes(rows, x.DV, num_splits));
     x.p.n_split = num_splits;
+    x.p.split_recip = std::nextafter(1.0f / float(num_splits), 2.0f);
     x.p.part_o = part_o;
     x.p.part_lse = part_lse;
     if ((st = attn_enqueue(x, s)) != LCX_OK) return st;
-    return launch_merge(part_o, part_lse, num_splits, a->B, a->Hq, a->L, a->D, a->o, a->dtype,
+    return launch_merge(part_o, part_lse, num_splits, a->B, a->Hq, a->L, x.DV, a->o, a->dtype,
                         a->o_strides, a->lse, s);
 }

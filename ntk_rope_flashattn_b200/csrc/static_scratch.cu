@@ -54,7 +54,8 @@ extern "C" lcx_status lcx_attn_fwd_split_static(const lcx_attn_args *a, int32_t 
     clear_error();
     if (!a) return fail(LCX_ERR_INVALID_ARG, "args is NULL");
     if (num_splits == 1) return lcx_attn_fwd_split(a, 1, nullptr, 0, stream);
-    const int64_t need = lcx_attn_split_workspace_bytes(a->B, a->Hq, a->L, a->D, num_splits);
+    const int64_t dv = a->Dv > 0 ? a->Dv : a->D;   // the partial outputs' head dim
+    const int64_t need = lcx_attn_split_workspace_bytes(a->B, a->Hq, a->L, dv, num_splits);
     if (need < 0)
         return fail(LCX_ERR_INVALID_ARG, "invalid sizes or num_splits for split-KV attention");
     if (need > kStaticScratchBytes)

@@ -67,7 +67,8 @@ int main(void) {
   P(lcx_attn_args, q_strides) P(lcx_attn_args, o_strides) P(lcx_attn_args, rope)
   P(lcx_attn_args, window) P(lcx_attn_args, sinks) P(lcx_attn_args, softmax_scale)
   P(lcx_attn_args, flags) P(lcx_attn_args, watchdog_ms) P(lcx_attn_args, reserved0)
-  P(lcx_attn_args, Lk) P(lcx_attn_args, q_offset)
+  P(lcx_attn_args, Lk) P(lcx_attn_args, q_offset) P(lcx_attn_args, Dv)
+  P(lcx_attn_args, k_rope) P(lcx_attn_args, k_rope_strides)
   return 0;
 }
 ''')
@@ -211,7 +212,7 @@ def _attn_args(**kw):
 @pytest.mark.parametrize("kw,expect", [
     (dict(Hkv=3), lcx.LCX_ERR_INVALID_ARG),
     (dict(D=96, rope=_params("plain", 96)), lcx.LCX_ERR_UNSUPPORTED),
-    (dict(rope=_params("plain", 64)), lcx.LCX_ERR_INVALID_ARG),
+    (dict(rope=_params("plain", 130)), lcx.LCX_ERR_INVALID_ARG),     # rotated dims > D
     (dict(dtype=5), lcx.LCX_ERR_INVALID_ARG),
     (dict(causal=2), lcx.LCX_ERR_INVALID_ARG),
     (dict(window=-1), lcx.LCX_ERR_INVALID_ARG),
@@ -232,6 +233,16 @@ def _attn_args(**kw):
     (dict(q_offset=1), lcx.LCX_ERR_INVALID_ARG),            # causal: q_offset + L > Lk
     (dict(Lk=255), lcx.LCX_ERR_INVALID_ARG),                # causal: L > Lk
     (dict(Lk=1 << 31, q_offset=(1 << 31) - 256), lcx.LCX_ERR_UNSUPPORTED),
+    (dict(Dv=-1), lcx.LCX_ERR_INVALID_ARG),
+    (dict(Dv=64), lcx.LCX_ERR_UNSUPPORTED),                           # (128, 64, 128)
+    (dict(rope=_params("plain", 256)), lcx.LCX_ERR_INVALID_ARG),      # rotated > D
+    (dict(rope=_params("plain", 32)), lcx.LCX_ERR_UNSUPPORTED),       # (128, 128, 32)
+    (dict(rope=_params("plain", 64), dtype=1), lcx.LCX_ERR_UNSUPPORTED),   # partial fp32
+    (dict(rope=_params("plain", 64), flags=2), lcx.LCX_ERR_UNSUPPORTED),   # partial split
+    (dict(k_rope=0x500000), lcx.LCX_ERR_INVALID_ARG),                 # k_rope, full rotary
+    (dict(D=192, rope=_params("plain", 192)), lcx.LCX_ERR_UNSUPPORTED),
+    (dict(D=192, Dv=128, rope=_params("plain", 64), k_rope=0x500008,
+          k_rope_strides=[256 * 64, 256 * 64, 64, 1]), lcx.LCX_ERR_UNSUPPORTED),  # misaligned
 ])
 def test_attn_validation_without_device(lib, kw, expect):
     a = _attn_args(**kw)
