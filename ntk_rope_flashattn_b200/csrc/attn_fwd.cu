@@ -88,6 +88,8 @@ struct AttnParams {
     int n_qb, heads_per_unit, units_per_qb;
     int rotate_q, rotate_k;
     int n_split;                       // key-range splits per unit (1: plain output)
+    int pack_lp, pack_hpt;             // head-packed query tiles (split-KV only): rows
+                                       // per head (multiple of 8), heads per tile; 0 = off
     float split_recip;                 // 1 / n_split, rounded up
     float *part_o;                     // n_split > 1: [n_split, B, Hq, L, D] partial o
     float *part_lse;                   //              [n_split, B, Hq, L] partial lse
@@ -142,6 +144,7 @@ struct Bars {
 // ---------------------------------------------------------------- schedule
 struct Unit {
     int b, g, hq0, nt, q0, split;
+    int hpt;  // heads per query tile: 1, or pack_hpt when the tiles are head-packed
 };
 
 // Work units are grouped by (batch, kv head) and, inside a group, numbered
@@ -160,9 +163,12 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
     r.b = grp / p.Hkv;
     r.g = grp % p.Hkv;
     r.q0 = (p.n_qb - 1 - rem / upq) * kBM;
-    r.nt = p.heads_per_unit;
     r.hq0 = r.g * p.G + p.heads_per_unit * (rem % upq);
     r.split = kKvSplit ? int(blockIdx.x) % p.n_split : 0;
+    // Head-packed (split-KV decode): one unit per kv group, its heads spread over
+    // the two query tiles.
+    r.hpt = (kKvSplit && p.pack_lp) ? p.pack_hpt : 1;
+    r.nt = p.heads_per_unit / r.hpt;
     return r;
 }
 
@@ -343,13 +349,68 @@ constexpr int kReseed = 16;
 // Rotate a ROWS x D bf16 tile in place (row r at position pos0 + r); only its
 // last RD columns are rotated (RD = D: all of them).  In the split mode also
 // write the residual part into `lo`.
+// Rotate (or, with rotate = false, only copy into hi/lo parts) this thread's
+// pairs of row r of a tile whose boxes are BOX bytes long; (c, s) the phasor.
+template <int D, int RD, bool kHalf, bool kSplit, int BOX>
+__device__ __forceinline__ void rotate_row(uint8_t *tile, uint8_t *lo, int r, int q,
+                                           const float *c, const float *s, bool rotate) {
+    constexpr int C0 = (D - RD) / 8;  // first rotated 16-byte chunk of a row
+    if (kHalf) {
+        const uint32_t oa = chunk_off(r, C0 + q, BOX);
+        const uint32_t ob = chunk_off(r, C0 + q + RD / 16, BOX);
+        float x1[8], x2[8];
+        unpack8(*reinterpret_cast<const uint4 *>(tile + oa), x1);
+        unpack8(*reinterpret_cast<const uint4 *>(tile + ob), x2);
+        if (rotate) rot_pairs<8>(x1, x2, c, s);
+        store8<kSplit>(tile, lo, oa, x1);
+        store8<kSplit>(tile, lo, ob, x2);
+    } else {
+        const uint32_t oa = chunk_off(r, C0 + q, BOX);
+        float x[8];
+        unpack8(*reinterpret_cast<const uint4 *>(tile + oa), x);
+        if (rotate) {
+            float x1[4], x2[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                x1[e] = x[2 * e];
+                x2[e] = x[2 * e + 1];
+            }
+            rot_pairs<4>(x1, x2, c, s);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                x[2 * e] = x1[e];
+                x[2 * e + 1] = x2[e];
+            }
+        }
+        store8<kSplit>(tile, lo, oa, x);
+    }
+}
+
+// A head-packed query tile (decode): row r = k Lp + i holds query i of the
+// tile's k-th head, at position pos0 + i; only rows < rows_used hold data.
+// Each row's phasor is evaluated from its exact angle (once per CTA).
+template <int D, int RD, bool kHalf, bool kSplit>
+__device__ __forceinline__ void rotate_packed_q(uint8_t *tile, uint8_t *lo, long long pos0,
+                                                int Lp, int rows_used,
+                                                const Phasor<RD, kHalf> &ph, const AttnParams &p,
+                                                bool rotate) {
+    using R = Rot<RD, kHalf>;
+    constexpr int NJ = kBM / R::RP;
+    for (int k = 0; k < NJ; ++k) {
+        const int r = ph.r0 + k * R::RP;
+        if (r >= rows_used) break;
+        float c[R::PPJ], s[R::PPJ];
+        if (rotate) ph.template start<(RD < D)>(pos0 + (r % Lp) - ph.r0, p, c, s);
+        rotate_row<D, RD, kHalf, kSplit, kBM * 128>(tile, lo, r, ph.q, c, s, rotate);
+    }
+}
+
 template <int D, int RD, bool kHalf, bool kSplit, int ROWS>
 __device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, uint8_t *lo, long long pos0,
                                                  const Phasor<RD, kHalf> &ph, const AttnParams &p,
                                                  bool rotate,
                                                  PhasorCarry<Rot<RD, kHalf>::PPJ> *carry = nullptr) {
     using R = Rot<RD, kHalf>;
-    constexpr int C0 = (D - RD) / 8;  // first rotated 16-byte chunk of a row
     constexpr int NJ = ROWS / R::RP;
     constexpr int BOX = ROWS * 128;
     float c[R::PPJ], s[R::PPJ];
@@ -369,35 +430,7 @@ __device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, uint8_t *lo, lon
 #pragma unroll kRotUnroll
     for (int k = 0; k < NJ; ++k) {
         const int r = ph.r0 + k * R::RP;
-        if (kHalf) {
-            const uint32_t oa = chunk_off(r, C0 + ph.q, BOX);
-            const uint32_t ob = chunk_off(r, C0 + ph.q + RD / 16, BOX);
-            float x1[8], x2[8];
-            unpack8(*reinterpret_cast<const uint4 *>(tile + oa), x1);
-            unpack8(*reinterpret_cast<const uint4 *>(tile + ob), x2);
-            if (rotate) rot_pairs<8>(x1, x2, c, s);
-            store8<kSplit>(tile, lo, oa, x1);
-            store8<kSplit>(tile, lo, ob, x2);
-        } else {
-            const uint32_t oa = chunk_off(r, C0 + ph.q, BOX);
-            float x[8];
-            unpack8(*reinterpret_cast<const uint4 *>(tile + oa), x);
-            if (rotate) {
-                float x1[4], x2[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    x1[e] = x[2 * e];
-                    x2[e] = x[2 * e + 1];
-                }
-                rot_pairs<4>(x1, x2, c, s);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    x[2 * e] = x1[e];
-                    x[2 * e + 1] = x2[e];
-                }
-            }
-            store8<kSplit>(tile, lo, oa, x);
-        }
+        rotate_row<D, RD, kHalf, kSplit, BOX>(tile, lo, r, ph.q, c, s, rotate);
         if (rotate) ph.step(c, s);
     }
     if (LCX_PHASOR_CARRY && carry && rotate) {
@@ -550,6 +583,28 @@ __device__ __forceinline__ void store_lse(const AttnParams &p, const Unit &U, in
         p.lse[(U.b * (long long)p.Hq + h) * p.L + i] = lse;
 }
 
+// Query row `row` of tile t: its head, its query index and whether it holds a
+// query (head-packed tiles: row = k Lp + i for the tile's k-th head).
+struct RowMap {
+    int h, i;
+    bool valid;
+};
+__device__ __forceinline__ RowMap map_row(const AttnParams &p, const Unit &U, int t, int row,
+                                          bool packed) {
+    RowMap m;
+    if (packed) {
+        const int k = row / p.pack_lp;
+        m.i = row - k * p.pack_lp;
+        m.h = U.hq0 + t * U.hpt + k;
+        m.valid = k < U.hpt && m.i < p.L;
+    } else {
+        m.h = U.hq0 + t;
+        m.i = U.q0 + row;
+        m.valid = m.i < p.L;
+    }
+    return m;
+}
+
 // ---------------------------------------------------------------- kernel
 // D: query/key head dim, DV: value/output head dim, RD: rotated (last) dims;
 // kKvSplit: this launch is one pass of split-KV (partial results per split).
@@ -579,6 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lane = threadIdx.x & 31;
     const Unit U = decode_unit<kKvSplit>(p);
     const Tiles T = make_tiles<BN, kKvSplit>(U.q0, U.split, p);   // this CTA's key tiles
+    const bool packed = kKvSplit && !kF32 && p.pack_lp > 0;       // head-packed query tiles
     volatile int *abort = &bar.abort;
     const uint64_t tmo = p.timeout_ns;
 
@@ -621,14 +677,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // A key split that received no tile (more splits than tiles): the
         // empty partial result, o = 0 and lse = -inf.
         if (warp < 8 && (warp >> 2) < U.nt) {
-            const int h = U.hq0 + (warp >> 2), i = U.q0 + (warp & 3) * 32 + lane;
-            if (i < p.L) {
+            const RowMap rm = map_row(p, U, warp >> 2, (warp & 3) * 32 + lane, packed);
+            if (rm.valid) {
                 float z[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) z[e] = 0.f;
                 for (int c = 0; c < DV / 32; ++c)
-                    store_o32<DV, kF32, kKvSplit>(p, U, h, i, c, z, 0.f);
-                store_lse<kKvSplit>(p, U, h, i, -INFINITY);
+                    store_o32<DV, kF32, kKvSplit>(p, U, rm.h, rm.i, c, z, 0.f);
+                store_lse<kKvSplit>(p, U, rm.h, rm.i, -INFINITY);
             }
         }
     } else if ((warp >> 2) == 3) {
@@ -645,11 +701,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // come from that tensor's single head.
                 constexpr int kNopeBoxes = (D - RD) / 64;
                 int issued_k[NSK] = {}, issued_v[NSV] = {};
-                mbar_arrive_expect_tx(&bar.full_q, U.nt * C::kTileQ);
-                for (int t = 0; t < U.nt; ++t)
-                    for (int bx = 0; bx < D / 64; ++bx)
-                        tma_load_4d(sQ + t * C::kParts * C::kTileQ + bx * C::kBoxQ, &tmq, &bar.full_q,
-                                    bx * 64, U.q0, U.hq0 + t, U.b);
+                if (packed) {
+                    // each head's pack_lp rows at row k pack_lp of its tile (the Q
+                    // map's box is pack_lp rows high; 8-row multiples keep the
+                    // 128-byte swizzle phase of the full tile)
+                    mbar_arrive_expect_tx(&bar.full_q,
+                                          U.nt * U.hpt * (D / 64) * p.pack_lp * 128);
+                    for (int t = 0; t < U.nt; ++t)
+                        for (int k = 0; k < U.hpt; ++k)
+                            for (int bx = 0; bx < D / 64; ++bx)
+                                tma_load_4d(sQ + t * C::kParts * C::kTileQ + bx * C::kBoxQ +
+                                                k * p.pack_lp * 128,
+                                            &tmq, &bar.full_q, bx * 64, 0, U.hq0 + t * U.hpt + k,
+                                            U.b);
+                } else {
+                    mbar_arrive_expect_tx(&bar.full_q, U.nt * C::kTileQ);
+                    for (int t = 0; t < U.nt; ++t)
+                        for (int bx = 0; bx < D / 64; ++bx)
+                            tma_load_4d(sQ + t * C::kParts * C::kTileQ + bx * C::kBoxQ, &tmq,
+                                        &bar.full_q, bx * 64, U.q0, U.hq0 + t, U.b);
+                }
                 bool ok = true;
                 for (int j = 0; ok && j < T.n; ++j) {
                     const int jt = T.tile(j);
@@ -779,8 +850,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok && (rotq || kSplit))
                 for (int t = 0; t < U.nt; ++t) {
                     uint8_t *qt = sQ + t * C::kParts * C::kTileQ;
-                    rotate_tile_bf16<D, RD, kHalf, kSplit, kBM>(
-                        qt, qt + C::kTileQ, (long long)U.q0 + p.qoff, ph, p, rotq);
+                    if (packed)
+                        rotate_packed_q<D, RD, kHalf, kSplit>(qt, qt + C::kTileQ, p.qoff,
+                                                              p.pack_lp, U.hpt * p.pack_lp, ph,
+                                                              p, rotq);
+                    else
+                        rotate_tile_bf16<D, RD, kHalf, kSplit, kBM>(
+                            qt, qt + C::kTileQ, (long long)U.q0 + p.qoff, ph, p, rotq);
                 }
         } else {
             for (int t = 0; t < U.nt; ++t) {
@@ -838,8 +914,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int row = wq * 32 + lane;
             const uint32_t trow = tmem + (uint32_t(wq * 32) << 16);
             const uint32_t s_col = t * BN, o_col = C::kColO + t * DV;
-            const int i = U.q0 + row;      // query row; its position is qoff + i
-            const int pi = i + p.qoff;
+            const RowMap rm = map_row(p, U, t, row, packed);
+            const int pi = rm.i + p.qoff;  // this row's query position
             const float cl2 = p.c_log2;
             float m = -INFINITY, l = 0.f;
             bool ok = true;
@@ -920,17 +996,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok) {
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.f / l : 0.f;
-                const int h = U.hq0 + t;
-                const bool valid = i < p.L;
     #pragma unroll 1
                 for (int c = 0; c < DV / 32; ++c) {
                     float v[32];
                     tmem_ld32(trow + o_col + c * 32, v);
-                    if (valid) store_o32<DV, kF32, kKvSplit>(p, U, h, i, c, v, inv);
+                    if (rm.valid) store_o32<DV, kF32, kKvSplit>(p, U, rm.h, rm.i, c, v, inv);
                 }
-                if (valid) {
+                if (rm.valid) {
                     const float ln2 = 0.69314718055994531f;
-                    store_lse<kKvSplit>(p, U, h, i, l > 0.f ? (m + __log2f(l)) * ln2 : -INFINITY);
+                    store_lse<kKvSplit>(p, U, rm.h, rm.i,
+                                        l > 0.f ? (m + __log2f(l)) * ln2 : -INFINITY);
                 }
             }
         }
@@ -1294,6 +1369,22 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
                                                 split_o_bytes(rows, x.DV, num_splits));
     x.p.n_split = num_splits;
     x.p.split_recip = std::nextafter(1.0f / float(num_splits), 2.0f);
+    // Head-packed query tiles: with few queries per head (decode, short chunks)
+    // the G heads of a kv group share the CTA's two 128-row query tiles, G/2
+    // heads of pack_lp rows each (L rounded up to 8 rows), so every K/V tile is
+    // read and rotated once per kv group instead of once per head pair.
+    const int64_t lp = (a->L + 7) / 8 * 8;
+    if (!x.f32 && x.p.G % 2 == 0 && x.D <= 128 && lp * (x.p.G / 2) <= kBM) {
+        x.p.pack_lp = int(lp);
+        x.p.pack_hpt = x.p.G / 2;
+        x.p.heads_per_unit = x.p.G;
+        x.p.n_qb = 1;
+        x.p.units_per_qb = x.p.B * x.p.Hkv;
+        x.units = (long long)x.p.B * x.p.Hkv;
+        if ((st = make_map(&x.m.q, a->q, a->B, a->Hq, a->L, a->D, a->q_strides, uint32_t(lp),
+                           "q")) != LCX_OK)
+            return st;
+    }
     x.p.part_o = part_o;
     x.p.part_lse = part_lse;
     if ((st = attn_enqueue(x, s)) != LCX_OK) return st;

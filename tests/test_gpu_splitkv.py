@@ -112,3 +112,25 @@ def test_merge_matches_oracle(D, dtype):
     finite = np.isfinite(ref_lse)
     assert np.isneginf(lse_np[~finite]).all() and (got[~finite] == 0).all()
     assert np.abs(lse_np[finite] - ref_lse[finite]).max() <= 1e-5
+
+
+@pytest.mark.parametrize("L,Hq,Hkv,extra", [
+    (3, 8, 1, {}),                                   # G = 8: 4 heads x 8 rows per tile
+    (33, 8, 2, dict(window=500, sinks=4)),           # G = 4, 40-row head blocks
+    (1, 8, 2, dict(pairing="interleaved")),
+    (8, 16, 1, {}),                                  # G = 16: 8 heads x 8 rows
+    (2, 6, 1, dict(mode="ntk", scale=4.0)),          # G = 6: 3 heads per tile
+    (5, 4, 2, dict(split_qk=True, D=64)),            # hi/lo parts, D = 64
+])
+def test_splitkv_head_packed_decode(L, Hq, Hkv, extra):
+    """Few queries per head: the kv group's heads share the two query tiles
+    (head-packed layout); every head's rows against the oracle."""
+    Lk = 2000
+    w = W0.with_(Hq=Hq, Hkv=Hkv, **extra, L=Lk)
+    q_all, k, v = make_inputs(w, device="cuda")
+    q = q_all[:, :, Lk - L:]
+    rope = rope_of(w)
+    o, lse = run_split(q, k, v, rope, 4, window=w.window, sinks=w.sinks, q_offset=Lk - L,
+                       split_qk=w.split_qk)
+    ref = oracle_rows(q, k, v, rope, Lk - L, True, w.window, w.sinks)
+    compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref[0], ref[1])
