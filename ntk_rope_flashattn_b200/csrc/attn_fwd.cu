@@ -1280,7 +1280,13 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     x.D = int(a->D);
     x.DV = int(Dv);
     x.RD = int(RD);
-    const uint32_t bn = x.split_qk ? 64u : 128u;
+    // K/V boxes are one key tile high: the kernel's expect-tx byte counts and
+    // stage layout assume exactly Cfg::BN rows per box.
+    const uint32_t bn = x.split_qk ? uint32_t(Cfg<64, 64, true>::BN) : uint32_t(Cfg<64, 64, false>::BN);
+    static_assert(Cfg<64, 64, true>::BN == Cfg<128, 128, true>::BN &&
+                      Cfg<64, 64, false>::BN == Cfg<128, 128, false>::BN &&
+                      Cfg<64, 64, false>::BN == Cfg<192, 128, false>::BN,
+                  "one key-tile height per QK^T mode");
     if (!x.f32) {
         const int64_t dk = a->k_rope ? a->D - RD : a->D;   // columns k itself holds
         if ((st = make_map(&x.m.q, a->q, a->B, a->Hq, a->L, a->D, a->q_strides, 128, "q")) != LCX_OK)
