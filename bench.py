@@ -42,9 +42,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
 # launch on the headline workload (yarn_L131072_s16), from a one-pass ncu capture
-# of the current kernel: 3.01 GB read + 1.07 GB written (algorithmic: q, k, v
+# of the current kernel: 3.00 GB read + 1.07 GB written (algorithmic: q, k, v
 # read once = 1.61 GB, o written once = 1.07 GB).  Only valid for that workload.
-ATTN_TRAFFIC_BYTES = {"yarn_L131072_s16": 4.08e9}
+ATTN_TRAFFIC_BYTES = {"yarn_L131072_s16": 4.07e9}
 
 
 def load_peaks():
@@ -265,6 +265,7 @@ def bench_gpu(args, world, rank, local):
 
     # --- split-KV decode: one new token per query head against the whole cache
     decode = bench_decode(lcx, w, q, k, v, rope, stream, status)
+    mla = bench_mla(lcx, dev, stream, status) if rank == 0 else None
 
     # --- end to end through host buffers
     qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
@@ -340,7 +341,11 @@ def bench_gpu(args, world, rank, local):
                 "d2h_bytes_per_step": d2h},
         "clocks": clk.summary(),
         "splitkv_decode": decode,
+        "mla_prefill": mla,
     }
+    if mla is not None:
+        mla["peak"] = float(peaks["bf16_tflops_sustained"])
+        mla["frac"] = round(mla["achieved"] / mla["peak"], 4)
     if decode is not None:
         decode["peak"] = float(peaks["hbm_gbs"])
         decode["frac"] = round(decode["achieved"] / decode["peak"], 4)
@@ -380,15 +385,64 @@ def bench_decode(lcx, w, q, k, v, rope, stream, status, reps=20):
         b.record(stream)
         torch.cuda.synchronize()
         sweep[splits] = a.elapsed_time(b) / reps
-    assert int(status.item()) == 0, "device watchdog fired in decode"
     best = min(sweep, key=sweep.get)
+    # the same step on a cache of keys rotated beforehand (LCX_ATTN_PREROTATED_K)
+    k_rot = lcx.apply_rope(k, rope)
+    ws = torch.empty(max(1, lcx.split_workspace_bytes(w.B, w.Hq, 1, w.D, best)),
+                     dtype=torch.uint8, device=q.device)
+    for _ in range(3):
+        lcx.attn_fwd(qd, k_rot, v, rope, num_splits=best, workspace=ws, k_prerotated=True, **kw)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        lcx.attn_fwd(qd, k_rot, v, rope, num_splits=best, workspace=ws, k_prerotated=True, **kw)
+    b.record(stream)
+    torch.cuda.synchronize()
+    us_rot = a.elapsed_time(b) / reps * 1e3
+    del k_rot
+    assert int(status.item()) == 0, "device watchdog fired in decode"
     us = sweep[best] * 1e3
     return {"what": "1 new token per head (B=%d, Hq=%d) against %d cached keys, q_offset = "
                     "L - 1, keys rotated on chip" % (w.B, w.Hq, w.L),
             "bound": "hbm", "num_splits": best, "us_per_call": round(us, 2),
             "us_by_splits": {str(s_): round(t * 1e3, 2) for s_, t in sweep.items()},
             "bytes": nbytes, "achieved": round(nbytes / (us * 1e-6) / 1e9, 1), "unit": "GB/s",
-            "launches": (1 if best == 1 else 2) * reps}
+            "us_per_call_prerotated_keys": round(us_rot, 2),
+            "achieved_prerotated_keys": round(nbytes / (us_rot * 1e-6) / 1e9, 1),
+            "launches": (1 if best == 1 else 2) * reps * 2}
+
+
+def bench_mla(lcx, dev, stream, status, reps=5):
+    """Decoupled-RoPE prefill in DeepSeek-V2's head shape (q/k 128 + 64 rotary
+    dims with one shared rotary key, v 128): B 1, 16 heads, L 16384, YaRN s=16
+    from 4096, causal.  Algorithmic FLOPs: 2 (192 + 128) per visible pair and
+    head."""
+    B, H, L, Dc, Dr, Dv = 1, 16, 16384, 128, 64, 128
+    g = torch.Generator(device=dev).manual_seed(0)
+    q = torch.randn((B, H, L, Dc + Dr), generator=g, device=dev).bfloat16()
+    kc = torch.randn((B, H, L, Dc), generator=g, device=dev).bfloat16()
+    kr = torch.randn((B, 1, L, Dr), generator=g, device=dev).bfloat16()
+    v = torch.randn((B, H, L, Dv), generator=g, device=dev).bfloat16()
+    o = torch.empty((B, H, L, Dv), dtype=torch.bfloat16, device=dev)
+    rope = lcx.RopeParams("yarn", Dr, scale=16.0, original_max_pos=4096)
+    kw = dict(out=o, status=status, k_rope=kr)
+    for _ in range(2):
+        lcx.attn_fwd(q, kc, v, rope, **kw)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        lcx.attn_fwd(q, kc, v, rope, **kw)
+    b.record(stream)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, "device watchdog fired in the decoupled-RoPE run"
+    ms = a.elapsed_time(b) / reps
+    flops = 2 * (Dc + Dr + Dv) * visible_pairs(L) * B * H
+    return {"what": "decoupled RoPE prefill, B 1, 16 heads, L 16384, q/k 128+64 (shared rotary "
+                    "key), v 128, YaRN s=16", "ms_per_call": round(ms, 3),
+            "achieved": round(flops / (ms * 1e-3) / 1e12, 1), "unit": "TFLOP/s",
+            "launches": reps}
 
 
 def bench_reference(args, world, rank):
