@@ -919,9 +919,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float cl2 = p.c_log2;
             float m = -INFINITY, l = 0.f;
             bool ok = true;
+            // Split-KV (decode) tiles hold few queries: a warp whose 32 rows hold
+            // none only keeps step with the barriers, which leaves its SMSP to the
+            // rotation warp (its P rows are never used: their O rows are not stored).
+            const bool idle = kKvSplit && !__any_sync(0xffffffffu, rm.valid);
             for (int j = 0; j < T.n; ++j) {
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_ready[t], j & 1, abort, tmo));
                 if (!ok) break;
+                if (idle) {
+                    mbar_arrive(&bar.p_ready[t]);
+                    continue;
+                }
                 tc_fence_after();
                 const int jt = T.tile(j), k0 = jt * BN;
                 const bool partial = !tile_full<BN>(U.q0, jt, p);
