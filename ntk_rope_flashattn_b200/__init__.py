@@ -364,30 +364,77 @@ def attn_merge(o_parts, lse_parts, out=None, lse=None, dtype=None):
     return out, lse
 
 
-def attn_fwd_host(q, k, v, rope: RopeParams, device="cuda", workspace=None, **kw):
-    """attn_fwd on HOST tensors: copies q/k/v to the device (pinned memory makes
-    the copies asynchronous), runs the kernel and copies o back to the host.
+def attn_fwd_host(q, k, v, rope: RopeParams, device="cuda", workspace=None, chunks=8, **kw):
+    """attn_fwd on HOST tensors [B, H, L, D]: copies q/k/v to the device, runs
+    the kernel and copies o back to the host (pinned host memory makes the
+    copies asynchronous).
 
-    ``workspace`` (dict) keeps the device buffers between calls.
+    The work is cut into about ``chunks`` pieces of whole kv-head groups (one
+    batch entry at a time), and the pieces are pipelined over three streams:
+    while the kernel runs on piece c, the inputs of piece c + 1 travel to the
+    device and the output of piece c - 1 travels back.  Each piece is one
+    lcx_attn_fwd call on views of the device buffers, so the arithmetic is the
+    same as one call over everything.  ``workspace`` (dict) keeps the device
+    buffers and streams between calls.  Returns the pinned host o; the current
+    stream is ordered after the last copy.
     """
     import torch
     ws = workspace if workspace is not None else {}
+    B, Hq, L, D = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
     dev = {}
     for name, t in (("q", q), ("k", k), ("v", v)):
         buf = ws.get(name)
         if buf is None or buf.shape != t.shape or buf.dtype != t.dtype:
             buf = torch.empty(t.shape, dtype=t.dtype, device=device)
             ws[name] = buf
-        buf.copy_(t, non_blocking=True)
         dev[name] = buf
+    o_shape = (B, Hq, L, v.shape[3])
     o_dev = ws.get("o")
-    if o_dev is None or o_dev.shape != q.shape or o_dev.dtype != q.dtype:
-        o_dev = torch.empty(q.shape, dtype=q.dtype, device=device)
+    if o_dev is None or tuple(o_dev.shape) != o_shape or o_dev.dtype != q.dtype:
+        o_dev = torch.empty(o_shape, dtype=q.dtype, device=device)
         ws["o"] = o_dev
-    attn_fwd(dev["q"], dev["k"], dev["v"], rope, out=o_dev, **kw)
     o_host = ws.get("o_host")
-    if o_host is None or o_host.shape != q.shape or o_host.dtype != q.dtype:
-        o_host = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    if o_host is None or tuple(o_host.shape) != o_shape or o_host.dtype != q.dtype:
+        o_host = torch.empty(o_shape, dtype=q.dtype, pin_memory=True)
         ws["o_host"] = o_host
-    o_host.copy_(o_dev, non_blocking=True)
+    # pieces: (batch, first kv head, end kv head); one piece when the caller
+    # wants per-row statistics back (lse / status buffers cover everything)
+    per_b = max(1, min(Hkv, -(-int(chunks) // B)))
+    if "lse" in kw or kw.get("return_lse"):
+        pieces = [(None, 0, Hkv)]
+    else:
+        bounds = [round(i * Hkv / per_b) for i in range(per_b + 1)]
+        pieces = [(b, g0, g1) for b in range(B) for g0, g1 in zip(bounds, bounds[1:])
+                  if g1 > g0]
+
+    def view(t, b, h0, h1):
+        return t[:, h0:h1] if b is None else t[b:b + 1, h0:h1]
+
+    cur = torch.cuda.current_stream(device)
+    s_in = ws.setdefault("stream_in", torch.cuda.Stream(device))
+    s_out = ws.setdefault("stream_out", torch.cuda.Stream(device))
+    s_in.wait_stream(cur)
+    s_out.wait_stream(cur)
+    arrived = []
+    with torch.cuda.stream(s_in):
+        for b, g0, g1 in pieces:
+            view(dev["q"], b, g0 * G, g1 * G).copy_(view(q, b, g0 * G, g1 * G), non_blocking=True)
+            view(dev["k"], b, g0, g1).copy_(view(k, b, g0, g1), non_blocking=True)
+            view(dev["v"], b, g0, g1).copy_(view(v, b, g0, g1), non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(s_in)
+            arrived.append(ev)
+    for (b, g0, g1), ev in zip(pieces, arrived):
+        cur.wait_event(ev)
+        o_piece = view(o_dev, b, g0 * G, g1 * G)
+        attn_fwd(view(dev["q"], b, g0 * G, g1 * G), view(dev["k"], b, g0, g1),
+                 view(dev["v"], b, g0, g1), rope, out=o_piece, **kw)
+        done = torch.cuda.Event()
+        done.record(cur)
+        s_out.wait_event(done)
+        with torch.cuda.stream(s_out):
+            view(o_host, b, g0 * G, g1 * G).copy_(o_piece, non_blocking=True)
+    cur.wait_stream(s_out)
     return o_host

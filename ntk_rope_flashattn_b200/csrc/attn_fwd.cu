@@ -89,6 +89,7 @@ struct AttnParams {
     int rotate_q, rotate_k;
     int n_split;                       // key-range splits per unit (1: plain output)
     int pack_lp, pack_hpt;             // head-packed query tiles (split-KV only): rows
+    int pack_stride, pack_off;         // head k of tile t starts at row k stride + t off;
                                        // per head (multiple of 8), heads per tile; 0 = off
     float split_recip;                 // 1 / n_split, rounded up
     float *part_o;                     // n_split > 1: [n_split, B, Hq, L, D] partial o
@@ -386,21 +387,23 @@ __device__ __forceinline__ void rotate_row(uint8_t *tile, uint8_t *lo, int r, in
     }
 }
 
-// A head-packed query tile (decode): row r = k Lp + i holds query i of the
-// tile's k-th head, at position pos0 + i; only rows < rows_used hold data.
-// Each row's phasor is evaluated from its exact angle (once per CTA).
+// A head-packed query tile (decode): row off + k stride + i holds query i
+// (i < Lp) of the tile's k-th head (k < heads), at position pos0 + i; other
+// rows hold no data.  Each row's phasor comes from its exact angle (once per
+// CTA).
 template <int D, int RD, bool kHalf, bool kSplit>
 __device__ __forceinline__ void rotate_packed_q(uint8_t *tile, uint8_t *lo, long long pos0,
-                                                int Lp, int rows_used,
+                                                int Lp, int stride, int off, int heads,
                                                 const Phasor<RD, kHalf> &ph, const AttnParams &p,
                                                 bool rotate) {
     using R = Rot<RD, kHalf>;
     constexpr int NJ = kBM / R::RP;
     for (int k = 0; k < NJ; ++k) {
         const int r = ph.r0 + k * R::RP;
-        if (r >= rows_used) break;
+        const int rel = r - off;
+        if (rel < 0 || rel >= heads * stride || rel % stride >= Lp) continue;
         float c[R::PPJ], s[R::PPJ];
-        if (rotate) ph.template start<(RD < D)>(pos0 + (r % Lp) - ph.r0, p, c, s);
+        if (rotate) ph.template start<(RD < D)>(pos0 + rel % stride - ph.r0, p, c, s);
         rotate_row<D, RD, kHalf, kSplit, kBM * 128>(tile, lo, r, ph.q, c, s, rotate);
     }
 }
@@ -584,7 +587,10 @@ __device__ __forceinline__ void store_lse(const AttnParams &p, const Unit &U, in
 }
 
 // Query row `row` of tile t: its head, its query index and whether it holds a
-// query (head-packed tiles: row = k Lp + i for the tile's k-th head).
+// query.  Head-packed tiles: the tile's k-th head starts at row
+// k stride + t off (stride >= Lp rows per head; tile 1 shifted by a warp when
+// the room allows, so the few busy softmax warps of the two tiles sit on
+// different SMSPs).
 struct RowMap {
     int h, i;
     bool valid;
@@ -593,10 +599,11 @@ __device__ __forceinline__ RowMap map_row(const AttnParams &p, const Unit &U, in
                                           bool packed) {
     RowMap m;
     if (packed) {
-        const int k = row / p.pack_lp;
-        m.i = row - k * p.pack_lp;
+        const int rel = row - t * p.pack_off;
+        const int k = rel >= 0 ? rel / p.pack_stride : U.hpt;
+        m.i = rel - k * p.pack_stride;
         m.h = U.hq0 + t * U.hpt + k;
-        m.valid = k < U.hpt && m.i < p.L;
+        m.valid = rel >= 0 && k < U.hpt && m.i < p.L;
     } else {
         m.h = U.hq0 + t;
         m.i = U.q0 + row;
@@ -711,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int k = 0; k < U.hpt; ++k)
                             for (int bx = 0; bx < D / 64; ++bx)
                                 tma_load_4d(sQ + t * C::kParts * C::kTileQ + bx * C::kBoxQ +
-                                                k * p.pack_lp * 128,
+                                                (k * p.pack_stride + t * p.pack_off) * 128,
                                             &tmq, &bar.full_q, bx * 64, 0, U.hq0 + t * U.hpt + k,
                                             U.b);
                 } else {
@@ -852,8 +859,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t *qt = sQ + t * C::kParts * C::kTileQ;
                     if (packed)
                         rotate_packed_q<D, RD, kHalf, kSplit>(qt, qt + C::kTileQ, p.qoff,
-                                                              p.pack_lp, U.hpt * p.pack_lp, ph,
-                                                              p, rotq);
+                                                              p.pack_lp, p.pack_stride,
+                                                              t * p.pack_off, U.hpt, ph, p, rotq);
                     else
                         rotate_tile_bf16<D, RD, kHalf, kSplit, kBM>(
                             qt, qt + C::kTileQ, (long long)U.q0 + p.qoff, ph, p, rotq);
@@ -1391,6 +1398,11 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
     if (!x.f32 && x.p.G % 2 == 0 && x.D <= 128 && lp * (x.p.G / 2) <= kBM) {
         x.p.pack_lp = int(lp);
         x.p.pack_hpt = x.p.G / 2;
+        // Heads spread over the tile (multiples of 8 rows keep the 128-byte
+        // swizzle phase), and tile 1 shifted by one warp's 32 rows when that
+        // still fits, so the busy softmax warps of both tiles use different SMSPs.
+        x.p.pack_stride = (kBM / x.p.pack_hpt) / 8 * 8;
+        x.p.pack_off = (x.p.pack_stride - x.p.pack_lp >= 32) ? 32 : 0;
         x.p.heads_per_unit = x.p.G;
         x.p.n_qb = 1;
         x.p.units_per_qb = x.p.B * x.p.Hkv;

@@ -236,3 +236,21 @@ def test_attn_length_dependent_tables(mode):
                                       v.float().cpu().numpy(), table, ms, "half", 0, True,
                                       w.window, w.sinks)
     compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_lse)
+
+
+@pytest.mark.parametrize("chunks", [1, 3, 8])
+def test_attn_fwd_host_pipelined_equals_device_call(chunks):
+    """attn_fwd_host cuts the work into kv-head pieces pipelined over copy
+    streams; every row's arithmetic is that of one device call, bit for bit."""
+    w = BASE.with_(B=2, Hq=8, Hkv=4, L=600, mode="yarn", scale=8.0, original_max_pos=128,
+                   window=300, sinks=4)
+    q, k, v = make_inputs(w, device="cuda")
+    rope = rope_of(w)
+    ref = lcx.attn_fwd(q, k, v, rope, window=w.window, sinks=w.sinks)
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    ws = {}
+    for _ in range(2):                     # the second call reuses buffers and streams
+        oh = lcx.attn_fwd_host(qh, kh, vh, rope, device="cuda", workspace=ws, chunks=chunks,
+                               window=w.window, sinks=w.sinks)
+        torch.cuda.synchronize()
+        assert torch.equal(oh, ref.cpu())
