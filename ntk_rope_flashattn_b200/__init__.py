@@ -67,7 +67,8 @@ class _AttnArgs(ctypes.Structure):
                 ("softmax_scale", ctypes.c_float), ("flags", ctypes.c_uint32),
                 ("watchdog_ms", ctypes.c_int32), ("reserved0", ctypes.c_int32),
                 ("Lk", ctypes.c_int64), ("q_offset", ctypes.c_int64), ("Dv", ctypes.c_int64),
-                ("k_rope", ctypes.c_void_p), ("k_rope_strides", ctypes.c_int64 * 4)]
+                ("k_rope", ctypes.c_void_p), ("k_rope_strides", ctypes.c_int64 * 4),
+                ("k_rot", ctypes.c_void_p), ("k_rot_bytes", ctypes.c_int64)]
 
 
 @dataclass
@@ -216,7 +217,8 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
              softmax_scale: float = 0.0, return_lse: bool = False, prerotated: bool = False,
              split_qk: bool = False, out=None, lse=None, status=None, watchdog_ms: int = 0,
              q_offset: int = 0, k_prerotated: bool = False, num_splits: int = 1,
-             workspace=None, k_rope=None, _test_stall: bool = False):
+             workspace=None, k_rope=None, rotate_k_once: bool = False, k_rot=None,
+             _test_stall: bool = False):
     """Fused RoPE + causal attention (prefill, chunked prefill, decode).
 
     q [B, Hq, L, D], k/v [B, Hkv, Lk, D] CUDA tensors (bf16 or fp32, last dim
@@ -233,6 +235,10 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
     rope.head_dim dims of q and k; ``k_rope`` [B, 1, Lk, rope.head_dim] then
     supplies that part of every key once for all heads and k holds the first
     D - rope.head_dim dims.  v / o may have their own head dim (v.shape[-1]).
+    ``rotate_k_once`` (or a ``k_rot`` buffer shaped like k): the keys are
+    rotated once into that buffer by the rotate pass before the kernel, which
+    then reads them pre-rotated, instead of rotating each key tile on chip in
+    every CTA that reads it (ignored where the kernel does not rotate keys).
     ``split_qk`` forms QK^T from hi/lo bf16 parts of the rotated operands
     (LCX_ATTN_SPLIT_QK) for inputs whose large logits bf16 rounding would spoil.
     ``status`` (optional int32 CUDA tensor of one element) receives
@@ -276,6 +282,11 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
     a.Lk = Lk
     a.q_offset = int(q_offset)
     a.Dv = Dv
+    if rotate_k_once and k_rot is None:
+        k_rot = torch.empty((B, Hkv, Lk, Dk), dtype=k.dtype, device=k.device)
+    if k_rot is not None:
+        a.k_rot = k_rot.data_ptr()
+        a.k_rot_bytes = k_rot.numel() * k_rot.element_size()
     if k_rope is not None:
         a.k_rope = k_rope.data_ptr()
         a.k_rope_strides = _strides(k_rope)

@@ -125,10 +125,14 @@ struct Cfg {
     static constexpr int kOffV = kOffK + kStagesK * kParts * kTileK;
     static constexpr int kOffBar = kOffV + kStagesV * kTileV;
     static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers + alignment slack
-    // TMEM columns: S_t at t*BN (P_t aliased over its first BN/2 columns), O_t after.
-    static constexpr int kColO = 2 * BN;
+    // S buffers per query tile: the split mode's 64-key tiles leave TMEM room
+    // for two, so its S runs two key tiles ahead of PV.
+    static constexpr int kNB = kSplit ? 2 : 1;
+    // TMEM columns: S_t,b at (t kNB + b) BN (P_t,b aliased over its first BN/2
+    // columns), O_t after.
+    static constexpr int kColO = 2 * kNB * BN;
     static_assert(kSmemBytes <= 232448, "shared memory budget");
-    static_assert(2 * BN + 2 * DV <= 512, "TMEM budget");
+    static_assert(2 * kNB * BN + 2 * DV <= 512, "TMEM budget");
 };
 
 template <int NSK, int NSV>
@@ -136,7 +140,7 @@ struct Bars {
     uint64_t full_q, ready_q;
     uint64_t full_k[NSK], ready_k[NSK], empty_k[NSK];
     uint64_t full_v[NSV], empty_v[NSV];
-    uint64_t s_ready[2], p_ready[2], o_ready[2];
+    uint64_t s_ready[2][2], p_ready[2][2], pv_done[2], o_ready[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -658,8 +662,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bar.empty_v[s], 1);
         }
         for (int t = 0; t < 2; ++t) {
-            mbar_init(&bar.s_ready[t], 1);
-            mbar_init(&bar.p_ready[t], 128);
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&bar.s_ready[t][b], 1);
+                mbar_init(&bar.p_ready[t][b], 128);
+            }
+            mbar_init(&bar.pv_done[t], 1);
             mbar_init(&bar.o_ready[t], 1);
         }
         mbar_init(&bar.drain, 1);
@@ -777,10 +784,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t dq0 = sdesc_sw128(q_addr, 16, 1024);
                 const uint64_t dk0 = sdesc_sw128(k_addr, 16, 1024);
                 const uint64_t dv0 = sdesc_sw128(v_addr, C::kBoxK, 1024);
-                auto issue_s = [&](int t, int s) {
+                constexpr int NB = C::kNB;
+                auto issue_s = [&](int t, int s, int b) {
                     const uint64_t qa = dq0 + ((t * C::kParts * C::kTileQ) >> 4);
                     const uint64_t ka = dk0 + ((s * C::kParts * C::kTileK) >> 4);
-                    const uint32_t dst = tmem + t * BN;
+                    const uint32_t dst = tmem + (t * NB + b) * BN;
                     constexpr int NPROD = kSplit ? 3 : 1;
 #pragma unroll
                     for (int pr = 0; pr < NPROD; ++pr) {
@@ -795,45 +803,69 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 };
                 // O_t += P_t V: P from TMEM (BN/2 columns of bf16 pairs), V MN-major.
-                auto issue_pv = [&](int t, int s, bool acc) {
+                auto issue_pv = [&](int t, int s, int b, bool acc) {
                     const uint64_t va = dv0 + ((s * C::kTileV) >> 4);
-                    const uint32_t dst = tmem + C::kColO + t * DV, pa = tmem + t * BN;
+                    const uint32_t dst = tmem + C::kColO + t * DV, pa = tmem + (t * NB + b) * BN;
 #pragma unroll
                     for (int kk = 0; kk < BN / 16; ++kk)
                         mma_ts(dst, pa + kk * 8, va + ((kk * 2048) >> 4), kIdPV, (acc || kk > 0));
                 };
+                // S_t(j + NB) is issued after PV_t(j), into the buffer P_t(j)
+                // occupied (MMAs of one thread execute in order).  With NB = 1
+                // the order is PV0(j), S0(j+1), PV1(j), S1(j+1): one query tile's
+                // softmax overlaps the other tile's products.  With NB = 2 it is
+                // PV0(j), PV1(j), S0(j+2), S1(j+2), and a softmax never waits for
+                // its own previous PV.
                 bool ok = mbar_wait(&bar.ready_q, 0, abort, tmo);
-                if (ok) ok = mbar_wait(&bar.ready_k[0], 0, abort, tmo);
-                tc_fence_after();
-                if (ok) {
+                for (int jj = 0; ok && jj < NB && jj < T.n; ++jj) {
+                    ok = mbar_wait(&bar.ready_k[jj % NSK], (jj / NSK) & 1, abort, tmo);
+                    tc_fence_after();
+                    if (!ok) break;
                     for (int t = 0; t < U.nt; ++t) {
-                        issue_s(t, 0);
-                        mma_commit(&bar.s_ready[t]);
+                        issue_s(t, jj % NSK, jj % NB);
+                        mma_commit(&bar.s_ready[t][jj % NB]);
                     }
-                    mma_commit(&bar.empty_k[0]);
+                    mma_commit(&bar.empty_k[jj % NSK]);
                 }
                 for (int j = 0; ok && j < T.n; ++j) {
-                    const int sv = j % NSV;
+                    const int sv = j % NSV, jn = j + NB;
                     ok = mbar_wait(&bar.full_v[sv], (j / NSV) & 1, abort, tmo);
                     for (int t = 0; ok && t < U.nt; ++t) {
-                        ok = mbar_wait(&bar.p_ready[t], j & 1, abort, tmo);
+                        ok = mbar_wait(&bar.p_ready[t][j % NB], (j / NB) & 1, abort, tmo);
                         tc_fence_after();
                         if (!ok) break;
-                        issue_pv(t, sv, j > 0);
-                        if (j + 1 < T.n) {
-                            const int sk = (j + 1) % NSK;
+                        issue_pv(t, sv, j % NB, j > 0);
+                        if (NB > 1) {
+                            mma_commit(&bar.pv_done[t]);
+                        } else if (jn < T.n) {
+                            const int sk = jn % NSK;
                             if (t == 0) {
-                                ok = mbar_wait(&bar.ready_k[sk], ((j + 1) / NSK) & 1, abort, tmo);
+                                ok = mbar_wait(&bar.ready_k[sk], (jn / NSK) & 1, abort, tmo);
                                 tc_fence_after();
                                 if (!ok) break;
                             }
-                            issue_s(t, sk);
-                            mma_commit(&bar.s_ready[t]);
+                            issue_s(t, sk, jn % NB);
+                            mma_commit(&bar.s_ready[t][jn % NB]);
                         }
                     }
-                    if (ok) {
+                    // Two S buffers: both PVs of tile j go first and release their
+                    // V stage, so a key tile that is still being rotated holds back
+                    // only the S products.
+                    if (NB > 1 && ok) {
                         mma_commit(&bar.empty_v[sv]);
-                        if (j + 1 < T.n) mma_commit(&bar.empty_k[(j + 1) % NSK]);
+                        if (jn < T.n) {
+                            const int sk = jn % NSK;
+                            ok = mbar_wait(&bar.ready_k[sk], (jn / NSK) & 1, abort, tmo);
+                            tc_fence_after();
+                            for (int t = 0; ok && t < U.nt; ++t) {
+                                issue_s(t, sk, jn % NB);
+                                mma_commit(&bar.s_ready[t][jn % NB]);
+                            }
+                            if (ok) mma_commit(&bar.empty_k[sk]);
+                        }
+                    } else if (ok) {
+                        mma_commit(&bar.empty_v[sv]);
+                        if (jn < T.n) mma_commit(&bar.empty_k[jn % NSK]);
                     }
                 }
                 if (ok)
@@ -920,7 +952,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int wq = warp & 3;
             const int row = wq * 32 + lane;
             const uint32_t trow = tmem + (uint32_t(wq * 32) << 16);
-            const uint32_t s_col = t * BN, o_col = C::kColO + t * DV;
+            const uint32_t o_col = C::kColO + t * DV;
+            constexpr int NB = C::kNB;
             const RowMap rm = map_row(p, U, t, row, packed);
             const int pi = rm.i + p.qoff;  // this row's query position
             const float cl2 = p.c_log2;
@@ -931,10 +964,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             // rotation warp (its P rows are never used: their O rows are not stored).
             const bool idle = kKvSplit && !__any_sync(0xffffffffu, rm.valid);
             for (int j = 0; j < T.n; ++j) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_ready[t], j & 1, abort, tmo));
+                const int b = j % NB;
+                const uint32_t s_col = (t * NB + b) * BN;
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(&bar.s_ready[t][b], (j / NB) & 1, abort, tmo));
                 if (!ok) break;
                 if (idle) {
-                    mbar_arrive(&bar.p_ready[t]);
+                    mbar_arrive(&bar.p_ready[t][b]);
                     continue;
                 }
                 tc_fence_after();
@@ -961,6 +997,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // result is exact either way, only O's rescale is saved.
                 const bool need = (m != -INFINITY) && (m_new > m + kRescaleLog2);
                 if (__any_sync(0xffffffffu, need)) {
+                    if (NB > 1) {
+                        // O_t must not be in flight: wait for PV_t(j - 1), the j-th
+                        // completion of pv_done (S_t(j) done implies PV_t(j - 2) was,
+                        // and PV_t(j) needs this tile's P, so no other phase can be
+                        // pending).  With one S buffer, S_t(j) done implies it.
+                        ok = __all_sync(0xffffffffu,
+                                        mbar_wait(&bar.pv_done[t], (j - 1) & 1, abort, tmo));
+                        if (!ok) break;
+                        tc_fence_after();
+                    }
                     const float alpha = need ? ex2_approx(m - m_new) : 1.f;
     #pragma unroll 1
                     for (int c = 0; c < DV / 32; ++c) {
@@ -1005,7 +1051,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_st_row(trow + s_col, pk);
                 l += lsum.x + lsum.y;
                 tc_fence_before();
-                mbar_arrive(&bar.p_ready[t]);
+                mbar_arrive(&bar.p_ready[t][b]);
             }
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.o_ready[t], 0, abort, tmo));
             if (ok) {
@@ -1163,6 +1209,12 @@ struct AttnLaunch : AttnLaunchShape {
     AttnParams p;
     Maps m;
     long long units;  // CTAs without key splits
+    // Keys rotated once before the attention kernel (args.k_rot): the rotate
+    // pass reads k_src and writes the contiguous buffer the kernel then reads.
+    bool rotate_k_once;
+    lcx_rope_params rope;
+    const void *k_src;
+    int64_t k_src_strides[4];
 };
 
 // Validate `a` and fill `x`.  *noop is set for empty problems (B or L zero),
@@ -1232,18 +1284,38 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     if ((st = check_tensor(a->o, a->o_strides, es, "o")) != LCX_OK) return st;
     if (a->k_rope && (st = check_tensor(a->k_rope, a->k_rope_strides, es, "k_rope")) != LCX_OK)
         return st;
+    // Keys rotated once into args.k_rot (by the rotate pass, mscale included)
+    // instead of once per key tile per CTA: only where the kernel would
+    // otherwise rotate them on chip in the plain QK^T mode with full rotary.
+    const bool rotate_k_once =
+        a->k_rot != nullptr && !(a->flags & (LCX_ATTN_PREROTATED | LCX_ATTN_PREROTATED_K |
+                                             LCX_ATTN_SPLIT_QK | LCX_ATTN_TEST_STALL)) &&
+        !partial && !a->k_rope && a->D % 16 == 0;
+    const int64_t kst_rot[4] = {a->Hkv * Lk * a->D, Lk * a->D, a->D, 1};
+    if (rotate_k_once) {
+        if (!aligned16(a->k_rot)) return fail(LCX_ERR_UNSUPPORTED, "k_rot must be 16-byte aligned");
+        if (a->k_rot_bytes < a->B * a->Hkv * Lk * a->D * es)
+            return fail(LCX_ERR_INVALID_ARG, "k_rot holds %lld bytes; %lld needed",
+                        (long long)a->k_rot_bytes, (long long)(a->B * a->Hkv * Lk * a->D * es));
+    }
+    const void *kptr = rotate_k_once ? a->k_rot : a->k;
+    const int64_t *kst = rotate_k_once ? kst_rot : a->k_strides;
 
     memset(&x, 0, sizeof(x));
+    x.rotate_k_once = rotate_k_once;
+    x.rope = a->rope;
+    x.k_src = a->k;
+    for (int d = 0; d < 4; ++d) x.k_src_strides[d] = a->k_strides[d];
     AttnParams &p = x.p;
     p.q = static_cast<const char *>(a->q);
-    p.k = static_cast<const char *>(a->k);
+    p.k = static_cast<const char *>(kptr);
     p.v = static_cast<const char *>(a->v);
     p.o = static_cast<char *>(a->o);
     p.lse = a->lse;
     p.status = a->dev_status;
     for (int d = 0; d < 3; ++d) {
         p.qs[d] = a->q_strides[d];
-        p.ks[d] = a->k_strides[d];
+        p.ks[d] = kst[d];
         p.vs[d] = a->v_strides[d];
         p.os[d] = a->o_strides[d];
     }
@@ -1267,7 +1339,8 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     x.units = (long long)p.n_qb * p.units_per_qb;
     if (x.units > 0x7fffffffLL) return fail(LCX_ERR_UNSUPPORTED, "too many work units");
     p.rotate_q = (a->flags & LCX_ATTN_PREROTATED) ? 0 : 1;
-    p.rotate_k = (a->flags & (LCX_ATTN_PREROTATED | LCX_ATTN_PREROTATED_K)) ? 0 : 1;
+    p.rotate_k = (rotate_k_once || (a->flags & (LCX_ATTN_PREROTATED | LCX_ATTN_PREROTATED_K)))
+                     ? 0 : 1;
     float ms = 1.f;
     // The length-dependent modes see the whole context: the Lk keys.
     rope_table_unchecked(&a->rope, effective_seq_len(&a->rope, Lk), p.theta, &ms);
@@ -1306,7 +1379,7 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
         const int64_t dk = a->k_rope ? a->D - RD : a->D;   // columns k itself holds
         if ((st = make_map(&x.m.q, a->q, a->B, a->Hq, a->L, a->D, a->q_strides, 128, "q")) != LCX_OK)
             return st;
-        if ((st = make_map(&x.m.k, a->k, a->B, a->Hkv, Lk, dk, a->k_strides, bn, "k")) != LCX_OK)
+        if ((st = make_map(&x.m.k, kptr, a->B, a->Hkv, Lk, dk, kst, bn, "k")) != LCX_OK)
             return st;
         if ((st = make_map(&x.m.v, a->v, a->B, a->Hkv, Lk, Dv, a->v_strides, bn, "v")) != LCX_OK)
             return st;
@@ -1324,6 +1397,16 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
 lcx_status attn_enqueue(const AttnLaunch &x, cudaStream_t s) {
     const long long grid = x.units * x.p.n_split;
     if (grid > 0x7fffffffLL) return fail(LCX_ERR_UNSUPPORTED, "too many work units");
+    if (x.rotate_k_once) {
+        // the rotate pass over all keys (positions 0..Lk-1), same stream first
+        lcx_rope_params rp = x.rope;
+        if (rp.seq_len <= 0) rp.seq_len = x.p.Lk;   // the context of the call, as the kernel's
+        const int64_t kst[4] = {(int64_t)x.p.Hkv * x.p.Lk * x.D, (int64_t)x.p.Lk * x.D, x.D, 1};
+        const lcx_status st =
+            lcx_apply_rope(&rp, x.k_src, const_cast<char *>(x.p.k), x.f32 ? LCX_F32 : LCX_BF16,
+                           x.p.B, x.p.Hkv, x.p.Lk, x.k_src_strides, kst, 0, s);
+        if (st != LCX_OK) return st;
+    }
     const unsigned g = unsigned(grid);
     return x.p.n_split > 1 ? launch_shape<true>(x, x.m, x.p, g, s)
                            : launch_shape<false>(x, x.m, x.p, g, s);

@@ -68,7 +68,8 @@ int main(void) {
   P(lcx_attn_args, window) P(lcx_attn_args, sinks) P(lcx_attn_args, softmax_scale)
   P(lcx_attn_args, flags) P(lcx_attn_args, watchdog_ms) P(lcx_attn_args, reserved0)
   P(lcx_attn_args, Lk) P(lcx_attn_args, q_offset) P(lcx_attn_args, Dv)
-  P(lcx_attn_args, k_rope) P(lcx_attn_args, k_rope_strides)
+  P(lcx_attn_args, k_rope) P(lcx_attn_args, k_rope_strides) P(lcx_attn_args, k_rot)
+  P(lcx_attn_args, k_rot_bytes)
   return 0;
 }
 ''')
@@ -241,6 +242,8 @@ def _attn_args(**kw):
     (dict(rope=_params("plain", 64), flags=2), lcx.LCX_ERR_UNSUPPORTED),   # partial split
     (dict(k_rope=0x500000), lcx.LCX_ERR_INVALID_ARG),                 # k_rope, full rotary
     (dict(D=192, rope=_params("plain", 192)), lcx.LCX_ERR_UNSUPPORTED),
+    (dict(k_rot=0x500008, k_rot_bytes=1 << 30), lcx.LCX_ERR_UNSUPPORTED),  # misaligned
+    (dict(k_rot=0x500000, k_rot_bytes=1000), lcx.LCX_ERR_INVALID_ARG),      # too small
     (dict(D=192, Dv=128, rope=_params("plain", 64), k_rope=0x500008,
           k_rope_strides=[256 * 64, 256 * 64, 64, 1]), lcx.LCX_ERR_UNSUPPORTED),  # misaligned
 ])

@@ -254,3 +254,38 @@ def test_attn_fwd_host_pipelined_equals_device_call(chunks):
                                window=w.window, sinks=w.sinks)
         torch.cuda.synchronize()
         assert torch.equal(oh, ref.cpu())
+
+
+@pytest.mark.parametrize("name", ["L1", "L127_yarn_G2", "L1000_window_sinks", "L700_D64",
+                                  "L400_interleaved", "L600_f32", "L2048_outliers_split",
+                                  "L300_pi_MHA_B2"])
+def test_attn_rotate_keys_once(name):
+    """Keys rotated once into a buffer by the rotate pass (args.k_rot) before
+    the kernel, instead of per key tile on chip: same parity (split-QK^T cases
+    keep the on-chip rotation and must be unaffected)."""
+    full_check(BASE.with_(**SMALL[name]), rotate_k_once=True)
+
+
+@pytest.mark.parametrize("mode,kw", [("dynamic_ntk", dict(original_max_pos=256)),
+                                     ("yarn", dict(scale=8.0, original_max_pos=128))])
+def test_attn_rotate_keys_once_decode_and_split(mode, kw):
+    """Rotate-once keys with a query offset (the rotate pass covers every key at
+    its own position; dynamic NTK sees the call's Lk) and with split-KV."""
+    w = BASE.with_(L=900, mode=mode, window=400, sinks=4, **kw)
+    q, k, v = make_inputs(w, device="cuda")
+    rope = rope_of(w)
+    table, ms, _ = oracle.rope_table(w.mode, w.D, w.base, w.scale, w.original_max_pos,
+                                     w.alpha, w.beta, seq_len=w.L)
+    a = 880
+    qs = q[:, :, a:]
+    bb, hh, ii = np.meshgrid(np.arange(w.B), np.arange(w.Hq), np.arange(w.L - a), indexing="ij")
+    ref_o, ref_lse = oracle.attn_rows(qs.float().cpu().numpy().reshape(-1, w.D), bb.ravel(),
+                                      hh.ravel(), ii.ravel() + a, k.float().cpu().numpy(),
+                                      v.float().cpu().numpy(), w.Hq, table, ms, "half", 0, True,
+                                      w.window, w.sinks)
+    for splits in (1, 4):
+        o, lse = lcx.attn_fwd(qs, k, v, rope, window=w.window, sinks=w.sinks, q_offset=a,
+                              rotate_k_once=True, num_splits=splits, return_lse=True)
+        torch.cuda.synchronize()
+        compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o.reshape(o.shape),
+                ref_lse.reshape(lse.shape))
