@@ -2,9 +2,12 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
-One step = one pass of the hot path over one batch of the workload: the RoPE
-table for the mode (host) and the fused rotate + QK^T + online softmax + PV
-kernel (lcx_attn_fwd).  Prints ONE JSON line (rank 0).
+One step = one pass of the hot path over one batch of the workload, one
+lcx_attn_fwd call: the RoPE table for the mode (host), the rotate pass over the
+keys into a buffer (args.k_rot: every key rotated once, mscale included), and
+the fused kernel (queries rotated on chip, QK^T, online softmax, PV).  In the
+split-QK^T mode the keys are rotated on chip instead.  Prints ONE JSON line
+(rank 0).
 
 * value      : attention TFLOP/s, algorithmic FLOPs = 4 * D * (visible query/key
                pairs) * B * Hq summed over all ranks, divided by the max over ranks
@@ -42,9 +45,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
 # launch on the headline workload (yarn_L131072_s16), from a one-pass ncu capture
-# of the current kernel: 3.00 GB read + 1.07 GB written (algorithmic: q, k, v
-# read once = 1.61 GB, o written once = 1.07 GB).  Only valid for that workload.
-ATTN_TRAFFIC_BYTES = {"yarn_L131072_s16": 4.07e9}
+# of the current kernel (keys pre-rotated by the rotate pass): 2.97 GB read +
+# 1.07 GB written (algorithmic: q, k, v read once = 1.61 GB, o written once =
+# 1.07 GB).  Only valid for that workload.
+ATTN_TRAFFIC_BYTES = {"yarn_L131072_s16": 4.04e9}
 
 
 def load_peaks():
@@ -211,8 +215,11 @@ def bench_gpu(args, world, rank, local):
                           w.pairing)
     o = torch.empty_like(q)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
+    # keys rotated once per step into k_rot (the library ignores it in split-QK^T mode)
+    rotate_once = not w.split_qk
+    k_rot = torch.empty_like(k) if rotate_once else None
     kw = dict(causal=w.causal, window=w.window, sinks=w.sinks, softmax_scale=w.softmax_scale,
-              split_qk=w.split_qk, out=o, status=status)
+              split_qk=w.split_qk, out=o, status=status, k_rot=k_rot)
     stream = torch.cuda.current_stream(dev)
 
     def step():
@@ -261,6 +268,16 @@ def bench_gpu(args, world, rank, local):
         rope_ev.append((a, b))
     torch.cuda.synchronize()
     rope_ms = statistics.median(a.elapsed_time(b) for a, b in rope_ev)
+    # the keys' rotate pass alone (part of every step when rotate_once)
+    k_ev = []
+    for _ in range(max(3, args.steps)):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        lcx.apply_rope(k, rope, out=kr)
+        b.record(stream)
+        k_ev.append((a, b))
+    torch.cuda.synchronize()
+    k_rope_ms = statistics.median(a.elapsed_time(b) for a, b in k_ev) if rotate_once else 0.0
     del qr, kr
 
     # --- split-KV decode: one new token per query head against the whole cache
@@ -273,7 +290,7 @@ def bench_gpu(args, world, rank, local):
     for _ in range(max(1, min(args.warmup, 2))):
         lcx.attn_fwd_host(qh, kh, vh, rope, device=dev, workspace=ws, causal=w.causal,
                           window=w.window, sinks=w.sinks, softmax_scale=w.softmax_scale,
-                          split_qk=w.split_qk)
+                          split_qk=w.split_qk, rotate_k_once=rotate_once)
     torch.cuda.synchronize()
     barrier(world)
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -281,7 +298,7 @@ def bench_gpu(args, world, rank, local):
     for _ in range(args.steps):
         oh = lcx.attn_fwd_host(qh, kh, vh, rope, device=dev, workspace=ws, causal=w.causal,
                                window=w.window, sinks=w.sinks, softmax_scale=w.softmax_scale,
-                               split_qk=w.split_qk)
+                               split_qk=w.split_qk, rotate_k_once=rotate_once)
     e_end.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), world)
@@ -291,7 +308,8 @@ def bench_gpu(args, world, rank, local):
     del qh, kh, vh, ws
 
     peaks, peak_src = load_peaks()
-    avg_launch = statistics.mean(launch_ms)
+    # the attention kernel's own time: the step minus the keys' rotate pass
+    avg_launch = statistics.mean(launch_ms) - k_rope_ms
     achieved = flops_rank / (avg_launch * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops_sustained"])
     rope_gbs = rope_bytes(w) / (rope_ms * 1e-3) / 1e9
@@ -320,7 +338,7 @@ def bench_gpu(args, world, rank, local):
                 sum(t.numel() * t.element_size() for t in (q, k, v)) / 1e9),
             "parallelism": "replicas x%d (independent batches, no collective)" % world,
         },
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * (2 if rotate_once else 1),
         "roofline": {
             "bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
             "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
@@ -330,6 +348,7 @@ def bench_gpu(args, world, rank, local):
             "algorithmic_bytes": (sum(t.numel() * t.element_size() for t in (q, k, v))
                                   + o.numel() * o.element_size()),
             "kernel": "attn_fwd_kernel", "avg_launch_ms": round(avg_launch, 3),
+            "k_rotate_pass_ms": round(k_rope_ms, 4),
             "launch_ms": [round(x, 3) for x in launch_ms],
         },
         "apply_rope": {
