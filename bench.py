@@ -6,8 +6,8 @@ One step = one pass of the hot path over one batch of the workload, one
 lcx_attn_fwd call: the RoPE table for the mode (host), the rotate pass over the
 keys into a buffer (args.k_rot: every key rotated once, mscale included), and
 the fused kernel (queries rotated on chip, QK^T, online softmax, PV).  In the
-split-QK^T mode the keys are rotated on chip instead.  Prints ONE JSON line
-(rank 0).
+split-QK^T mode the pass writes the keys as hi/lo bf16 parts.  Prints ONE
+JSON line (rank 0).
 
 * value      : attention TFLOP/s, algorithmic FLOPs = 4 * D * (visible query/key
                pairs) * B * Hq summed over all ranks, divided by the max over ranks
@@ -215,9 +215,10 @@ def bench_gpu(args, world, rank, local):
                           w.pairing)
     o = torch.empty_like(q)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    # keys rotated once per step into k_rot (the library ignores it in split-QK^T mode)
-    rotate_once = not w.split_qk
-    k_rot = torch.empty_like(k) if rotate_once else None
+    # keys rotated once per step into k_rot (split-QK^T with bf16 keys: hi then lo parts)
+    rotate_once = True
+    parts = 2 if (w.split_qk and k.dtype == torch.bfloat16) else 1
+    k_rot = torch.empty((parts,) + tuple(k.shape), dtype=k.dtype, device=dev)
     kw = dict(causal=w.causal, window=w.window, sinks=w.sinks, softmax_scale=w.softmax_scale,
               split_qk=w.split_qk, out=o, status=status, k_rot=k_rot)
     stream = torch.cuda.current_stream(dev)

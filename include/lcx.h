@@ -195,14 +195,18 @@ typedef struct {
     int64_t k_rope_strides[4]; /* elements; the head stride is not used        */
     void *k_rot;               /* DEVICE scratch or NULL.  When set, and the keys
                                   would be rotated on chip (no PREROTATED flags,
-                                  plain QK^T, every dim rotated, no k_rope), the
-                                  keys are rotated once into it by the rotate pass
-                                  of lcx_apply_rope (mscale included) and the
+                                  every dim rotated, no k_rope), the keys are
+                                  rotated once into it by the rotate pass of
+                                  lcx_apply_rope (mscale included) and the
                                   attention kernel reads them from there: one
                                   rotation per key instead of one per key tile
                                   and CTA.  Contiguous [B, Hkv, Lk, D] of dtype;
-                                  16-byte aligned.  Ignored otherwise          */
-    int64_t k_rot_bytes;       /* bytes at k_rot (>= B*Hkv*Lk*D*element size)  */
+                                  in the split-QK^T mode with bf16 operands the
+                                  hi parts, then the lo parts (bf16 of the
+                                  rounding residual).  16-byte aligned.  Ignored
+                                  otherwise                                    */
+    int64_t k_rot_bytes;       /* bytes at k_rot: >= B*Hkv*Lk*D*element size,
+                                  twice that for split-QK^T with bf16          */
 } lcx_attn_args;
 
 /*

@@ -235,10 +235,11 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
     rope.head_dim dims of q and k; ``k_rope`` [B, 1, Lk, rope.head_dim] then
     supplies that part of every key once for all heads and k holds the first
     D - rope.head_dim dims.  v / o may have their own head dim (v.shape[-1]).
-    ``rotate_k_once`` (or a ``k_rot`` buffer shaped like k): the keys are
-    rotated once into that buffer by the rotate pass before the kernel, which
-    then reads them pre-rotated, instead of rotating each key tile on chip in
-    every CTA that reads it (ignored where the kernel does not rotate keys).
+    ``rotate_k_once`` (or a ``k_rot`` buffer shaped like k, twice that in the
+    split-QK^T mode with bf16 keys): the keys are rotated once into that buffer
+    by the rotate pass before the kernel, which then reads them pre-rotated
+    (split mode: as hi/lo bf16 parts), instead of rotating each key tile on chip
+    in every CTA that reads it (ignored where the kernel does not rotate keys).
     ``split_qk`` forms QK^T from hi/lo bf16 parts of the rotated operands
     (LCX_ATTN_SPLIT_QK) for inputs whose large logits bf16 rounding would spoil.
     ``status`` (optional int32 CUDA tensor of one element) receives
@@ -283,7 +284,9 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
     a.q_offset = int(q_offset)
     a.Dv = Dv
     if rotate_k_once and k_rot is None:
-        k_rot = torch.empty((B, Hkv, Lk, Dk), dtype=k.dtype, device=k.device)
+        # split QK^T with bf16 keys: the pass writes hi parts, then lo parts
+        parts = 2 if (split_qk and k.dtype == torch.bfloat16) else 1
+        k_rot = torch.empty((parts, B, Hkv, Lk, Dk), dtype=k.dtype, device=k.device)
     if k_rot is not None:
         a.k_rot = k_rot.data_ptr()
         a.k_rot_bytes = k_rot.numel() * k_rot.element_size()

@@ -24,6 +24,7 @@ constexpr int kMaxHalf = 256;  // head_dim <= 512
 struct RopeArgs {
     const char *x;
     char *y;
+    char *y_lo;                  // bf16 only, or NULL: y_lo = bf16(y' - bf16(y'))
     long long xs_b, xs_h, xs_l;  // element strides
     long long ys_b, ys_h, ys_l;
     int H, L;
@@ -70,6 +71,28 @@ __device__ __forceinline__ uint4 pack(const float (&y)[8]) {
 __device__ __forceinline__ uint4 pack(const float (&y)[4]) {
     return make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]), __float_as_uint(y[2]),
                       __float_as_uint(y[3]));
+}
+
+// The residual of the bf16 rounding, y - bf16(y), rounded to bf16 again: the
+// "lo" half of a hi/lo pair (hi + lo carries y to ~16 significant bits).  Same
+// layout as y; e2 < 0 means only the vector at e1 exists.
+template <int N>
+__device__ __forceinline__ void store_lo(const RopeArgs &a, int b, int l, int h, int e1, int e2,
+                                         const float (&y1)[N], const float (&y2)[N],
+                                         const uint4 &h1, const uint4 &h2) {
+    __nv_bfloat16 *lr = reinterpret_cast<__nv_bfloat16 *>(
+        a.y_lo + 2 * (b * a.ys_b + l * a.ys_l + (long long)h * a.ys_h));
+    float r1[8], r2[8], f[8];
+    unpack(h1, f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) r1[e] = y1[e] - f[e];
+    __stcs(reinterpret_cast<uint4 *>(lr + e1), pack(r1));
+    if (e2 >= 0) {
+        unpack(h2, f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) r2[e] = y2[e] - f[e];
+        __stcs(reinterpret_cast<uint4 *>(lr + e2), pack(r2));
+    }
 }
 
 // HALF pairing: a job covers N consecutive pairs i0..i0+N-1, i.e. the vector
@@ -128,8 +151,11 @@ __global__ void __launch_bounds__(256) apply_rope_kernel(const __grid_constant__
                     y1[e] = fmaf(x1[e], c[e], -x2[e] * s[e]);
                     y2[e] = fmaf(x1[e], s[e], x2[e] * c[e]);
                 }
-                __stcs(reinterpret_cast<uint4 *>(yr + e1), pack(y1));
-                __stcs(reinterpret_cast<uint4 *>(yr + e2), pack(y2));
+                const uint4 h1 = pack(y1), h2 = pack(y2);
+                __stcs(reinterpret_cast<uint4 *>(yr + e1), h1);
+                __stcs(reinterpret_cast<uint4 *>(yr + e2), h2);
+                if constexpr (sizeof(T) == 2)
+                    if (a.y_lo) store_lo(a, b, l, h0 + u, e1, e2, y1, y2, h1, h2);
             } else {
                 float x[N], y[N];
                 unpack(va[u], x);
@@ -138,21 +164,21 @@ __global__ void __launch_bounds__(256) apply_rope_kernel(const __grid_constant__
                     y[2 * e] = fmaf(x[2 * e], c[e], -x[2 * e + 1] * s[e]);
                     y[2 * e + 1] = fmaf(x[2 * e], s[e], x[2 * e + 1] * c[e]);
                 }
-                __stcs(reinterpret_cast<uint4 *>(yr + e1), pack(y));
+                const uint4 h = pack(y);
+                __stcs(reinterpret_cast<uint4 *>(yr + e1), h);
+                if constexpr (sizeof(T) == 2)
+                    if (a.y_lo) store_lo(a, b, l, h0 + u, e1, -1, y, y, h, h);
             }
         }
     }
 }
 
 }  // namespace
-}  // namespace lcx
 
-extern "C" lcx_status lcx_apply_rope(const lcx_rope_params *params, const void *x, void *y,
-                                     int32_t dtype, int64_t B, int64_t H, int64_t L,
-                                     const int64_t *x_strides, const int64_t *y_strides,
-                                     int64_t pos_offset, void *stream) {
-    using namespace lcx;
-    clear_error();
+lcx_status apply_rope_impl(const lcx_rope_params *params, const void *x, void *y, void *y_lo,
+                           int32_t dtype, int64_t B, int64_t H, int64_t L,
+                           const int64_t *x_strides, const int64_t *y_strides, int64_t pos_offset,
+                           cudaStream_t s) {
     lcx_status st = check_rope_params(params);
     if (st != LCX_OK) return st;
     if (dtype != LCX_BF16 && dtype != LCX_F32)
@@ -180,8 +206,9 @@ extern "C" lcx_status lcx_apply_rope(const lcx_rope_params *params, const void *
         if (x_strides[d] % vec != 0 || ys[d] % vec != 0)
             return fail(LCX_ERR_UNSUPPORTED, "strides must be multiples of 16 bytes");
     }
-    if (!aligned16(x) || !aligned16(y))
+    if (!aligned16(x) || !aligned16(y) || !aligned16(y_lo))
         return fail(LCX_ERR_UNSUPPORTED, "x and y must be 16-byte aligned");
+    if (y_lo && dtype != LCX_BF16) return fail(LCX_ERR_UNSUPPORTED, "a lo part needs bf16");
     if (x == y) {
         for (int d = 0; d < 3; ++d)
             if (x_strides[d] != ys[d])
@@ -191,6 +218,7 @@ extern "C" lcx_status lcx_apply_rope(const lcx_rope_params *params, const void *
     RopeArgs a;
     a.x = static_cast<const char *>(x);
     a.y = static_cast<char *>(y);
+    a.y_lo = static_cast<char *>(y_lo);
     a.xs_b = x_strides[0];
     a.xs_h = x_strides[1];
     a.xs_l = x_strides[2];
@@ -207,7 +235,6 @@ extern "C" lcx_status lcx_apply_rope(const lcx_rope_params *params, const void *
     if (a.rows_per_cta < 1) a.rows_per_cta = 1;
     const int threads = a.rows_per_cta * a.jobs_per_row;
     dim3 grid(unsigned((L + a.rows_per_cta - 1) / a.rows_per_cta), unsigned(B));
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (dtype == LCX_BF16) {
         if (half)
             apply_rope_kernel<__nv_bfloat16, true><<<grid, threads, 0, s>>>(a);
@@ -223,4 +250,15 @@ extern "C" lcx_status lcx_apply_rope(const lcx_rope_params *params, const void *
     if (e != cudaSuccess)
         return fail(LCX_ERR_CUDA, "apply_rope launch failed: %s", cudaGetErrorString(e));
     return LCX_OK;
+}
+
+}  // namespace lcx
+
+extern "C" lcx_status lcx_apply_rope(const lcx_rope_params *params, const void *x, void *y,
+                                     int32_t dtype, int64_t B, int64_t H, int64_t L,
+                                     const int64_t *x_strides, const int64_t *y_strides,
+                                     int64_t pos_offset, void *stream) {
+    lcx::clear_error();
+    return lcx::apply_rope_impl(params, x, y, nullptr, dtype, B, H, L, x_strides, y_strides,
+                                pos_offset, static_cast<cudaStream_t>(stream));
 }

@@ -96,6 +96,7 @@ struct AttnParams {
     float *part_lse;                   //              [n_split, B, Hq, L] partial lse
     int test_stall;                    // loader issues nothing (watchdog test hook)
     int k_rope_shared;                 // rotated key columns come from one shared head
+    int k_lo_tma;                      // split mode: the keys' lo parts arrive by TMA
     float rot_ms;                      // factor on rotated values (partial rotary: mscale)
     float c_log2;                      // logit scale in log2 units
     unsigned long long timeout_ns;
@@ -710,7 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_prefetch_desc(&tmq);
                 tma_prefetch_desc(&tmk);
                 tma_prefetch_desc(&tmv);
-                if (RD < D && p.k_rope_shared) tma_prefetch_desc(&tmkr);
+                if ((RD < D && p.k_rope_shared) || p.k_lo_tma) tma_prefetch_desc(&tmkr);
                 // With a shared rotary key, the K boxes from column D - RD on
                 // come from that tensor's single head.
                 constexpr int kNopeBoxes = (D - RD) / 64;
@@ -741,7 +742,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int sk = j % NSK, uk = j / NSK, sv = j % NSV, uv = j / NSV;
                     if (uk > 0) ok = mbar_wait(&bar.empty_k[sk], (uk - 1) & 1, abort, tmo);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(&bar.full_k[sk], C::kTileK);
+                    // split mode with keys split by the rotate pass: the lo part
+                    // (fourth tensor map) lands in the stage's second part
+                    const bool lo = kSplit && p.k_lo_tma;
+                    mbar_arrive_expect_tx(&bar.full_k[sk], lo ? 2 * C::kTileK : C::kTileK);
+                    if (lo)
+                        for (int bx = 0; bx < D / 64; ++bx)
+                            tma_load_4d(sK + sk * C::kParts * C::kTileK + C::kTileK + bx * C::kBoxK,
+                                        &tmkr, &bar.full_k[sk], bx * 64, jt * BN, U.g, U.b);
                     for (int bx = 0; bx < D / 64; ++bx) {
                         uint8_t *dst = sK + sk * C::kParts * C::kTileK + bx * C::kBoxK;
                         if constexpr (RD < D) {
@@ -816,9 +824,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // softmax overlaps the other tile's products.  With NB = 2 it is
                 // PV0(j), PV1(j), S0(j+2), S1(j+2), and a softmax never waits for
                 // its own previous PV.
+                // Keys already rotated (and no hi/lo split) need no pass through
+                // the rotation warpgroup: the MMA waits for the TMA itself.
+                uint64_t *kready = (kF32 || (kSplit && !p.k_lo_tma) || p.rotate_k) ? bar.ready_k
+                                                                                    : bar.full_k;
                 bool ok = mbar_wait(&bar.ready_q, 0, abort, tmo);
                 for (int jj = 0; ok && jj < NB && jj < T.n; ++jj) {
-                    ok = mbar_wait(&bar.ready_k[jj % NSK], (jj / NSK) & 1, abort, tmo);
+                    ok = mbar_wait(&kready[jj % NSK], (jj / NSK) & 1, abort, tmo);
                     tc_fence_after();
                     if (!ok) break;
                     for (int t = 0; t < U.nt; ++t) {
@@ -840,7 +852,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         } else if (jn < T.n) {
                             const int sk = jn % NSK;
                             if (t == 0) {
-                                ok = mbar_wait(&bar.ready_k[sk], (jn / NSK) & 1, abort, tmo);
+                                ok = mbar_wait(&kready[sk], (jn / NSK) & 1, abort, tmo);
                                 tc_fence_after();
                                 if (!ok) break;
                             }
@@ -855,7 +867,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_commit(&bar.empty_v[sv]);
                         if (jn < T.n) {
                             const int sk = jn % NSK;
-                            ok = mbar_wait(&bar.ready_k[sk], (jn / NSK) & 1, abort, tmo);
+                            ok = mbar_wait(&kready[sk], (jn / NSK) & 1, abort, tmo);
                             tc_fence_after();
                             for (int t = 0; ok && t < U.nt; ++t) {
                                 issue_s(t, sk, jn % NB);
@@ -910,7 +922,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             mbar_arrive(&bar.ready_q);
         }
-        for (int j = 0; ok && j < T.n; ++j) {
+        // bf16 keys that are already rotated go straight from the TMA to the MMA
+        const bool relay_k = kF32 || (kSplit && !p.k_lo_tma) || rotk;
+        for (int j = 0; ok && relay_k && j < T.n; ++j) {
             const int jt = T.tile(j);
             const int s = j % NSK, use = j / NSK, sv = j % NSV, usev = j / NSV;
             uint8_t *tk = sK + s * C::kParts * C::kTileK;
@@ -1215,6 +1229,7 @@ struct AttnLaunch : AttnLaunchShape {
     lcx_rope_params rope;
     const void *k_src;
     int64_t k_src_strides[4];
+    void *k_lo;       // split mode: where the pass writes the keys' lo parts, or NULL
 };
 
 // Validate `a` and fill `x`.  *noop is set for empty problems (B or L zero),
@@ -1287,22 +1302,28 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     // Keys rotated once into args.k_rot (by the rotate pass, mscale included)
     // instead of once per key tile per CTA: only where the kernel would
     // otherwise rotate them on chip in the plain QK^T mode with full rotary.
+    // In the split-QK^T mode with bf16 keys the pass also writes the lo parts
+    // (bf16 of the rounding residual) right after the hi parts.
     const bool rotate_k_once =
         a->k_rot != nullptr && !(a->flags & (LCX_ATTN_PREROTATED | LCX_ATTN_PREROTATED_K |
-                                             LCX_ATTN_SPLIT_QK | LCX_ATTN_TEST_STALL)) &&
+                                             LCX_ATTN_TEST_STALL)) &&
         !partial && !a->k_rope && a->D % 16 == 0;
+    const bool k_lo = rotate_k_once && (a->flags & LCX_ATTN_SPLIT_QK) && a->dtype == LCX_BF16;
     const int64_t kst_rot[4] = {a->Hkv * Lk * a->D, Lk * a->D, a->D, 1};
+    const int64_t k_part_bytes = a->B * a->Hkv * Lk * a->D * es;
     if (rotate_k_once) {
         if (!aligned16(a->k_rot)) return fail(LCX_ERR_UNSUPPORTED, "k_rot must be 16-byte aligned");
-        if (a->k_rot_bytes < a->B * a->Hkv * Lk * a->D * es)
+        if (a->k_rot_bytes < k_part_bytes * (k_lo ? 2 : 1))
             return fail(LCX_ERR_INVALID_ARG, "k_rot holds %lld bytes; %lld needed",
-                        (long long)a->k_rot_bytes, (long long)(a->B * a->Hkv * Lk * a->D * es));
+                        (long long)a->k_rot_bytes, (long long)(k_part_bytes * (k_lo ? 2 : 1)));
     }
+    void *k_lo_ptr = k_lo ? static_cast<char *>(a->k_rot) + k_part_bytes : nullptr;
     const void *kptr = rotate_k_once ? a->k_rot : a->k;
     const int64_t *kst = rotate_k_once ? kst_rot : a->k_strides;
 
     memset(&x, 0, sizeof(x));
     x.rotate_k_once = rotate_k_once;
+    x.k_lo = k_lo_ptr;
     x.rope = a->rope;
     x.k_src = a->k;
     for (int d = 0; d < 4; ++d) x.k_src_strides[d] = a->k_strides[d];
@@ -1358,6 +1379,7 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     }
     p.c_log2 = float(scale * msq * 1.4426950408889634);
     p.k_rope_shared = a->k_rope ? 1 : 0;
+    p.k_lo_tma = k_lo ? 1 : 0;
     // Legitimate waits last microseconds; the default limit is 2 s.
     p.timeout_ns = 1000000ull * (unsigned long long)(a->watchdog_ms > 0 ? a->watchdog_ms : 2000);
     p.test_stall = (a->flags & LCX_ATTN_TEST_STALL) ? 1 : 0;
@@ -1383,6 +1405,11 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
             return st;
         if ((st = make_map(&x.m.v, a->v, a->B, a->Hkv, Lk, Dv, a->v_strides, bn, "v")) != LCX_OK)
             return st;
+        if (k_lo) {
+            if ((st = make_map(&x.m.kr, k_lo_ptr, a->B, a->Hkv, Lk, a->D, kst_rot, bn, "k_lo")) !=
+                LCX_OK)
+                return st;
+        }
         if (a->k_rope) {
             // one head: the head stride never matters, any valid value will do
             int64_t krs[4] = {a->k_rope_strides[0], Lk * RD, a->k_rope_strides[2], 1};
@@ -1403,8 +1430,9 @@ lcx_status attn_enqueue(const AttnLaunch &x, cudaStream_t s) {
         if (rp.seq_len <= 0) rp.seq_len = x.p.Lk;   // the context of the call, as the kernel's
         const int64_t kst[4] = {(int64_t)x.p.Hkv * x.p.Lk * x.D, (int64_t)x.p.Lk * x.D, x.D, 1};
         const lcx_status st =
-            lcx_apply_rope(&rp, x.k_src, const_cast<char *>(x.p.k), x.f32 ? LCX_F32 : LCX_BF16,
-                           x.p.B, x.p.Hkv, x.p.Lk, x.k_src_strides, kst, 0, s);
+            apply_rope_impl(&rp, x.k_src, const_cast<char *>(x.p.k), x.k_lo,
+                            x.f32 ? LCX_F32 : LCX_BF16, x.p.B, x.p.Hkv, x.p.Lk, x.k_src_strides,
+                            kst, 0, s);
         if (st != LCX_OK) return st;
     }
     const unsigned g = unsigned(grid);

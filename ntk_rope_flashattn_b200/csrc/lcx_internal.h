@@ -32,6 +32,13 @@ inline int64_t effective_seq_len(const lcx_rope_params *p, int64_t call_len) {
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The rotate pass of lcx_apply_rope (argument checks included), optionally also
+// writing y_lo = bf16(y' - bf16(y')) (bf16 only; same strides as y; NULL = none).
+lcx_status apply_rope_impl(const lcx_rope_params *params, const void *x, void *y, void *y_lo,
+                           int32_t dtype, int64_t B, int64_t H, int64_t L,
+                           const int64_t *x_strides, const int64_t *y_strides, int64_t pos_offset,
+                           cudaStream_t stream);
+
 // Enqueue the merge of n_parts partial results ([n_parts, B, Hq, L, D] fp32 o,
 // [n_parts, B, Hq, L] fp32 lse) into o (dtype, strides) and optionally lse.
 // Arguments are assumed valid.

@@ -258,11 +258,14 @@ def test_attn_fwd_host_pipelined_equals_device_call(chunks):
 
 @pytest.mark.parametrize("name", ["L1", "L127_yarn_G2", "L1000_window_sinks", "L700_D64",
                                   "L400_interleaved", "L600_f32", "L2048_outliers_split",
+                                  "L640_outliers_split", "L333_split_D64_interleaved",
+                                  "L300_split_f32", "L257_split_G3", "L200_split_noncausal",
                                   "L300_pi_MHA_B2"])
 def test_attn_rotate_keys_once(name):
     """Keys rotated once into a buffer by the rotate pass (args.k_rot) before
-    the kernel, instead of per key tile on chip: same parity (split-QK^T cases
-    keep the on-chip rotation and must be unaffected)."""
+    the kernel, instead of per key tile on chip: same parity.  Split-QK^T cases
+    with bf16 keys get hi/lo parts from the pass (loaded by TMA); with fp32
+    keys the kernel splits the pre-rotated fp32 values itself."""
     full_check(BASE.with_(**SMALL[name]), rotate_k_once=True)
 
 
