@@ -253,6 +253,23 @@ def bench_gpu(args, world, rank, local):
     flops_rank = attn_flops(w)
     tflops = job_tflops(flops_rank, world, args.steps, total_ms)
 
+    # --- the same step with every K tile rotated on chip by each CTA that reads
+    # it (no key buffer): the kernel-only variant of the path, for comparison
+    kw_chip = dict(kw, k_rot=None)
+    for _ in range(2):
+        lcx.attn_fwd(q, k, v, rope, **kw_chip)
+    torch.cuda.synchronize()
+    a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps_chip = max(2, min(args.steps, 3))
+    a_ev.record(stream)
+    for _ in range(reps_chip):
+        lcx.attn_fwd(q, k, v, rope, **kw_chip)
+    b_ev.record(stream)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, "device watchdog fired (keys rotated on chip)"
+    chip_ms = a_ev.elapsed_time(b_ev) / reps_chip
+    chip_tflops = flops_rank / (chip_ms * 1e-3) / 1e12
+
     # --- apply_rope (the unfused rotate-pairs pass) on Q and K, for its own roofline
     qr, kr = torch.empty_like(q), torch.empty_like(k)
     for _ in range(3):
@@ -360,6 +377,11 @@ def bench_gpu(args, world, rank, local):
         "e2e": {"value": round(e2e_tflops, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "clocks": clk.summary(),
+        "keys_rotated_on_chip": {
+            "what": "the same step without a key buffer: every K tile rotated in shared "
+                    "memory by each CTA that reads it (the single-kernel variant)",
+            "ms_per_step": round(chip_ms, 3), "value": round(chip_tflops, 2),
+            "unit": "TFLOP/s", "launches": reps_chip},
         "splitkv_decode": decode,
         "mla_prefill": mla,
     }
