@@ -45,10 +45,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
 # launch on the headline workload (yarn_L131072_s16), from a one-pass ncu capture
-# of the current kernel (keys pre-rotated by the rotate pass): 2.97 GB read +
+# of the current kernel (keys pre-rotated by the rotate pass): 3.00 GB read +
 # 1.07 GB written (algorithmic: q, k, v read once = 1.61 GB, o written once =
 # 1.07 GB).  Only valid for that workload.
-ATTN_TRAFFIC_BYTES = {"yarn_L131072_s16": 4.04e9}
+ATTN_TRAFFIC_BYTES = {"yarn_L131072_s16": 4.07e9}
 
 
 def load_peaks():
@@ -381,7 +381,7 @@ def bench_gpu(args, world, rank, local):
             "what": "the same step without a key buffer: every K tile rotated in shared "
                     "memory by each CTA that reads it (the single-kernel variant)",
             "ms_per_step": round(chip_ms, 3), "value": round(chip_tflops, 2),
-            "unit": "TFLOP/s", "launches": reps_chip},
+            "unit": "TFLOP/s", "launches_per_step": 1, "steps": reps_chip},
         "splitkv_decode": decode,
         "mla_prefill": mla,
     }
