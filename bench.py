@@ -414,7 +414,10 @@ def bench_decode(lcx, w, q, k, v, rope, stream, status, reps=20):
               split_qk=w.split_qk, out=od, status=status, q_offset=w.L - 1)
     nbytes = sum(t.numel() * t.element_size() for t in (k, v, qd, od))
     sweep = {}
-    for splits in (1, 8, 16, 32, 64):
+    # the powers of two, and the count that gives every SM one CTA of a kv group
+    sms = torch.cuda.get_device_properties(q.device).multi_processor_count
+    fill = max(1, min(256, sms // (w.B * w.Hkv)))
+    for splits in sorted({1, 8, 16, 32, 64, fill}):
         ws = torch.empty(max(1, lcx.split_workspace_bytes(w.B, w.Hq, 1, w.D, splits)),
                          dtype=torch.uint8, device=q.device)
         for _ in range(3):

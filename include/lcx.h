@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define LCX_VERSION 101
+#define LCX_VERSION 102
 
 #if defined(__GNUC__)
 #define LCX_API __attribute__((visibility("default")))
@@ -263,11 +263,15 @@ LCX_API lcx_status lcx_attn_fwd(const lcx_attn_args *args, void *stream);
 LCX_API lcx_status lcx_attn_fwd_split(const lcx_attn_args *args, int32_t num_splits,
                                       void *workspace, int64_t workspace_bytes, void *stream);
 
-/* Workspace bytes lcx_attn_fwd_split needs: [num_splits, B, Hq, L, D] fp32
- * partial outputs (D here: the output head dim, args.Dv or args.D when Dv is
- * 0) then [num_splits, B, Hq, L] fp32 partial LSEs, each block
- * rounded up to 256 bytes.  0 when num_splits == 1; -1 for invalid sizes
- * (D not 64/128, num_splits outside 1..256, or more than 2^40 query rows). */
+/* Workspace bytes lcx_attn_fwd_split needs: room for two partial results
+ * per split, [2 num_splits, B, Hq, L, D] fp32 partial outputs (D here: the
+ * output head dim, args.Dv or args.D when Dv is 0) then [2 num_splits, B, Hq,
+ * L] fp32 partial LSEs, each block rounded up to 256 bytes.  (Launches whose
+ * query tiles are head-packed -- few queries per head, as in decode -- give
+ * each of a split's two query tiles every other key tile and so write two
+ * partial results per split; the others use the first num_splits.)  0 when
+ * num_splits == 1; -1 for invalid sizes (D not 64/128, num_splits outside
+ * 1..256, or more than 2^40 query rows). */
 LCX_API int64_t lcx_attn_split_workspace_bytes(int64_t B, int64_t Hq, int64_t L, int64_t D,
                                                int32_t num_splits);
 

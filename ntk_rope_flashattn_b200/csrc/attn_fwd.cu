@@ -91,6 +91,8 @@ struct AttnParams {
     int pack_lp, pack_hpt;             // head-packed query tiles (split-KV only): rows
     int pack_stride, pack_off;         // head k of tile t starts at row k stride + t off;
                                        // per head (multiple of 8), heads per tile; 0 = off
+    int pack_ilv;                      // packed: both tiles hold all heads of the group, tile t
+                                       // takes key tiles j = t mod 2, partial 2 split + t
     float split_recip;                 // 1 / n_split, rounded up
     float *part_o;                     // n_split > 1: [n_split, B, Hq, L, D] partial o
     float *part_lse;                   //              [n_split, B, Hq, L] partial lse
@@ -174,7 +176,7 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
     // Head-packed (split-KV decode): one unit per kv group, its heads spread over
     // the two query tiles.
     r.hpt = (kKvSplit && p.pack_lp) ? p.pack_hpt : 1;
-    r.nt = p.heads_per_unit / r.hpt;
+    r.nt = (kKvSplit && p.pack_lp && p.pack_ilv) ? 2 : p.heads_per_unit / r.hpt;
     return r;
 }
 
@@ -552,10 +554,10 @@ __device__ __forceinline__ float row_max(const float (&v)[N]) {
 // inv: fp32 into the partial buffer of the unit's key split when there is one,
 // else rounded once to the output type.
 template <int D, bool kF32, bool kKvSplit>
-__device__ __forceinline__ void store_o32(const AttnParams &p, const Unit &U, int h, int i, int c,
-                                          const float (&v)[32], float inv) {
+__device__ __forceinline__ void store_o32(const AttnParams &p, const Unit &U, int slot, int h,
+                                          int i, int c, const float (&v)[32], float inv) {
     if constexpr (kKvSplit) {
-        const long long prow = (((long long)U.split * p.B + U.b) * p.Hq + h) * p.L + i;
+        const long long prow = (((long long)slot * p.B + U.b) * p.Hq + h) * p.L + i;
         float4 *dst = reinterpret_cast<float4 *>(p.part_o + prow * D + c * 32);
 #pragma unroll
         for (int e = 0; e < 8; ++e)
@@ -583,10 +585,10 @@ __device__ __forceinline__ void store_o32(const AttnParams &p, const Unit &U, in
 
 // The row's log-sum-exp (natural log) into the partial buffer or the output.
 template <bool kKvSplit>
-__device__ __forceinline__ void store_lse(const AttnParams &p, const Unit &U, int h, int i,
-                                          float lse) {
+__device__ __forceinline__ void store_lse(const AttnParams &p, const Unit &U, int slot, int h,
+                                          int i, float lse) {
     if constexpr (kKvSplit)
-        p.part_lse[(((long long)U.split * p.B + U.b) * p.Hq + h) * p.L + i] = lse;
+        p.part_lse[(((long long)slot * p.B + U.b) * p.Hq + h) * p.L + i] = lse;
     else if (p.lse)
         p.lse[(U.b * (long long)p.Hq + h) * p.L + i] = lse;
 }
@@ -607,7 +609,7 @@ __device__ __forceinline__ RowMap map_row(const AttnParams &p, const Unit &U, in
         const int rel = row - t * p.pack_off;
         const int k = rel >= 0 ? rel / p.pack_stride : U.hpt;
         m.i = rel - k * p.pack_stride;
-        m.h = U.hq0 + t * U.hpt + k;
+        m.h = U.hq0 + (p.pack_ilv ? 0 : t * U.hpt) + k;
         m.valid = rel >= 0 && k < U.hpt && m.i < p.L;
     } else {
         m.h = U.hq0 + t;
@@ -692,14 +694,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // A key split that received no tile (more splits than tiles): the
         // empty partial result, o = 0 and lse = -inf.
         if (warp < 8 && (warp >> 2) < U.nt) {
-            const RowMap rm = map_row(p, U, warp >> 2, (warp & 3) * 32 + lane, packed);
+            const int t = warp >> 2;
+            const RowMap rm = map_row(p, U, t, (warp & 3) * 32 + lane, packed);
             if (rm.valid) {
                 float z[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) z[e] = 0.f;
+                const int slot = p.pack_ilv ? 2 * U.split + t : U.split;
                 for (int c = 0; c < DV / 32; ++c)
-                    store_o32<DV, kF32, kKvSplit>(p, U, rm.h, rm.i, c, z, 0.f);
-                store_lse<kKvSplit>(p, U, rm.h, rm.i, -INFINITY);
+                    store_o32<DV, kF32, kKvSplit>(p, U, slot, rm.h, rm.i, c, z, 0.f);
+                store_lse<kKvSplit>(p, U, slot, rm.h, rm.i, -INFINITY);
             }
         }
     } else if ((warp >> 2) == 3) {
@@ -727,8 +731,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int bx = 0; bx < D / 64; ++bx)
                                 tma_load_4d(sQ + t * C::kParts * C::kTileQ + bx * C::kBoxQ +
                                                 (k * p.pack_stride + t * p.pack_off) * 128,
-                                            &tmq, &bar.full_q, bx * 64, 0, U.hq0 + t * U.hpt + k,
-                                            U.b);
+                                            &tmq, &bar.full_q, bx * 64, 0,
+                                            U.hq0 + (p.pack_ilv ? 0 : t * U.hpt) + k, U.b);
                 } else {
                     mbar_arrive_expect_tx(&bar.full_q, U.nt * C::kTileQ);
                     for (int t = 0; t < U.nt; ++t)
@@ -829,55 +833,87 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint64_t *kready = (kF32 || (kSplit && !p.k_lo_tma) || p.rotate_k) ? bar.ready_k
                                                                                     : bar.full_k;
                 bool ok = mbar_wait(&bar.ready_q, 0, abort, tmo);
-                for (int jj = 0; ok && jj < NB && jj < T.n; ++jj) {
-                    ok = mbar_wait(&kready[jj % NSK], (jj / NSK) & 1, abort, tmo);
-                    tc_fence_after();
-                    if (!ok) break;
-                    for (int t = 0; t < U.nt; ++t) {
-                        issue_s(t, jj % NSK, jj % NB);
-                        mma_commit(&bar.s_ready[t][jj % NB]);
-                    }
-                    mma_commit(&bar.empty_k[jj % NSK]);
-                }
-                for (int j = 0; ok && j < T.n; ++j) {
-                    const int sv = j % NSV, jn = j + NB;
-                    ok = mbar_wait(&bar.full_v[sv], (j / NSV) & 1, abort, tmo);
-                    for (int t = 0; ok && t < U.nt; ++t) {
-                        ok = mbar_wait(&bar.p_ready[t][j % NB], (j / NB) & 1, abort, tmo);
+                if (kKvSplit && NB == 1 && p.pack_ilv) {
+                    // Both query tiles hold the same queries and tile t takes the
+                    // key tiles j = t mod 2, so two K/V tiles are in flight per
+                    // CTA: S_t(j + 2) follows PV_t(j) into the buffer P_t(j) held.
+                    for (int j = 0; ok && j < 2 && j < T.n; ++j) {
+                        ok = mbar_wait(&kready[j % NSK], (j / NSK) & 1, abort, tmo);
                         tc_fence_after();
                         if (!ok) break;
-                        issue_pv(t, sv, j % NB, j > 0);
-                        if (NB > 1) {
-                            mma_commit(&bar.pv_done[t]);
-                        } else if (jn < T.n) {
-                            const int sk = jn % NSK;
-                            if (t == 0) {
-                                ok = mbar_wait(&kready[sk], (jn / NSK) & 1, abort, tmo);
-                                tc_fence_after();
-                                if (!ok) break;
-                            }
-                            issue_s(t, sk, jn % NB);
-                            mma_commit(&bar.s_ready[t][jn % NB]);
-                        }
+                        issue_s(j, j % NSK, 0);
+                        mma_commit(&bar.s_ready[j][0]);
+                        mma_commit(&bar.empty_k[j % NSK]);
                     }
-                    // Two S buffers: both PVs of tile j go first and release their
-                    // V stage, so a key tile that is still being rotated holds back
-                    // only the S products.
-                    if (NB > 1 && ok) {
+                    for (int j = 0; ok && j < T.n; ++j) {
+                        const int t = j & 1, sv = j % NSV, jn = j + 2;
+                        ok = mbar_wait(&bar.full_v[sv], (j / NSV) & 1, abort, tmo);
+                        if (ok) ok = mbar_wait(&bar.p_ready[t][0], (j >> 1) & 1, abort, tmo);
+                        tc_fence_after();
+                        if (!ok) break;
+                        issue_pv(t, sv, 0, j >= 2);
                         mma_commit(&bar.empty_v[sv]);
                         if (jn < T.n) {
                             const int sk = jn % NSK;
                             ok = mbar_wait(&kready[sk], (jn / NSK) & 1, abort, tmo);
                             tc_fence_after();
-                            for (int t = 0; ok && t < U.nt; ++t) {
+                            if (!ok) break;
+                            issue_s(t, sk, 0);
+                            mma_commit(&bar.s_ready[t][0]);
+                            mma_commit(&bar.empty_k[sk]);
+                        }
+                    }
+                } else {
+                    for (int jj = 0; ok && jj < NB && jj < T.n; ++jj) {
+                        ok = mbar_wait(&kready[jj % NSK], (jj / NSK) & 1, abort, tmo);
+                        tc_fence_after();
+                        if (!ok) break;
+                        for (int t = 0; t < U.nt; ++t) {
+                            issue_s(t, jj % NSK, jj % NB);
+                            mma_commit(&bar.s_ready[t][jj % NB]);
+                        }
+                        mma_commit(&bar.empty_k[jj % NSK]);
+                    }
+                    for (int j = 0; ok && j < T.n; ++j) {
+                        const int sv = j % NSV, jn = j + NB;
+                        ok = mbar_wait(&bar.full_v[sv], (j / NSV) & 1, abort, tmo);
+                        for (int t = 0; ok && t < U.nt; ++t) {
+                            ok = mbar_wait(&bar.p_ready[t][j % NB], (j / NB) & 1, abort, tmo);
+                            tc_fence_after();
+                            if (!ok) break;
+                            issue_pv(t, sv, j % NB, j > 0);
+                            if (NB > 1) {
+                                mma_commit(&bar.pv_done[t]);
+                            } else if (jn < T.n) {
+                                const int sk = jn % NSK;
+                                if (t == 0) {
+                                    ok = mbar_wait(&kready[sk], (jn / NSK) & 1, abort, tmo);
+                                    tc_fence_after();
+                                    if (!ok) break;
+                                }
                                 issue_s(t, sk, jn % NB);
                                 mma_commit(&bar.s_ready[t][jn % NB]);
                             }
-                            if (ok) mma_commit(&bar.empty_k[sk]);
                         }
-                    } else if (ok) {
-                        mma_commit(&bar.empty_v[sv]);
-                        if (jn < T.n) mma_commit(&bar.empty_k[jn % NSK]);
+                        // Two S buffers: both PVs of tile j go first and release their
+                        // V stage, so a key tile that is still being rotated holds back
+                        // only the S products.
+                        if (NB > 1 && ok) {
+                            mma_commit(&bar.empty_v[sv]);
+                            if (jn < T.n) {
+                                const int sk = jn % NSK;
+                                ok = mbar_wait(&kready[sk], (jn / NSK) & 1, abort, tmo);
+                                tc_fence_after();
+                                for (int t = 0; ok && t < U.nt; ++t) {
+                                    issue_s(t, sk, jn % NB);
+                                    mma_commit(&bar.s_ready[t][jn % NB]);
+                                }
+                                if (ok) mma_commit(&bar.empty_k[sk]);
+                            }
+                        } else if (ok) {
+                            mma_commit(&bar.empty_v[sv]);
+                            if (jn < T.n) mma_commit(&bar.empty_k[jn % NSK]);
+                        }
                     }
                 }
                 if (ok)
@@ -977,11 +1013,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             // none only keeps step with the barriers, which leaves its SMSP to the
             // rotation warp (its P rows are never used: their O rows are not stored).
             const bool idle = kKvSplit && !__any_sync(0xffffffffu, rm.valid);
-            for (int j = 0; j < T.n; ++j) {
-                const int b = j % NB;
+            // Interleaved key tiles (head-packed split-KV): this tile takes the
+            // key tiles j = t mod 2 of the split and writes partial 2 split + t.
+            const bool ilv = kKvSplit && NB == 1 && p.pack_ilv;
+            const int n_it = ilv ? (T.n - t + 1) / 2 : T.n;
+            for (int it = 0; it < n_it; ++it) {
+                const int j = ilv ? 2 * it + t : it;
+                const int b = it % NB;
                 const uint32_t s_col = (t * NB + b) * BN;
                 ok = __all_sync(0xffffffffu,
-                                mbar_wait(&bar.s_ready[t][b], (j / NB) & 1, abort, tmo));
+                                mbar_wait(&bar.s_ready[t][b], (it / NB) & 1, abort, tmo));
                 if (!ok) break;
                 if (idle) {
                     mbar_arrive(&bar.p_ready[t][b]);
@@ -1017,7 +1058,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // and PV_t(j) needs this tile's P, so no other phase can be
                         // pending).  With one S buffer, S_t(j) done implies it.
                         ok = __all_sync(0xffffffffu,
-                                        mbar_wait(&bar.pv_done[t], (j - 1) & 1, abort, tmo));
+                                        mbar_wait(&bar.pv_done[t], (it - 1) & 1, abort, tmo));
                         if (!ok) break;
                         tc_fence_after();
                     }
@@ -1071,15 +1112,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok) {
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.f / l : 0.f;
+                const int slot = ilv ? 2 * U.split + t : U.split;
     #pragma unroll 1
                 for (int c = 0; c < DV / 32; ++c) {
                     float v[32];
-                    tmem_ld32(trow + o_col + c * 32, v);
-                    if (rm.valid) store_o32<DV, kF32, kKvSplit>(p, U, rm.h, rm.i, c, v, inv);
+                    if (n_it > 0) {
+                        tmem_ld32(trow + o_col + c * 32, v);
+                    } else {
+                        // no key tile reached this tile: O_t was never written
+    #pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] = 0.f;
+                    }
+                    if (rm.valid)
+                        store_o32<DV, kF32, kKvSplit>(p, U, slot, rm.h, rm.i, c, v, inv);
                 }
                 if (rm.valid) {
                     const float ln2 = 0.69314718055994531f;
-                    store_lse<kKvSplit>(p, U, rm.h, rm.i,
+                    store_lse<kKvSplit>(p, U, slot, rm.h, rm.i,
                                         l > 0.f ? (m + __log2f(l)) * ln2 : -INFINITY);
                 }
             }
@@ -1473,7 +1522,9 @@ extern "C" int64_t lcx_attn_split_workspace_bytes(int64_t B, int64_t Hq, int64_t
         B * Hq * L > lcx::kMaxSplitRows)
         return -1;
     if (num_splits == 1) return 0;
-    return lcx::split_ws_bytes(B * Hq * L, D, num_splits);
+    // room for two partial results per split (head-packed launches write one
+    // per query tile)
+    return lcx::split_ws_bytes(B * Hq * L, D, 2 * int64_t(num_splits));
 }
 
 extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_splits,
@@ -1490,23 +1541,40 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
     if (num_splits == 1) return attn_enqueue(x, s);
     const int64_t rows = a->B * a->Hq * a->L;
     if (rows > kMaxSplitRows) return fail(LCX_ERR_UNSUPPORTED, "too many query rows to split");
-    const int64_t need = split_ws_bytes(rows, x.DV, num_splits);
+    const int64_t need = split_ws_bytes(rows, x.DV, 2 * int64_t(num_splits));
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(LCX_ERR_INVALID_ARG, "workspace must be a 256-byte aligned device pointer");
     if (workspace_bytes < need)
         return fail(LCX_ERR_INVALID_ARG, "workspace holds %lld bytes; %lld needed",
                     (long long)workspace_bytes, (long long)need);
     float *part_o = static_cast<float *>(workspace);
-    float *part_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) +
-                                                split_o_bytes(rows, x.DV, num_splits));
+    float *part_lse = reinterpret_cast<float *>(
+        static_cast<char *>(workspace) + split_o_bytes(rows, x.DV, 2 * int64_t(num_splits)));
     x.p.n_split = num_splits;
     x.p.split_recip = std::nextafter(1.0f / float(num_splits), 2.0f);
     // Head-packed query tiles: with few queries per head (decode, short chunks)
-    // the G heads of a kv group share the CTA's two 128-row query tiles, G/2
-    // heads of pack_lp rows each (L rounded up to 8 rows), so every K/V tile is
-    // read and rotated once per kv group instead of once per head pair.
+    // the G heads of a kv group share the CTA's query tiles (pack_lp rows per
+    // head: L rounded up to 8 rows), so every K/V tile is read and rotated once
+    // per kv group instead of once per head pair.
+    //  - bf16, plain QK^T, G pack_lp <= 128: both tiles hold all G heads (rows
+    //    [0, G pack_lp), tile 1 shifted by whole warps when that fits, so the
+    //    busy softmax warps of the two tiles use different SMSPs) and tile t
+    //    takes the key tiles j = t mod 2: two K/V tiles in flight per CTA, two
+    //    partial results per split.
+    //  - otherwise, G even and G/2 pack_lp <= 128: G/2 heads per tile, both
+    //    tiles multiply every key tile.
     const int64_t lp = (a->L + 7) / 8 * 8;
-    if (!x.f32 && x.p.G % 2 == 0 && x.D <= 128 && lp * (x.p.G / 2) <= kBM) {
+    int n_parts = num_splits;
+    if (!x.f32 && !x.split_qk && x.D <= 128 && lp * x.p.G <= kBM) {
+        const int used = int(lp) * x.p.G;
+        x.p.pack_lp = int(lp);
+        x.p.pack_hpt = x.p.G;
+        x.p.pack_stride = int(lp);
+        x.p.pack_off = (used + 31) / 32 * 32;
+        if (x.p.pack_off + used > kBM) x.p.pack_off = 0;
+        x.p.pack_ilv = 1;
+        n_parts = 2 * num_splits;
+    } else if (!x.f32 && x.p.G % 2 == 0 && x.D <= 128 && lp * (x.p.G / 2) <= kBM) {
         x.p.pack_lp = int(lp);
         x.p.pack_hpt = x.p.G / 2;
         // Heads spread over the tile (multiples of 8 rows keep the 128-byte
@@ -1514,6 +1582,8 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
         // still fits, so the busy softmax warps of both tiles use different SMSPs.
         x.p.pack_stride = (kBM / x.p.pack_hpt) / 8 * 8;
         x.p.pack_off = (x.p.pack_stride - x.p.pack_lp >= 32) ? 32 : 0;
+    }
+    if (x.p.pack_lp) {
         x.p.heads_per_unit = x.p.G;
         x.p.n_qb = 1;
         x.p.units_per_qb = x.p.B * x.p.Hkv;
@@ -1525,6 +1595,6 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
     x.p.part_o = part_o;
     x.p.part_lse = part_lse;
     if ((st = attn_enqueue(x, s)) != LCX_OK) return st;
-    return launch_merge(part_o, part_lse, num_splits, a->B, a->Hq, a->L, x.DV, a->o, a->dtype,
+    return launch_merge(part_o, part_lse, n_parts, a->B, a->Hq, a->L, x.DV, a->o, a->dtype,
                         a->o_strides, a->lse, s);
 }

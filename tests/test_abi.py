@@ -43,7 +43,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lcx.version() == 101
+    assert lcx.version() == 102
     for st in range(5):
         assert lib.lcx_status_string(st).decode()
     assert lib.lcx_status_string(99).decode() == "unknown status"
@@ -273,8 +273,11 @@ def test_attn_split_validation_without_device(lib, splits, ws, nbytes):
 def test_split_workspace_bytes(lib):
     f = lib.lcx_attn_split_workspace_bytes
     assert f(1, 32, 1, 128, 1) == 0
-    assert f(1, 32, 1, 128, 16) == 16 * 32 * 128 * 4 + 2048
-    assert f(2, 3, 5, 64, 3) == -(-(3 * 30 * 64 * 4) // 256) * 256 + 512
+    # room for two partial results per split (head-packed launches write one
+    # per query tile): [2 S, rows, D] fp32 o then [2 S, rows] fp32 lse, each
+    # rounded up to 256 bytes
+    assert f(1, 32, 1, 128, 16) == 2 * 16 * 32 * 128 * 4 + 2 * 16 * 32 * 4
+    assert f(2, 3, 5, 64, 3) == -(-(6 * 30 * 64 * 4) // 256) * 256 + 768
     for bad in ((1, 32, 1, 96, 4), (1, 32, 1, 128, 0), (1, 32, 1, 128, 257), (-1, 1, 1, 64, 2),
                 (1 << 20, 65536, 1 << 30, 128, 2)):
         assert f(*bad) == -1

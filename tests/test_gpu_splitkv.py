@@ -134,3 +134,28 @@ def test_splitkv_head_packed_decode(L, Hq, Hkv, extra):
                        split_qk=w.split_qk)
     ref = oracle_rows(q, k, v, rope, Lk - L, True, w.window, w.sinks)
     compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref[0], ref[1])
+
+
+@pytest.mark.parametrize("L,Lk,splits,extra", [
+    (1, 1800, 2, dict(Hq=8, Hkv=2)),                 # 15 key tiles: splits of 8 and 7
+    (1, 777, 7, dict(Hq=8, Hkv=2)),                  # one key tile per split: tile 1 gets none
+    (2, 1000, 3, dict(Hq=6, Hkv=2)),                 # G = 3 (odd): packed only this way
+    (1, 1500, 5, dict(Hq=2, Hkv=2)),                 # G = 1
+    (4, 3000, 6, dict(Hq=8, Hkv=2, window=700, sinks=4)),
+    (1, 2000, 4, dict(Hq=8, Hkv=2, k_prerotated=True)),
+])
+def test_splitkv_interleaved_key_tiles(L, Lk, splits, extra):
+    """bf16 head-packed split-KV: both query tiles hold all G heads and take
+    alternate key tiles of the split (two partial results per split); every
+    head's rows against the oracle, edge counts of key tiles included."""
+    extra = dict(extra)
+    prerot = extra.pop("k_prerotated", False)
+    w = W0.with_(**extra, L=Lk)
+    q_all, k, v = make_inputs(w, device="cuda")
+    q = q_all[:, :, Lk - L:]
+    rope = rope_of(w)
+    kk = lcx.apply_rope(k, rope) if prerot else k
+    o, lse = run_split(q, kk, v, rope, splits, window=w.window, sinks=w.sinks, q_offset=Lk - L,
+                       k_prerotated=prerot)
+    ref = oracle_rows(q, k, v, rope, Lk - L, True, w.window, w.sinks)
+    compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref[0], ref[1])
