@@ -86,6 +86,8 @@ struct AttnParams {
     int Lk, qoff;                      // key rows; position of query row 0
     int causal, window, sinks;
     int n_qb, heads_per_unit, units_per_qb;
+    int qpair;                         // unit = two consecutive 128-row query blocks of one
+                                       // head (odd G); n_qb then counts 256-row blocks
     int rotate_q, rotate_k;
     int n_split;                       // key-range splits per unit (1: plain output)
     int pack_lp, pack_hpt;             // head-packed query tiles (split-KV only): rows
@@ -153,6 +155,10 @@ struct Bars {
 struct Unit {
     int b, g, hq0, nt, q0, split;
     int hpt;  // heads per query tile: 1, or pack_hpt when the tiles are head-packed
+    // query tile t holds head hq0 + t hstep, rows q0 + t qstep (+ the row)
+    int hstep, qstep;
+    __device__ __forceinline__ int tq0(int t) const { return q0 + t * qstep; }
+    __device__ __forceinline__ int th(int t) const { return hq0 + t * hstep; }
 };
 
 // Work units are grouped by (batch, kv head) and, inside a group, numbered
@@ -170,13 +176,23 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
     Unit r;
     r.b = grp / p.Hkv;
     r.g = grp % p.Hkv;
-    r.q0 = (p.n_qb - 1 - rem / upq) * kBM;
+    const int rows = p.qpair ? 2 * kBM : kBM;   // query rows of a unit
+    r.q0 = (p.n_qb - 1 - rem / upq) * rows;
     r.hq0 = r.g * p.G + p.heads_per_unit * (rem % upq);
     r.split = kKvSplit ? int(blockIdx.x) % p.n_split : 0;
     // Head-packed (split-KV decode): one unit per kv group, its heads spread over
     // the two query tiles.
     r.hpt = (kKvSplit && p.pack_lp) ? p.pack_hpt : 1;
     r.nt = (kKvSplit && p.pack_lp && p.pack_ilv) ? 2 : p.heads_per_unit / r.hpt;
+    r.hstep = 1;
+    r.qstep = 0;
+    if (p.qpair) {
+        // odd G: the two tiles are consecutive query blocks of head hq0 (one,
+        // when the second would start past the last query)
+        r.hstep = 0;
+        r.qstep = kBM;
+        r.nt = (r.q0 + kBM < p.L) ? 2 : 1;
+    }
     return r;
 }
 
@@ -194,7 +210,8 @@ struct Tiles {
 
 template <int BN, bool kKvSplit>
 __device__ __forceinline__ Tiles make_tiles(int q0, int split, const AttnParams &p) {
-    const int i1 = min(q0 + kBM - 1, p.L - 1) + p.qoff;
+    const int rows = p.qpair ? 2 * kBM : kBM;   // the unit's query rows from q0
+    const int i1 = min(q0 + rows - 1, p.L - 1) + p.qoff;
     const int jhi = p.causal ? i1 / BN : (p.Lk - 1) / BN;
     int jlo = 0, ns = 0;
     if (p.causal && p.window > 0) {
@@ -612,8 +629,8 @@ __device__ __forceinline__ RowMap map_row(const AttnParams &p, const Unit &U, in
         m.h = U.hq0 + (p.pack_ilv ? 0 : t * U.hpt) + k;
         m.valid = rel >= 0 && k < U.hpt && m.i < p.L;
     } else {
-        m.h = U.hq0 + t;
-        m.i = U.q0 + row;
+        m.h = U.th(t);
+        m.i = U.tq0(t) + row;
         m.valid = m.i < p.L;
     }
     return m;
@@ -738,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int t = 0; t < U.nt; ++t)
                         for (int bx = 0; bx < D / 64; ++bx)
                             tma_load_4d(sQ + t * C::kParts * C::kTileQ + bx * C::kBoxQ, &tmq,
-                                        &bar.full_q, bx * 64, U.q0, U.hq0 + t, U.b);
+                                        &bar.full_q, bx * 64, U.tq0(t), U.th(t), U.b);
                 }
                 bool ok = true;
                 for (int j = 0; ok && j < T.n; ++j) {
@@ -943,15 +960,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                               t * p.pack_off, U.hpt, ph, p, rotq);
                     else
                         rotate_tile_bf16<D, RD, kHalf, kSplit, kBM>(
-                            qt, qt + C::kTileQ, (long long)U.q0 + p.qoff, ph, p, rotq);
+                            qt, qt + C::kTileQ, (long long)U.tq0(t) + p.qoff, ph, p, rotq);
                 }
         } else {
             for (int t = 0; t < U.nt; ++t) {
                 const float *base = reinterpret_cast<const float *>(p.q) + U.b * p.qs[0] +
-                                    (long long)(U.hq0 + t) * p.qs[1];
+                                    (long long)U.th(t) * p.qs[1];
                 uint8_t *qt = sQ + t * C::kParts * C::kTileQ;
-                load_tile_f32<D, kHalf, kSplit, kBM>(qt, qt + C::kTileQ, base, p.qs[2], U.q0, p.L,
-                                                     (long long)U.q0 + p.qoff, rotq, ph, p);
+                load_tile_f32<D, kHalf, kSplit, kBM>(qt, qt + C::kTileQ, base, p.qs[2], U.tq0(t),
+                                                     p.L, (long long)U.tq0(t) + p.qoff, rotq, ph,
+                                                     p);
             }
         }
         if (ok) {
@@ -1006,6 +1024,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr int NB = C::kNB;
             const RowMap rm = map_row(p, U, t, row, packed);
             const int pi = rm.i + p.qoff;  // this row's query position
+            const int tq0 = U.tq0(t);      // the tile's first query row
             const float cl2 = p.c_log2;
             float m = -INFINITY, l = 0.f;
             bool ok = true;
@@ -1030,7 +1049,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 const int jt = T.tile(j), k0 = jt * BN;
-                const bool partial = !tile_full<BN>(U.q0, jt, p);
+                const bool partial = !tile_full<BN>(tq0, jt, p);
                 // visible columns: col <= hi and (no window or col >= lo or col < sk)
                 const int hi = p.causal ? min(pi - k0, p.Lk - 1 - k0) : p.Lk - 1 - k0;
                 const int lo = pi - p.window + 1 - k0;
@@ -1400,10 +1419,12 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     // A window of Lk or more keys, or Lk sinks, no longer restricts anything.
     p.window = int(a->window > Lk ? Lk : a->window);
     p.sinks = int(a->sinks > Lk ? Lk : a->sinks);
-    p.n_qb = int((a->L + kBM - 1) / kBM);
     // Two query heads share a CTA's K/V tiles when the group allows it and
-    // two query tiles fit (D = 192 leaves room for one).
+    // two query tiles fit (D = 192 leaves room for one); with an odd group the
+    // two tiles are consecutive query blocks of one head instead.
     p.heads_per_unit = (p.G % 2 == 0 && a->D <= 128) ? 2 : 1;
+    p.qpair = (p.G % 2 == 1 && a->D <= 128) ? 1 : 0;
+    p.n_qb = int((a->L + (p.qpair ? 2 * kBM : kBM) - 1) / (p.qpair ? 2 * kBM : kBM));
     p.units_per_qb = p.B * p.Hq / p.heads_per_unit;
     p.n_split = 1;
     x.units = (long long)p.n_qb * p.units_per_qb;
@@ -1584,6 +1605,7 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
         x.p.pack_off = (x.p.pack_stride - x.p.pack_lp >= 32) ? 32 : 0;
     }
     if (x.p.pack_lp) {
+        x.p.qpair = 0;
         x.p.heads_per_unit = x.p.G;
         x.p.n_qb = 1;
         x.p.units_per_qb = x.p.B * x.p.Hkv;

@@ -105,6 +105,14 @@ SMALL = {
     "L300_split_f32": dict(L=300, dtype="f32", mode="pi", scale=2.0, split_qk=True),
     "L200_split_noncausal": dict(L=200, Hq=2, Hkv=1, causal=False, split_qk=True),
     "L256_scale": dict(L=256, softmax_scale=0.05),
+    # odd G: a unit is two consecutive 128-row query blocks of one head
+    "L129_MHA_pair": dict(L=129, Hq=2, Hkv=2),       # second block of one row
+    "L128_MHA_single": dict(L=128, Hq=1, Hkv=1),      # no second block
+    "L700_G3_window_sinks": dict(L=700, Hq=3, Hkv=1, mode="yarn", scale=8.0,
+                                 original_max_pos=128, window=200, sinks=4),
+    "L520_MHA_f32": dict(L=520, Hq=1, Hkv=1, dtype="f32", mode="pi", scale=2.0),
+    "L600_MHA_noncausal": dict(L=600, Hq=2, Hkv=2, causal=False),
+    "L384_G5_D64_interleaved": dict(L=384, Hq=5, Hkv=1, D=64, pairing="interleaved"),
 }
 
 

@@ -38,6 +38,7 @@ def run_split(q, k, v, rope, num_splits, **kw):
     (2, 900, 5, dict(split_qk=True, window=300, sinks=2)),
     (3, 640, 4, dict(dtype="f32", mode="pi", scale=2.0)),
     (1, 500, 7, dict(D=64, pairing="interleaved")),
+    (300, 2000, 3, dict(Hq=2, Hkv=2)),       # G = 1, too many rows to pack: query-block pairs
 ])
 def test_splitkv_decode(L, Lk, splits, extra):
     w = W0.with_(**extra, L=Lk)
