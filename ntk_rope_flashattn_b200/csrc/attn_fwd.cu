@@ -59,6 +59,9 @@ constexpr float kRescaleLog2 = 8.0f;    // rescale O only if the max grows by > 
 #ifndef LCX_EMU_EVERY
 #define LCX_EMU_EVERY 0
 #endif
+#ifndef LCX_D192_TWO_TILES
+#define LCX_D192_TWO_TILES 1
+#endif
 #ifndef LCX_KSTAGES_D128
 #define LCX_KSTAGES_D128 2
 #endif
@@ -111,20 +114,20 @@ struct AttnParams {
 // R rows x 128 bytes with the 128-byte swizzle.  In the split mode every Q and
 // K tile has a second "lo" part holding bf16(x' - bf16(x')), and key tiles are
 // 64 rows so that both parts fit.  D is the query/key head dim, DV the
-// value/output head dim; at D = 192 (decoupled RoPE: 128 + 64) one query tile
-// per CTA leaves room for two K and two V stages.
+// value/output head dim; at D = 192 (decoupled RoPE: 128 + 64) two query tiles
+// (96 KB) leave room for two K stages (48 KB each) and one V stage.
 template <int D, int DV, bool kSplit>
 struct Cfg {
     static constexpr int BN = kSplit ? 64 : 128;        // keys per tile
     static constexpr int kParts = kSplit ? 2 : 1;       // hi (+ lo) parts of Q and K
-    static constexpr int kNTQ = D > 128 ? 1 : 2;        // query tiles per CTA
+    static constexpr int kNTQ = (D > 128 && !LCX_D192_TWO_TILES) ? 1 : 2;  // query tiles per CTA
     static constexpr int kTileQ = kBM * D * 2;          // one part of a Q tile
     static constexpr int kTileK = BN * D * 2;           // one part of a K tile
     static constexpr int kTileV = BN * DV * 2;          // a V tile
     static constexpr int kBoxQ = kBM * 128;
     static constexpr int kBoxK = BN * 128;
     static constexpr int kStagesK = (D == 64) ? 4 : (D == 128 && !kSplit) ? LCX_KSTAGES_D128 : 2;
-    static constexpr int kStagesV = (D == 64) ? 4 : 2;
+    static constexpr int kStagesV = (D == 64) ? 4 : (D > 128 && kNTQ == 2) ? 1 : 2;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kNTQ * kParts * kTileQ;
     static constexpr int kOffV = kOffK + kStagesK * kParts * kTileK;
@@ -1422,8 +1425,9 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     // Two query heads share a CTA's K/V tiles when the group allows it and
     // two query tiles fit (D = 192 leaves room for one); with an odd group the
     // two tiles are consecutive query blocks of one head instead.
-    p.heads_per_unit = (p.G % 2 == 0 && a->D <= 128) ? 2 : 1;
-    p.qpair = (p.G % 2 == 1 && a->D <= 128) ? 1 : 0;
+    const bool two_tiles = a->D <= 128 || LCX_D192_TWO_TILES;
+    p.heads_per_unit = (p.G % 2 == 0 && two_tiles) ? 2 : 1;
+    p.qpair = (p.G % 2 == 1 && two_tiles) ? 1 : 0;
     p.n_qb = int((a->L + (p.qpair ? 2 * kBM : kBM) - 1) / (p.qpair ? 2 * kBM : kBM));
     p.units_per_qb = p.B * p.Hq / p.heads_per_unit;
     p.n_split = 1;

@@ -60,6 +60,7 @@ YARN = dict(mode="yarn", scale=8.0, original_max_pos=128)
     (128, 2, 2, 257, "interleaved", 0, 0),
     (64, 4, 4, 520, "half", 0, 0),             # d_C = d_R = 64
     (64, 4, 2, 300, "interleaved", 100, 2),
+    (128, 6, 2, 600, "half", 200, 4),          # G = 3: query-block pairs of one head
 ])
 def test_mla_shared_rope_key(Dc, Hq, Hkv, L, pairing, window, sinks):
     Dr, Dv = 64, 128
