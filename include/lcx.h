@@ -194,19 +194,22 @@ typedef struct {
                                   D - rope.head_dim columns of each key       */
     int64_t k_rope_strides[4]; /* elements; the head stride is not used        */
     void *k_rot;               /* DEVICE scratch or NULL.  When set, and the keys
-                                  would be rotated on chip (no PREROTATED flags,
-                                  every dim rotated, no k_rope), the keys are
-                                  rotated once into it by the rotate pass of
-                                  lcx_apply_rope (mscale included) and the
-                                  attention kernel reads them from there: one
-                                  rotation per key instead of one per key tile
-                                  and CTA.  Contiguous [B, Hkv, Lk, D] of dtype;
-                                  in the split-QK^T mode with bf16 operands the
-                                  hi parts, then the lo parts (bf16 of the
-                                  rounding residual).  16-byte aligned.  Ignored
-                                  otherwise                                    */
+                                  would be rotated on chip (no PREROTATED flags),
+                                  the rotated keys are written once into it by
+                                  the rotate pass of lcx_apply_rope (mscale
+                                  included) and the attention kernel reads them
+                                  from there: one rotation per key instead of
+                                  one per key tile and CTA.  Every dim rotated,
+                                  no k_rope: contiguous [B, Hkv, Lk, D] of
+                                  dtype; in the split-QK^T mode with bf16
+                                  operands the hi parts, then the lo parts (bf16
+                                  of the rounding residual).  With k_rope: the
+                                  shared rotary key, contiguous [B, 1, Lk,
+                                  rope.head_dim].  16-byte aligned.  Ignored
+                                  otherwise (partial rotary without k_rope)    */
     int64_t k_rot_bytes;       /* bytes at k_rot: >= B*Hkv*Lk*D*element size,
-                                  twice that for split-QK^T with bf16          */
+                                  twice that for split-QK^T with bf16, or
+                                  B*Lk*rope.head_dim*element size with k_rope */
 } lcx_attn_args;
 
 /*

@@ -284,9 +284,13 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
     a.q_offset = int(q_offset)
     a.Dv = Dv
     if rotate_k_once and k_rot is None:
-        # split QK^T with bf16 keys: the pass writes hi parts, then lo parts
-        parts = 2 if (split_qk and k.dtype == torch.bfloat16) else 1
-        k_rot = torch.empty((parts, B, Hkv, Lk, Dk), dtype=k.dtype, device=k.device)
+        if k_rope is not None:
+            # decoupled RoPE: the pass rotates only the shared rotary key
+            k_rot = torch.empty((B, 1, Lk, k_rope.shape[-1]), dtype=k.dtype, device=k.device)
+        else:
+            # split QK^T with bf16 keys: the pass writes hi parts, then lo parts
+            parts = 2 if (split_qk and k.dtype == torch.bfloat16) else 1
+            k_rot = torch.empty((parts, B, Hkv, Lk, Dk), dtype=k.dtype, device=k.device)
     if k_rot is not None:
         a.k_rot = k_rot.data_ptr()
         a.k_rot_bytes = k_rot.numel() * k_rot.element_size()

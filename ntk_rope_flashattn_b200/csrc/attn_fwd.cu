@@ -1301,6 +1301,8 @@ struct AttnLaunch : AttnLaunchShape {
     const void *k_src;
     int64_t k_src_strides[4];
     void *k_lo;       // split mode: where the pass writes the keys' lo parts, or NULL
+    int rot_h, rot_d; // heads and columns the pass rotates (Hkv, D; or 1, d_R)
+    void *k_rot;      // where the pass writes
 };
 
 // Validate `a` and fill `x`.  *noop is set for empty problems (B or L zero),
@@ -1371,17 +1373,20 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     if (a->k_rope && (st = check_tensor(a->k_rope, a->k_rope_strides, es, "k_rope")) != LCX_OK)
         return st;
     // Keys rotated once into args.k_rot (by the rotate pass, mscale included)
-    // instead of once per key tile per CTA: only where the kernel would
-    // otherwise rotate them on chip in the plain QK^T mode with full rotary.
-    // In the split-QK^T mode with bf16 keys the pass also writes the lo parts
-    // (bf16 of the rounding residual) right after the hi parts.
+    // instead of once per key tile per CTA, where the kernel would otherwise
+    // rotate them on chip: full-rotary keys ([B, Hkv, Lk, D]), or the shared
+    // rotary key of decoupled RoPE ([B, 1, Lk, d_R]; k keeps its un-rotated
+    // columns).  In the split-QK^T mode with bf16 keys the pass also writes
+    // the lo parts (bf16 of the rounding residual) right after the hi parts.
+    const bool rot_shared = partial && a->k_rope != nullptr;
     const bool rotate_k_once =
         a->k_rot != nullptr && !(a->flags & (LCX_ATTN_PREROTATED | LCX_ATTN_PREROTATED_K |
                                              LCX_ATTN_TEST_STALL)) &&
-        !partial && !a->k_rope && a->D % 16 == 0;
+        ((!partial && !a->k_rope && a->D % 16 == 0) || rot_shared);
     const bool k_lo = rotate_k_once && (a->flags & LCX_ATTN_SPLIT_QK) && a->dtype == LCX_BF16;
-    const int64_t kst_rot[4] = {a->Hkv * Lk * a->D, Lk * a->D, a->D, 1};
-    const int64_t k_part_bytes = a->B * a->Hkv * Lk * a->D * es;
+    const int64_t rot_h = rot_shared ? 1 : a->Hkv, rot_d = rot_shared ? RD : a->D;
+    const int64_t kst_rot[4] = {rot_h * Lk * rot_d, Lk * rot_d, rot_d, 1};
+    const int64_t k_part_bytes = a->B * rot_h * Lk * rot_d * es;
     if (rotate_k_once) {
         if (!aligned16(a->k_rot)) return fail(LCX_ERR_UNSUPPORTED, "k_rot must be 16-byte aligned");
         if (a->k_rot_bytes < k_part_bytes * (k_lo ? 2 : 1))
@@ -1389,15 +1394,20 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
                         (long long)a->k_rot_bytes, (long long)(k_part_bytes * (k_lo ? 2 : 1)));
     }
     void *k_lo_ptr = k_lo ? static_cast<char *>(a->k_rot) + k_part_bytes : nullptr;
-    const void *kptr = rotate_k_once ? a->k_rot : a->k;
-    const int64_t *kst = rotate_k_once ? kst_rot : a->k_strides;
+    const bool k_from_rot = rotate_k_once && !rot_shared;   // k itself read from k_rot
+    const void *kptr = k_from_rot ? a->k_rot : a->k;
+    const int64_t *kst = k_from_rot ? kst_rot : a->k_strides;
 
     memset(&x, 0, sizeof(x));
     x.rotate_k_once = rotate_k_once;
     x.k_lo = k_lo_ptr;
     x.rope = a->rope;
-    x.k_src = a->k;
-    for (int d = 0; d < 4; ++d) x.k_src_strides[d] = a->k_strides[d];
+    x.k_src = rot_shared ? a->k_rope : a->k;
+    for (int d = 0; d < 4; ++d)
+        x.k_src_strides[d] = rot_shared ? a->k_rope_strides[d] : a->k_strides[d];
+    x.rot_h = int(rot_h);
+    x.rot_d = int(rot_d);
+    x.k_rot = rotate_k_once ? a->k_rot : nullptr;
     AttnParams &p = x.p;
     p.q = static_cast<const char *>(a->q);
     p.k = static_cast<const char *>(kptr);
@@ -1485,9 +1495,15 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
                 return st;
         }
         if (a->k_rope) {
-            // one head: the head stride never matters, any valid value will do
+            // one head: the head stride never matters, any valid value will do;
+            // rotated once, the shared key is read from k_rot
+            const void *kr = rot_shared && rotate_k_once ? a->k_rot : a->k_rope;
             int64_t krs[4] = {a->k_rope_strides[0], Lk * RD, a->k_rope_strides[2], 1};
-            if ((st = make_map(&x.m.kr, a->k_rope, a->B, 1, Lk, RD, krs, bn, "k_rope")) != LCX_OK)
+            if (rot_shared && rotate_k_once) {
+                krs[0] = kst_rot[0];
+                krs[2] = kst_rot[2];
+            }
+            if ((st = make_map(&x.m.kr, kr, a->B, 1, Lk, RD, krs, bn, "k_rope")) != LCX_OK)
                 return st;
         }
     }
@@ -1502,11 +1518,11 @@ lcx_status attn_enqueue(const AttnLaunch &x, cudaStream_t s) {
         // the rotate pass over all keys (positions 0..Lk-1), same stream first
         lcx_rope_params rp = x.rope;
         if (rp.seq_len <= 0) rp.seq_len = x.p.Lk;   // the context of the call, as the kernel's
-        const int64_t kst[4] = {(int64_t)x.p.Hkv * x.p.Lk * x.D, (int64_t)x.p.Lk * x.D, x.D, 1};
+        const int64_t kst[4] = {(int64_t)x.rot_h * x.p.Lk * x.rot_d, (int64_t)x.p.Lk * x.rot_d,
+                                x.rot_d, 1};
         const lcx_status st =
-            apply_rope_impl(&rp, x.k_src, const_cast<char *>(x.p.k), x.k_lo,
-                            x.f32 ? LCX_F32 : LCX_BF16, x.p.B, x.p.Hkv, x.p.Lk, x.k_src_strides,
-                            kst, 0, s);
+            apply_rope_impl(&rp, x.k_src, x.k_rot, x.k_lo, x.f32 ? LCX_F32 : LCX_BF16, x.p.B,
+                            x.rot_h, x.p.Lk, x.k_src_strides, kst, 0, s);
         if (st != LCX_OK) return st;
     }
     const unsigned g = unsigned(grid);

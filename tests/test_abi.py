@@ -246,6 +246,10 @@ def _attn_args(**kw):
     (dict(k_rot=0x500000, k_rot_bytes=1000), lcx.LCX_ERR_INVALID_ARG),      # too small
     (dict(D=192, Dv=128, rope=_params("plain", 64), k_rope=0x500008,
           k_rope_strides=[256 * 64, 256 * 64, 64, 1]), lcx.LCX_ERR_UNSUPPORTED),  # misaligned
+    # the shared rotary key rotated once: k_rot must hold [B, 1, Lk, 64]
+    (dict(D=192, Dv=128, rope=_params("plain", 64), k_rope=0x500000,
+          k_rope_strides=[256 * 64, 256 * 64, 64, 1], k_rot=0x600000, k_rot_bytes=1000),
+     lcx.LCX_ERR_INVALID_ARG),
 ])
 def test_attn_validation_without_device(lib, kw, expect):
     a = _attn_args(**kw)

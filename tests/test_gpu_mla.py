@@ -111,3 +111,21 @@ def test_mla_prerotated():
     check(o, lse, ref)
     o2, lse2 = run(q, kc, v, rope, k_rope=kr_rot, k_prerotated=True)
     check(o2, lse2, ref)
+
+
+@pytest.mark.parametrize("Dc,Hq,Hkv,L,pairing,window,sinks", [
+    (128, 4, 4, 700, "half", 0, 0),            # MHA: query-block pairs
+    (128, 8, 2, 333, "half", 150, 4),          # GQA, window + sinks
+    (64, 4, 2, 300, "interleaved", 100, 2),
+])
+def test_mla_rotate_k_once(Dc, Hq, Hkv, L, pairing, window, sinks):
+    """The shared rotary key rotated once into k_rot by the rotate pass, the
+    kernel reading it from there: the oracle's result, and k_rot equal to
+    lcx_apply_rope of the shared key."""
+    Dr, Dv = 64, 128
+    q, kc, kr, v = mla_inputs(1, Hq, Hkv, L, Dc, Dr, Dv, seed=Dc + L + 1)
+    rope = lcx.RopeParams(head_dim=Dr, pairing=pairing, **YARN)
+    k_rot = torch.empty_like(kr)
+    o, lse = run(q, kc, v, rope, k_rope=kr, window=window, sinks=sinks, k_rot=k_rot)
+    check(o, lse, oracle_mla(q, kc, kr, v, rope, 0, window, sinks))
+    assert torch.equal(k_rot, lcx.apply_rope(kr, rope))
