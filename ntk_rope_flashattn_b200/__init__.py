@@ -417,18 +417,48 @@ def attn_fwd_host(q, k, v, rope: RopeParams, device="cuda", workspace=None, chun
     if o_host is None or tuple(o_host.shape) != o_shape or o_host.dtype != q.dtype:
         o_host = torch.empty(o_shape, dtype=q.dtype, pin_memory=True)
         ws["o_host"] = o_host
-    # pieces: (batch, first kv head, end kv head); one piece when the caller
-    # wants per-row statistics back (lse / status buffers cover everything)
+    # pieces: (batch, first kv head, end kv head, first query row, end query
+    # row); one piece when the caller wants per-row statistics back (lse /
+    # status buffers cover everything)
     per_b = max(1, min(Hkv, -(-int(chunks) // B)))
     if "lse" in kw or kw.get("return_lse"):
-        pieces = [(None, 0, Hkv)]
+        pieces = [(None, 0, Hkv, 0, L)]
     else:
         bounds = [round(i * Hkv / per_b) for i in range(per_b + 1)]
-        pieces = [(b, g0, g1) for b in range(B) for g0, g1 in zip(bounds, bounds[1:])
+        pieces = [(b, g0, g1, 0, L) for b in range(B) for g0, g1 in zip(bounds, bounds[1:])
                   if g1 > g0]
+        # Causal prefill: a query range [i0, i1) needs only the keys [0, i1),
+        # so the first piece starts with about its first quarter of query rows
+        # (less input to copy before the first kernel) and the last piece ends
+        # with about its last quarter (less output to copy after the last
+        # kernel).  Cuts sit on 128-row query blocks, so every query tile
+        # starts where it does in one call over everything (its rows are
+        # rotated from the same start) and meets the same key tiles in the
+        # same order.
+        q4 = (L // 4) // 128 * 128
+        if kw.get("causal", True) and not kw.get("q_offset", 0) and q4 >= 128:
+            c = (L - q4) // 128 * 128           # start of the last piece's rows
+            b0, g00, g01, _, _ = pieces[0]
+            head = [(b0, g00, g01, 0, q4), (b0, g00, g01, q4, L)]
+            if len(pieces) == 1:
+                pieces = head[:1] + [(b0, g00, g01, q4, c), (b0, g00, g01, c, L)]
+            else:
+                bl, gl0, gl1, _, _ = pieces[-1]
+                pieces = head + pieces[1:-1] + [(bl, gl0, gl1, 0, c), (bl, gl0, gl1, c, L)]
 
-    def view(t, b, h0, h1):
-        return t[:, h0:h1] if b is None else t[b:b + 1, h0:h1]
+    def view(t, b, h0, h1, r0=None, r1=None):
+        t = t[:, h0:h1] if b is None else t[b:b + 1, h0:h1]
+        return t if r0 is None else t[:, :, r0:r1]
+
+    def copy_rows(dst, src, b, h0, h1, r0, r1):
+        # rows [r0, r1) of heads [h0, h1): one copy per contiguous block (a
+        # strided host <-> device copy would go through a slow staging path)
+        if r0 == 0 and r1 == dst.shape[2] and b is not None:
+            view(dst, b, h0, h1).copy_(view(src, b, h0, h1), non_blocking=True)
+            return
+        for bb in (range(dst.shape[0]) if b is None else (b,)):
+            for h in range(h0, h1):
+                dst[bb, h, r0:r1].copy_(src[bb, h, r0:r1], non_blocking=True)
 
     cur = torch.cuda.current_stream(device)
     s_in = ws.setdefault("stream_in", torch.cuda.Stream(device))
@@ -436,23 +466,34 @@ def attn_fwd_host(q, k, v, rope: RopeParams, device="cuda", workspace=None, chun
     s_in.wait_stream(cur)
     s_out.wait_stream(cur)
     arrived = []
+    have = {}   # (batch, kv head range) -> key rows already on the device
     with torch.cuda.stream(s_in):
-        for b, g0, g1 in pieces:
-            view(dev["q"], b, g0 * G, g1 * G).copy_(view(q, b, g0 * G, g1 * G), non_blocking=True)
-            view(dev["k"], b, g0, g1).copy_(view(k, b, g0, g1), non_blocking=True)
-            view(dev["v"], b, g0, g1).copy_(view(v, b, g0, g1), non_blocking=True)
+        for b, g0, g1, i0, i1 in pieces:
+            copy_rows(dev["q"], q, b, g0 * G, g1 * G, i0, i1)
+            # keys and values up to the piece's last query (all of them unless
+            # causal), from where the group's earlier pieces stopped
+            k1 = i1 if i1 < L else k.shape[2]
+            k0 = have.get((b, g0, g1), 0)
+            if k1 > k0:
+                copy_rows(dev["k"], k, b, g0, g1, k0, k1)
+                copy_rows(dev["v"], v, b, g0, g1, k0, k1)
+                have[(b, g0, g1)] = k1
             ev = torch.cuda.Event()
             ev.record(s_in)
             arrived.append(ev)
-    for (b, g0, g1), ev in zip(pieces, arrived):
+    for (b, g0, g1, i0, i1), ev in zip(pieces, arrived):
         cur.wait_event(ev)
-        o_piece = view(o_dev, b, g0 * G, g1 * G)
-        attn_fwd(view(dev["q"], b, g0 * G, g1 * G), view(dev["k"], b, g0, g1),
-                 view(dev["v"], b, g0, g1), rope, out=o_piece, **kw)
+        o_piece = view(o_dev, b, g0 * G, g1 * G, i0, i1)
+        pkw = dict(kw)
+        if i0 > 0 or i1 < L:
+            pkw["q_offset"] = i0
+        k1 = i1 if i1 < L else k.shape[2]
+        attn_fwd(view(dev["q"], b, g0 * G, g1 * G, i0, i1), view(dev["k"], b, g0, g1, 0, k1),
+                 view(dev["v"], b, g0, g1, 0, k1), rope, out=o_piece, **pkw)
         done = torch.cuda.Event()
         done.record(cur)
         s_out.wait_event(done)
         with torch.cuda.stream(s_out):
-            view(o_host, b, g0 * G, g1 * G).copy_(o_piece, non_blocking=True)
+            copy_rows(o_host, o_dev, b, g0 * G, g1 * G, i0, i1)
     cur.wait_stream(s_out)
     return o_host

@@ -246,20 +246,29 @@ def test_attn_length_dependent_tables(mode):
     compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_lse)
 
 
-@pytest.mark.parametrize("chunks", [1, 3, 8])
-def test_attn_fwd_host_pipelined_equals_device_call(chunks):
-    """attn_fwd_host cuts the work into kv-head pieces pipelined over copy
-    streams; every row's arithmetic is that of one device call, bit for bit."""
-    w = BASE.with_(B=2, Hq=8, Hkv=4, L=600, mode="yarn", scale=8.0, original_max_pos=128,
-                   window=300, sinks=4)
+@pytest.mark.parametrize("chunks,extra", [
+    (1, {}), (3, {}), (8, {}),
+    (8, dict(rotate_k_once=True)),                       # the bench's e2e path
+    (3, dict(causal=False, window=0, sinks=0)),          # no query-range pieces
+    (2, dict(L=1100)),                                   # query cuts at 256 / 768
+])
+def test_attn_fwd_host_pipelined_equals_device_call(chunks, extra):
+    """attn_fwd_host cuts the work into kv-head pieces (and, causal, the first
+    and last into query ranges) pipelined over copy streams; every row's
+    arithmetic is that of one device call, bit for bit."""
+    extra = dict(extra)
+    L = extra.pop("L", 600)
+    causal = extra.pop("causal", True)
+    w = BASE.with_(B=2, Hq=8, Hkv=4, L=L, mode="yarn", scale=8.0, original_max_pos=128,
+                   window=extra.pop("window", 300), sinks=extra.pop("sinks", 4), causal=causal)
     q, k, v = make_inputs(w, device="cuda")
     rope = rope_of(w)
-    ref = lcx.attn_fwd(q, k, v, rope, window=w.window, sinks=w.sinks)
+    ref = lcx.attn_fwd(q, k, v, rope, causal=causal, window=w.window, sinks=w.sinks, **extra)
     qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
     ws = {}
     for _ in range(2):                     # the second call reuses buffers and streams
         oh = lcx.attn_fwd_host(qh, kh, vh, rope, device="cuda", workspace=ws, chunks=chunks,
-                               window=w.window, sinks=w.sinks)
+                               causal=causal, window=w.window, sinks=w.sinks, **extra)
         torch.cuda.synchronize()
         assert torch.equal(oh, ref.cpu())
 
