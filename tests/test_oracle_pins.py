@@ -361,9 +361,13 @@ def test_attention_matches_torch_sdpa_fp64(causal, W, S):
     m = torch.from_numpy(oracle.mask(L, causal, W, S))
     ref = torch.nn.functional.scaled_dot_product_attention(qr, kr, vv, attn_mask=m, scale=0.3)
     np.testing.assert_allclose(o, ref.numpy(), atol=1e-12, rtol=0)
-    logits = (qr @ kr.transpose(-1, -2)) * 0.3
-    ref_lse = torch.logsumexp(logits.masked_fill(~m, float("-inf")), dim=-1)
-    np.testing.assert_allclose(lse, ref_lse.numpy(), atol=1e-12, rtol=0)
+    # lse = max + ln sum exp(s - max) over the visible keys, evaluated in numpy
+    # fp64 on numpy's own matmul of the rotated operands
+    logits = np.where(m.numpy(), np.matmul(qr.numpy(), np.swapaxes(kr.numpy(), -1, -2)) * 0.3,
+                      -np.inf)
+    mx = logits.max(axis=-1, keepdims=True)
+    ref_lse = mx[..., 0] + np.log(np.exp(logits - mx).sum(axis=-1))
+    np.testing.assert_allclose(lse, ref_lse, atol=1e-12, rtol=0)
 
 
 def test_attention_equals_online_softmax_blocks():
