@@ -536,7 +536,22 @@ def main():
     ap.add_argument("--impl", default="lcx", choices=["lcx", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="only the split-KV decode measurement on the workload's cache "
+                         "(prints its object; for profiling, not a bench line)")
     args = ap.parse_args()
+    if args.decode_only:
+        import ntk_rope_flashattn_b200 as lcx
+        w = WORKLOADS[args.workload]
+        dev = torch.device("cuda", 0)
+        q, k, v = make_inputs(w, device=dev, seed=rank_seed(w, 0))
+        rope = lcx.RopeParams(w.mode, w.D, w.base, w.scale, w.original_max_pos, w.alpha,
+                              w.beta, w.pairing)
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        res = bench_decode(lcx, w, q, k, v, rope, torch.cuda.current_stream(dev), status,
+                           reps=args.steps)
+        print(json.dumps(res), flush=True)
+        return
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
