@@ -56,6 +56,12 @@ constexpr int kRegsIssue = 64;          // warpgroup 3: TMA and MMA issuing warp
 static_assert(2 * kRegsSoftmax + kRegsRotate + kRegsIssue == 4 * 128, "register file split");
 constexpr int kBM = 128;                // query rows per tile
 constexpr float kRescaleLog2 = 8.0f;    // rescale O only if the max grows by > 2^8
+// Build-time switches (-D...; the defaults are the measured-fastest choices):
+//   LCX_EMU_EVERY       1 column pair in N takes 2^x on the FMA pipe (0: none)
+//   LCX_D192_TWO_TILES  two query tiles and one V stage at D = 192 (0: one tile)
+//   LCX_KSTAGES_D128    K ring depth at D = 128 without split QK^T
+//   LCX_ROT_UNROLL      rows in flight per rotation thread
+//   LCX_PHASOR_CARRY    reuse the phasor a K tile ends with for the next tile
 #ifndef LCX_EMU_EVERY
 #define LCX_EMU_EVERY 0
 #endif
