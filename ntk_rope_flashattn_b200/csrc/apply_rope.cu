@@ -96,8 +96,9 @@ __device__ __forceinline__ void store_lo(const RopeArgs &a, int b, int l, int h,
 }
 
 // HALF pairing: a job covers N consecutive pairs i0..i0+N-1, i.e. the vector
-// at element i0 and the vector at element i0 + D/2.
-template <typename T, bool kHalf>
+// at element i0 and the vector at element i0 + D/2.  kLo: also write the lo
+// parts (bf16 only).
+template <typename T, bool kHalf, bool kLo>
 __global__ void __launch_bounds__(256) apply_rope_kernel(const __grid_constant__ RopeArgs a) {
     constexpr int N = Vec<T>::N;
     constexpr int P = kHalf ? N : N / 2;  // pairs per job
@@ -154,8 +155,8 @@ __global__ void __launch_bounds__(256) apply_rope_kernel(const __grid_constant__
                 const uint4 h1 = pack(y1), h2 = pack(y2);
                 __stcs(reinterpret_cast<uint4 *>(yr + e1), h1);
                 __stcs(reinterpret_cast<uint4 *>(yr + e2), h2);
-                if constexpr (sizeof(T) == 2)
-                    if (a.y_lo) store_lo(a, b, l, h0 + u, e1, e2, y1, y2, h1, h2);
+                if constexpr (sizeof(T) == 2 && kLo)
+                    store_lo(a, b, l, h0 + u, e1, e2, y1, y2, h1, h2);
             } else {
                 float x[N], y[N];
                 unpack(va[u], x);
@@ -166,8 +167,8 @@ __global__ void __launch_bounds__(256) apply_rope_kernel(const __grid_constant__
                 }
                 const uint4 h = pack(y);
                 __stcs(reinterpret_cast<uint4 *>(yr + e1), h);
-                if constexpr (sizeof(T) == 2)
-                    if (a.y_lo) store_lo(a, b, l, h0 + u, e1, -1, y, y, h, h);
+                if constexpr (sizeof(T) == 2 && kLo)
+                    store_lo(a, b, l, h0 + u, e1, -1, y, y, h, h);
             }
         }
     }
@@ -236,15 +237,17 @@ lcx_status apply_rope_impl(const lcx_rope_params *params, const void *x, void *y
     const int threads = a.rows_per_cta * a.jobs_per_row;
     dim3 grid(unsigned((L + a.rows_per_cta - 1) / a.rows_per_cta), unsigned(B));
     if (dtype == LCX_BF16) {
-        if (half)
-            apply_rope_kernel<__nv_bfloat16, true><<<grid, threads, 0, s>>>(a);
+        if (y_lo)
+            half ? apply_rope_kernel<__nv_bfloat16, true, true><<<grid, threads, 0, s>>>(a)
+                 : apply_rope_kernel<__nv_bfloat16, false, true><<<grid, threads, 0, s>>>(a);
         else
-            apply_rope_kernel<__nv_bfloat16, false><<<grid, threads, 0, s>>>(a);
+            half ? apply_rope_kernel<__nv_bfloat16, true, false><<<grid, threads, 0, s>>>(a)
+                 : apply_rope_kernel<__nv_bfloat16, false, false><<<grid, threads, 0, s>>>(a);
     } else {
         if (half)
-            apply_rope_kernel<float, true><<<grid, threads, 0, s>>>(a);
+            apply_rope_kernel<float, true, false><<<grid, threads, 0, s>>>(a);
         else
-            apply_rope_kernel<float, false><<<grid, threads, 0, s>>>(a);
+            apply_rope_kernel<float, false, false><<<grid, threads, 0, s>>>(a);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
