@@ -69,3 +69,45 @@ def test_random_configuration(i):
     ref_o, ref_lse = oracle_rows(q, k, v, rope, w.L - Lq, w.causal, w.window, w.sinks)
     compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_lse,
             24 if w.dtype == "f32" else 8)
+
+
+N_DRAWS_MLA = 40
+
+
+def draw_mla(i):
+    """Decoupled-RoPE configuration i: q/k head dim d_C + d_R with d_R = 64 (d_C
+    128 or 64), value dim 128, the rotary key shared by every head."""
+    r = np.random.default_rng(104729 + i)
+    Dc = int(r.choice([128, 64]))
+    G = int(r.choice([1, 2, 3, 4]))
+    Hkv = int(r.choice([1, 2]))
+    Lk = int(r.integers(1, 700))
+    window = int(r.integers(1, Lk + 1)) if r.random() < 0.35 else 0
+    sinks = int(r.integers(0, 100)) if window and r.random() < 0.5 else 0
+    Lq = Lk if r.random() < 0.5 else int(r.integers(1, Lk + 1))
+    rope = dict(mode=str(r.choice(["plain", "pi", "ntk", "yarn"])),
+                scale=float(r.choice([2.0, 4.0, 8.0])), original_max_pos=128,
+                pairing=str(r.choice(["half", "interleaved"])))
+    opts = dict(rotate_k_once=bool(r.random() < 0.5), num_splits=int(r.choice([1, 1, 3])))
+    return dict(B=int(r.choice([1, 2])), Hq=G * Hkv, Hkv=Hkv, Lk=Lk, Lq=Lq, Dc=Dc,
+                window=window, sinks=sinks, seed=int(r.integers(0, 1000)), rope=rope,
+                opts=opts)
+
+
+@pytest.mark.parametrize("i", range(N_DRAWS_MLA))
+def test_random_decoupled_rope(i):
+    from test_gpu_mla import mla_inputs, oracle_mla
+    c = draw_mla(i)
+    Dr, Dv = 64, 128
+    q_all, kc, kr, v = mla_inputs(c["B"], c["Hq"], c["Hkv"], c["Lk"], c["Dc"], Dr, Dv,
+                                  seed=c["seed"])
+    q = q_all[:, :, c["Lk"] - c["Lq"]:]
+    rope = lcx.RopeParams(head_dim=Dr, **c["rope"])
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = lcx.attn_fwd(q, kc, v, rope, k_rope=kr, window=c["window"], sinks=c["sinks"],
+                          q_offset=c["Lk"] - c["Lq"], return_lse=True, status=status,
+                          **c["opts"])
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, c
+    ref = oracle_mla(q, kc, kr, v, rope, c["Lk"] - c["Lq"], c["window"], c["sinks"])
+    compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref[0], ref[1])
