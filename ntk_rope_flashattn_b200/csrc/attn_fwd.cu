@@ -60,6 +60,8 @@ constexpr float kRescaleLog2 = 8.0f;    // rescale O only if the max grows by > 
 //   LCX_EMU_EVERY       1 column pair in N takes 2^x on the FMA pipe (0: none)
 //   LCX_D192_TWO_TILES  two query tiles and one V stage at D = 192 (0: one tile)
 //   LCX_KSTAGES_D128    K ring depth at D = 128 without split QK^T
+//   LCX_SPLIT_FUSED     split QK^T: Qhi [Klo; Khi]^T as one N = 128 product (key
+//                       parts interleaved by box) plus Qlo Khi^T, one S buffer
 //   LCX_ROT_UNROLL      rows in flight per rotation thread
 //   LCX_PHASOR_CARRY    reuse the phasor a K tile ends with for the next tile
 #ifndef LCX_EMU_EVERY
@@ -70,6 +72,9 @@ constexpr float kRescaleLog2 = 8.0f;    // rescale O only if the max grows by > 
 #endif
 #ifndef LCX_KSTAGES_D128
 #define LCX_KSTAGES_D128 2
+#endif
+#ifndef LCX_SPLIT_FUSED
+#define LCX_SPLIT_FUSED 1
 #endif
 #ifndef LCX_ROT_UNROLL
 #define LCX_ROT_UNROLL 2
@@ -139,14 +144,23 @@ struct Cfg {
     static constexpr int kOffV = kOffK + kStagesK * kParts * kTileK;
     static constexpr int kOffBar = kOffV + kStagesV * kTileV;
     static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers + alignment slack
-    // S buffers per query tile: the split mode's 64-key tiles leave TMEM room
-    // for two, so its S runs two key tiles ahead of PV.
-    static constexpr int kNB = kSplit ? 2 : 1;
-    // TMEM columns: S_t,b at (t kNB + b) BN (P_t,b aliased over its first BN/2
-    // columns), O_t after.
-    static constexpr int kColO = 2 * kNB * BN;
+    // Split mode, fused: the hi and lo parts of a K stage are interleaved box by
+    // box (lo box b, then hi box b), so that [Klo; Khi] is one 2 BN-row operand
+    // and Qhi [Klo; Khi]^T one N = 2 BN product; its S buffer is 2 BN columns
+    // (Qhi Klo^T, then Qhi Khi^T + Qlo Khi^T), one per query tile.  Otherwise
+    // the split mode's 64-key tiles leave TMEM room for two S buffers per query
+    // tile, so its S runs two key tiles ahead of PV.
+    static constexpr bool kFused = kSplit && LCX_SPLIT_FUSED != 0;
+    static constexpr int kNB = (kSplit && !kFused) ? 2 : 1;   // S buffers per query tile
+    static constexpr int kSCols = kFused ? 2 * BN : BN;       // TMEM columns of an S buffer
+    static constexpr int kKBoxStride = kFused ? 2 * kBoxK : kBoxK;  // between a part's boxes
+    static constexpr int kKHi = kFused ? kBoxK : 0;           // hi part in a K stage
+    static constexpr int kKLo = kFused ? 0 : kTileK;          // lo part in a K stage
+    // TMEM columns: S_t,b at (t kNB + b) kSCols (P_t,b aliased over its first
+    // BN/2 columns), O_t after.
+    static constexpr int kColO = 2 * kNB * kSCols;
     static_assert(kSmemBytes <= 232448, "shared memory budget");
-    static_assert(2 * kNB * BN + 2 * DV <= 512, "TMEM budget");
+    static_assert(2 * kNB * kSCols + 2 * DV <= 512, "TMEM budget");
 };
 
 template <int NSK, int NSV>
@@ -441,14 +455,16 @@ __device__ __forceinline__ void rotate_packed_q(uint8_t *tile, uint8_t *lo, long
     }
 }
 
-template <int D, int RD, bool kHalf, bool kSplit, int ROWS>
+// BS: bytes between the tile's 64-column boxes (ROWS x 128 unless the parts
+// of a split key tile are interleaved box by box).
+template <int D, int RD, bool kHalf, bool kSplit, int ROWS, int BS = ROWS * 128>
 __device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, uint8_t *lo, long long pos0,
                                                  const Phasor<RD, kHalf> &ph, const AttnParams &p,
                                                  bool rotate,
                                                  PhasorCarry<Rot<RD, kHalf>::PPJ> *carry = nullptr) {
     using R = Rot<RD, kHalf>;
     constexpr int NJ = ROWS / R::RP;
-    constexpr int BOX = ROWS * 128;
+    constexpr int BOX = BS;
     float c[R::PPJ], s[R::PPJ];
     if (rotate) {
         if (LCX_PHASOR_CARRY && carry && carry->next == pos0 && carry->age < kReseed) {
@@ -482,14 +498,14 @@ __device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, uint8_t *lo, lon
 // fp32 operands: load ROWS rows from global (rows >= L read as zero), rotate in
 // fp32 when asked (row r at position pos0 + r), round to bf16 (hi, and lo in
 // the split mode) into the tile.
-template <int D, bool kHalf, bool kSplit, int ROWS>
+template <int D, bool kHalf, bool kSplit, int ROWS, int BS = ROWS * 128>
 __device__ __forceinline__ void load_tile_f32(uint8_t *tile, uint8_t *lo, const float *base,
                                               long long rs, int row0, int L, long long pos0,
                                               bool rotate, const Phasor<D, kHalf> &ph,
                                               const AttnParams &p) {
     using R = Rot<D, kHalf>;
     constexpr int NJ = ROWS / R::RP;
-    constexpr int BOX = ROWS * 128;
+    constexpr int BOX = BS;
     float c[R::PPJ], s[R::PPJ];
     if (rotate) ph.start(pos0, p, c, s);
     for (int k = 0; k < NJ; ++k) {
@@ -778,10 +794,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(&bar.full_k[sk], lo ? 2 * C::kTileK : C::kTileK);
                     if (lo)
                         for (int bx = 0; bx < D / 64; ++bx)
-                            tma_load_4d(sK + sk * C::kParts * C::kTileK + C::kTileK + bx * C::kBoxK,
+                            tma_load_4d(sK + sk * C::kParts * C::kTileK + C::kKLo +
+                                            bx * C::kKBoxStride,
                                         &tmkr, &bar.full_k[sk], bx * 64, jt * BN, U.g, U.b);
                     for (int bx = 0; bx < D / 64; ++bx) {
-                        uint8_t *dst = sK + sk * C::kParts * C::kTileK + bx * C::kBoxK;
+                        uint8_t *dst =
+                            sK + sk * C::kParts * C::kTileK + C::kKHi + bx * C::kKBoxStride;
                         if constexpr (RD < D) {
                             if (p.k_rope_shared && bx >= kNopeBoxes) {
                                 tma_load_4d(dst, &tmkr, &bar.full_k[sk], (bx - kNopeBoxes) * 64,
@@ -812,6 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // ------------------------------------------------ MMA issuer
             if (lane == 0) {
                 constexpr uint32_t kIdS = idesc_bf16_f32(128, BN, 0, 0);
+                constexpr uint32_t kIdS2 = idesc_bf16_f32(128, 2 * BN, 0, 0);   // fused split
                 constexpr uint32_t kIdPV = idesc_bf16_f32(128, DV, 0, 1);
                 const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
                 // S_t = Q_t K^T over D in steps of 16 (32 bytes inside a 128-byte
@@ -826,7 +845,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 auto issue_s = [&](int t, int s, int b) {
                     const uint64_t qa = dq0 + ((t * C::kParts * C::kTileQ) >> 4);
                     const uint64_t ka = dk0 + ((s * C::kParts * C::kTileK) >> 4);
-                    const uint32_t dst = tmem + (t * NB + b) * BN;
+                    const uint32_t dst = tmem + (t * NB + b) * C::kSCols;
+                    if constexpr (C::kFused) {
+                        // Qhi [Klo; Khi]^T over the 2 BN rows of a box pair (lo box,
+                        // then hi box: 8-row groups 1024 bytes apart throughout),
+                        // then Qlo Khi^T onto the Qhi Khi^T half
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t oq = ((kk >> 2) * C::kBoxQ + (kk & 3) * 32) >> 4;
+                            const uint32_t ok_ = ((kk >> 2) * C::kKBoxStride + (kk & 3) * 32) >> 4;
+                            mma_ss(dst, qa + oq, ka + ok_, kIdS2, kk > 0);
+                        }
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t oq = ((kk >> 2) * C::kBoxQ + (kk & 3) * 32) >> 4;
+                            const uint32_t ok_ = ((kk >> 2) * C::kKBoxStride + (kk & 3) * 32) >> 4;
+                            mma_ss(dst + BN, qa + (C::kTileQ >> 4) + oq, ka + (C::kKHi >> 4) + ok_,
+                                   kIdS, true);
+                        }
+                        return;
+                    }
                     constexpr int NPROD = kSplit ? 3 : 1;
 #pragma unroll
                     for (int pr = 0; pr < NPROD; ++pr) {
@@ -843,7 +881,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // O_t += P_t V: P from TMEM (BN/2 columns of bf16 pairs), V MN-major.
                 auto issue_pv = [&](int t, int s, int b, bool acc) {
                     const uint64_t va = dv0 + ((s * C::kTileV) >> 4);
-                    const uint32_t dst = tmem + C::kColO + t * DV, pa = tmem + (t * NB + b) * BN;
+                    const uint32_t dst = tmem + C::kColO + t * DV;
+                    const uint32_t pa = tmem + (t * NB + b) * C::kSCols;
 #pragma unroll
                     for (int kk = 0; kk < BN / 16; ++kk)
                         mma_ts(dst, pa + kk * 8, va + ((kk * 2048) >> 4), kIdPV, (acc || kk > 0));
@@ -995,8 +1034,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_k[s], use & 1, abort, tmo));
                 if (!ok) break;
                 if (rotk || kSplit)
-                    rotate_tile_bf16<D, RD, kHalf, kSplit, BN>(
-                        tk, tk + C::kTileK, (long long)jt * BN, ph, p, rotk, &kcarry);
+                    rotate_tile_bf16<D, RD, kHalf, kSplit, BN, C::kKBoxStride>(
+                        tk + C::kKHi, tk + C::kKLo, (long long)jt * BN, ph, p, rotk, &kcarry);
             } else {
                 if (use > 0)
                     ok = __all_sync(0xffffffffu,
@@ -1004,8 +1043,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 const float *base = reinterpret_cast<const float *>(p.k) + U.b * p.ks[0] +
                                     (long long)U.g * p.ks[1];
-                load_tile_f32<D, kHalf, kSplit, BN>(tk, tk + C::kTileK, base, p.ks[2], jt * BN,
-                                                    p.Lk, (long long)jt * BN, rotk, ph, p);
+                load_tile_f32<D, kHalf, kSplit, BN, C::kKBoxStride>(
+                    tk + C::kKHi, tk + C::kKLo, base, p.ks[2], jt * BN, p.Lk, (long long)jt * BN,
+                    rotk, ph, p);
             }
             fence_proxy_async_smem();
             mbar_arrive(&bar.ready_k[s]);
@@ -1048,7 +1088,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int it = 0; it < n_it; ++it) {
                 const int j = ilv ? 2 * it + t : it;
                 const int b = it % NB;
-                const uint32_t s_col = (t * NB + b) * BN;
+                const uint32_t s_col = (t * NB + b) * C::kSCols;
                 ok = __all_sync(0xffffffffu,
                                 mbar_wait(&bar.s_ready[t][b], (it / NB) & 1, abort, tmo));
                 if (!ok) break;
@@ -1068,7 +1108,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
                 // The whole S row of this thread in one TMEM load.
                 float v[BN];
-                tmem_ld_row(trow + s_col, v);
+                if constexpr (C::kFused) {
+                    // columns [0, BN): Qhi Klo^T; [BN, 2 BN): Qhi Khi^T + Qlo Khi^T
+                    float w[2 * BN];
+                    tmem_ld_row(trow + s_col, w);
+    #pragma unroll
+                    for (int e = 0; e < BN; ++e) v[e] = w[e] + w[e + BN];
+                } else {
+                    tmem_ld_row(trow + s_col, v);
+                }
                 if (partial) {
     #pragma unroll
                     for (int e = 0; e < BN; ++e)
