@@ -412,7 +412,11 @@ def bench_decode(lcx, w, q, k, v, rope, stream, status, reps=20):
     od = torch.empty_like(qd)
     kw = dict(causal=True, window=w.window, sinks=w.sinks, softmax_scale=w.softmax_scale,
               split_qk=w.split_qk, out=od, status=status, q_offset=w.L - 1)
-    nbytes = sum(t.numel() * t.element_size() for t in (k, v, qd, od))
+    # algorithmic bytes: q and o, and the K and V rows of the keys the new token
+    # sees (the whole cache, or its window and sinks)
+    n_vis = _row_visible(w, w.L - 1)
+    kv_row = (k.shape[3] * k.element_size() + v.shape[3] * v.element_size()) * w.B * w.Hkv
+    nbytes = n_vis * kv_row + sum(t.numel() * t.element_size() for t in (qd, od))
     sweep = {}
     # the powers of two, and the count that gives every SM one CTA of a kv group
     sms = torch.cuda.get_device_properties(q.device).multi_processor_count
@@ -448,8 +452,8 @@ def bench_decode(lcx, w, q, k, v, rope, stream, status, reps=20):
     del k_rot
     assert int(status.item()) == 0, "device watchdog fired in decode"
     us = sweep[best] * 1e3
-    return {"what": "1 new token per head (B=%d, Hq=%d) against %d cached keys, q_offset = "
-                    "L - 1, keys rotated on chip" % (w.B, w.Hq, w.L),
+    return {"what": "1 new token per head (B=%d, Hq=%d) against %d cached keys (%d of them "
+                    "visible), q_offset = L - 1, keys rotated on chip" % (w.B, w.Hq, w.L, n_vis),
             "bound": "hbm", "num_splits": best, "us_per_call": round(us, 2),
             "us_by_splits": {str(s_): round(t * 1e3, 2) for s_, t in sweep.items()},
             "bytes": nbytes, "achieved": round(nbytes / (us * 1e-6) / 1e9, 1), "unit": "GB/s",

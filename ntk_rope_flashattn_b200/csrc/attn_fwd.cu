@@ -1651,16 +1651,18 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
     // the G heads of a kv group share the CTA's query tiles (pack_lp rows per
     // head: L rounded up to 8 rows), so every K/V tile is read and rotated once
     // per kv group instead of once per head pair.
-    //  - bf16, plain QK^T, G pack_lp <= 128: both tiles hold all G heads (rows
+    //  - bf16, one S buffer per query tile (plain QK^T, or split QK^T with its
+    //    products fused), G pack_lp <= 128: both tiles hold all G heads (rows
     //    [0, G pack_lp), tile 1 shifted by whole warps when that fits, so the
     //    busy softmax warps of the two tiles use different SMSPs) and tile t
     //    takes the key tiles j = t mod 2: two K/V tiles in flight per CTA, two
     //    partial results per split.
-    //  - otherwise, G even and G/2 pack_lp <= 128: G/2 heads per tile, both
-    //    tiles multiply every key tile.
+    //  - otherwise (fp32, unfused split QK^T, G pack_lp > 128), G even and
+    //    G/2 pack_lp <= 128: G/2 heads per tile, both tiles multiply every key
+    //    tile.
     const int64_t lp = (a->L + 7) / 8 * 8;
     int n_parts = num_splits;
-    if (!x.f32 && !x.split_qk && x.D <= 128 && lp * x.p.G <= kBM) {
+    if (!x.f32 && (!x.split_qk || LCX_SPLIT_FUSED) && x.D <= 128 && lp * x.p.G <= kBM) {
         const int used = int(lp) * x.p.G;
         x.p.pack_lp = int(lp);
         x.p.pack_hpt = x.p.G;

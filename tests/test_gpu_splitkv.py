@@ -144,6 +144,11 @@ def test_splitkv_head_packed_decode(L, Hq, Hkv, extra):
     (1, 1500, 5, dict(Hq=2, Hkv=2)),                 # G = 1
     (4, 3000, 6, dict(Hq=8, Hkv=2, window=700, sinks=4)),
     (1, 2000, 4, dict(Hq=8, Hkv=2, k_prerotated=True)),
+    # split QK^T (64-key tiles, fused products): odd counts, one tile per split,
+    # keys split by the rotate pass
+    (1, 1800, 2, dict(Hq=8, Hkv=2, split_qk=True)),
+    (2, 777, 13, dict(Hq=6, Hkv=2, split_qk=True)),
+    (3, 2000, 5, dict(Hq=8, Hkv=2, split_qk=True, rotate_k_once=True)),
 ])
 def test_splitkv_interleaved_key_tiles(L, Lk, splits, extra):
     """bf16 head-packed split-KV: both query tiles hold all G heads and take
@@ -151,12 +156,13 @@ def test_splitkv_interleaved_key_tiles(L, Lk, splits, extra):
     head's rows against the oracle, edge counts of key tiles included."""
     extra = dict(extra)
     prerot = extra.pop("k_prerotated", False)
+    once = extra.pop("rotate_k_once", False)
     w = W0.with_(**extra, L=Lk)
     q_all, k, v = make_inputs(w, device="cuda")
     q = q_all[:, :, Lk - L:]
     rope = rope_of(w)
     kk = lcx.apply_rope(k, rope) if prerot else k
     o, lse = run_split(q, kk, v, rope, splits, window=w.window, sinks=w.sinks, q_offset=Lk - L,
-                       k_prerotated=prerot)
+                       k_prerotated=prerot, split_qk=w.split_qk, rotate_k_once=once)
     ref = oracle_rows(q, k, v, rope, Lk - L, True, w.window, w.sinks)
     compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref[0], ref[1])
