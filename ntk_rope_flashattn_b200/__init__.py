@@ -236,7 +236,8 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
     supplies that part of every key once for all heads and k holds the first
     D - rope.head_dim dims.  v / o may have their own head dim (v.shape[-1]).
     ``rotate_k_once`` (or a ``k_rot`` buffer shaped like k, twice that in the
-    split-QK^T mode with bf16 keys): the keys are rotated once into that buffer
+    split-QK^T mode with bf16 keys, or like k_rope with decoupled RoPE): the
+    keys (with k_rope: the shared rotary key) are rotated once into that buffer
     by the rotate pass before the kernel, which then reads them pre-rotated
     (split mode: as hi/lo bf16 parts), instead of rotating each key tile on chip
     in every CTA that reads it (ignored where the kernel does not rotate keys).
