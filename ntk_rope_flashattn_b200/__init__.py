@@ -383,6 +383,35 @@ def attn_merge(o_parts, lse_parts, out=None, lse=None, dtype=None):
     return out, lse
 
 
+def host_pieces(B, Hkv, L, chunks, causal=True, q_offset=0, one_piece=False):
+    """The pieces attn_fwd_host cuts a call into: (batch or None, first kv head,
+    end kv head, first query row, end query row).  About ``chunks`` pieces of
+    whole kv-head groups, one batch entry at a time (one piece covering
+    everything when ``one_piece``).  Causal prefill (q_offset 0): the first
+    piece starts with about its first quarter of query rows and the last piece
+    ends with about its last quarter, cut on 128-row query blocks -- a query
+    range [i0, i1) needs only the keys [0, i1), so less input is copied before
+    the first kernel and less output after the last, and every query tile
+    starts where it does in one call over everything."""
+    if one_piece:
+        return [(None, 0, Hkv, 0, L)]
+    per_b = max(1, min(Hkv, -(-int(chunks) // B)))
+    bounds = [round(i * Hkv / per_b) for i in range(per_b + 1)]
+    pieces = [(b, g0, g1, 0, L) for b in range(B) for g0, g1 in zip(bounds, bounds[1:])
+              if g1 > g0]
+    q4 = (L // 4) // 128 * 128
+    if causal and not q_offset and q4 >= 128:
+        c = (L - q4) // 128 * 128           # start of the last piece's rows
+        b0, g00, g01, _, _ = pieces[0]
+        head = [(b0, g00, g01, 0, q4), (b0, g00, g01, q4, L)]
+        if len(pieces) == 1:
+            pieces = head[:1] + [(b0, g00, g01, q4, c), (b0, g00, g01, c, L)]
+        else:
+            bl, gl0, gl1, _, _ = pieces[-1]
+            pieces = head + pieces[1:-1] + [(bl, gl0, gl1, 0, c), (bl, gl0, gl1, c, L)]
+    return pieces
+
+
 def attn_fwd_host(q, k, v, rope: RopeParams, device="cuda", workspace=None, chunks=8, **kw):
     """attn_fwd on HOST tensors [B, H, L, D]: copies q/k/v to the device, runs
     the kernel and copies o back to the host (pinned host memory makes the
@@ -418,34 +447,9 @@ def attn_fwd_host(q, k, v, rope: RopeParams, device="cuda", workspace=None, chun
     if o_host is None or tuple(o_host.shape) != o_shape or o_host.dtype != q.dtype:
         o_host = torch.empty(o_shape, dtype=q.dtype, pin_memory=True)
         ws["o_host"] = o_host
-    # pieces: (batch, first kv head, end kv head, first query row, end query
-    # row); one piece when the caller wants per-row statistics back (lse /
-    # status buffers cover everything)
-    per_b = max(1, min(Hkv, -(-int(chunks) // B)))
-    if "lse" in kw or kw.get("return_lse"):
-        pieces = [(None, 0, Hkv, 0, L)]
-    else:
-        bounds = [round(i * Hkv / per_b) for i in range(per_b + 1)]
-        pieces = [(b, g0, g1, 0, L) for b in range(B) for g0, g1 in zip(bounds, bounds[1:])
-                  if g1 > g0]
-        # Causal prefill: a query range [i0, i1) needs only the keys [0, i1),
-        # so the first piece starts with about its first quarter of query rows
-        # (less input to copy before the first kernel) and the last piece ends
-        # with about its last quarter (less output to copy after the last
-        # kernel).  Cuts sit on 128-row query blocks, so every query tile
-        # starts where it does in one call over everything (its rows are
-        # rotated from the same start) and meets the same key tiles in the
-        # same order.
-        q4 = (L // 4) // 128 * 128
-        if kw.get("causal", True) and not kw.get("q_offset", 0) and q4 >= 128:
-            c = (L - q4) // 128 * 128           # start of the last piece's rows
-            b0, g00, g01, _, _ = pieces[0]
-            head = [(b0, g00, g01, 0, q4), (b0, g00, g01, q4, L)]
-            if len(pieces) == 1:
-                pieces = head[:1] + [(b0, g00, g01, q4, c), (b0, g00, g01, c, L)]
-            else:
-                bl, gl0, gl1, _, _ = pieces[-1]
-                pieces = head + pieces[1:-1] + [(bl, gl0, gl1, 0, c), (bl, gl0, gl1, c, L)]
+    pieces = host_pieces(B, Hkv, L, chunks, causal=kw.get("causal", True),
+                         q_offset=kw.get("q_offset", 0),
+                         one_piece="lse" in kw or bool(kw.get("return_lse")))
 
     def view(t, b, h0, h1, r0=None, r1=None):
         t = t[:, h0:h1] if b is None else t[b:b + 1, h0:h1]
