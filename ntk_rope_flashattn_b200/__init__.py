@@ -350,7 +350,9 @@ def attn_fwd_split_static(q, k, v, rope: RopeParams, num_splits: int, causal: bo
 
 
 def split_workspace_bytes(B, Hq, L, D, num_splits):
-    """Bytes of workspace lcx_attn_fwd_split needs (0 for one split)."""
+    """Bytes of workspace lcx_attn_fwd_split needs (0 for one split): fp32
+    partial outputs and LSEs for two partial results per split (head-packed
+    launches give each of a split's query tiles every other key tile)."""
     n = int(load().lcx_attn_split_workspace_bytes(B, Hq, L, D, int(num_splits)))
     if n < 0:
         raise ValueError("invalid split-KV sizes")
