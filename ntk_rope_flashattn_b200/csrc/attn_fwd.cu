@@ -126,7 +126,11 @@ struct AttnParams {
 // K tile has a second "lo" part holding bf16(x' - bf16(x')), and key tiles are
 // 64 rows so that both parts fit.  D is the query/key head dim, DV the
 // value/output head dim; at D = 192 (decoupled RoPE: 128 + 64) two query tiles
-// (96 KB) leave room for two K stages (48 KB each) and one V stage.
+// (96 KB) leave room for one K stage (48 KB) and two V stages (32 KB each).
+// The K stage is released as soon as both S products of key tile j are done,
+// so key tile j + 1 lands while the softmax of j runs; the second V stage lets
+// V(j + 1) land while PV(j) still reads V(j).  That beats two K stages with one
+// V stage (1038 vs 942 TFLOP/s on a 16-head L 16384 prefill).
 template <int D, int DV, bool kSplit>
 struct Cfg {
     static constexpr int BN = kSplit ? 64 : 128;        // keys per tile
@@ -137,8 +141,10 @@ struct Cfg {
     static constexpr int kTileV = BN * DV * 2;          // a V tile
     static constexpr int kBoxQ = kBM * 128;
     static constexpr int kBoxK = BN * 128;
-    static constexpr int kStagesK = (D == 64) ? 4 : (D == 128 && !kSplit) ? LCX_KSTAGES_D128 : 2;
-    static constexpr int kStagesV = (D == 64) ? 4 : (D > 128 && kNTQ == 2) ? 1 : 2;
+    static constexpr int kStagesK = (D == 64) ? 4
+                                  : (D == 128 && !kSplit) ? LCX_KSTAGES_D128
+                                  : (D > 128 && kNTQ == 2) ? 1 : 2;
+    static constexpr int kStagesV = (D == 64) ? 4 : 2;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kNTQ * kParts * kTileQ;
     static constexpr int kOffV = kOffK + kStagesK * kParts * kTileK;
