@@ -58,7 +58,7 @@ constexpr int kBM = 128;                // query rows per tile
 constexpr float kRescaleLog2 = 8.0f;    // rescale O only if the max grows by > 2^8
 // Build-time switches (-D...; the defaults are the measured-fastest choices):
 //   LCX_EMU_EVERY       1 column pair in N takes 2^x on the FMA pipe (0: none)
-//   LCX_D192_TWO_TILES  two query tiles and one V stage at D = 192 (0: one tile)
+//   LCX_D192_TWO_TILES  two query tiles and one K stage at D = 192 (0: one tile)
 //   LCX_KSTAGES_D128    K ring depth at D = 128 without split QK^T
 //   LCX_SPLIT_FUSED     split QK^T: Qhi [Klo; Khi]^T as one N = 128 product (key
 //                       parts interleaved by box) plus Qlo Khi^T, one S buffer
