@@ -667,12 +667,15 @@ def test_mla_without_nope_part_is_shared_key_attention():
     np.testing.assert_allclose(lse.reshape(B, Hq, L), ref_l, atol=1e-12, rtol=0)
 
 
-@pytest.mark.parametrize("pairing", ["half", "interleaved"])
-def test_mla_matches_torch_sdpa_on_concatenated_vectors(pairing):
+@pytest.mark.parametrize("pairing,Hkv", [("half", 4), ("interleaved", 4), ("half", 2)])
+def test_mla_matches_torch_sdpa_on_concatenated_vectors(pairing, Hkv):
     """Reduction to a library routine: torch's fp64 scaled_dot_product_attention
     on explicitly concatenated [q_C ; rotated q_R] and [k_C ; rotated k_R] (the
-    rotation pinned above, mscale on the rotated parts), value dim d_v != d_qk."""
-    B, Hq, Hkv, L, Dc, Dr, Dv = 2, 4, 4, 29, 48, 16, 24
+    rotation pinned above, mscale on the rotated parts), value dim d_v != d_qk;
+    with Hkv < Hq, query head h takes the k_C and v of head h // G (K/V
+    replicated G times before the library call)."""
+    B, Hq, L, Dc, Dr, Dv = 2, 4, 29, 48, 16, 24
+    G = Hq // Hkv
     table, ms, _ = oracle.rope_table("yarn", Dr, scale=8.0, original_max_pos=4)
     assert ms > 1.0
     q, kc, kr, v = _mla_inputs(B, Hq, Hkv, L, Dc, Dr, Dv, 61)
@@ -684,11 +687,11 @@ def test_mla_matches_torch_sdpa_on_concatenated_vectors(pairing):
     krr = oracle.rotate_rows(kr.reshape(-1, Dr), np.tile(np.arange(L), B), table, ms,
                              pairing).reshape(B, 1, L, Dr)
     qcat = torch.from_numpy(np.concatenate([q[..., :Dc].astype(np.float64), qr], axis=-1))
-    kcat = torch.from_numpy(np.concatenate([kc.astype(np.float64),
-                                            np.repeat(krr, Hkv, axis=1)], axis=-1))
+    kcat = torch.from_numpy(np.concatenate([np.repeat(kc, G, axis=1).astype(np.float64),
+                                            np.repeat(krr, Hq, axis=1)], axis=-1))
     m = torch.from_numpy(oracle.mask(L, True, 11, 3))
     ref = torch.nn.functional.scaled_dot_product_attention(
-        qcat, kcat, torch.from_numpy(v.astype(np.float64)), attn_mask=m,
+        qcat, kcat, torch.from_numpy(np.repeat(v, G, axis=1).astype(np.float64)), attn_mask=m,
         scale=1.0 / math.sqrt(Dc + Dr))
     np.testing.assert_allclose(o.reshape(B, Hq, L, Dv), ref.numpy(), atol=1e-12, rtol=0)
     logits = (qcat @ kcat.transpose(-1, -2)) / math.sqrt(Dc + Dr)
