@@ -92,6 +92,19 @@ MUTANTS = {
     "sinks_one_too_many": (
         "S + 1 sink keys (10.2)", C_SRC,
         [("if (j < sinks) return 1;", "if (j <= sinks) return 1;")]),
+    "noncausal_hides_future": (
+        "attention without the causal mask still hides later keys (2.4)", C_SRC,
+        [("if (!causal) return 1;", "if (!causal) return j <= i;")]),
+    "sinks_seen_by_earlier_queries": (
+        "sink keys visible to queries before them (10.2: sinks are earlier tokens)", C_SRC,
+        [("    if (j > i) return 0;\n    if (window <= 0) return 1;",
+          "    if (window > 0 && j < sinks) return 1;\n    if (j > i) return 0;\n"
+          "    if (window <= 0) return 1;")]),
+    "table_truncated": (
+        "the fp32 table truncated toward zero instead of rounded to nearest", C_SRC,
+        [("table[i] = (float)tp[i];",
+          "{ float f_ = (float)tp[i]; if ((double)f_ > tp[i]) f_ = nextafterf(f_, 0.0f); "
+          "table[i] = f_; }")]),
     "gqa_heads_interleaved": (
         "query head h reads kv head h mod Hkv instead of floor(h / G)", C_SRC,
         [("if (row_b[r] == b && row_h[r] / G == g) sel[ns++] = r;",
