@@ -1492,9 +1492,9 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     // A window of Lk or more keys, or Lk sinks, no longer restricts anything.
     p.window = int(a->window > Lk ? Lk : a->window);
     p.sinks = int(a->sinks > Lk ? Lk : a->sinks);
-    // Two query heads share a CTA's K/V tiles when the group allows it and
-    // two query tiles fit (D = 192 leaves room for one); with an odd group the
-    // two tiles are consecutive query blocks of one head instead.
+    // Two query heads share a CTA's K/V tiles when the group allows it and the
+    // CTA holds two query tiles (at D = 192 only with LCX_D192_TWO_TILES); with
+    // an odd group the two tiles are consecutive query blocks of one head.
     const bool two_tiles = a->D <= 128 || LCX_D192_TWO_TILES;
     p.heads_per_unit = (p.G % 2 == 0 && two_tiles) ? 2 : 1;
     p.qpair = (p.G % 2 == 1 && two_tiles) ? 1 : 0;
