@@ -23,7 +23,8 @@
  *
  * Parity pins: every function here is pinned by tests/test_oracle_pins.py
  * (printed worked values, closed forms, invariants, brute force).  No function
- * is "parity unpinned".
+ * is "parity unpinned".  tests/test_oracle_mutants.py plants single mistakes in
+ * copies of this file and checks that those pins fail on each.
  */
 #include <math.h>
 #include <stdint.h>
