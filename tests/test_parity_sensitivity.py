@@ -1,0 +1,145 @@
+"""The GPU parity comparison is sharp enough to see a kernel that gets its own
+arithmetic wrong.
+
+A kernel can make the same mistakes as the oracle's mutants: a mask
+off-by-one, a wrong pairing or rotation sign, mscale on one component only,
+the wrong kv head, a missing score scale, or bad softmax statistics.  For each
+such mistake, a copy of the oracle with it planted stands in for the kernel.
+It is compared with the unchanged oracle by the GPU tests' own comparison
+(test_gpu_attn.compare: max-abs 2e-2 beyond the output's rounding, mean-abs
+2e-3, LSE 2e-2), on inputs drawn like the GPU tests' small cases.  At least one
+of those cases must fail the comparison.  Everything runs on the CPU.  The
+RoPE table is the unchanged oracle's on both sides, because the kernel takes
+its table from the host.
+"""
+import importlib.util
+import os
+import sys
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from test_gpu_attn import BASE, SMALL, compare, table_of
+from test_oracle_mutants import MUTANTS, _copy_oracle
+from workloads import make_inputs
+
+# mistakes a kernel could make in its own arithmetic (the table comes from the host)
+PREFILL_MUTANTS = [
+    "causal_sees_next_key", "causal_hides_diagonal", "window_one_too_wide",
+    "sinks_one_too_many", "sinks_seen_by_earlier_queries", "noncausal_hides_future",
+    "rotation_first_sign", "rotation_second_sign", "rotation_mscale_one_component",
+    "half_pairing_mirrored", "interleaved_pair_reversed", "gqa_heads_interleaved",
+    "lse_without_max", "output_not_normalised", "default_scale_one_over_d",
+]
+MLA_MUTANTS = [
+    "mla_rope_slice_first", "mla_key_without_mscale", "mla_key_positions_across_batch",
+    "mla_heads_interleaved", "mla_lse_without_max", "mla_default_scale_rope_dims",
+]
+
+# decoupled-RoPE shapes of the GPU tests (test_gpu_mla.py and the random
+# decoupled-RoPE draws, which include batch 2): (B, Dc, Hq, Hkv, L, pairing, W, S)
+MLA_CASES = [
+    (1, 128, 4, 4, 700, "half", 0, 0),
+    (1, 128, 8, 2, 333, "half", 150, 4),
+    (1, 128, 2, 2, 257, "interleaved", 0, 0),
+    (2, 64, 3, 1, 200, "half", 0, 0),
+]
+
+
+@pytest.fixture(scope="module")
+def copies(tmp_path_factory):
+    """name -> the oracle package copy with that mistake planted, imported
+    under its own module name (its library built in its own folder); the
+    "unchanged" copy has none."""
+    mods = {}
+    for name in ["unchanged"] + PREFILL_MUTANTS + MLA_MUTANTS:
+        _, file, edits = MUTANTS[name] if name in MUTANTS else ("", "lcx_oracle.c", [])
+        dst = str(tmp_path_factory.mktemp("sens_" + name))
+        err = _copy_oracle(dst, edits, file)
+        assert err is None, err
+        pkg = os.path.join(dst, "oracle")
+        modname = "oracle_mutant_" + name
+        spec = importlib.util.spec_from_file_location(
+            modname, os.path.join(pkg, "__init__.py"), submodule_search_locations=[pkg])
+        mod = importlib.util.module_from_spec(spec)
+        sys.modules[modname] = mod
+        spec.loader.exec_module(mod)
+        assert os.path.dirname(mod.__file__) == pkg
+        mods[name] = mod
+    yield mods
+    for name in mods:
+        sys.modules.pop("oracle_mutant_" + name, None)
+
+
+def _cases():
+    ws = [BASE.with_(**kw) for kw in SMALL.values()]
+    return sorted(ws, key=lambda w: w.B * w.Hq * w.L * w.L * w.D)   # cheapest first
+
+
+_ref_cache = {}
+
+
+def _prefill(lib, w):
+    q, k, v = (t.float().numpy() for t in make_inputs(w, device="cpu"))
+    table, ms = table_of(w)
+    scale = w.softmax_scale if w.softmax_scale > 0 else None
+    return lib.attn_full(q, k, v, table, ms, w.pairing, 0, w.causal, w.window, w.sinks, scale)
+
+
+def _caught(got, ref, out_bits):
+    try:
+        compare(got[0], got[1], ref[0], ref[1], out_bits)
+    except AssertionError:
+        return True
+    return False
+
+
+def test_unchanged_copy_passes_the_comparison(copies):
+    """The harness itself: a copy without a planted mistake passes (on the
+    cheapest cases), so a failure below comes from the mistake."""
+    for w in _cases()[:6]:
+        ref = _ref_cache.setdefault(repr(w), _prefill(oracle, w))
+        assert not _caught(_prefill(copies["unchanged"], w), ref, 24 if w.dtype == "f32" else 8)
+    for case in MLA_CASES[:2]:
+        ref = _ref_cache.setdefault(("mla",) + case, _mla(oracle, case))
+        assert not _caught(_mla(copies["unchanged"], case), ref, 8)
+
+
+@pytest.mark.parametrize("name", PREFILL_MUTANTS)
+def test_prefill_comparison_sees_kernel_mistake(copies, name):
+    for w in _cases():
+        key = repr(w)
+        if key not in _ref_cache:
+            _ref_cache[key] = _prefill(oracle, w)
+        got = _prefill(copies[name], w)
+        if _caught(got, _ref_cache[key], 24 if w.dtype == "f32" else 8):
+            return
+    pytest.fail("no GPU small case's comparison sees %r (%s)" % (name, MUTANTS[name][0]))
+
+
+def _mla(lib, case, seed=11):
+    B, Dc, Hq, Hkv, L, pairing, W, S = case
+    Dr, Dv = 64, 128
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn((B, Hq, L, Dc + Dr), generator=g).bfloat16().float().numpy()
+    kc = torch.randn((B, Hkv, L, Dc), generator=g).bfloat16().float().numpy()
+    kr = torch.randn((B, L, Dr), generator=g).bfloat16().float().numpy()
+    v = torch.randn((B, Hkv, L, Dv), generator=g).bfloat16().float().numpy()
+    table, ms, _ = oracle.rope_table("yarn", Dr, scale=8.0, original_max_pos=128)
+    bb, hh, ii = np.meshgrid(np.arange(B), np.arange(Hq), np.arange(L), indexing="ij")
+    o, lse = lib.attn_rows_mla(q.reshape(-1, Dc + Dr), bb.ravel(), hh.ravel(), ii.ravel(), kc,
+                               kr, v, Hq, table, ms, pairing, 0, True, W, S)
+    return o, lse
+
+
+@pytest.mark.parametrize("name", MLA_MUTANTS)
+def test_decoupled_rope_comparison_sees_kernel_mistake(copies, name):
+    for case in MLA_CASES:
+        key = ("mla",) + case
+        if key not in _ref_cache:
+            _ref_cache[key] = _mla(oracle, case)
+        if _caught(_mla(copies[name], case), _ref_cache[key], 8):
+            return
+    pytest.fail("no decoupled-RoPE case's comparison sees %r (%s)" % (name, MUTANTS[name][0]))
