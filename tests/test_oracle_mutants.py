@@ -127,6 +127,10 @@ MUTANTS = {
         "a partial result over keys [k_begin, k_end) that also takes keys before k_begin",
         C_SRC,
         [("if (j < c->k_begin || j >= c->k_end ||", "if (j >= c->k_end ||")]),
+    "key_range_end_ignored": (
+        "a partial result over keys [k_begin, k_end) that also takes keys from k_end on",
+        C_SRC,
+        [("if (j < c->k_begin || j >= c->k_end ||", "if (j < c->k_begin ||")]),
     "merge_equal_weights": (
         "merge averages the partial outputs instead of weighting by e^lse (8.3.4)", C_SRC,
         [("double w = exp(l - m);", "double w = 1.0;")]),
@@ -152,6 +156,10 @@ MUTANTS = {
         "the short factor table used for long sequences and the long one for short (7.4)",
         C_SRC,
         [("(factors_short && seq_len <= L_train)", "(factors_short && seq_len > L_train)")]),
+    "short_factors_threshold": (
+        "the short factor table dropped at seq_len = L_train already (7.4: it holds up to "
+        "the training length)", C_SRC,
+        [("(factors_short && seq_len <= L_train)", "(factors_short && seq_len < L_train)")]),
     "mla_rope_slice_first": (
         "decoupled RoPE takes q_R from the front of the query row (9.5)", C_SRC,
         [("xr[d] = (double)c->q[r * Dq + c->Dc + d];", "xr[d] = (double)c->q[r * Dq + d];")]),
