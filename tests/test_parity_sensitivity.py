@@ -3,7 +3,8 @@ arithmetic wrong.
 
 A kernel can make the same mistakes as the oracle's mutants: a mask
 off-by-one, a wrong pairing or rotation sign, mscale on one component only,
-the wrong kv head, a missing score scale, or bad softmax statistics.  For each
+the wrong kv head, a missing score scale, bad softmax statistics, a key split
+that reads outside its stretch, or a merge that weights its parts wrongly.  For each
 such mistake, a copy of the oracle with it planted stands in for the kernel.
 It is compared with the unchanged oracle by the GPU tests' own comparison
 (test_gpu_attn.compare: max-abs 2e-2 beyond the output's rounding, mean-abs
@@ -22,6 +23,7 @@ import torch
 
 import oracle
 from test_gpu_attn import BASE, SMALL, compare, table_of
+from test_gpu_decode import W0, oracle_rows, rope_of
 from test_oracle_mutants import MUTANTS, _copy_oracle
 from workloads import make_inputs
 
@@ -32,6 +34,12 @@ PREFILL_MUTANTS = [
     "rotation_first_sign", "rotation_second_sign", "rotation_mscale_one_component",
     "half_pairing_mirrored", "interleaved_pair_reversed", "gqa_heads_interleaved",
     "lse_without_max", "output_not_normalised", "default_scale_one_over_d",
+]
+# mistakes of a split-KV launch: a split that reads outside its stretch of keys,
+# or a merge that combines the partial results wrongly
+SPLIT_MUTANTS = [
+    "key_range_start_ignored", "key_range_end_ignored", "merge_equal_weights",
+    "merge_lse_without_max", "merge_not_normalised",
 ]
 MLA_MUTANTS = [
     "mla_rope_slice_first", "mla_key_without_mscale", "mla_key_positions_across_batch",
@@ -54,7 +62,7 @@ def copies(tmp_path_factory):
     under its own module name (its library built in its own folder); the
     "unchanged" copy has none."""
     mods = {}
-    for name in ["unchanged"] + PREFILL_MUTANTS + MLA_MUTANTS:
+    for name in ["unchanged"] + PREFILL_MUTANTS + SPLIT_MUTANTS + MLA_MUTANTS:
         _, file, edits = MUTANTS[name] if name in MUTANTS else ("", "lcx_oracle.c", [])
         dst = str(tmp_path_factory.mktemp("sens_" + name))
         err = _copy_oracle(dst, edits, file)
@@ -143,3 +151,55 @@ def test_decoupled_rope_comparison_sees_kernel_mistake(copies, name):
         if _caught(_mla(copies[name], case), _ref_cache[key], 8):
             return
     pytest.fail("no decoupled-RoPE case's comparison sees %r (%s)" % (name, MUTANTS[name][0]))
+
+
+# split-KV shapes of the GPU tests (test_gpu_splitkv.py): (L, Lk, splits, extra)
+SPLIT_CASES = [
+    (1, 777, 3, {}),
+    (4, 5000, 8, dict(window=1000, sinks=4)),
+    (2, 900, 5, dict(window=300, sinks=2)),
+    (1, 4096, 32, dict(Hq=8, Hkv=2)),
+]
+
+
+def _split(rows_lib, merge_lib, case):
+    """Split-KV the way the kernel partitions it (reading 27: split s takes the
+    s-th stretch of ceil(n / splits) key tiles of 128, later ones may be empty),
+    each split by rows_lib over its key range, combined by merge_lib."""
+    L, Lk, splits, extra = case
+    w = W0.with_(**extra, L=Lk)
+    q_all, k, v = make_inputs(w, device="cpu")
+    q = q_all[:, :, Lk - L:]
+    rope = rope_of(w)
+    B, Hq, _, D = q.shape
+    table, ms, _ = oracle.rope_table(rope.mode, D, rope.base, rope.scale, rope.original_max_pos,
+                                     rope.alpha, rope.beta, seq_len=Lk)
+    bb, hh, ii = (x.ravel() for x in np.meshgrid(np.arange(B), np.arange(Hq), np.arange(L),
+                                                 indexing="ij"))
+    qr, kk, vv = (t.float().numpy() for t in (q, k, v))
+    n_tiles = -(-Lk // 128)
+    c = -(-n_tiles // splits) * 128          # keys per split
+    parts = [rows_lib.attn_rows(qr.reshape(-1, D), bb, hh, ii + Lk - L, kk, vv, Hq, table, ms,
+                                rope.pairing, 0, True, w.window, w.sinks,
+                                k_begin=min(Lk, s * c), k_end=min(Lk, (s + 1) * c))
+             for s in range(splits)]
+    o, lse = merge_lib.merge(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+    ref = oracle_rows(q, k, v, rope, Lk - L, True, w.window, w.sinks)
+    return (o.reshape(B, Hq, L, D), lse.reshape(B, Hq, L)), ref
+
+
+def test_unchanged_split_passes_the_comparison(copies):
+    for case in SPLIT_CASES[:2]:
+        got, ref = _split(copies["unchanged"], copies["unchanged"], case)
+        assert not _caught(got, ref, 8)
+
+
+@pytest.mark.parametrize("name", SPLIT_MUTANTS)
+def test_splitkv_comparison_sees_kernel_mistake(copies, name):
+    mod = copies[name]
+    for case in SPLIT_CASES:
+        rows_lib, merge_lib = (oracle, mod) if name.startswith("merge") else (mod, oracle)
+        got, ref = _split(rows_lib, merge_lib, case)
+        if _caught(got, ref, 8):
+            return
+    pytest.fail("no split-KV case's comparison sees %r (%s)" % (name, MUTANTS[name][0]))
