@@ -24,6 +24,7 @@ import torch
 import oracle
 from test_gpu_attn import BASE, SMALL, compare, table_of
 from test_gpu_decode import W0, oracle_rows, rope_of
+from test_gpu_rope import CASES as ROPE_CASES, check_rotation
 from test_oracle_mutants import MUTANTS, _copy_oracle
 from workloads import make_inputs
 
@@ -34,6 +35,12 @@ PREFILL_MUTANTS = [
     "rotation_first_sign", "rotation_second_sign", "rotation_mscale_one_component",
     "half_pairing_mirrored", "interleaved_pair_reversed", "gqa_heads_interleaved",
     "lse_without_max", "output_not_normalised", "default_scale_one_over_d",
+]
+# mistakes of the rotate pass (lcx_apply_rope): rotation signs, mscale on one
+# component, pairings, and the angle of position m + 1
+ROPE_MUTANTS = [
+    "rotation_first_sign", "rotation_second_sign", "rotation_mscale_one_component",
+    "half_pairing_mirrored", "interleaved_pair_reversed", "position_plus_one",
 ]
 # mistakes of a split-KV launch: a split that reads outside its stretch of keys,
 # or a merge that combines the partial results wrongly
@@ -62,7 +69,8 @@ def copies(tmp_path_factory):
     under its own module name (its library built in its own folder); the
     "unchanged" copy has none."""
     mods = {}
-    for name in ["unchanged"] + PREFILL_MUTANTS + SPLIT_MUTANTS + MLA_MUTANTS:
+    names = PREFILL_MUTANTS + SPLIT_MUTANTS + MLA_MUTANTS
+    for name in ["unchanged"] + names + [m for m in ROPE_MUTANTS if m not in names]:
         _, file, edits = MUTANTS[name] if name in MUTANTS else ("", "lcx_oracle.c", [])
         dst = str(tmp_path_factory.mktemp("sens_" + name))
         err = _copy_oracle(dst, edits, file)
@@ -203,3 +211,31 @@ def test_splitkv_comparison_sees_kernel_mistake(copies, name):
         if _caught(got, ref, 8):
             return
     pytest.fail("no split-KV case's comparison sees %r (%s)" % (name, MUTANTS[name][0]))
+
+
+def _rotate(lib, case):
+    """The rotate pass's output as a kernel would store it (the copy's fp64
+    rotation rounded once to the tensor's type), with the unchanged table."""
+    B, H, L, D, dt, mode, s, pairing, off = case
+    g = torch.Generator().manual_seed(0)
+    x = torch.randn((B, H, L, D), generator=g).to(dt)
+    rope = rope_of(W0.with_(D=D, mode=mode, scale=s, original_max_pos=2048, pairing=pairing))
+    table, ms, _ = oracle.rope_table(mode, D, rope.base, s, 2048, rope.alpha, rope.beta)
+    pos = np.tile(np.arange(L) + off, B * H)
+    y = lib.rotate_rows(x.float().numpy().reshape(-1, D), pos, table, ms, pairing)
+    return x, torch.from_numpy(y.reshape(B, H, L, D)).to(dt), rope, off
+
+
+def test_unchanged_rotation_passes_the_check(copies):
+    for case in ROPE_CASES:
+        check_rotation(*_rotate(copies["unchanged"], case))
+
+
+@pytest.mark.parametrize("name", ROPE_MUTANTS)
+def test_rotation_check_sees_kernel_mistake(copies, name):
+    for case in ROPE_CASES:
+        try:
+            check_rotation(*_rotate(copies[name], case))
+        except AssertionError:
+            return
+    pytest.fail("no apply_rope case's check sees %r (%s)" % (name, MUTANTS[name][0]))
