@@ -197,11 +197,22 @@ def _stream(t):
     return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
 
 
+def _same_device(ref, **tensors):
+    """Every tensor given (None skipped) must be a CUDA tensor on ref's device:
+    the library takes device pointers only, so a host buffer is refused here
+    rather than handed to a kernel."""
+    for name, t in tensors.items():
+        if t is not None and (not t.is_cuda or t.device != ref.device):
+            raise ValueError("%s must be a CUDA tensor on %s (got %s)" % (name, ref.device,
+                                                                         t.device))
+
+
 def apply_rope(x, rope: RopeParams, out=None, pos_offset: int = 0, inplace: bool = False):
     """Rotate x [B, H, L, D] (bf16/fp32, CUDA) by positions pos_offset + l."""
     import torch
     if x.dim() != 4 or not x.is_cuda:
         raise ValueError("x must be a 4-D CUDA tensor [B, H, L, D]")
+    _same_device(x, out=out)
     y = x if inplace else (out if out is not None else torch.empty_like(x))
     B, H, L, D = x.shape
     if D != rope.head_dim:
@@ -260,6 +271,8 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
         raise ValueError("k_rope must be [B, 1, Lk, rope.head_dim], got %s" % (k_rope.shape,))
     if not (q.dtype == k.dtype == v.dtype) or (k_rope is not None and k_rope.dtype != q.dtype):
         raise ValueError("q, k, v (and k_rope) must share a dtype")
+    _same_device(q, k=k, v=v, out=out, lse=lse, status=status, workspace=workspace,
+                 k_rope=k_rope, k_rot=k_rot)
     o = out if out is not None else torch.empty((B, Hq, L, Dv), dtype=q.dtype, device=q.device)
     if return_lse and lse is None:
         lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
@@ -325,6 +338,9 @@ def attn_fwd_split_static(q, k, v, rope: RopeParams, num_splits: int, causal: bo
     Hkv, Lk = k.shape[1], k.shape[2]
     if k.shape != (B, Hkv, Lk, D) or v.shape != k.shape or not (q.dtype == k.dtype == v.dtype):
         raise ValueError("shape / dtype mismatch: q %s k %s v %s" % (q.shape, k.shape, v.shape))
+    if not q.is_cuda:
+        raise ValueError("q, k, v must be CUDA tensors")
+    _same_device(q, k=k, v=v, out=out, lse=lse, status=status)
     o = out if out is not None else torch.empty_like(q)
     a = _AttnArgs()
     a.q, a.k, a.v, a.o = q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr()
@@ -367,6 +383,9 @@ def attn_merge(o_parts, lse_parts, out=None, lse=None, dtype=None):
     otherwise) and lse [B, Hq, L] fp32.
     """
     import torch
+    if not o_parts.is_cuda:
+        raise ValueError("o_parts must be a CUDA tensor")
+    _same_device(o_parts, lse_parts=lse_parts, out=out, lse=lse)
     if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32:
         raise ValueError("partial results must be fp32")
     if not (o_parts.is_contiguous() and lse_parts.is_contiguous()):
