@@ -28,6 +28,11 @@
  *   - Tensors are [B, H, L, D] with element strides given per dimension; the
  *     last dimension must be contiguous (stride 1).  Pointers and strides must
  *     keep every row 16-byte aligned.
+ *   - Every tensor, workspace and status pointer is device memory of the
+ *     current device, unless a call says otherwise (lcx_rope_table works on
+ *     host arrays).  The library does not query a pointer's kind, so a host
+ *     pointer reaches the kernel that reads it; the Python binding refuses
+ *     host tensors before the call.
  *   - Errors: argument problems are detected on the host before any device
  *     work and return LCX_ERR_INVALID_ARG (malformed) or LCX_ERR_UNSUPPORTED
  *     (well-formed but outside what the kernels implement).  A failed launch
