@@ -8,7 +8,6 @@ Thin ctypes wrappers around ``liblcx_oracle.so`` (plain C, fp64); see
 ``lcx_oracle.c`` for the definitions and their sources.
 """
 import ctypes
-import os
 
 import numpy as np
 

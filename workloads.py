@@ -11,8 +11,7 @@ Input recipe (one fresh generator per workload, seed 0):
   same generator multiply the selected entries by 8; then the tensors are cast
   (round-to-nearest-even) to the workload's dtype.
 """
-from dataclasses import dataclass, field, asdict
-import math
+from dataclasses import dataclass, asdict
 
 import torch
 
