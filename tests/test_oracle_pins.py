@@ -195,6 +195,40 @@ def test_table_is_rounded_fp64():
 # rotation
 # --------------------------------------------------------------------------
 
+def test_window_angle_table_d64():
+    """"长上下文外推", sections 5.2, 6.1 and 6.2 (d=64, a 4096-position training
+    window): each pair's frequency, the angle it covers over the window and the
+    turns that makes; the slowest pair's cos / sin at the window's end (taken
+    from the oracle's rotation of a unit pair at position 4095); and its angle
+    at position 8191, whose sin / cos the page takes at the angle rounded to
+    the printed 63 degrees."""
+    pins = load_pins()
+
+    def near(name, got):
+        val, tol, src = pins[name]
+        assert abs(got - val) <= tol, (name, got, val, src)
+
+    table, ms, _ = oracle.rope_table("plain", 64)
+    near("d64_i8_freq", float(table[8]))
+    near("d64_i24_freq", float(table[24]))
+    for i in (0, 8, 16, 24, 31):
+        rad = 4096 * float(table[i])
+        if "d64_i%d_window_rad" % i in pins:
+            near("d64_i%d_window_rad" % i, rad)
+        near("d64_i%d_window_turns" % i, rad / (2 * math.pi))
+    x = np.zeros((1, 64), dtype=np.float32)
+    x[0, 31] = 1.0                                  # unit vector on pair 31's first component
+    y = oracle.rotate_rows(x, np.array([4095]), table, ms, "half")
+    near("d64_i31_window_cos", y[0, 31])
+    near("d64_i31_window_sin", y[0, 63])
+    rad = 8191 * float(table[31])
+    near("d64_i31_pos8191_rad", rad)
+    near("d64_i31_pos8191_deg", math.degrees(rad))
+    deg = round(math.degrees(rad))
+    near("d64_i31_pos8191_sin", math.sin(math.radians(deg)))
+    near("d64_i31_pos8191_cos", math.cos(math.radians(deg)))
+
+
 @pytest.mark.parametrize("pairing", ["half", "interleaved"])
 def test_homework_angles(pairing):
     """"长上下文外推", homework 2: base 1e4, d=4, m=100: pair 0 turns by 100 rad,
