@@ -18,9 +18,23 @@ JSON line (rank 0).
 * cpu_baseline: the fp64 CPU oracle on a bounded sample of the same workload.
 * --impl reference: the oracle alone, as the reference arm (rank 0 only).
 
-Multi-GPU (torchrun): every rank runs an independent replica (its own seeded
-batch) -- the path has no exchange step, so there is no data-path collective and
-scaling is weak.  Inputs are larger than L2 (126 MB), so no flush is needed.
+* configs    : every workload of workloads.WORKLOADS measured the same way (one
+               lcx_attn_fwd call per step, inputs resident in HBM, L2 flushed
+               between calls whose inputs fit in L2): attention TFLOP/s and its
+               fraction of the sustained and burst bf16 peaks, the mean call
+               time, apply_rope GB/s against HBM, the tiny workload's latency,
+               and the oracle's extrapolated full-size CPU time (an estimate).
+
+Multi-GPU: `--gpus N` with N > 1 runs N ranks, one per GPU (started with
+torchrun by this script when it was not launched under torchrun itself; under
+torchrun WORLD_SIZE must equal N).  `--shard replicas` (default): every rank
+runs an independent replica (its own seeded batch) -- the path has no exchange
+step, so there is no data-path collective and scaling is weak.  `--shard heads`:
+the ranks split one batch's kv heads (rank r takes kv heads
+[r Hkv / N, (r + 1) Hkv / N) and their query heads, and writes that slice of
+O), again with no data-path collective; the total work is fixed, so scaling is
+strong.  The NCCL process group carries only the barriers and the max-over-ranks
+timing.  The headline inputs are larger than L2 (126 MB), so no flush is needed.
 """
 import argparse
 import json
@@ -151,9 +165,20 @@ def max_over_ranks(x, world):
     return float(t.item())
 
 
-def rank_seed(w, rank):
-    """Each rank runs an independent replica of the workload with its own seed."""
-    return w.seed + rank
+def rank_seed(w, rank, shard="replicas"):
+    """Replicas: each rank runs an independent replica of the workload with its
+    own seed.  Head shards: every rank draws the same batch (the workload's seed)
+    and keeps its slice of the heads."""
+    return w.seed if shard == "heads" else w.seed + rank
+
+
+def shard_heads(Hkv, world, rank):
+    """The kv heads [g0, g1) rank `rank` of `world` takes when the ranks split
+    one batch by heads (its query heads are [g0 G, g1 G)).  Contiguous, disjoint,
+    covering every kv head; sizes differ by at most one."""
+    if not 1 <= world <= Hkv:
+        raise ValueError("cannot split %d kv heads over %d ranks" % (Hkv, world))
+    return rank * Hkv // world, (rank + 1) * Hkv // world
 
 
 def job_tflops(flops_per_rank, world, steps, max_ms):
@@ -210,7 +235,14 @@ def bench_gpu(args, world, rank, local):
     import ntk_rope_flashattn_b200 as lcx
     w = WORKLOADS[args.workload]
     dev = torch.device("cuda", local)
-    q, k, v = make_inputs(w, device=dev, seed=rank_seed(w, rank))
+    q, k, v = make_inputs(w, device=dev, seed=rank_seed(w, rank, args.shard))
+    g0, g1 = 0, w.Hkv
+    if args.shard == "heads":
+        G = w.Hq // w.Hkv
+        g0, g1 = shard_heads(w.Hkv, world, rank)
+        q, k, v = (q[:, g0 * G:g1 * G].contiguous(), k[:, g0:g1].contiguous(),
+                   v[:, g0:g1].contiguous())
+        torch.cuda.empty_cache()
     rope = lcx.RopeParams(w.mode, w.D, w.base, w.scale, w.original_max_pos, w.alpha, w.beta,
                           w.pairing)
     o = torch.empty_like(q)
@@ -250,8 +282,10 @@ def bench_gpu(args, world, rank, local):
     launch_ms = [a.elapsed_time(b) for a, b in evs]
     assert int(status.item()) == 0, "device watchdog fired"
     total_ms = max_over_ranks(total_ms, world)
-    flops_rank = attn_flops(w)
-    tflops = job_tflops(flops_rank, world, args.steps, total_ms)
+    flops_rank = attn_flops(w) * (g1 - g0) // w.Hkv
+    # whole-job work: all replicas, or the one batch the head shards split
+    flops_job = attn_flops(w) if args.shard == "heads" else flops_rank * world
+    tflops = flops_job * args.steps / (total_ms * 1e-3) / 1e12
 
     # --- the same step with every K tile rotated on chip by each CTA that reads
     # it (no key buffer): the kernel-only variant of the path, for comparison
@@ -299,8 +333,9 @@ def bench_gpu(args, world, rank, local):
     del qr, kr
 
     # --- split-KV decode: one new token per query head against the whole cache
-    decode = bench_decode(lcx, w, q, k, v, rope, stream, status)
-    mla = bench_mla(lcx, dev, stream, status) if rank == 0 else None
+    extras = world == 1 and not args.no_extras
+    decode = bench_decode(lcx, w, q, k, v, rope, stream, status) if extras else None
+    mla = bench_mla(lcx, dev, stream, status) if extras else None
 
     # --- end to end through host buffers
     qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
@@ -320,7 +355,7 @@ def bench_gpu(args, world, rank, local):
     e_end.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), world)
-    e2e_tflops = job_tflops(flops_rank, world, args.steps, e2e_ms)
+    e2e_tflops = flops_job * args.steps / (e2e_ms * 1e-3) / 1e12
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
     d2h = oh.numel() * oh.element_size()
     del qh, kh, vh, ws
@@ -340,10 +375,11 @@ def bench_gpu(args, world, rank, local):
         "warmup": args.warmup,
         "ms_per_step": round(total_ms / args.steps, 3),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if args.shard == "heads" else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) q/k/v, seed 0 + rank)",
+        "data": ("synthetic (seeded N(0,1) q/k/v, seed 0, kv heads split over the ranks)"
+                 if args.shard == "heads" else "synthetic (seeded N(0,1) q/k/v, seed 0 + rank)"),
         "impl": "lcx",
         "config": {
             "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "D": w.D,
@@ -354,7 +390,11 @@ def bench_gpu(args, world, rank, local):
             "flops_per_step_per_gpu": flops_rank,
             "l2": "inputs larger than L2 (q+k+v = %.2f GB), no flush" % (
                 sum(t.numel() * t.element_size() for t in (q, k, v)) / 1e9),
-            "parallelism": "replicas x%d (independent batches, no collective)" % world,
+            "parallelism": ("heads sharded over %d ranks (rank r: kv heads [r Hkv/N, (r+1) "
+                            "Hkv/N) and their query heads), no data-path collective" % world
+                            if args.shard == "heads" else
+                            "replicas x%d (independent batches, no collective)" % world),
+            "flops_per_step_job": flops_job,
         },
         "gpu_launches": args.steps * (2 if rotate_once else 1),
         "roofline": {
@@ -394,11 +434,144 @@ def bench_gpu(args, world, rank, local):
         res["gpu_launches_decode"] = decode["launches"]
     del q, k, v, o
     torch.cuda.empty_cache()
+    if extras and not args.no_configs:
+        res["configs"] = bench_configs(lcx, dev, stream, status, peaks, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         val, secs, cores, desc = oracle_sample(w, budget_s=args.cpu_budget)
         res["cpu_baseline"] = {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                                "sample": desc, "seconds": round(secs, 2)}
+        if "configs" in res:
+            oracle_estimates(res["configs"], budget_s=args.cpu_budget_per_config)
     return res
+
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _call_ms(fn, stream, reps, flush=None, warm=2):
+    """Mean device time of one fn() over reps calls (CUDA events on the launching
+    stream).  With `flush` (a buffer larger than L2) every call is timed alone
+    after the buffer was rewritten, so no call finds the previous one's data in
+    L2."""
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    if flush is None:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+    evs = []
+    for _ in range(reps):
+        flush.add_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+
+def bench_configs(lcx, dev, stream, status, peaks, local, reps=5):
+    """Every workload measured like the headline: one lcx_attn_fwd call per
+    step (host table, the keys' rotate pass into a buffer, the attention kernel),
+    inputs resident in HBM.  Workloads whose inputs fit in L2 are timed call by
+    call with L2 flushed in between.  The tiny workload is launch-bound: its
+    number is the latency of one call."""
+    out = {}
+    burst, sust, hbm = (float(peaks["bf16_tflops"]), float(peaks["bf16_tflops_sustained"]),
+                        float(peaks["hbm_gbs"]))
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    with ClockSampler(local) as clk:
+        for name, w in WORKLOADS.items():
+            q, k, v = make_inputs(w, device=dev, seed=w.seed)
+            rope = lcx.RopeParams(w.mode, w.D, w.base, w.scale, w.original_max_pos, w.alpha,
+                                  w.beta, w.pairing)
+            o = torch.empty_like(q)
+            parts = 2 if (w.split_qk and k.dtype == torch.bfloat16) else 1
+            k_rot = torch.empty((parts,) + tuple(k.shape), dtype=k.dtype, device=dev)
+            kw = dict(causal=w.causal, window=w.window, sinks=w.sinks,
+                      softmax_scale=w.softmax_scale, split_qk=w.split_qk, out=o,
+                      status=status, k_rot=k_rot)
+            in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+            fl = flush if in_bytes < L2_BYTES else None
+            tiny = w.L * w.B * w.Hq <= 4096
+            n = 200 if tiny else reps
+            ms = _call_ms(lambda: lcx.attn_fwd(q, k, v, rope, **kw), stream, n,
+                          flush=None if tiny else fl)
+            flops = attn_flops(w)
+            tf = flops / (ms * 1e-3) / 1e12
+            qr, kr = torch.empty_like(q), torch.empty_like(k)
+
+            def rope_qk():
+                lcx.apply_rope(q, rope, out=qr)
+                lcx.apply_rope(k, rope, out=kr)
+            rope_ms = _call_ms(rope_qk, stream, max(reps, 5), flush=fl)
+            k_pass_ms = _call_ms(lambda: lcx.apply_rope(k, rope, out=kr), stream,
+                                 max(reps, 5), flush=fl)
+            rb = rope_bytes(w)
+            e = {
+                "what": w.description, "ms_per_call": round(ms, 4), "calls": n,
+                "attn_tflops": round(tf, 2), "frac_sustained": round(tf / sust, 4),
+                "frac_burst": round(tf / burst, 4),
+                "apply_rope_gbs": round(rb / (rope_ms * 1e-3) / 1e9, 1),
+                "apply_rope_frac_hbm": round(rb / (rope_ms * 1e-3) / 1e9 / hbm, 4),
+                "apply_rope_ms": round(rope_ms, 4),
+                "l2": "flushed between calls" if fl is not None else (
+                    "inputs larger than L2" if not tiny else "launch-bound latency, L2 warm"),
+                "qk_mode": "split" if w.split_qk else "bf16",
+                "dtype": w.dtype, "flops_per_call": flops,
+            }
+            if not w.split_qk:
+                # the attention kernel alone: the call minus the keys' rotate pass
+                kern = ms - k_pass_ms
+                e["kernel_ms"] = round(kern, 4)
+                e["kernel_tflops"] = round(flops / (kern * 1e-3) / 1e12, 2)
+            if tiny:
+                e["latency_us"] = round(ms * 1e3, 2)
+            assert int(status.item()) == 0, "device watchdog fired in %s" % name
+            out[name] = e
+            del q, k, v, o, k_rot, qr, kr
+            torch.cuda.empty_cache()
+    del flush
+    torch.cuda.empty_cache()
+    out["clocks"] = clk.summary()
+    out["peaks"] = {"bf16_tflops": burst, "bf16_tflops_sustained": sust, "hbm_gbs": hbm}
+    return out
+
+
+def oracle_estimates(configs, budget_s=1.5):
+    """The oracle beside each workload: the tiny workload timed over its whole
+    tensor; for the others a short sample (the heaviest rows of one kv head)
+    gives the oracle's FLOP rate, and the full-size CPU time is extrapolated
+    from it (labelled an estimate)."""
+    import oracle
+    for name, e in configs.items():
+        w = WORKLOADS.get(name)
+        if w is None:
+            continue
+        if w.L * w.B * w.Hq <= 4096:
+            q, k, v = make_inputs(w, device="cpu", seed=w.seed)
+            table, ms, _ = oracle.rope_table(w.mode, w.D, w.base, w.scale, w.original_max_pos,
+                                             w.alpha, w.beta)
+            scale = w.softmax_scale if w.softmax_scale > 0 else None
+            t0 = time.perf_counter()
+            oracle.attn_full(q.float().numpy(), k.float().numpy(), v.float().numpy(), table, ms,
+                             w.pairing, 0, w.causal, w.window, w.sinks, scale)
+            secs = time.perf_counter() - t0
+            e["oracle_full_s"] = round(secs, 4)
+            e["oracle_full_threads"] = oracle.num_threads(0)
+            continue
+        rate, secs, cores, desc = oracle_sample(w, budget_s=budget_s)
+        e["oracle_tflops_sample"] = rate
+        e["oracle_full_s_estimate"] = round(attn_flops(w) / (rate * 1e12), 1)
+        e["oracle_estimate_from"] = "%s (%.1f s, %d threads); extrapolated, not run" % (
+            desc, secs, cores)
 
 
 def bench_decode(lcx, w, q, k, v, rope, stream, status, reps=20):
@@ -531,6 +704,20 @@ def bench_reference(args, world, rank):
     }
 
 
+def relaunch(n):
+    """Run this script as n ranks under torchrun (one per GPU, rendezvous on
+    127.0.0.1) with the same arguments; returns torchrun's exit status.  Rank 0
+    prints the JSON line."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           "--nproc-per-node", str(n), "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -539,11 +726,27 @@ def main():
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="lcx", choices=["lcx", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--cpu-budget-per-config", type=float, default=1.5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload measurements (the configs object)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip decode, decoupled-RoPE and per-workload measurements")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="N > 1: independent replicas (weak scaling) or one batch split by "
+                         "kv heads (strong scaling)")
     ap.add_argument("--decode-only", action="store_true",
                     help="only the split-KV decode measurement on the workload's cache "
                          "(prints its object; for profiling, not a bench line)")
     args = ap.parse_args()
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is None and args.gpus > 1:
+        # not launched under torchrun: start the N ranks here
+        sys.exit(relaunch(args.gpus))
+    if env_world is not None and int(env_world) != args.gpus:
+        print("bench.py: --gpus %d but WORLD_SIZE=%s; launch one rank per GPU with "
+              "--gpus equal to the number of ranks" % (args.gpus, env_world), file=sys.stderr)
+        sys.exit(2)
     if args.decode_only:
         import ntk_rope_flashattn_b200 as lcx
         w = WORKLOADS[args.workload]

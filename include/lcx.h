@@ -169,7 +169,11 @@ typedef struct {
     float *lse;                /* DEVICE [B, Hq, L] fp32 natural-log sum-exp of the
                                   scaled logits, or NULL                          */
     int32_t *dev_status;       /* DEVICE int32 or NULL: set to LCX_ERR_TIMEOUT by a
-                                  kernel whose bounded wait expired; never cleared */
+                                  kernel whose bounded wait expired; never cleared.
+                                  After an expiry o and lse are undefined (the call
+                                  still returns LCX_OK: the expiry happens on the
+                                  device after the call returned), so callers that
+                                  must detect it pass this word and read it      */
     int32_t dtype;             /* lcx_dtype of q, k, v, o                         */
     int32_t causal;            /* 1 = key j visible to query i only if j <= i    */
     int64_t B, Hq, Hkv, L, D;  /* Hq % Hkv == 0; D = query/key head dim           */
@@ -314,20 +318,27 @@ LCX_API lcx_status lcx_attn_merge(const float *o_parts, const float *lse_parts, 
  * The pages describe no counterpart of this call; it exists for callers that
  * have no device allocator at hand.
  *   Scratch : one static __device__ array of LCX_STATIC_SCRATCH_BYTES per
- *             device (256-byte aligned), resolved with cudaGetSymbolAddress
- *             on the first call on each device (a checked call; failure is
- *             LCX_ERR_CUDA; under lazy module loading the CUDA runtime also
- *             materialises the array at that point).  Make that first call
- *             before capturing the stream into a graph; later calls allocate
- *             nothing.  Nothing in it must start at zero (every partial
- *             row the merge reads is written earlier in the same call), so it
- *             is never cleared.
+ *             CUDA context (256-byte aligned).  Every call looks up the
+ *             current context's copy with cudaGetSymbolAddress (a checked
+ *             call; failure is LCX_ERR_CUDA), so a context that was destroyed
+ *             and created again (cudaDeviceReset) is never handed a stale
+ *             address.  The first call in a context is the set-up: under lazy
+ *             module loading the CUDA runtime loads the library's module, and
+ *             with it the array, at that lookup; make that first call before
+ *             capturing the stream into a graph.  Later calls allocate
+ *             nothing.  Nothing in the array must start at zero (every
+ *             partial row the merge reads is written earlier in the same
+ *             call), so it is never cleared.
  *   Limit   : requests whose lcx_attn_split_workspace_bytes exceeds
  *             LCX_STATIC_SCRATCH_BYTES return LCX_ERR_UNSUPPORTED before any
  *             device work.
  *   Races   : every call on a device shares the one array, so two calls whose
  *             executions overlap (different streams, or threads without
  *             ordering) corrupt each other's partial results; order them.
+ *   Watchdog: if a bounded device wait expires (args.watchdog_ms), o and lse
+ *             are undefined -- the merge may read partial rows that an
+ *             earlier call left in the array.  Pass args.dev_status to learn
+ *             of it.
  *   Otherwise as lcx_attn_fwd_split (num_splits 1..256; 1 uses no scratch).
  */
 LCX_API lcx_status lcx_attn_fwd_split_static(const lcx_attn_args *args, int32_t num_splits,

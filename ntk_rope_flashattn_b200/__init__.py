@@ -89,14 +89,20 @@ class RopeParams:
     @classmethod
     def from_hf(cls, cfg: dict, head_dim: int):
         """From a HuggingFace-style ``rope_scaling`` dict plus ``rope_theta``
-        (keys: type/rope_type, factor, original_max_position_embeddings,
-        beta_slow -> alpha, beta_fast -> beta, rope_theta)."""
+        (keys: type/rope_type, factor, original_max_position_embeddings or
+        max_position_embeddings, beta_slow -> alpha, beta_fast -> beta,
+        rope_theta).  Rope types: default -> plain, linear -> pi, ntk -> ntk,
+        yarn -> yarn, dynamic -> dynamic_ntk.  Dynamic NTK here takes its scale
+        from the call's context length (s = seq_len / original_max_pos, plain
+        RoPE up to the training length), so ``factor`` does not enter it."""
         kind = cfg.get("rope_type", cfg.get("type", "default"))
-        mode = {"default": "plain", "linear": "pi", "dynamic": "ntk", "ntk": "ntk",
+        mode = {"default": "plain", "linear": "pi", "dynamic": "dynamic_ntk", "ntk": "ntk",
                 "yarn": "yarn"}.get(kind, kind)
+        if mode not in MODES or mode in ("none", "factors"):
+            raise ValueError("rope type %r has no equivalent here" % (kind,))
+        lmax = cfg.get("original_max_position_embeddings", cfg.get("max_position_embeddings", 4096))
         return cls(mode=mode, head_dim=head_dim, base=float(cfg.get("rope_theta", 10000.0)),
-                   scale=float(cfg.get("factor", 1.0)),
-                   original_max_pos=int(cfg.get("original_max_position_embeddings", 4096)),
+                   scale=float(cfg.get("factor", 1.0)), original_max_pos=int(lmax),
                    alpha=float(cfg.get("beta_slow", 1.0)), beta=float(cfg.get("beta_fast", 32.0)))
 
     def _c(self):
@@ -255,7 +261,9 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
     ``split_qk`` forms QK^T from hi/lo bf16 parts of the rotated operands
     (LCX_ATTN_SPLIT_QK) for inputs whose large logits bf16 rounding would spoil.
     ``status`` (optional int32 CUDA tensor of one element) receives
-    LCX_ERR_TIMEOUT if a kernel's bounded wait expired.
+    LCX_ERR_TIMEOUT if a kernel's bounded wait expired (``watchdog_ms``, 0 =
+    2000); o and lse are then undefined, and without ``status`` nothing
+    reports it.
     """
     import torch
     for t in (q, k, v):
@@ -327,12 +335,15 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
 
 def attn_fwd_split_static(q, k, v, rope: RopeParams, num_splits: int, causal: bool = True,
                           window: int = 0, sinks: int = 0, softmax_scale: float = 0.0,
-                          q_offset: int = 0, out=None, lse=None, status=None):
+                          q_offset: int = 0, out=None, lse=None, status=None,
+                          watchdog_ms: int = 0):
     """Split-KV attention through lcx_attn_fwd_split_static: the partial results
     live in the library's static device scratch (LCX_STATIC_SCRATCH_BYTES per
-    device), so nothing is allocated for them.  Calls on one device must not
-    overlap in time (they share the scratch).  q [B, Hq, L, D], k/v
-    [B, Hkv, Lk, D]; returns o (and fills ``lse`` when given)."""
+    CUDA context), so nothing is allocated for them.  Calls on one device must
+    not overlap in time (they share the scratch).  q [B, Hq, L, D], k/v
+    [B, Hkv, Lk, D]; returns o (and fills ``lse`` when given).  If a bounded
+    device wait expires (``watchdog_ms``, 0 = 2000) o and lse are undefined;
+    pass ``status`` to learn of it (it receives LCX_ERR_TIMEOUT)."""
     import torch
     B, Hq, L, D = q.shape
     Hkv, Lk = k.shape[1], k.shape[2]
@@ -356,7 +367,7 @@ def attn_fwd_split_static(q, k, v, rope: RopeParams, num_splits: int, causal: bo
     a.window, a.sinks = int(window), int(sinks)
     a.softmax_scale = float(softmax_scale)
     a.flags = 0
-    a.watchdog_ms = 0
+    a.watchdog_ms = int(watchdog_ms)
     a.reserved0 = 0
     a.Lk = Lk
     a.q_offset = int(q_offset)

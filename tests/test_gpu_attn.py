@@ -2,12 +2,17 @@
 fp64 oracle.
 
 Tolerance (from the target): output max-abs <= 2e-2 and mean-abs <= 2e-3 against
-the fp64 result; LSE max-abs <= 2e-2.  The max-abs bound is applied beyond the
-output's own rounding: a bf16 output cannot hold |o| in [2^e, 2^(e+1)) closer than
-half an ulp (2^(e-8)), which is 0.031-0.063 for the |o| of 8-32 that outlier-heavy
-inputs produce, so the check is |o - o_ref| - ulp(o_ref)/2 <= 2e-2.  Small cases compare every element and span
-several 128-row tiles with ragged tails; the full-size workloads compare sampled
-query rows (boundary rows plus seeded random rows, all heads).
+the fp64 result; LSE max-abs <= 2e-2.  The max-abs bound is literal (raw
+|o - o_ref| <= 2e-2) wherever |o_ref| < 4.  From |o_ref| = 4 up it is applied
+beyond the output's own rounding: a bf16 output cannot hold |o| in
+[2^e, 2^(e+1)) closer than half an ulp (2^(e-8)), which is 0.016 at 4 and
+0.031-0.063 for the |o| of 8-32 that outlier-heavy inputs produce, so there the
+check is |o - o_ref| - ulp(o_ref)/2 <= 2e-2.  N(0,1) inputs (all workloads but
+the outlier one) practically never reach |o| >= 4, so for them the bound is the
+literal one.  Small cases compare every element and span several 128-row tiles
+with ragged tails; the full-size workloads compare sampled query rows (boundary
+rows plus seeded random rows, all heads).  Each comparison prints its raw max and
+mean error (pytest -s shows them).
 """
 import numpy as np
 import pytest
@@ -20,6 +25,7 @@ from workloads import WORKLOADS, Workload, make_inputs, sample_rows
 pytestmark = pytest.mark.gpu
 
 MAX_ABS, MEAN_ABS, LSE_ABS = 2e-2, 2e-3, 2e-2
+ROUNDING_ALLOWANCE_FROM = 4.0   # |o_ref| from which the output's half-ulp is allowed
 
 
 def rope_of(w):
@@ -49,14 +55,19 @@ def half_ulp(ref, out_bits):
     return np.exp2(np.floor(np.log2(a)) - out_bits)
 
 
-def compare(got_o, got_lse, ref_o, ref_lse, out_bits=8):
+def compare(got_o, got_lse, ref_o, ref_lse, out_bits=8, label=""):
     err = np.abs(got_o.astype(np.float64) - ref_o)
     assert np.isfinite(got_o).all()
-    excess = err - half_ulp(ref_o, out_bits)
-    assert excess.max() <= MAX_ABS, "max-abs beyond output rounding %.4g (raw %.4g)" % (
-        excess.max(), err.max())
-    assert err.mean() <= MEAN_ABS, "mean-abs %.4g" % err.mean()
+    big = np.abs(ref_o) >= ROUNDING_ALLOWANCE_FROM
+    excess = np.where(big, err - half_ulp(ref_o, out_bits), err)
     lerr = np.abs(got_lse.astype(np.float64) - ref_lse)
+    raw_small = err[~big].max() if (~big).any() else 0.0
+    print("[parity] %s raw max %.4g (|o_ref| < 4: %.4g), mean %.3g, checked max %.4g, "
+          "%d of %d elements with |o_ref| >= 4, lse max %.3g" % (
+              label, err.max(), raw_small, err.mean(), excess.max(), int(big.sum()), err.size,
+              lerr.max()))
+    assert excess.max() <= MAX_ABS, "max-abs %.4g (raw %.4g)" % (excess.max(), err.max())
+    assert err.mean() <= MEAN_ABS, "mean-abs %.4g" % err.mean()
     assert lerr.max() <= LSE_ABS, "lse max-abs %.4g" % lerr.max()
     return err.max(), err.mean()
 
@@ -70,7 +81,7 @@ def full_check(w, **kw):
                                       v.float().cpu().numpy(), table, ms, w.pairing, 0,
                                       w.causal, w.window, w.sinks, scale)
     return compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o, ref_lse,
-                   24 if w.dtype == "f32" else 8)
+                   24 if w.dtype == "f32" else 8, label=w.name)
 
 
 BASE = Workload("case", B=1, Hq=4, Hkv=2, L=256, D=128, dtype="bf16", mode="plain")
@@ -206,7 +217,9 @@ def sampled_check(w, n_random=16, max_heads=None):
                                         np.zeros(hh.size), hh.ravel(), rr.ravel(), kb, vb, w.Hq,
                                         table, ms, w.pairing, 0, w.causal, w.window, w.sinks,
                                         scale)
-        errs.append(compare(ob.reshape(-1, w.D), lb.ravel(), ref_o, ref_l))
+        errs.append(compare(ob.reshape(-1, w.D), lb.ravel(), ref_o, ref_l,
+                            label="%s batch %d, %d rows x %d heads" % (w.name, b, len(rows),
+                                                                      len(heads))))
     del q, k, v, o, lse
     torch.cuda.empty_cache()
     return errs
@@ -215,7 +228,13 @@ def sampled_check(w, n_random=16, max_heads=None):
 @pytest.mark.parametrize("name", ["llama3_8b_L8192", "pi_L32768_s4", "ntk_L32768_s4",
                                   "yarn_L131072_s16", "sink_window_L65536"])
 def test_attn_full_size_sampled_rows(name):
-    sampled_check(WORKLOADS[name])
+    """Sampled rows of each full-size workload.  The four N(0,1) workloads must
+    meet the literal bound with no rounding allowance at all."""
+    w = WORKLOADS[name]
+    errs = sampled_check(w)
+    if w.outlier_frac == 0:
+        assert max(e[0] for e in errs) <= MAX_ABS
+        assert max(e[1] for e in errs) <= MEAN_ABS
 
 
 @pytest.mark.parametrize("mode", ["dynamic_ntk", "factors", "factors_short"])

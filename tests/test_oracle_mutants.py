@@ -105,6 +105,14 @@ MUTANTS = {
         [("table[i] = (float)tp[i];",
           "{ float f_ = (float)tp[i]; if ((double)f_ > tp[i]) f_ = nextafterf(f_, 0.0f); "
           "table[i] = f_; }")]),
+    "midpoint_never_flags": (
+        "the midpoint flag never set, so a table entry on an fp32 rounding midpoint "
+        "would still be compared bit for bit", C_SRC,
+        [("return (fabs(v - mid_up) < tol || fabs(v - mid_dn) < tol) ? 1 : 0;",
+          "return 0 * ((fabs(v - mid_up) < tol || fabs(v - mid_dn) < tol) ? 1 : 0);")]),
+    "midpoint_flags_everything": (
+        "the midpoint tolerance far too wide (2^-20), flagging ordinary entries", C_SRC,
+        [("double tol = fabs(v) * ldexp(1.0, -40);", "double tol = fabs(v) * ldexp(1.0, -20);")]),
     "gqa_heads_interleaved": (
         "query head h reads kv head h mod Hkv instead of floor(h / G)", C_SRC,
         [("if (row_b[r] == b && row_h[r] / G == g) sel[ns++] = r;",

@@ -191,6 +191,28 @@ def test_table_is_rounded_fp64():
         assert abs(float(ms) - ms64) <= 2.0 ** -24 * ms64
 
 
+def test_midpoint_flag_marks_fp32_midpoints():
+    """The flag that exempts a table entry from the bit-exact comparison is set
+    exactly where the fp64 value sits on an fp32 rounding midpoint.  With the
+    per-pair factor mode theta'_0 = 1 / lambda_0, so lambda_0 = 1 / v puts v
+    (to within a few fp64 ulps) into entry 0: a midpoint must flag, and values
+    2^-30 (relative) to either side, or an fp32 number itself, must not."""
+    D = 64
+    for f in (np.float32(1.5), np.float32(0.01), np.float32(3.0517578125e-05)):
+        up = np.nextafter(f, np.float32(np.inf))
+        mid = 0.5 * (float(f) + float(up))
+        cases = [(mid, 1), (mid * (1 + 2.0 ** -30), 0), (mid * (1 - 2.0 ** -30), 0),
+                 (float(f), 0), (float(up), 0)]
+        for v, expect in cases:
+            lam = np.ones(D // 2)
+            lam[0] = 1.0 / v
+            th, _ = oracle.rope_theta_ext("factors", D, factors=lam)
+            assert abs(th[0] - v) <= 4 * np.spacing(v)
+            t, ms, flags = oracle.rope_table("factors", D, factors=lam)
+            assert flags[0] == expect, (float(f), v)
+            assert flags[1:].sum() == 0
+
+
 # --------------------------------------------------------------------------
 # rotation
 # --------------------------------------------------------------------------

@@ -18,6 +18,9 @@ from workloads import Workload, make_inputs
 W = Workload("static_scratch", B=2, Hq=8, Hkv=2, L=3000, D=128, dtype="bf16", mode="yarn",
              scale=8.0, original_max_pos=256, window=1200, sinks=4)
 SCRATCH = 32 * 1024 * 1024
+# the first static call: more rows and splits than any checked call, so the
+# partial results it leaves cover everything a checked call reads
+POISON_L, POISON_SPLITS = 200, 8
 
 
 def _rope(w):
@@ -57,21 +60,30 @@ def test_static_scratch_refuses_before_device_work():
 @pytest.mark.parametrize("L,splits", [(1, 8), (4, 16), (1, 1), (200, 3)])
 def test_static_scratch_equals_workspace_entry(L, splits):
     """Two calls in a row through each entry point: bit-identical o and lse, and
-    the static entry allocates no device memory."""
+    the static entry allocates no device memory, although an earlier static
+    call on other inputs left different partial results in the scratch."""
     q_all, k, v = make_inputs(W, device="cuda")
     q = q_all[:, :, W.L - L:]
     rope = _rope(W)
     kw = dict(window=W.window, sinks=W.sinks, q_offset=W.L - L)
     assert lcx.split_workspace_bytes(W.B, W.Hq, L, W.D, splits) <= SCRATCH
+    assert L <= POISON_L and lcx.split_workspace_bytes(W.B, W.Hq, POISON_L, W.D,
+                                                       POISON_SPLITS) <= SCRATCH
     ref = [lcx.attn_fwd(q, k, v, rope, num_splits=splits, return_lse=True, **kw)
            for _ in range(2)]
     outs = [(torch.empty_like(q), torch.empty((W.B, W.Hq, L), dtype=torch.float32,
                                               device="cuda")) for _ in range(2)]
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    # The first call on a device resolves the scratch array (with lazy module
+    # The first call in a context loads the scratch array (with lazy module
     # loading the CUDA runtime materialises it then); the calls after it are
-    # the ones that must allocate nothing.
-    lcx.attn_fwd_split_static(q, k, v, rope, splits, out=outs[0][0], lse=outs[0][1], **kw)
+    # the ones that must allocate nothing.  That first call runs on OTHER
+    # inputs (another seed) with more rows and splits, so every byte of the
+    # scratch the checked calls read first holds a different, stale value: a
+    # partial row the checked call failed to write would show up below.
+    q2_all, k2, v2 = make_inputs(W, device="cuda", seed=7)
+    lp = POISON_L
+    lcx.attn_fwd_split_static(q2_all[:, :, W.L - lp:], k2, v2, rope, POISON_SPLITS,
+                              window=W.window, sinks=W.sinks, q_offset=W.L - lp)
     torch.cuda.synchronize()
     allocated, free = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
     for o, lse in outs:
