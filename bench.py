@@ -6,7 +6,7 @@ One step = one pass of the hot path over one batch of the workload, one
 lcx_attn_fwd call: the RoPE table for the mode (host), the rotate pass over the
 keys into a buffer (args.k_rot: every key rotated once, mscale included), and
 the fused kernel (queries rotated on chip, QK^T, online softmax, PV).  In the
-split-QK^T mode the pass writes the keys as hi/lo bf16 parts.  Prints ONE
+split-QK^T mode the pass writes the keys' fp16 and 8-bit cross parts.  Prints ONE
 JSON line (rank 0).
 
 * value      : attention TFLOP/s, algorithmic FLOPs = 4 * D * (visible query/key
@@ -247,7 +247,8 @@ def bench_gpu(args, world, rank, local):
                           w.pairing)
     o = torch.empty_like(q)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    # keys rotated once per step into k_rot (split-QK^T with bf16 keys: hi then lo parts)
+    # keys rotated once per step into k_rot (split-QK^T with bf16 keys: fp16 parts, then
+    # 8-bit cross parts of as many bytes)
     rotate_once = True
     parts = 2 if (w.split_qk and k.dtype == torch.bfloat16) else 1
     k_rot = torch.empty((parts,) + tuple(k.shape), dtype=k.dtype, device=dev)

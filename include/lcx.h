@@ -144,13 +144,18 @@ LCX_API lcx_status lcx_apply_rope(const lcx_rope_params *params, const void *x, 
                                    lcx_apply_rope with the same params, mscale
                                    included): skip the on-chip rotation and the
                                    mscale^2 factor on the logits.             */
-#define LCX_ATTN_SPLIT_QK 2u    /* split mode: hold each rotated q' and k' as a bf16
-                                   pair hi + lo (lo = bf16(x' - hi)) and form
-                                   QK^T as hi.hi + hi.lo + lo.hi, so the logits
-                                   are no longer limited by bf16 rounding of the
-                                   rotated operands (needed when the logits are
-                                   large, e.g. outlier-heavy activations); about
-                                   twice the tensor-core work for QK^T        */
+#define LCX_ATTN_SPLIT_QK 2u    /* split mode: hold each rotated q' and k' as an
+                                   fp16 part h = f16(x') plus the residual
+                                   r = x' - h and form QK^T as
+                                   qh.kh (fp16 tensor cores) + [e5m2(qh) |
+                                   e5m2(qr)].[e5m2(kr) | e5m2(kh)] (one e5m2
+                                   product over 2 D at twice the fp16 rate),
+                                   so the logits are accurate to ~2^-15
+                                   relative instead of bf16's 2^-9 (needed when
+                                   the logits are large, e.g. outlier-heavy
+                                   activations); twice the tensor-core time
+                                   of plain QK^T.  The rotated values must lie
+                                   inside fp16's range (|x'| < 65504)        */
 #define LCX_ATTN_PREROTATED_K 4u /* k alone already holds rotated vectors (a KV
                                    cache filled by lcx_apply_rope with the same
                                    params, mscale included); q is rotated on
@@ -211,11 +216,14 @@ typedef struct {
                                   one per key tile and CTA.  Every dim rotated,
                                   no k_rope: contiguous [B, Hkv, Lk, D] of
                                   dtype; in the split-QK^T mode with bf16
-                                  operands the hi parts, then the lo parts (bf16
-                                  of the rounding residual).  With k_rope: the
-                                  shared rotary key, contiguous [B, 1, Lk,
-                                  rope.head_dim].  16-byte aligned.  Ignored
-                                  otherwise (partial rotary without k_rope)    */
+                                  operands the keys' fp16 parts ([B, Hkv, Lk,
+                                  D] fp16) followed by their 8-bit cross parts
+                                  ([B, Hkv, Lk, 2 D] bytes: e5m2 of the
+                                  residual, then of the fp16 part).  With
+                                  k_rope: the shared rotary key, contiguous
+                                  [B, 1, Lk, rope.head_dim].  16-byte aligned.
+                                  Ignored otherwise (partial rotary without
+                                  k_rope)                                        */
     int64_t k_rot_bytes;       /* bytes at k_rot: >= B*Hkv*Lk*D*element size,
                                   twice that for split-QK^T with bf16, or
                                   B*Lk*rope.head_dim*element size with k_rope */
@@ -242,9 +250,11 @@ typedef struct {
  *   the rotated parts only, as the scaled cos/sin do), the first D - d_R are
  *   used as they are, and the default scale 1/sqrt(D) is 1/sqrt(d_h + d_R).
  *   k_rope supplies the rotated key part once for all heads.
- *   Arithmetic: q', k' rounded to bf16 on chip, QK^T and PV on bf16 tensor
- *   cores with fp32 accumulation, softmax statistics in fp32, o rounded once
- *   to the output dtype.  fp32 inputs are rounded to bf16 operands.
+ *   Arithmetic: q', k' rounded to bf16 on chip (split mode: an fp16 part
+ *   and e5m2 cross parts, see LCX_ATTN_SPLIT_QK), QK^T and PV on tensor cores
+ *   with fp32 accumulation, P rounded to bf16 for PV, softmax statistics in
+ *   fp32, o rounded once to the output dtype.  fp32 inputs are rounded to
+ *   bf16 operands.
  *   Supported (D, Dv, rope.head_dim): (64, 64, 64), (128, 128, 128) with bf16
  *   or fp32 and either QK^T mode; (128, 128, 64) and (192, 128, 64) with bf16
  *   and plain QK^T.  Pointers 16-byte aligned, strides multiples of 16 bytes,

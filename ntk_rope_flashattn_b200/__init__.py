@@ -256,10 +256,12 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
     split-QK^T mode with bf16 keys, or like k_rope with decoupled RoPE): the
     keys (with k_rope: the shared rotary key) are rotated once into that buffer
     by the rotate pass before the kernel, which then reads them pre-rotated
-    (split mode: as hi/lo bf16 parts), instead of rotating each key tile on chip
-    in every CTA that reads it (ignored where the kernel does not rotate keys).
-    ``split_qk`` forms QK^T from hi/lo bf16 parts of the rotated operands
-    (LCX_ATTN_SPLIT_QK) for inputs whose large logits bf16 rounding would spoil.
+    (split mode: as fp16 parts and 8-bit cross parts), instead of rotating each
+    key tile on chip in every CTA that reads it (ignored where the kernel does
+    not rotate keys).
+    ``split_qk`` (LCX_ATTN_SPLIT_QK) forms QK^T from an fp16 part and e5m2
+    cross parts of the rotated operands, for inputs whose large logits bf16
+    rounding would spoil (rotated values must stay inside fp16's range).
     ``status`` (optional int32 CUDA tensor of one element) receives
     LCX_ERR_TIMEOUT if a kernel's bounded wait expired (``watchdog_ms``, 0 =
     2000); o and lse are then undefined, and without ``status`` nothing
@@ -310,7 +312,8 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
             # decoupled RoPE: the pass rotates only the shared rotary key
             k_rot = torch.empty((B, 1, Lk, k_rope.shape[-1]), dtype=k.dtype, device=k.device)
         else:
-            # split QK^T with bf16 keys: the pass writes hi parts, then lo parts
+            # split QK^T with bf16 keys: the pass writes the fp16 parts, then the
+            # 8-bit cross parts (2 D bytes per key: as many bytes again)
             parts = 2 if (split_qk and k.dtype == torch.bfloat16) else 1
             k_rot = torch.empty((parts, B, Hkv, Lk, Dk), dtype=k.dtype, device=k.device)
     if k_rot is not None:

@@ -24,11 +24,13 @@ constexpr int kMaxHalf = 256;  // head_dim <= 512
 struct RopeArgs {
     const char *x;
     char *y;
-    char *y_lo;                  // bf16 only, or NULL: y_lo = bf16(y' - bf16(y'))
+    char *y_x8;                  // bf16 x only, or NULL: y then receives the fp16 parts
+                                 // h = f16(y') and y_x8 the 8-bit cross parts (below)
     long long xs_b, xs_h, xs_l;  // element strides
     long long ys_b, ys_h, ys_l;
     int H, L;
     long long pos_offset;
+    int D;                // head_dim
     int jobs_per_row;     // 16-byte jobs per (position, head)
     int rows_per_cta;     // positions per CTA
     float ms;
@@ -73,32 +75,59 @@ __device__ __forceinline__ uint4 pack(const float (&y)[4]) {
                       __float_as_uint(y[3]));
 }
 
-// The residual of the bf16 rounding, y - bf16(y), rounded to bf16 again: the
-// "lo" half of a hi/lo pair (hi + lo carries y to ~16 significant bits).  Same
-// layout as y; e2 < 0 means only the vector at e1 exists.
-template <int N>
-__device__ __forceinline__ void store_lo(const RopeArgs &a, int b, int l, int h, int e1, int e2,
-                                         const float (&y1)[N], const float (&y2)[N],
-                                         const uint4 &h1, const uint4 &h2) {
-    __nv_bfloat16 *lr = reinterpret_cast<__nv_bfloat16 *>(
-        a.y_lo + 2 * (b * a.ys_b + l * a.ys_l + (long long)h * a.ys_h));
-    float r1[8], r2[8], f[8];
-    unpack(h1, f);
+__device__ __forceinline__ uint32_t pk16(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ float2 unpk16(uint32_t v) {
+    float lo, hi;
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "cvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(v));
+    return make_float2(lo, hi);
+}
+__device__ __forceinline__ uint32_t pk8x4(float x0, float x1, float x2, float x3) {
+    uint16_t lo, hi;
+    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(x1), "f"(x0));
+    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(x3), "f"(x2));
+    return uint32_t(lo) | (uint32_t(hi) << 16);
+}
+
+// Split-QK^T keys: the 8 rotated values y of the vector at element e of a row
+// are stored as fp16 parts h = f16(y) (16 bytes at y's place, which is fp16
+// here) and, in the 8-bit cross row of 2 D bytes, the e5m2 bytes of the
+// residual y - h at bytes e .. e + 7 and of h at bytes D + e .. D + e + 7 (the
+// key order [r8 | h8] the attention kernel's cross product expects).  The
+// cross row of (b, h, l) starts at twice the element offset of y's row.
+__device__ __forceinline__ void store_split(const RopeArgs &a, int b, int l, int h, int e,
+                                            const float (&y)[8]) {
+    const long long row = b * a.ys_b + l * a.ys_l + (long long)h * a.ys_h;
+    const uint4 hv = make_uint4(pk16(y[0], y[1]), pk16(y[2], y[3]), pk16(y[4], y[5]),
+                                pk16(y[6], y[7]));
+    __stcs(reinterpret_cast<uint4 *>(a.y + 2 * (row + e)), hv);
+    const uint32_t w[4] = {hv.x, hv.y, hv.z, hv.w};
+    float hf[8], r[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) r1[e] = y1[e] - f[e];
-    __stcs(reinterpret_cast<uint4 *>(lr + e1), pack(r1));
-    if (e2 >= 0) {
-        unpack(h2, f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) r2[e] = y2[e] - f[e];
-        __stcs(reinterpret_cast<uint4 *>(lr + e2), pack(r2));
+    for (int k = 0; k < 4; ++k) {
+        const float2 f = unpk16(w[k]);
+        hf[2 * k] = f.x;
+        hf[2 * k + 1] = f.y;
     }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) r[k] = y[k] - hf[k];   // exact in fp32
+    char *x8 = a.y_x8 + 2 * row;
+    __stcs(reinterpret_cast<uint2 *>(x8 + e),
+           make_uint2(pk8x4(r[0], r[1], r[2], r[3]), pk8x4(r[4], r[5], r[6], r[7])));
+    __stcs(reinterpret_cast<uint2 *>(x8 + a.D + e),
+           make_uint2(pk8x4(hf[0], hf[1], hf[2], hf[3]), pk8x4(hf[4], hf[5], hf[6], hf[7])));
 }
 
 // HALF pairing: a job covers N consecutive pairs i0..i0+N-1, i.e. the vector
-// at element i0 and the vector at element i0 + D/2.  kLo: also write the lo
-// parts (bf16 only).
-template <typename T, bool kHalf, bool kLo>
+// at element i0 and the vector at element i0 + D/2.  kX8: write the split
+// mode's fp16 and 8-bit cross parts instead of y in x's type (bf16 x only).
+template <typename T, bool kHalf, bool kX8>
 __global__ void __launch_bounds__(256) apply_rope_kernel(const __grid_constant__ RopeArgs a) {
     constexpr int N = Vec<T>::N;
     constexpr int P = kHalf ? N : N / 2;  // pairs per job
@@ -152,11 +181,13 @@ __global__ void __launch_bounds__(256) apply_rope_kernel(const __grid_constant__
                     y1[e] = fmaf(x1[e], c[e], -x2[e] * s[e]);
                     y2[e] = fmaf(x1[e], s[e], x2[e] * c[e]);
                 }
-                const uint4 h1 = pack(y1), h2 = pack(y2);
-                __stcs(reinterpret_cast<uint4 *>(yr + e1), h1);
-                __stcs(reinterpret_cast<uint4 *>(yr + e2), h2);
-                if constexpr (sizeof(T) == 2 && kLo)
-                    store_lo(a, b, l, h0 + u, e1, e2, y1, y2, h1, h2);
+                if constexpr (sizeof(T) == 2 && kX8) {
+                    store_split(a, b, l, h0 + u, e1, y1);
+                    store_split(a, b, l, h0 + u, e2, y2);
+                } else {
+                    __stcs(reinterpret_cast<uint4 *>(yr + e1), pack(y1));
+                    __stcs(reinterpret_cast<uint4 *>(yr + e2), pack(y2));
+                }
             } else {
                 float x[N], y[N];
                 unpack(va[u], x);
@@ -165,10 +196,14 @@ __global__ void __launch_bounds__(256) apply_rope_kernel(const __grid_constant__
                     y[2 * e] = fmaf(x[2 * e], c[e], -x[2 * e + 1] * s[e]);
                     y[2 * e + 1] = fmaf(x[2 * e], s[e], x[2 * e + 1] * c[e]);
                 }
-                const uint4 h = pack(y);
-                __stcs(reinterpret_cast<uint4 *>(yr + e1), h);
-                if constexpr (sizeof(T) == 2 && kLo)
-                    store_lo(a, b, l, h0 + u, e1, -1, y, y, h, h);
+                if constexpr (sizeof(T) == 2 && kX8) {
+                    float y8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) y8[e] = y[e];
+                    store_split(a, b, l, h0 + u, e1, y8);
+                } else {
+                    __stcs(reinterpret_cast<uint4 *>(yr + e1), pack(y));
+                }
             }
         }
     }
@@ -176,7 +211,7 @@ __global__ void __launch_bounds__(256) apply_rope_kernel(const __grid_constant__
 
 }  // namespace
 
-lcx_status apply_rope_impl(const lcx_rope_params *params, const void *x, void *y, void *y_lo,
+lcx_status apply_rope_impl(const lcx_rope_params *params, const void *x, void *y, void *y_x8,
                            int32_t dtype, int64_t B, int64_t H, int64_t L,
                            const int64_t *x_strides, const int64_t *y_strides, int64_t pos_offset,
                            cudaStream_t s) {
@@ -207,9 +242,10 @@ lcx_status apply_rope_impl(const lcx_rope_params *params, const void *x, void *y
         if (x_strides[d] % vec != 0 || ys[d] % vec != 0)
             return fail(LCX_ERR_UNSUPPORTED, "strides must be multiples of 16 bytes");
     }
-    if (!aligned16(x) || !aligned16(y) || !aligned16(y_lo))
+    if (!aligned16(x) || !aligned16(y) || !aligned16(y_x8))
         return fail(LCX_ERR_UNSUPPORTED, "x and y must be 16-byte aligned");
-    if (y_lo && dtype != LCX_BF16) return fail(LCX_ERR_UNSUPPORTED, "a lo part needs bf16");
+    if (y_x8 && (dtype != LCX_BF16 || x == y))
+        return fail(LCX_ERR_UNSUPPORTED, "split parts need bf16 x and a separate y");
     if (x == y) {
         for (int d = 0; d < 3; ++d)
             if (x_strides[d] != ys[d])
@@ -219,7 +255,8 @@ lcx_status apply_rope_impl(const lcx_rope_params *params, const void *x, void *y
     RopeArgs a;
     a.x = static_cast<const char *>(x);
     a.y = static_cast<char *>(y);
-    a.y_lo = static_cast<char *>(y_lo);
+    a.y_x8 = static_cast<char *>(y_x8);
+    a.D = D;
     a.xs_b = x_strides[0];
     a.xs_h = x_strides[1];
     a.xs_l = x_strides[2];
@@ -237,7 +274,7 @@ lcx_status apply_rope_impl(const lcx_rope_params *params, const void *x, void *y
     const int threads = a.rows_per_cta * a.jobs_per_row;
     dim3 grid(unsigned((L + a.rows_per_cta - 1) / a.rows_per_cta), unsigned(B));
     if (dtype == LCX_BF16) {
-        if (y_lo)
+        if (y_x8)
             half ? apply_rope_kernel<__nv_bfloat16, true, true><<<grid, threads, 0, s>>>(a)
                  : apply_rope_kernel<__nv_bfloat16, false, true><<<grid, threads, 0, s>>>(a);
         else

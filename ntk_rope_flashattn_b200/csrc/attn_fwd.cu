@@ -60,8 +60,6 @@ constexpr float kRescaleLog2 = 8.0f;    // rescale O only if the max grows by > 
 //   LCX_EMU_EVERY       1 column pair in N takes 2^x on the FMA pipe (0: none)
 //   LCX_D192_TWO_TILES  two query tiles and one K stage at D = 192 (0: one tile)
 //   LCX_KSTAGES_D128    K ring depth at D = 128 without split QK^T
-//   LCX_SPLIT_FUSED     split QK^T: Qhi [Klo; Khi]^T as one N = 128 product (key
-//                       parts interleaved by box) plus Qlo Khi^T, one S buffer
 //   LCX_ROT_UNROLL      rows in flight per rotation thread
 //   LCX_PHASOR_CARRY    reuse the phasor a K tile ends with for the next tile
 #ifndef LCX_EMU_EVERY
@@ -72,9 +70,6 @@ constexpr float kRescaleLog2 = 8.0f;    // rescale O only if the max grows by > 
 #endif
 #ifndef LCX_KSTAGES_D128
 #define LCX_KSTAGES_D128 2
-#endif
-#ifndef LCX_SPLIT_FUSED
-#define LCX_SPLIT_FUSED 1
 #endif
 #ifndef LCX_ROT_UNROLL
 #define LCX_ROT_UNROLL 2
@@ -113,60 +108,65 @@ struct AttnParams {
     float *part_o;                     // n_split > 1: [n_split, B, Hq, L, D] partial o
     float *part_lse;                   //              [n_split, B, Hq, L] partial lse
     int test_stall;                    // loader issues nothing (watchdog test hook)
+    int rot_help;                      // head-packed split-KV with keys rotated on chip: the
+                                       // softmax warps (bit w = warp w; 0 or 4 of them) whose
+                                       // rows hold no query in either tile and that rotate key
+                                       // tiles with warps 8-11
     int k_rope_shared;                 // rotated key columns come from one shared head
-    int k_lo_tma;                      // split mode: the keys' lo parts arrive by TMA
+    int k_x8_tma;                      // split mode: the keys' 8-bit cross parts arrive by TMA
     float rot_ms;                      // factor on rotated values (partial rotary: mscale)
     float c_log2;                      // logit scale in log2 units
     unsigned long long timeout_ns;
     float theta[64];
 };
 
-// Shared-memory plan.  A tile of R rows x D bf16 is stored as D/64 TMA boxes of
-// R rows x 128 bytes with the 128-byte swizzle.  In the split mode every Q and
-// K tile has a second "lo" part holding bf16(x' - bf16(x')), and key tiles are
-// 64 rows so that both parts fit.  D is the query/key head dim, DV the
-// value/output head dim; at D = 192 (decoupled RoPE: 128 + 64) two query tiles
-// (96 KB) leave room for one K stage (48 KB) and two V stages (32 KB each).
-// The K stage is released as soon as both S products of key tile j are done,
-// so key tile j + 1 lands while the softmax of j runs; the second V stage lets
-// V(j + 1) land while PV(j) still reads V(j).  That beats two K stages with one
-// V stage (1038 vs 942 TFLOP/s on a 16-head L 16384 prefill).
+// Shared-memory plan.  A tile of R rows x D 16-bit values is stored as D/64 TMA
+// boxes of R rows x 128 bytes with the 128-byte swizzle.  D is the query/key
+// head dim, DV the value/output head dim; at D = 192 (decoupled RoPE: 128 + 64)
+// two query tiles (96 KB) leave room for one K stage (48 KB) and two V stages
+// (32 KB each).  The K stage is released as soon as both S products of key
+// tile j are done, so key tile j + 1 lands while the softmax of j runs; the
+// second V stage lets V(j + 1) land while PV(j) still reads V(j).  That beats
+// two K stages with one V stage (1038 vs 942 TFLOP/s on a 16-head L 16384
+// prefill).
+//
+// Split QK^T mode: every rotated value x' is held as an fp16 part h = f16(x')
+// and the rounding residual r = x' - h, and
+//   S = Qh Kh^T + [e5m2(Qh) | e5m2(Qr)] [e5m2(Kr) | e5m2(Kh)]^T,
+// one fp16 product (kind::f16) plus one e5m2 product over K = 2D
+// (kind::f8f6f4, twice the fp16 rate, so it costs what one more fp16 product
+// over K = D would).  The cross terms h r' are ~2^-11 of S, so their 3-bit
+// e5m2 operands still leave the logits accurate to about 2^-15 relative;
+// only the product of the two residuals (~2^-22) is dropped.  Each Q and K
+// tile then has a second part, the 8-bit cross operand: 2D bytes per row, the
+// size of a 16-bit part, stored as D/64 boxes of 128-byte rows ([h8 | r8] for
+// a query row, [r8 | h8] for a key row).  Key tiles stay 128 rows; at D = 128
+// the parts fill shared memory with one K stage (64 KB) and one V stage.
 template <int D, int DV, bool kSplit>
 struct Cfg {
-    static constexpr int BN = kSplit ? 64 : 128;        // keys per tile
-    static constexpr int kParts = kSplit ? 2 : 1;       // hi (+ lo) parts of Q and K
+    static constexpr int BN = 128;                      // keys per tile
+    static constexpr int kParts = kSplit ? 2 : 1;       // 16-bit part (+ 8-bit cross part)
     static constexpr int kNTQ = (D > 128 && !LCX_D192_TWO_TILES) ? 1 : 2;  // query tiles per CTA
     static constexpr int kTileQ = kBM * D * 2;          // one part of a Q tile
     static constexpr int kTileK = BN * D * 2;           // one part of a K tile
     static constexpr int kTileV = BN * DV * 2;          // a V tile
     static constexpr int kBoxQ = kBM * 128;
     static constexpr int kBoxK = BN * 128;
-    static constexpr int kStagesK = (D == 64) ? 4
-                                  : (D == 128 && !kSplit) ? LCX_KSTAGES_D128
-                                  : (D > 128 && kNTQ == 2) ? 1 : 2;
-    static constexpr int kStagesV = (D == 64) ? 4 : 2;
+    static constexpr int kStagesK = kSplit ? (D == 64 ? 3 : 1)
+                                  : (D == 64) ? 4
+                                  : (D == 128) ? LCX_KSTAGES_D128
+                                  : (kNTQ == 2) ? 1 : 2;
+    static constexpr int kStagesV = kSplit ? (D == 64 ? 3 : 1) : (D == 64) ? 4 : 2;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kNTQ * kParts * kTileQ;
     static constexpr int kOffV = kOffK + kStagesK * kParts * kTileK;
     static constexpr int kOffBar = kOffV + kStagesV * kTileV;
     static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers + alignment slack
-    // Split mode, fused: the hi and lo parts of a K stage are interleaved box by
-    // box (lo box b, then hi box b), so that [Klo; Khi] is one 2 BN-row operand
-    // and Qhi [Klo; Khi]^T one N = 2 BN product; its S buffer is 2 BN columns
-    // (Qhi Klo^T, then Qhi Khi^T + Qlo Khi^T), one per query tile.  Otherwise
-    // the split mode's 64-key tiles leave TMEM room for two S buffers per query
-    // tile, so its S runs two key tiles ahead of PV.
-    static constexpr bool kFused = kSplit && LCX_SPLIT_FUSED != 0;
-    static constexpr int kNB = (kSplit && !kFused) ? 2 : 1;   // S buffers per query tile
-    static constexpr int kSCols = kFused ? 2 * BN : BN;       // TMEM columns of an S buffer
-    static constexpr int kKBoxStride = kFused ? 2 * kBoxK : kBoxK;  // between a part's boxes
-    static constexpr int kKHi = kFused ? kBoxK : 0;           // hi part in a K stage
-    static constexpr int kKLo = kFused ? 0 : kTileK;          // lo part in a K stage
-    // TMEM columns: S_t,b at (t kNB + b) kSCols (P_t,b aliased over its first
-    // BN/2 columns), O_t after.
-    static constexpr int kColO = 2 * kNB * kSCols;
+    // TMEM columns: S_t at t BN (P_t aliased over its first BN/2 columns), O_t
+    // from 2 BN on.
+    static constexpr int kColO = 2 * BN;
     static_assert(kSmemBytes <= 232448, "shared memory budget");
-    static_assert(2 * kNB * kSCols + 2 * DV <= 512, "TMEM budget");
+    static_assert(2 * BN + 2 * DV <= 512, "TMEM budget");
 };
 
 template <int NSK, int NSV>
@@ -174,7 +174,7 @@ struct Bars {
     uint64_t full_q, ready_q;
     uint64_t full_k[NSK], ready_k[NSK], empty_k[NSK];
     uint64_t full_v[NSV], empty_v[NSV];
-    uint64_t s_ready[2][2], p_ready[2][2], pv_done[2], o_ready[2];
+    uint64_t s_ready[2], p_ready[2], o_ready[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -283,11 +283,14 @@ __device__ __forceinline__ uint32_t chunk_off(int r, int fc, int box_bytes) {
     return (fc >> 3) * box_bytes + r * 128 + (((fc & 7) ^ (r & 7)) << 4);
 }
 
-template <int D, bool kHalf>
+// The rotation's work split among NT threads (the rotation warpgroup's 128, or
+// 256 when idle softmax warps of a decode launch help with the key tiles).
+template <int D, bool kHalf, int NT = 128>
 struct Rot {
     static constexpr int CPR = kHalf ? D / 16 : D / 8;  // jobs per row
-    static constexpr int RP = 128 / CPR;                 // rows per pass of the WG
+    static constexpr int RP = NT / CPR;                  // rows per pass of the NT threads
     static constexpr int PPJ = kHalf ? 8 : 4;            // pairs per job
+    static_assert(NT % CPR == 0 && 128 % RP == 0, "rotation work split");
 };
 
 // Rotate one job's pairs, two pairs per packed instruction: x1/x2 are the pair
@@ -321,34 +324,53 @@ __device__ __forceinline__ uint4 pack8(const float (&y)[8]) {
     return make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
                       pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
 }
-// hi = bf16(y) (returned packed), y -= hi (the residual, for the lo part).
-__device__ __forceinline__ uint4 pack8_hi(float (&y)[8]) {
-    const uint4 h = pack8(y);
-    float hf[8];
-    unpack8(h, hf);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) y[e] -= hf[e];
-    return h;
+// Byte offset of byte x of row r in a tile of 128-byte swizzled rows whose
+// boxes are box_bytes long (x < 128 per box: box x / 128, 16-byte chunk x / 16
+// of that box's row at chunk (x / 16) ^ (r & 7)).
+__device__ __forceinline__ uint32_t byte_off(int r, int x, int box_bytes) {
+    return (x >> 7) * box_bytes + r * 128 + ((((x >> 4) & 7) ^ (r & 7)) << 4) + (x & 15);
 }
 
-// Store 8 rotated values: bf16 hi part at `hi`, and in the split mode the bf16
-// residual at the same offset of the lo part.
-template <bool kSplit>
-__device__ __forceinline__ void store8(uint8_t *hi, uint8_t *lo, uint32_t off, float (&y)[8]) {
-    if (kSplit) {
-        *reinterpret_cast<uint4 *>(hi + off) = pack8_hi(y);
-        *reinterpret_cast<uint4 *>(lo + off) = pack8(y);
+// Store the 8 rotated values of 16-byte chunk fc (columns 8 fc .. 8 fc + 7) of
+// row r.  Plain mode: bf16 into the tile.  Split mode: the fp16 part h into the
+// tile and, into the 8-bit cross part x8, e5m2(h) and e5m2(x' - h): a query row
+// holds [h8 | r8] (column c at bytes c and D + c), a key row [r8 | h8].
+template <bool kSplit, bool kKey, int D, int BOX>
+__device__ __forceinline__ void store8(uint8_t *tile, uint8_t *x8, int r, int fc,
+                                       const float (&y)[8]) {
+    const uint32_t off = chunk_off(r, fc, BOX);
+    if constexpr (!kSplit) {
+        *reinterpret_cast<uint4 *>(tile + off) = pack8(y);
     } else {
-        *reinterpret_cast<uint4 *>(hi + off) = pack8(y);
+        const uint4 h = make_uint4(pack_f16x2(y[0], y[1]), pack_f16x2(y[2], y[3]),
+                                   pack_f16x2(y[4], y[5]), pack_f16x2(y[6], y[7]));
+        *reinterpret_cast<uint4 *>(tile + off) = h;
+        const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
+        float hf[8], rr[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = f16x2_to_f32x2(hw[k]);
+            hf[2 * k] = f.x;
+            hf[2 * k + 1] = f.y;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) rr[e] = y[e] - hf[e];   // exact in fp32
+        const uint2 h8 = make_uint2(pack_e5m2x4(hf[0], hf[1], hf[2], hf[3]),
+                                    pack_e5m2x4(hf[4], hf[5], hf[6], hf[7]));
+        const uint2 r8 = make_uint2(pack_e5m2x4(rr[0], rr[1], rr[2], rr[3]),
+                                    pack_e5m2x4(rr[4], rr[5], rr[6], rr[7]));
+        const int c = 8 * fc;
+        *reinterpret_cast<uint2 *>(x8 + byte_off(r, kKey ? D + c : c, BOX)) = h8;
+        *reinterpret_cast<uint2 *>(x8 + byte_off(r, kKey ? c : D + c, BOX)) = r8;
     }
 }
 
 // Per-thread phasor state of the rotation warpgroup: the thread always handles
 // the same pairs i0..i0+PPJ-1 and rows r0 + RP k, so it starts each tile at
 // e^{i (pos0 + r0) theta} and steps by e^{i RP theta}.
-template <int D, bool kHalf>
+template <int D, bool kHalf, int NT = 128>
 struct Phasor {
-    using R = Rot<D, kHalf>;
+    using R = Rot<D, kHalf, NT>;
     float sc[R::PPJ], ss[R::PPJ];  // step
     int q, r0, i0;
     __device__ __forceinline__ void init(int tw, const AttnParams &p) {
@@ -400,28 +422,25 @@ struct PhasorCarry {
 };
 constexpr int kReseed = 16;
 
-// Rotate a ROWS x D bf16 tile in place (row r at position pos0 + r); only its
-// last RD columns are rotated (RD = D: all of them).  In the split mode also
-// write the residual part into `lo`.
-// Rotate (or, with rotate = false, only copy into hi/lo parts) this thread's
-// pairs of row r of a tile whose boxes are BOX bytes long; (c, s) the phasor.
-template <int D, int RD, bool kHalf, bool kSplit, int BOX>
-__device__ __forceinline__ void rotate_row(uint8_t *tile, uint8_t *lo, int r, int q,
+// Rotate (or, with rotate = false, only copy into the split mode's parts) this
+// thread's pairs of row r of a tile whose boxes are BOX bytes long; (c, s) the
+// phasor.  Only the last RD of the D columns are rotated.
+template <int D, int RD, bool kHalf, bool kSplit, bool kKey, int BOX>
+__device__ __forceinline__ void rotate_row(uint8_t *tile, uint8_t *x8, int r, int q,
                                            const float *c, const float *s, bool rotate) {
     constexpr int C0 = (D - RD) / 8;  // first rotated 16-byte chunk of a row
     if (kHalf) {
-        const uint32_t oa = chunk_off(r, C0 + q, BOX);
-        const uint32_t ob = chunk_off(r, C0 + q + RD / 16, BOX);
+        const int fa = C0 + q, fb = C0 + q + RD / 16;
         float x1[8], x2[8];
-        unpack8(*reinterpret_cast<const uint4 *>(tile + oa), x1);
-        unpack8(*reinterpret_cast<const uint4 *>(tile + ob), x2);
+        unpack8(*reinterpret_cast<const uint4 *>(tile + chunk_off(r, fa, BOX)), x1);
+        unpack8(*reinterpret_cast<const uint4 *>(tile + chunk_off(r, fb, BOX)), x2);
         if (rotate) rot_pairs<8>(x1, x2, c, s);
-        store8<kSplit>(tile, lo, oa, x1);
-        store8<kSplit>(tile, lo, ob, x2);
+        store8<kSplit, kKey, D, BOX>(tile, x8, r, fa, x1);
+        store8<kSplit, kKey, D, BOX>(tile, x8, r, fb, x2);
     } else {
-        const uint32_t oa = chunk_off(r, C0 + q, BOX);
+        const int fa = C0 + q;
         float x[8];
-        unpack8(*reinterpret_cast<const uint4 *>(tile + oa), x);
+        unpack8(*reinterpret_cast<const uint4 *>(tile + chunk_off(r, fa, BOX)), x);
         if (rotate) {
             float x1[4], x2[4];
 #pragma unroll
@@ -436,7 +455,7 @@ __device__ __forceinline__ void rotate_row(uint8_t *tile, uint8_t *lo, int r, in
                 x[2 * e + 1] = x2[e];
             }
         }
-        store8<kSplit>(tile, lo, oa, x);
+        store8<kSplit, kKey, D, BOX>(tile, x8, r, fa, x);
     }
 }
 
@@ -457,20 +476,22 @@ __device__ __forceinline__ void rotate_packed_q(uint8_t *tile, uint8_t *lo, long
         if (rel < 0 || rel >= heads * stride || rel % stride >= Lp) continue;
         float c[R::PPJ], s[R::PPJ];
         if (rotate) ph.template start<(RD < D)>(pos0 + rel % stride - ph.r0, p, c, s);
-        rotate_row<D, RD, kHalf, kSplit, kBM * 128>(tile, lo, r, ph.q, c, s, rotate);
+        rotate_row<D, RD, kHalf, kSplit, false, kBM * 128>(tile, lo, r, ph.q, c, s, rotate);
     }
 }
 
-// BS: bytes between the tile's 64-column boxes (ROWS x 128 unless the parts
-// of a split key tile are interleaved box by box).
-template <int D, int RD, bool kHalf, bool kSplit, int ROWS, int BS = ROWS * 128>
+// Rotate a ROWS x D bf16 tile in place (row r at position pos0 + r); only its
+// last RD columns are rotated (RD = D: all of them).  In the split mode the
+// tile receives the fp16 parts and `lo` the 8-bit cross parts (kKey: the key
+// order [r8 | h8]).
+template <int D, int RD, bool kHalf, bool kSplit, bool kKey, int ROWS, int NT = 128>
 __device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, uint8_t *lo, long long pos0,
-                                                 const Phasor<RD, kHalf> &ph, const AttnParams &p,
-                                                 bool rotate,
+                                                 const Phasor<RD, kHalf, NT> &ph,
+                                                 const AttnParams &p, bool rotate,
                                                  PhasorCarry<Rot<RD, kHalf>::PPJ> *carry = nullptr) {
-    using R = Rot<RD, kHalf>;
+    using R = Rot<RD, kHalf, NT>;
     constexpr int NJ = ROWS / R::RP;
-    constexpr int BOX = BS;
+    constexpr int BOX = ROWS * 128;
     float c[R::PPJ], s[R::PPJ];
     if (rotate) {
         if (LCX_PHASOR_CARRY && carry && carry->next == pos0 && carry->age < kReseed) {
@@ -485,10 +506,12 @@ __device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, uint8_t *lo, lon
             if (carry) carry->age = 0;
         }
     }
-#pragma unroll kRotUnroll
+    // the split mode's stores take more registers: one row in flight
+    constexpr int kUnroll = kSplit ? 1 : kRotUnroll;
+#pragma unroll kUnroll
     for (int k = 0; k < NJ; ++k) {
         const int r = ph.r0 + k * R::RP;
-        rotate_row<D, RD, kHalf, kSplit, BOX>(tile, lo, r, ph.q, c, s, rotate);
+        rotate_row<D, RD, kHalf, kSplit, kKey, BOX>(tile, lo, r, ph.q, c, s, rotate);
         if (rotate) ph.step(c, s);
     }
     if (LCX_PHASOR_CARRY && carry && rotate) {
@@ -502,16 +525,16 @@ __device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, uint8_t *lo, lon
 }
 
 // fp32 operands: load ROWS rows from global (rows >= L read as zero), rotate in
-// fp32 when asked (row r at position pos0 + r), round to bf16 (hi, and lo in
-// the split mode) into the tile.
-template <int D, bool kHalf, bool kSplit, int ROWS, int BS = ROWS * 128>
+// fp32 when asked (row r at position pos0 + r), round to bf16 (split mode: the
+// fp16 part, and the 8-bit cross part into `lo`) into the tile.
+template <int D, bool kHalf, bool kSplit, bool kKey, int ROWS>
 __device__ __forceinline__ void load_tile_f32(uint8_t *tile, uint8_t *lo, const float *base,
                                               long long rs, int row0, int L, long long pos0,
                                               bool rotate, const Phasor<D, kHalf> &ph,
                                               const AttnParams &p) {
     using R = Rot<D, kHalf>;
     constexpr int NJ = ROWS / R::RP;
-    constexpr int BOX = BS;
+    constexpr int BOX = ROWS * 128;
     float c[R::PPJ], s[R::PPJ];
     if (rotate) ph.start(pos0, p, c, s);
     for (int k = 0; k < NJ; ++k) {
@@ -526,8 +549,8 @@ __device__ __forceinline__ void load_tile_f32(uint8_t *tile, uint8_t *lo, const 
                 x2[e] = valid ? src[ph.i0 + e + D / 2] : 0.f;
             }
             if (rotate) rot_pairs<8>(x1, x2, c, s);
-            store8<kSplit>(tile, lo, chunk_off(r, ph.q, BOX), x1);
-            store8<kSplit>(tile, lo, chunk_off(r, ph.q + D / 16, BOX), x2);
+            store8<kSplit, kKey, D, BOX>(tile, lo, r, ph.q, x1);
+            store8<kSplit, kKey, D, BOX>(tile, lo, r, ph.q + D / 16, x2);
         } else {
             float x[8];
 #pragma unroll
@@ -546,7 +569,7 @@ __device__ __forceinline__ void load_tile_f32(uint8_t *tile, uint8_t *lo, const 
                     x[2 * e + 1] = x2[e];
                 }
             }
-            store8<kSplit>(tile, lo, chunk_off(r, ph.q, BOX), x);
+            store8<kSplit, kKey, D, BOX>(tile, lo, r, ph.q, x);
         }
         if (rotate) ph.step(c, s);
     }
@@ -569,15 +592,6 @@ __device__ __forceinline__ void load_v_f32(uint8_t *tile, const float *base, lon
     }
 }
 
-// Whole-row TMEM access for the softmax (128 or 64 columns).
-__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, float (&v)[128]) { tmem_ld128(taddr, v); }
-__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, float (&v)[64]) { tmem_ld64(taddr, v); }
-__device__ __forceinline__ void tmem_st_row(uint32_t taddr, const uint32_t (&u)[64]) {
-    tmem_st64(taddr, u);
-}
-__device__ __forceinline__ void tmem_st_row(uint32_t taddr, const uint32_t (&u)[32]) {
-    tmem_st32(taddr, u);
-}
 
 // Max of N values (N % 8 == 0) with four independent chains of 3-input max:
 // v[0..3] start the chains, v[4 .. N-5] are taken 8 at a time, v[N-4 .. N-1]
@@ -667,6 +681,31 @@ __device__ __forceinline__ RowMap map_row(const AttnParams &p, const Unit &U, in
     return m;
 }
 
+// Key tiles of a head-packed split-KV launch rotated by 256 threads: the
+// rotation warpgroup (tw 0..127) and four softmax warps that hold no query
+// (tw 128..255), each thread taking every 32nd row of its pairs.  The same
+// stage protocol as the rotation warpgroup alone: wait for the TMA, rotate in
+// place (split mode: into the fp16 and 8-bit cross parts), arrive on ready_k.
+template <int D, int RD, bool kHalf, bool kSplit, int NSK, int BN, int kParts, int kTileK,
+          typename Bar>
+__device__ __forceinline__ void rotate_keys_helped(int tw, const Tiles &T, uint8_t *sK, Bar &bar,
+                                                   const AttnParams &p, volatile int *abort,
+                                                   uint64_t tmo) {
+    Phasor<RD, kHalf, 256> ph;
+    ph.init(tw, p);
+    PhasorCarry<Rot<RD, kHalf>::PPJ> carry;
+    for (int j = 0; j < T.n; ++j) {
+        const int jt = T.tile(j), s = j % NSK;
+        uint8_t *tk = sK + s * kParts * kTileK;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar.full_k[s], (j / NSK) & 1, abort, tmo)))
+            break;
+        rotate_tile_bf16<D, RD, kHalf, kSplit, true, BN, 256>(tk, tk + kTileK, (long long)jt * BN,
+                                                              ph, p, true, &carry);
+        fence_proxy_async_smem();
+        mbar_arrive(&bar.ready_k[s]);
+    }
+}
+
 // ---------------------------------------------------------------- kernel
 // D: query/key head dim, DV: value/output head dim, RD: rotated (last) dims;
 // kKvSplit: this launch is one pass of split-KV (partial results per split).
@@ -705,7 +744,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bar.ready_q, 128);
         for (int s = 0; s < NSK; ++s) {
             mbar_init(&bar.full_k[s], 1);
-            mbar_init(&bar.ready_k[s], 128);
+            mbar_init(&bar.ready_k[s], 128 + 32 * __popc(p.rot_help));
             mbar_init(&bar.empty_k[s], 1);
         }
         for (int s = 0; s < NSV; ++s) {
@@ -713,11 +752,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bar.empty_v[s], 1);
         }
         for (int t = 0; t < 2; ++t) {
-            for (int b = 0; b < 2; ++b) {
-                mbar_init(&bar.s_ready[t][b], 1);
-                mbar_init(&bar.p_ready[t][b], 128);
-            }
-            mbar_init(&bar.pv_done[t], 1);
+            mbar_init(&bar.s_ready[t], 1);
+            // every softmax warp hands over P of every tile, except the ones that
+            // help rotate keys
+            mbar_init(&bar.p_ready[t], 32 * (8 - __popc(p.rot_help)));
             mbar_init(&bar.o_ready[t], 1);
         }
         mbar_init(&bar.drain, 1);
@@ -763,7 +801,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_prefetch_desc(&tmq);
                 tma_prefetch_desc(&tmk);
                 tma_prefetch_desc(&tmv);
-                if ((RD < D && p.k_rope_shared) || p.k_lo_tma) tma_prefetch_desc(&tmkr);
+                if ((RD < D && p.k_rope_shared) || p.k_x8_tma) tma_prefetch_desc(&tmkr);
                 // With a shared rotary key, the K boxes from column D - RD on
                 // come from that tensor's single head.
                 constexpr int kNopeBoxes = (D - RD) / 64;
@@ -794,18 +832,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int sk = j % NSK, uk = j / NSK, sv = j % NSV, uv = j / NSV;
                     if (uk > 0) ok = mbar_wait(&bar.empty_k[sk], (uk - 1) & 1, abort, tmo);
                     if (!ok) break;
-                    // split mode with keys split by the rotate pass: the lo part
-                    // (fourth tensor map) lands in the stage's second part
-                    const bool lo = kSplit && p.k_lo_tma;
-                    mbar_arrive_expect_tx(&bar.full_k[sk], lo ? 2 * C::kTileK : C::kTileK);
-                    if (lo)
+                    // split mode with keys split by the rotate pass: the fp16 parts
+                    // come through tmk, the 8-bit cross parts (fourth tensor map,
+                    // 2 D bytes per key, 128-byte boxes) into the stage's second part
+                    const bool x8 = kSplit && p.k_x8_tma;
+                    mbar_arrive_expect_tx(&bar.full_k[sk], x8 ? 2 * C::kTileK : C::kTileK);
+                    if (x8)
                         for (int bx = 0; bx < D / 64; ++bx)
-                            tma_load_4d(sK + sk * C::kParts * C::kTileK + C::kKLo +
-                                            bx * C::kKBoxStride,
-                                        &tmkr, &bar.full_k[sk], bx * 64, jt * BN, U.g, U.b);
+                            tma_load_4d(sK + sk * C::kParts * C::kTileK + C::kTileK +
+                                            bx * C::kBoxK,
+                                        &tmkr, &bar.full_k[sk], bx * 128, jt * BN, U.g, U.b);
                     for (int bx = 0; bx < D / 64; ++bx) {
-                        uint8_t *dst =
-                            sK + sk * C::kParts * C::kTileK + C::kKHi + bx * C::kKBoxStride;
+                        uint8_t *dst = sK + sk * C::kParts * C::kTileK + bx * C::kBoxK;
                         if constexpr (RD < D) {
                             if (p.k_rope_shared && bx >= kNopeBoxes) {
                                 tma_load_4d(dst, &tmkr, &bar.full_k[sk], (bx - kNopeBoxes) * 64,
@@ -835,76 +873,63 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (warp == kWarpMma) {
             // ------------------------------------------------ MMA issuer
             if (lane == 0) {
-                constexpr uint32_t kIdS = idesc_bf16_f32(128, BN, 0, 0);
-                constexpr uint32_t kIdS2 = idesc_bf16_f32(128, 2 * BN, 0, 0);   // fused split
+                // S: bf16 (plain) or fp16 (split: the Qh Kh^T product) operands;
+                // the split mode's cross product takes e5m2 operands.
+                constexpr uint32_t kIdS = kSplit ? idesc_f32acc(128, BN, kFmtF16, kFmtF16, 0, 0)
+                                                 : idesc_bf16_f32(128, BN, 0, 0);
+                constexpr uint32_t kIdX8 = idesc_f32acc(128, BN, kFmtE5M2, kFmtE5M2, 0, 0);
                 constexpr uint32_t kIdPV = idesc_bf16_f32(128, DV, 0, 1);
                 const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
                 // S_t = Q_t K^T over D in steps of 16 (32 bytes inside a 128-byte
-                // swizzle row, then the next 64-column box).  Split mode:
-                // S = Qhi Klo + Qlo Khi + Qhi Khi, all accumulated in fp32.
-                // Descriptors of the first K step; later steps only move the start
-                // address (in 16-byte units, well inside the 14-bit field).
+                // swizzle row, then the next 64-column box).  Descriptors of the
+                // first K step; later steps only move the start address (in
+                // 16-byte units, well inside the 14-bit field).
                 const uint64_t dq0 = sdesc_sw128(q_addr, 16, 1024);
                 const uint64_t dk0 = sdesc_sw128(k_addr, 16, 1024);
                 const uint64_t dv0 = sdesc_sw128(v_addr, C::kBoxK, 1024);
-                constexpr int NB = C::kNB;
-                auto issue_s = [&](int t, int s, int b) {
+                auto issue_s = [&](int t, int s) {
                     const uint64_t qa = dq0 + ((t * C::kParts * C::kTileQ) >> 4);
                     const uint64_t ka = dk0 + ((s * C::kParts * C::kTileK) >> 4);
-                    const uint32_t dst = tmem + (t * NB + b) * C::kSCols;
-                    if constexpr (C::kFused) {
-                        // Qhi [Klo; Khi]^T over the 2 BN rows of a box pair (lo box,
-                        // then hi box: 8-row groups 1024 bytes apart throughout),
-                        // then Qlo Khi^T onto the Qhi Khi^T half
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t oq = ((kk >> 2) * C::kBoxQ + (kk & 3) * 32) >> 4;
-                            const uint32_t ok_ = ((kk >> 2) * C::kKBoxStride + (kk & 3) * 32) >> 4;
-                            mma_ss(dst, qa + oq, ka + ok_, kIdS2, kk > 0);
-                        }
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t oq = ((kk >> 2) * C::kBoxQ + (kk & 3) * 32) >> 4;
-                            const uint32_t ok_ = ((kk >> 2) * C::kKBoxStride + (kk & 3) * 32) >> 4;
-                            mma_ss(dst + BN, qa + (C::kTileQ >> 4) + oq, ka + (C::kKHi >> 4) + ok_,
-                                   kIdS, true);
-                        }
-                        return;
-                    }
-                    constexpr int NPROD = kSplit ? 3 : 1;
-#pragma unroll
-                    for (int pr = 0; pr < NPROD; ++pr) {
-                        const uint64_t qp = qa + (((kSplit && pr == 1) ? C::kTileQ : 0) >> 4);
-                        const uint64_t kp = ka + (((kSplit && pr == 0) ? C::kTileK : 0) >> 4);
+                    const uint32_t dst = tmem + t * BN;
+                    if constexpr (kSplit) {
+                        // the e5m2 cross product first, into a fresh accumulator:
+                        // [h8 | r8]_q [r8 | h8]_k^T over K = 2 D in steps of 32
+                        // bytes -- the same byte walk as the 16-bit product
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint32_t oq = ((kk >> 2) * C::kBoxQ + (kk & 3) * 32) >> 4;
                             const uint32_t ok_ = ((kk >> 2) * C::kBoxK + (kk & 3) * 32) >> 4;
-                            mma_ss(dst, qp + oq, kp + ok_, kIdS, (pr > 0 || kk > 0));
+                            mma_ss_f8(dst, qa + (C::kTileQ >> 4) + oq, ka + (C::kTileK >> 4) + ok_,
+                                      kIdX8, kk > 0);
                         }
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t oq = ((kk >> 2) * C::kBoxQ + (kk & 3) * 32) >> 4;
+                        const uint32_t ok_ = ((kk >> 2) * C::kBoxK + (kk & 3) * 32) >> 4;
+                        mma_ss(dst, qa + oq, ka + ok_, kIdS, kSplit || kk > 0);
                     }
                 };
                 // O_t += P_t V: P from TMEM (BN/2 columns of bf16 pairs), V MN-major.
-                auto issue_pv = [&](int t, int s, int b, bool acc) {
+                auto issue_pv = [&](int t, int s, bool acc) {
                     const uint64_t va = dv0 + ((s * C::kTileV) >> 4);
                     const uint32_t dst = tmem + C::kColO + t * DV;
-                    const uint32_t pa = tmem + (t * NB + b) * C::kSCols;
+                    const uint32_t pa = tmem + t * BN;
 #pragma unroll
                     for (int kk = 0; kk < BN / 16; ++kk)
                         mma_ts(dst, pa + kk * 8, va + ((kk * 2048) >> 4), kIdPV, (acc || kk > 0));
                 };
-                // S_t(j + NB) is issued after PV_t(j), into the buffer P_t(j)
-                // occupied (MMAs of one thread execute in order).  With NB = 1
-                // the order is PV0(j), S0(j+1), PV1(j), S1(j+1): one query tile's
-                // softmax overlaps the other tile's products.  With NB = 2 it is
-                // PV0(j), PV1(j), S0(j+2), S1(j+2), and a softmax never waits for
-                // its own previous PV.
-                // Keys already rotated (and no hi/lo split) need no pass through
-                // the rotation warpgroup: the MMA waits for the TMA itself.
-                uint64_t *kready = (kF32 || (kSplit && !p.k_lo_tma) || p.rotate_k) ? bar.ready_k
+                // S_t(j + 1) is issued after PV_t(j), into the buffer P_t(j)
+                // occupied (MMAs of one thread execute in order): the order is
+                // PV0(j), S0(j+1), PV1(j), S1(j+1), so one query tile's softmax
+                // overlaps the other tile's products.
+                // Keys already rotated (and, in the split mode, already in parts)
+                // need no pass through the rotation warpgroup: the MMA waits for
+                // the TMA itself.
+                uint64_t *kready = (kF32 || (kSplit && !p.k_x8_tma) || p.rotate_k) ? bar.ready_k
                                                                                     : bar.full_k;
                 bool ok = mbar_wait(&bar.ready_q, 0, abort, tmo);
-                if (kKvSplit && NB == 1 && p.pack_ilv) {
+                if (kKvSplit && p.pack_ilv) {
                     // Both query tiles hold the same queries and tile t takes the
                     // key tiles j = t mod 2, so two K/V tiles are in flight per
                     // CTA: S_t(j + 2) follows PV_t(j) into the buffer P_t(j) held.
@@ -912,76 +937,60 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = mbar_wait(&kready[j % NSK], (j / NSK) & 1, abort, tmo);
                         tc_fence_after();
                         if (!ok) break;
-                        issue_s(j, j % NSK, 0);
-                        mma_commit(&bar.s_ready[j][0]);
+                        issue_s(j, j % NSK);
+                        mma_commit(&bar.s_ready[j]);
                         mma_commit(&bar.empty_k[j % NSK]);
                     }
                     for (int j = 0; ok && j < T.n; ++j) {
                         const int t = j & 1, sv = j % NSV, jn = j + 2;
                         ok = mbar_wait(&bar.full_v[sv], (j / NSV) & 1, abort, tmo);
-                        if (ok) ok = mbar_wait(&bar.p_ready[t][0], (j >> 1) & 1, abort, tmo);
+                        if (ok) ok = mbar_wait(&bar.p_ready[t], (j >> 1) & 1, abort, tmo);
                         tc_fence_after();
                         if (!ok) break;
-                        issue_pv(t, sv, 0, j >= 2);
+                        issue_pv(t, sv, j >= 2);
                         mma_commit(&bar.empty_v[sv]);
                         if (jn < T.n) {
                             const int sk = jn % NSK;
                             ok = mbar_wait(&kready[sk], (jn / NSK) & 1, abort, tmo);
                             tc_fence_after();
                             if (!ok) break;
-                            issue_s(t, sk, 0);
-                            mma_commit(&bar.s_ready[t][0]);
+                            issue_s(t, sk);
+                            mma_commit(&bar.s_ready[t]);
                             mma_commit(&bar.empty_k[sk]);
                         }
                     }
                 } else {
-                    for (int jj = 0; ok && jj < NB && jj < T.n; ++jj) {
-                        ok = mbar_wait(&kready[jj % NSK], (jj / NSK) & 1, abort, tmo);
+                    if (T.n > 0) {
+                        ok = ok && mbar_wait(&kready[0], 0, abort, tmo);
                         tc_fence_after();
-                        if (!ok) break;
-                        for (int t = 0; t < U.nt; ++t) {
-                            issue_s(t, jj % NSK, jj % NB);
-                            mma_commit(&bar.s_ready[t][jj % NB]);
+                        if (ok) {
+                            for (int t = 0; t < U.nt; ++t) {
+                                issue_s(t, 0);
+                                mma_commit(&bar.s_ready[t]);
+                            }
+                            mma_commit(&bar.empty_k[0]);
                         }
-                        mma_commit(&bar.empty_k[jj % NSK]);
                     }
                     for (int j = 0; ok && j < T.n; ++j) {
-                        const int sv = j % NSV, jn = j + NB;
+                        const int sv = j % NSV, jn = j + 1;
                         ok = mbar_wait(&bar.full_v[sv], (j / NSV) & 1, abort, tmo);
                         for (int t = 0; ok && t < U.nt; ++t) {
-                            ok = mbar_wait(&bar.p_ready[t][j % NB], (j / NB) & 1, abort, tmo);
+                            ok = mbar_wait(&bar.p_ready[t], j & 1, abort, tmo);
                             tc_fence_after();
                             if (!ok) break;
-                            issue_pv(t, sv, j % NB, j > 0);
-                            if (NB > 1) {
-                                mma_commit(&bar.pv_done[t]);
-                            } else if (jn < T.n) {
+                            issue_pv(t, sv, j > 0);
+                            if (jn < T.n) {
                                 const int sk = jn % NSK;
                                 if (t == 0) {
                                     ok = mbar_wait(&kready[sk], (jn / NSK) & 1, abort, tmo);
                                     tc_fence_after();
                                     if (!ok) break;
                                 }
-                                issue_s(t, sk, jn % NB);
-                                mma_commit(&bar.s_ready[t][jn % NB]);
+                                issue_s(t, sk);
+                                mma_commit(&bar.s_ready[t]);
                             }
                         }
-                        // Two S buffers: both PVs of tile j go first and release their
-                        // V stage, so a key tile that is still being rotated holds back
-                        // only the S products.
-                        if (NB > 1 && ok) {
-                            mma_commit(&bar.empty_v[sv]);
-                            if (jn < T.n) {
-                                const int sk = jn % NSK;
-                                ok = mbar_wait(&kready[sk], (jn / NSK) & 1, abort, tmo);
-                                tc_fence_after();
-                                for (int t = 0; ok && t < U.nt; ++t) {
-                                    issue_s(t, sk, jn % NB);
-                                    mma_commit(&bar.s_ready[t][jn % NB]);
-                                }
-                                if (ok) mma_commit(&bar.empty_k[sk]);
-                            }
-                        } else if (ok) {
+                        if (ok) {
                             mma_commit(&bar.empty_v[sv]);
                             if (jn < T.n) mma_commit(&bar.empty_k[jn % NSK]);
                         }
@@ -1013,7 +1022,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                               p.pack_lp, p.pack_stride,
                                                               t * p.pack_off, U.hpt, ph, p, rotq);
                     else
-                        rotate_tile_bf16<D, RD, kHalf, kSplit, kBM>(
+                        rotate_tile_bf16<D, RD, kHalf, kSplit, false, kBM>(
                             qt, qt + C::kTileQ, (long long)U.tq0(t) + p.qoff, ph, p, rotq);
                 }
         } else {
@@ -1021,17 +1030,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float *base = reinterpret_cast<const float *>(p.q) + U.b * p.qs[0] +
                                     (long long)U.th(t) * p.qs[1];
                 uint8_t *qt = sQ + t * C::kParts * C::kTileQ;
-                load_tile_f32<D, kHalf, kSplit, kBM>(qt, qt + C::kTileQ, base, p.qs[2], U.tq0(t),
-                                                     p.L, (long long)U.tq0(t) + p.qoff, rotq, ph,
-                                                     p);
+                load_tile_f32<D, kHalf, kSplit, false, kBM>(qt, qt + C::kTileQ, base, p.qs[2],
+                                                            U.tq0(t), p.L,
+                                                            (long long)U.tq0(t) + p.qoff, rotq,
+                                                            ph, p);
             }
         }
         if (ok) {
             fence_proxy_async_smem();
             mbar_arrive(&bar.ready_q);
         }
-        // bf16 keys that are already rotated go straight from the TMA to the MMA
-        const bool relay_k = kF32 || (kSplit && !p.k_lo_tma) || rotk;
+        // bf16 keys that are already rotated (and, split, already in parts) go
+        // straight from the TMA to the MMA
+        bool relay_k = kF32 || (kSplit && !p.k_x8_tma) || rotk;
+        if constexpr (kKvSplit && !kF32) {
+            if (ok && p.rot_help) {
+                rotate_keys_helped<D, RD, kHalf, kSplit, NSK, BN, C::kParts, C::kTileK>(
+                    tw, T, sK, bar, p, abort, tmo);
+                relay_k = false;
+            }
+        }
         for (int j = 0; ok && relay_k && j < T.n; ++j) {
             const int jt = T.tile(j);
             const int s = j % NSK, use = j / NSK, sv = j % NSV, usev = j / NSV;
@@ -1040,8 +1058,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_k[s], use & 1, abort, tmo));
                 if (!ok) break;
                 if (rotk || kSplit)
-                    rotate_tile_bf16<D, RD, kHalf, kSplit, BN, C::kKBoxStride>(
-                        tk + C::kKHi, tk + C::kKLo, (long long)jt * BN, ph, p, rotk, &kcarry);
+                    rotate_tile_bf16<D, RD, kHalf, kSplit, true, BN>(
+                        tk, tk + C::kTileK, (long long)jt * BN, ph, p, rotk, &kcarry);
             } else {
                 if (use > 0)
                     ok = __all_sync(0xffffffffu,
@@ -1049,9 +1067,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 const float *base = reinterpret_cast<const float *>(p.k) + U.b * p.ks[0] +
                                     (long long)U.g * p.ks[1];
-                load_tile_f32<D, kHalf, kSplit, BN, C::kKBoxStride>(
-                    tk + C::kKHi, tk + C::kKLo, base, p.ks[2], jt * BN, p.Lk, (long long)jt * BN,
-                    rotk, ph, p);
+                load_tile_f32<D, kHalf, kSplit, true, BN>(tk, tk + C::kTileK, base, p.ks[2],
+                                                          jt * BN, p.Lk, (long long)jt * BN,
+                                                          rotk, ph, p);
             }
             fence_proxy_async_smem();
             mbar_arrive(&bar.ready_k[s]);
@@ -1069,42 +1087,57 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         setmaxnreg_inc<kRegsSoftmax>();
-        if ((warp >> 2) < U.nt) {
-            // ------------------------------------------------ softmax, tile t
-            const int t = warp >> 2;
-            const int wq = warp & 3;
-            const int row = wq * 32 + lane;
-            const uint32_t trow = tmem + (uint32_t(wq * 32) << 16);
-            const uint32_t o_col = C::kColO + t * DV;
-            constexpr int NB = C::kNB;
-            const RowMap rm = map_row(p, U, t, row, packed);
-            const int pi = rm.i + p.qoff;  // this row's query position
-            const int tq0 = U.tq0(t);      // the tile's first query row
+        if (kKvSplit && !kF32 && ((p.rot_help >> warp) & 1)) {
+            // a softmax warp whose rows hold no query: it helps rotate key tiles
+            const int ord = __popc(p.rot_help & ((1u << warp) - 1u));
+            rotate_keys_helped<D, RD, kHalf, kSplit, NSK, BN, C::kParts, C::kTileK>(
+                128 + 32 * ord + lane, T, sK, bar, p, abort, tmo);
+        } else {
+            // ------------------------------------------------ softmax
+            // All eight softmax warps work on one query tile at a time, two
+            // threads per row: warp w takes rows 32 (w % 4) + 16 (w / 4) ..
+            // + 15 of every query tile (TMEM lanes of its quadrant), its lanes
+            // 0-15 the first half of those rows' columns (keys of S, output
+            // dims of O) and lanes 16-31 the second half.  The row max and sum
+            // combine with one shuffle.  The tiles alternate in the order the
+            // MMA warp produces them (S_0(j), S_1(j), S_0(j + 1), ...), so one
+            // tile's softmax runs at the full width of the SM while the tensor
+            // core works on the other tile.
+            const int hf = lane >> 4;                        // column half
+            const int row = (warp & 3) * 32 + (warp >> 2) * 16 + (lane & 15);
+            const uint32_t tlane = uint32_t((warp & 3) * 32 + (warp >> 2) * 16) << 16;
             const float cl2 = p.c_log2;
-            float m = -INFINITY, l = 0.f;
+            constexpr int HB = BN / 2;                       // keys per thread
+            // Interleaved key tiles (head-packed split-KV): tile t takes the key
+            // tiles j = t mod 2 of the split and writes partial 2 split + t.
+            const bool ilv = kKvSplit && p.pack_ilv;
+            const int nt = U.nt;
+            // per-tile state in scalars (t is a run-time index: arrays would live
+            // in local memory)
+            const RowMap rm0 = map_row(p, U, 0, row, packed);
+            const RowMap rm1 = map_row(p, U, nt > 1 ? 1 : 0, row, packed);
+            float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+            // Split-KV (decode) tiles hold few queries: a warp whose rows of the
+            // tile hold none only keeps step with the barriers (its P rows are
+            // never used: their O rows are not stored).
+            const bool idle0 = kKvSplit && !__any_sync(0xffffffffu, rm0.valid);
+            const bool idle1 = kKvSplit && !__any_sync(0xffffffffu, rm1.valid);
             bool ok = true;
-            // Split-KV (decode) tiles hold few queries: a warp whose 32 rows hold
-            // none only keeps step with the barriers, which leaves its SMSP to the
-            // rotation warp (its P rows are never used: their O rows are not stored).
-            const bool idle = kKvSplit && !__any_sync(0xffffffffu, rm.valid);
-            // Interleaved key tiles (head-packed split-KV): this tile takes the
-            // key tiles j = t mod 2 of the split and writes partial 2 split + t.
-            const bool ilv = kKvSplit && NB == 1 && p.pack_ilv;
-            const int n_it = ilv ? (T.n - t + 1) / 2 : T.n;
-            for (int it = 0; it < n_it; ++it) {
-                const int j = ilv ? 2 * it + t : it;
-                const int b = it % NB;
-                const uint32_t s_col = (t * NB + b) * C::kSCols;
-                ok = __all_sync(0xffffffffu,
-                                mbar_wait(&bar.s_ready[t][b], (it / NB) & 1, abort, tmo));
+            const int n_steps = ilv ? T.n : T.n * nt;
+            for (int k = 0; k < n_steps; ++k) {
+                const int t = ilv ? (k & 1) : (k % nt);
+                const int j = ilv ? k : k / nt;               // key tile of the list
+                const int it = ilv ? (k >> 1) : j;            // the tile's own step count
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_ready[t], it & 1, abort, tmo));
                 if (!ok) break;
-                if (idle) {
-                    mbar_arrive(&bar.p_ready[t][b]);
+                if (t ? idle1 : idle0) {
+                    mbar_arrive(&bar.p_ready[t]);
                     continue;
                 }
                 tc_fence_after();
-                const int jt = T.tile(j), k0 = jt * BN;
-                const bool partial = !tile_full<BN>(tq0, jt, p);
+                const int jt = T.tile(j), k0 = jt * BN + hf * HB;   // this thread's first key
+                const bool partial = !tile_full<BN>(U.tq0(t), jt, p);
+                const int pi = (t ? rm1.i : rm0.i) + p.qoff;   // this row's query position
                 // visible columns: col <= hi and (no window or col >= lo or col < sk)
                 const int hi = p.causal ? min(pi - k0, p.Lk - 1 - k0) : p.Lk - 1 - k0;
                 const int lo = pi - p.window + 1 - k0;
@@ -1112,62 +1145,52 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool win = p.causal && p.window > 0;
                 auto vis = [&](int col) { return col <= hi && (!win || col >= lo || col < sk); };
 
-                // The whole S row of this thread in one TMEM load.
-                float v[BN];
-                if constexpr (C::kFused) {
-                    // columns [0, BN): Qhi Klo^T; [BN, 2 BN): Qhi Khi^T + Qlo Khi^T
-                    float w[2 * BN];
-                    tmem_ld_row(trow + s_col, w);
-    #pragma unroll
-                    for (int e = 0; e < BN; ++e) v[e] = w[e] + w[e + BN];
-                } else {
-                    tmem_ld_row(trow + s_col, v);
-                }
+                // This thread's half of its S row in one TMEM load.
+                const uint32_t trow = tmem + tlane + uint32_t(t * BN);
+                float v[HB];
+                tmem_ld16x2_64(trow, v);
                 if (partial) {
-    #pragma unroll
-                    for (int e = 0; e < BN; ++e)
+#pragma unroll
+                    for (int e = 0; e < HB; ++e)
                         if (!vis(e)) v[e] = -INFINITY;
                 }
-                const float mx = row_max(v);
-                const float m_new = fmaxf(m, mx * cl2);
+                const float mh = row_max(v);
+                const float mx = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 16));
+                float mt = t ? m1 : m0;
+                float lt = t ? l1 : l0;
+                const float m_new = fmaxf(mt, mx * cl2);
                 // Keep the old reference unless the max grew by more than 2^8: the
                 // result is exact either way, only O's rescale is saved.
-                const bool need = (m != -INFINITY) && (m_new > m + kRescaleLog2);
+                const bool need = (mt != -INFINITY) && (m_new > mt + kRescaleLog2);
                 if (__any_sync(0xffffffffu, need)) {
-                    if (NB > 1) {
-                        // O_t must not be in flight: wait for PV_t(j - 1), the j-th
-                        // completion of pv_done (S_t(j) done implies PV_t(j - 2) was,
-                        // and PV_t(j) needs this tile's P, so no other phase can be
-                        // pending).  With one S buffer, S_t(j) done implies it.
-                        ok = __all_sync(0xffffffffu,
-                                        mbar_wait(&bar.pv_done[t], (it - 1) & 1, abort, tmo));
-                        if (!ok) break;
-                        tc_fence_after();
-                    }
-                    const float alpha = need ? ex2_approx(m - m_new) : 1.f;
-    #pragma unroll 1
-                    for (int c = 0; c < DV / 32; ++c) {
+                    // O_t is not in flight: S_t(j) is issued after PV_t(j - 1), so
+                    // its completion implies PV_t(j - 1)'s.  Each thread rescales its
+                    // half of the row's output dims (32-column chunks 2c + hf).
+                    const float alpha = need ? ex2_approx(mt - m_new) : 1.f;
+                    const uint32_t orow = tmem + tlane + uint32_t(C::kColO + t * DV);
+#pragma unroll 1
+                    for (int c = 0; c < DV / 64; ++c) {
                         float o[32];
-                        tmem_ld32(trow + o_col + c * 32, o);
+                        tmem_ld16x2_32(orow + c * 64, o);
                         uint32_t u[32];
-    #pragma unroll
+#pragma unroll
                         for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(o[e] * alpha);
-                        tmem_st32(trow + o_col + c * 32, u);
+                        tmem_st16x2_32(orow + c * 64, u);
                     }
                     if (need) {
-                        l *= alpha;
-                        m = m_new;
+                        lt *= alpha;
+                        mt = m_new;
                     }
                 }
-                if (m == -INFINITY) m = m_new;
-                const float mref = (m == -INFINITY) ? 0.f : m;
-                // P = 2^(s c - m) as bf16 pairs, written over the first half of S.
-                // One column pair in kEmuEvery takes 2^x on the FMA pipe.
+                if (mt == -INFINITY) mt = m_new;
+                const float mref = (mt == -INFINITY) ? 0.f : mt;
+                // P = 2^(s c - m) as bf16 pairs, written over the first half of S
+                // (this thread's 64 keys: P columns 32 hf .. 32 hf + 31).
                 const float2 c2 = make_float2(cl2, cl2), nm2 = make_float2(-mref, -mref);
                 float2 lsum = make_float2(0.f, 0.f);
-                uint32_t pk[BN / 2];
-    #pragma unroll
-                for (int e = 0; e < BN / 2; ++e) {
+                uint32_t pk[HB / 2];
+#pragma unroll
+                for (int e = 0; e < HB / 2; ++e) {
                     const float2 x = fma2(make_float2(v[2 * e], v[2 * e + 1]), c2, nm2);
                     float2 pe;
                     if (kEmuEvery > 0 && (e % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1)
@@ -1185,33 +1208,46 @@ __global__ void __launch_bounds__(kThreads, 1)
                         lsum = add2(lsum, pe);
                     }
                 }
-                tmem_st_row(trow + s_col, pk);
-                l += lsum.x + lsum.y;
+                tmem_st16x2_32(tmem + tlane + uint32_t(t * BN), pk);
+                lt += lsum.x + lsum.y;
+                if (t) {
+                    m1 = mt;
+                    l1 = lt;
+                } else {
+                    m0 = mt;
+                    l0 = lt;
+                }
                 tc_fence_before();
-                mbar_arrive(&bar.p_ready[t][b]);
+                mbar_arrive(&bar.p_ready[t]);
             }
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.o_ready[t], 0, abort, tmo));
-            if (ok) {
+            for (int t = 0; ok && t < nt; ++t) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar.o_ready[t], 0, abort, tmo));
+                if (!ok) break;
                 tc_fence_after();
-                const float inv = l > 0.f ? 1.f / l : 0.f;
+                const RowMap rm = t ? rm1 : rm0;
+                const float lh = t ? l1 : l0, mt = t ? m1 : m0;
+                const float lt = lh + __shfl_xor_sync(0xffffffffu, lh, 16);   // the row's sum
+                const float inv = lt > 0.f ? 1.f / lt : 0.f;
                 const int slot = ilv ? 2 * U.split + t : U.split;
-    #pragma unroll 1
-                for (int c = 0; c < DV / 32; ++c) {
+                const int n_it = ilv ? (T.n - t + 1) / 2 : T.n;
+                const uint32_t orow = tmem + tlane + uint32_t(C::kColO + t * DV);
+#pragma unroll 1
+                for (int c = 0; c < DV / 64; ++c) {
                     float v[32];
                     if (n_it > 0) {
-                        tmem_ld32(trow + o_col + c * 32, v);
+                        tmem_ld16x2_32(orow + c * 64, v);
                     } else {
                         // no key tile reached this tile: O_t was never written
-    #pragma unroll
+#pragma unroll
                         for (int e = 0; e < 32; ++e) v[e] = 0.f;
                     }
                     if (rm.valid)
-                        store_o32<DV, kF32, kKvSplit>(p, U, slot, rm.h, rm.i, c, v, inv);
+                        store_o32<DV, kF32, kKvSplit>(p, U, slot, rm.h, rm.i, 2 * c + hf, v, inv);
                 }
-                if (rm.valid) {
+                if (rm.valid && hf == 0) {
                     const float ln2 = 0.69314718055994531f;
                     store_lse<kKvSplit>(p, U, slot, rm.h, rm.i,
-                                        l > 0.f ? (m + __log2f(l)) * ln2 : -INFINITY);
+                                        lt > 0.f ? (mt + __log2f(lt)) * ln2 : -INFINITY);
                 }
             }
         }
@@ -1245,17 +1281,21 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [B, H, L, D] bf16 tensor -> 4-D tensor map with 64 x box_rows boxes, 128-byte swizzle.
+// [B, H, L, D] tensor of es-byte elements (2: bf16 or fp16 bits, 1: bytes) ->
+// 4-D tensor map whose boxes are 128 bytes (64 or 128 elements) x box_rows,
+// 128-byte swizzle.  TMA copies the bits; it never converts them.
 lcx_status make_map(CUtensorMap *map, const void *ptr, int64_t B, int64_t H, int64_t L, int64_t D,
-                    const int64_t *st, uint32_t box_rows, const char *name) {
+                    const int64_t *st, uint32_t box_rows, const char *name, int es = 2) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(LCX_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(L), cuuint64_t(H), cuuint64_t(B)};
-    cuuint64_t strides[3] = {cuuint64_t(st[2] * 2), cuuint64_t(st[1] * 2), cuuint64_t(st[0] * 2)};
-    cuuint32_t box[4] = {64, box_rows, 1, 1};
+    cuuint64_t strides[3] = {cuuint64_t(st[2] * es), cuuint64_t(st[1] * es),
+                             cuuint64_t(st[0] * es)};
+    cuuint32_t box[4] = {cuuint32_t(128 / es), box_rows, 1, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    CUresult r = fn(map, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                    4, const_cast<void *>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         return fail(LCX_ERR_UNSUPPORTED, "tensor map for %s rejected (CUresult %d)", name, int(r));
@@ -1360,7 +1400,7 @@ struct AttnLaunch : AttnLaunchShape {
     lcx_rope_params rope;
     const void *k_src;
     int64_t k_src_strides[4];
-    void *k_lo;       // split mode: where the pass writes the keys' lo parts, or NULL
+    void *k_x8;       // split mode: where the pass writes the keys' 8-bit cross parts, or NULL
     int rot_h, rot_d; // heads and columns the pass rotates (Hkv, D; or 1, d_R)
     void *k_rot;      // where the pass writes
 };
@@ -1436,31 +1476,32 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     // instead of once per key tile per CTA, where the kernel would otherwise
     // rotate them on chip: full-rotary keys ([B, Hkv, Lk, D]), or the shared
     // rotary key of decoupled RoPE ([B, 1, Lk, d_R]; k keeps its un-rotated
-    // columns).  In the split-QK^T mode with bf16 keys the pass also writes
-    // the lo parts (bf16 of the rounding residual) right after the hi parts.
+    // columns).  In the split-QK^T mode with bf16 keys the pass writes the
+    // keys' fp16 parts there, followed by their 8-bit cross parts ([r8 | h8],
+    // 2 D bytes per key: as many bytes again).
     const bool rot_shared = partial && a->k_rope != nullptr;
     const bool rotate_k_once =
         a->k_rot != nullptr && !(a->flags & (LCX_ATTN_PREROTATED | LCX_ATTN_PREROTATED_K |
                                              LCX_ATTN_TEST_STALL)) &&
         ((!partial && !a->k_rope && a->D % 16 == 0) || rot_shared);
-    const bool k_lo = rotate_k_once && (a->flags & LCX_ATTN_SPLIT_QK) && a->dtype == LCX_BF16;
+    const bool k_x8 = rotate_k_once && (a->flags & LCX_ATTN_SPLIT_QK) && a->dtype == LCX_BF16;
     const int64_t rot_h = rot_shared ? 1 : a->Hkv, rot_d = rot_shared ? RD : a->D;
     const int64_t kst_rot[4] = {rot_h * Lk * rot_d, Lk * rot_d, rot_d, 1};
     const int64_t k_part_bytes = a->B * rot_h * Lk * rot_d * es;
     if (rotate_k_once) {
         if (!aligned16(a->k_rot)) return fail(LCX_ERR_UNSUPPORTED, "k_rot must be 16-byte aligned");
-        if (a->k_rot_bytes < k_part_bytes * (k_lo ? 2 : 1))
+        if (a->k_rot_bytes < k_part_bytes * (k_x8 ? 2 : 1))
             return fail(LCX_ERR_INVALID_ARG, "k_rot holds %lld bytes; %lld needed",
-                        (long long)a->k_rot_bytes, (long long)(k_part_bytes * (k_lo ? 2 : 1)));
+                        (long long)a->k_rot_bytes, (long long)(k_part_bytes * (k_x8 ? 2 : 1)));
     }
-    void *k_lo_ptr = k_lo ? static_cast<char *>(a->k_rot) + k_part_bytes : nullptr;
+    void *k_x8_ptr = k_x8 ? static_cast<char *>(a->k_rot) + k_part_bytes : nullptr;
     const bool k_from_rot = rotate_k_once && !rot_shared;   // k itself read from k_rot
     const void *kptr = k_from_rot ? a->k_rot : a->k;
     const int64_t *kst = k_from_rot ? kst_rot : a->k_strides;
 
     memset(&x, 0, sizeof(x));
     x.rotate_k_once = rotate_k_once;
-    x.k_lo = k_lo_ptr;
+    x.k_x8 = k_x8_ptr;
     x.rope = a->rope;
     x.k_src = rot_shared ? a->k_rope : a->k;
     for (int d = 0; d < 4; ++d)
@@ -1523,7 +1564,7 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     }
     p.c_log2 = float(scale * msq * 1.4426950408889634);
     p.k_rope_shared = a->k_rope ? 1 : 0;
-    p.k_lo_tma = k_lo ? 1 : 0;
+    p.k_x8_tma = k_x8 ? 1 : 0;
     // Legitimate waits last microseconds; the default limit is 2 s.
     p.timeout_ns = 1000000ull * (unsigned long long)(a->watchdog_ms > 0 ? a->watchdog_ms : 2000);
     p.test_stall = (a->flags & LCX_ATTN_TEST_STALL) ? 1 : 0;
@@ -1536,11 +1577,12 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     x.RD = int(RD);
     // K/V boxes are one key tile high: the kernel's expect-tx byte counts and
     // stage layout assume exactly Cfg::BN rows per box.
-    const uint32_t bn = x.split_qk ? uint32_t(Cfg<64, 64, true>::BN) : uint32_t(Cfg<64, 64, false>::BN);
-    static_assert(Cfg<64, 64, true>::BN == Cfg<128, 128, true>::BN &&
-                      Cfg<64, 64, false>::BN == Cfg<128, 128, false>::BN &&
-                      Cfg<64, 64, false>::BN == Cfg<192, 128, false>::BN,
-                  "one key-tile height per QK^T mode");
+    const uint32_t bn = uint32_t(Cfg<64, 64, false>::BN);
+    static_assert(Cfg<64, 64, true>::BN == Cfg<64, 64, false>::BN &&
+                      Cfg<128, 128, true>::BN == Cfg<64, 64, false>::BN &&
+                      Cfg<128, 128, false>::BN == Cfg<64, 64, false>::BN &&
+                      Cfg<192, 128, false>::BN == Cfg<64, 64, false>::BN,
+                  "one key-tile height for every kernel instance");
     if (!x.f32) {
         const int64_t dk = a->k_rope ? a->D - RD : a->D;   // columns k itself holds
         if ((st = make_map(&x.m.q, a->q, a->B, a->Hq, a->L, a->D, a->q_strides, 128, "q")) != LCX_OK)
@@ -1549,9 +1591,12 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
             return st;
         if ((st = make_map(&x.m.v, a->v, a->B, a->Hkv, Lk, Dv, a->v_strides, bn, "v")) != LCX_OK)
             return st;
-        if (k_lo) {
-            if ((st = make_map(&x.m.kr, k_lo_ptr, a->B, a->Hkv, Lk, a->D, kst_rot, bn, "k_lo")) !=
-                LCX_OK)
+        if (k_x8) {
+            // the keys' 8-bit cross parts: [B, Hkv, Lk, 2 D] bytes, boxes of
+            // 128 bytes x one key tile
+            const int64_t bst[4] = {kst_rot[0] * 2, kst_rot[1] * 2, kst_rot[2] * 2, 1};
+            if ((st = make_map(&x.m.kr, k_x8_ptr, a->B, a->Hkv, Lk, 2 * a->D, bst, bn, "k_x8",
+                               1)) != LCX_OK)
                 return st;
         }
         if (a->k_rope) {
@@ -1581,7 +1626,7 @@ lcx_status attn_enqueue(const AttnLaunch &x, cudaStream_t s) {
         const int64_t kst[4] = {(int64_t)x.rot_h * x.p.Lk * x.rot_d, (int64_t)x.p.Lk * x.rot_d,
                                 x.rot_d, 1};
         const lcx_status st =
-            apply_rope_impl(&rp, x.k_src, x.k_rot, x.k_lo, x.f32 ? LCX_F32 : LCX_BF16, x.p.B,
+            apply_rope_impl(&rp, x.k_src, x.k_rot, x.k_x8, x.f32 ? LCX_F32 : LCX_BF16, x.p.B,
                             x.rot_h, x.p.Lk, x.k_src_strides, kst, 0, s);
         if (st != LCX_OK) return st;
     }
@@ -1657,18 +1702,17 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
     // the G heads of a kv group share the CTA's query tiles (pack_lp rows per
     // head: L rounded up to 8 rows), so every K/V tile is read and rotated once
     // per kv group instead of once per head pair.
-    //  - bf16, one S buffer per query tile (plain QK^T, or split QK^T with its
-    //    products fused), G pack_lp <= 128: both tiles hold all G heads (rows
+    //  - bf16, G pack_lp <= 128: both tiles hold all G heads (rows
     //    [0, G pack_lp), tile 1 shifted by whole warps when that fits, so the
     //    busy softmax warps of the two tiles use different SMSPs) and tile t
     //    takes the key tiles j = t mod 2: two K/V tiles in flight per CTA, two
     //    partial results per split.
-    //  - otherwise (fp32, unfused split QK^T, G pack_lp > 128), G even and
+    //  - otherwise (fp32, or G pack_lp > 128), G even and
     //    G/2 pack_lp <= 128: G/2 heads per tile, both tiles multiply every key
     //    tile.
     const int64_t lp = (a->L + 7) / 8 * 8;
     int n_parts = num_splits;
-    if (!x.f32 && (!x.split_qk || LCX_SPLIT_FUSED) && x.D <= 128 && lp * x.p.G <= kBM) {
+    if (!x.f32 && x.D <= 128 && lp * x.p.G <= kBM) {
         const int used = int(lp) * x.p.G;
         x.p.pack_lp = int(lp);
         x.p.pack_hpt = x.p.G;
@@ -1677,6 +1721,27 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
         if (x.p.pack_off + used > kBM) x.p.pack_off = 0;
         x.p.pack_ilv = 1;
         n_parts = 2 * num_splits;
+        // Keys rotated on chip: softmax warps whose 16 rows hold no query in
+        // either tile (warp w: rows 32 (w % 4) + 16 (w / 4) .. + 15) rotate key
+        // tiles beside warps 8-11 (four of them, which halves each thread's
+        // rows; with fewer idle warps nobody helps).
+        if (x.p.rotate_k) {
+            int mask = 0, n = 0;
+            for (int w = 0; w < 8 && n < 4; ++w) {
+                bool any = false;
+                const int r0 = 32 * (w % 4) + 16 * (w / 4);
+                for (int t = 0; t < 2 && !any; ++t)
+                    for (int r = r0; r < r0 + 16 && !any; ++r) {
+                        const int rel = r - t * x.p.pack_off;
+                        any = rel >= 0 && rel < used && rel % x.p.pack_stride < a->L;
+                    }
+                if (!any) {
+                    mask |= 1 << w;
+                    ++n;
+                }
+            }
+            x.p.rot_help = n == 4 ? mask : 0;
+        }
     } else if (!x.f32 && x.p.G % 2 == 0 && x.D <= 128 && lp * (x.p.G / 2) <= kBM) {
         x.p.pack_lp = int(lp);
         x.p.pack_hpt = x.p.G / 2;

@@ -32,9 +32,11 @@ inline int64_t effective_seq_len(const lcx_rope_params *p, int64_t call_len) {
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// The rotate pass of lcx_apply_rope (argument checks included), optionally also
-// writing y_lo = bf16(y' - bf16(y')) (bf16 only; same strides as y; NULL = none).
-lcx_status apply_rope_impl(const lcx_rope_params *params, const void *x, void *y, void *y_lo,
+// The rotate pass of lcx_apply_rope (argument checks included).  With y_x8
+// (bf16 x only, NULL = none) it writes the split-QK^T key parts instead: y the
+// fp16 parts h = f16(y'), and y_x8, a row of 2 D bytes per (b, h, l) starting at
+// twice y's element offset, the e5m2 bytes of y' - h then those of h.
+lcx_status apply_rope_impl(const lcx_rope_params *params, const void *x, void *y, void *y_x8,
                            int32_t dtype, int64_t B, int64_t H, int64_t L,
                            const int64_t *x_strides, const int64_t *y_strides, int64_t pos_offset,
                            cudaStream_t stream);

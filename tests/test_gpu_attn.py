@@ -300,7 +300,7 @@ def test_attn_fwd_host_pipelined_equals_device_call(chunks, extra):
 def test_attn_rotate_keys_once(name):
     """Keys rotated once into a buffer by the rotate pass (args.k_rot) before
     the kernel, instead of per key tile on chip: same parity.  Split-QK^T cases
-    with bf16 keys get hi/lo parts from the pass (loaded by TMA); with fp32
+    with bf16 keys get fp16 and 8-bit cross parts from the pass (loaded by TMA); with fp32
     keys the kernel splits the pre-rotated fp32 values itself."""
     full_check(BASE.with_(**SMALL[name]), rotate_k_once=True)
 

@@ -121,7 +121,7 @@ def test_merge_matches_oracle(D, dtype):
     (1, 8, 2, dict(pairing="interleaved")),
     (8, 16, 1, {}),                                  # G = 16: 8 heads x 8 rows
     (2, 6, 1, dict(mode="ntk", scale=4.0)),          # G = 6: 3 heads per tile
-    (5, 4, 2, dict(split_qk=True, D=64)),            # hi/lo parts, D = 64
+    (5, 4, 2, dict(split_qk=True, D=64)),            # split parts, D = 64
 ])
 def test_splitkv_head_packed_decode(L, Hq, Hkv, extra):
     """Few queries per head: the kv group's heads share the two query tiles
@@ -144,8 +144,8 @@ def test_splitkv_head_packed_decode(L, Hq, Hkv, extra):
     (1, 1500, 5, dict(Hq=2, Hkv=2)),                 # G = 1
     (4, 3000, 6, dict(Hq=8, Hkv=2, window=700, sinks=4)),
     (1, 2000, 4, dict(Hq=8, Hkv=2, k_prerotated=True)),
-    # split QK^T (64-key tiles, fused products): odd counts, one tile per split,
-    # keys split by the rotate pass
+    # split QK^T: odd counts, one tile per split, keys split into their parts by
+    # the rotate pass
     (1, 1800, 2, dict(Hq=8, Hkv=2, split_qk=True)),
     (2, 777, 13, dict(Hq=6, Hkv=2, split_qk=True)),
     (3, 2000, 5, dict(Hq=8, Hkv=2, split_qk=True, rotate_k_once=True)),
@@ -153,7 +153,9 @@ def test_splitkv_head_packed_decode(L, Hq, Hkv, extra):
 def test_splitkv_interleaved_key_tiles(L, Lk, splits, extra):
     """bf16 head-packed split-KV: both query tiles hold all G heads and take
     alternate key tiles of the split (two partial results per split); every
-    head's rows against the oracle, edge counts of key tiles included."""
+    head's rows against the oracle, edge counts of key tiles included.  With
+    keys rotated on chip and G L <= 32, four softmax warps that hold no query
+    help rotate the key tiles (256 rotating threads)."""
     extra = dict(extra)
     prerot = extra.pop("k_prerotated", False)
     once = extra.pop("rotate_k_once", False)

@@ -38,7 +38,7 @@ class Workload:
     softmax_scale: float = 0.0  # 0 -> 1/sqrt(D)
     outlier_frac: float = 0.0
     outlier_mult: float = 8.0
-    split_qk: bool = False     # form QK^T from hi/lo bf16 parts (outlier-heavy inputs)
+    split_qk: bool = False     # form QK^T from fp16 + e5m2 cross parts (outlier-heavy inputs)
     seed: int = 0
     description: str = ""
 
