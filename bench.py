@@ -234,6 +234,8 @@ def _row_visible(w, i):
 def bench_gpu(args, world, rank, local):
     import ntk_rope_flashattn_b200 as lcx
     w = WORKLOADS[args.workload]
+    if args.batch > 0:
+        w = w.with_(B=args.batch)
     dev = torch.device("cuda", local)
     q, k, v = make_inputs(w, device=dev, seed=rank_seed(w, rank, args.shard))
     g0, g1 = 0, w.Hkv
@@ -733,6 +735,9 @@ def main():
                     help="skip the per-workload measurements (the configs object)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip decode, decoupled-RoPE and per-workload measurements")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch size (smaller captures for profiling; "
+                         "the line's config records it)")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="N > 1: independent replicas (weak scaling) or one batch split by "
                          "kv heads (strong scaling)")

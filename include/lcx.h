@@ -253,8 +253,10 @@ typedef struct {
  *   Arithmetic: q', k' rounded to bf16 on chip (split mode: an fp16 part
  *   and e5m2 cross parts, see LCX_ATTN_SPLIT_QK), QK^T and PV on tensor cores
  *   with fp32 accumulation, P rounded to bf16 for PV, softmax statistics in
- *   fp32, o rounded once to the output dtype.  fp32 inputs are rounded to
- *   bf16 operands.
+ *   fp32, o rounded once to the output dtype.  fp32 inputs at D = 64 keep
+ *   32-bit operands: q', k', v and P rounded to tf32 (10-bit mantissa) for
+ *   tf32 tensor-core products; at D = 128 (and in the split mode) fp32 inputs
+ *   are rounded to the 16-bit operands above.
  *   Supported (D, Dv, rope.head_dim): (64, 64, 64), (128, 128, 128) with bf16
  *   or fp32 and either QK^T mode; (128, 128, 64) and (192, 128, 64) with bf16
  *   and plain QK^T.  Pointers 16-byte aligned, strides multiples of 16 bytes,

@@ -142,21 +142,29 @@ struct AttnParams {
 // size of a 16-bit part, stored as D/64 boxes of 128-byte rows ([h8 | r8] for
 // a query row, [r8 | h8] for a key row).  Key tiles stay 128 rows; at D = 128
 // the parts fill shared memory with one K stage (64 KB) and one V stage.
-template <int D, int DV, bool kSplit>
+//
+// tf32 operands (fp32 inputs at D = 64): Q, K and V tiles hold fp32 values
+// rounded to tf32, 32 per 128-byte row of a box (2 boxes per row at D = 64);
+// P is written to TMEM as fp32 over the whole S buffer.  Two K and two V
+// stages of 32 KB beside two 32 KB query tiles.
+template <int D, int DV, bool kSplit, bool kTF = false>
 struct Cfg {
     static constexpr int BN = 128;                      // keys per tile
+    static constexpr int ES = kTF ? 4 : 2;              // bytes per operand element
     static constexpr int kParts = kSplit ? 2 : 1;       // 16-bit part (+ 8-bit cross part)
     static constexpr int kNTQ = (D > 128 && !LCX_D192_TWO_TILES) ? 1 : 2;  // query tiles per CTA
-    static constexpr int kTileQ = kBM * D * 2;          // one part of a Q tile
-    static constexpr int kTileK = BN * D * 2;           // one part of a K tile
-    static constexpr int kTileV = BN * DV * 2;          // a V tile
+    static constexpr int kTileQ = kBM * D * ES;         // one part of a Q tile
+    static constexpr int kTileK = BN * D * ES;          // one part of a K tile
+    static constexpr int kTileV = BN * DV * ES;         // a V tile
     static constexpr int kBoxQ = kBM * 128;
     static constexpr int kBoxK = BN * 128;
+    static constexpr int kKSteps = D * ES / 32;         // QK^T instructions over D (32 bytes each)
     static constexpr int kStagesK = kSplit ? (D == 64 ? 3 : 1)
+                                  : kTF ? 2
                                   : (D == 64) ? 4
                                   : (D == 128) ? LCX_KSTAGES_D128
                                   : (kNTQ == 2) ? 1 : 2;
-    static constexpr int kStagesV = kSplit ? (D == 64 ? 3 : 1) : (D == 64) ? 4 : 2;
+    static constexpr int kStagesV = kSplit ? (D == 64 ? 3 : 1) : kTF ? 2 : (D == 64) ? 4 : 2;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kNTQ * kParts * kTileQ;
     static constexpr int kOffV = kOffK + kStagesK * kParts * kTileK;
@@ -335,9 +343,17 @@ __device__ __forceinline__ uint32_t byte_off(int r, int x, int box_bytes) {
 // row r.  Plain mode: bf16 into the tile.  Split mode: the fp16 part h into the
 // tile and, into the 8-bit cross part x8, e5m2(h) and e5m2(x' - h): a query row
 // holds [h8 | r8] (column c at bytes c and D + c), a key row [r8 | h8].
-template <bool kSplit, bool kKey, int D, int BOX>
+template <bool kSplit, bool kKey, int D, int BOX, bool kTF = false>
 __device__ __forceinline__ void store8(uint8_t *tile, uint8_t *x8, int r, int fc,
                                        const float (&y)[8]) {
+    if constexpr (kTF) {
+        // tf32 tile: the 8 values are two 16-byte chunks (columns 8 fc ..)
+        *reinterpret_cast<float4 *>(tile + chunk_off(r, 2 * fc, BOX)) =
+            make_float4(round_tf32(y[0]), round_tf32(y[1]), round_tf32(y[2]), round_tf32(y[3]));
+        *reinterpret_cast<float4 *>(tile + chunk_off(r, 2 * fc + 1, BOX)) =
+            make_float4(round_tf32(y[4]), round_tf32(y[5]), round_tf32(y[6]), round_tf32(y[7]));
+        return;
+    }
     const uint32_t off = chunk_off(r, fc, BOX);
     if constexpr (!kSplit) {
         *reinterpret_cast<uint4 *>(tile + off) = pack8(y);
@@ -526,8 +542,9 @@ __device__ __forceinline__ void rotate_tile_bf16(uint8_t *tile, uint8_t *lo, lon
 
 // fp32 operands: load ROWS rows from global (rows >= L read as zero), rotate in
 // fp32 when asked (row r at position pos0 + r), round to bf16 (split mode: the
-// fp16 part, and the 8-bit cross part into `lo`) into the tile.
-template <int D, bool kHalf, bool kSplit, bool kKey, int ROWS>
+// fp16 part, and the 8-bit cross part into `lo`; kTF: to tf32, kept in fp32)
+// into the tile.
+template <int D, bool kHalf, bool kSplit, bool kKey, int ROWS, bool kTF = false>
 __device__ __forceinline__ void load_tile_f32(uint8_t *tile, uint8_t *lo, const float *base,
                                               long long rs, int row0, int L, long long pos0,
                                               bool rotate, const Phasor<D, kHalf> &ph,
@@ -549,8 +566,8 @@ __device__ __forceinline__ void load_tile_f32(uint8_t *tile, uint8_t *lo, const 
                 x2[e] = valid ? src[ph.i0 + e + D / 2] : 0.f;
             }
             if (rotate) rot_pairs<8>(x1, x2, c, s);
-            store8<kSplit, kKey, D, BOX>(tile, lo, r, ph.q, x1);
-            store8<kSplit, kKey, D, BOX>(tile, lo, r, ph.q + D / 16, x2);
+            store8<kSplit, kKey, D, BOX, kTF>(tile, lo, r, ph.q, x1);
+            store8<kSplit, kKey, D, BOX, kTF>(tile, lo, r, ph.q + D / 16, x2);
         } else {
             float x[8];
 #pragma unroll
@@ -569,14 +586,14 @@ __device__ __forceinline__ void load_tile_f32(uint8_t *tile, uint8_t *lo, const 
                     x[2 * e + 1] = x2[e];
                 }
             }
-            store8<kSplit, kKey, D, BOX>(tile, lo, r, ph.q, x);
+            store8<kSplit, kKey, D, BOX, kTF>(tile, lo, r, ph.q, x);
         }
         if (rotate) ph.step(c, s);
     }
 }
 
-// fp32 V tile: convert only.
-template <int D, int ROWS>
+// fp32 V tile: convert only (to bf16, or with kTF round to tf32).
+template <int D, int ROWS, bool kTF = false>
 __device__ __forceinline__ void load_v_f32(uint8_t *tile, const float *base, long long rs, int row0,
                                            int L, int tw) {
     constexpr int CPR = D / 8;
@@ -588,7 +605,7 @@ __device__ __forceinline__ void load_v_f32(uint8_t *tile, const float *base, lon
         float x[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[e] = valid ? src[e] : 0.f;
-        *reinterpret_cast<uint4 *>(tile + chunk_off(r, fc, BOX)) = pack8(x);
+        store8<false, false, D, BOX, kTF>(tile, nullptr, r, fc, x);
     }
 }
 
@@ -715,7 +732,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv,
                     const __grid_constant__ CUtensorMap tmkr, const __grid_constant__ AttnParams p) {
-    using C = Cfg<D, DV, kSplit>;
+    // fp32 operands at D = 64 stay 32-bit (rounded to tf32) for kind::tf32
+    // products; at D = 128 two query tiles of them would not fit beside the
+    // K/V stages, so they are rounded to bf16 like the split mode's values.
+    constexpr bool kTF = kF32 && !kSplit && D == 64;
+    using C = Cfg<D, DV, kSplit, kTF>;
     static_assert(!kF32 || (RD == D && DV == D), "fp32 operands: full rotary, DV = D");
     static_assert(!kSplit || (RD == D && DV == D), "split QK^T: full rotary, DV = D");
     constexpr int NSK = C::kStagesK;
@@ -876,9 +897,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // S: bf16 (plain) or fp16 (split: the Qh Kh^T product) operands;
                 // the split mode's cross product takes e5m2 operands.
                 constexpr uint32_t kIdS = kSplit ? idesc_f32acc(128, BN, kFmtF16, kFmtF16, 0, 0)
-                                                 : idesc_bf16_f32(128, BN, 0, 0);
+                                          : kTF ? idesc_f32acc(128, BN, kFmtTF32, kFmtTF32, 0, 0)
+                                                : idesc_bf16_f32(128, BN, 0, 0);
                 constexpr uint32_t kIdX8 = idesc_f32acc(128, BN, kFmtE5M2, kFmtE5M2, 0, 0);
-                constexpr uint32_t kIdPV = idesc_bf16_f32(128, DV, 0, 1);
+                constexpr uint32_t kIdPV = kTF ? idesc_f32acc(128, DV, kFmtTF32, kFmtTF32, 0, 1)
+                                               : idesc_bf16_f32(128, DV, 0, 1);
                 const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
                 // S_t = Q_t K^T over D in steps of 16 (32 bytes inside a 128-byte
                 // swizzle row, then the next 64-column box).  Descriptors of the
@@ -904,20 +927,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
+                    for (int kk = 0; kk < C::kKSteps; ++kk) {
                         const uint32_t oq = ((kk >> 2) * C::kBoxQ + (kk & 3) * 32) >> 4;
                         const uint32_t ok_ = ((kk >> 2) * C::kBoxK + (kk & 3) * 32) >> 4;
-                        mma_ss(dst, qa + oq, ka + ok_, kIdS, kSplit || kk > 0);
+                        if constexpr (kTF)
+                            mma_ss_tf32(dst, qa + oq, ka + ok_, kIdS, kk > 0);
+                        else
+                            mma_ss(dst, qa + oq, ka + ok_, kIdS, kSplit || kk > 0);
                     }
                 };
-                // O_t += P_t V: P from TMEM (BN/2 columns of bf16 pairs), V MN-major.
+                // O_t += P_t V: P from TMEM (BN/2 columns of bf16 pairs, or BN of
+                // tf32), V MN-major; each instruction takes 32 bytes of keys per
+                // row of P (8 TMEM columns) and as many 128-byte rows of V.
                 auto issue_pv = [&](int t, int s, bool acc) {
                     const uint64_t va = dv0 + ((s * C::kTileV) >> 4);
                     const uint32_t dst = tmem + C::kColO + t * DV;
                     const uint32_t pa = tmem + t * BN;
+                    constexpr int KS = 32 / C::ES;   // keys per instruction
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk)
-                        mma_ts(dst, pa + kk * 8, va + ((kk * 2048) >> 4), kIdPV, (acc || kk > 0));
+                    for (int kk = 0; kk < BN / KS; ++kk) {
+                        if constexpr (kTF)
+                            mma_ts_tf32(dst, pa + kk * 8, va + ((kk * KS * 128) >> 4), kIdPV,
+                                        (acc || kk > 0));
+                        else
+                            mma_ts(dst, pa + kk * 8, va + ((kk * KS * 128) >> 4), kIdPV,
+                                   (acc || kk > 0));
+                    }
                 };
                 // S_t(j + 1) is issued after PV_t(j), into the buffer P_t(j)
                 // occupied (MMAs of one thread execute in order): the order is
@@ -1030,10 +1065,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float *base = reinterpret_cast<const float *>(p.q) + U.b * p.qs[0] +
                                     (long long)U.th(t) * p.qs[1];
                 uint8_t *qt = sQ + t * C::kParts * C::kTileQ;
-                load_tile_f32<D, kHalf, kSplit, false, kBM>(qt, qt + C::kTileQ, base, p.qs[2],
-                                                            U.tq0(t), p.L,
-                                                            (long long)U.tq0(t) + p.qoff, rotq,
-                                                            ph, p);
+                load_tile_f32<D, kHalf, kSplit, false, kBM, kTF>(qt, qt + C::kTileQ, base,
+                                                                 p.qs[2], U.tq0(t), p.L,
+                                                                 (long long)U.tq0(t) + p.qoff,
+                                                                 rotq, ph, p);
             }
         }
         if (ok) {
@@ -1067,9 +1102,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 const float *base = reinterpret_cast<const float *>(p.k) + U.b * p.ks[0] +
                                     (long long)U.g * p.ks[1];
-                load_tile_f32<D, kHalf, kSplit, true, BN>(tk, tk + C::kTileK, base, p.ks[2],
-                                                          jt * BN, p.Lk, (long long)jt * BN,
-                                                          rotk, ph, p);
+                load_tile_f32<D, kHalf, kSplit, true, BN, kTF>(tk, tk + C::kTileK, base,
+                                                               p.ks[2], jt * BN, p.Lk,
+                                                               (long long)jt * BN, rotk, ph, p);
             }
             fence_proxy_async_smem();
             mbar_arrive(&bar.ready_k[s]);
@@ -1080,7 +1115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 const float *base = reinterpret_cast<const float *>(p.v) + U.b * p.vs[0] +
                                     (long long)U.g * p.vs[1];
-                load_v_f32<D, BN>(sV + sv * C::kTileV, base, p.vs[2], jt * BN, p.Lk, tw);
+                load_v_f32<D, BN, kTF>(sV + sv * C::kTileV, base, p.vs[2], jt * BN, p.Lk, tw);
                 fence_proxy_async_smem();
                 mbar_arrive(&bar.full_v[sv]);
             }
@@ -1185,30 +1220,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (mt == -INFINITY) mt = m_new;
                 const float mref = (mt == -INFINITY) ? 0.f : mt;
                 // P = 2^(s c - m) as bf16 pairs, written over the first half of S
-                // (this thread's 64 keys: P columns 32 hf .. 32 hf + 31).
+                // (this thread's 64 keys: P columns 32 hf .. 32 hf + 31); tf32
+                // operands: as tf32 values over all of S (columns 64 hf ..).
                 const float2 c2 = make_float2(cl2, cl2), nm2 = make_float2(-mref, -mref);
                 float2 lsum = make_float2(0.f, 0.f);
-                uint32_t pk[HB / 2];
+                if constexpr (kTF) {
+                    uint32_t pw[HB];
 #pragma unroll
-                for (int e = 0; e < HB / 2; ++e) {
-                    const float2 x = fma2(make_float2(v[2 * e], v[2 * e + 1]), c2, nm2);
-                    float2 pe;
-                    if (kEmuEvery > 0 && (e % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1)
-                        pe = exp2_fma2(x);
-                    else
-                        pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-                    pk[e] = pack_bf16x2(pe.x, pe.y);
-                    if (kSplit) {
-                        // Normalise by the weights the tensor core actually
-                        // multiplies V with (bf16), not their fp32 values: with
-                        // the stale max reference the dominant weight is 2^d,
-                        // d in [0, 8], and its rounding must cancel in o.
-                        lsum = add2(lsum, make_float2(bf16lo_to_f32(pk[e]), bf16hi_to_f32(pk[e])));
-                    } else {
+                    for (int e = 0; e < HB / 2; ++e) {
+                        const float2 x = fma2(make_float2(v[2 * e], v[2 * e + 1]), c2, nm2);
+                        // the weights the tensor core multiplies V with (tf32), and
+                        // the normalisation by their sum
+                        const float2 pe = make_float2(round_tf32(ex2_approx(x.x)),
+                                                      round_tf32(ex2_approx(x.y)));
+                        pw[2 * e] = __float_as_uint(pe.x);
+                        pw[2 * e + 1] = __float_as_uint(pe.y);
                         lsum = add2(lsum, pe);
                     }
+                    tmem_st16x2_64(tmem + tlane + uint32_t(t * BN), pw);
+                } else {
+                    uint32_t pk[HB / 2];
+#pragma unroll
+                    for (int e = 0; e < HB / 2; ++e) {
+                        const float2 x = fma2(make_float2(v[2 * e], v[2 * e + 1]), c2, nm2);
+                        float2 pe;
+                        if (kEmuEvery > 0 && (e % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1)
+                            pe = exp2_fma2(x);
+                        else
+                            pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                        pk[e] = pack_bf16x2(pe.x, pe.y);
+                        if (kSplit) {
+                            // Normalise by the weights the tensor core actually
+                            // multiplies V with (bf16), not their fp32 values: with
+                            // the stale max reference the dominant weight is 2^d,
+                            // d in [0, 8], and its rounding must cancel in o.
+                            lsum = add2(lsum,
+                                        make_float2(bf16lo_to_f32(pk[e]), bf16hi_to_f32(pk[e])));
+                        } else {
+                            lsum = add2(lsum, pe);
+                        }
+                    }
+                    tmem_st16x2_32(tmem + tlane + uint32_t(t * BN), pk);
                 }
-                tmem_st16x2_32(tmem + tlane + uint32_t(t * BN), pk);
                 lt += lsum.x + lsum.y;
                 if (t) {
                     m1 = mt;
@@ -1317,7 +1370,7 @@ struct AttnLaunchShape {
 template <int D, int DV, int RD, bool kF32, bool kHalf, bool kSplit, bool kKvSplit>
 lcx_status launch(const Maps &m, const AttnParams &p, unsigned grid, cudaStream_t s) {
     auto kern = attn_fwd_kernel<D, DV, RD, kF32, kHalf, kSplit, kKvSplit>;
-    const int smem = Cfg<D, DV, kSplit>::kSmemBytes;
+    const int smem = Cfg<D, DV, kSplit, kF32 && !kSplit && D == 64>::kSmemBytes;
     // The warpgroups re-balance registers with setmaxnreg, which waits until the
     // registers it asks for are free: the launch must hold the whole split.
     static const int regs = []() {
