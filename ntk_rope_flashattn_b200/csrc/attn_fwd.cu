@@ -74,6 +74,11 @@ constexpr float kRescaleLog2 = 8.0f;    // rescale O only if the max grows by > 
 #ifndef LCX_ROT_UNROLL
 #define LCX_ROT_UNROLL 2
 #endif
+// LCX_SPLIT_P_F16: the split mode's PV takes P and V in fp16 (V converted in
+// shared memory) rather than bf16
+#ifndef LCX_SPLIT_P_F16
+#define LCX_SPLIT_P_F16 1
+#endif
 #ifndef LCX_PHASOR_CARRY
 #define LCX_PHASOR_CARRY 1
 #endif
@@ -181,7 +186,7 @@ template <int NSK, int NSV>
 struct Bars {
     uint64_t full_q, ready_q;
     uint64_t full_k[NSK], ready_k[NSK], empty_k[NSK];
-    uint64_t full_v[NSV], empty_v[NSV];
+    uint64_t full_v[NSV], empty_v[NSV], fp16_v[NSV];
     uint64_t s_ready[2], p_ready[2], o_ready[2];
     uint64_t drain;
     uint32_t tmem_base;
@@ -592,10 +597,47 @@ __device__ __forceinline__ void load_tile_f32(uint8_t *tile, uint8_t *lo, const 
     }
 }
 
-// fp32 V tile: convert only (to bf16, or with kTF round to tf32).
-template <int D, int ROWS, bool kTF = false>
+// A bf16 tile converted to fp16 in place (exact for |x| in fp16's normal range;
+// smaller values keep fp16's subnormal spacing, 2^-24), 16 bytes per thread
+// and step.
+template <int BYTES>
+__device__ __forceinline__ void bf16_tile_to_f16(uint8_t *tile, int tw) {
+    for (int i = tw; i < BYTES / 16; i += 128) {
+        uint4 *c = reinterpret_cast<uint4 *>(tile) + i;
+        const uint4 x = *c;
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t h[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) h[k] = pack_f16x2(bf16lo_to_f32(w[k]), bf16hi_to_f32(w[k]));
+        *c = make_uint4(h[0], h[1], h[2], h[3]);
+    }
+}
+
+// fp32 V tile: convert only (to bf16, with kF16 to fp16, or with kTF round to
+// tf32).  The tf32
+// tile is stored transposed, K-major for the PV product: row d (output dim)
+// holds the ROWS keys' values, 32 keys per 128-byte row of a box of D rows
+// (ROWS / 32 boxes), 16-byte chunks swizzled by d; each thread gathers four
+// consecutive keys of one dim into one chunk.
+template <int D, int ROWS, bool kTF = false, bool kF16 = false>
 __device__ __forceinline__ void load_v_f32(uint8_t *tile, const float *base, long long rs, int row0,
                                            int L, int tw) {
+    if constexpr (kTF) {
+        constexpr int VBOX = D * 128;   // one box: D rows of 32 keys
+        for (int idx = tw; idx < D * (ROWS / 4); idx += 128) {
+            const int d = idx % D, g = idx / D;    // dim, group of 4 keys
+            float x[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = 4 * g + e;
+                x[e] = row0 + r < L ? round_tf32(base[(long long)(row0 + r) * rs + d]) : 0.f;
+            }
+            *reinterpret_cast<float4 *>(tile + (g >> 3) * VBOX + d * 128 +
+                                        (((g & 7) ^ (d & 7)) << 4)) =
+                make_float4(x[0], x[1], x[2], x[3]);
+        }
+        return;
+    }
     constexpr int CPR = D / 8;
     constexpr int BOX = ROWS * 128;
     for (int idx = tw; idx < ROWS * CPR; idx += 128) {
@@ -605,7 +647,10 @@ __device__ __forceinline__ void load_v_f32(uint8_t *tile, const float *base, lon
         float x[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[e] = valid ? src[e] : 0.f;
-        store8<false, false, D, BOX, kTF>(tile, nullptr, r, fc, x);
+        *reinterpret_cast<uint4 *>(tile + chunk_off(r, fc, BOX)) =
+            kF16 ? make_uint4(pack_f16x2(x[0], x[1]), pack_f16x2(x[2], x[3]),
+                              pack_f16x2(x[4], x[5]), pack_f16x2(x[6], x[7]))
+                 : pack8(x);
     }
 }
 
@@ -736,6 +781,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // products; at D = 128 two query tiles of them would not fit beside the
     // K/V stages, so they are rounded to bf16 like the split mode's values.
     constexpr bool kTF = kF32 && !kSplit && D == 64;
+    // split mode: P and V in fp16 for PV (bf16 V tiles from the TMA are
+    // converted in shared memory by the rotation warpgroup)
+    constexpr bool kPF16 = kSplit && LCX_SPLIT_P_F16;
+    constexpr bool kConvV = kPF16 && !kF32;
     using C = Cfg<D, DV, kSplit, kTF>;
     static_assert(!kF32 || (RD == D && DV == D), "fp32 operands: full rotary, DV = D");
     static_assert(!kSplit || (RD == D && DV == D), "split QK^T: full rotary, DV = D");
@@ -770,6 +819,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < NSV; ++s) {
             mbar_init(&bar.full_v[s], kF32 ? 128 : 1);
+            mbar_init(&bar.fp16_v[s], 128);
             mbar_init(&bar.empty_v[s], 1);
         }
         for (int t = 0; t < 2; ++t) {
@@ -900,8 +950,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                           : kTF ? idesc_f32acc(128, BN, kFmtTF32, kFmtTF32, 0, 0)
                                                 : idesc_bf16_f32(128, BN, 0, 0);
                 constexpr uint32_t kIdX8 = idesc_f32acc(128, BN, kFmtE5M2, kFmtE5M2, 0, 0);
-                constexpr uint32_t kIdPV = kTF ? idesc_f32acc(128, DV, kFmtTF32, kFmtTF32, 0, 1)
-                                               : idesc_bf16_f32(128, DV, 0, 1);
+                // PV: V MN-major (bf16 tiles as the TMA lands them), or K-major
+                // (the tf32 tile, which the loader writes transposed)
+                constexpr uint32_t kIdPV = kTF ? idesc_f32acc(128, DV, kFmtTF32, kFmtTF32, 0, 0)
+                                          : kPF16 ? idesc_f32acc(128, DV, kFmtF16, kFmtF16, 0, 1)
+                                                  : idesc_bf16_f32(128, DV, 0, 1);
+                // V ready for PV: landed (TMA, or written by the fp32 loader), or
+                // converted to fp16 by the rotation warpgroup
+                uint64_t *vready = kConvV ? bar.fp16_v : bar.full_v;
                 const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
                 // S_t = Q_t K^T over D in steps of 16 (32 bytes inside a 128-byte
                 // swizzle row, then the next 64-column box).  Descriptors of the
@@ -909,7 +965,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // 16-byte units, well inside the 14-bit field).
                 const uint64_t dq0 = sdesc_sw128(q_addr, 16, 1024);
                 const uint64_t dk0 = sdesc_sw128(k_addr, 16, 1024);
-                const uint64_t dv0 = sdesc_sw128(v_addr, C::kBoxK, 1024);
+                const uint64_t dv0 = kTF ? sdesc_sw128(v_addr, 16, 1024)
+                                         : sdesc_sw128(v_addr, C::kBoxK, 1024);
                 auto issue_s = [&](int t, int s) {
                     const uint64_t qa = dq0 + ((t * C::kParts * C::kTileQ) >> 4);
                     const uint64_t ka = dk0 + ((s * C::kParts * C::kTileK) >> 4);
@@ -937,8 +994,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 };
                 // O_t += P_t V: P from TMEM (BN/2 columns of bf16 pairs, or BN of
-                // tf32), V MN-major; each instruction takes 32 bytes of keys per
-                // row of P (8 TMEM columns) and as many 128-byte rows of V.
+                // tf32); each instruction takes 32 bytes of keys per row of P (8
+                // TMEM columns).  bf16 V is MN-major (as many 128-byte rows of V
+                // per step); the tf32 tile is V^T, K-major (32 bytes of each row).
                 auto issue_pv = [&](int t, int s, bool acc) {
                     const uint64_t va = dv0 + ((s * C::kTileV) >> 4);
                     const uint32_t dst = tmem + C::kColO + t * DV;
@@ -947,8 +1005,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < BN / KS; ++kk) {
                         if constexpr (kTF)
-                            mma_ts_tf32(dst, pa + kk * 8, va + ((kk * KS * 128) >> 4), kIdPV,
-                                        (acc || kk > 0));
+                            // K-major V^T: 32 keys per box row, four 8-key steps per box
+                            mma_ts_tf32(dst, pa + kk * 8,
+                                        va + ((((kk >> 2) * DV * 128) + (kk & 3) * 32) >> 4),
+                                        kIdPV, (acc || kk > 0));
                         else
                             mma_ts(dst, pa + kk * 8, va + ((kk * KS * 128) >> 4), kIdPV,
                                    (acc || kk > 0));
@@ -978,7 +1038,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     for (int j = 0; ok && j < T.n; ++j) {
                         const int t = j & 1, sv = j % NSV, jn = j + 2;
-                        ok = mbar_wait(&bar.full_v[sv], (j / NSV) & 1, abort, tmo);
+                        ok = mbar_wait(&vready[sv], (j / NSV) & 1, abort, tmo);
                         if (ok) ok = mbar_wait(&bar.p_ready[t], (j >> 1) & 1, abort, tmo);
                         tc_fence_after();
                         if (!ok) break;
@@ -1008,7 +1068,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     for (int j = 0; ok && j < T.n; ++j) {
                         const int sv = j % NSV, jn = j + 1;
-                        ok = mbar_wait(&bar.full_v[sv], (j / NSV) & 1, abort, tmo);
+                        ok = mbar_wait(&vready[sv], (j / NSV) & 1, abort, tmo);
                         for (int t = 0; ok && t < U.nt; ++t) {
                             ok = mbar_wait(&bar.p_ready[t], j & 1, abort, tmo);
                             tc_fence_after();
@@ -1085,16 +1145,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 relay_k = false;
             }
         }
-        for (int j = 0; ok && relay_k && j < T.n; ++j) {
+        // key tile j (when the keys pass through this warpgroup), then, split
+        // mode, value tile j converted to fp16 -- the order the MMA needs them
+        for (int j = 0; ok && (relay_k || kConvV) && j < T.n; ++j) {
             const int jt = T.tile(j);
             const int s = j % NSK, use = j / NSK, sv = j % NSV, usev = j / NSV;
             uint8_t *tk = sK + s * C::kParts * C::kTileK;
             if constexpr (!kF32) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_k[s], use & 1, abort, tmo));
-                if (!ok) break;
-                if (rotk || kSplit)
-                    rotate_tile_bf16<D, RD, kHalf, kSplit, true, BN>(
-                        tk, tk + C::kTileK, (long long)jt * BN, ph, p, rotk, &kcarry);
+                if (relay_k) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_k[s], use & 1, abort, tmo));
+                    if (!ok) break;
+                    if (rotk || kSplit)
+                        rotate_tile_bf16<D, RD, kHalf, kSplit, true, BN>(
+                            tk, tk + C::kTileK, (long long)jt * BN, ph, p, rotk, &kcarry);
+                }
             } else {
                 if (use > 0)
                     ok = __all_sync(0xffffffffu,
@@ -1106,8 +1170,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                                p.ks[2], jt * BN, p.Lk,
                                                                (long long)jt * BN, rotk, ph, p);
             }
-            fence_proxy_async_smem();
-            mbar_arrive(&bar.ready_k[s]);
+            if (relay_k) {
+                fence_proxy_async_smem();
+                mbar_arrive(&bar.ready_k[s]);
+            }
+            if constexpr (kConvV) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_v[sv], usev & 1, abort, tmo));
+                if (!ok) break;
+                bf16_tile_to_f16<C::kTileV>(sV + sv * C::kTileV, tw);
+                fence_proxy_async_smem();
+                mbar_arrive(&bar.fp16_v[sv]);
+            }
             if constexpr (kF32) {
                 if (usev > 0)
                     ok = __all_sync(0xffffffffu,
@@ -1115,7 +1188,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 const float *base = reinterpret_cast<const float *>(p.v) + U.b * p.vs[0] +
                                     (long long)U.g * p.vs[1];
-                load_v_f32<D, BN, kTF>(sV + sv * C::kTileV, base, p.vs[2], jt * BN, p.Lk, tw);
+                load_v_f32<D, BN, kTF, kPF16>(sV + sv * C::kTileV, base, p.vs[2], jt * BN, p.Lk,
+                                              tw);
                 fence_proxy_async_smem();
                 mbar_arrive(&bar.full_v[sv]);
             }
@@ -1248,8 +1322,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             pe = exp2_fma2(x);
                         else
                             pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-                        pk[e] = pack_bf16x2(pe.x, pe.y);
-                        if (kSplit) {
+                        if (kPF16) {
+                            // fp16 weights (11 significant bits; at most 2^8 with
+                            // the stale reference, far inside fp16's range)
+                            pk[e] = pack_f16x2(pe.x, pe.y);
+                            lsum = add2(lsum, f16x2_to_f32x2(pk[e]));
+                        } else if (kSplit) {
+                            pk[e] = pack_bf16x2(pe.x, pe.y);
                             // Normalise by the weights the tensor core actually
                             // multiplies V with (bf16), not their fp32 values: with
                             // the stale max reference the dominant weight is 2^d,
@@ -1257,6 +1336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             lsum = add2(lsum,
                                         make_float2(bf16lo_to_f32(pk[e]), bf16hi_to_f32(pk[e])));
                         } else {
+                            pk[e] = pack_bf16x2(pe.x, pe.y);
                             lsum = add2(lsum, pe);
                         }
                     }
@@ -1777,8 +1857,9 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
         // Keys rotated on chip: softmax warps whose 16 rows hold no query in
         // either tile (warp w: rows 32 (w % 4) + 16 (w / 4) .. + 15) rotate key
         // tiles beside warps 8-11 (four of them, which halves each thread's
-        // rows; with fewer idle warps nobody helps).
-        if (x.p.rotate_k) {
+        // rows; with fewer idle warps nobody helps).  Not in the split mode,
+        // whose rotation warpgroup also converts every V tile to fp16.
+        if (x.p.rotate_k && !x.split_qk) {
             int mask = 0, n = 0;
             for (int w = 0; w < 8 && n < 4; ++w) {
                 bool any = false;
