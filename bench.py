@@ -59,10 +59,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
 # launch on the headline workload (yarn_L131072_s16), from a one-pass ncu capture
-# of the current kernel (keys pre-rotated by the rotate pass): 3.02 GB read +
-# 1.09 GB written (algorithmic: q, k, v read once = 1.61 GB, o written once =
-# 1.07 GB).  Only valid for that workload.
-ATTN_TRAFFIC_BYTES = {"yarn_L131072_s16": 4.11e9}
+# of the current kernel (keys pre-rotated by the rotate pass); None until the
+# current kernel has been captured.  Only valid for that workload.
+ATTN_TRAFFIC_BYTES = {"yarn_L131072_s16": None}
 
 
 def load_peaks():
@@ -527,7 +526,8 @@ def bench_configs(lcx, dev, stream, status, peaks, local, reps=5):
                 "apply_rope_ms": round(rope_ms, 4),
                 "l2": "flushed between calls" if fl is not None else (
                     "inputs larger than L2" if not tiny else "launch-bound latency, L2 warm"),
-                "qk_mode": "split" if w.split_qk else "bf16",
+                "qk_mode": ("split: fp16 q'k' + e5m2 cross terms, fp16 P and V" if w.split_qk
+                            else "tf32" if w.dtype == "f32" and w.D == 64 else "bf16"),
                 "dtype": w.dtype, "flops_per_call": flops,
             }
             if not w.split_qk:

@@ -115,8 +115,8 @@ struct AttnParams {
     int test_stall;                    // loader issues nothing (watchdog test hook)
     int rot_help;                      // head-packed split-KV with keys rotated on chip: the
                                        // softmax warps (bit w = warp w; 0 or 4 of them) whose
-                                       // rows hold no query in either tile and that rotate key
-                                       // tiles with warps 8-11
+                                       // rows hold no query and that rotate key tiles with
+                                       // warps 8-11
     int k_rope_shared;                 // rotated key columns come from one shared head
     int k_x8_tma;                      // split mode: the keys' 8-bit cross parts arrive by TMA
     float rot_ms;                      // factor on rotated values (partial rotary: mscale)
@@ -824,9 +824,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&bar.s_ready[t], 1);
-            // every softmax warp hands over P of every tile, except the ones that
+            // the tile's four softmax warps hand over P, except the ones that
             // help rotate keys
-            mbar_init(&bar.p_ready[t], 32 * (8 - __popc(p.rot_help)));
+            mbar_init(&bar.p_ready[t], 32 * (4 - __popc((p.rot_help >> (4 * t)) & 0xF)));
             mbar_init(&bar.o_ready[t], 1);
         }
         mbar_init(&bar.drain, 1);
@@ -974,8 +974,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if constexpr (kSplit) {
                         // the e5m2 cross product first, into a fresh accumulator:
                         // [h8 | r8]_q [r8 | h8]_k^T over K = 2 D in steps of 32
-                        // bytes -- the same byte walk as the 16-bit product
-#pragma unroll
+                        // bytes -- the same byte walk as the 16-bit product (loops
+                        // not unrolled: the issuing warp has 64 registers)
+#pragma unroll 1
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint32_t oq = ((kk >> 2) * C::kBoxQ + (kk & 3) * 32) >> 4;
                             const uint32_t ok_ = ((kk >> 2) * C::kBoxK + (kk & 3) * 32) >> 4;
@@ -983,7 +984,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       kIdX8, kk > 0);
                         }
                     }
-#pragma unroll
+#pragma unroll(kSplit ? 1 : C::kKSteps)
                     for (int kk = 0; kk < C::kKSteps; ++kk) {
                         const uint32_t oq = ((kk >> 2) * C::kBoxQ + (kk & 3) * 32) >> 4;
                         const uint32_t ok_ = ((kk >> 2) * C::kBoxK + (kk & 3) * 32) >> 4;
@@ -1201,52 +1202,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int ord = __popc(p.rot_help & ((1u << warp) - 1u));
             rotate_keys_helped<D, RD, kHalf, kSplit, NSK, BN, C::kParts, C::kTileK>(
                 128 + 32 * ord + lane, T, sK, bar, p, abort, tmo);
-        } else {
-            // ------------------------------------------------ softmax
-            // All eight softmax warps work on one query tile at a time, two
-            // threads per row: warp w takes rows 32 (w % 4) + 16 (w / 4) ..
-            // + 15 of every query tile (TMEM lanes of its quadrant), its lanes
-            // 0-15 the first half of those rows' columns (keys of S, output
-            // dims of O) and lanes 16-31 the second half.  The row max and sum
-            // combine with one shuffle.  The tiles alternate in the order the
-            // MMA warp produces them (S_0(j), S_1(j), S_0(j + 1), ...), so one
-            // tile's softmax runs at the full width of the SM while the tensor
-            // core works on the other tile.
-            const int hf = lane >> 4;                        // column half
-            const int row = (warp & 3) * 32 + (warp >> 2) * 16 + (lane & 15);
-            const uint32_t tlane = uint32_t((warp & 3) * 32 + (warp >> 2) * 16) << 16;
+        } else if ((warp >> 2) < U.nt) {
+            // ------------------------------------------------ softmax, tile t
+            // Warps 0-3 serve query tile 0 and warps 4-7 tile 1, one thread per
+            // row (TMEM lane), the whole S row in registers.  (All eight warps
+            // on one tile at a time, two threads per row, was measured 5%
+            // slower: twice the per-row overhead for the same MUFU work.)
+            const int t = warp >> 2;
+            const int wq = warp & 3;
+            const int row = wq * 32 + lane;
+            const uint32_t trow = tmem + (uint32_t(wq * 32) << 16);
+            const uint32_t o_col = C::kColO + t * DV;
+            const RowMap rm = map_row(p, U, t, row, packed);
+            const int pi = rm.i + p.qoff;  // this row's query position
+            const int tq0 = U.tq0(t);      // the tile's first query row
             const float cl2 = p.c_log2;
-            constexpr int HB = BN / 2;                       // keys per thread
-            // Interleaved key tiles (head-packed split-KV): tile t takes the key
-            // tiles j = t mod 2 of the split and writes partial 2 split + t.
-            const bool ilv = kKvSplit && p.pack_ilv;
-            const int nt = U.nt;
-            // per-tile state in scalars (t is a run-time index: arrays would live
-            // in local memory)
-            const RowMap rm0 = map_row(p, U, 0, row, packed);
-            const RowMap rm1 = map_row(p, U, nt > 1 ? 1 : 0, row, packed);
-            float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-            // Split-KV (decode) tiles hold few queries: a warp whose rows of the
-            // tile hold none only keeps step with the barriers (its P rows are
-            // never used: their O rows are not stored).
-            const bool idle0 = kKvSplit && !__any_sync(0xffffffffu, rm0.valid);
-            const bool idle1 = kKvSplit && !__any_sync(0xffffffffu, rm1.valid);
+            float m = -INFINITY, l = 0.f;
             bool ok = true;
-            const int n_steps = ilv ? T.n : T.n * nt;
-            for (int k = 0; k < n_steps; ++k) {
-                const int t = ilv ? (k & 1) : (k % nt);
-                const int j = ilv ? k : k / nt;               // key tile of the list
-                const int it = ilv ? (k >> 1) : j;            // the tile's own step count
+            // Split-KV (decode) tiles hold few queries: a warp whose 32 rows hold
+            // none only keeps step with the barriers, which leaves its SMSP to the
+            // rotation warp (its P rows are never used: their O rows are not stored).
+            const bool idle = kKvSplit && !__any_sync(0xffffffffu, rm.valid);
+            // Interleaved key tiles (head-packed split-KV): this tile takes the
+            // key tiles j = t mod 2 of the split and writes partial 2 split + t.
+            const bool ilv = kKvSplit && p.pack_ilv;
+            const int n_it = ilv ? (T.n - t + 1) / 2 : T.n;
+            for (int it = 0; it < n_it; ++it) {
+                const int j = ilv ? 2 * it + t : it;
+                const uint32_t s_col = t * BN;
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_ready[t], it & 1, abort, tmo));
                 if (!ok) break;
-                if (t ? idle1 : idle0) {
+                if (idle) {
                     mbar_arrive(&bar.p_ready[t]);
                     continue;
                 }
                 tc_fence_after();
-                const int jt = T.tile(j), k0 = jt * BN + hf * HB;   // this thread's first key
-                const bool partial = !tile_full<BN>(U.tq0(t), jt, p);
-                const int pi = (t ? rm1.i : rm0.i) + p.qoff;   // this row's query position
+                const int jt = T.tile(j), k0 = jt * BN;
+                const bool partial = !tile_full<BN>(tq0, jt, p);
                 // visible columns: col <= hi and (no window or col >= lo or col < sk)
                 const int hi = p.causal ? min(pi - k0, p.Lk - 1 - k0) : p.Lk - 1 - k0;
                 const int lo = pi - p.window + 1 - k0;
@@ -1254,68 +1246,67 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool win = p.causal && p.window > 0;
                 auto vis = [&](int col) { return col <= hi && (!win || col >= lo || col < sk); };
 
-                // This thread's half of its S row in one TMEM load.
-                const uint32_t trow = tmem + tlane + uint32_t(t * BN);
-                float v[HB];
-                tmem_ld16x2_64(trow, v);
+                // The whole S row of this thread in one TMEM load.
+                float v[BN];
+                tmem_ld128(trow + s_col, v);
                 if (partial) {
 #pragma unroll
-                    for (int e = 0; e < HB; ++e)
+                    for (int e = 0; e < BN; ++e)
                         if (!vis(e)) v[e] = -INFINITY;
                 }
-                const float mh = row_max(v);
-                const float mx = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 16));
-                float mt = t ? m1 : m0;
-                float lt = t ? l1 : l0;
-                const float m_new = fmaxf(mt, mx * cl2);
+                const float mx = row_max(v);
+                const float m_new = fmaxf(m, mx * cl2);
                 // Keep the old reference unless the max grew by more than 2^8: the
                 // result is exact either way, only O's rescale is saved.
-                const bool need = (mt != -INFINITY) && (m_new > mt + kRescaleLog2);
+                const bool need = (m != -INFINITY) && (m_new > m + kRescaleLog2);
                 if (__any_sync(0xffffffffu, need)) {
                     // O_t is not in flight: S_t(j) is issued after PV_t(j - 1), so
-                    // its completion implies PV_t(j - 1)'s.  Each thread rescales its
-                    // half of the row's output dims (32-column chunks 2c + hf).
-                    const float alpha = need ? ex2_approx(mt - m_new) : 1.f;
-                    const uint32_t orow = tmem + tlane + uint32_t(C::kColO + t * DV);
+                    // its completion implies PV_t(j - 1)'s.
+                    const float alpha = need ? ex2_approx(m - m_new) : 1.f;
 #pragma unroll 1
-                    for (int c = 0; c < DV / 64; ++c) {
+                    for (int c = 0; c < DV / 32; ++c) {
                         float o[32];
-                        tmem_ld16x2_32(orow + c * 64, o);
+                        tmem_ld32(trow + o_col + c * 32, o);
                         uint32_t u[32];
 #pragma unroll
                         for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(o[e] * alpha);
-                        tmem_st16x2_32(orow + c * 64, u);
+                        tmem_st32(trow + o_col + c * 32, u);
                     }
                     if (need) {
-                        lt *= alpha;
-                        mt = m_new;
+                        l *= alpha;
+                        m = m_new;
                     }
                 }
-                if (mt == -INFINITY) mt = m_new;
-                const float mref = (mt == -INFINITY) ? 0.f : mt;
-                // P = 2^(s c - m) as bf16 pairs, written over the first half of S
-                // (this thread's 64 keys: P columns 32 hf .. 32 hf + 31); tf32
-                // operands: as tf32 values over all of S (columns 64 hf ..).
+                if (m == -INFINITY) m = m_new;
+                const float mref = (m == -INFINITY) ? 0.f : m;
+                // P = 2^(s c - m): as bf16 pairs (fp16 pairs in the split mode)
+                // over the first half of S, or, tf32 operands, as tf32 values over
+                // all of S.  One column pair in kEmuEvery takes 2^x on the FMA pipe.
                 const float2 c2 = make_float2(cl2, cl2), nm2 = make_float2(-mref, -mref);
                 float2 lsum = make_float2(0.f, 0.f);
                 if constexpr (kTF) {
-                    uint32_t pw[HB];
 #pragma unroll
-                    for (int e = 0; e < HB / 2; ++e) {
+                    for (int e = 0; e < BN / 2; ++e) {
                         const float2 x = fma2(make_float2(v[2 * e], v[2 * e + 1]), c2, nm2);
                         // the weights the tensor core multiplies V with (tf32), and
                         // the normalisation by their sum
                         const float2 pe = make_float2(round_tf32(ex2_approx(x.x)),
                                                       round_tf32(ex2_approx(x.y)));
-                        pw[2 * e] = __float_as_uint(pe.x);
-                        pw[2 * e + 1] = __float_as_uint(pe.y);
+                        v[2 * e] = pe.x;
+                        v[2 * e + 1] = pe.y;
                         lsum = add2(lsum, pe);
                     }
-                    tmem_st16x2_64(tmem + tlane + uint32_t(t * BN), pw);
-                } else {
-                    uint32_t pk[HB / 2];
+                    uint32_t pw[64];
 #pragma unroll
-                    for (int e = 0; e < HB / 2; ++e) {
+                    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                        for (int e = 0; e < 64; ++e) pw[e] = __float_as_uint(v[64 * h + e]);
+                        tmem_st64(trow + s_col + 64 * h, pw);
+                    }
+                } else {
+                    uint32_t pk[BN / 2];
+#pragma unroll
+                    for (int e = 0; e < BN / 2; ++e) {
                         const float2 x = fma2(make_float2(v[2 * e], v[2 * e + 1]), c2, nm2);
                         float2 pe;
                         if (kEmuEvery > 0 && (e % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1)
@@ -1340,47 +1331,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                             lsum = add2(lsum, pe);
                         }
                     }
-                    tmem_st16x2_32(tmem + tlane + uint32_t(t * BN), pk);
+                    tmem_st64(trow + s_col, pk);
                 }
-                lt += lsum.x + lsum.y;
-                if (t) {
-                    m1 = mt;
-                    l1 = lt;
-                } else {
-                    m0 = mt;
-                    l0 = lt;
-                }
+                l += lsum.x + lsum.y;
                 tc_fence_before();
                 mbar_arrive(&bar.p_ready[t]);
             }
-            for (int t = 0; ok && t < nt; ++t) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&bar.o_ready[t], 0, abort, tmo));
-                if (!ok) break;
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.o_ready[t], 0, abort, tmo));
+            if (ok) {
                 tc_fence_after();
-                const RowMap rm = t ? rm1 : rm0;
-                const float lh = t ? l1 : l0, mt = t ? m1 : m0;
-                const float lt = lh + __shfl_xor_sync(0xffffffffu, lh, 16);   // the row's sum
-                const float inv = lt > 0.f ? 1.f / lt : 0.f;
+                const float inv = l > 0.f ? 1.f / l : 0.f;
                 const int slot = ilv ? 2 * U.split + t : U.split;
-                const int n_it = ilv ? (T.n - t + 1) / 2 : T.n;
-                const uint32_t orow = tmem + tlane + uint32_t(C::kColO + t * DV);
 #pragma unroll 1
-                for (int c = 0; c < DV / 64; ++c) {
+                for (int c = 0; c < DV / 32; ++c) {
                     float v[32];
                     if (n_it > 0) {
-                        tmem_ld16x2_32(orow + c * 64, v);
+                        tmem_ld32(trow + o_col + c * 32, v);
                     } else {
                         // no key tile reached this tile: O_t was never written
 #pragma unroll
                         for (int e = 0; e < 32; ++e) v[e] = 0.f;
                     }
                     if (rm.valid)
-                        store_o32<DV, kF32, kKvSplit>(p, U, slot, rm.h, rm.i, 2 * c + hf, v, inv);
+                        store_o32<DV, kF32, kKvSplit>(p, U, slot, rm.h, rm.i, c, v, inv);
                 }
-                if (rm.valid && hf == 0) {
+                if (rm.valid) {
                     const float ln2 = 0.69314718055994531f;
                     store_lse<kKvSplit>(p, U, slot, rm.h, rm.i,
-                                        lt > 0.f ? (mt + __log2f(lt)) * ln2 : -INFINITY);
+                                        l > 0.f ? (m + __log2f(l)) * ln2 : -INFINITY);
                 }
             }
         }
@@ -1854,8 +1832,8 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
         if (x.p.pack_off + used > kBM) x.p.pack_off = 0;
         x.p.pack_ilv = 1;
         n_parts = 2 * num_splits;
-        // Keys rotated on chip: softmax warps whose 16 rows hold no query in
-        // either tile (warp w: rows 32 (w % 4) + 16 (w / 4) .. + 15) rotate key
+        // Keys rotated on chip: softmax warps whose 32 rows of their tile (warp
+        // w: rows 32 (w % 4) .. + 31 of tile w / 4) hold no query rotate key
         // tiles beside warps 8-11 (four of them, which halves each thread's
         // rows; with fewer idle warps nobody helps).  Not in the split mode,
         // whose rotation warpgroup also converts every V tile to fp16.
@@ -1863,12 +1841,10 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
             int mask = 0, n = 0;
             for (int w = 0; w < 8 && n < 4; ++w) {
                 bool any = false;
-                const int r0 = 32 * (w % 4) + 16 * (w / 4);
-                for (int t = 0; t < 2 && !any; ++t)
-                    for (int r = r0; r < r0 + 16 && !any; ++r) {
-                        const int rel = r - t * x.p.pack_off;
-                        any = rel >= 0 && rel < used && rel % x.p.pack_stride < a->L;
-                    }
+                for (int r = 32 * (w % 4); r < 32 * (w % 4) + 32 && !any; ++r) {
+                    const int rel = r - (w / 4) * x.p.pack_off;
+                    any = rel >= 0 && rel < used && rel % x.p.pack_stride < a->L;
+                }
                 if (!any) {
                     mask |= 1 << w;
                     ++n;
