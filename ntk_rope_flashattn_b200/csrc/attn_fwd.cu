@@ -23,7 +23,7 @@
 //   warps 0-3 / 4-7  softmax for query tile 0 / 1: one thread per query row
 //               reads its S row from TMEM, masks partial tiles, keeps the
 //               running max/sum, writes P (bf16) back over S, rescales its O
-//               row only when the max grew by more than 2^8, and finally
+//               row only when the max grew by more than 2^15, and finally
 //               normalises O and stores it.
 // Positions: query row i sits at q_offset + i and key j at j, so one kernel
 // serves prefill (q_offset 0, Lk = L), chunked prefill and decode (the new
@@ -55,7 +55,11 @@ constexpr int kRegsRotate = 96;         // warpgroup 2
 constexpr int kRegsIssue = 64;          // warpgroup 3: TMA and MMA issuing warps
 static_assert(2 * kRegsSoftmax + kRegsRotate + kRegsIssue == 4 * 128, "register file split");
 constexpr int kBM = 128;                // query rows per tile
-constexpr float kRescaleLog2 = 8.0f;    // rescale O only if the max grows by > 2^8
+// Rescale O only if the row max grew by more than 2^15: until then the weights
+// stay <= 2^15, inside the range of every P format used (bf16, fp16, tf32), and
+// O and l stay far from fp32's.  (At 2^8, outlier-heavy inputs had a rescale
+// in 53% of a warp's key tiles, N(0,1) inputs in 5%; at 2^15 36% and ~0%.)
+constexpr float kRescaleLog2 = 15.0f;
 // Build-time switches (-D...; the defaults are the measured-fastest choices):
 //   LCX_EMU_EVERY       1 column pair in N takes 2^x on the FMA pipe (0: none)
 //   LCX_D192_TWO_TILES  two query tiles and one K stage at D = 192 (0: one tile)
@@ -78,6 +82,11 @@ constexpr float kRescaleLog2 = 8.0f;    // rescale O only if the max grows by > 
 // shared memory) rather than bf16
 #ifndef LCX_SPLIT_P_F16
 #define LCX_SPLIT_P_F16 1
+#endif
+// LCX_CORR_WG: when the rotation warpgroup relays no key tiles, it rescales O
+// for the softmax (off the softmax's critical path)
+#ifndef LCX_CORR_WG
+#define LCX_CORR_WG 1
 #endif
 #ifndef LCX_PHASOR_CARRY
 #define LCX_PHASOR_CARRY 1
@@ -188,7 +197,9 @@ struct Bars {
     uint64_t full_k[NSK], ready_k[NSK], empty_k[NSK];
     uint64_t full_v[NSV], empty_v[NSV], fp16_v[NSV];
     uint64_t s_ready[2], p_ready[2], o_ready[2];
+    uint64_t corr_req[2], corr_done[2];   // O rescale handed to the rotation warpgroup
     uint64_t drain;
+    int corr_need[2][4];                  // per tile and warp: some row needs a rescale
     uint32_t tmem_base;
     int abort;
 };
@@ -808,6 +819,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool packed = kKvSplit && !kF32 && p.pack_lp > 0;       // head-packed query tiles
     volatile int *abort = &bar.abort;
     const uint64_t tmo = p.timeout_ns;
+    // The rotation warpgroup rescales O for the softmax (a correction
+    // warpgroup) when it relays no key tiles: keys pre-rotated or rotated once
+    // (and, split, split into their parts), bf16 operands, no rotation helpers.
+    // The softmax then only publishes each row's factor and goes on with its
+    // exponentials while the rescale runs beside them.
+    const bool corr = LCX_CORR_WG && !kF32 && !((kSplit && !p.k_x8_tma) || p.rotate_k) &&
+                      !p.rot_help;
 
     if (threadIdx.x == 0) {
         mbar_init(&bar.full_q, 1);
@@ -828,6 +846,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // help rotate keys
             mbar_init(&bar.p_ready[t], 32 * (4 - __popc((p.rot_help >> (4 * t)) & 0xF)));
             mbar_init(&bar.o_ready[t], 1);
+            mbar_init(&bar.corr_req[t], 128);
+            mbar_init(&bar.corr_done[t], 128);
         }
         mbar_init(&bar.drain, 1);
         // A CTA that starts after another one's watchdog fired does no work.
@@ -1041,6 +1061,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int t = j & 1, sv = j % NSV, jn = j + 2;
                         ok = mbar_wait(&vready[sv], (j / NSV) & 1, abort, tmo);
                         if (ok) ok = mbar_wait(&bar.p_ready[t], (j >> 1) & 1, abort, tmo);
+                        if (ok && corr) ok = mbar_wait(&bar.corr_done[t], (j >> 1) & 1, abort, tmo);
                         tc_fence_after();
                         if (!ok) break;
                         issue_pv(t, sv, j >= 2);
@@ -1072,6 +1093,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = mbar_wait(&vready[sv], (j / NSV) & 1, abort, tmo);
                         for (int t = 0; ok && t < U.nt; ++t) {
                             ok = mbar_wait(&bar.p_ready[t], j & 1, abort, tmo);
+                            if (ok && corr) ok = mbar_wait(&bar.corr_done[t], j & 1, abort, tmo);
                             tc_fence_after();
                             if (!ok) break;
                             issue_pv(t, sv, j > 0);
@@ -1147,8 +1169,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         // key tile j (when the keys pass through this warpgroup), then, split
-        // mode, value tile j converted to fp16 -- the order the MMA needs them
-        for (int j = 0; ok && (relay_k || kConvV) && j < T.n; ++j) {
+        // mode, value tile j converted to fp16, then the O rescales of the query
+        // tiles that take key tile j (correction warpgroup) -- the order the MMA
+        // needs them
+        const bool ilv = kKvSplit && p.pack_ilv;
+        for (int j = 0; ok && (relay_k || kConvV || corr) && j < T.n; ++j) {
             const int jt = T.tile(j);
             const int s = j % NSK, use = j / NSK, sv = j % NSV, usev = j / NSV;
             uint8_t *tk = sK + s * C::kParts * C::kTileK;
@@ -1181,6 +1206,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bf16_tile_to_f16<C::kTileV>(sV + sv * C::kTileV, tw);
                 fence_proxy_async_smem();
                 mbar_arrive(&bar.fp16_v[sv]);
+            }
+            if (corr) {
+                // warp 8 + q serves TMEM lanes 32 q .. 32 q + 31 (its quadrant),
+                // the rows of softmax warps q and 4 + q
+                const int wq = warp - kWarpRot0;
+                const uint32_t trow = tmem + (uint32_t(wq * 32) << 16);
+                const int it = ilv ? (j >> 1) : j;
+                const int tb = ilv ? (j & 1) : 0, te = ilv ? (j & 1) + 1 : U.nt;
+                for (int t = tb; ok && t < te; ++t) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(&bar.corr_req[t], it & 1, abort, tmo));
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (reinterpret_cast<volatile int *>(bar.corr_need[t])[wq]) {
+                        const float alpha = tmem_ld1(trow + t * BN + BN - 1);
+                        const uint32_t o_col = C::kColO + t * DV;
+#pragma unroll 1
+                        for (int c = 0; c < DV / 32; ++c) {
+                            float o[32];
+                            tmem_ld32(trow + o_col + c * 32, o);
+                            uint32_t u[32];
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(o[e] * alpha);
+                            tmem_st32_nowait(trow + o_col + c * 32, u);
+                        }
+                        tmem_wait_st();
+                    }
+                    tc_fence_before();
+                    mbar_arrive(&bar.corr_done[t]);
+                }
             }
             if constexpr (kF32) {
                 if (usev > 0)
@@ -1233,6 +1287,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_ready[t], it & 1, abort, tmo));
                 if (!ok) break;
                 if (idle) {
+                    if (corr) {
+                        if (lane == 0) bar.corr_need[t][wq] = 0;
+                        mbar_arrive(&bar.corr_req[t]);
+                    }
                     mbar_arrive(&bar.p_ready[t]);
                     continue;
                 }
@@ -1256,13 +1314,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const float mx = row_max(v);
                 const float m_new = fmaxf(m, mx * cl2);
-                // Keep the old reference unless the max grew by more than 2^8: the
+                // Keep the old reference unless the max grew by more than 2^15: the
                 // result is exact either way, only O's rescale is saved.
                 const bool need = (m != -INFINITY) && (m_new > m + kRescaleLog2);
-                if (__any_sync(0xffffffffu, need)) {
+                if (corr) {
+                    // publish the warp's need and each row's factor (in the last
+                    // column of S_t, free once S is in registers and outside P)
+                    // for the rotation warpgroup, which rescales O_t meanwhile
+                    const bool any = __any_sync(0xffffffffu, need);
+                    if (lane == 0) bar.corr_need[t][wq] = any ? 1 : 0;
+                    if (any) tmem_st1(trow + s_col + BN - 1, need ? ex2_approx(m - m_new) : 1.f);
+                    tc_fence_before();
+                    mbar_arrive(&bar.corr_req[t]);
+                    if (need) {
+                        l *= ex2_approx(m - m_new);
+                        m = m_new;
+                    }
+                } else if (__any_sync(0xffffffffu, need)) {
                     // O_t is not in flight: S_t(j) is issued after PV_t(j - 1), so
                     // its completion implies PV_t(j - 1)'s.
                     const float alpha = need ? ex2_approx(m - m_new) : 1.f;
+                    // chunk by chunk; the stores are not waited for one by one,
+                    // only once before P is handed over
 #pragma unroll 1
                     for (int c = 0; c < DV / 32; ++c) {
                         float o[32];
@@ -1270,8 +1343,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         uint32_t u[32];
 #pragma unroll
                         for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(o[e] * alpha);
-                        tmem_st32(trow + o_col + c * 32, u);
+                        tmem_st32_nowait(trow + o_col + c * 32, u);
                     }
+                    tmem_wait_st();
                     if (need) {
                         l *= alpha;
                         m = m_new;
@@ -1314,7 +1388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         else
                             pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                         if (kPF16) {
-                            // fp16 weights (11 significant bits; at most 2^8 with
+                            // fp16 weights (11 significant bits; at most 2^15 with
                             // the stale reference, far inside fp16's range)
                             pk[e] = pack_f16x2(pe.x, pe.y);
                             lsum = add2(lsum, f16x2_to_f32x2(pk[e]));
@@ -1323,7 +1397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             // Normalise by the weights the tensor core actually
                             // multiplies V with (bf16), not their fp32 values: with
                             // the stale max reference the dominant weight is 2^d,
-                            // d in [0, 8], and its rounding must cancel in o.
+                            // d in [0, 15], and its rounding must cancel in o.
                             lsum = add2(lsum,
                                         make_float2(bf16lo_to_f32(pk[e]), bf16hi_to_f32(pk[e])));
                         } else {
