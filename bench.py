@@ -249,9 +249,9 @@ def bench_gpu(args, world, rank, local):
     o = torch.empty_like(q)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     # keys rotated once per step into k_rot (split-QK^T with bf16 keys: fp16 parts, then
-    # 8-bit cross parts of as many bytes)
+    # 8-bit cross parts of as many bytes, then V in fp16)
     rotate_once = True
-    parts = 2 if (w.split_qk and k.dtype == torch.bfloat16) else 1
+    parts = 3 if (w.split_qk and k.dtype == torch.bfloat16) else 1
     k_rot = torch.empty((parts,) + tuple(k.shape), dtype=k.dtype, device=dev)
     kw = dict(causal=w.causal, window=w.window, sinks=w.sinks, softmax_scale=w.softmax_scale,
               split_qk=w.split_qk, out=o, status=status, k_rot=k_rot)
@@ -495,7 +495,7 @@ def bench_configs(lcx, dev, stream, status, peaks, local, reps=5):
             rope = lcx.RopeParams(w.mode, w.D, w.base, w.scale, w.original_max_pos, w.alpha,
                                   w.beta, w.pairing)
             o = torch.empty_like(q)
-            parts = 2 if (w.split_qk and k.dtype == torch.bfloat16) else 1
+            parts = 3 if (w.split_qk and k.dtype == torch.bfloat16) else 1
             k_rot = torch.empty((parts,) + tuple(k.shape), dtype=k.dtype, device=dev)
             kw = dict(causal=w.causal, window=w.window, sinks=w.sinks,
                       softmax_scale=w.softmax_scale, split_qk=w.split_qk, out=o,

@@ -219,13 +219,14 @@ typedef struct {
                                   operands the keys' fp16 parts ([B, Hkv, Lk,
                                   D] fp16) followed by their 8-bit cross parts
                                   ([B, Hkv, Lk, 2 D] bytes: e5m2 of the
-                                  residual, then of the fp16 part).  With
+                                  residual, then of the fp16 part) and by the
+                                  values in fp16 ([B, Hkv, Lk, D]).  With
                                   k_rope: the shared rotary key, contiguous
                                   [B, 1, Lk, rope.head_dim].  16-byte aligned.
                                   Ignored otherwise (partial rotary without
                                   k_rope)                                        */
     int64_t k_rot_bytes;       /* bytes at k_rot: >= B*Hkv*Lk*D*element size,
-                                  twice that for split-QK^T with bf16, or
+                                  three times that for split-QK^T with bf16, or
                                   B*Lk*rope.head_dim*element size with k_rope */
 } lcx_attn_args;
 

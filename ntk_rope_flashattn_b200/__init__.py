@@ -252,11 +252,12 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
     rope.head_dim dims of q and k; ``k_rope`` [B, 1, Lk, rope.head_dim] then
     supplies that part of every key once for all heads and k holds the first
     D - rope.head_dim dims.  v / o may have their own head dim (v.shape[-1]).
-    ``rotate_k_once`` (or a ``k_rot`` buffer shaped like k, twice that in the
-    split-QK^T mode with bf16 keys, or like k_rope with decoupled RoPE): the
+    ``rotate_k_once`` (or a ``k_rot`` buffer shaped like k, three times that in
+    the split-QK^T mode with bf16 keys, or like k_rope with decoupled RoPE): the
     keys (with k_rope: the shared rotary key) are rotated once into that buffer
     by the rotate pass before the kernel, which then reads them pre-rotated
-    (split mode: as fp16 parts and 8-bit cross parts), instead of rotating each
+    (split mode: as fp16 parts and 8-bit cross parts, with V in fp16 beside
+    them), instead of rotating each
     key tile on chip in every CTA that reads it (ignored where the kernel does
     not rotate keys).
     ``split_qk`` (LCX_ATTN_SPLIT_QK) forms QK^T from an fp16 part and e5m2
@@ -313,8 +314,9 @@ def attn_fwd(q, k, v, rope: RopeParams, causal: bool = True, window: int = 0, si
             k_rot = torch.empty((B, 1, Lk, k_rope.shape[-1]), dtype=k.dtype, device=k.device)
         else:
             # split QK^T with bf16 keys: the pass writes the fp16 parts, then the
-            # 8-bit cross parts (2 D bytes per key: as many bytes again)
-            parts = 2 if (split_qk and k.dtype == torch.bfloat16) else 1
+            # 8-bit cross parts (2 D bytes per key: as many bytes again), then
+            # V in fp16 (as many bytes again)
+            parts = 3 if (split_qk and k.dtype == torch.bfloat16) else 1
             k_rot = torch.empty((parts, B, Hkv, Lk, Dk), dtype=k.dtype, device=k.device)
     if k_rot is not None:
         a.k_rot = k_rot.data_ptr()

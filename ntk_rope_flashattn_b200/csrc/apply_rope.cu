@@ -10,6 +10,8 @@
 // range reduction + libm sincosf) and reuses them across all H heads, so the
 // trigonometry costs 1/H of a pass and the kernel streams HBM with 128-bit
 // loads and stores.
+#include <algorithm>
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -209,7 +211,47 @@ __global__ void __launch_bounds__(256) apply_rope_kernel(const __grid_constant__
     }
 }
 
+// bf16 [B, H, L, D] (element strides, last one 1) -> contiguous fp16 copy:
+// one 16-byte vector (8 values) per thread and step, grid-stride over the rows.
+__global__ void __launch_bounds__(256) bf16_to_f16_kernel(const __nv_bfloat16 *x,
+                                                          long long xs_b, long long xs_h,
+                                                          long long xs_l, uint16_t *y, int H,
+                                                          int L, int vpr, long long n) {
+    for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n; i += (long long)gridDim.x * 256) {
+        const long long row = i / vpr;
+        const int c = int(i % vpr);
+        const int l = int(row % L);
+        const long long bh = row / L;
+        const int h = int(bh % H), b = int(bh / H);
+        const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(x + b * xs_b + h * xs_h + l * xs_l) + c);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            o[k] = pk16(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xFFFF0000u));
+        __stcs(reinterpret_cast<uint4 *>(y) + i, make_uint4(o[0], o[1], o[2], o[3]));
+    }
+}
+
 }  // namespace
+
+lcx_status bf16_to_f16_impl(const void *x, const int64_t *x_strides, void *y, int64_t B,
+                            int64_t H, int64_t L, int64_t D, cudaStream_t s) {
+    if (D % 8 != 0) return fail(LCX_ERR_UNSUPPORTED, "head dim must be a multiple of 8");
+    const long long n = (long long)B * H * L * (D / 8);
+    if (n == 0) return LCX_OK;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long blocks = std::min<long long>((n + 255) / 256, (long long)sms * 8);
+    bf16_to_f16_kernel<<<unsigned(blocks), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16 *>(x), x_strides[0], x_strides[1], x_strides[2],
+        static_cast<uint16_t *>(y), int(H), int(L), int(D / 8), n);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return fail(LCX_ERR_CUDA, "bf16 -> fp16 launch failed: %s", cudaGetErrorString(e));
+    return LCX_OK;
+}
 
 lcx_status apply_rope_impl(const lcx_rope_params *params, const void *x, void *y, void *y_x8,
                            int32_t dtype, int64_t B, int64_t H, int64_t L,

@@ -12,7 +12,9 @@
 //   unit      = (batch b, two query heads of one GQA group, 128 query rows);
 //               both query tiles read the same K/V tiles, so each K tile is
 //               loaded and rotated once for 256 query rows.
-//   warp 12   TMA producer: Q tiles once, then K/V tiles into a ring of stages.
+//   warp 12   TMA producer: Q tiles once, then K tiles into a ring of stages;
+//   warp 14   TMA producer of the V tiles (a V stage that frees late never
+//             holds back the next K tile).
 //   warps 8-11 rotation warpgroup: rotates the Q tiles and every K tile in
 //               shared memory (bf16 -> fp32 -> rotate -> bf16) right after the
 //               TMA lands, then hands the tile to the tensor core.
@@ -83,11 +85,6 @@ constexpr float kRescaleLog2 = 15.0f;
 #ifndef LCX_SPLIT_P_F16
 #define LCX_SPLIT_P_F16 1
 #endif
-// LCX_CORR_WG: when the rotation warpgroup relays no key tiles, it rescales O
-// for the softmax (off the softmax's critical path)
-#ifndef LCX_CORR_WG
-#define LCX_CORR_WG 1
-#endif
 #ifndef LCX_PHASOR_CARRY
 #define LCX_PHASOR_CARRY 1
 #endif
@@ -96,7 +93,8 @@ constexpr int kRotUnroll = LCX_ROT_UNROLL;  // rows in flight per rotation threa
 // measured fastest here, since the MUFU is not the binding limit).
 constexpr int kEmuEvery = LCX_EMU_EVERY;
 constexpr int kWarpMma = 13;
-constexpr int kWarpTma = 12;
+constexpr int kWarpTma = 12;    // Q and K tiles
+constexpr int kWarpTmaV = 14;   // V tiles
 constexpr int kWarpRot0 = 8;
 
 struct AttnParams {
@@ -128,6 +126,7 @@ struct AttnParams {
                                        // warps 8-11
     int k_rope_shared;                 // rotated key columns come from one shared head
     int k_x8_tma;                      // split mode: the keys' 8-bit cross parts arrive by TMA
+    int v_f16;                         // split mode: V arrives in fp16 (converted by a pass)
     float rot_ms;                      // factor on rotated values (partial rotary: mscale)
     float c_log2;                      // logit scale in log2 units
     unsigned long long timeout_ns;
@@ -166,14 +165,19 @@ struct Cfg {
     static constexpr int BN = 128;                      // keys per tile
     static constexpr int ES = kTF ? 4 : 2;              // bytes per operand element
     static constexpr int kParts = kSplit ? 2 : 1;       // 16-bit part (+ 8-bit cross part)
-    static constexpr int kNTQ = (D > 128 && !LCX_D192_TWO_TILES) ? 1 : 2;  // query tiles per CTA
+    // query tiles per CTA: two that ping-pong on the tensor core, or (split
+    // mode, and D = 192 without LCX_D192_TWO_TILES) one
+    static constexpr int kNTQ = (kSplit || (D > 128 && !LCX_D192_TWO_TILES)) ? 1 : 2;
+    // S buffers per query tile: the single split-mode tile keeps two, so S(j + 2)
+    // is computed while the softmax works on key tile j
+    static constexpr int kNB = kSplit ? 2 : 1;
     static constexpr int kTileQ = kBM * D * ES;         // one part of a Q tile
     static constexpr int kTileK = BN * D * ES;          // one part of a K tile
     static constexpr int kTileV = BN * DV * ES;         // a V tile
     static constexpr int kBoxQ = kBM * 128;
     static constexpr int kBoxK = BN * 128;
     static constexpr int kKSteps = D * ES / 32;         // QK^T instructions over D (32 bytes each)
-    static constexpr int kStagesK = kSplit ? (D == 64 ? 3 : 1)
+    static constexpr int kStagesK = kSplit ? (D == 64 ? 3 : 2)
                                   : kTF ? 2
                                   : (D == 64) ? 4
                                   : (D == 128) ? LCX_KSTAGES_D128
@@ -184,11 +188,11 @@ struct Cfg {
     static constexpr int kOffV = kOffK + kStagesK * kParts * kTileK;
     static constexpr int kOffBar = kOffV + kStagesV * kTileV;
     static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers + alignment slack
-    // TMEM columns: S_t at t BN (P_t aliased over its first BN/2 columns), O_t
-    // from 2 BN on.
-    static constexpr int kColO = 2 * BN;
+    // TMEM columns: S_t,b at (t kNB + b) BN (P_t,b aliased over its first BN/2
+    // columns, or all of it with tf32), then O_t.
+    static constexpr int kColO = kNTQ * kNB * BN;
     static_assert(kSmemBytes <= 232448, "shared memory budget");
-    static_assert(2 * BN + 2 * DV <= 512, "TMEM budget");
+    static_assert(kColO + kNTQ * DV <= 512, "TMEM budget");
 };
 
 template <int NSK, int NSV>
@@ -196,10 +200,8 @@ struct Bars {
     uint64_t full_q, ready_q;
     uint64_t full_k[NSK], ready_k[NSK], empty_k[NSK];
     uint64_t full_v[NSV], empty_v[NSV], fp16_v[NSV];
-    uint64_t s_ready[2], p_ready[2], o_ready[2];
-    uint64_t corr_req[2], corr_done[2];   // O rescale handed to the rotation warpgroup
+    uint64_t s_ready[2][2], p_ready[2][2], pv_done[2], o_ready[2];
     uint64_t drain;
-    int corr_need[2][4];                  // per tile and warp: some row needs a rescale
     uint32_t tmem_base;
     int abort;
 };
@@ -819,13 +821,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool packed = kKvSplit && !kF32 && p.pack_lp > 0;       // head-packed query tiles
     volatile int *abort = &bar.abort;
     const uint64_t tmo = p.timeout_ns;
-    // The rotation warpgroup rescales O for the softmax (a correction
-    // warpgroup) when it relays no key tiles: keys pre-rotated or rotated once
-    // (and, split, split into their parts), bf16 operands, no rotation helpers.
-    // The softmax then only publishes each row's factor and goes on with its
-    // exponentials while the rescale runs beside them.
-    const bool corr = LCX_CORR_WG && !kF32 && !((kSplit && !p.k_x8_tma) || p.rotate_k) &&
-                      !p.rot_help;
 
     if (threadIdx.x == 0) {
         mbar_init(&bar.full_q, 1);
@@ -841,13 +836,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bar.empty_v[s], 1);
         }
         for (int t = 0; t < 2; ++t) {
-            mbar_init(&bar.s_ready[t], 1);
-            // the tile's four softmax warps hand over P, except the ones that
-            // help rotate keys
-            mbar_init(&bar.p_ready[t], 32 * (4 - __popc((p.rot_help >> (4 * t)) & 0xF)));
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&bar.s_ready[t][b], 1);
+                // the tile's four softmax warps hand over P, except the ones
+                // that help rotate keys
+                mbar_init(&bar.p_ready[t][b],
+                          32 * (4 - __popc((p.rot_help >> (4 * t)) & 0xF)));
+            }
+            mbar_init(&bar.pv_done[t], 1);
             mbar_init(&bar.o_ready[t], 1);
-            mbar_init(&bar.corr_req[t], 128);
-            mbar_init(&bar.corr_done[t], 128);
         }
         mbar_init(&bar.drain, 1);
         // A CTA that starts after another one's watchdog fired does no work.
@@ -884,7 +881,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if ((warp >> 2) == 3) {
-        // warpgroup 3: warp 12 issues the TMA copies, warp 13 the MMAs
+        // warpgroup 3: warps 12 and 14 issue the TMA copies (Q and K; V), warp 13
+        // the MMAs
         setmaxnreg_dec<kRegsIssue>();
         if (warp == kWarpTma) {
             // ------------------------------------------------ TMA producer
@@ -896,7 +894,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // With a shared rotary key, the K boxes from column D - RD on
                 // come from that tensor's single head.
                 constexpr int kNopeBoxes = (D - RD) / 64;
-                int issued_k[NSK] = {}, issued_v[NSV] = {};
+                int issued_k[NSK] = {};
                 if (packed) {
                     // each head's pack_lp rows at row k pack_lp of its tile (the Q
                     // map's box is pack_lp rows high; 8-row multiples keep the
@@ -920,7 +918,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bool ok = true;
                 for (int j = 0; ok && j < T.n; ++j) {
                     const int jt = T.tile(j);
-                    const int sk = j % NSK, uk = j / NSK, sv = j % NSV, uv = j / NSV;
+                    const int sk = j % NSK, uk = j / NSK;
                     if (uk > 0) ok = mbar_wait(&bar.empty_k[sk], (uk - 1) & 1, abort, tmo);
                     if (!ok) break;
                     // split mode with keys split by the rotate pass: the fp16 parts
@@ -945,6 +943,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_load_4d(dst, &tmk, &bar.full_k[sk], bx * 64, jt * BN, U.g, U.b);
                     }
                     ++issued_k[sk];
+                }
+                // Never leave the CTA with copies in flight: wait (bounded, even
+                // after an abort) for the last load issued to every buffer.
+                mbar_wait(&bar.full_q, 0, nullptr, tmo);
+                for (int s = 0; s < NSK; ++s)
+                    if (issued_k[s]) mbar_wait(&bar.full_k[s], (issued_k[s] - 1) & 1, nullptr, tmo);
+            }
+        } else if (warp == kWarpTmaV) {
+            // ------------------------------------------------ TMA producer of V
+            // V tiles come from their own warp, so a V stage that frees late (one
+            // V stage: after the last PV of the previous tile) never holds back the
+            // next K tile behind it.
+            if (!kF32 && lane == 0 && !p.test_stall) {
+                int issued_v[NSV] = {};
+                bool ok = true;
+                for (int j = 0; ok && j < T.n; ++j) {
+                    const int jt = T.tile(j);
+                    const int sv = j % NSV, uv = j / NSV;
                     if (uv > 0) ok = mbar_wait(&bar.empty_v[sv], (uv - 1) & 1, abort, tmo);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&bar.full_v[sv], C::kTileV);
@@ -953,11 +969,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     bx * 64, jt * BN, U.g, U.b);
                     ++issued_v[sv];
                 }
-                // Never leave the CTA with copies in flight: wait (bounded, even
-                // after an abort) for the last load issued to every buffer.
-                mbar_wait(&bar.full_q, 0, nullptr, tmo);
-                for (int s = 0; s < NSK; ++s)
-                    if (issued_k[s]) mbar_wait(&bar.full_k[s], (issued_k[s] - 1) & 1, nullptr, tmo);
                 for (int s = 0; s < NSV; ++s)
                     if (issued_v[s]) mbar_wait(&bar.full_v[s], (issued_v[s] - 1) & 1, nullptr, tmo);
             }
@@ -977,7 +988,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                   : idesc_bf16_f32(128, DV, 0, 1);
                 // V ready for PV: landed (TMA, or written by the fp32 loader), or
                 // converted to fp16 by the rotation warpgroup
-                uint64_t *vready = kConvV ? bar.fp16_v : bar.full_v;
+                uint64_t *vready = (kConvV && !p.v_f16) ? bar.fp16_v : bar.full_v;
                 const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
                 // S_t = Q_t K^T over D in steps of 16 (32 bytes inside a 128-byte
                 // swizzle row, then the next 64-column box).  Descriptors of the
@@ -987,10 +998,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t dk0 = sdesc_sw128(k_addr, 16, 1024);
                 const uint64_t dv0 = kTF ? sdesc_sw128(v_addr, 16, 1024)
                                          : sdesc_sw128(v_addr, C::kBoxK, 1024);
-                auto issue_s = [&](int t, int s) {
+                constexpr int NB = C::kNB;
+                auto issue_s = [&](int t, int s, int b) {
                     const uint64_t qa = dq0 + ((t * C::kParts * C::kTileQ) >> 4);
                     const uint64_t ka = dk0 + ((s * C::kParts * C::kTileK) >> 4);
-                    const uint32_t dst = tmem + t * BN;
+                    const uint32_t dst = tmem + (t * NB + b) * BN;
                     if constexpr (kSplit) {
                         // the e5m2 cross product first, into a fresh accumulator:
                         // [h8 | r8]_q [r8 | h8]_k^T over K = 2 D in steps of 32
@@ -1018,10 +1030,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // tf32); each instruction takes 32 bytes of keys per row of P (8
                 // TMEM columns).  bf16 V is MN-major (as many 128-byte rows of V
                 // per step); the tf32 tile is V^T, K-major (32 bytes of each row).
-                auto issue_pv = [&](int t, int s, bool acc) {
+                auto issue_pv = [&](int t, int s, int b, bool acc) {
                     const uint64_t va = dv0 + ((s * C::kTileV) >> 4);
                     const uint32_t dst = tmem + C::kColO + t * DV;
-                    const uint32_t pa = tmem + t * BN;
+                    const uint32_t pa = tmem + (t * NB + b) * BN;
                     constexpr int KS = 32 / C::ES;   // keys per instruction
 #pragma unroll
                     for (int kk = 0; kk < BN / KS; ++kk) {
@@ -1053,37 +1065,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = mbar_wait(&kready[j % NSK], (j / NSK) & 1, abort, tmo);
                         tc_fence_after();
                         if (!ok) break;
-                        issue_s(j, j % NSK);
-                        mma_commit(&bar.s_ready[j]);
+                        issue_s(j, j % NSK, 0);
+                        mma_commit(&bar.s_ready[j][0]);
                         mma_commit(&bar.empty_k[j % NSK]);
                     }
                     for (int j = 0; ok && j < T.n; ++j) {
                         const int t = j & 1, sv = j % NSV, jn = j + 2;
                         ok = mbar_wait(&vready[sv], (j / NSV) & 1, abort, tmo);
-                        if (ok) ok = mbar_wait(&bar.p_ready[t], (j >> 1) & 1, abort, tmo);
-                        if (ok && corr) ok = mbar_wait(&bar.corr_done[t], (j >> 1) & 1, abort, tmo);
+                        if (ok) ok = mbar_wait(&bar.p_ready[t][0], (j >> 1) & 1, abort, tmo);
                         tc_fence_after();
                         if (!ok) break;
-                        issue_pv(t, sv, j >= 2);
+                        issue_pv(t, sv, 0, j >= 2);
                         mma_commit(&bar.empty_v[sv]);
                         if (jn < T.n) {
                             const int sk = jn % NSK;
                             ok = mbar_wait(&kready[sk], (jn / NSK) & 1, abort, tmo);
                             tc_fence_after();
                             if (!ok) break;
-                            issue_s(t, sk);
-                            mma_commit(&bar.s_ready[t]);
+                            issue_s(t, sk, 0);
+                            mma_commit(&bar.s_ready[t][0]);
                             mma_commit(&bar.empty_k[sk]);
                         }
                     }
-                } else {
+                } else if constexpr (NB == 1) {
                     if (T.n > 0) {
                         ok = ok && mbar_wait(&kready[0], 0, abort, tmo);
                         tc_fence_after();
                         if (ok) {
                             for (int t = 0; t < U.nt; ++t) {
-                                issue_s(t, 0);
-                                mma_commit(&bar.s_ready[t]);
+                                issue_s(t, 0, 0);
+                                mma_commit(&bar.s_ready[t][0]);
                             }
                             mma_commit(&bar.empty_k[0]);
                         }
@@ -1092,11 +1103,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int sv = j % NSV, jn = j + 1;
                         ok = mbar_wait(&vready[sv], (j / NSV) & 1, abort, tmo);
                         for (int t = 0; ok && t < U.nt; ++t) {
-                            ok = mbar_wait(&bar.p_ready[t], j & 1, abort, tmo);
-                            if (ok && corr) ok = mbar_wait(&bar.corr_done[t], j & 1, abort, tmo);
+                            ok = mbar_wait(&bar.p_ready[t][0], j & 1, abort, tmo);
                             tc_fence_after();
                             if (!ok) break;
-                            issue_pv(t, sv, j > 0);
+                            issue_pv(t, sv, 0, j > 0);
                             if (jn < T.n) {
                                 const int sk = jn % NSK;
                                 if (t == 0) {
@@ -1104,13 +1114,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     tc_fence_after();
                                     if (!ok) break;
                                 }
-                                issue_s(t, sk);
-                                mma_commit(&bar.s_ready[t]);
+                                issue_s(t, sk, 0);
+                                mma_commit(&bar.s_ready[t][0]);
                             }
                         }
                         if (ok) {
                             mma_commit(&bar.empty_v[sv]);
                             if (jn < T.n) mma_commit(&bar.empty_k[jn % NSK]);
+                        }
+                    }
+                } else {
+                    // Two S buffers per query tile (the split mode's single tile):
+                    // S(j + 2) goes into the buffer P(j) held, right after PV(j),
+                    // so the softmax of key tile j + 1 can start while PV(j) and
+                    // S(j + 2) run; a softmax that rescales O first waits for the
+                    // previous PV (pv_done).
+                    for (int jj = 0; ok && jj < NB && jj < T.n; ++jj) {
+                        ok = mbar_wait(&kready[jj % NSK], (jj / NSK) & 1, abort, tmo);
+                        tc_fence_after();
+                        if (!ok) break;
+                        for (int t = 0; t < U.nt; ++t) {
+                            issue_s(t, jj % NSK, jj % NB);
+                            mma_commit(&bar.s_ready[t][jj % NB]);
+                        }
+                        mma_commit(&bar.empty_k[jj % NSK]);
+                    }
+                    for (int j = 0; ok && j < T.n; ++j) {
+                        const int sv = j % NSV, jn = j + NB, b = j % NB;
+                        ok = mbar_wait(&vready[sv], (j / NSV) & 1, abort, tmo);
+                        for (int t = 0; ok && t < U.nt; ++t) {
+                            ok = mbar_wait(&bar.p_ready[t][b], (j / NB) & 1, abort, tmo);
+                            tc_fence_after();
+                            if (!ok) break;
+                            issue_pv(t, sv, b, j > 0);
+                            mma_commit(&bar.pv_done[t]);
+                        }
+                        if (!ok) break;
+                        mma_commit(&bar.empty_v[sv]);
+                        if (jn < T.n) {
+                            const int sk = jn % NSK;
+                            ok = mbar_wait(&kready[sk], (jn / NSK) & 1, abort, tmo);
+                            tc_fence_after();
+                            if (!ok) break;
+                            for (int t = 0; t < U.nt; ++t) {
+                                issue_s(t, sk, b);
+                                mma_commit(&bar.s_ready[t][b]);
+                            }
+                            mma_commit(&bar.empty_k[sk]);
                         }
                     }
                 }
@@ -1168,23 +1218,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 relay_k = false;
             }
         }
-        // key tile j (when the keys pass through this warpgroup), then, split
-        // mode, value tile j converted to fp16, then the O rescales of the query
-        // tiles that take key tile j (correction warpgroup) -- the order the MMA
-        // needs them
-        const bool ilv = kKvSplit && p.pack_ilv;
-        for (int j = 0; ok && (relay_k || kConvV || corr) && j < T.n; ++j) {
+        for (int j = 0; ok && relay_k && j < T.n; ++j) {
             const int jt = T.tile(j);
             const int s = j % NSK, use = j / NSK, sv = j % NSV, usev = j / NSV;
             uint8_t *tk = sK + s * C::kParts * C::kTileK;
             if constexpr (!kF32) {
-                if (relay_k) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_k[s], use & 1, abort, tmo));
-                    if (!ok) break;
-                    if (rotk || kSplit)
-                        rotate_tile_bf16<D, RD, kHalf, kSplit, true, BN>(
-                            tk, tk + C::kTileK, (long long)jt * BN, ph, p, rotk, &kcarry);
-                }
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_k[s], use & 1, abort, tmo));
+                if (!ok) break;
+                if (rotk || kSplit)
+                    rotate_tile_bf16<D, RD, kHalf, kSplit, true, BN>(
+                        tk, tk + C::kTileK, (long long)jt * BN, ph, p, rotk, &kcarry);
             } else {
                 if (use > 0)
                     ok = __all_sync(0xffffffffu,
@@ -1196,46 +1239,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                                p.ks[2], jt * BN, p.Lk,
                                                                (long long)jt * BN, rotk, ph, p);
             }
-            if (relay_k) {
-                fence_proxy_async_smem();
-                mbar_arrive(&bar.ready_k[s]);
-            }
-            if constexpr (kConvV) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_v[sv], usev & 1, abort, tmo));
-                if (!ok) break;
-                bf16_tile_to_f16<C::kTileV>(sV + sv * C::kTileV, tw);
-                fence_proxy_async_smem();
-                mbar_arrive(&bar.fp16_v[sv]);
-            }
-            if (corr) {
-                // warp 8 + q serves TMEM lanes 32 q .. 32 q + 31 (its quadrant),
-                // the rows of softmax warps q and 4 + q
-                const int wq = warp - kWarpRot0;
-                const uint32_t trow = tmem + (uint32_t(wq * 32) << 16);
-                const int it = ilv ? (j >> 1) : j;
-                const int tb = ilv ? (j & 1) : 0, te = ilv ? (j & 1) + 1 : U.nt;
-                for (int t = tb; ok && t < te; ++t) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(&bar.corr_req[t], it & 1, abort, tmo));
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (reinterpret_cast<volatile int *>(bar.corr_need[t])[wq]) {
-                        const float alpha = tmem_ld1(trow + t * BN + BN - 1);
-                        const uint32_t o_col = C::kColO + t * DV;
-#pragma unroll 1
-                        for (int c = 0; c < DV / 32; ++c) {
-                            float o[32];
-                            tmem_ld32(trow + o_col + c * 32, o);
-                            uint32_t u[32];
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(o[e] * alpha);
-                            tmem_st32_nowait(trow + o_col + c * 32, u);
-                        }
-                        tmem_wait_st();
-                    }
-                    tc_fence_before();
-                    mbar_arrive(&bar.corr_done[t]);
-                }
-            }
+            fence_proxy_async_smem();
+            mbar_arrive(&bar.ready_k[s]);
             if constexpr (kF32) {
                 if (usev > 0)
                     ok = __all_sync(0xffffffffu,
@@ -1256,6 +1261,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int ord = __popc(p.rot_help & ((1u << warp) - 1u));
             rotate_keys_helped<D, RD, kHalf, kSplit, NSK, BN, C::kParts, C::kTileK>(
                 128 + 32 * ord + lane, T, sK, bar, p, abort, tmo);
+        } else if (kConvV && warp >= 4) {
+            // split mode: its one query tile leaves softmax warps 4-7 free; unless
+            // V arrives in fp16 already, they convert every V tile to fp16 for the
+            // PV product, in key-tile order
+            const int tw = threadIdx.x - 128;
+            bool ok = !p.v_f16;
+            for (int j = 0; ok && j < T.n; ++j) {
+                const int sv = j % NSV;
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar.full_v[sv], (j / NSV) & 1, abort, tmo));
+                if (!ok) break;
+                bf16_tile_to_f16<C::kTileV>(sV + sv * C::kTileV, tw);
+                fence_proxy_async_smem();
+                mbar_arrive(&bar.fp16_v[sv]);
+            }
         } else if ((warp >> 2) < U.nt) {
             // ------------------------------------------------ softmax, tile t
             // Warps 0-3 serve query tile 0 and warps 4-7 tile 1, one thread per
@@ -1281,17 +1300,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             // key tiles j = t mod 2 of the split and writes partial 2 split + t.
             const bool ilv = kKvSplit && p.pack_ilv;
             const int n_it = ilv ? (T.n - t + 1) / 2 : T.n;
+            constexpr int NB = C::kNB;
             for (int it = 0; it < n_it; ++it) {
                 const int j = ilv ? 2 * it + t : it;
-                const uint32_t s_col = t * BN;
-                ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_ready[t], it & 1, abort, tmo));
+                const int b = it % NB;
+                const uint32_t s_col = (t * NB + b) * BN;
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(&bar.s_ready[t][b], (it / NB) & 1, abort, tmo));
                 if (!ok) break;
                 if (idle) {
-                    if (corr) {
-                        if (lane == 0) bar.corr_need[t][wq] = 0;
-                        mbar_arrive(&bar.corr_req[t]);
-                    }
-                    mbar_arrive(&bar.p_ready[t]);
+                    mbar_arrive(&bar.p_ready[t][b]);
                     continue;
                 }
                 tc_fence_after();
@@ -1317,22 +1335,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // Keep the old reference unless the max grew by more than 2^15: the
                 // result is exact either way, only O's rescale is saved.
                 const bool need = (m != -INFINITY) && (m_new > m + kRescaleLog2);
-                if (corr) {
-                    // publish the warp's need and each row's factor (in the last
-                    // column of S_t, free once S is in registers and outside P)
-                    // for the rotation warpgroup, which rescales O_t meanwhile
-                    const bool any = __any_sync(0xffffffffu, need);
-                    if (lane == 0) bar.corr_need[t][wq] = any ? 1 : 0;
-                    if (any) tmem_st1(trow + s_col + BN - 1, need ? ex2_approx(m - m_new) : 1.f);
-                    tc_fence_before();
-                    mbar_arrive(&bar.corr_req[t]);
-                    if (need) {
-                        l *= ex2_approx(m - m_new);
-                        m = m_new;
+                if (__any_sync(0xffffffffu, need)) {
+                    if (NB > 1) {
+                        // O_t must not be in flight: wait for PV_t(j - 1), the j-th
+                        // completion of pv_done (S_t(j) done implies PV_t(j - 2)
+                        // was, and PV_t(j) needs this tile's P, so no other phase
+                        // can be pending).  With one S buffer, S_t(j) is issued
+                        // after PV_t(j - 1), so its completion implies it.
+                        ok = __all_sync(0xffffffffu,
+                                        mbar_wait(&bar.pv_done[t], (it - 1) & 1, abort, tmo));
+                        if (!ok) break;
+                        tc_fence_after();
                     }
-                } else if (__any_sync(0xffffffffu, need)) {
-                    // O_t is not in flight: S_t(j) is issued after PV_t(j - 1), so
-                    // its completion implies PV_t(j - 1)'s.
                     const float alpha = need ? ex2_approx(m - m_new) : 1.f;
                     // chunk by chunk; the stores are not waited for one by one,
                     // only once before P is handed over
@@ -1389,9 +1403,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                         if (kPF16) {
                             // fp16 weights (11 significant bits; at most 2^15 with
-                            // the stale reference, far inside fp16's range)
+                            // the stale reference, inside fp16's range).  Summed
+                            // before rounding: an fp16 weight is within 2^-12 of
+                            // its fp32 value, and unpacking every pair would put
+                            // two more conversions per pair on the pipe the
+                            // exponentials use.
                             pk[e] = pack_f16x2(pe.x, pe.y);
-                            lsum = add2(lsum, f16x2_to_f32x2(pk[e]));
+                            lsum = add2(lsum, pe);
                         } else if (kSplit) {
                             pk[e] = pack_bf16x2(pe.x, pe.y);
                             // Normalise by the weights the tensor core actually
@@ -1409,7 +1427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 l += lsum.x + lsum.y;
                 tc_fence_before();
-                mbar_arrive(&bar.p_ready[t]);
+                mbar_arrive(&bar.p_ready[t][b]);
             }
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.o_ready[t], 0, abort, tmo));
             if (ok) {
@@ -1586,6 +1604,9 @@ struct AttnLaunch : AttnLaunchShape {
     const void *k_src;
     int64_t k_src_strides[4];
     void *k_x8;       // split mode: where the pass writes the keys' 8-bit cross parts, or NULL
+    void *v16;        // split mode: where a pass writes V in fp16 (contiguous), or NULL
+    const void *v_src;
+    int64_t v_src_strides[4];
     int rot_h, rot_d; // heads and columns the pass rotates (Hkv, D; or 1, d_R)
     void *k_rot;      // where the pass writes
 };
@@ -1663,7 +1684,9 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     // rotary key of decoupled RoPE ([B, 1, Lk, d_R]; k keeps its un-rotated
     // columns).  In the split-QK^T mode with bf16 keys the pass writes the
     // keys' fp16 parts there, followed by their 8-bit cross parts ([r8 | h8],
-    // 2 D bytes per key: as many bytes again).
+    // 2 D bytes per key: as many bytes again), and a second pass the values in
+    // fp16 (as many bytes again), so the kernel loads every PV operand as it
+    // multiplies it.
     const bool rot_shared = partial && a->k_rope != nullptr;
     const bool rotate_k_once =
         a->k_rot != nullptr && !(a->flags & (LCX_ATTN_PREROTATED | LCX_ATTN_PREROTATED_K |
@@ -1675,11 +1698,12 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     const int64_t k_part_bytes = a->B * rot_h * Lk * rot_d * es;
     if (rotate_k_once) {
         if (!aligned16(a->k_rot)) return fail(LCX_ERR_UNSUPPORTED, "k_rot must be 16-byte aligned");
-        if (a->k_rot_bytes < k_part_bytes * (k_x8 ? 2 : 1))
+        if (a->k_rot_bytes < k_part_bytes * (k_x8 ? 3 : 1))
             return fail(LCX_ERR_INVALID_ARG, "k_rot holds %lld bytes; %lld needed",
-                        (long long)a->k_rot_bytes, (long long)(k_part_bytes * (k_x8 ? 2 : 1)));
+                        (long long)a->k_rot_bytes, (long long)(k_part_bytes * (k_x8 ? 3 : 1)));
     }
     void *k_x8_ptr = k_x8 ? static_cast<char *>(a->k_rot) + k_part_bytes : nullptr;
+    void *v16_ptr = k_x8 ? static_cast<char *>(a->k_rot) + 2 * k_part_bytes : nullptr;
     const bool k_from_rot = rotate_k_once && !rot_shared;   // k itself read from k_rot
     const void *kptr = k_from_rot ? a->k_rot : a->k;
     const int64_t *kst = k_from_rot ? kst_rot : a->k_strides;
@@ -1687,6 +1711,9 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     memset(&x, 0, sizeof(x));
     x.rotate_k_once = rotate_k_once;
     x.k_x8 = k_x8_ptr;
+    x.v16 = v16_ptr;
+    x.v_src = a->v;
+    for (int d = 0; d < 4; ++d) x.v_src_strides[d] = a->v_strides[d];
     x.rope = a->rope;
     x.k_src = rot_shared ? a->k_rope : a->k;
     for (int d = 0; d < 4; ++d)
@@ -1719,9 +1746,11 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     p.window = int(a->window > Lk ? Lk : a->window);
     p.sinks = int(a->sinks > Lk ? Lk : a->sinks);
     // Two query heads share a CTA's K/V tiles when the group allows it and the
-    // CTA holds two query tiles (at D = 192 only with LCX_D192_TWO_TILES); with
-    // an odd group the two tiles are consecutive query blocks of one head.
-    const bool two_tiles = a->D <= 128 || LCX_D192_TWO_TILES;
+    // CTA holds two query tiles (at D = 192 only with LCX_D192_TWO_TILES; never
+    // in the split mode, whose CTA holds one tile with two S buffers); with an
+    // odd group the two tiles are consecutive query blocks of one head.
+    const bool two_tiles =
+        (a->D <= 128 || LCX_D192_TWO_TILES) && !(a->flags & LCX_ATTN_SPLIT_QK);
     p.heads_per_unit = (p.G % 2 == 0 && two_tiles) ? 2 : 1;
     p.qpair = (p.G % 2 == 1 && two_tiles) ? 1 : 0;
     p.n_qb = int((a->L + (p.qpair ? 2 * kBM : kBM) - 1) / (p.qpair ? 2 * kBM : kBM));
@@ -1750,6 +1779,7 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     p.c_log2 = float(scale * msq * 1.4426950408889634);
     p.k_rope_shared = a->k_rope ? 1 : 0;
     p.k_x8_tma = k_x8 ? 1 : 0;
+    p.v_f16 = v16_ptr ? 1 : 0;
     // Legitimate waits last microseconds; the default limit is 2 s.
     p.timeout_ns = 1000000ull * (unsigned long long)(a->watchdog_ms > 0 ? a->watchdog_ms : 2000);
     p.test_stall = (a->flags & LCX_ATTN_TEST_STALL) ? 1 : 0;
@@ -1774,7 +1804,10 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
             return st;
         if ((st = make_map(&x.m.k, kptr, a->B, a->Hkv, Lk, dk, kst, bn, "k")) != LCX_OK)
             return st;
-        if ((st = make_map(&x.m.v, a->v, a->B, a->Hkv, Lk, Dv, a->v_strides, bn, "v")) != LCX_OK)
+        // V, or (split mode with the key buffer) its contiguous fp16 copy
+        const int64_t v16_st[4] = {a->Hkv * Lk * Dv, Lk * Dv, Dv, 1};
+        if ((st = make_map(&x.m.v, v16_ptr ? v16_ptr : a->v, a->B, a->Hkv, Lk, Dv,
+                           v16_ptr ? v16_st : a->v_strides, bn, "v")) != LCX_OK)
             return st;
         if (k_x8) {
             // the keys' 8-bit cross parts: [B, Hkv, Lk, 2 D] bytes, boxes of
@@ -1810,10 +1843,14 @@ lcx_status attn_enqueue(const AttnLaunch &x, cudaStream_t s) {
         if (rp.seq_len <= 0) rp.seq_len = x.p.Lk;   // the context of the call, as the kernel's
         const int64_t kst[4] = {(int64_t)x.rot_h * x.p.Lk * x.rot_d, (int64_t)x.p.Lk * x.rot_d,
                                 x.rot_d, 1};
-        const lcx_status st =
+        lcx_status st =
             apply_rope_impl(&rp, x.k_src, x.k_rot, x.k_x8, x.f32 ? LCX_F32 : LCX_BF16, x.p.B,
                             x.rot_h, x.p.Lk, x.k_src_strides, kst, 0, s);
         if (st != LCX_OK) return st;
+        if (x.v16) {
+            st = bf16_to_f16_impl(x.v_src, x.v_src_strides, x.v16, x.p.B, x.p.Hkv, x.p.Lk, x.DV, s);
+            if (st != LCX_OK) return st;
+        }
     }
     const unsigned g = unsigned(grid);
     return x.p.n_split > 1 ? launch_shape<true>(x, x.m, x.p, g, s)
@@ -1895,9 +1932,19 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
     //  - otherwise (fp32, or G pack_lp > 128), G even and
     //    G/2 pack_lp <= 128: G/2 heads per tile, both tiles multiply every key
     //    tile.
+    //  - split QK^T (one query tile per CTA): all G heads in that tile when
+    //    G pack_lp <= 128, its two S buffers walking the key tiles in turn.
     const int64_t lp = (a->L + 7) / 8 * 8;
     int n_parts = num_splits;
-    if (!x.f32 && x.D <= 128 && lp * x.p.G <= kBM) {
+    if (x.split_qk) {
+        // one query tile per CTA: all G heads in it when they fit
+        if (!x.f32 && lp * x.p.G <= kBM) {
+            x.p.pack_lp = int(lp);
+            x.p.pack_hpt = x.p.G;
+            x.p.pack_stride = int(lp);
+            x.p.pack_off = 0;
+        }
+    } else if (!x.f32 && x.D <= 128 && lp * x.p.G <= kBM) {
         const int used = int(lp) * x.p.G;
         x.p.pack_lp = int(lp);
         x.p.pack_hpt = x.p.G;

@@ -41,6 +41,11 @@ lcx_status apply_rope_impl(const lcx_rope_params *params, const void *x, void *y
                            const int64_t *x_strides, const int64_t *y_strides, int64_t pos_offset,
                            cudaStream_t stream);
 
+// Contiguous fp16 copy of a bf16 [B, H, L, D] tensor (element strides, the last
+// one 1), values converted exactly where fp16 holds them (the split mode's V).
+lcx_status bf16_to_f16_impl(const void *x, const int64_t *x_strides, void *y, int64_t B,
+                            int64_t H, int64_t L, int64_t D, cudaStream_t stream);
+
 // Enqueue the merge of n_parts partial results ([n_parts, B, Hq, L, D] fp32 o,
 // [n_parts, B, Hq, L] fp32 lse) into o (dtype, strides) and optionally lse.
 // Arguments are assumed valid.

@@ -173,6 +173,18 @@ __device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint
         : "memory");
 }
 
+// D(tmem) = A(tmem) x B(smem) (+ D if accumulate), kind::f8f6f4 (A: 4 elements
+// per 32-bit TMEM column).
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // D(tmem) = A(smem) x B(smem) (+ D if accumulate), kind::tf32 (fp32 storage,
 // 10-bit mantissa used; K = 8 per instruction).
 __device__ __forceinline__ void mma_ss_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -255,26 +267,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
         : "memory");
 #pragma unroll
     for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(u[i]);
-}
-
-// One 32-bit TMEM column of 32 lanes (thread t reads lane base + t), then wait.
-__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
-    uint32_t u;
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(u)
-        : "r"(taddr)
-        : "memory");
-    return __uint_as_float(u);
-}
-// One 32-bit value per thread -> one TMEM column of 32 lanes, then wait.
-__device__ __forceinline__ void tmem_st1(uint32_t taddr, float x) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};\n\t"
-        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-        "r"(__float_as_uint(x))
-        : "memory");
 }
 
 // 32 lanes x 64 columns of 32-bit TMEM -> 64 registers per thread, one wait.

@@ -244,6 +244,9 @@ def _attn_args(**kw):
     (dict(D=192, rope=_params("plain", 192)), lcx.LCX_ERR_UNSUPPORTED),
     (dict(k_rot=0x500008, k_rot_bytes=1 << 30), lcx.LCX_ERR_UNSUPPORTED),  # misaligned
     (dict(k_rot=0x500000, k_rot_bytes=1000), lcx.LCX_ERR_INVALID_ARG),      # too small
+    # split QK^T with bf16: the keys' fp16 parts, their cross parts and V in fp16
+    # (three times the keys' 131072 bytes); twice is too small
+    (dict(k_rot=0x500000, k_rot_bytes=2 * 131072, flags=2), lcx.LCX_ERR_INVALID_ARG),
     (dict(D=192, Dv=128, rope=_params("plain", 64), k_rope=0x500008,
           k_rope_strides=[256 * 64, 256 * 64, 64, 1]), lcx.LCX_ERR_UNSUPPORTED),  # misaligned
     # the shared rotary key rotated once: k_rot must hold [B, 1, Lk, 64]
