@@ -182,17 +182,28 @@ struct Cfg {
                                   : (D == 64) ? 4
                                   : (D == 128) ? LCX_KSTAGES_D128
                                   : (kNTQ == 2) ? 1 : 2;
-    static constexpr int kStagesV = kSplit ? (D == 64 ? 3 : 1) : kTF ? 2 : (D == 64) ? 4 : 2;
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kNTQ * kParts * kTileQ;
+    static constexpr int kStagesV = kSplit ? 3 : kTF ? 2 : (D == 64) ? 4 : 2;
+    // Split mode: the query tile's two parts are the A operands of QK^T from
+    // TMEM, so its shared-memory copy is only a staging area for the rotation
+    // and the last K stage reuses it once the parts have moved to TMEM.
+    static constexpr bool kQT = kSplit;
+    static constexpr int kOffK = kQT ? 0 : kNTQ * kParts * kTileQ;
+    static constexpr int kOffQ = kQT ? kOffK + (kStagesK - 1) * kParts * kTileK : 0;
     static constexpr int kOffV = kOffK + kStagesK * kParts * kTileK;
     static constexpr int kOffBar = kOffV + kStagesV * kTileV;
     static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers + alignment slack
     // TMEM columns: S_t,b at (t kNB + b) BN (P_t,b aliased over its first BN/2
-    // columns, or all of it with tf32), then O_t.
+    // columns, or all of it with tf32), then O_t, then (split mode) the query
+    // tile's fp16 part (D/2 columns, two values each) and its 8-bit cross part
+    // (D/2 columns, four bytes each).
+    // With as many K stages as S buffers, the completion of S(j) (s_ready of
+    // buffer j mod kNB) is also the release of K stage j mod kStagesK.
+    static constexpr bool kKFreeOnS = kNB > 1 && kStagesK == kNB;
     static constexpr int kColO = kNTQ * kNB * BN;
+    static constexpr int kColQ = kColO + kNTQ * DV;
+    static_assert(!kQT || (kNTQ == 1 && kTileQ == kTileK), "query staging in a K stage");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
-    static_assert(kColO + kNTQ * DV <= 512, "TMEM budget");
+    static_assert(kColQ + (kQT ? D : 0) <= 512, "TMEM budget");
 };
 
 template <int NSK, int NSV>
@@ -200,7 +211,7 @@ struct Bars {
     uint64_t full_q, ready_q;
     uint64_t full_k[NSK], ready_k[NSK], empty_k[NSK];
     uint64_t full_v[NSV], empty_v[NSV], fp16_v[NSV];
-    uint64_t s_ready[2][2], p_ready[2][2], pv_done[2], o_ready[2];
+    uint64_t s_ready[2][2], p_ready[2][2], o_ready[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -397,6 +408,36 @@ __device__ __forceinline__ void store8(uint8_t *tile, uint8_t *x8, int r, int fc
         *reinterpret_cast<uint2 *>(x8 + byte_off(r, kKey ? D + c : c, BOX)) = h8;
         *reinterpret_cast<uint2 *>(x8 + byte_off(r, kKey ? c : D + c, BOX)) = r8;
     }
+}
+
+// Copy row r of a split-mode query tile into TMEM lane r (taddr: the lane's
+// address at the first query column): the fp16 part (128-byte swizzled rows,
+// D/64 boxes) to D/2 columns of two values, then the 8-bit cross part (2 D
+// bytes, as many boxes) to D/2 columns of four bytes, both in K order with the
+// lower index in the lower bits -- the A-operand layout of the TMEM form of the
+// MMA, 32 bytes of K (8 columns) per instruction.
+template <int D, int BOX>
+__device__ __forceinline__ void q_parts_to_tmem(const uint8_t *hi, const uint8_t *x8, int r,
+                                                uint32_t taddr) {
+#pragma unroll 1
+    for (int part = 0; part < 2; ++part) {
+        const uint8_t *src = part ? x8 : hi;
+#pragma unroll 1
+        for (int g = 0; g < D / 64; ++g) {
+            uint32_t u[32];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 w =
+                    *reinterpret_cast<const uint4 *>(src + chunk_off(r, g * 8 + c, BOX));
+                u[4 * c] = w.x;
+                u[4 * c + 1] = w.y;
+                u[4 * c + 2] = w.z;
+                u[4 * c + 3] = w.w;
+            }
+            tmem_st32_nowait(taddr + part * (D / 2) + g * 32, u);
+        }
+    }
+    tmem_wait_st();
 }
 
 // Per-thread phasor state of the rotation warpgroup: the thread always handles
@@ -807,7 +848,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // Q part x of tile t at sQ + (t * kParts + x) * kTileQ; K part x of stage s at
+    // Q part x of tile t at sQ + (t * kParts + x) * kTileQ (split mode: staging
+    // in the last K stage); K part x of stage s at
     // sK + (s * kParts + x) * kTileK; V stage s at sV + s * kTileK.
     uint8_t *sQ = smem + C::kOffQ;
     uint8_t *sK = smem + C::kOffK;
@@ -840,10 +882,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_init(&bar.s_ready[t][b], 1);
                 // the tile's four softmax warps hand over P, except the ones
                 // that help rotate keys
-                mbar_init(&bar.p_ready[t][b],
-                          32 * (4 - __popc((p.rot_help >> (4 * t)) & 0xF)));
+                mbar_init(&bar.p_ready[t][b], 32 * (4 - __popc((p.rot_help >> (4 * t)) & 0xF)));
             }
-            mbar_init(&bar.pv_done[t], 1);
             mbar_init(&bar.o_ready[t], 1);
         }
         mbar_init(&bar.drain, 1);
@@ -919,7 +959,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int j = 0; ok && j < T.n; ++j) {
                     const int jt = T.tile(j);
                     const int sk = j % NSK, uk = j / NSK;
-                    if (uk > 0) ok = mbar_wait(&bar.empty_k[sk], (uk - 1) & 1, abort, tmo);
+                    if (uk > 0)
+                        ok = mbar_wait(C::kKFreeOnS ? &bar.s_ready[0][sk] : &bar.empty_k[sk],
+                                       (uk - 1) & 1, abort, tmo);
+                    // the last K stage is the query tile's staging area until its
+                    // parts are in TMEM
+                    if (C::kQT && j == NSK - 1) ok = ok && mbar_wait(&bar.ready_q, 0, abort, tmo);
                     if (!ok) break;
                     // split mode with keys split by the rotate pass: the fp16 parts
                     // come through tmk, the 8-bit cross parts (fourth tensor map,
@@ -994,36 +1039,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // swizzle row, then the next 64-column box).  Descriptors of the
                 // first K step; later steps only move the start address (in
                 // 16-byte units, well inside the 14-bit field).
+                // All descriptors share their upper word (1024-byte stride), so
+                // the loops below carry only the lower words.
                 const uint64_t dq0 = sdesc_sw128(q_addr, 16, 1024);
-                const uint64_t dk0 = sdesc_sw128(k_addr, 16, 1024);
-                const uint64_t dv0 = kTF ? sdesc_sw128(v_addr, 16, 1024)
-                                         : sdesc_sw128(v_addr, C::kBoxK, 1024);
+                const uint32_t dhi = uint32_t(dq0 >> 32);
+                const uint32_t q_lo = uint32_t(dq0);
+                const uint32_t k_lo = uint32_t(sdesc_sw128(k_addr, 16, 1024));
+                const uint32_t v_lo = uint32_t(kTF ? sdesc_sw128(v_addr, 16, 1024)
+                                                   : sdesc_sw128(v_addr, C::kBoxK, 1024));
                 constexpr int NB = C::kNB;
                 auto issue_s = [&](int t, int s, int b) {
-                    const uint64_t qa = dq0 + ((t * C::kParts * C::kTileQ) >> 4);
-                    const uint64_t ka = dk0 + ((s * C::kParts * C::kTileK) >> 4);
+                    const uint32_t ka = k_lo + ((s * C::kParts * C::kTileK) >> 4);
                     const uint32_t dst = tmem + (t * NB + b) * BN;
-                    if constexpr (kSplit) {
-                        // the e5m2 cross product first, into a fresh accumulator:
-                        // [h8 | r8]_q [r8 | h8]_k^T over K = 2 D in steps of 32
-                        // bytes -- the same byte walk as the 16-bit product (loops
-                        // not unrolled: the issuing warp has 64 registers)
-#pragma unroll 1
+                    if constexpr (C::kQT) {
+                        // Split mode, query parts in TMEM (8 columns = 32 bytes of
+                        // K per instruction): the e5m2 cross product first, into a
+                        // fresh accumulator, [h8 | r8]_q [r8 | h8]_k^T over K = 2 D,
+                        // then the fp16 product on top of it.
+                        const uint32_t qh = tmem + C::kColQ, qx = qh + D / 2;
+#pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t ok_ = ((kk >> 2) * C::kBoxK + (kk & 3) * 32) >> 4;
+                            mma_ts_w<1>(dst, qx + kk * 8, ka + (C::kTileK >> 4) + ok_, dhi, kIdX8,
+                                        kk > 0);
+                        }
+#pragma unroll
+                        for (int kk = 0; kk < C::kKSteps; ++kk) {
+                            const uint32_t ok_ = ((kk >> 2) * C::kBoxK + (kk & 3) * 32) >> 4;
+                            mma_ts_w<0>(dst, qh + kk * 8, ka + ok_, dhi, kIdS, 1);
+                        }
+                    } else {
+                        const uint32_t qa = q_lo + ((t * C::kParts * C::kTileQ) >> 4);
+#pragma unroll
+                        for (int kk = 0; kk < C::kKSteps; ++kk) {
                             const uint32_t oq = ((kk >> 2) * C::kBoxQ + (kk & 3) * 32) >> 4;
                             const uint32_t ok_ = ((kk >> 2) * C::kBoxK + (kk & 3) * 32) >> 4;
-                            mma_ss_f8(dst, qa + (C::kTileQ >> 4) + oq, ka + (C::kTileK >> 4) + ok_,
-                                      kIdX8, kk > 0);
+                            mma_ss_w<kTF ? 2 : 0>(dst, qa + oq, ka + ok_, dhi, kIdS, kk > 0);
                         }
-                    }
-#pragma unroll(kSplit ? 1 : C::kKSteps)
-                    for (int kk = 0; kk < C::kKSteps; ++kk) {
-                        const uint32_t oq = ((kk >> 2) * C::kBoxQ + (kk & 3) * 32) >> 4;
-                        const uint32_t ok_ = ((kk >> 2) * C::kBoxK + (kk & 3) * 32) >> 4;
-                        if constexpr (kTF)
-                            mma_ss_tf32(dst, qa + oq, ka + ok_, kIdS, kk > 0);
-                        else
-                            mma_ss(dst, qa + oq, ka + ok_, kIdS, kSplit || kk > 0);
                     }
                 };
                 // O_t += P_t V: P from TMEM (BN/2 columns of bf16 pairs, or BN of
@@ -1031,20 +1083,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // TMEM columns).  bf16 V is MN-major (as many 128-byte rows of V
                 // per step); the tf32 tile is V^T, K-major (32 bytes of each row).
                 auto issue_pv = [&](int t, int s, int b, bool acc) {
-                    const uint64_t va = dv0 + ((s * C::kTileV) >> 4);
+                    const uint32_t va = v_lo + ((s * C::kTileV) >> 4);
                     const uint32_t dst = tmem + C::kColO + t * DV;
                     const uint32_t pa = tmem + (t * NB + b) * BN;
                     constexpr int KS = 32 / C::ES;   // keys per instruction
 #pragma unroll
                     for (int kk = 0; kk < BN / KS; ++kk) {
-                        if constexpr (kTF)
-                            // K-major V^T: 32 keys per box row, four 8-key steps per box
-                            mma_ts_tf32(dst, pa + kk * 8,
-                                        va + ((((kk >> 2) * DV * 128) + (kk & 3) * 32) >> 4),
-                                        kIdPV, (acc || kk > 0));
-                        else
-                            mma_ts(dst, pa + kk * 8, va + ((kk * KS * 128) >> 4), kIdPV,
-                                   (acc || kk > 0));
+                        // K-major V^T (tf32): 32 keys per box row, four 8-key steps
+                        // per box; MN-major V: KS rows of 128 bytes per step
+                        const uint32_t ov = kTF ? ((((kk >> 2) * DV * 128) + (kk & 3) * 32) >> 4)
+                                                : ((kk * KS * 128) >> 4);
+                        mma_ts_w<kTF ? 2 : 0>(dst, pa + kk * 8, va + ov, dhi, kIdPV,
+                                              (acc || kk > 0));
                     }
                 };
                 // S_t(j + 1) is issued after PV_t(j), into the buffer P_t(j)
@@ -1124,43 +1174,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 } else {
-                    // Two S buffers per query tile (the split mode's single tile):
-                    // S(j + 2) goes into the buffer P(j) held, right after PV(j),
-                    // so the softmax of key tile j + 1 can start while PV(j) and
-                    // S(j + 2) run; a softmax that rescales O first waits for the
-                    // previous PV (pv_done).
+                    // Two S buffers (the split mode's single query tile): S(j + 2)
+                    // goes into the buffer P(j) held, right after PV(j), so the
+                    // softmax of key tile j + 1 runs while PV(j) and S(j + 2) do.
+                    // Every wait of iteration j comes before PV(j), so PV(j) and
+                    // S(j + 2) reach the tensor core back to back.  PV(j)'s
+                    // completion is signalled once, on its V stage's barrier (a
+                    // softmax that rescales O waits there); with as many K stages
+                    // as S buffers, S(j)'s completion also frees its K stage.
+                    static_assert(C::kNTQ == 1, "one query tile with two S buffers");
                     for (int jj = 0; ok && jj < NB && jj < T.n; ++jj) {
                         ok = mbar_wait(&kready[jj % NSK], (jj / NSK) & 1, abort, tmo);
                         tc_fence_after();
                         if (!ok) break;
-                        for (int t = 0; t < U.nt; ++t) {
-                            issue_s(t, jj % NSK, jj % NB);
-                            mma_commit(&bar.s_ready[t][jj % NB]);
-                        }
-                        mma_commit(&bar.empty_k[jj % NSK]);
+                        issue_s(0, jj % NSK, jj % NB);
+                        mma_commit(&bar.s_ready[0][jj % NB]);
+                        if (!C::kKFreeOnS) mma_commit(&bar.empty_k[jj % NSK]);
                     }
                     for (int j = 0; ok && j < T.n; ++j) {
-                        const int sv = j % NSV, jn = j + NB, b = j % NB;
-                        ok = mbar_wait(&vready[sv], (j / NSV) & 1, abort, tmo);
-                        for (int t = 0; ok && t < U.nt; ++t) {
-                            ok = mbar_wait(&bar.p_ready[t][b], (j / NB) & 1, abort, tmo);
-                            tc_fence_after();
-                            if (!ok) break;
-                            issue_pv(t, sv, b, j > 0);
-                            mma_commit(&bar.pv_done[t]);
+                        const int sv = j % NSV, jn = j + NB, b = j % NB, sk = jn % NSK;
+                        // The three phases are polled together first: each test's
+                        // result takes ~100 cycles to come back, so polling them
+                        // one after the other would keep the tensor core waiting.
+                        const bool kr = jn >= T.n || mbar_try_wait(&kready[sk], (jn / NSK) & 1);
+                        const bool all = kr & mbar_try_wait(&vready[sv], (j / NSV) & 1) &
+                                         mbar_try_wait(&bar.p_ready[0][b], (j / NB) & 1);
+                        if (!all) {
+                            if (jn < T.n) ok = mbar_wait(&kready[sk], (jn / NSK) & 1, abort, tmo);
+                            if (ok) ok = mbar_wait(&vready[sv], (j / NSV) & 1, abort, tmo);
+                            if (ok) ok = mbar_wait(&bar.p_ready[0][b], (j / NB) & 1, abort, tmo);
                         }
+                        tc_fence_after();
                         if (!ok) break;
+                        issue_pv(0, sv, b, j > 0);
                         mma_commit(&bar.empty_v[sv]);
                         if (jn < T.n) {
-                            const int sk = jn % NSK;
-                            ok = mbar_wait(&kready[sk], (jn / NSK) & 1, abort, tmo);
-                            tc_fence_after();
-                            if (!ok) break;
-                            for (int t = 0; t < U.nt; ++t) {
-                                issue_s(t, sk, b);
-                                mma_commit(&bar.s_ready[t][b]);
-                            }
-                            mma_commit(&bar.empty_k[sk]);
+                            issue_s(0, sk, b);
+                            mma_commit(&bar.s_ready[0][b]);
+                            if (!C::kKFreeOnS) mma_commit(&bar.empty_k[sk]);
                         }
                     }
                 }
@@ -1204,6 +1255,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                                  rotq, ph, p);
             }
         }
+        if constexpr (C::kQT) {
+            // the query tile's parts move to TMEM (A operands of QK^T); the
+            // staging area then serves as the last K stage.  Each thread copies
+            // one row, which other threads of the warpgroup rotated.
+            named_bar_sync(1, 128);
+            if (ok) {
+                const uint8_t *qt = sQ;
+                q_parts_to_tmem<D, C::kBoxQ>(qt, qt + C::kTileQ, tw,
+                                             tmem + (uint32_t((warp & 3) * 32) << 16) + C::kColQ);
+                tc_fence_before();
+            }
+            named_bar_sync(1, 128);   // every row copied before keys overwrite the area
+        }
         if (ok) {
             fence_proxy_async_smem();
             mbar_arrive(&bar.ready_q);
@@ -1231,7 +1295,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
                 if (use > 0)
                     ok = __all_sync(0xffffffffu,
-                                    mbar_wait(&bar.empty_k[s], (use - 1) & 1, abort, tmo));
+                                    mbar_wait(C::kKFreeOnS ? &bar.s_ready[0][s] : &bar.empty_k[s],
+                                              (use - 1) & 1, abort, tmo));
                 if (!ok) break;
                 const float *base = reinterpret_cast<const float *>(p.k) + U.b * p.ks[0] +
                                     (long long)U.g * p.ks[1];
@@ -1337,13 +1402,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool need = (m != -INFINITY) && (m_new > m + kRescaleLog2);
                 if (__any_sync(0xffffffffu, need)) {
                     if (NB > 1) {
-                        // O_t must not be in flight: wait for PV_t(j - 1), the j-th
-                        // completion of pv_done (S_t(j) done implies PV_t(j - 2)
-                        // was, and PV_t(j) needs this tile's P, so no other phase
-                        // can be pending).  With one S buffer, S_t(j) is issued
-                        // after PV_t(j - 1), so its completion implies it.
+                        // O must not be in flight: wait for PV(j - 1), whose
+                        // completion is signalled on its V stage's barrier (S(j)
+                        // done implies PV(j - 2) was, and PV(j) needs this tile's
+                        // P, so no other phase of that barrier can be pending).
+                        // With one S buffer, S_t(j) is issued after PV_t(j - 1), so
+                        // its completion implies it.
                         ok = __all_sync(0xffffffffu,
-                                        mbar_wait(&bar.pv_done[t], (it - 1) & 1, abort, tmo));
+                                        mbar_wait(&bar.empty_v[(it - 1) % NSV],
+                                                  ((it - 1) / NSV) & 1, abort, tmo));
                         if (!ok) break;
                         tc_fence_after();
                     }

@@ -132,6 +132,12 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
                  : "memory");
 }
 
+// Barrier among `count` threads (whole warps) on hardware barrier `id` (0 is
+// __syncthreads').
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -159,6 +165,42 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// The same MMAs with the shared-memory descriptors passed as their lower 32-bit
+// words: every 128-byte-swizzle descriptor with a 1024-byte stride has the same
+// upper word (stride, version, layout), so an issuing loop keeps one register
+// per operand and steps it by immediates.  K in {0: kind::f16, 1: kind::f8f6f4,
+// 2: kind::tf32}.
+template <int K>
+__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
+                                         uint32_t idesc, uint32_t accumulate) {
+#define LCX_MMA_SS_W(KIND)                                                                 \
+    asm volatile("{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"                           \
+                 "mov.b64 da, {%1, %3};\n\tmov.b64 db, {%2, %3};\n\t"                      \
+                 "setp.ne.b32 p, %5, 0;\n\t"                                               \
+                 "tcgen05.mma.cta_group::1.kind::" KIND " [%0], da, db, %4, p;\n\t}" ::"r"(d_tmem), \
+                 "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)                 \
+                 : "memory")
+    if constexpr (K == 0) LCX_MMA_SS_W("f16");
+    else if constexpr (K == 1) LCX_MMA_SS_W("f8f6f4");
+    else LCX_MMA_SS_W("tf32");
+#undef LCX_MMA_SS_W
+}
+template <int K>
+__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t hi,
+                                         uint32_t idesc, uint32_t accumulate) {
+#define LCX_MMA_TS_W(KIND)                                                                 \
+    asm volatile("{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"                                 \
+                 "mov.b64 db, {%2, %3};\n\t"                                               \
+                 "setp.ne.b32 p, %5, 0;\n\t"                                               \
+                 "tcgen05.mma.cta_group::1.kind::" KIND " [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem), \
+                 "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)               \
+                 : "memory")
+    if constexpr (K == 0) LCX_MMA_TS_W("f16");
+    else if constexpr (K == 1) LCX_MMA_TS_W("f8f6f4");
+    else LCX_MMA_TS_W("tf32");
+#undef LCX_MMA_TS_W
 }
 
 // D(tmem) = A(smem) x B(smem) (+ D if accumulate), kind::f8f6f4 (8-bit A/B as the
