@@ -1385,15 +1385,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int lo = pi - p.window + 1 - k0;
                 const int sk = p.sinks - k0;
                 const bool win = p.causal && p.window > 0;
-                auto vis = [&](int col) { return col <= hi && (!win || col >= lo || col < sk); };
 
                 // The whole S row of this thread in one TMEM load.
                 float v[BN];
                 tmem_ld128(trow + s_col, v);
                 if (partial) {
+                    // A select per column, no branch: the rows of a warp see
+                    // different columns, and a branch per column (divergent across
+                    // the warp) cost ~13k cycles per partial tile.
 #pragma unroll
-                    for (int e = 0; e < BN; ++e)
-                        if (!vis(e)) v[e] = -INFINITY;
+                    for (int e = 0; e < BN; ++e) {
+                        const bool keep = (e <= hi) & (!win | (e >= lo) | (e < sk));
+                        v[e] = keep ? v[e] : -INFINITY;
+                    }
                 }
                 const float mx = row_max(v);
                 const float m_new = fmaxf(m, mx * cl2);
