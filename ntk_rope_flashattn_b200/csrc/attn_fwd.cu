@@ -881,8 +881,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int b = 0; b < 2; ++b) {
                 mbar_init(&bar.s_ready[t][b], 1);
                 // the tile's four softmax warps hand over P, except the ones
-                // that help rotate keys
-                mbar_init(&bar.p_ready[t][b], 32 * (4 - __popc((p.rot_help >> (4 * t)) & 0xF)));
+                // that help rotate keys; all eight in the split mode with fp16 V
+                mbar_init(&bar.p_ready[t][b], (kSplit && !kKvSplit && p.v_f16)
+                                                  ? 256
+                                                  : 32 * (4 - __popc((p.rot_help >> (4 * t)) & 0xF)));
             }
             mbar_init(&bar.o_ready[t], 1);
         }
@@ -1326,6 +1328,115 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int ord = __popc(p.rot_help & ((1u << warp) - 1u));
             rotate_keys_helped<D, RD, kHalf, kSplit, NSK, BN, C::kParts, C::kTileK>(
                 128 + 32 * ord + lane, T, sK, bar, p, abort, tmo);
+        } else if (kSplit && !kKvSplit && p.v_f16) {
+            // ------------------------------------------------ softmax, split mode
+            // With V already in fp16 the one query tile takes all eight softmax
+            // warps, two threads per row: warp w holds rows 32 (w % 4) + 16 (w / 4)
+            // .. + 15 (TMEM lanes of its quadrant), its lanes 0-15 keys 0-63 of
+            // those rows (output dims 0-63) and lanes 16-31 keys 64-127 (dims
+            // 64-127).  Row max and sum combine with one shuffle; the two warps
+            // of an SMSP overlap one's exponentials with the other's other work.
+            constexpr int NB = C::kNB;
+            constexpr int HB = BN / 2;                        // keys per thread
+            static_assert(kPF16 || !kSplit, "the split mode's P is fp16");
+            const int hf = lane >> 4;                         // column half
+            const int row = (warp & 3) * 32 + (warp >> 2) * 16 + (lane & 15);
+            const uint32_t tl = tmem + (uint32_t((warp & 3) * 32 + (warp >> 2) * 16) << 16);
+            const RowMap rm = map_row(p, U, 0, row, false);
+            const int pi = rm.i + p.qoff;                     // this row's query position
+            const int tq0 = U.tq0(0);
+            const float cl2 = p.c_log2;
+            float m = -INFINITY, l = 0.f;                     // l: this thread's half
+            bool ok = true;
+            for (int it = 0; it < T.n; ++it) {
+                const int b = it % NB;
+                const uint32_t s_col = b * BN;
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(&bar.s_ready[0][b], (it / NB) & 1, abort, tmo));
+                if (!ok) break;
+                tc_fence_after();
+                const int jt = T.tile(it), k0 = jt * BN + hf * HB;   // this thread's first key
+                const bool partial = !tile_full<BN>(tq0, jt, p);
+                // visible columns: col <= hi and (no window or col >= lo or col < sk)
+                const int hi = p.causal ? min(pi - k0, p.Lk - 1 - k0) : p.Lk - 1 - k0;
+                const int lo = pi - p.window + 1 - k0;
+                const int sk = p.sinks - k0;
+                const bool win = p.causal && p.window > 0;
+                float v[HB];
+                tmem_ld16x2_64(tl + s_col, v);
+                if (partial) {
+#pragma unroll
+                    for (int e = 0; e < HB; ++e) {
+                        const bool keep = (e <= hi) & (!win | (e >= lo) | (e < sk));
+                        v[e] = keep ? v[e] : -INFINITY;
+                    }
+                }
+                const float mh = row_max(v);
+                const float mx = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 16));
+                const float m_new = fmaxf(m, mx * cl2);
+                // Keep the old reference unless the max grew by more than 2^15.
+                const bool need = (m != -INFINITY) && (m_new > m + kRescaleLog2);
+                if (__any_sync(0xffffffffu, need)) {
+                    // O must not be in flight: PV(j - 1), signalled on its V
+                    // stage's barrier.  Each thread rescales its half of the row's
+                    // output dims.
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(&bar.empty_v[(it - 1) % NSV], ((it - 1) / NSV) & 1,
+                                              abort, tmo));
+                    if (!ok) break;
+                    tc_fence_after();
+                    const float alpha = need ? ex2_approx(m - m_new) : 1.f;
+#pragma unroll 1
+                    for (int c = 0; c < DV / 64; ++c) {
+                        float o[32];
+                        tmem_ld16x2_32(tl + C::kColO + c * 64, o);
+                        uint32_t u[32];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(o[e] * alpha);
+                        tmem_st16x2_32(tl + C::kColO + c * 64, u);
+                    }
+                    if (need) {
+                        l *= alpha;
+                        m = m_new;
+                    }
+                }
+                if (m == -INFINITY) m = m_new;
+                const float mref = (m == -INFINITY) ? 0.f : m;
+                // P = 2^(s c - m) as fp16 pairs over the first half of S (this
+                // thread's keys: P columns 32 hf .. 32 hf + 31), summed in fp32
+                const float2 c2 = make_float2(cl2, cl2), nm2 = make_float2(-mref, -mref);
+                float2 lsum = make_float2(0.f, 0.f);
+                uint32_t pk[HB / 2];
+#pragma unroll
+                for (int e = 0; e < HB / 2; ++e) {
+                    const float2 x = fma2(make_float2(v[2 * e], v[2 * e + 1]), c2, nm2);
+                    const float2 pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                    pk[e] = pack_f16x2(pe.x, pe.y);
+                    lsum = add2(lsum, pe);
+                }
+                tmem_st16x2_32(tl + s_col, pk);
+                l += lsum.x + lsum.y;
+                tc_fence_before();
+                mbar_arrive(&bar.p_ready[0][b]);
+            }
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.o_ready[0], 0, abort, tmo));
+            if (ok) {
+                tc_fence_after();
+                const float lt = l + __shfl_xor_sync(0xffffffffu, l, 16);   // the row's sum
+                const float inv = lt > 0.f ? 1.f / lt : 0.f;
+#pragma unroll 1
+                for (int c = 0; c < DV / 64; ++c) {
+                    float o[32];
+                    tmem_ld16x2_32(tl + C::kColO + c * 64, o);
+                    if (rm.valid)
+                        store_o32<DV, kF32, kKvSplit>(p, U, U.split, rm.h, rm.i, 2 * c + hf, o, inv);
+                }
+                if (rm.valid && hf == 0) {
+                    const float ln2 = 0.69314718055994531f;
+                    store_lse<kKvSplit>(p, U, U.split, rm.h, rm.i,
+                                        lt > 0.f ? (m + __log2f(lt)) * ln2 : -INFINITY);
+                }
+            }
         } else if (kConvV && warp >= 4) {
             // split mode: its one query tile leaves softmax warps 4-7 free; unless
             // V arrives in fp16 already, they convert every V tile to fp16 for the
