@@ -65,7 +65,7 @@ constexpr float kRescaleLog2 = 15.0f;
 // Build-time switches (-D...; the defaults are the measured-fastest choices):
 //   LCX_EMU_EVERY       1 column pair in N takes 2^x on the FMA pipe (0: none)
 //   LCX_D192_TWO_TILES  two query tiles and one K stage at D = 192 (0: one tile)
-//   LCX_KSTAGES_D128    K ring depth at D = 128 without split QK^T
+//   LCX_KSTAGES_D128    K ring depth at D = 128 without split QK^T (key-split launches: 3)
 //   LCX_ROT_UNROLL      rows in flight per rotation thread
 //   LCX_PHASOR_CARRY    reuse the phasor a K tile ends with for the next tile
 #ifndef LCX_EMU_EVERY
@@ -160,7 +160,7 @@ struct AttnParams {
 // rounded to tf32, 32 per 128-byte row of a box (2 boxes per row at D = 64);
 // P is written to TMEM as fp32 over the whole S buffer.  Two K and two V
 // stages of 32 KB beside two 32 KB query tiles.
-template <int D, int DV, bool kSplit, bool kTF = false>
+template <int D, int DV, bool kSplit, bool kTF = false, bool kKv = false>
 struct Cfg {
     static constexpr int BN = 128;                      // keys per tile
     static constexpr int ES = kTF ? 4 : 2;              // bytes per operand element
@@ -180,7 +180,7 @@ struct Cfg {
     static constexpr int kStagesK = kSplit ? (D == 64 ? 3 : 2)
                                   : kTF ? 2
                                   : (D == 64) ? 4
-                                  : (D == 128) ? LCX_KSTAGES_D128
+                                  : (D == 128) ? (kKv ? 3 : LCX_KSTAGES_D128)
                                   : (kNTQ == 2) ? 1 : 2;
     static constexpr int kStagesV = kSplit ? 3 : kTF ? 2 : (D == 64) ? 4 : 2;
     // Split mode: the query tile's two parts are the A operands of QK^T from
@@ -839,7 +839,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // converted in shared memory by the rotation warpgroup)
     constexpr bool kPF16 = kSplit && LCX_SPLIT_P_F16;
     constexpr bool kConvV = kPF16 && !kF32;
-    using C = Cfg<D, DV, kSplit, kTF>;
+    using C = Cfg<D, DV, kSplit, kTF, kKvSplit>;
     static_assert(!kF32 || (RD == D && DV == D), "fp32 operands: full rotary, DV = D");
     static_assert(!kSplit || (RD == D && DV == D), "split QK^T: full rotary, DV = D");
     constexpr int NSK = C::kStagesK;
@@ -1702,7 +1702,7 @@ struct AttnLaunchShape {
 template <int D, int DV, int RD, bool kF32, bool kHalf, bool kSplit, bool kKvSplit>
 lcx_status launch(const Maps &m, const AttnParams &p, unsigned grid, cudaStream_t s) {
     auto kern = attn_fwd_kernel<D, DV, RD, kF32, kHalf, kSplit, kKvSplit>;
-    const int smem = Cfg<D, DV, kSplit, kF32 && !kSplit && D == 64>::kSmemBytes;
+    const int smem = Cfg<D, DV, kSplit, kF32 && !kSplit && D == 64, kKvSplit>::kSmemBytes;
     // The warpgroups re-balance registers with setmaxnreg, which waits until the
     // registers it asks for are free: the launch must hold the whole split.
     static const int regs = []() {
