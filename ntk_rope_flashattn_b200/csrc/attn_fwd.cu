@@ -80,8 +80,9 @@ constexpr float kRescaleLog2 = 15.0f;
 #ifndef LCX_ROT_UNROLL
 #define LCX_ROT_UNROLL 2
 #endif
-// LCX_SPLIT_P_F16: the split mode's PV takes P and V in fp16 (V converted in
-// shared memory) rather than bf16
+// LCX_SPLIT_P_F16: the split mode's PV takes P and V in fp16 (V converted once
+// by the rotate pass, or in shared memory by softmax warps 4-7 when keys are
+// rotated on chip) rather than bf16
 #ifndef LCX_SPLIT_P_F16
 #define LCX_SPLIT_P_F16 1
 #endif
@@ -147,14 +148,16 @@ struct AttnParams {
 // and the rounding residual r = x' - h, and
 //   S = Qh Kh^T + [e5m2(Qh) | e5m2(Qr)] [e5m2(Kr) | e5m2(Kh)]^T,
 // one fp16 product (kind::f16) plus one e5m2 product over K = 2D
-// (kind::f8f6f4, twice the fp16 rate, so it costs what one more fp16 product
-// over K = D would).  The cross terms h r' are ~2^-11 of S, so their 3-bit
-// e5m2 operands still leave the logits accurate to about 2^-15 relative;
-// only the product of the two residuals (~2^-22) is dropped.  Each Q and K
-// tile then has a second part, the 8-bit cross operand: 2D bytes per row, the
-// size of a 16-bit part, stored as D/64 boxes of 128-byte rows ([h8 | r8] for
-// a query row, [r8 | h8] for a key row).  Key tiles stay 128 rows; at D = 128
-// the parts fill shared memory with one K stage (64 KB) and one V stage.
+// (kind::f8f6f4: at M = N = 128 each instruction takes the same ~64 cycles as
+// an fp16 one, so the cross product costs one more fp16 product).  The cross
+// terms h r' are ~2^-11 of S, so their 3-bit e5m2 operands still leave the
+// logits accurate to about 2^-15 relative; only the product of the two
+// residuals (~2^-22) is dropped.  Each Q and K tile then has a second part,
+// the 8-bit cross operand: 2D bytes per row, the size of a 16-bit part, stored
+// as D/64 boxes of 128-byte rows ([h8 | r8] for a query row, [r8 | h8] for a
+// key row).  One query tile per CTA, whose parts are TMEM A operands (their
+// shared-memory staging is the last K stage); two K stages (64 KB each at
+// D = 128) and three V stages of fp16.
 //
 // tf32 operands (fp32 inputs at D = 64): Q, K and V tiles hold fp32 values
 // rounded to tf32, 32 per 128-byte row of a box (2 boxes per row at D = 64);
