@@ -149,7 +149,8 @@ LCX_API lcx_status lcx_apply_rope(const lcx_rope_params *params, const void *x, 
                                    r = x' - h and form QK^T as
                                    qh.kh (fp16 tensor cores) + [e5m2(qh) |
                                    e5m2(qr)].[e5m2(kr) | e5m2(kh)] (one e5m2
-                                   product over 2 D at twice the fp16 rate),
+                                   product over 2 D, about one fp16 product's
+                                   time), with P and V in fp16 for PV,
                                    so the logits are accurate to ~2^-15
                                    relative instead of bf16's 2^-9 (needed when
                                    the logits are large, e.g. outlier-heavy
@@ -253,7 +254,8 @@ typedef struct {
  *   k_rope supplies the rotated key part once for all heads.
  *   Arithmetic: q', k' rounded to bf16 on chip (split mode: an fp16 part
  *   and e5m2 cross parts, see LCX_ATTN_SPLIT_QK), QK^T and PV on tensor cores
- *   with fp32 accumulation, P rounded to bf16 for PV, softmax statistics in
+ *   with fp32 accumulation, P rounded to bf16 for PV (split mode: P and V in
+ *   fp16), softmax statistics in
  *   fp32, o rounded once to the output dtype.  fp32 inputs at D = 64 keep
  *   32-bit operands: q', k', v and P rounded to tf32 (10-bit mantissa) for
  *   tf32 tensor-core products; at D = 128 (and in the split mode) fp32 inputs
