@@ -39,6 +39,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cmath>
 #include <cstring>
 
@@ -1650,6 +1651,420 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicExch(p.status, int(LCX_ERR_TIMEOUT));
 }
 
+// ---------------------------------------------------------------- decode kernel
+// Split-KV decode with the scores transposed: S^T = K Q^T puts one key per TMEM
+// lane and one query per column, the queries being the kv group's G heads times
+// the L rows of the call (G L <= NQ).  The query-tile kernel above gives each
+// query row a thread that evaluates all 128 keys of a tile, so a decode tile
+// of 4 heads keeps 4 of a warp's 32 rows busy and computes 8 times the
+// exponentials it needs.  Here the thread of key r evaluates only that key's
+// G L weights; the column maxima and sums are reduced over the 128 key threads
+// (shuffles, then four warps through shared memory).  The weights go to shared
+// memory as the K-major B operand of O^T = V^T P^T, whose A operand is the V
+// tile read MN-major exactly as the TMA lands it, and O^T keeps one output
+// column per TMEM lane.  The query block takes 4 KB of shared memory instead of
+// two 32 KB query tiles, which leaves room for three K and three V stages.
+namespace dec {
+constexpr int kThreads = 480;  // warps 0-3 softmax, 4-11 rotation, 12 K, 13 MMA, 14 V
+constexpr int D = 128, BN = 128, NQ = 16;
+constexpr int NSK = 3, NSV = 3, NBS = 4, NBP = 2;  // K, V stages; S^T, P buffers
+constexpr int kTile = BN * D * 2;                  // a K or V tile, bf16
+constexpr int kBox = BN * 128;                     // its 64-column boxes
+constexpr int kQBox = NQ * 128;                    // a 64-column box of the query or P block
+constexpr int kOffK = 0;
+constexpr int kOffV = kOffK + NSK * kTile;
+constexpr int kOffQ = kOffV + NSV * kTile;
+constexpr int kOffP = kOffQ + (D / 64) * kQBox;
+constexpr int kOffX = kOffP + NBP * (BN / 64) * kQBox;
+constexpr int kOffBar = kOffX + 1024;
+constexpr int kSmemBytes = kOffBar + 256 + 1024;  // barriers + alignment slack
+constexpr int kColO = NBS * NQ;                   // TMEM: NBS S^T buffers of NQ columns, then O^T
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+struct Bars {
+    uint64_t ready_q;
+    uint64_t full_k[NSK], ready_k[NSK], empty_k[NSK];
+    uint64_t full_v[NSV], empty_v[NSV];
+    uint64_t s_ready[NBS], p_ready[NBP], p_free[NBP];
+    uint64_t o_ready, drain;
+    uint32_t tmem_base;
+    int abort;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block");
+}  // namespace dec
+
+// The group's query block: row n = k L + i holds query i of head hq0 + k
+// (n < nq; the other rows are zero), rotated at position qoff + i unless the
+// queries arrive rotated, stored as the K-major B operand of S^T (two 64-column
+// boxes of NQ 128-byte rows, 128-byte swizzle).  Thread tw (of 128) takes row
+// tw / 8 and its pairs 8 (tw % 8) .. + 7: two 16-byte loads, two 16-byte
+// stores; each angle from the accurate sine and cosine.
+template <bool kHalf>
+__device__ __forceinline__ void load_q_decode(uint8_t *sQ, const AttnParams &p, const Unit &U,
+                                              int nq, int tw) {
+    using namespace dec;
+    static_assert(NQ * 8 == 128, "one row segment per thread");
+    const int n = tw >> 3, g = tw & 7;
+    // the 16-byte chunks (8 columns each) that hold the thread's pairs
+    const int c1 = kHalf ? g : 2 * g, c2 = kHalf ? g + D / 16 : 2 * g + 1;
+    uint4 a = make_uint4(0u, 0u, 0u, 0u), b = a;
+    if (n < nq) {
+        const int i = n % p.L;
+        const uint4 *row = reinterpret_cast<const uint4 *>(
+            reinterpret_cast<const __nv_bfloat16 *>(p.q) + U.b * p.qs[0] +
+            (long long)(U.hq0 + n / p.L) * p.qs[1] + (long long)i * p.qs[2]);
+        a = row[c1];
+        b = row[c2];
+        if (p.rotate_q) {
+            float x[8], y[8], c[8], s[8];
+            unpack8(a, x);
+            unpack8(b, y);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                rope_sincos((long long)p.qoff + i, p.theta[8 * g + e], &c[e], &s[e]);
+            // half pairing: pair 8 g + e is (x[e], y[e]); interleaved: pairs
+            // 8 g + e and 8 g + 4 + e are (x[2e], x[2e+1]) and (y[2e], y[2e+1])
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                float &u = kHalf ? x[e] : (e < 4 ? x[2 * e] : y[2 * (e - 4)]);
+                float &v = kHalf ? y[e] : (e < 4 ? x[2 * e + 1] : y[2 * (e - 4) + 1]);
+                const float u0 = u, v0 = v;
+                u = u0 * c[e] - v0 * s[e];
+                v = v0 * c[e] + u0 * s[e];
+            }
+            a = pack8(x);
+            b = pack8(y);
+        }
+    }
+    *reinterpret_cast<uint4 *>(sQ + chunk_off(n, c1, kQBox)) = a;
+    *reinterpret_cast<uint4 *>(sQ + chunk_off(n, c2, kQBox)) = b;
+}
+
+// One CTA per (batch, kv group, key split): bf16 operands, D = DV = 128, full
+// rotary, partial results (o normalised, lse) into the split workspace.  kNQ:
+// the query columns the softmax reads (4, 8 or 16 >= G L).
+template <bool kHalf, int kNQ>
+__global__ void __launch_bounds__(dec::kThreads, 1)
+    attn_decode_kernel(const __grid_constant__ CUtensorMap tmk,
+                       const __grid_constant__ CUtensorMap tmv,
+                       const __grid_constant__ AttnParams p) {
+    using namespace dec;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sK = smem + kOffK;
+    uint8_t *sV = smem + kOffV;
+    uint8_t *sQ = smem + kOffQ;
+    uint8_t *sP = smem + kOffP;
+    float *xmax = reinterpret_cast<float *>(smem + kOffX);  // [2][4][kNQ] column maxima per warp
+    float *xsum = xmax + 2 * 4 * kNQ;                        // [4][kNQ] column sums per warp
+    dec::Bars &bar = *reinterpret_cast<dec::Bars *>(smem + kOffBar);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const Unit U = decode_unit<true>(p);
+    const Tiles T = make_tiles<BN, true>(U.q0, U.split, p);
+    const int nq = p.G * p.L;  // query columns in use
+    volatile int *abort = &bar.abort;
+    const uint64_t tmo = p.timeout_ns;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bar.ready_q, 128);
+        for (int s = 0; s < NSK; ++s) {
+            mbar_init(&bar.full_k[s], 1);
+            mbar_init(&bar.ready_k[s], 256);
+            mbar_init(&bar.empty_k[s], 1);
+        }
+        for (int s = 0; s < NSV; ++s) {
+            mbar_init(&bar.full_v[s], 1);
+            mbar_init(&bar.empty_v[s], 1);
+        }
+        for (int b = 0; b < NBS; ++b) mbar_init(&bar.s_ready[b], 1);
+        for (int b = 0; b < NBP; ++b) {
+            mbar_init(&bar.p_ready[b], 128);
+            mbar_init(&bar.p_free[b], 1);
+        }
+        mbar_init(&bar.o_ready, 1);
+        mbar_init(&bar.drain, 1);
+        // A CTA that starts after another one's watchdog fired does no work.
+        bar.abort = p.status ? *reinterpret_cast<volatile int *>(p.status) : 0;
+        fence_mbar_init();
+    }
+    if (warp == 13) {
+        tmem_alloc(&bar.tmem_base, 128);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bar.tmem_base;
+    const bool skip = bar.abort != 0;
+
+    if (skip) {
+        // nothing to do: fall through to the common exit
+    } else if (T.n == 0) {
+        // a split that received no key tile: the empty partial result
+        if (warp < 4) {
+            for (int n = 0; n < nq; ++n) {
+                const long long prow =
+                    (((long long)U.split * p.B + U.b) * p.Hq + U.hq0 + n / p.L) * p.L + n % p.L;
+                p.part_o[prow * D + threadIdx.x] = 0.f;
+                if (threadIdx.x == 0) p.part_lse[prow] = -INFINITY;
+            }
+        }
+    } else if (warp == 12 || warp == 14) {
+        // ------------------------------------------------ TMA producers: K (12), V (14)
+        if (lane == 0 && !p.test_stall) {
+            const bool isk = warp == 12;
+            constexpr int NS = NSK > NSV ? NSK : NSV;
+            const int ns = isk ? NSK : NSV;
+            uint64_t *full = isk ? bar.full_k : bar.full_v;
+            uint64_t *empty = isk ? bar.empty_k : bar.empty_v;
+            uint8_t *base = isk ? sK : sV;
+            const CUtensorMap *map = isk ? &tmk : &tmv;
+            tma_prefetch_desc(map);
+            int issued[NS] = {};
+            bool ok = true;
+            for (int j = 0; ok && j < T.n; ++j) {
+                const int jt = T.tile(j), s = j % ns, u = j / ns;
+                if (u > 0) ok = mbar_wait(&empty[s], (u - 1) & 1, abort, tmo);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&full[s], kTile);
+                for (int bx = 0; bx < D / 64; ++bx)
+                    tma_load_4d(base + s * kTile + bx * kBox, map, &full[s], bx * 64, jt * BN,
+                                U.g, U.b);
+                ++issued[s];
+            }
+            // never leave the CTA with copies in flight (bounded, even after an abort)
+            for (int s = 0; s < ns; ++s)
+                if (issued[s]) mbar_wait(&full[s], (issued[s] - 1) & 1, nullptr, tmo);
+        }
+    } else if (warp == 13) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            // S^T: A = the K tile, B = the query block, both K-major.  O^T: A = the
+            // V tile, MN-major; B = the weights, K-major.  M = 128, N = NQ.
+            constexpr uint32_t kIdS = idesc_bf16_f32(128, NQ, 0, 0);
+            constexpr uint32_t kIdO = idesc_bf16_f32(128, NQ, 1, 0);
+            const uint64_t dv0 = sdesc_sw128(smem_u32(sV), kBox, 1024);
+            const uint32_t dhi = uint32_t(dv0 >> 32);  // the same for every descriptor here
+            const uint32_t v_lo = uint32_t(dv0);
+            const uint32_t k_lo = uint32_t(sdesc_sw128(smem_u32(sK), 16, 1024));
+            const uint32_t q_lo = uint32_t(sdesc_sw128(smem_u32(sQ), 16, 1024));
+            const uint32_t p_lo = uint32_t(sdesc_sw128(smem_u32(sP), 16, 1024));
+            uint64_t *kready = p.rotate_k ? bar.ready_k : bar.full_k;
+            auto issue_s = [&](int j) {
+                const uint32_t ka = k_lo + (((j % NSK) * kTile) >> 4);
+                const uint32_t dst = tmem + (j % NBS) * NQ;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t ok_ = ((kk >> 2) * kBox + (kk & 3) * 32) >> 4;
+                    const uint32_t oq = ((kk >> 2) * kQBox + (kk & 3) * 32) >> 4;
+                    mma_ss_w<0>(dst, ka + ok_, q_lo + oq, dhi, kIdS, kk > 0);
+                }
+            };
+            auto issue_pv = [&](int j) {
+                const uint32_t va = v_lo + (((j % NSV) * kTile) >> 4);
+                const uint32_t pa = p_lo + (((j % NBP) * (BN / 64) * kQBox) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    const uint32_t ov = (kk * 16 * 128) >> 4;  // 16 keys: 16 rows of the V tile
+                    const uint32_t op = ((kk >> 2) * kQBox + (kk & 3) * 32) >> 4;
+                    mma_ss_w<0>(tmem + kColO, va + ov, pa + op, dhi, kIdO, (j > 0 || kk > 0));
+                }
+            };
+            bool ok = mbar_wait(&bar.ready_q, 0, abort, tmo);
+            // S^T runs up to NBS key tiles ahead of the softmax
+            for (int j = 0; ok && j < NBS && j < T.n; ++j) {
+                ok = mbar_wait(&kready[j % NSK], (j / NSK) & 1, abort, tmo);
+                tc_fence_after();
+                if (!ok) break;
+                issue_s(j);
+                mma_commit(&bar.s_ready[j % NBS]);
+                mma_commit(&bar.empty_k[j % NSK]);
+            }
+            for (int j = 0; ok && j < T.n; ++j) {
+                ok = mbar_wait(&bar.full_v[j % NSV], (j / NSV) & 1, abort, tmo);
+                if (ok) ok = mbar_wait(&bar.p_ready[j % NBP], (j / NBP) & 1, abort, tmo);
+                tc_fence_after();
+                if (!ok) break;
+                issue_pv(j);
+                mma_commit(&bar.empty_v[j % NSV]);
+                mma_commit(&bar.p_free[j % NBP]);
+                // S^T(j + NBS) into the buffer the softmax of j has read
+                const int jn = j + NBS;
+                if (jn < T.n) {
+                    ok = mbar_wait(&kready[jn % NSK], (jn / NSK) & 1, abort, tmo);
+                    tc_fence_after();
+                    if (!ok) break;
+                    issue_s(jn);
+                    mma_commit(&bar.s_ready[jn % NBS]);
+                    mma_commit(&bar.empty_k[jn % NSK]);
+                }
+            }
+            if (ok) mma_commit(&bar.o_ready);
+            // every product done before the CTA frees its TMEM (bounded)
+            mma_commit(&bar.drain);
+            mbar_wait(&bar.drain, 0, nullptr, tmo);
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ------------------------------------------------ queries, then key rotation
+        const int tw = threadIdx.x - 128;  // 0..255
+        if (tw < 128) {
+            load_q_decode<kHalf>(sQ, p, U, nq, tw);
+            fence_proxy_async_smem();
+            mbar_arrive(&bar.ready_q);
+        }
+        if (p.rotate_k)
+            rotate_keys_helped<D, D, kHalf, false, NSK, BN, 1, kTile>(tw, T, sK, bar, p, abort,
+                                                                      tmo);
+    } else {
+        // ------------------------------------------------ softmax, warps 0-3
+        // Thread r holds key r of every key tile (TMEM lane r of S^T) and output
+        // column r (lane r of O^T).  Every iteration passes named barrier 2 once,
+        // whatever happened, so the four warps always meet.
+        const int r = threadIdx.x;
+        const uint32_t tl = tmem + (uint32_t(warp * 32) << 16);
+        const float cl2 = p.c_log2;
+        // the weight buffers' rows n >= nq stay zero
+        for (int i = r; i < NBP * (BN / 64) * kQBox / 16; i += 128)
+            reinterpret_cast<uint4 *>(sP)[i] = make_uint4(0u, 0u, 0u, 0u);
+        // column n sees the keys [lo, hi] and the sinks (none when n >= nq)
+        int hi[kNQ], lo[kNQ];
+        float m[kNQ], l[kNQ];
+#pragma unroll
+        for (int n = 0; n < kNQ; ++n) {
+            const int pi = p.qoff + n % p.L;  // the query's position
+            hi[n] = n >= nq ? -1 : p.causal ? min(pi, p.Lk - 1) : p.Lk - 1;
+            lo[n] = (p.causal && p.window > 0) ? pi - p.window + 1 : INT_MIN;
+            m[n] = -INFINITY;
+            l[n] = 0.f;
+        }
+        bool ok = true;
+        for (int j = 0; j < T.n; ++j) {
+            const int pb = j % NBP;
+            const uint32_t ps = (j / NBS) & 1, pp = ((j - NBP) / NBP) & 1;
+            if (ok) {
+                // S^T(j) computed and the weight buffer free (PV(j - NBP) done):
+                // both tested at once first, the full waits only if one is pending
+                const bool rdy = mbar_try_wait(&bar.s_ready[j % NBS], ps) &&
+                                 (j < NBP || mbar_try_wait(&bar.p_free[pb], pp));
+                if (!__all_sync(0xffffffffu, rdy)) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_ready[j % NBS], ps, abort, tmo));
+                    if (ok && j >= NBP)
+                        ok = __all_sync(0xffffffffu, mbar_wait(&bar.p_free[pb], pp, abort, tmo));
+                }
+            }
+            float x[kNQ];
+            if (ok) {
+                tc_fence_after();
+                tmem_ldn<kNQ>(tl + (j % NBS) * NQ, x);
+            }
+            const int key = T.tile(j) * BN + r;
+            // logits in log2 units, masked.  The reference m of a column moves
+            // only when a logit passes m + 2^15 (exact either way; O^T's
+            // rescale is saved): a vote per column, and the warp's maximum only
+            // for the columns where the vote says so.
+            bool grow[kNQ];
+#pragma unroll
+            for (int n = 0; n < kNQ; ++n) {
+                const bool vis = ok && key <= hi[n] && (key >= lo[n] || key < p.sinks);
+                x[n] = vis ? x[n] * cl2 : -INFINITY;
+                grow[n] = __any_sync(0xffffffffu, x[n] > m[n] + kRescaleLog2);
+            }
+#pragma unroll
+            for (int n = 0; n < kNQ; ++n) {
+                float mx = -INFINITY;
+                if (grow[n]) {
+                    mx = x[n];
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1)
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                }
+                if (lane == 0) xmax[((j & 1) * 4 + warp) * kNQ + n] = mx;
+            }
+            named_bar_sync(2, 128);
+            bool rescale = false;
+            float alpha[NQ];
+#pragma unroll
+            for (int n = 0; n < NQ; ++n) alpha[n] = 1.f;
+#pragma unroll
+            for (int n = 0; n < kNQ; ++n) {
+                const float *xm = xmax + (j & 1) * 4 * kNQ + n;
+                const float mt = fmaxf(fmaxf(xm[0], xm[kNQ]), fmaxf(xm[2 * kNQ], xm[3 * kNQ]));
+                if (mt > m[n] + kRescaleLog2) {
+                    if (m[n] != -INFINITY) {
+                        alpha[n] = ex2_approx(m[n] - mt);
+                        l[n] *= alpha[n];
+                        rescale = true;
+                    }
+                    m[n] = mt;
+                }
+            }
+            if (ok && rescale) {
+                // O^T must not be in flight: PV(j - 1) done
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar.p_free[(j - 1) % NBP],
+                                                       ((j - 1) / NBP) & 1, abort, tmo));
+                if (ok) {
+                    tc_fence_after();
+                    float o[NQ];
+                    tmem_ld16(tl + kColO, o);
+#pragma unroll
+                    for (int n = 0; n < NQ; ++n) o[n] *= alpha[n];
+                    tmem_st16(tl + kColO, o);
+                }
+            }
+            if (ok) {
+                // the weights 2^(s c - m), bf16, into row n of the K-major P block
+                uint8_t *pbuf = sP + pb * (BN / 64) * kQBox;
+#pragma unroll
+                for (int n = 0; n < kNQ; ++n) {
+                    const float w = ex2_approx(x[n] - (m[n] == -INFINITY ? 0.f : m[n]));
+                    l[n] += w;
+                    *reinterpret_cast<__nv_bfloat16 *>(pbuf + chunk_off(n, r >> 3, kQBox) +
+                                                       (r & 7) * 2) = __float2bfloat16_rn(w);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&bar.p_ready[pb]);
+            }
+        }
+        // each column's sum over the 128 keys
+#pragma unroll
+        for (int n = 0; n < kNQ; ++n) {
+            float sum = l[n];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            if (lane == 0) xsum[warp * kNQ + n] = sum;
+        }
+        named_bar_sync(2, 128);
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.o_ready, 0, abort, tmo));
+        if (ok) {
+            tc_fence_after();
+            float o[kNQ];
+            tmem_ldn<kNQ>(tl + kColO, o);
+            const float ln2 = 0.69314718055994531f;
+#pragma unroll
+            for (int n = 0; n < kNQ; ++n) {
+                if (n >= nq) break;
+                const float lt = xsum[n] + xsum[kNQ + n] + xsum[2 * kNQ + n] + xsum[3 * kNQ + n];
+                const long long prow =
+                    (((long long)U.split * p.B + U.b) * p.Hq + U.hq0 + n / p.L) * p.L + n % p.L;
+                p.part_o[prow * D + r] = lt > 0.f ? o[n] * (1.f / lt) : 0.f;
+                if (r == 0) p.part_lse[prow] = lt > 0.f ? (m[n] + __log2f(lt)) * ln2 : -INFINITY;
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 13) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+    if (threadIdx.x == 0 && !skip && bar.abort && p.status)
+        atomicExch(p.status, int(LCX_ERR_TIMEOUT));
+}
+
 // ---------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -1759,6 +2174,29 @@ lcx_status launch_shape(const AttnLaunchShape &x, const Maps &m, const AttnParam
                       : launch_full<64, false, kKv>(x.f32, x.half, m, p, g, s);
 }
 
+// The transposed decode kernel (bf16, D = DV = 128, full rotary, G L <= 16).
+template <bool kHalf, int kNQ>
+lcx_status launch_decode(const Maps &m, const AttnParams &p, unsigned grid, cudaStream_t s) {
+    auto kern = attn_decode_kernel<kHalf, kNQ>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kSmemBytes);
+    if (e != cudaSuccess)
+        return fail(LCX_ERR_CUDA, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
+    kern<<<grid, dec::kThreads, dec::kSmemBytes, s>>>(m.k, m.v, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return fail(LCX_ERR_CUDA, "attn_decode launch failed: %s", cudaGetErrorString(e));
+    return LCX_OK;
+}
+
+template <bool kHalf>
+lcx_status launch_decode_nq(int nq, const Maps &m, const AttnParams &p, unsigned grid,
+                            cudaStream_t s) {
+    return nq <= 4 ? launch_decode<kHalf, 4>(m, p, grid, s)
+                   : nq <= 8 ? launch_decode<kHalf, 8>(m, p, grid, s)
+                             : launch_decode<kHalf, 16>(m, p, grid, s);
+}
+
 lcx_status check_tensor(const void *ptr, const int64_t *st, int es, const char *name) {
     if (!ptr) return fail(LCX_ERR_INVALID_ARG, "%s is NULL", name);
     if (!aligned16(ptr)) return fail(LCX_ERR_UNSUPPORTED, "%s must be 16-byte aligned", name);
@@ -1794,6 +2232,7 @@ struct AttnLaunch : AttnLaunchShape {
     int64_t v_src_strides[4];
     int rot_h, rot_d; // heads and columns the pass rotates (Hkv, D; or 1, d_R)
     void *k_rot;      // where the pass writes
+    bool decode;      // split-KV launch of the transposed decode kernel
 };
 
 // Validate `a` and fill `x`.  *noop is set for empty problems (B or L zero),
@@ -2038,6 +2477,11 @@ lcx_status attn_enqueue(const AttnLaunch &x, cudaStream_t s) {
         }
     }
     const unsigned g = unsigned(grid);
+    if (x.decode) {
+        const int nq = x.p.G * x.p.L;
+        return x.half ? launch_decode_nq<true>(nq, x.m, x.p, g, s)
+                      : launch_decode_nq<false>(nq, x.m, x.p, g, s);
+    }
     return x.p.n_split > 1 ? launch_shape<true>(x, x.m, x.p, g, s)
                            : launch_shape<false>(x, x.m, x.p, g, s);
 }
@@ -2121,7 +2565,18 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
     //    G pack_lp <= 128, its two S buffers walking the key tiles in turn.
     const int64_t lp = (a->L + 7) / 8 * 8;
     int n_parts = num_splits;
-    if (x.split_qk) {
+    // A kv group's G L queries fit in the columns of one transposed score
+    // block (bf16, D = DV = 128, full rotary): the decode kernel, one CTA per
+    // (batch, kv group, split), one partial result per split.
+    x.decode = !x.f32 && !x.split_qk && x.D == 128 && x.DV == 128 && x.RD == 128 &&
+               !x.p.k_rope_shared && !x.p.test_stall && int64_t(x.p.G) * a->L <= dec::NQ;
+    if (x.decode) {
+        x.p.qpair = 0;
+        x.p.heads_per_unit = x.p.G;
+        x.p.n_qb = 1;
+        x.p.units_per_qb = x.p.B * x.p.Hkv;
+        x.units = (long long)x.p.B * x.p.Hkv;
+    } else if (x.split_qk) {
         // one query tile per CTA: all G heads in it when they fit
         if (!x.f32 && lp * x.p.G <= kBM) {
             x.p.pack_lp = int(lp);

@@ -311,6 +311,67 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
     for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(u[i]);
 }
 
+// 32 lanes x 16 columns of 32-bit TMEM -> 16 registers per thread, then the wait.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16]) {
+    uint32_t u[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+          "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]),
+          "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) r[i] = __uint_as_float(u[i]);
+}
+
+// 32 lanes x N columns (N = 4, 8 or 16) -> N registers per thread, then the wait.
+template <int N>
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, float (&r)[N]) {
+    static_assert(N == 4 || N == 8 || N == 16, "tmem_ldn width");
+    if constexpr (N == 16) {
+        tmem_ld16(taddr, r);
+    } else if constexpr (N == 8) {
+        uint32_t u[8];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
+            "tcgen05.wait::ld.sync.aligned;"
+            : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+              "=r"(u[7])
+            : "r"(taddr)
+            : "memory");
+#pragma unroll
+        for (int i = 0; i < 8; ++i) r[i] = __uint_as_float(u[i]);
+    } else {
+        uint32_t u[4];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];\n\t"
+            "tcgen05.wait::ld.sync.aligned;"
+            : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
+            : "r"(taddr)
+            : "memory");
+#pragma unroll
+        for (int i = 0; i < 4; ++i) r[i] = __uint_as_float(u[i]);
+    }
+}
+
+// 16 registers per thread -> 32 lanes x 16 columns of TMEM, then the wait.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+        "r"(__float_as_uint(r[0])), "r"(__float_as_uint(r[1])), "r"(__float_as_uint(r[2])),
+        "r"(__float_as_uint(r[3])), "r"(__float_as_uint(r[4])), "r"(__float_as_uint(r[5])),
+        "r"(__float_as_uint(r[6])), "r"(__float_as_uint(r[7])), "r"(__float_as_uint(r[8])),
+        "r"(__float_as_uint(r[9])), "r"(__float_as_uint(r[10])), "r"(__float_as_uint(r[11])),
+        "r"(__float_as_uint(r[12])), "r"(__float_as_uint(r[13])), "r"(__float_as_uint(r[14])),
+        "r"(__float_as_uint(r[15]))
+        : "memory");
+}
+
 // 32 lanes x 64 columns of 32-bit TMEM -> 64 registers per thread, one wait.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&r)[64]) {
     uint32_t u[64];
