@@ -906,7 +906,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = bar.tmem_base;
     const bool skip = bar.abort != 0;
-
+    // key splits: the merge may be scheduled now (it waits for this grid to
+    // finish before it reads the partial results)
+    if constexpr (kKvSplit) pdl_launch_dependents();
 
     if (skip) {
         // nothing to do: fall through to the common exit
@@ -1798,6 +1800,9 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = bar.tmem_base;
     const bool skip = bar.abort != 0;
+    // the merge of the partial results may be scheduled now (it waits for this
+    // grid to finish before it reads them)
+    pdl_launch_dependents();
 
     if (skip) {
         // nothing to do: fall through to the common exit

@@ -30,6 +30,10 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
     merge_kernel(const float *__restrict__ o_parts, const float *__restrict__ lse_parts,
                  int n_parts, long long rows, int Hq, int L, void *o, long long os0,
                  long long os1, long long os2, float *lse_out) {
+    // Launched as a programmatic dependent of the attention kernel that writes
+    // the parts: wait here until that grid has completed and its writes are
+    // visible (a plain launch passes straight through).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     constexpr int V = D / 32;  // values per lane: 4 (D=128) or 2 (D=64)
     const int lane = threadIdx.x & 31;
     const long long row = (long long)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
@@ -41,26 +45,38 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
     float acc[V];
 #pragma unroll
     for (int e = 0; e < V; ++e) acc[e] = 0.f;
-    float z = 0.f;
+    float z = 0.f;  // this lane's parts' weights
     if (m != -INFINITY) {
-        for (int s = 0; s < n_parts; ++s) {
-            const float l = lse_parts[(long long)s * rows + row];
-            if (l == -INFINITY) continue;
-            const float w = expf(l - m);
-            z += w;
-            const float *src = o_parts + ((long long)s * rows + row) * D + lane * V;
-            if constexpr (V == 4) {
-                const float4 x = __ldcs(reinterpret_cast<const float4 *>(src));
-                acc[0] += w * x.x;
-                acc[1] += w * x.y;
-                acc[2] += w * x.z;
-                acc[3] += w * x.w;
-            } else {
-                const float2 x = __ldcs(reinterpret_cast<const float2 *>(src));
-                acc[0] += w * x.x;
-                acc[1] += w * x.y;
+        // 32 parts at a time: lane u computes the weight of part s0 + u (0 for
+        // an empty part), the warp takes it by shuffle; the parts' rows have no
+        // dependence on one another, so eight of them are loaded at once.
+        for (int s0 = 0; s0 < n_parts; s0 += 32) {
+            const int s = s0 + lane;
+            const float l = s < n_parts ? lse_parts[(long long)s * rows + row] : -INFINITY;
+            const float wl = l == -INFINITY ? 0.f : expf(l - m);
+            z += wl;
+            const int nu = min(32, n_parts - s0);
+#pragma unroll 8
+            for (int u = 0; u < nu; ++u) {
+                const float w = __shfl_sync(0xffffffffu, wl, u);
+                const float *src = o_parts + ((long long)(s0 + u) * rows + row) * D + lane * V;
+                if constexpr (V == 4) {
+                    float4 x = __ldcs(reinterpret_cast<const float4 *>(src));
+                    if (w == 0.f) x = make_float4(0.f, 0.f, 0.f, 0.f);
+                    acc[0] += w * x.x;
+                    acc[1] += w * x.y;
+                    acc[2] += w * x.z;
+                    acc[3] += w * x.w;
+                } else {
+                    float2 x = __ldcs(reinterpret_cast<const float2 *>(src));
+                    if (w == 0.f) x = make_float2(0.f, 0.f);
+                    acc[0] += w * x.x;
+                    acc[1] += w * x.y;
+                }
             }
         }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
     }
     const float inv = z > 0.f ? 1.f / z : 0.f;
     const long long h_all = row / L;                  // b * Hq + h
@@ -89,28 +105,35 @@ lcx_status launch_merge(const float *o_parts, const float *lse_parts, int n_part
     if (rows == 0) return LCX_OK;
     const long long blocks = (rows + kMergeWarps - 1) / kMergeWarps;
     if (blocks > 0x7fffffffLL) return fail(LCX_ERR_UNSUPPORTED, "too many rows to merge");
-    const dim3 grid{unsigned(blocks)}, block{unsigned(kMergeWarps * 32)};
+    // A programmatic dependent launch: the grid may be scheduled while the
+    // attention kernel that writes the parts finishes (the kernel waits for
+    // it), which hides this launch's latency behind that kernel's tail.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(blocks));
+    cfg.blockDim = dim3(unsigned(kMergeWarps * 32));
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     const bool f32 = dtype == LCX_F32;
     const long long s0 = o_strides[0], s1 = o_strides[1], s2 = o_strides[2];
-    if (D == 128) {
-        if (f32)
-            merge_kernel<128, true><<<grid, block, 0, stream>>>(o_parts, lse_parts, n_parts, rows,
-                                                                int(Hq), int(L), o, s0, s1, s2,
-                                                                lse_out);
-        else
-            merge_kernel<128, false><<<grid, block, 0, stream>>>(o_parts, lse_parts, n_parts, rows,
-                                                                 int(Hq), int(L), o, s0, s1, s2,
-                                                                 lse_out);
-    } else {
-        if (f32)
-            merge_kernel<64, true><<<grid, block, 0, stream>>>(o_parts, lse_parts, n_parts, rows,
-                                                               int(Hq), int(L), o, s0, s1, s2,
-                                                               lse_out);
-        else
-            merge_kernel<64, false><<<grid, block, 0, stream>>>(o_parts, lse_parts, n_parts, rows,
-                                                                int(Hq), int(L), o, s0, s1, s2,
-                                                                lse_out);
-    }
+    const int hq = int(Hq), l = int(L);
+    cudaError_t le;
+    if (D == 128)
+        le = f32 ? cudaLaunchKernelEx(&cfg, merge_kernel<128, true>, o_parts, lse_parts, n_parts,
+                                      rows, hq, l, o, s0, s1, s2, lse_out)
+                 : cudaLaunchKernelEx(&cfg, merge_kernel<128, false>, o_parts, lse_parts, n_parts,
+                                      rows, hq, l, o, s0, s1, s2, lse_out);
+    else
+        le = f32 ? cudaLaunchKernelEx(&cfg, merge_kernel<64, true>, o_parts, lse_parts, n_parts,
+                                      rows, hq, l, o, s0, s1, s2, lse_out)
+                 : cudaLaunchKernelEx(&cfg, merge_kernel<64, false>, o_parts, lse_parts, n_parts,
+                                      rows, hq, l, o, s0, s1, s2, lse_out);
+    if (le != cudaSuccess)
+        return fail(LCX_ERR_CUDA, "merge launch failed: %s", cudaGetErrorString(le));
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return fail(LCX_ERR_CUDA, "merge launch failed: %s", cudaGetErrorString(e));

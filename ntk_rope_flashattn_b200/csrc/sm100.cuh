@@ -138,6 +138,14 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched after this one with the
+// programmatic-serialization attribute may be scheduled once every CTA of this
+// grid has executed this (or exited); that kernel waits for this grid's
+// completion with griddepcontrol.wait before it reads what this one wrote.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }

@@ -168,3 +168,38 @@ def test_splitkv_interleaved_key_tiles(L, Lk, splits, extra):
                        k_prerotated=prerot, split_qk=w.split_qk, rotate_k_once=once)
     ref = oracle_rows(q, k, v, rope, Lk - L, True, w.window, w.sinks)
     compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref[0], ref[1])
+
+
+@pytest.mark.parametrize("L,Lk,splits,extra", [
+    (1, 2000, 5, dict(Hq=16, Hkv=4)),                          # G L = 4: 4 query columns
+    (1, 2000, 5, dict(Hq=10, Hkv=2)),                          # G L = 5: 8 columns, 3 unused
+    (2, 1500, 3, dict(Hq=8, Hkv=2, pairing="interleaved")),    # G L = 8
+    (3, 3000, 6, dict(Hq=6, Hkv=2, window=900, sinks=5)),      # G L = 9: 16 columns
+    (16, 2100, 4, dict(Hq=2, Hkv=2)),                          # G = 1, a 16-row chunk
+    (1, 900, 12, dict(Hq=8, Hkv=2)),                           # 8 key tiles, 12 splits
+    (1, 2000, 5, dict(Hq=8, Hkv=2, rotate_k_once=True)),       # keys rotated by the pass
+    (1, 2000, 5, dict(Hq=8, Hkv=2, prerotated=True)),          # q and k arrive rotated
+    (4, 1000, 3, dict(Hq=8, Hkv=2, causal=False)),
+])
+def test_splitkv_transposed_decode(L, Lk, splits, extra):
+    """Key-split launches whose kv group holds at most 16 queries (bf16, D = 128,
+    full rotary) run the transposed-score decode kernel: one key per TMEM lane
+    and one query per column, 4, 8 or 16 columns read.  Every row of every head
+    against the oracle, empty splits, both pairings and the rotated-input modes
+    included."""
+    extra = dict(extra)
+    once = extra.pop("rotate_k_once", False)
+    prerot = extra.pop("prerotated", False)
+    causal = extra.pop("causal", True)
+    w = W0.with_(**extra, L=Lk)
+    q_all, k, v = make_inputs(w, device="cuda")
+    rope = rope_of(w)
+    q = q_all[:, :, Lk - L:]
+    q_in, k_in = q, k
+    if prerot:
+        q_in = lcx.apply_rope(q_all, rope)[:, :, Lk - L:]
+        k_in = lcx.apply_rope(k, rope)
+    o, lse = run_split(q_in, k_in, v, rope, splits, causal=causal, window=w.window,
+                       sinks=w.sinks, q_offset=Lk - L, prerotated=prerot, rotate_k_once=once)
+    ref = oracle_rows(q, k, v, rope, Lk - L, causal, w.window, w.sinks)
+    compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref[0], ref[1])
