@@ -2574,7 +2574,7 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
     // block (bf16, D = DV = 128, full rotary): the decode kernel, one CTA per
     // (batch, kv group, split), one partial result per split.
     x.decode = !x.f32 && !x.split_qk && x.D == 128 && x.DV == 128 && x.RD == 128 &&
-               !x.p.k_rope_shared && !x.p.test_stall && int64_t(x.p.G) * a->L <= dec::NQ;
+               !x.p.k_rope_shared && int64_t(x.p.G) * a->L <= dec::NQ;
     if (x.decode) {
         x.p.qpair = 0;
         x.p.heads_per_unit = x.p.G;
