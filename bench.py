@@ -479,6 +479,39 @@ def _call_ms(fn, stream, reps, flush=None, warm=2):
     return statistics.mean(a.elapsed_time(b) for a, b in evs)
 
 
+def _graph_and_host_us(fn, n=50):
+    """A launch-bound call measured two more ways: the host time to issue one
+    call (no synchronisation in between), and the device time per call when n
+    calls captured once into a CUDA graph are replayed (no host work between
+    the launches)."""
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(n):
+        fn()
+    host_us = (time.perf_counter() - t0) / n * 1e6
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for _ in range(n):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream()
+    a.record(cur)
+    g.replay()
+    b.record(cur)
+    torch.cuda.synchronize()
+    graph_us = a.elapsed_time(b) / n * 1e3
+    del g
+    return graph_us, host_us
+
+
 def bench_configs(lcx, dev, stream, status, peaks, local, reps=5):
     """Every workload measured like the headline: one lcx_attn_fwd call per
     step (host table, the keys' rotate pass into a buffer, the attention kernel),
@@ -537,6 +570,11 @@ def bench_configs(lcx, dev, stream, status, peaks, local, reps=5):
                 e["kernel_tflops"] = round(flops / (kern * 1e-3) / 1e12, 2)
             if tiny:
                 e["latency_us"] = round(ms * 1e3, 2)
+                # back-to-back calls from Python are bound by the host's issue
+                # time; replayed from a CUDA graph they show the device's own
+                g_us, h_us = _graph_and_host_us(lambda: lcx.attn_fwd(q, k, v, rope, **kw))
+                e["latency_graph_us"] = round(g_us, 2)
+                e["host_issue_us"] = round(h_us, 2)
             assert int(status.item()) == 0, "device watchdog fired in %s" % name
             out[name] = e
             del q, k, v, o, k_rot, qr, kr

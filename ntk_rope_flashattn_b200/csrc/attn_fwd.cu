@@ -2380,8 +2380,19 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     // odd group the two tiles are consecutive query blocks of one head.
     const bool two_tiles =
         (a->D <= 128 || LCX_D192_TWO_TILES) && !(a->flags & LCX_ATTN_SPLIT_QK);
-    p.heads_per_unit = (p.G % 2 == 0 && two_tiles) ? 2 : 1;
-    p.qpair = (p.G % 2 == 1 && two_tiles) ? 1 : 0;
+    // Pairs only when the paired units still fill the GPU: a problem of few
+    // query blocks (the tiny workload is one pair) runs faster spread over
+    // twice the CTAs, one query tile each.
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sms = 148;
+    const int64_t paired_units =
+        p.G % 2 == 0 ? (a->L + kBM - 1) / kBM * (a->B * a->Hq / 2)
+                     : (a->L + 2 * kBM - 1) / (2 * kBM) * (a->B * a->Hq);
+    const bool pair = two_tiles && paired_units >= sms;
+    p.heads_per_unit = (p.G % 2 == 0 && pair) ? 2 : 1;
+    p.qpair = (p.G % 2 == 1 && pair) ? 1 : 0;
     p.n_qb = int((a->L + (p.qpair ? 2 * kBM : kBM) - 1) / (p.qpair ? 2 * kBM : kBM));
     p.units_per_qb = p.B * p.Hq / p.heads_per_unit;
     p.n_split = 1;
