@@ -1660,8 +1660,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // query row a thread that evaluates all 128 keys of a tile, so a decode tile
 // of 4 heads keeps 4 of a warp's 32 rows busy and computes 8 times the
 // exponentials it needs.  Here the thread of key r evaluates only that key's
-// G L weights; the column maxima and sums are reduced over the 128 key threads
-// (shuffles, then four warps through shared memory).  The weights go to shared
+// G L weights.  A column's maximum is reduced over the 128 key threads
+// (shuffles, then four warps through shared memory) only when a vote finds a
+// logit past the column's lazy reference; its sum once, at the end.  The weights go to shared
 // memory as the K-major B operand of O^T = V^T P^T, whose A operand is the V
 // tile read MN-major exactly as the TMA lands it, and O^T keeps one output
 // column per TMEM lane.  The query block takes 4 KB of shared memory instead of
