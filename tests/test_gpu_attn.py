@@ -341,3 +341,25 @@ def test_attn_rotate_keys_once_decode_and_split(mode, kw):
         torch.cuda.synchronize()
         compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref_o.reshape(o.shape),
                 ref_lse.reshape(lse.shape))
+
+
+@pytest.mark.parametrize("extra", [
+    # G = 3 (odd): 50 pairs of consecutive 128-row query blocks x 3 heads = 150
+    # paired units, so each CTA takes two query blocks of one head
+    dict(Hq=3, Hkv=1, L=256 * 50, mode="yarn", scale=8.0, original_max_pos=1024),
+    # G = 4 (even): 37 query blocks x 4 head pairs = 148 paired units, so each
+    # CTA takes one query block of two heads of a group
+    dict(Hq=8, Hkv=2, L=128 * 37, mode="ntk", scale=4.0, window=1500, sinks=3),
+])
+def test_attn_paired_units(extra):
+    """Query tiles are paired in a CTA (two heads of a group, or two consecutive
+    query blocks of one head) only when the paired units still number at least
+    the SM count; these shapes sit at that edge on a 148-SM B200, so the paired
+    forms stay under test (the smaller shapes above run one tile per CTA)."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    w = BASE.with_(**extra)
+    paired = (-(-w.L // 256) * w.Hq) if w.Hq // w.Hkv % 2 else (-(-w.L // 128) * w.Hq // 2)
+    assert paired >= sms or sms > 150
+    errs = sampled_check(w)
+    assert max(e[0] for e in errs) <= MAX_ABS
+    assert max(e[1] for e in errs) <= MEAN_ABS
