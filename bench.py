@@ -450,16 +450,16 @@ def bench_gpu(args, world, rank, local):
 L2_BYTES = 126 * 1024 * 1024
 
 
-def _call_ms(fn, stream, reps, flush=None, warm=2):
-    """Mean device time of one fn() over reps calls (CUDA events on the launching
-    stream).  With `flush` (a buffer larger than L2) every call is timed alone
-    after the buffer was rewritten, so no call finds the previous one's data in
-    L2."""
+def _call_ms(fn, stream, reps, flush=None, warm=2, per_call=False):
+    """Device time of one fn() (CUDA events on the launching stream): the mean
+    over reps back-to-back calls, or, with `flush` or `per_call`, the median of
+    reps calls each timed alone.  With `flush` (a buffer larger than L2) the
+    buffer is rewritten before every call, so no call finds the previous one's
+    data in L2."""
     for _ in range(warm):
         fn()
     torch.cuda.synchronize()
-    times = []
-    if flush is None:
+    if flush is None and not per_call:
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(reps):
@@ -469,14 +469,15 @@ def _call_ms(fn, stream, reps, flush=None, warm=2):
         return a.elapsed_time(b) / reps
     evs = []
     for _ in range(reps):
-        flush.add_(1)
+        if flush is not None:
+            flush.add_(1)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         fn()
         b.record(stream)
         evs.append((a, b))
     torch.cuda.synchronize()
-    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+    return statistics.median(a.elapsed_time(b) for a, b in evs)
 
 
 def _graph_and_host_us(fn, n=50):
@@ -512,12 +513,13 @@ def _graph_and_host_us(fn, n=50):
     return graph_us, host_us
 
 
-def bench_configs(lcx, dev, stream, status, peaks, local, reps=5):
+def bench_configs(lcx, dev, stream, status, peaks, local, reps=10):
     """Every workload measured like the headline: one lcx_attn_fwd call per
     step (host table, the keys' rotate pass into a buffer, the attention kernel),
-    inputs resident in HBM.  Workloads whose inputs fit in L2 are timed call by
-    call with L2 flushed in between.  The tiny workload is launch-bound: its
-    number is the latency of one call."""
+    inputs resident in HBM; the median of `reps` calls, each timed alone.
+    Workloads whose inputs fit in L2 have L2 flushed before every call.  The
+    tiny workload is launch-bound: its number is the latency of one call (mean
+    of 200 back to back, and from a CUDA-graph replay)."""
     out = {}
     burst, sust, hbm = (float(peaks["bf16_tflops"]), float(peaks["bf16_tflops_sustained"]),
                         float(peaks["hbm_gbs"]))
@@ -538,7 +540,7 @@ def bench_configs(lcx, dev, stream, status, peaks, local, reps=5):
             tiny = w.L * w.B * w.Hq <= 4096
             n = 200 if tiny else reps
             ms = _call_ms(lambda: lcx.attn_fwd(q, k, v, rope, **kw), stream, n,
-                          flush=None if tiny else fl)
+                          flush=None if tiny else fl, per_call=not tiny)
             flops = attn_flops(w)
             tf = flops / (ms * 1e-3) / 1e12
             qr, kr = torch.empty_like(q), torch.empty_like(k)
@@ -546,12 +548,14 @@ def bench_configs(lcx, dev, stream, status, peaks, local, reps=5):
             def rope_qk():
                 lcx.apply_rope(q, rope, out=qr)
                 lcx.apply_rope(k, rope, out=kr)
-            rope_ms = _call_ms(rope_qk, stream, max(reps, 5), flush=fl)
+            rope_ms = _call_ms(rope_qk, stream, max(reps, 5), flush=fl, per_call=True)
             k_pass_ms = _call_ms(lambda: lcx.apply_rope(k, rope, out=kr), stream,
-                                 max(reps, 5), flush=fl)
+                                 max(reps, 5), flush=fl, per_call=True)
             rb = rope_bytes(w)
             e = {
                 "what": w.description, "ms_per_call": round(ms, 4), "calls": n,
+                "timing": ("mean of %d back to back" % n) if tiny else (
+                    "median of %d calls, each timed alone" % n),
                 "attn_tflops": round(tf, 2), "frac_sustained": round(tf / sust, 4),
                 "frac_burst": round(tf / burst, 4),
                 "apply_rope_gbs": round(rb / (rope_ms * 1e-3) / 1e9, 1),
