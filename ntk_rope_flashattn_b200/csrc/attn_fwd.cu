@@ -1670,19 +1670,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 namespace dec {
 constexpr int kThreads = 480;  // warps 0-3 softmax, 4-11 rotation, 12 K, 13 MMA, 14 V
 constexpr int D = 128, BN = 128, NQ = 16;
-constexpr int NSK = 3, NSV = 3, NBS = 4, NBP = 2;  // K, V stages; S^T, P buffers
-constexpr int kTile = BN * D * 2;                  // a K or V tile, bf16
-constexpr int kBox = BN * 128;                     // its 64-column boxes
-constexpr int kQBox = NQ * 128;                    // a 64-column box of the query or P block
-constexpr int kOffK = 0;
-constexpr int kOffV = kOffK + NSK * kTile;
-constexpr int kOffQ = kOffV + NSV * kTile;
-constexpr int kOffP = kOffQ + (D / 64) * kQBox;
-constexpr int kOffX = kOffP + NBP * (BN / 64) * kQBox;
-constexpr int kOffBar = kOffX + 1024;
-constexpr int kSmemBytes = kOffBar + 256 + 1024;  // barriers + alignment slack
-constexpr int kColO = NBS * NQ;                   // TMEM: NBS S^T buffers of NQ columns, then O^T
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+constexpr int NBS = 4, NBP = 2;    // S^T buffers, P buffers
+constexpr int kTile = BN * D * 2;  // a K (or K part) or V tile of 16-bit values
+constexpr int kBox = BN * 128;     // its 128-byte-wide boxes
+constexpr int kQBox = NQ * 128;    // a 128-byte-wide box of the query or P block
+constexpr int kColO = NBS * NQ;    // TMEM: NBS S^T buffers of NQ columns, then O^T
+// Shared-memory plan.  bf16 QK^T: three K and three V stages.  Split QK^T
+// (keys as the fp16 part plus the 8-bit cross part, 64 KB a stage; V in fp16):
+// two of each.  Then the query block (its parts), two P buffers, the column
+// exchange area and the barriers.
+template <bool kSplitQK>
+struct Cfg {
+    static constexpr int kParts = kSplitQK ? 2 : 1;
+    static constexpr int NSK = kSplitQK ? 2 : 3, NSV = kSplitQK ? 2 : 3;
+    static constexpr int kOffK = 0;
+    static constexpr int kOffV = kOffK + NSK * kParts * kTile;
+    static constexpr int kOffQ = kOffV + NSV * kTile;
+    static constexpr int kOffP = kOffQ + kParts * (D / 64) * kQBox;
+    static constexpr int kOffX = kOffP + NBP * (BN / 64) * kQBox;
+    static constexpr int kOffBar = kOffX + 1024;
+    static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // barriers + alignment slack
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+template <int NSK, int NSV>
 struct Bars {
     uint64_t ready_q;
     uint64_t full_k[NSK], ready_k[NSK], empty_k[NSK];
@@ -1692,16 +1702,17 @@ struct Bars {
     uint32_t tmem_base;
     int abort;
 };
-static_assert(sizeof(Bars) <= 256, "barrier block");
+static_assert(sizeof(Bars<3, 3>) <= 256, "barrier block");
 }  // namespace dec
 
 // The group's query block: row n = k L + i holds query i of head hq0 + k
 // (n < nq; the other rows are zero), rotated at position qoff + i unless the
 // queries arrive rotated, stored as the K-major B operand of S^T (two 64-column
-// boxes of NQ 128-byte rows, 128-byte swizzle).  Thread tw (of 128) takes row
-// tw / 8 and its pairs 8 (tw % 8) .. + 7: two 16-byte loads, two 16-byte
-// stores; each angle from the accurate sine and cosine.
-template <bool kHalf>
+// boxes of NQ 128-byte rows, 128-byte swizzle; split QK^T: the fp16 part, then
+// the 8-bit cross part in as many boxes).  Thread tw (of 128) takes row tw / 8
+// and its pairs 8 (tw % 8) .. + 7: two 16-byte loads; each angle from the
+// accurate sine and cosine.
+template <bool kHalf, bool kSplitQK>
 __device__ __forceinline__ void load_q_decode(uint8_t *sQ, const AttnParams &p, const Unit &U,
                                               int nq, int tw) {
     using namespace dec;
@@ -1709,18 +1720,18 @@ __device__ __forceinline__ void load_q_decode(uint8_t *sQ, const AttnParams &p, 
     const int n = tw >> 3, g = tw & 7;
     // the 16-byte chunks (8 columns each) that hold the thread's pairs
     const int c1 = kHalf ? g : 2 * g, c2 = kHalf ? g + D / 16 : 2 * g + 1;
-    uint4 a = make_uint4(0u, 0u, 0u, 0u), b = a;
+    float x[8], y[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = y[e] = 0.f;
     if (n < nq) {
         const int i = n % p.L;
         const uint4 *row = reinterpret_cast<const uint4 *>(
             reinterpret_cast<const __nv_bfloat16 *>(p.q) + U.b * p.qs[0] +
             (long long)(U.hq0 + n / p.L) * p.qs[1] + (long long)i * p.qs[2]);
-        a = row[c1];
-        b = row[c2];
+        unpack8(row[c1], x);
+        unpack8(row[c2], y);
         if (p.rotate_q) {
-            float x[8], y[8], c[8], s[8];
-            unpack8(a, x);
-            unpack8(b, y);
+            float c[8], s[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
                 rope_sincos((long long)p.qoff + i, p.theta[8 * g + e], &c[e], &s[e]);
@@ -1734,33 +1745,43 @@ __device__ __forceinline__ void load_q_decode(uint8_t *sQ, const AttnParams &p, 
                 u = u0 * c[e] - v0 * s[e];
                 v = v0 * c[e] + u0 * s[e];
             }
-            a = pack8(x);
-            b = pack8(y);
         }
     }
-    *reinterpret_cast<uint4 *>(sQ + chunk_off(n, c1, kQBox)) = a;
-    *reinterpret_cast<uint4 *>(sQ + chunk_off(n, c2, kQBox)) = b;
+    if constexpr (kSplitQK) {
+        // the fp16 part, and the 8-bit cross part [h8 | r8], of the rotated values
+        store8<true, false, D, kQBox>(sQ, sQ + (D / 64) * kQBox, n, c1, x);
+        store8<true, false, D, kQBox>(sQ, sQ + (D / 64) * kQBox, n, c2, y);
+    } else {
+        *reinterpret_cast<uint4 *>(sQ + chunk_off(n, c1, kQBox)) = pack8(x);
+        *reinterpret_cast<uint4 *>(sQ + chunk_off(n, c2, kQBox)) = pack8(y);
+    }
 }
 
 // One CTA per (batch, kv group, key split): bf16 operands, D = DV = 128, full
 // rotary, partial results (o normalised, lse) into the split workspace.  kNQ:
-// the query columns the softmax reads (4, 8 or 16 >= G L).
-template <bool kHalf, int kNQ>
+// the query columns the softmax reads (4, 8 or 16 >= G L).  kSplitQK: the
+// split mode's S = Qh Kh^T + [Qh8 | Qr8] [Kr8 | Kh8]^T, transposed, with the
+// keys' parts and V in fp16 as the rotate pass wrote them (tmk: the fp16 parts,
+// tmkr: the 8-bit cross parts), and fp16 weights for PV.
+template <bool kHalf, int kNQ, bool kSplitQK>
 __global__ void __launch_bounds__(dec::kThreads, 1)
     attn_decode_kernel(const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmv,
+                       const __grid_constant__ CUtensorMap tmkr,
                        const __grid_constant__ AttnParams p) {
     using namespace dec;
+    using C = dec::Cfg<kSplitQK>;
+    constexpr int NSK = C::NSK, NSV = C::NSV;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sK = smem + kOffK;
-    uint8_t *sV = smem + kOffV;
-    uint8_t *sQ = smem + kOffQ;
-    uint8_t *sP = smem + kOffP;
-    float *xmax = reinterpret_cast<float *>(smem + kOffX);  // [2][4][kNQ] column maxima per warp
-    float *xsum = xmax + 2 * 4 * kNQ;                        // [4][kNQ] column sums per warp
-    dec::Bars &bar = *reinterpret_cast<dec::Bars *>(smem + kOffBar);
+    uint8_t *sK = smem + C::kOffK;  // stage s at sK + s kParts kTile (split: fp16 part, 8-bit part)
+    uint8_t *sV = smem + C::kOffV;
+    uint8_t *sQ = smem + C::kOffQ;
+    uint8_t *sP = smem + C::kOffP;
+    float *xmax = reinterpret_cast<float *>(smem + C::kOffX);  // [2][4][kNQ] column maxima per warp
+    float *xsum = xmax + 2 * 4 * kNQ;                           // [4][kNQ] column sums per warp
+    dec::Bars<NSK, NSV> &bar = *reinterpret_cast<dec::Bars<NSK, NSV> *>(smem + C::kOffBar);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -1828,16 +1849,23 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
             uint8_t *base = isk ? sK : sV;
             const CUtensorMap *map = isk ? &tmk : &tmv;
             tma_prefetch_desc(map);
+            if (kSplitQK && isk) tma_prefetch_desc(&tmkr);
+            // split mode: a K stage is the fp16 part then the 8-bit cross part
+            const int parts = (kSplitQK && isk) ? 2 : 1;
             int issued[NS] = {};
             bool ok = true;
             for (int j = 0; ok && j < T.n; ++j) {
                 const int jt = T.tile(j), s = j % ns, u = j / ns;
                 if (u > 0) ok = mbar_wait(&empty[s], (u - 1) & 1, abort, tmo);
                 if (!ok) break;
-                mbar_arrive_expect_tx(&full[s], kTile);
+                uint8_t *dst = base + s * parts * kTile;
+                mbar_arrive_expect_tx(&full[s], parts * kTile);
                 for (int bx = 0; bx < D / 64; ++bx)
-                    tma_load_4d(base + s * kTile + bx * kBox, map, &full[s], bx * 64, jt * BN,
-                                U.g, U.b);
+                    tma_load_4d(dst + bx * kBox, map, &full[s], bx * 64, jt * BN, U.g, U.b);
+                if (parts == 2)   // 2 D bytes per key: D / 64 boxes of 128 bytes
+                    for (int bx = 0; bx < D / 64; ++bx)
+                        tma_load_4d(dst + kTile + bx * kBox, &tmkr, &full[s], bx * 128, jt * BN,
+                                    U.g, U.b);
                 ++issued[s];
             }
             // never leave the CTA with copies in flight (bounded, even after an abort)
@@ -1849,8 +1877,11 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
         if (lane == 0) {
             // S^T: A = the K tile, B = the query block, both K-major.  O^T: A = the
             // V tile, MN-major; B = the weights, K-major.  M = 128, N = NQ.
-            constexpr uint32_t kIdS = idesc_bf16_f32(128, NQ, 0, 0);
-            constexpr uint32_t kIdO = idesc_bf16_f32(128, NQ, 1, 0);
+            constexpr uint32_t kIdS = kSplitQK ? idesc_f32acc(128, NQ, kFmtF16, kFmtF16, 0, 0)
+                                               : idesc_bf16_f32(128, NQ, 0, 0);
+            constexpr uint32_t kIdX8 = idesc_f32acc(128, NQ, kFmtE5M2, kFmtE5M2, 0, 0);
+            constexpr uint32_t kIdO = kSplitQK ? idesc_f32acc(128, NQ, kFmtF16, kFmtF16, 1, 0)
+                                               : idesc_bf16_f32(128, NQ, 1, 0);
             const uint64_t dv0 = sdesc_sw128(smem_u32(sV), kBox, 1024);
             const uint32_t dhi = uint32_t(dv0 >> 32);  // the same for every descriptor here
             const uint32_t v_lo = uint32_t(dv0);
@@ -1859,13 +1890,24 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
             const uint32_t p_lo = uint32_t(sdesc_sw128(smem_u32(sP), 16, 1024));
             uint64_t *kready = p.rotate_k ? bar.ready_k : bar.full_k;
             auto issue_s = [&](int j) {
-                const uint32_t ka = k_lo + (((j % NSK) * kTile) >> 4);
+                const uint32_t ka = k_lo + (((j % NSK) * C::kParts * kTile) >> 4);
                 const uint32_t dst = tmem + (j % NBS) * NQ;
+                if constexpr (kSplitQK) {
+                    // the e5m2 cross product over K = 2 D bytes (32 per
+                    // instruction, the same box geometry as the 16-bit parts)
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t ok_ = ((kk >> 2) * kBox + (kk & 3) * 32) >> 4;
+                        const uint32_t oq = ((kk >> 2) * kQBox + (kk & 3) * 32) >> 4;
+                        mma_ss_w<1>(dst, ka + (kTile >> 4) + ok_,
+                                    q_lo + (((D / 64) * kQBox) >> 4) + oq, dhi, kIdX8, kk > 0);
+                    }
+                }
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ok_ = ((kk >> 2) * kBox + (kk & 3) * 32) >> 4;
                     const uint32_t oq = ((kk >> 2) * kQBox + (kk & 3) * 32) >> 4;
-                    mma_ss_w<0>(dst, ka + ok_, q_lo + oq, dhi, kIdS, kk > 0);
+                    mma_ss_w<0>(dst, ka + ok_, q_lo + oq, dhi, kIdS, kSplitQK || kk > 0);
                 }
             };
             auto issue_pv = [&](int j) {
@@ -1917,11 +1959,12 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
         // ------------------------------------------------ queries, then key rotation
         const int tw = threadIdx.x - 128;  // 0..255
         if (tw < 128) {
-            load_q_decode<kHalf>(sQ, p, U, nq, tw);
+            load_q_decode<kHalf, kSplitQK>(sQ, p, U, nq, tw);
             fence_proxy_async_smem();
             mbar_arrive(&bar.ready_q);
         }
-        if (p.rotate_k)
+        // (split mode: the keys always arrive in their parts from the rotate pass)
+        if (!kSplitQK && p.rotate_k)
             rotate_keys_helped<D, D, kHalf, false, NSK, BN, 1, kTile>(tw, T, sK, bar, p, abort,
                                                                       tmo);
     } else {
@@ -2021,14 +2064,18 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
                 }
             }
             if (ok) {
-                // the weights 2^(s c - m), bf16, into row n of the K-major P block
+                // the weights 2^(s c - m), bf16 (split mode: fp16, for the fp16
+                // V), into row n of the K-major P block
                 uint8_t *pbuf = sP + pb * (BN / 64) * kQBox;
 #pragma unroll
                 for (int n = 0; n < kNQ; ++n) {
                     const float w = ex2_approx(x[n] - (m[n] == -INFINITY ? 0.f : m[n]));
                     l[n] += w;
-                    *reinterpret_cast<__nv_bfloat16 *>(pbuf + chunk_off(n, r >> 3, kQBox) +
-                                                       (r & 7) * 2) = __float2bfloat16_rn(w);
+                    uint8_t *dst = pbuf + chunk_off(n, r >> 3, kQBox) + (r & 7) * 2;
+                    if constexpr (kSplitQK)
+                        *reinterpret_cast<uint16_t *>(dst) = uint16_t(pack_f16x2(w, 0.f) & 0xFFFFu);
+                    else
+                        *reinterpret_cast<__nv_bfloat16 *>(dst) = __float2bfloat16_rn(w);
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
@@ -2181,26 +2228,26 @@ lcx_status launch_shape(const AttnLaunchShape &x, const Maps &m, const AttnParam
 }
 
 // The transposed decode kernel (bf16, D = DV = 128, full rotary, G L <= 16).
-template <bool kHalf, int kNQ>
+template <bool kHalf, int kNQ, bool kSplitQK>
 lcx_status launch_decode(const Maps &m, const AttnParams &p, unsigned grid, cudaStream_t s) {
-    auto kern = attn_decode_kernel<kHalf, kNQ>;
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kSmemBytes);
+    auto kern = attn_decode_kernel<kHalf, kNQ, kSplitQK>;
+    constexpr int smem = dec::Cfg<kSplitQK>::kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess)
         return fail(LCX_ERR_CUDA, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
-    kern<<<grid, dec::kThreads, dec::kSmemBytes, s>>>(m.k, m.v, p);
+    kern<<<grid, dec::kThreads, smem, s>>>(m.k, m.v, m.kr, p);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return fail(LCX_ERR_CUDA, "attn_decode launch failed: %s", cudaGetErrorString(e));
     return LCX_OK;
 }
 
-template <bool kHalf>
+template <bool kHalf, bool kSplitQK>
 lcx_status launch_decode_nq(int nq, const Maps &m, const AttnParams &p, unsigned grid,
                             cudaStream_t s) {
-    return nq <= 4 ? launch_decode<kHalf, 4>(m, p, grid, s)
-                   : nq <= 8 ? launch_decode<kHalf, 8>(m, p, grid, s)
-                             : launch_decode<kHalf, 16>(m, p, grid, s);
+    return nq <= 4 ? launch_decode<kHalf, 4, kSplitQK>(m, p, grid, s)
+                   : nq <= 8 ? launch_decode<kHalf, 8, kSplitQK>(m, p, grid, s)
+                             : launch_decode<kHalf, 16, kSplitQK>(m, p, grid, s);
 }
 
 lcx_status check_tensor(const void *ptr, const int64_t *st, int es, const char *name) {
@@ -2496,8 +2543,11 @@ lcx_status attn_enqueue(const AttnLaunch &x, cudaStream_t s) {
     const unsigned g = unsigned(grid);
     if (x.decode) {
         const int nq = x.p.G * x.p.L;
-        return x.half ? launch_decode_nq<true>(nq, x.m, x.p, g, s)
-                      : launch_decode_nq<false>(nq, x.m, x.p, g, s);
+        if (x.split_qk)
+            return x.half ? launch_decode_nq<true, true>(nq, x.m, x.p, g, s)
+                          : launch_decode_nq<false, true>(nq, x.m, x.p, g, s);
+        return x.half ? launch_decode_nq<true, false>(nq, x.m, x.p, g, s)
+                      : launch_decode_nq<false, false>(nq, x.m, x.p, g, s);
     }
     return x.p.n_split > 1 ? launch_shape<true>(x, x.m, x.p, g, s)
                            : launch_shape<false>(x, x.m, x.p, g, s);
@@ -2585,8 +2635,10 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
     // A kv group's G L queries fit in the columns of one transposed score
     // block (bf16, D = DV = 128, full rotary): the decode kernel, one CTA per
     // (batch, kv group, split), one partial result per split.
-    x.decode = !x.f32 && !x.split_qk && x.D == 128 && x.DV == 128 && x.RD == 128 &&
-               !x.p.k_rope_shared && int64_t(x.p.G) * a->L <= dec::NQ;
+    // Split QK^T: with the keys' parts and V in fp16 from the rotate pass.
+    x.decode = !x.f32 && x.D == 128 && x.DV == 128 && x.RD == 128 && !x.p.k_rope_shared &&
+               int64_t(x.p.G) * a->L <= dec::NQ &&
+               (!x.split_qk || (x.p.k_x8_tma && x.p.v_f16));
     if (x.decode) {
         x.p.qpair = 0;
         x.p.heads_per_unit = x.p.G;

@@ -180,6 +180,10 @@ def test_splitkv_interleaved_key_tiles(L, Lk, splits, extra):
     (1, 2000, 5, dict(Hq=8, Hkv=2, rotate_k_once=True)),       # keys rotated by the pass
     (1, 2000, 5, dict(Hq=8, Hkv=2, prerotated=True)),          # q and k arrive rotated
     (4, 1000, 3, dict(Hq=8, Hkv=2, causal=False)),
+    # split QK^T (keys' fp16 and 8-bit parts and V in fp16 from the rotate pass)
+    (1, 2000, 5, dict(Hq=8, Hkv=2, split_qk=True, rotate_k_once=True)),
+    (2, 1500, 3, dict(Hq=8, Hkv=2, pairing="interleaved", split_qk=True, rotate_k_once=True)),
+    (3, 3000, 6, dict(Hq=6, Hkv=2, window=900, sinks=5, split_qk=True, rotate_k_once=True)),
 ])
 def test_splitkv_transposed_decode(L, Lk, splits, extra):
     """Key-split launches whose kv group holds at most 16 queries (bf16, D = 128,
@@ -200,6 +204,23 @@ def test_splitkv_transposed_decode(L, Lk, splits, extra):
         q_in = lcx.apply_rope(q_all, rope)[:, :, Lk - L:]
         k_in = lcx.apply_rope(k, rope)
     o, lse = run_split(q_in, k_in, v, rope, splits, causal=causal, window=w.window,
-                       sinks=w.sinks, q_offset=Lk - L, prerotated=prerot, rotate_k_once=once)
+                       sinks=w.sinks, q_offset=Lk - L, prerotated=prerot, rotate_k_once=once,
+                       split_qk=w.split_qk)
     ref = oracle_rows(q, k, v, rope, Lk - L, causal, w.window, w.sinks)
+    compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref[0], ref[1])
+
+
+@pytest.mark.parametrize("splits", [4, 9])
+def test_splitkv_decode_outlier_workload(splits):
+    """A decode step of the outlier workload (8x outliers on 1% of the channels,
+    YaRN s=8, a 4096-key window and 4 sinks) in its split-QK^T mode with the
+    keys split once by the rotate pass: the transposed decode kernel's fp16 and
+    e5m2 products against the oracle, every head, two batches."""
+    w = WORKLOADS["sink_window_L65536"].with_(B=2, L=9000)
+    q_all, k, v = make_inputs(w, device="cuda")
+    q = q_all[:, :, w.L - 1:]
+    rope = rope_of(w)
+    o, lse = run_split(q, k, v, rope, splits, window=w.window, sinks=w.sinks,
+                       q_offset=w.L - 1, split_qk=True, rotate_k_once=True)
+    ref = oracle_rows(q, k, v, rope, w.L - 1, True, w.window, w.sinks)
     compare(o.float().cpu().numpy(), lse.cpu().numpy(), ref[0], ref[1])
