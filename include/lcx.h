@@ -288,9 +288,10 @@ LCX_API lcx_status lcx_attn_fwd(const lcx_attn_args *args, void *stream);
  *   programmatic dependent launch that waits for the attention kernel before
  *   reading its results).  With bf16 operands, D = Dv = rope.head_dim = 128,
  *   no k_rope and at most 16 queries per kv group (G L <= 16, e.g. a decode
- *   step), the attention kernel is the transposed-score decode kernel (one CTA
- *   per batch, kv group and split; keys along the tensor-memory lanes, the
- *   group's queries along its columns).  Errors as for lcx_attn_fwd; a short
+ *   step), and in the split-QK^T mode only with args.k_rot (keys split by the
+ *   rotate pass), the attention kernel is the transposed-score decode kernel
+ *   (one CTA per batch, kv group and split; keys along the tensor-memory
+ *   lanes, the group's queries along its columns).  Errors as for lcx_attn_fwd; a short
  *   workspace is LCX_ERR_INVALID_ARG.
  */
 LCX_API lcx_status lcx_attn_fwd_split(const lcx_attn_args *args, int32_t num_splits,
