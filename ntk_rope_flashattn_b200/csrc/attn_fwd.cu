@@ -893,8 +893,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bar.o_ready[t], 1);
         }
         mbar_init(&bar.drain, 1);
-        // A CTA that starts after another one's watchdog fired does no work.
-        bar.abort = p.status ? *reinterpret_cast<volatile int *>(p.status) : 0;
+        bar.abort = 0;
         fence_mbar_init();
     }
     if (warp == kWarpMma) {
@@ -905,14 +904,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar.tmem_base;
-    const bool skip = bar.abort != 0;
+    // A CTA that starts after another one's watchdog fired gives up at its
+    // first wait that does not complete at once: thread 0 reads the status
+    // word here, after the barrier, so no role waits for that load to start.
+    bool pre = false;   // thread 0: the word was already set
+    if (threadIdx.x == 0 && p.status && *reinterpret_cast<volatile int *>(p.status) != 0) {
+        pre = true;
+        *abort = 1;
+    }
     // key splits: the merge may be scheduled now (it waits for this grid to
     // finish before it reads the partial results)
     if constexpr (kKvSplit) pdl_launch_dependents();
 
-    if (skip) {
-        // nothing to do: fall through to the common exit
-    } else if (kKvSplit && T.n == 0) {
+    if (kKvSplit && T.n == 0) {
         // A key split that received no tile (more splits than tiles): the
         // empty partial result, o = 0 and lse = -inf.
         if (warp < 8 && (warp >> 2) < U.nt) {
@@ -1649,7 +1653,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
-    if (threadIdx.x == 0 && !skip && bar.abort && p.status)
+    if (threadIdx.x == 0 && !pre && bar.abort && p.status)
         atomicExch(p.status, int(LCX_ERR_TIMEOUT));
 }
 
@@ -1809,8 +1813,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
         }
         mbar_init(&bar.o_ready, 1);
         mbar_init(&bar.drain, 1);
-        // A CTA that starts after another one's watchdog fired does no work.
-        bar.abort = p.status ? *reinterpret_cast<volatile int *>(p.status) : 0;
+        bar.abort = 0;
         fence_mbar_init();
     }
     if (warp == 13) {
@@ -1821,14 +1824,19 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar.tmem_base;
-    const bool skip = bar.abort != 0;
+    // A CTA that starts after another one's watchdog fired gives up at its
+    // first wait that does not complete at once (the status word is read by
+    // thread 0 after the barrier, off the roles' path).
+    bool pre = false;   // thread 0: the word was already set
+    if (threadIdx.x == 0 && p.status && *reinterpret_cast<volatile int *>(p.status) != 0) {
+        pre = true;
+        *abort = 1;
+    }
     // the merge of the partial results may be scheduled now (it waits for this
     // grid to finish before it reads them)
     pdl_launch_dependents();
 
-    if (skip) {
-        // nothing to do: fall through to the common exit
-    } else if (T.n == 0) {
+    if (T.n == 0) {
         // a split that received no key tile: the empty partial result
         if (warp < 4) {
             for (int n = 0; n < nq; ++n) {
@@ -2114,7 +2122,7 @@ __global__ void __launch_bounds__(dec::kThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, 128);
     }
-    if (threadIdx.x == 0 && !skip && bar.abort && p.status)
+    if (threadIdx.x == 0 && !pre && bar.abort && p.status)
         atomicExch(p.status, int(LCX_ERR_TIMEOUT));
 }
 
