@@ -61,7 +61,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # launch on the headline workload (yarn_L131072_s16), from a one-pass ncu capture
 # of the current kernel (keys pre-rotated by the rotate pass); None until the
 # current kernel has been captured.  Only valid for that workload.
-ATTN_TRAFFIC_BYTES = {"yarn_L131072_s16": 3034403072 + 1091801856}
+ATTN_TRAFFIC_BYTES = {"yarn_L131072_s16": 2987733248 + 1077540864}
 
 
 def load_peaks():
