@@ -129,6 +129,8 @@ struct AttnParams {
     int k_rope_shared;                 // rotated key columns come from one shared head
     int k_x8_tma;                      // split mode: the keys' 8-bit cross parts arrive by TMA
     int v_f16;                         // split mode: V arrives in fp16 (converted by a pass)
+    int persist;                       // split mode: each CTA takes units blockIdx.x + k gridDim.x
+    int n_units;                       //   of the n_units, one after the other
     float rot_ms;                      // factor on rotated values (partial rotary: mscale)
     float c_log2;                      // logit scale in log2 units
     unsigned long long timeout_ns;
@@ -216,6 +218,7 @@ struct Bars {
     uint64_t full_k[NSK], ready_k[NSK], empty_k[NSK];
     uint64_t full_v[NSV], empty_v[NSV], fp16_v[NSV];
     uint64_t s_ready[2][2], p_ready[2][2], o_ready[2];
+    uint64_t o_free;   // persistent split mode: the epilogue has read O
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -238,8 +241,8 @@ struct Unit {
 // -- and still hands out the longest units of every group first.  With key
 // splits (kKvSplit), the n_split CTAs of a unit are consecutive.
 template <bool kKvSplit>
-__device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
-    const int u = kKvSplit ? int(blockIdx.x) / p.n_split : int(blockIdx.x);
+__device__ __forceinline__ Unit decode_unit(const AttnParams &p, int unit = -1) {
+    const int u = unit >= 0 ? unit : kKvSplit ? int(blockIdx.x) / p.n_split : int(blockIdx.x);
     const int upq = p.G / p.heads_per_unit;          // units per query block of a group
     const int per_group = p.n_qb * upq;
     const int grp = u / per_group, rem = u % per_group;
@@ -829,7 +832,8 @@ __device__ __forceinline__ void rotate_keys_helped(int tw, const Tiles &T, uint8
 // ---------------------------------------------------------------- kernel
 // D: query/key head dim, DV: value/output head dim, RD: rotated (last) dims;
 // kKvSplit: this launch is one pass of split-KV (partial results per split).
-template <int D, int DV, int RD, bool kF32, bool kHalf, bool kSplit, bool kKvSplit>
+template <int D, int DV, int RD, bool kF32, bool kHalf, bool kSplit, bool kKvSplit,
+          bool kPersist = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq,
                     const __grid_constant__ CUtensorMap tmk,
@@ -893,6 +897,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bar.o_ready[t], 1);
         }
         mbar_init(&bar.drain, 1);
+        mbar_init(&bar.o_free, 256);
         bar.abort = 0;
         fence_mbar_init();
     }
@@ -938,7 +943,73 @@ __global__ void __launch_bounds__(kThreads, 1)
         setmaxnreg_dec<kRegsIssue>();
         if (warp == kWarpTma) {
             // ------------------------------------------------ TMA producer
-            if (!kF32 && lane == 0 && !p.test_stall) {
+            constexpr bool persistent = kPersist;
+            if constexpr (kPersist) {
+                static_assert(kSplit && !kKvSplit && C::kKFreeOnS, "persistent split mode");
+                // Persistent split mode: per unit, the query tile into its staging
+                // area (the last K stage) once the last key tile there has been
+                // multiplied, then the unit's key tiles, stages counted across
+                // units; the first key tile into the staging stage waits until the
+                // query's parts have moved to TMEM.
+                if (lane == 0) {
+                    tma_prefetch_desc(&tmq);
+                    tma_prefetch_desc(&tmk);
+                    if (p.k_x8_tma) tma_prefetch_desc(&tmkr);
+                    int issued_k[NSK] = {};
+                    int nq = 0, g = 0;
+                    bool ok = true;
+                    for (int ku = 0; ok; ++ku) {
+                        const int uu = int(blockIdx.x) + ku * int(gridDim.x);
+                        if (uu >= p.n_units) break;
+                        const Unit Uu = decode_unit<kKvSplit>(p, uu);
+                        const Tiles Tu = make_tiles<BN, kKvSplit>(Uu.q0, Uu.split, p);
+                        if (ku > 0) {
+                            // the previous query tile has left the staging area (a
+                            // unit whose key tiles all went to other stages never
+                            // waited for that below) ...
+                            ok = mbar_wait(&bar.ready_q, (ku - 1) & 1, abort, tmo);
+                            // ... and the last key tile (index < g) in that stage
+                            // has been multiplied
+                            const int gl = (g - 1) - (((g - 1) - (NSK - 1)) % NSK + NSK) % NSK;
+                            if (ok && gl >= 0)
+                                ok = mbar_wait(&bar.s_ready[0][gl % C::kNB], (gl / C::kNB) & 1,
+                                               abort, tmo);
+                        }
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(&bar.full_q, C::kTileQ);
+                        for (int bx = 0; bx < D / 64; ++bx)
+                            tma_load_4d(sQ + bx * C::kBoxQ, &tmq, &bar.full_q, bx * 64, Uu.tq0(0),
+                                        Uu.th(0), Uu.b);
+                        ++nq;
+                        bool staged = true;
+                        for (int j = 0; ok && j < Tu.n; ++j, ++g) {
+                            const int jt = Tu.tile(j), sk = g % NSK, uk = g / NSK;
+                            if (uk > 0) ok = mbar_wait(&bar.s_ready[0][sk], (uk - 1) & 1, abort, tmo);
+                            if (ok && sk == NSK - 1 && staged) {
+                                ok = mbar_wait(&bar.ready_q, ku & 1, abort, tmo);
+                                staged = false;
+                            }
+                            if (!ok) break;
+                            const bool x8 = p.k_x8_tma != 0;
+                            uint8_t *st = sK + sk * C::kParts * C::kTileK;
+                            mbar_arrive_expect_tx(&bar.full_k[sk], x8 ? 2 * C::kTileK : C::kTileK);
+                            if (x8)
+                                for (int bx = 0; bx < D / 64; ++bx)
+                                    tma_load_4d(st + C::kTileK + bx * C::kBoxK, &tmkr, &bar.full_k[sk],
+                                                bx * 128, jt * BN, Uu.g, Uu.b);
+                            for (int bx = 0; bx < D / 64; ++bx)
+                                tma_load_4d(st + bx * C::kBoxK, &tmk, &bar.full_k[sk], bx * 64,
+                                            jt * BN, Uu.g, Uu.b);
+                            ++issued_k[sk];
+                        }
+                    }
+                    // never leave the CTA with copies in flight (bounded)
+                    if (nq) mbar_wait(&bar.full_q, (nq - 1) & 1, nullptr, tmo);
+                    for (int s = 0; s < NSK; ++s)
+                        if (issued_k[s]) mbar_wait(&bar.full_k[s], (issued_k[s] - 1) & 1, nullptr, tmo);
+                }
+            }
+            if (!persistent && !kF32 && lane == 0 && !p.test_stall) {
                 tma_prefetch_desc(&tmq);
                 tma_prefetch_desc(&tmk);
                 tma_prefetch_desc(&tmv);
@@ -1012,7 +1083,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             // V tiles come from their own warp, so a V stage that frees late (one
             // V stage: after the last PV of the previous tile) never holds back the
             // next K tile behind it.
-            if (!kF32 && lane == 0 && !p.test_stall) {
+            constexpr bool persistent = kPersist;
+            if constexpr (kPersist) {
+                // persistent split mode: the units' V tiles, stages counted across units
+                if (lane == 0) {
+                    int issued_v[NSV] = {};
+                    int g = 0;
+                    bool ok = true;
+                    for (int ku = 0; ok; ++ku) {
+                        const int uu = int(blockIdx.x) + ku * int(gridDim.x);
+                        if (uu >= p.n_units) break;
+                        const Unit Uu = decode_unit<kKvSplit>(p, uu);
+                        const Tiles Tu = make_tiles<BN, kKvSplit>(Uu.q0, Uu.split, p);
+                        for (int j = 0; ok && j < Tu.n; ++j, ++g) {
+                            const int jt = Tu.tile(j), sv = g % NSV, uv = g / NSV;
+                            if (uv > 0) ok = mbar_wait(&bar.empty_v[sv], (uv - 1) & 1, abort, tmo);
+                            if (!ok) break;
+                            mbar_arrive_expect_tx(&bar.full_v[sv], C::kTileV);
+                            for (int bx = 0; bx < DV / 64; ++bx)
+                                tma_load_4d(sV + sv * C::kTileV + bx * C::kBoxK, &tmv, &bar.full_v[sv],
+                                            bx * 64, jt * BN, Uu.g, Uu.b);
+                            ++issued_v[sv];
+                        }
+                    }
+                    for (int s = 0; s < NSV; ++s)
+                        if (issued_v[s]) mbar_wait(&bar.full_v[s], (issued_v[s] - 1) & 1, nullptr, tmo);
+                }
+            }
+            if (!persistent && !kF32 && lane == 0 && !p.test_stall) {
                 int issued_v[NSV] = {};
                 bool ok = true;
                 for (int j = 0; ok && j < T.n; ++j) {
@@ -1195,39 +1293,64 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // softmax that rescales O waits there); with as many K stages
                     // as S buffers, S(j)'s completion also frees its K stage.
                     static_assert(C::kNTQ == 1, "one query tile with two S buffers");
-                    for (int jj = 0; ok && jj < NB && jj < T.n; ++jj) {
-                        ok = mbar_wait(&kready[jj % NSK], (jj / NSK) & 1, abort, tmo);
-                        tc_fence_after();
-                        if (!ok) break;
-                        issue_s(0, jj % NSK, jj % NB);
-                        mma_commit(&bar.s_ready[0][jj % NB]);
-                        if (!C::kKFreeOnS) mma_commit(&bar.empty_k[jj % NSK]);
-                    }
-                    for (int j = 0; ok && j < T.n; ++j) {
-                        const int sv = j % NSV, jn = j + NB, b = j % NB, sk = jn % NSK;
-                        // The three phases are polled together first: each test's
-                        // result takes ~100 cycles to come back, so polling them
-                        // one after the other would keep the tensor core waiting.
-                        const bool kr = jn >= T.n || mbar_try_wait(&kready[sk], (jn / NSK) & 1);
-                        const bool all = kr & mbar_try_wait(&vready[sv], (j / NSV) & 1) &
-                                         mbar_try_wait(&bar.p_ready[0][b], (j / NB) & 1);
-                        if (!all) {
-                            if (jn < T.n) ok = mbar_wait(&kready[sk], (jn / NSK) & 1, abort, tmo);
-                            if (ok) ok = mbar_wait(&vready[sv], (j / NSV) & 1, abort, tmo);
-                            if (ok) ok = mbar_wait(&bar.p_ready[0][b], (j / NB) & 1, abort, tmo);
+                    // Persistent launches: the units of this CTA one after the
+                    // other, S buffers, K and V stages counted across them (g);
+                    // a later unit's first PV waits until the previous unit's
+                    // epilogue has read O.
+                    int g = 0;
+                    for (int ku = 0; ok; ++ku) {
+                        const int uu = int(blockIdx.x) + ku * int(gridDim.x);
+                        if (kPersist ? uu >= p.n_units : ku > 0) break;
+                        const Tiles Tu =
+                            kPersist ? make_tiles<BN, kKvSplit>(decode_unit<kKvSplit>(p, uu).q0, 0, p)
+                                     : T;
+                        if (ku > 0) {
+                            ok = mbar_wait(&bar.ready_q, ku & 1, abort, tmo);
+                            tc_fence_after();
+                            if (!ok) break;
                         }
-                        tc_fence_after();
-                        if (!ok) break;
-                        issue_pv(0, sv, b, j > 0);
-                        mma_commit(&bar.empty_v[sv]);
-                        if (jn < T.n) {
-                            issue_s(0, sk, b);
-                            mma_commit(&bar.s_ready[0][b]);
-                            if (!C::kKFreeOnS) mma_commit(&bar.empty_k[sk]);
+                        for (int jj = 0; ok && jj < NB && jj < Tu.n; ++jj) {
+                            const int gj = g + jj;
+                            ok = mbar_wait(&kready[gj % NSK], (gj / NSK) & 1, abort, tmo);
+                            tc_fence_after();
+                            if (!ok) break;
+                            issue_s(0, gj % NSK, gj % NB);
+                            mma_commit(&bar.s_ready[0][gj % NB]);
+                            if (!C::kKFreeOnS) mma_commit(&bar.empty_k[gj % NSK]);
                         }
+                        for (int j = 0; ok && j < Tu.n; ++j) {
+                            const int gj = g + j;
+                            const int sv = gj % NSV, jn = gj + NB, b = gj % NB, sk = jn % NSK;
+                            const bool more = j + NB < Tu.n;
+                            // The three phases are polled together first: each test's
+                            // result takes ~100 cycles to come back, so polling them
+                            // one after the other would keep the tensor core waiting.
+                            const bool kr = !more || mbar_try_wait(&kready[sk], (jn / NSK) & 1);
+                            const bool all = kr & mbar_try_wait(&vready[sv], (gj / NSV) & 1) &
+                                             mbar_try_wait(&bar.p_ready[0][b], (gj / NB) & 1);
+                            if (!all) {
+                                if (more) ok = mbar_wait(&kready[sk], (jn / NSK) & 1, abort, tmo);
+                                if (ok) ok = mbar_wait(&vready[sv], (gj / NSV) & 1, abort, tmo);
+                                if (ok) ok = mbar_wait(&bar.p_ready[0][b], (gj / NB) & 1, abort, tmo);
+                            }
+                            if (kPersist && ok && j == 0 && ku > 0)
+                                ok = mbar_wait(&bar.o_free, (ku - 1) & 1, abort, tmo);
+                            tc_fence_after();
+                            if (!ok) break;
+                            issue_pv(0, sv, b, j > 0);
+                            mma_commit(&bar.empty_v[sv]);
+                            if (more) {
+                                issue_s(0, sk, b);
+                                mma_commit(&bar.s_ready[0][b]);
+                                if (!C::kKFreeOnS) mma_commit(&bar.empty_k[sk]);
+                            }
+                        }
+                        if (ok) mma_commit(&bar.o_ready[0]);
+                        g += Tu.n;
                     }
                 }
-                if (ok)
+                // (two S buffers: O ready is signalled per unit inside the loop)
+                if (ok && NB == 1)
                     for (int t = 0; t < U.nt; ++t) mma_commit(&bar.o_ready[t]);
                 // Drain: all issued MMAs complete before TMEM is released.
                 mma_commit(&bar.drain);
@@ -1283,6 +1406,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
             fence_proxy_async_smem();
             mbar_arrive(&bar.ready_q);
+        }
+        if constexpr (kPersist) {
+            // Persistent split mode: the query tile of every later unit of this
+            // CTA, rotated into its parts in the staging area as soon as it lands,
+            // and copied to TMEM once the previous unit's last S product is done.
+            // Both named barriers run in every iteration, whatever the waits
+            // returned, so the four warps always meet.
+            {
+                int g = T.n;   // key tiles of the units before
+                for (int ku = 1;; ++ku) {
+                    const int uu = int(blockIdx.x) + ku * int(gridDim.x);
+                    if (uu >= p.n_units) break;
+                    const Unit Uu = decode_unit<kKvSplit>(p, uu);
+                    const Tiles Tu = make_tiles<BN, kKvSplit>(Uu.q0, Uu.split, p);
+                    bool okq = __all_sync(0xffffffffu, mbar_wait(&bar.full_q, ku & 1, abort, tmo));
+                    if (okq)
+                        rotate_tile_bf16<D, RD, kHalf, kSplit, false, kBM>(
+                            sQ, sQ + C::kTileQ, (long long)Uu.tq0(0) + p.qoff, ph, p, rotq);
+                    named_bar_sync(1, 128);
+                    if (okq)
+                        okq = __all_sync(0xffffffffu,
+                                         mbar_wait(&bar.s_ready[0][(g - 1) % C::kNB],
+                                                   ((g - 1) / C::kNB) & 1, abort, tmo));
+                    if (okq) {
+                        tc_fence_after();
+                        q_parts_to_tmem<D, C::kBoxQ>(sQ, sQ + C::kTileQ, tw,
+                                                     tmem + (uint32_t((warp & 3) * 32) << 16) +
+                                                         C::kColQ);
+                        tc_fence_before();
+                    }
+                    named_bar_sync(1, 128);
+                    if (okq) {
+                        fence_proxy_async_smem();
+                        mbar_arrive(&bar.ready_q);
+                    }
+                    g += Tu.n;
+                }
+            }
         }
         // bf16 keys that are already rotated (and, split, already in parts) go
         // straight from the TMA to the MMA
@@ -1352,20 +1513,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int hf = lane >> 4;                         // column half
             const int row = (warp & 3) * 32 + (warp >> 2) * 16 + (lane & 15);
             const uint32_t tl = tmem + (uint32_t((warp & 3) * 32 + (warp >> 2) * 16) << 16);
-            const RowMap rm = map_row(p, U, 0, row, false);
-            const int pi = rm.i + p.qoff;                     // this row's query position
-            const int tq0 = U.tq0(0);
             const float cl2 = p.c_log2;
-            float m = -INFINITY, l = 0.f;                     // l: this thread's half
             bool ok = true;
-            for (int it = 0; it < T.n; ++it) {
-                const int b = it % NB;
+            // Persistent launches take their units one after the other; S
+            // buffers and V stages keep counting across them (g: the key tiles
+            // of the units before).
+            int g = 0;
+            for (int ku = 0; ok; ++ku) {
+            const int uu = int(blockIdx.x) + ku * int(gridDim.x);
+            if (kPersist ? uu >= p.n_units : ku > 0) break;
+            const Unit Uu = kPersist ? decode_unit<kKvSplit>(p, uu) : U;
+            const Tiles Tu = kPersist ? make_tiles<BN, kKvSplit>(Uu.q0, Uu.split, p) : T;
+            const RowMap rm = map_row(p, Uu, 0, row, false);
+            const int pi = rm.i + p.qoff;                     // this row's query position
+            const int tq0 = Uu.tq0(0);
+            float m = -INFINITY, l = 0.f;                     // l: this thread's half
+            for (int it = 0; it < Tu.n; ++it) {
+                const int gi = g + it;
+                const int b = gi % NB;
                 const uint32_t s_col = b * BN;
                 ok = __all_sync(0xffffffffu,
-                                mbar_wait(&bar.s_ready[0][b], (it / NB) & 1, abort, tmo));
+                                mbar_wait(&bar.s_ready[0][b], (gi / NB) & 1, abort, tmo));
                 if (!ok) break;
                 tc_fence_after();
-                const int jt = T.tile(it), k0 = jt * BN + hf * HB;   // this thread's first key
+                const int jt = Tu.tile(it), k0 = jt * BN + hf * HB;   // this thread's first key
                 const bool partial = !tile_full<BN>(tq0, jt, p);
                 // visible columns: col <= hi and (no window or col >= lo or col < sk)
                 const int hi = p.causal ? min(pi - k0, p.Lk - 1 - k0) : p.Lk - 1 - k0;
@@ -1391,7 +1562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // stage's barrier.  Each thread rescales its half of the row's
                     // output dims.
                     ok = __all_sync(0xffffffffu,
-                                    mbar_wait(&bar.empty_v[(it - 1) % NSV], ((it - 1) / NSV) & 1,
+                                    mbar_wait(&bar.empty_v[(gi - 1) % NSV], ((gi - 1) / NSV) & 1,
                                               abort, tmo));
                     if (!ok) break;
                     tc_fence_after();
@@ -1429,7 +1600,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 mbar_arrive(&bar.p_ready[0][b]);
             }
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.o_ready[0], 0, abort, tmo));
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.o_ready[0], ku & 1, abort, tmo));
             if (ok) {
                 tc_fence_after();
                 const float lt = l + __shfl_xor_sync(0xffffffffu, l, 16);   // the row's sum
@@ -1438,14 +1609,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < DV / 64; ++c) {
                     float o[32];
                     tmem_ld16x2_32(tl + C::kColO + c * 64, o);
+                    if constexpr (kPersist) {
+                        // O read: a persistent launch's next unit may start its
+                        // first PV into the same columns
+                        if (c == DV / 64 - 1) {
+                            tc_fence_before();
+                            mbar_arrive(&bar.o_free);
+                        }
+                    }
                     if (rm.valid)
-                        store_o32<DV, kF32, kKvSplit>(p, U, U.split, rm.h, rm.i, 2 * c + hf, o, inv);
+                        store_o32<DV, kF32, kKvSplit>(p, Uu, Uu.split, rm.h, rm.i, 2 * c + hf, o, inv);
                 }
                 if (rm.valid && hf == 0) {
                     const float ln2 = 0.69314718055994531f;
-                    store_lse<kKvSplit>(p, U, U.split, rm.h, rm.i,
+                    store_lse<kKvSplit>(p, Uu, Uu.split, rm.h, rm.i,
                                         lt > 0.f ? (m + __log2f(lt)) * ln2 : -INFINITY);
                 }
+            }
+            g += Tu.n;
             }
         } else if (kConvV && warp >= 4) {
             // split mode: its one query tile leaves softmax warps 4-7 free; unless
@@ -2178,16 +2359,17 @@ struct AttnLaunchShape {
     int D, DV, RD;    // query/key head dim, value head dim, rotated dims
 };
 
-template <int D, int DV, int RD, bool kF32, bool kHalf, bool kSplit, bool kKvSplit>
-lcx_status launch(const Maps &m, const AttnParams &p, unsigned grid, cudaStream_t s) {
-    auto kern = attn_fwd_kernel<D, DV, RD, kF32, kHalf, kSplit, kKvSplit>;
+template <int D, int DV, int RD, bool kF32, bool kHalf, bool kSplit, bool kKvSplit,
+          bool kPersist>
+lcx_status launch_instance(const Maps &m, const AttnParams &p, unsigned grid, cudaStream_t s) {
+    auto kern = attn_fwd_kernel<D, DV, RD, kF32, kHalf, kSplit, kKvSplit, kPersist>;
     const int smem = Cfg<D, DV, kSplit, kF32 && !kSplit && D == 64, kKvSplit>::kSmemBytes;
     // The warpgroups re-balance registers with setmaxnreg, which waits until the
     // registers it asks for are free: the launch must hold the whole split.
     static const int regs = []() {
         cudaFuncAttributes fa;
         return cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, DV, RD, kF32, kHalf, kSplit,
-                                                         kKvSplit>) == cudaSuccess
+                                                         kKvSplit, kPersist>) == cudaSuccess
                    ? fa.numRegs
                    : -1;
     }();
@@ -2202,6 +2384,16 @@ lcx_status launch(const Maps &m, const AttnParams &p, unsigned grid, cudaStream_
     if (e != cudaSuccess)
         return fail(LCX_ERR_CUDA, "attn_fwd launch failed: %s", cudaGetErrorString(e));
     return LCX_OK;
+}
+
+// The persistent instance for the split mode's CTA-per-SM launches (see
+// AttnParams::persist), the plain instance otherwise.
+template <int D, int DV, int RD, bool kF32, bool kHalf, bool kSplit, bool kKvSplit>
+lcx_status launch(const Maps &m, const AttnParams &p, unsigned grid, cudaStream_t s) {
+    if constexpr (kSplit && !kKvSplit && !kF32 && D == 128)
+        if (p.persist)
+            return launch_instance<D, DV, RD, kF32, kHalf, kSplit, kKvSplit, true>(m, p, grid, s);
+    return launch_instance<D, DV, RD, kF32, kHalf, kSplit, kKvSplit, false>(m, p, grid, s);
 }
 
 // Full rotary (RD = D = DV): bf16 or fp32 operands, plain or split QK^T.
@@ -2294,6 +2486,7 @@ struct AttnLaunch : AttnLaunchShape {
     int rot_h, rot_d; // heads and columns the pass rotates (Hkv, D; or 1, d_R)
     void *k_rot;      // where the pass writes
     bool decode;      // split-KV launch of the transposed decode kernel
+    int sms;          // the device's SM count
 };
 
 // Validate `a` and fill `x`.  *noop is set for empty problems (B or L zero),
@@ -2454,6 +2647,7 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     p.n_split = 1;
     x.units = (long long)p.n_qb * p.units_per_qb;
     if (x.units > 0x7fffffffLL) return fail(LCX_ERR_UNSUPPORTED, "too many work units");
+    x.sms = sms;
     p.rotate_q = (a->flags & LCX_ATTN_PREROTATED) ? 0 : 1;
     p.rotate_k = (rotate_k_once || (a->flags & (LCX_ATTN_PREROTATED | LCX_ATTN_PREROTATED_K)))
                      ? 0 : 1;
@@ -2476,6 +2670,13 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
     p.k_rope_shared = a->k_rope ? 1 : 0;
     p.k_x8_tma = k_x8 ? 1 : 0;
     p.v_f16 = v16_ptr ? 1 : 0;
+    // Split QK^T with the key parts and V from the rotate pass at D = 128: a
+    // CTA per SM takes its units one after the other, the next unit's query
+    // tile loaded, rotated and copied to TMEM while the current one finishes
+    // (cleared again for key-split launches).
+    p.n_units = int(x.units);
+    p.persist = ((a->flags & LCX_ATTN_SPLIT_QK) && a->dtype == LCX_BF16 && a->D == 128 &&
+                 v16_ptr && !(a->flags & LCX_ATTN_TEST_STALL) && x.units > sms) ? 1 : 0;
     // Legitimate waits last microseconds; the default limit is 2 s.
     p.timeout_ns = 1000000ull * (unsigned long long)(a->watchdog_ms > 0 ? a->watchdog_ms : 2000);
     p.test_stall = (a->flags & LCX_ATTN_TEST_STALL) ? 1 : 0;
@@ -2531,7 +2732,8 @@ lcx_status attn_prepare(const lcx_attn_args *a, AttnLaunch &x, bool *noop) {
 
 // Launch the attention kernel described by x (x.p.n_split CTAs per unit).
 lcx_status attn_enqueue(const AttnLaunch &x, cudaStream_t s) {
-    const long long grid = x.units * x.p.n_split;
+    const long long grid =
+        x.p.persist ? std::min<long long>(x.units, x.sms) : x.units * x.p.n_split;
     if (grid > 0x7fffffffLL) return fail(LCX_ERR_UNSUPPORTED, "too many work units");
     if (x.rotate_k_once) {
         // the rotate pass over all keys (positions 0..Lk-1), same stream first
@@ -2624,6 +2826,7 @@ extern "C" lcx_status lcx_attn_fwd_split(const lcx_attn_args *a, int32_t num_spl
         static_cast<char *>(workspace) + split_o_bytes(rows, x.DV, 2 * int64_t(num_splits)));
     x.p.n_split = num_splits;
     x.p.split_recip = std::nextafter(1.0f / float(num_splits), 2.0f);
+    x.p.persist = 0;
     // Head-packed query tiles: with few queries per head (decode, short chunks)
     // the G heads of a kv group share the CTA's query tiles (pack_lp rows per
     // head: L rounded up to 8 rows), so every K/V tile is read and rotated once

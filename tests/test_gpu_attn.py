@@ -363,3 +363,22 @@ def test_attn_paired_units(extra):
     errs = sampled_check(w)
     assert max(e[0] for e in errs) <= MAX_ABS
     assert max(e[1] for e in errs) <= MEAN_ABS
+
+
+@pytest.mark.parametrize("extra", [
+    dict(),                                   # causal: units of 1 to 40 key tiles
+    dict(window=1000, sinks=4, B=2),          # window and sinks, two batches
+])
+def test_attn_split_persistent_units(extra):
+    """Split QK^T with the keys split once by the rotate pass runs as one CTA per
+    SM taking its units one after the other (the next unit's query tile staged,
+    rotated and moved to TMEM while the current unit finishes) whenever the units
+    outnumber the SMs.  Units of every length, including the first query block
+    of each head, whose one key tile never reaches the query's staging stage;
+    sampled rows of every head against the oracle."""
+    w = BASE.with_(Hq=8, Hkv=2, L=128 * 40, mode="yarn", scale=8.0, original_max_pos=1024,
+                   split_qk=True, **extra)
+    assert w.L // 128 * w.Hq * w.B > torch.cuda.get_device_properties(0).multi_processor_count
+    errs = sampled_check(w, n_random=24, rotate_k_once=True)
+    assert max(e[0] for e in errs) <= MAX_ABS
+    assert max(e[1] for e in errs) <= MEAN_ABS
